@@ -1,0 +1,471 @@
+"""Benchmark of the speculative-decoding verify step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {0..4}] [--impl {ours,reference}]
+
+One step = one verify round (one C-ABI call) over the workload's whole batch.
+Default workload 1: chain speculative sampling, B=64, gamma=5, V=32000, bf16
+target + draft logits, T in {0.6, 1.0} per sequence.  With N > 1 (torchrun)
+every rank verifies its own batch of the same shape (the batch axis shards
+with no exchange): weak scaling, time = max over ranks.
+
+Rank 0 prints ONE JSON line.  ``value`` is whole-job verify rounds/s with the
+inputs already in HBM (CUDA-graph replays, CUDA events); L2 is kept cold by
+rotating several input sets whose total exceeds the 126 MB L2 (workload 1) or
+by inputs larger than L2 (workloads 2-4).  ``e2e`` is the same metric through
+the Python binding with pinned host buffers copied in and results copied out
+every step.  ``roofline`` reports the row kernel (the dominant one) against
+the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 oracle on a
+bounded sample on the host cores.  ``--impl reference`` runs that oracle
+alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def make_inputs(wid: int, rnd: int, device, rank: int = 0):
+    from speculative_decoding_verify_temperature_b200 import workloads as wl
+    r = rnd + 100 * rank
+    if wid == 0:
+        t, d = wl.chain_config0_logits(device)
+        return wl.chain_config0_round(r, t, d, device)
+    if wid == 1:
+        return wl.chain_config1(r, device)
+    if wid == 2:
+        return wl.tree_config2(r, device)
+    if wid == 3:
+        return wl.tree_config3(r, device)
+    return wl.chain_config4(r, device)
+
+
+def input_bytes(inp) -> int:
+    n = 0
+    for v in vars(inp).values():
+        if hasattr(v, "element_size") and hasattr(v, "numel"):
+            n += v.numel() * v.element_size()
+    return n
+
+
+def describe(wid: int, inp) -> dict:
+    from speculative_decoding_verify_temperature_b200 import workloads as wl
+    d = {"workload": wl.WORKLOADS[wid], "global_batch": inp.B}
+    if wid in (0, 1, 4):
+        d.update(gamma=inp.gamma, V=inp.V, target_dtype=str(inp.target.dtype).split(".")[-1],
+                 draft="f32 probabilities" if inp.draft_is_probs else str(inp.draft.dtype).split(".")[-1] + " logits")
+    else:
+        d.update(nodes=inp.N, V=inp.V, max_depth=inp.max_depth, target_dtype=str(inp.target.dtype).split(".")[-1])
+    return d
+
+
+class Runner:
+    """Calls the verify entry point of a workload through the Python binding."""
+
+    def __init__(self, wid, inp, ws):
+        self.wid, self.inp, self.ws = wid, inp, ws
+        import torch
+        B = inp.B
+        dev = inp.target.device
+        if wid in (0, 1, 4):
+            self.out = (torch.empty((B, inp.gamma + 1), dtype=torch.int32, device=dev),
+                        torch.empty((B,), dtype=torch.int32, device=dev))
+        else:
+            W = inp.max_depth + 1
+            self.out = (torch.empty((B, W), dtype=torch.int32, device=dev),
+                        torch.empty((B, W), dtype=torch.int32, device=dev),
+                        torch.empty((B,), dtype=torch.int32, device=dev))
+
+    def __call__(self):
+        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+        i = self.inp
+        if self.wid in (0, 1, 4):
+            sv.spec_verify_chain(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
+                                 draft_is_probs=i.draft_is_probs, V=i.V, out_tokens=self.out[0],
+                                 out_num_accepted=self.out[1], workspace=self.ws)
+        elif self.wid == 2:
+            sv.spec_verify_tree_greedy(i.target, i.tokens, i.parents, i.max_depth, V=i.V,
+                                       out_accept_index=self.out[0], out_tokens=self.out[1],
+                                       out_num_accepted=self.out[2], workspace=self.ws)
+        else:
+            sv.spec_verify_tree_sample(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
+                                       i.max_depth, draft_probs=i.draft_probs, V=i.V,
+                                       out_accept_index=self.out[0], out_tokens=self.out[1],
+                                       out_num_accepted=self.out[2], workspace=self.ws)
+
+    def num_accepted(self):
+        return self.out[-1]
+
+
+def kernels_per_step(wid, inp) -> int:
+    """Launches per verify call: the row-statistics kernel and the finalize kernel."""
+    return 2
+
+
+def workspace_for(wid, inp):
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    ws = sv.Workspace(inp.target.device)
+    if wid in (0, 1, 4):
+        return ws.get(sv.SPEC_ENTRY_CHAIN, inp.B, inp.gamma, inp.V)
+    e = sv.SPEC_ENTRY_TREE_GREEDY if wid == 2 else sv.SPEC_ENTRY_TREE_SAMPLE
+    return ws.get(e, inp.B, inp.N, inp.V)
+
+
+def algorithmic_bytes(wid, inp) -> int:
+    """Bytes of logits / probabilities the row kernel must read once per round."""
+    b = inp.target[:, :, :inp.V].numel() * inp.target.element_size()
+    if wid in (0, 1):
+        b += inp.draft[:, :, :inp.V].numel() * inp.draft.element_size()
+    return b
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons in a background thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self.stop_ev = threading.Event()
+        self.mark = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:          # NVML missing: report it rather than guess
+            self.nv = None
+            self.err = repr(e)
+            self.max_mhz = None
+
+    def run(self):
+        while not self.stop_ev.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((self.mark, mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self.run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop_ev.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        timed = [s for s in self.samples if s[0]]
+        window = "timed region"
+        if len(timed) < 3:
+            timed = self.samples
+            window = "warm-up + timed region (timed region shorter than the sampling period)"
+        mhz = [s[1] for s in timed]
+        mask = 0
+        for s in timed:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and b != 0x1]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(timed), "window": window}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+
+def cpu_baseline(wid, inp, seconds, nthreads=None):
+    """Time the fp64 oracle, as it stands, on whole rounds of the same inputs until
+    ``seconds`` have elapsed (at least one round).  Returns rounds/s."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity
+    import oracle
+    oracle.build()
+    cores = nthreads or len(os.sched_getaffinity(0))
+    # Copy the inputs to host once; the oracle reads the same bytes the GPU reads.
+    n = 0
+    fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain,
+          2: parity.oracle_greedy, 3: parity.oracle_sample}[wid]
+    B = inp.B
+    # Large workloads: a bounded sample of whole sequences per "round" of work,
+    # scaled to full rounds below.
+    per = B if wid in (0, 1) else max(1, min(B, {2: 8, 3: 4, 4: 16}[wid]))
+    rows = None if per == B else list(range(per))
+    elapsed = 0.0
+    while n == 0 or elapsed < seconds:
+        t1 = time.perf_counter()
+        fn(inp, rows, nthreads=cores)
+        elapsed += time.perf_counter() - t1
+        n += 1
+    rounds = n * per / B
+    return {"value": rounds / elapsed, "unit": "rounds/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} x {per} of {B} sequences of one round (whole sequences), fp64 C oracle, "
+                      f"OpenMP over sequences, {elapsed:.1f} s of CPU time; rounds/s scaled by {per}/{B}"}
+
+
+# ----------------------------------------------------------------------------- main
+
+def profile_traffic(wid):
+    """Per-launch DRAM traffic of the row kernel from a committed ncu summary,
+    valid only while the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "speculative_decoding_verify_temperature_b200", "csrc", "spec_verify.cu")
+    try:
+        rec = json.load(open(path)).get(str(wid))
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec and rec.get("source_sha256_16") == h:
+            return rec.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0}, "fallback"
+
+
+def run_reference(args, ws_, rank):
+    import torch
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(args.workload, 0, dev)
+    steps = max(1, args.steps)
+    # each step is a bounded sample of the workload (see cpu_baseline)
+    cb = cpu_baseline(args.workload, inp, seconds=min(60.0, max(5.0, 0.02 * steps)))
+    cfg = describe(args.workload, inp)
+    line = {"impl": "reference", "metric": "verify rounds/s", "value": cb["value"], "unit": "rounds/s",
+            "n_gpus": ws_, "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg, "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    ws_, rank, local = dist_env()
+    import torch
+    import torch.distributed as dist
+    if ws_ > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if args.impl == "reference":
+        run_reference(args, ws_, rank)
+        if ws_ > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    wid = args.workload
+
+    # --- inputs: enough rotating sets to keep L2 cold between steps
+    first = make_inputs(wid, 0, dev, rank)
+    nbytes = input_bytes(first)
+    nsets = 1 if nbytes > 2 * L2_BYTES else min(16, -(-2 * L2_BYTES // nbytes))
+    sets = [first] + [make_inputs(wid, r, dev, rank) for r in range(1, nsets)]
+    ws = workspace_for(wid, first)
+    runners = [Runner(wid, s, ws) for s in sets]
+    kps = kernels_per_step(wid, first)
+    stream = torch.cuda.current_stream()
+
+    for i in range(max(3, args.warmup)):
+        runners[i % nsets]()
+    torch.cuda.synchronize()
+
+    # --- one CUDA graph per rotation of the input sets
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for r in runners:
+            r()
+    torch.cuda.synchronize()
+    singles = []
+    for r in runners:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            r()
+        singles.append(g)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.02)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        if ws_ > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler.mark = True
+        e0.record(stream)
+        full, rem = divmod(K, nsets)
+        for _ in range(full):
+            graph.replay()
+        for i in range(rem):
+            singles[i].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sampler.mark = False
+        if ws_ > 1:
+            dist.barrier()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], device=dev)
+    if ws_ > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = ws_ * K / (ms_max / 1e3)
+
+    # --- dominant kernel duration (row kernel), events recorded by the library
+    nk = max(50, min(2000, K))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    torch.cuda.synchronize()
+    for i in range(nk):
+        sv.spec_profile_events(*evs[i])
+        runners[i % nsets]()
+    sv.spec_profile_events()
+    torch.cuda.synchronize()
+    kms = [a.elapsed_time(b) for a, b in evs]
+    k_avg_ms = sum(kms) / len(kms)
+    alg = algorithmic_bytes(wid, first)
+    peaks, peak_kind = measured_peaks()
+    achieved = alg / (k_avg_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profile_traffic(wid),
+                "kernel": "k_stats (streams every logit row once)",
+                "kernel_ms": round(k_avg_ms, 5), "algorithmic_bytes_per_launch": alg,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"}
+    round_gbs = alg / (ms_max / K / 1e3) / 1e9
+
+    # --- acceptance statistics of the benchmarked rounds
+    torch.cuda.synchronize()
+    acc = []
+    for r in runners:
+        r()
+        acc.append(r.num_accepted().float())
+    acc = torch.cat(acc)
+    mean_tau = float((acc + 1).mean())
+    B = first.B
+    draft_per_round = B * (first.gamma if wid in (0, 1, 4) else first.N - 1)
+
+    # --- end to end through the binding with host buffers
+    e2e = run_e2e(wid, first, ws, args.e2e_steps, dev)
+
+    cfg = describe(wid, first)
+    cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",
+               l2=(f"{nsets} rotating input sets of {nbytes / 1e6:.1f} MB ({nsets * nbytes / 1e6:.0f} MB > 126 MB L2)"
+                   if nsets > 1 else f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2"),
+               timing="CUDA-graph replays, CUDA events, max over ranks")
+    line = {
+        "metric": "verify rounds/s", "value": round(value, 2), "unit": "rounds/s", "n_gpus": ws_,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+        "roofline": roofline,
+        "round_hbm_gbs": round(round_gbs, 1),
+        "draft_tokens_verified_per_s": round(value * draft_per_round, 1),
+        "accepted_tokens_per_s": round(value * B * mean_tau, 1), "mean_tau": round(mean_tau, 4),
+        "e2e": e2e, "gpu_launches": K * kps, "clocks": sampler.summary(),
+    }
+    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wid, first, args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_ > 1:
+        dist.barrier()
+        del graph, singles
+        dist.destroy_process_group()
+
+
+def run_e2e(wid, inp, ws, steps, dev):
+    """Same metric through the binding: every step copies this round's inputs from
+    pinned host memory, verifies, and copies the outputs back."""
+    import torch
+    host = {k: v.detach().cpu().pin_memory() for k, v in vars(inp).items() if isinstance(v, torch.Tensor)}
+    dev_bufs = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    import copy
+    dinp = copy.copy(inp)
+    for k, v in dev_bufs.items():
+        setattr(dinp, k, v)
+    runner = Runner(wid, dinp, ws)
+    out_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in runner.out]
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(o.numel() * o.element_size() for o in out_host)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k, v in host.items():
+            dev_bufs[k].copy_(v, non_blocking=True)
+        runner()
+        for o, h in zip(runner.out, out_host):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": round(steps / (ms / 1e3), 2), "unit": "rounds/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

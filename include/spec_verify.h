@@ -1,0 +1,249 @@
+/*
+ * spec_verify.h -- C ABI of libspecverify, the verify/accept step of
+ * speculative decoding on NVIDIA B200 (sm_100a).
+ *
+ * The method comes from three web pages, cited by title and section:
+ *   [atlas]   "Speculative Decoding —— 无损加速自回归 decode" (llm-infra-atlas):
+ *             §0 latency formula, §2 notation (p = target, q = draft, gamma,
+ *             bonus token, correction / residual, tree attention).
+ *   [kevins]  "Speculative Decoding：投机解码的真实收益、校正采样与生产边界"
+ *             (ricardokevins notes): "draft / verify / accept" steps,
+ *             "sampling correction" a(x) = min(1, p(x)/q(x)) and
+ *             r(x) = max(p(x)-q(x),0) / sum_y max(p(y)-q(y),0).
+ *   [origins] zdszero "spec_origins" page: "Blockwise Parallel Decoding"
+ *             (verify = longest prefix equal to the argmax), "Speculative
+ *             Decoding" (acceptance rules 1-3, why lossless, closed form),
+ *             "SpecInfer" (token tree, ancestor-only mask), "In SGLang"
+ *             (verify_tree_greedy, target-only tree sampling with prob_acc,
+ *             threshold_single / threshold_acc, relu(target - draft_probs)).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is DEVICE memory owned by the caller, except the
+ *   host output of spec_read_device_status.  The library allocates nothing.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *   default stream).  Argument errors are detected on the host before any
+ *   launch and returned synchronously; nothing is enqueued then.  A failed
+ *   launch returns SPEC_ERR_CUDA.
+ * - Per-sequence input errors found on the device (non-finite logits, an
+ *   all -inf row, a token id outside [0, V), a temperature that is not a
+ *   finite normal positive f32, a malformed parent array) never trap: the
+ *   sequence gets out_num_accepted[b] = -1 and every output slot -1, and the
+ *   bit (1 << SPEC_ERR_DEVICE_INPUT) is OR-ed into the workspace status word
+ *   (read it with spec_read_device_status).
+ * - Logit rows: row r of sequence b starts at element (b*R + r) * row_stride
+ *   of its array (R = rows per sequence of that array).  Each row's first
+ *   byte must be 16-byte aligned: base pointer 16-byte aligned and
+ *   row_stride * element size a multiple of 16 bytes (a multiple of 8 bf16
+ *   or 4 f32 elements).  row_stride >= V.
+ * - Temperature softmax: p = softmax(logits / T) per row, computed in f32
+ *   with f32 accumulation (fp64 across chunks); T is per sequence.
+ * - Uniforms (coins, final_u) are caller-supplied f32 values in [0, 1).
+ *   Every random choice of a call is a deterministic function of them: the
+ *   same inputs give bit-identical outputs.
+ * - Inverse-CDF draws scan the vocabulary in index order 0..V-1 and pick
+ *   the smallest j with u * S < C_j (C = running sum of the weights, S the
+ *   total): zero-weight tokens are never drawn.
+ * - Workspace: caller-owned device scratch of spec_workspace_bytes() bytes,
+ *   256-byte aligned, zero-filled once by spec_workspace_init() before first
+ *   use and again whenever it is reused for another entry point or another
+ *   batch size.  Its arrival counters reset themselves, so it can be reused
+ *   by any number of calls of that shape, and captured in CUDA graphs, on
+ *   ONE stream at a time (concurrent calls sharing a workspace race).
+ * - Limits: 1 <= gamma <= SPEC_MAX_GAMMA, 1 <= N <= SPEC_MAX_NODES,
+ *   0 <= max_depth <= SPEC_MAX_DEPTH, 1 <= V <= SPEC_MAX_V, B >= 0
+ *   (B == 0 returns SPEC_OK and launches nothing).
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPEC_MAX_GAMMA 16
+#define SPEC_MAX_NODES 256
+#define SPEC_MAX_DEPTH 64
+#define SPEC_MAX_V (1 << 20)
+
+typedef enum {
+    SPEC_OK = 0,
+    SPEC_ERR_INVALID_ARG = 1,   /* host-side argument check failed; nothing launched */
+    SPEC_ERR_UNSUPPORTED = 2,   /* valid but unsupported combination (e.g. no sm_100 device) */
+    SPEC_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    SPEC_ERR_DEVICE_INPUT = 4,  /* (status bit) a sequence had invalid device-side inputs */
+    SPEC_ERR_TIMEOUT = 5,       /* (status bit) a bounded device-side wait gave up */
+    SPEC_ERR_WORKSPACE = 6      /* workspace too small or misaligned */
+} spec_status;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
+
+typedef enum {
+    SPEC_ENTRY_CHAIN = 0,
+    SPEC_ENTRY_TREE_GREEDY = 1,
+    SPEC_ENTRY_TREE_SAMPLE = 2
+} spec_entry;
+
+/*
+ * spec_verify_chain -- chain speculative sampling, one round for B sequences.
+ * [origins] "Speculative Decoding", acceptance rules 1-3; [kevins] "sampling
+ * correction" a(x), r(x); the p/q rejection path that [origins] "In SGLang"
+ * runs for chains (topk = 1).
+ *
+ * For each sequence b, with p_i = softmax(target row i / T_b), i in [0,gamma],
+ * and q_i the draft distribution at position i:
+ *   1. draft token x_i is accepted iff coins[b,i] <= p_i(x_i) / q_i(x_i)
+ *      (ratio +inf when q_i(x_i) = 0), for i = 0, 1, ... until the first
+ *      rejection k (k = gamma if none);
+ *   2. if k < gamma the correction token is drawn with final_u[b] from
+ *      norm(max(0, p_k - q_k)); if that mass is zero (rounding only) it is
+ *      drawn from p_k;
+ *   3. if k = gamma the bonus token is drawn with final_u[b] from p_gamma.
+ *
+ * target_logits  [B, gamma+1, t_row_stride] of tdt, read-only.
+ * draft          [B, gamma, d_row_stride]: logits of ddt when draft_is_probs
+ *                = 0 (q_i = softmax(draft row i / T_b), same T as the
+ *                target), or f32 probabilities used as given when
+ *                draft_is_probs = 1 (ddt must be SPEC_F32).  Read-only.
+ * draft_tokens   [B, gamma] int32 in [0, V).
+ * temperature    [B] f32.
+ * coins          [B, gamma] f32, coins[b,i] is the uniform of position i.
+ * final_u        [B] f32.
+ * out_tokens     [B, gamma+1] int32: x_0..x_{k-1}, then the correction or
+ *                bonus token at index k, then -1.
+ * out_num_accepted [B] int32: k in [0, gamma], or -1 (invalid sequence).
+ * diag           nullable, [B, 2*gamma+1] f32: p_i(x_i) for i < gamma,
+ *                then q_i(x_i) for i < gamma, then S = the mass of the
+ *                distribution the last token was drawn from before
+ *                normalisation (sum_j max(0, p_k(j) - q_k(j)) on a
+ *                rejection, 1 for a bonus).
+ * workspace      >= spec_workspace_bytes(SPEC_ENTRY_CHAIN, B, gamma, V).
+ */
+spec_status spec_verify_chain(int B, int gamma, int V,
+                              const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                              const void* draft, spec_dtype ddt, int draft_is_probs,
+                              int64_t d_row_stride,
+                              const int32_t* draft_tokens, const float* temperature,
+                              const float* coins, const float* final_u,
+                              int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * spec_verify_tree_greedy -- greedy verify of a draft token tree.
+ * [origins] "In SGLang" (greedy goes through verify_tree_greedy) and
+ * "Blockwise Parallel Decoding" (verify keeps the longest prefix equal to
+ * the scoring model's own argmax, so the output equals greedy decoding);
+ * [origins] "SpecInfer" (tree flattened, ancestors before descendants).
+ *
+ * g_n = argmax_j target[b, n, j] (lowest index among equal maxima; a NaN
+ * anywhere in the sequence's rows makes it invalid).  Walk: cur = 0; the
+ * first child c of cur in increasing node index with tokens[b,c] == g_cur is
+ * accepted and becomes cur; stop when no child matches.  Emitted: the
+ * accepted draft tokens, then the bonus g_cur.
+ *
+ * target_logits  [B, N, t_row_stride]; row n holds the target logits at tree
+ *                node n (node 0 = the last verified token, the root).
+ * tokens         [B, N] int32; tokens[b,0] is not read; others in [0, V).
+ * parents        [B, N] int32; parents[b,0] = -1; 0 <= parents[b,n] < n; every
+ *                node's depth (root = 0) <= max_depth.
+ * out_accept_index [B, max_depth+1] int32: node ids of the accepted path,
+ *                root first (k+1 entries), then -1.
+ * out_tokens     [B, max_depth+1] int32: the k accepted draft tokens, the
+ *                bonus token at index k, then -1.
+ * out_num_accepted [B] int32: k, or -1.
+ * workspace      >= spec_workspace_bytes(SPEC_ENTRY_TREE_GREEDY, B, N, V).
+ * Temperature plays no part.
+ */
+spec_status spec_verify_tree_greedy(int B, int N, int V, int max_depth,
+                                    const void* target_logits, spec_dtype tdt,
+                                    int64_t t_row_stride,
+                                    const int32_t* tokens, const int32_t* parents,
+                                    int32_t* out_accept_index, int32_t* out_tokens,
+                                    int32_t* out_num_accepted,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * spec_verify_tree_sample -- target-only tree sampling.
+ * [origins] "In SGLang": tree_speculative_sampling_target_only, a SpecInfer
+ * style walk down the tree that tries the next sibling after a rejection;
+ * draft probabilities are zeros and acceptance reads the target only.
+ *
+ * p_n = softmax(target row n / T_b).  cur = 0.  At cur the children c_1..c_m
+ * (increasing node index) are tried in order with prob_acc += p_cur(tok_c):
+ * c is accepted iff coins[b,cur] <= prob_acc / threshold_acc or
+ * p_cur(tok_c) >= threshold_single; on acceptance cur = c and the walk goes
+ * one level down (with coins[b,c]); a child that is not accepted is
+ * rejected.  The walk stops when no child of cur is accepted or cur has no
+ * children.  The last token is drawn with final_u[b] from
+ * relu(p_cur - d_cur), where d_cur is the draft_probs row of cur (zeros when
+ * draft_probs is NULL) with the entries of cur's rejected children replaced
+ * by their target probabilities.  draft_probs is never written: the
+ * replacement is kept on chip.  With both thresholds 1 the emitted tokens
+ * are distributed exactly as the target's.
+ *
+ * Arguments as spec_verify_tree_greedy, plus:
+ * temperature    [B] f32.
+ * coins          [B, N] f32: coins[b,n] is the uniform used while visiting n.
+ * final_u        [B] f32.
+ * draft_probs    nullable, [B, N, dp_row_stride] f32.
+ * threshold_single, threshold_acc  host f32, > 0 (1.0 = lossless).
+ * diag           nullable, [B, N+1] f32: p_parent(n)(tokens[b,n]) for n >= 1
+ *                (0 at n = 0), then S = the mass of relu(p_cur - d_cur).
+ * workspace      >= spec_workspace_bytes(SPEC_ENTRY_TREE_SAMPLE, B, N, V).
+ */
+spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
+                                    const void* target_logits, spec_dtype tdt,
+                                    int64_t t_row_stride,
+                                    const int32_t* tokens, const int32_t* parents,
+                                    const float* temperature, const float* coins,
+                                    const float* final_u,
+                                    const float* draft_probs, int64_t dp_row_stride,
+                                    float threshold_single, float threshold_acc,
+                                    int32_t* out_accept_index, int32_t* out_tokens,
+                                    int32_t* out_num_accepted, float* diag,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * spec_workspace_bytes -- workspace size for one entry point and shape.
+ * rows = gamma for SPEC_ENTRY_CHAIN (sized for draft logits, which also
+ * covers draft probabilities), N for the tree entry points.  Returns 0 for
+ * out-of-range arguments.  Pure host function.
+ */
+size_t spec_workspace_bytes(int entry, int B, int rows, int V);
+
+/* spec_workspace_init -- zero-fill `bytes` of the workspace on `stream`. */
+spec_status spec_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/*
+ * spec_read_device_status -- copy the workspace status word to *status_out
+ * (a bit mask: bit c set <=> status code c occurred since the last read),
+ * then clear it.  Synchronises `stream`.
+ */
+spec_status spec_read_device_status(void* workspace, int* status_out, void* stream);
+
+/*
+ * spec_profile_events -- kernel timing hook.  While set (non-NULL), every
+ * later verify call on this host thread records `start_event` on its stream
+ * just before launching its row-statistics kernel (the kernel that streams
+ * every logit row, which dominates each call) and `stop_event` just after it,
+ * so cudaEventElapsedTime gives that kernel's duration.  Both are
+ * cudaEvent_t handles owned by the caller; NULL, NULL switches the hook off.
+ * Inside stream capture the records become external event nodes.
+ */
+spec_status spec_profile_events(void* start_event, void* stop_event);
+
+/* spec_status_string -- static description of a status code. */
+const char* spec_status_string(spec_status status);
+
+/* spec_last_error_detail -- detail of the last SPEC_ERR_INVALID_ARG /
+ * SPEC_ERR_CUDA / SPEC_ERR_WORKSPACE returned on the calling host thread. */
+const char* spec_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H */

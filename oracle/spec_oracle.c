@@ -31,8 +31,9 @@
  *   - argmax ties go to the lowest index, comparing values (-0 == +0);
  *   - tree children are visited in increasing node index;
  *   - any invalid input of a sequence (non-finite row maximum, NaN or +inf
- *     logit, token id out of range, T <= 0, malformed parent array) marks the
- *     whole sequence invalid: num_accepted = -1 and every output slot -1.
+ *     logit, token id out of range, a temperature that is not a finite
+ *     normal positive f32, malformed parent array) marks the whole sequence
+ *     invalid: num_accepted = -1 and every output slot -1.
  *
  * Parity margins: for each sequence the oracle also reports how close each
  * random decision came to flipping (|u - ratio|, |coin - prob_acc/theta|,
@@ -127,6 +128,9 @@ static int inverse_cdf(const double* w, int V, double u, double* S_out, double* 
 
 static void fill_i32(int32_t* a, int n, int32_t v) { for (int i = 0; i < n; ++i) a[i] = v; }
 
+/* A usable temperature: finite, positive and not subnormal as an f32. */
+static int temperature_ok(double T) { return T >= 0x1p-126 && T <= 0x1.fffffep127; }
+
 /*
  * Chain verify, one call = one round for B independent sequences.
  *
@@ -173,7 +177,7 @@ void oracle_chain(int B, int gamma, int V,
             int32_t* toks = out_tokens + (int64_t)b * (gamma + 1);
             const int32_t* x = draft_tokens + (int64_t)b * gamma;
             double T = (double)temperature[b];
-            int bad = !(T > 0.0);
+            int bad = !temperature_ok(T);
             for (int i = 0; i <= gamma && !bad; ++i) {
                 const char* row = (const char*)target +
                     ((int64_t)b * (gamma + 1) + i) * t_row_stride * (tdt == OR_F32 ? 4 : 2);
@@ -405,7 +409,7 @@ void oracle_tree_sample(int B, int N, int V, int max_depth,
             int32_t* ai = out_accept_index + (int64_t)b * (max_depth + 1);
             int32_t* ot = out_tokens + (int64_t)b * (max_depth + 1);
             double T = (double)temperature[b];
-            int bad = !(T > 0.0) || !tree_ok(N, V, max_depth, tk, pa, depth);
+            int bad = !temperature_ok(T) || !tree_ok(N, V, max_depth, tk, pa, depth);
             for (int n = 0; n < N && !bad; ++n) {
                 const char* row = (const char*)target +
                     ((int64_t)b * N + n) * t_row_stride * (tdt == OR_F32 ? 4 : 2);

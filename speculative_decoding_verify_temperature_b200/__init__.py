@@ -1,0 +1,18 @@
+"""B200-native verify/accept step of speculative decoding.
+
+``spec_verify`` is the Python binding of ``libspecverify.so`` (C ABI in
+``include/spec_verify.h``); ``workloads`` makes the seeded synthetic inputs.
+"""
+from . import workloads  # noqa: F401
+from .spec_verify import (  # noqa: F401
+    SpecError,
+    Workspace,
+    lib,
+    spec_profile_events,
+    spec_read_device_status,
+    spec_verify_chain,
+    spec_verify_tree_greedy,
+    spec_verify_tree_sample,
+    spec_workspace_bytes,
+    spec_workspace_init,
+)

@@ -1,0 +1,1430 @@
+// spec_verify.cu -- sm_100a kernels and C ABI of libspecverify (see include/spec_verify.h).
+//
+// Data path (one call = one verify round over B sequences, two launches):
+//
+//   k_stats     streams every logit row once.  The (sequence, row, chunk) work
+//               items -- a chunk is 128 threads x 8 x 16-byte vectors = 16 KB
+//               (8192 bf16 or 4096 f32 elements) -- are split into contiguous
+//               per-CTA ranges.  Each warp reduces its 4 KB of a chunk to one
+//               statistic: online softmax (max m, sum 2^(x - m), x = l*log2e/T)
+//               for the sampling entry points, (max value, lowest index) for
+//               greedy.  No atomics, no fences: the next kernel in stream order
+//               reads the statistics.
+//
+//   k_chain_final / k_tree_final   per-sequence finalisation: combine the
+//               statistics per row (fp64 across chunks), gather the drafted
+//               tokens' probabilities, take the accept/reject decisions or walk
+//               the tree, and draw the last token by inverse CDF -- the chunk
+//               holding u*S is located from chunk masses, then rescanned with
+//               coalesced 8-element groups and a block-wide fp64 prefix scan.
+//               The chain residual max(0, p_k - q_k) over several chunks is
+//               summed by one CTA per chunk; the last to arrive (atomicAdd after
+//               __threadfence, no spin-wait) draws and resets its counter, so
+//               workspaces need no per-call memset.
+//
+// Nothing here is a dense contraction, so no tensor cores: the path is a
+// streaming reduction bounded by HBM bandwidth, with the exp2 unit (MUFU, 16
+// per clock per SM) as the secondary ceiling.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "spec_verify.h"
+
+namespace sv {
+
+constexpr int NT = 128;               // threads per CTA
+constexpr int NWARP = NT / 32;
+constexpr int VPT = 8;                // 16-byte vectors per thread per chunk
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1 or N)
+constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
+constexpr double LOG2E = 1.4426950408889634073599246810019;
+
+enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2 };
+enum { DK_NONE = 0, DK_LOGITS = 1, DK_PROBS = 2 };
+
+template <int DT> struct Tr;
+template <> struct Tr<SPEC_BF16> { static constexpr int EPV = 8; static constexpr int ESZ = 2; };
+template <> struct Tr<SPEC_F32> { static constexpr int EPV = 4; static constexpr int ESZ = 4; };
+template <int DT> __host__ __device__ constexpr int chunk_elems() { return NT * VPT * Tr<DT>::EPV; }
+
+struct Params {
+    int B, V, R, nch, gamma, N, max_depth;
+    int rows_tgt;                  // target rows per sequence
+    const char* tgt;
+    int64_t tstride;               // bytes between consecutive target rows
+    const char* drf;
+    int64_t dstride;               // bytes between consecutive draft rows
+    const int32_t* draft_tokens;
+    const int32_t* tokens;
+    const int32_t* parents;
+    const float* temperature;
+    const float* coins;
+    const float* final_u;
+    const float* draft_probs;      // tree sample, nullable
+    int64_t dpstride;              // bytes
+    float th_single, th_acc;
+    int32_t* out_tokens;
+    int32_t* out_accept_index;
+    int32_t* out_num_accepted;
+    float* diag;
+    float2* stats;                 // [B][R][nch][NWARP]
+    float2* stats2;                // [B][nch][NWARP]   (chain residual chunk sums)
+    unsigned* cnt2;                // [B]               (chain residual arrivals)
+    unsigned* status;
+};
+
+// ----------------------------------------------------------------------------- small helpers
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+template <int DT> __device__ __forceinline__ float ld_elem(const char* row, int64_t j) {
+    if constexpr (DT == SPEC_BF16) {
+        unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(row) + j);
+        return __uint_as_float((uint32_t)h << 16);
+    } else {
+        return __ldg(reinterpret_cast<const float*>(row) + j);
+    }
+}
+
+// One 16-byte vector starting at element e0; elements at or past V read as -inf.
+template <int DT> __device__ __forceinline__ uint4 ld_vec(const char* row, int64_t e0, int V) {
+    constexpr int EPV = Tr<DT>::EPV;
+    if (e0 + EPV <= V) return ld_stream(row + e0 * Tr<DT>::ESZ);
+    uint32_t w[4];
+    if constexpr (DT == SPEC_BF16) {
+        const unsigned short* h = reinterpret_cast<const unsigned short*>(row);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t lo = (e0 + 2 * i < V) ? (uint32_t)__ldg(h + e0 + 2 * i) : 0xFF80u;
+            uint32_t hi = (e0 + 2 * i + 1 < V) ? (uint32_t)__ldg(h + e0 + 2 * i + 1) : 0xFF80u;
+            w[i] = lo | (hi << 16);
+        }
+    } else {
+        const uint32_t* f = reinterpret_cast<const uint32_t*>(row);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = (e0 + i < V) ? __ldg(f + e0 + i) : 0xFF800000u;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int DT> __device__ __forceinline__ float vec_elem(const uint4& v, int i) {
+    uint32_t w = (i >> (DT == SPEC_BF16 ? 1 : 0)) == 0 ? v.x
+               : (i >> (DT == SPEC_BF16 ? 1 : 0)) == 1 ? v.y
+               : (i >> (DT == SPEC_BF16 ? 1 : 0)) == 2 ? v.z : v.w;
+    if constexpr (DT == SPEC_BF16) return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+    else return __uint_as_float(w);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+__device__ __forceinline__ float nanf_() { return __int_as_float(0x7fffffff); }
+
+__host__ __device__ __forceinline__ bool temperature_ok(float T) {
+    return T >= 1.17549435e-38f && T <= 3.40282347e38f;   // false for NaN
+}
+__device__ __forceinline__ float scale_of(float T) { return (float)(LOG2E / (double)T); }
+
+__device__ __forceinline__ float2 ldcg2(const float2* p) { return __ldcg(p); }
+
+__device__ __forceinline__ void flag_input_error(const Params& P) {
+    atomicOr(P.status, 1u << SPEC_ERR_DEVICE_INPUT);
+}
+
+// Block-wide exclusive scan of one double per thread; *total receives the sum.
+__device__ double block_excl_scan(double v, double* total) {
+    __shared__ double wsum[NWARP];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    double inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double n = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    double before = 0.0, tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < NWARP; ++w) {
+        if (w < warp) before += wsum[w];
+        tot += wsum[w];
+    }
+    __syncthreads();
+    *total = tot;
+    return before + inc - v;
+}
+
+// ----------------------------------------------------------------------------- row-chunk statistics
+
+// Per-thread online-softmax partial over NV 16-byte vectors starting at element
+// e_base: (max x, sum 2^(x - max)), x = l * s.  `bad` is set by a NaN or +inf.
+template <int DT, int NV>
+__device__ __forceinline__ void thread_softmax(const char* row, int V, int64_t e_base, float s,
+                                               float& mt, float& st, bool& bad) {
+    constexpr int EPV = Tr<DT>::EPV;
+    const int tid = threadIdx.x;
+    uint4 v[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) v[k] = ld_vec<DT>(row, e_base + (int64_t)(k * NT + tid) * EPV, V);
+    float lmax;
+    bool b = false;
+    if constexpr (DT == SPEC_BF16) {
+        __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&v[0].x);
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = __hmax2_nan(mx, h[i]);
+        }
+        float a = __low2float(mx), c = __high2float(mx);
+        b = (a != a) || (c != c);
+        lmax = fmaxf(a, c);
+    } else {
+        lmax = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) {
+                float x = vec_elem<DT>(v[k], i);
+                b |= (x != x);
+                lmax = fmaxf(lmax, x);
+            }
+    }
+    b |= (lmax == INFINITY);
+    mt = -INFINITY;
+    st = 0.f;
+    if (!b && lmax != -INFINITY) {
+        mt = lmax * s;
+        const float nm = -mt;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int i = 0; i < EPV; i += 2) {
+                a0 += ex2(fmaf(vec_elem<DT>(v[k], i), s, nm));
+                a1 += ex2(fmaf(vec_elem<DT>(v[k], i + 1), s, nm));
+            }
+        st = a0 + a1;
+    }
+    bad |= b;
+}
+
+// Online-softmax statistic of chunk c of a row, CH elements per chunk (the
+// target's chunking; rows of another dtype are split into as many 16-byte
+// vectors as that takes).  Per warp: (max x, sum 2^(x - max)); NaN sum for a
+// row holding a NaN or +inf.
+template <int DT, int CH>
+__device__ __forceinline__ float2 chunk_softmax(const char* row, int V, int c, float s) {
+    constexpr int EPV = Tr<DT>::EPV;
+    constexpr int NVT = CH / (NT * EPV);          // vectors per thread for this dtype
+    constexpr int NV = NVT < VPT ? NVT : VPT;
+    constexpr int NSUB = NVT / NV;
+    static_assert(NV * NSUB * NT * EPV == CH, "chunk geometry");
+    float mt, st;
+    bool bad = false;
+    thread_softmax<DT, NV>(row, V, (int64_t)c * CH, s, mt, st, bad);
+#pragma unroll
+    for (int sub = 1; sub < NSUB; ++sub) {
+        float m2, s2;
+        thread_softmax<DT, NV>(row, V, (int64_t)c * CH + (int64_t)sub * NV * NT * EPV, s, m2, s2, bad);
+        const float m = fmaxf(mt, m2);
+        if (m > -INFINITY) st = (mt > -INFINITY ? st * ex2(mt - m) : 0.f) + (m2 > -INFINITY ? s2 * ex2(m2 - m) : 0.f);
+        mt = m;
+    }
+    const float mw = warp_max(mt);
+    const bool anybad = __any_sync(FULL, bad);
+    float contrib = (mt == -INFINITY) ? 0.f : st * ex2(mt - mw);
+    float sw = warp_sum(contrib);
+    if (anybad) sw = nanf_();
+    return make_float2(mw, sw);
+}
+
+// (max value, lowest index) of one chunk per warp; value NaN if any NaN was seen.
+template <int DT>
+__device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
+    constexpr int EPV = Tr<DT>::EPV, CH = chunk_elems<DT>();
+    const int tid = threadIdx.x;
+    uint4 v[VPT];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+        v[k] = ld_vec<DT>(row, (int64_t)c * CH + (int64_t)(k * NT + tid) * EPV, V);
+    float best = -INFINITY;
+    int bestk = 0;
+    uint4 bw = v[0];
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        float mk;
+        if constexpr (DT == SPEC_BF16) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+            __nv_bfloat162 m2 = __hmax2_nan(__hmax2_nan(h[0], h[1]), __hmax2_nan(h[2], h[3]));
+            float a = __low2float(m2), b = __high2float(m2);
+            bad |= (a != a) || (b != b);
+            mk = fmaxf(a, b);
+        } else {
+            mk = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float x = vec_elem<DT>(v[k], i);
+                bad |= (x != x);
+                mk = fmaxf(mk, x);
+            }
+        }
+        if (mk > best) { best = mk; bestk = k; bw = v[k]; }
+    }
+    int j = EPV - 1;
+#pragma unroll
+    for (int i = EPV - 1; i >= 0; --i)
+        if (vec_elem<DT>(bw, i) == best) j = i;
+    int idx = c * CH + (bestk * NT + tid) * EPV + j;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        float ov = __shfl_xor_sync(FULL, best, o);
+        int oi = __shfl_xor_sync(FULL, idx, o);
+        if (ov > best || (ov == best && oi < idx)) { best = ov; idx = oi; }
+    }
+    if (__any_sync(FULL, bad)) best = nanf_();
+    return make_float2(best, __int_as_float(idx));
+}
+
+// ----------------------------------------------------------------------------- finaliser pieces
+
+struct FinShared {
+    float m[MAXR];
+    double z[MAXR];
+    int bad[MAXR];
+    int par[SPEC_MAX_NODES];
+    int tok[SPEC_MAX_NODES];
+    double pch[SPEC_MAX_NODES];
+    int rej[SPEC_MAX_NODES];
+    double M[MAXCH];
+    uint32_t bitmap[(NT * VPT * 8) / 32];
+    int ivals[8];
+    double dvals[4];
+};
+
+// Combine the per-warp softmax statistics of rows [0, R) into (m, Z, bad).
+__device__ void combine_softmax_rows(const Params& P, int b, int R, FinShared& sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = P.nch * NWARP;
+    for (int r = warp; r < R; r += NWARP) {
+        const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        float m = -INFINITY;
+        bool bad = false;
+#pragma unroll 4
+        for (int e = lane; e < E; e += 32) {
+            float2 x = ldcg2(st + e);
+            m = fmaxf(m, x.x);
+            bad |= (x.y != x.y);
+        }
+        m = warp_max(m);
+        bad = __any_sync(FULL, bad);
+        double z = 0.0;
+        if (m > -INFINITY && !bad) {
+#pragma unroll 4
+            for (int e = lane; e < E; e += 32) {
+                float2 x = ldcg2(st + e);
+                if (x.x > -INFINITY) z += (double)x.y * (double)ex2(x.x - m);
+            }
+        }
+        z = warp_sum_d(z);
+        if (lane == 0) {
+            sh.m[r] = m;
+            sh.z[r] = z;
+            sh.bad[r] = bad || !(m > -INFINITY) || !(m < INFINITY) || !(z > 0.0) || !(z < 1e300);
+        }
+    }
+}
+
+// p(x) of one element, fp64 exp2, in the units of the row statistics.
+__device__ __forceinline__ double prob_d(float l, float s, float m, double z) {
+    return exp2((double)l * (double)s - (double)m) / z;
+}
+
+// Eight consecutive elements e0..e0+7 of a row (e0 a multiple of 8) as f32;
+// elements at or past V read as `fill`.
+template <int DT> __device__ __forceinline__ void ld8(const char* row, int64_t e0, int V, float fill,
+                                                      float (&x)[8]) {
+    if constexpr (DT == SPEC_BF16) {
+        if (e0 + 8 <= V) {
+            uint4 v = ld_stream(row + e0 * 2);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = vec_elem<DT>(v, i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i) : fill;
+        }
+    } else {
+        if (e0 + 8 <= V) {
+            uint4 a = ld_stream(row + e0 * 4), b = ld_stream(row + e0 * 4 + 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { x[i] = vec_elem<DT>(a, i); x[4 + i] = vec_elem<DT>(b, i); }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i) : fill;
+        }
+    }
+}
+
+__device__ __forceinline__ bool excluded(const uint32_t* bitmap, int base, int64_t j) {
+    const int o = (int)(j - base);
+    return (bitmap[o >> 5] >> (o & 31)) & 1u;
+}
+
+// Weight functors of the inverse-CDF draws.  group(e0, w) gives the (f32)
+// weights of elements e0..e0+7 (0 past V); chunk sums and rescans both use it.
+template <int TDT> struct WTarget {          // 2^(x_j - m), excluded tokens 0
+    const char* row; float s, m; const uint32_t* bitmap; int base; int V;
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8];
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            w[i] = ex2(fmaf(x[i], s, -m));
+            if (bitmap && e0 + i < V && excluded(bitmap, base, e0 + i)) w[i] = 0.f;
+        }
+    }
+};
+template <int TDT, int DDT, int DK> struct WChainRes {   // max(0, p_j - q_j)
+    const char* trow; const char* drow; float s, mp, izp, mq, izq; int V;
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8<TDT>(trow, e0, V, -INFINITY, x);
+        if constexpr (DK == DK_PROBS) ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        else ld8<DDT>(drow, e0, V, -INFINITY, d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float p = ex2(fmaf(x[i], s, -mp)) * izp;
+            const float q = (DK == DK_PROBS) ? d[i] : ex2(fmaf(d[i], s, -mq)) * izq;
+            w[i] = fmaxf(0.f, p - q);
+        }
+    }
+};
+template <int TDT> struct WTreeRes {         // relu(p_j - d_j), excluded tokens 0
+    const char* row; const char* drow; float s, m, iz; const uint32_t* bitmap; int base; int V;
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+        ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            w[i] = fmaxf(0.f, ex2(fmaf(x[i], s, -m)) * iz - d[i]);
+            if (bitmap && e0 + i < V && excluded(bitmap, base, e0 + i)) w[i] = 0.f;
+        }
+    }
+};
+
+// Sum of the weights of chunk c, per thread (groups g = k*NT + tid, coalesced).
+template <int CH, class WF>
+__device__ __forceinline__ float chunk_weight_partial(const WF& wf, int c) {
+    constexpr int GPT = CH / 8 / NT;
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < GPT; ++k) {
+        const int64_t e0 = (int64_t)c * CH + (int64_t)(k * NT + threadIdx.x) * 8;
+        if (e0 < wf.V) {
+            float w[8];
+            wf.group(e0, w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc += w[i];
+        }
+    }
+    return acc;
+}
+
+// Inverse-CDF rescan of chunk c: the chunk is read as coalesced 8-element
+// groups (group g covers elements c*CH + 8g .. +7, thread tid owns groups
+// g = k*NT + tid), group sums are scanned block-wide in fp64 in index order,
+// and the thread owning t_loc recomputes its group and walks its 8 weights.
+// If t_loc < 0, t_loc = u * (chunk total) (single-chunk rows).  Returns the
+// drawn index, or -1 when the chunk has no positive weight; *chunk_total gets
+// the chunk's sum.
+template <int CH, class WF>
+__device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, double* chunk_total) {
+    constexpr int GPT = CH / 8 / NT;
+    __shared__ double wt[GPT][NWARP];
+    __shared__ int owner, found;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float gs[GPT];
+#pragma unroll
+    for (int k = 0; k < GPT; ++k) {
+        gs[k] = 0.f;
+        const int64_t e0 = (int64_t)c * CH + (int64_t)(k * NT + tid) * 8;
+        if (e0 < V) {
+            float w[8];
+            wf.group(e0, w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gs[k] += w[i];
+        }
+    }
+    double inc[GPT];
+#pragma unroll
+    for (int k = 0; k < GPT; ++k) {
+        inc[k] = (double)gs[k];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            double n = __shfl_up_sync(FULL, inc[k], o);
+            if (lane >= o) inc[k] += n;
+        }
+        if (lane == 31) wt[k][warp] = inc[k];
+    }
+    if (tid == 0) { owner = -1; found = -1; }
+    __syncthreads();
+    double total = 0.0;
+#pragma unroll
+    for (int k = 0; k < GPT; ++k)
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) total += wt[k][w];
+    if (chunk_total) *chunk_total = total;
+    if (t_loc < 0.0) t_loc = (double)u * total;
+    double base = 0.0;
+#pragma unroll
+    for (int k = 0; k < GPT; ++k) {
+        double before = base;
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) if (w < warp) before += wt[k][w];
+        const double excl = before + inc[k] - (double)gs[k];
+        if (gs[k] > 0.f && excl <= t_loc) atomicMax(&owner, k * NT + tid);
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) base += wt[k][w];
+    }
+    __syncthreads();
+    const int og = owner;
+    if (og >= 0 && (og % NT) == tid) {
+        const int k = og / NT;
+        double before = 0.0;
+        for (int kk = 0; kk < k; ++kk)
+            for (int w = 0; w < NWARP; ++w) before += wt[kk][w];
+        for (int w = 0; w < warp; ++w) before += wt[k][w];
+        double excl = 0.0;
+#pragma unroll
+        for (int kk = 0; kk < GPT; ++kk)
+            if (kk == k) excl = before + inc[kk] - (double)gs[kk];
+        const int64_t e0 = (int64_t)c * CH + (int64_t)og * 8;
+        float w[8];
+        wf.group(e0, w);
+        const double loc = t_loc - excl;
+        double acc = 0.0;
+        int pick = -1, last = -1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            acc += (double)w[i];
+            if (w[i] > 0.f) {
+                last = (int)(e0 + i);
+                if (pick < 0 && loc < acc) pick = (int)(e0 + i);
+            }
+        }
+        found = pick >= 0 ? pick : last;
+    }
+    __syncthreads();
+    const int r = found;
+    __syncthreads();
+    return r;
+}
+
+// Inverse-CDF draw from the target row `row` (statistics st: nch*NWARP entries)
+// with the tokens in excl[0..nexcl) removed.  Chunk masses come from the
+// statistics (fp64), excluded tokens are subtracted from their chunk, the
+// chunk holding u*S is rescanned.  *S_unnorm = remaining mass in units of
+// 2^(x - m).  Returns the token (or -1 if nothing is left).
+template <int TDT>
+__device__ int sample_target_row(const char* row, int V, int nch, const float2* st, float s, float m,
+                                 float u, const int* excl, int nexcl, FinShared& sh, double* S_unnorm) {
+    constexpr int CH = chunk_elems<TDT>();
+    const int tid = threadIdx.x;
+    for (int c = tid; c < nch; c += NT) {
+        double M = 0.0;
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) {
+            float2 x = ldcg2(st + c * NWARP + w);
+            if (x.x > -INFINITY) M += (double)x.y * (double)ex2(x.x - m);
+        }
+        sh.M[c] = M;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int i = 0; i < nexcl; ++i) {
+            int t = excl[i];
+            bool dup = false;
+            for (int j = 0; j < i; ++j) dup |= (excl[j] == t);
+            if (dup) continue;
+            double e = exp2((double)ld_elem<TDT>(row, t) * (double)s - (double)m);
+            double& M = sh.M[t / CH];
+            M = fmax(0.0, M - e);
+        }
+        double S = 0.0;
+        for (int c = 0; c < nch; ++c) S += sh.M[c];
+        sh.dvals[0] = S;
+    }
+    __syncthreads();
+    const double S = sh.dvals[0];
+    *S_unnorm = S;
+    const double t = (double)u * S;
+    int result = -1;
+    for (int attempt = 0; attempt < nch; ++attempt) {
+        if (tid == 0) {
+            double C = 0.0;
+            int cs = -1;
+            double before = 0.0;
+            for (int c = 0; c < nch; ++c) {
+                if (sh.M[c] <= 0.0) continue;
+                if (t < C + sh.M[c]) { cs = c; before = C; break; }
+                C += sh.M[c];
+            }
+            if (cs < 0) {                       // rounding past the end: last chunk with mass
+                for (int c = nch - 1; c >= 0; --c)
+                    if (sh.M[c] > 0.0) { cs = c; break; }
+                before = C - (cs >= 0 ? sh.M[cs] : 0.0);
+            }
+            sh.ivals[0] = cs;
+            sh.dvals[1] = before;
+        }
+        __syncthreads();
+        const int cs = sh.ivals[0];
+        if (cs < 0) break;
+        for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+        __syncthreads();
+        for (int i = tid; i < nexcl; i += NT) {
+            int o = excl[i] - cs * CH;
+            if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+        }
+        __syncthreads();
+        WTarget<TDT> wf{row, s, m, nexcl ? sh.bitmap : nullptr, cs * CH, V};
+        double tot;
+        result = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+        if (result >= 0) break;
+        if (tid == 0) sh.M[cs] = 0.0;         // nothing positive there after all: skip it
+        __syncthreads();
+    }
+    return result;
+}
+
+// Validate a tree held in sh.par / sh.tok (N nodes); returns 1 if well formed.
+__device__ int tree_valid(const Params& P, int N, int V, int max_depth, FinShared& sh) {
+    __shared__ int ok;
+    if (threadIdx.x == 0) ok = 1;
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += NT) {
+        int pa = sh.par[n];
+        bool good = (n == 0) ? (pa == -1) : (pa >= 0 && pa < n && sh.tok[n] >= 0 && sh.tok[n] < V);
+        if (!good) ok = 0;
+    }
+    __syncthreads();
+    if (ok) {
+        for (int n = threadIdx.x; n < N; n += NT) {
+            int d = 0, a = n;
+            while (a > 0 && d <= max_depth) { a = sh.par[a]; ++d; }
+            if (d > max_depth) ok = 0;
+        }
+    }
+    __syncthreads();
+    int r = ok;
+    __syncthreads();
+    return r;
+}
+
+// ----------------------------------------------------------------------------- finalisers
+
+// Chain decision for sequence b (rule 1), computed by thread 0 after the row
+// statistics were combined into sh.m / sh.z / sh.bad.  Writes sh.ivals[0] =
+// valid, sh.ivals[1] = k, sh.dvals[0] = s.  When `write` is set it also writes
+// the accepted tokens, the -1 tail (position k excluded), num_accepted and the
+// p/q diagnostics, and flags invalid sequences.
+template <int TDT, int DDT, int DK>
+__device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write) {
+    const int gamma = P.gamma, V = P.V, W = gamma + 1;
+    int32_t* toks = P.out_tokens + (size_t)b * W;
+    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+    const float T = P.temperature[b];
+    bool ok = temperature_ok(T);
+    for (int r = 0; r < P.R; ++r) ok &= !sh.bad[r];
+    const int32_t* x = P.draft_tokens + (size_t)b * gamma;
+    for (int i = 0; i < gamma; ++i) ok &= (x[i] >= 0 && x[i] < V);
+    const float s = ok ? scale_of(T) : 0.f;
+    int k = gamma;
+    if (ok) {
+        // p_i(x_i), q_i(x_i) for every position (diagnostics), then rule 1.
+        double pr[SPEC_MAX_GAMMA], qr[SPEC_MAX_GAMMA];
+        for (int i = 0; i < gamma; ++i) {
+            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride;
+            const char* drow = P.drf + ((size_t)b * gamma + i) * P.dstride;
+            pr[i] = prob_d(ld_elem<TDT>(trow, x[i]), s, sh.m[i], sh.z[i]);
+            if constexpr (DK == DK_PROBS) {
+                qr[i] = (double)__ldg(reinterpret_cast<const float*>(drow) + x[i]);
+                ok &= (qr[i] >= 0.0 && qr[i] <= 3.0e38);
+            } else {
+                qr[i] = prob_d(ld_elem<DDT>(drow, x[i]), s, sh.m[gamma + 1 + i], sh.z[gamma + 1 + i]);
+            }
+            if (dg && write) { dg[i] = (float)pr[i]; dg[gamma + i] = (float)qr[i]; }
+        }
+        for (int i = 0; i < gamma && ok; ++i) {
+            const double ratio = (qr[i] > 0.0) ? pr[i] / qr[i] : INFINITY;
+            if (!((double)P.coins[(size_t)b * gamma + i] <= ratio)) { k = i; break; }
+        }
+    }
+    sh.ivals[0] = ok;
+    sh.ivals[1] = k;
+    sh.dvals[0] = (double)s;
+    if (!write) return;
+    if (!ok) {
+        for (int i = 0; i < W; ++i) toks[i] = -1;
+        P.out_num_accepted[b] = -1;
+        if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
+        flag_input_error(P);
+    } else {
+        for (int i = 0; i < k; ++i) toks[i] = x[i];
+        for (int i = k + 1; i < W; ++i) toks[i] = -1;
+        P.out_num_accepted[b] = k;
+    }
+}
+
+template <int TDT>
+__device__ void finalize_greedy(const Params& P, int b, FinShared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = P.N, V = P.V, W = P.max_depth + 1;
+    const int E = P.nch * NWARP;
+    // per-node argmax (lowest index among equal maxima)
+    for (int r = warp; r < N; r += NWARP) {
+        const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        float best = -INFINITY;
+        int idx = 0x7fffffff;
+        bool bad = false;
+        for (int e = lane; e < E; e += 32) {
+            float2 x = ldcg2(st + e);
+            int xi = __float_as_int(x.y);
+            if (x.x != x.x) bad = true;
+            else if (x.x > best || (x.x == best && xi < idx)) { best = x.x; idx = xi; }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            float ov = __shfl_xor_sync(FULL, best, o);
+            int oi = __shfl_xor_sync(FULL, idx, o);
+            if (ov > best || (ov == best && oi < idx)) { best = ov; idx = oi; }
+        }
+        bad = __any_sync(FULL, bad);
+        if (lane == 0) { sh.rej[r] = idx; sh.bad[r] = bad; }
+    }
+    for (int n = tid; n < N; n += NT) {
+        sh.par[n] = P.parents[(size_t)b * N + n];
+        sh.tok[n] = P.tokens[(size_t)b * N + n];
+    }
+    __syncthreads();
+    int ok = tree_valid(P, N, V, P.max_depth, sh);
+    if (tid == 0) {
+        for (int r = 0; r < N; ++r) ok &= !sh.bad[r];
+        sh.ivals[0] = ok;
+    }
+    __syncthreads();
+    ok = sh.ivals[0];
+    int32_t* ai = P.out_accept_index + (size_t)b * W;
+    int32_t* ot = P.out_tokens + (size_t)b * W;
+    if (!ok) {
+        for (int i = tid; i < W; i += NT) { ai[i] = -1; ot[i] = -1; }
+        if (tid == 0) { P.out_num_accepted[b] = -1; flag_input_error(P); }
+        return;
+    }
+    if (warp == 0) {
+        const int* g = sh.rej;
+        int cur = 0, k = 0;
+        if (lane == 0) ai[0] = 0;
+        for (;;) {
+            int next = -1;
+            for (int base = cur + 1; base < N && next < 0; base += 32) {
+                int c = base + lane;
+                bool hit = c < N && sh.par[c] == cur && sh.tok[c] == g[cur];
+                unsigned m = __ballot_sync(FULL, hit);
+                if (m) next = base + __ffs(m) - 1;
+            }
+            if (next < 0) break;
+            if (lane == 0) { ot[k] = sh.tok[next]; ai[k + 1] = next; }
+            ++k;
+            cur = next;
+        }
+        if (lane == 0) {
+            ot[k] = g[cur];
+            for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+            P.out_num_accepted[b] = k;
+        }
+    }
+}
+
+template <int TDT>
+__device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = P.N, V = P.V, W = P.max_depth + 1;
+    combine_softmax_rows(P, b, N, sh);
+    for (int n = tid; n < N; n += NT) {
+        sh.par[n] = P.parents[(size_t)b * N + n];
+        sh.tok[n] = P.tokens[(size_t)b * N + n];
+    }
+    __syncthreads();
+    int ok = tree_valid(P, N, V, P.max_depth, sh);
+    const float T = P.temperature[b];
+    if (tid == 0) {
+        ok &= temperature_ok(T);
+        for (int r = 0; r < N; ++r) ok &= !sh.bad[r];
+        sh.ivals[0] = ok;
+    }
+    __syncthreads();
+    ok = sh.ivals[0];
+    int32_t* ai = P.out_accept_index + (size_t)b * W;
+    int32_t* ot = P.out_tokens + (size_t)b * W;
+    float* dg = P.diag ? P.diag + (size_t)b * (N + 1) : nullptr;
+    if (!ok) {
+        for (int i = tid; i < W; i += NT) { ai[i] = -1; ot[i] = -1; }
+        if (dg) for (int i = tid; i < N + 1; i += NT) dg[i] = nanf_();
+        if (tid == 0) { P.out_num_accepted[b] = -1; flag_input_error(P); }
+        return;
+    }
+    const float s = scale_of(T);
+    // p_parent(n)(tokens[n]) for every non-root node
+    for (int n = tid; n < N; n += NT) {
+        double pc = 0.0;
+        if (n > 0) {
+            int pa = sh.par[n];
+            const char* row = P.tgt + ((size_t)b * N + pa) * P.tstride;
+            pc = prob_d(ld_elem<TDT>(row, sh.tok[n]), s, sh.m[pa], sh.z[pa]);
+        }
+        sh.pch[n] = pc;
+        if (dg) dg[n] = (float)pc;
+    }
+    __syncthreads();
+    // sibling walk with prob_acc
+    if (warp == 0) {
+        const double ths = (double)P.th_single, tha = (double)P.th_acc;
+        int cur = 0, k = 0, nrej = 0;
+        if (lane == 0) ai[0] = 0;
+        for (;;) {
+            const double coin = (double)P.coins[(size_t)b * N + cur];
+            double acc = 0.0;
+            int next = -1;
+            nrej = 0;
+            for (int base = cur + 1; base < N && next < 0; base += 32) {
+                int c = base + lane;
+                unsigned m = __ballot_sync(FULL, c < N && sh.par[c] == cur);
+                if (lane == 0) {
+                    while (m && next < 0) {
+                        int cc = base + __ffs(m) - 1;
+                        m &= m - 1;
+                        double pc = sh.pch[cc];
+                        acc += pc;
+                        if (coin <= acc / tha || pc >= ths) next = cc;
+                        else sh.rej[nrej++] = sh.tok[cc];
+                    }
+                }
+                next = __shfl_sync(FULL, next, 0);
+            }
+            if (next < 0) break;
+            if (lane == 0) { ot[k] = sh.tok[next]; ai[k + 1] = next; }
+            ++k;
+            cur = next;
+        }
+        if (lane == 0) { sh.ivals[1] = cur; sh.ivals[2] = k; sh.ivals[3] = nrej; }
+    }
+    __syncthreads();
+    const int cur = sh.ivals[1], k = sh.ivals[2], nrej = sh.ivals[3];
+    const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
+    const float u = P.final_u[b];
+    int y;
+    double S;
+    if (!P.draft_probs) {
+        const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * NWARP;
+        double Su;
+        y = sample_target_row<TDT>(row, V, P.nch, st, s, sh.m[cur], u, sh.rej, nrej, sh, &Su);
+        S = Su / sh.z[cur];
+    } else {
+        // relu(p_cur - d_cur) over the whole row: chunk sums, then one rescan.
+        constexpr int CH = chunk_elems<TDT>();
+        const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * N + cur) * P.dpstride;
+        const float m = sh.m[cur], iz = (float)(1.0 / sh.z[cur]);
+        for (int c = 0; c < P.nch; ++c) {
+            for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+            __syncthreads();
+            for (int i = tid; i < nrej; i += NT) {
+                int o = sh.rej[i] - c * CH;
+                if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+            }
+            __syncthreads();
+            WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, c * CH, V};
+            double part = (double)chunk_weight_partial<CH>(wf, c);
+            part = warp_sum_d(part);
+            if (lane == 0) sh.dvals[warp % 4] = part;     // NWARP == 4
+            __syncthreads();
+            if (tid == 0) sh.M[c] = sh.dvals[0] + sh.dvals[1] + sh.dvals[2] + sh.dvals[3];
+            __syncthreads();
+        }
+        if (tid == 0) {
+            double tot = 0.0;
+            for (int c = 0; c < P.nch; ++c) tot += sh.M[c];
+            sh.dvals[0] = tot;
+        }
+        __syncthreads();
+        S = sh.dvals[0];
+        y = -1;
+        if (S > 0.0) {
+            const double t = (double)u * S;
+            for (int attempt = 0; attempt < P.nch && y < 0; ++attempt) {
+                if (tid == 0) {
+                    double C = 0.0, before = 0.0;
+                    int cs = -1;
+                    for (int c = 0; c < P.nch; ++c) {
+                        if (sh.M[c] <= 0.0) continue;
+                        if (t < C + sh.M[c]) { cs = c; before = C; break; }
+                        C += sh.M[c];
+                    }
+                    if (cs < 0)
+                        for (int c = P.nch - 1; c >= 0; --c)
+                            if (sh.M[c] > 0.0) { cs = c; before = C - sh.M[c]; break; }
+                    sh.ivals[4] = cs;
+                    sh.dvals[1] = before;
+                }
+                __syncthreads();
+                const int cs = sh.ivals[4];
+                if (cs < 0) break;
+                for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+                __syncthreads();
+                for (int i = tid; i < nrej; i += NT) {
+                    int o = sh.rej[i] - cs * CH;
+                    if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+                }
+                __syncthreads();
+                WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, cs * CH, V};
+                double tot;
+                y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+                if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+                __syncthreads();
+            }
+        }
+        if (y < 0) {
+            // empty residual (rounding only): draw from p_cur itself
+            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * NWARP;
+            double Su;
+            y = sample_target_row<TDT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
+        }
+    }
+    if (tid == 0) {
+        ot[k] = y;
+        for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+        P.out_num_accepted[b] = k;
+        if (dg) dg[N] = (float)S;
+    }
+}
+
+// ----------------------------------------------------------------------------- kernels
+
+// Row statistics (the streaming kernel).  The B*R*nch work items (sequence-
+// major, then row, then chunk) are split into gridDim.x contiguous ranges,
+// one per CTA.  Each warp writes one statistic per item; nothing else is
+// shared, so the kernel has no atomics and no fences: the finalize kernel
+// that follows in stream order reads the statistics.
+template <int MODE, int TDT, int DDT>
+__global__ void __launch_bounds__(NT) k_stats(const Params P) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int per_seq = P.R * P.nch;
+    const long long total = (long long)P.B * per_seq;
+    const long long lo = total * blockIdx.x / gridDim.x;
+    const long long hi = total * (blockIdx.x + 1) / gridDim.x;
+    for (long long item = lo; item < hi; ++item) {
+        const int b = (int)(item / per_seq);
+        const int rem = (int)(item - (long long)b * per_seq);
+        const int r = rem / P.nch, c = rem - r * P.nch;
+        float2 stat;
+        if constexpr (MODE == MODE_GREEDY) {
+            const char* row = P.tgt + ((size_t)b * P.R + r) * P.tstride;
+            stat = chunk_argmax<TDT>(row, P.V, c);
+        } else {
+            const float s = scale_of(__ldg(P.temperature + b));
+            if (r < P.rows_tgt) {
+                const char* row = P.tgt + ((size_t)b * P.rows_tgt + r) * P.tstride;
+                stat = chunk_softmax<TDT, chunk_elems<TDT>()>(row, P.V, c, s);
+            } else {
+                const char* row = P.drf + ((size_t)b * (P.R - P.rows_tgt) + (r - P.rows_tgt)) * P.dstride;
+                stat = chunk_softmax<DDT, chunk_elems<TDT>()>(row, P.V, c, s);
+            }
+        }
+        if (lane == 0) P.stats[(((size_t)b * P.R + r) * P.nch + c) * NWARP + warp] = stat;
+    }
+}
+
+// Chain finalisation, grid = B * nch: CTA (b, c) recomputes sequence b's
+// decision from the row statistics (cheap, identical in every CTA), then
+//  - k = gamma: CTA c = 0 draws the bonus token from p_gamma (rule 3);
+//  - k < gamma, one chunk per row: CTA 0 draws the correction directly;
+//  - k < gamma, several chunks: every CTA sums max(0, p_k - q_k) over its
+//    chunk; the last CTA of the sequence to arrive locates the chunk holding
+//    u*S and rescans it (rule 2).
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
+    __shared__ FinShared sh;
+    __shared__ int is_last;
+    constexpr int CH = chunk_elems<TDT>();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x / P.nch, c = blockIdx.x - b * P.nch;
+    const int gamma = P.gamma, V = P.V;
+    combine_softmax_rows(P, b, P.R, sh);
+    __syncthreads();
+    if (tid == 0) chain_decide<TDT, DDT, DK>(P, b, sh, c == 0);
+    __syncthreads();
+    const int ok = sh.ivals[0], k = sh.ivals[1];
+    const float s = (float)sh.dvals[0];
+    if (!ok) return;
+    const float u = P.final_u[b];
+    int32_t* toks = P.out_tokens + (size_t)b * (gamma + 1);
+    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
+    if (k == gamma) {
+        if (c != 0) return;
+        const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * NWARP;
+        double S;
+        int y = sample_target_row<TDT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        if (tid == 0) {
+            toks[k] = y;
+            if (dg) dg[2 * gamma] = 1.0f;
+        }
+        return;
+    }
+    const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
+    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]);
+    const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
+    const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
+    WChainRes<TDT, DDT, DK> wf{trow, drow, s, mp, izp, mq, izq, V};
+    const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * NWARP;
+    if (P.nch == 1) {
+        double S;
+        int y = rescan_chunk<CH>(wf, 0, V, -1.0, u, &S);
+        if (y < 0 || !(S > 0.0)) {
+            double S2;
+            y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &S2);
+        }
+        if (tid == 0) {
+            toks[k] = y;
+            if (dg) dg[2 * gamma] = (float)S;
+        }
+        return;
+    }
+    const float ws = warp_sum(chunk_weight_partial<CH>(wf, c));
+    if (lane == 0) {
+        P.stats2[((size_t)b * P.nch + c) * NWARP + warp] = make_float2(ws, 0.f);
+        __threadfence();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(P.cnt2 + b, 1u);
+        is_last = (prev == (unsigned)P.nch - 1u);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int cc = tid; cc < P.nch; cc += NT) {
+        double M = 0.0;
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) M += (double)ldcg2(P.stats2 + ((size_t)b * P.nch + cc) * NWARP + w).x;
+        sh.M[cc] = M;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double S = 0.0;
+        for (int cc = 0; cc < P.nch; ++cc) S += sh.M[cc];
+        sh.dvals[0] = S;
+    }
+    __syncthreads();
+    const double S = sh.dvals[0];
+    int y = -1;
+    if (S > 0.0) {
+        const double t = (double)u * S;
+        for (int attempt = 0; attempt < P.nch && y < 0; ++attempt) {
+            if (tid == 0) {
+                double C = 0.0, before = 0.0;
+                int cs = -1;
+                for (int cc = 0; cc < P.nch; ++cc) {
+                    if (sh.M[cc] <= 0.0) continue;
+                    if (t < C + sh.M[cc]) { cs = cc; before = C; break; }
+                    C += sh.M[cc];
+                }
+                if (cs < 0)
+                    for (int cc = P.nch - 1; cc >= 0; --cc)
+                        if (sh.M[cc] > 0.0) { cs = cc; before = C - sh.M[cc]; break; }
+                sh.ivals[2] = cs;
+                sh.dvals[1] = before;
+            }
+            __syncthreads();
+            const int cs = sh.ivals[2];
+            if (cs < 0) break;
+            double tot;
+            y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+            if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+            __syncthreads();
+        }
+    }
+    if (y < 0) {
+        // empty residual (rounding only): draw from p_k
+        double Su;
+        y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+    }
+    if (tid == 0) {
+        toks[k] = y;
+        if (dg) dg[2 * gamma] = (float)S;
+        __threadfence();
+        P.cnt2[b] = 0u;
+    }
+}
+
+// Tree finalisation, one CTA per sequence.
+template <int MODE, int TDT>
+__global__ void __launch_bounds__(NT) k_tree_final(const Params P) {
+    __shared__ FinShared sh;
+    if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT>(P, blockIdx.x, sh);
+    else finalize_sample<TDT>(P, blockIdx.x, sh);
+}
+
+}  // namespace sv
+
+// ============================================================================= host side
+
+using namespace sv;
+
+namespace {
+
+thread_local char g_detail[512];
+thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+
+cudaError_t record(cudaEvent_t ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return e;
+    return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                                               : cudaEventRecord(ev, st);
+}
+
+spec_status fail(spec_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+    size_t status, cnt2, stats, stats2, total;
+    int R, nch_max;
+};
+
+// Chunks are sized for the widest element (f32: 4096 per chunk) so that one
+// workspace size serves both input dtypes.
+Layout make_layout(int entry, int B, int rows, int V) {
+    Layout L{};
+    const int nch = (V + chunk_elems<SPEC_F32>() - 1) / chunk_elems<SPEC_F32>();
+    L.nch_max = nch;
+    L.R = (entry == SPEC_ENTRY_CHAIN) ? 2 * rows + 1 : rows;
+    size_t off = 0;
+    L.status = off; off = align256(off + 16);
+    L.cnt2 = off; off = align256(off + sizeof(unsigned) * (size_t)B);
+    L.stats = off; off = align256(off + sizeof(float2) * (size_t)B * L.R * nch * NWARP);
+    L.stats2 = off;
+    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(float2) * (size_t)B * nch * NWARP);
+    L.total = off;
+    return L;
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <class K>
+int blocks_per_sm(K kernel) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, NT, 0) != cudaSuccess || n <= 0) n = 1;
+    return n;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+spec_status check_rows(const char* what, const void* p, spec_dtype dt, int64_t stride, int V) {
+    if (!p) return fail(SPEC_ERR_INVALID_ARG, "%s is NULL", what);
+    if (dt != SPEC_F32 && dt != SPEC_BF16) return fail(SPEC_ERR_INVALID_ARG, "%s: unknown dtype %d", what, (int)dt);
+    if (stride < V) return fail(SPEC_ERR_INVALID_ARG, "%s: row stride %lld < V %d", what, (long long)stride, V);
+    const int esz = dt == SPEC_F32 ? 4 : 2;
+    if (!aligned16(p)) return fail(SPEC_ERR_INVALID_ARG, "%s: base pointer not 16-byte aligned", what);
+    if ((stride * esz) % 16 != 0)
+        return fail(SPEC_ERR_INVALID_ARG, "%s: row stride * element size (%lld bytes) not a multiple of 16",
+                    what, (long long)(stride * esz));
+    return SPEC_OK;
+}
+
+spec_status check_ws(void* ws, size_t bytes, const Layout& L) {
+    if (!ws) return fail(SPEC_ERR_WORKSPACE, "workspace is NULL");
+    if (((uintptr_t)ws & 255u) != 0) return fail(SPEC_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    if (bytes < L.total)
+        return fail(SPEC_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", bytes, L.total);
+    return SPEC_OK;
+}
+
+void bind_ws(Params& P, void* ws, const Layout& L) {
+    char* w = static_cast<char*>(ws);
+    P.status = reinterpret_cast<unsigned*>(w + L.status);
+    P.cnt2 = reinterpret_cast<unsigned*>(w + L.cnt2);
+    P.stats = reinterpret_cast<float2*>(w + L.stats);
+    P.stats2 = reinterpret_cast<float2*>(w + L.stats2);
+}
+
+spec_status launched(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return SPEC_OK;
+}
+
+template <int MODE, int TDT, int DDT>
+spec_status launch_stats(const Params& P, cudaStream_t st) {
+    auto kern = k_stats<MODE, TDT, DDT>;
+    static const int occ = blocks_per_sm(kern);
+    const long long items = (long long)P.B * P.R * P.nch;
+    long long grid = (long long)num_sms() * occ;
+    if (grid > items) grid = items;
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    kern<<<(unsigned)grid, NT, 0, st>>>(P);
+    spec_status s = launched("k_stats");
+    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
+        return fail(SPEC_ERR_CUDA, "profile event");
+    return s;
+}
+
+template <int TDT, int DDT, int DK>
+spec_status launch_chain(const Params& P, cudaStream_t st) {
+    spec_status s = launch_stats<MODE_CHAIN, TDT, DDT>(P, st);
+    if (s != SPEC_OK) return s;
+    k_chain_final<TDT, DDT, DK><<<(unsigned)(P.B * P.nch), NT, 0, st>>>(P);
+    return launched("k_chain_final");
+}
+
+template <int MODE, int TDT>
+spec_status launch_tree(const Params& P, cudaStream_t st) {
+    spec_status s = launch_stats<MODE, TDT, TDT>(P, st);
+    if (s != SPEC_OK) return s;
+    k_tree_final<MODE, TDT><<<(unsigned)P.B, NT, 0, st>>>(P);
+    return launched("k_tree_final");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t spec_workspace_bytes(int entry, int B, int rows, int V) {
+    if (B < 0 || V < 1 || V > SPEC_MAX_V) return 0;
+    if (entry == SPEC_ENTRY_CHAIN) {
+        if (rows < 1 || rows > SPEC_MAX_GAMMA) return 0;
+    } else if (entry == SPEC_ENTRY_TREE_GREEDY || entry == SPEC_ENTRY_TREE_SAMPLE) {
+        if (rows < 1 || rows > SPEC_MAX_NODES) return 0;
+    } else {
+        return 0;
+    }
+    return make_layout(entry, B, rows, V).total;
+}
+
+spec_status spec_workspace_init(void* workspace, size_t bytes, void* stream) {
+    if (!workspace) return fail(SPEC_ERR_WORKSPACE, "workspace is NULL");
+    cudaError_t e = cudaMemsetAsync(workspace, 0, bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    return SPEC_OK;
+}
+
+spec_status spec_read_device_status(void* workspace, int* status_out, void* stream) {
+    if (!workspace || !status_out) return fail(SPEC_ERR_INVALID_ARG, "NULL workspace or status_out");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof v, st);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "reading status: %s", cudaGetErrorString(e));
+    *status_out = (int)v;
+    return SPEC_OK;
+}
+
+const char* spec_status_string(spec_status s) {
+    switch (s) {
+        case SPEC_OK: return "ok";
+        case SPEC_ERR_INVALID_ARG: return "invalid argument";
+        case SPEC_ERR_UNSUPPORTED: return "unsupported";
+        case SPEC_ERR_CUDA: return "CUDA error";
+        case SPEC_ERR_DEVICE_INPUT: return "invalid device-side input in a sequence";
+        case SPEC_ERR_TIMEOUT: return "device-side wait timed out";
+        case SPEC_ERR_WORKSPACE: return "workspace too small or misaligned";
+    }
+    return "unknown status";
+}
+
+const char* spec_last_error_detail(void) { return g_detail; }
+
+spec_status spec_profile_events(void* start_event, void* stop_event) {
+    g_prof_start = static_cast<cudaEvent_t>(start_event);
+    g_prof_stop = static_cast<cudaEvent_t>(stop_event);
+    return SPEC_OK;
+}
+
+spec_status spec_verify_chain(int B, int gamma, int V,
+                              const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                              const void* draft, spec_dtype ddt, int draft_is_probs,
+                              int64_t d_row_stride,
+                              const int32_t* draft_tokens, const float* temperature,
+                              const float* coins, const float* final_u,
+                              int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
+    if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
+    if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
+    if (B == 0) return SPEC_OK;
+    spec_status s = check_rows("target_logits", target_logits, tdt, t_row_stride, V);
+    if (s != SPEC_OK) return s;
+    if (draft_is_probs && ddt != SPEC_F32) return fail(SPEC_ERR_INVALID_ARG, "draft probabilities must be SPEC_F32");
+    s = check_rows("draft", draft, ddt, d_row_stride, V);
+    if (s != SPEC_OK) return s;
+    if (!draft_tokens || !temperature || !coins || !final_u || !out_tokens || !out_num_accepted)
+        return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    const Layout L = make_layout(SPEC_ENTRY_CHAIN, B, gamma, V);
+    s = check_ws(workspace, workspace_bytes, L);
+    if (s != SPEC_OK) return s;
+    Params P{};
+    P.B = B; P.V = V; P.gamma = gamma;
+    P.rows_tgt = gamma + 1;
+    P.R = draft_is_probs ? gamma + 1 : 2 * gamma + 1;
+    P.nch = (V + (tdt == SPEC_BF16 ? chunk_elems<SPEC_BF16>() : chunk_elems<SPEC_F32>()) - 1) /
+            (tdt == SPEC_BF16 ? chunk_elems<SPEC_BF16>() : chunk_elems<SPEC_F32>());
+    P.tgt = static_cast<const char*>(target_logits);
+    P.tstride = t_row_stride * (tdt == SPEC_F32 ? 4 : 2);
+    P.drf = static_cast<const char*>(draft);
+    P.dstride = d_row_stride * (ddt == SPEC_F32 ? 4 : 2);
+    P.draft_tokens = draft_tokens; P.temperature = temperature; P.coins = coins; P.final_u = final_u;
+    P.out_tokens = out_tokens; P.out_num_accepted = out_num_accepted; P.diag = diag;
+    bind_ws(P, workspace, L);
+    // The statistics of a row are laid out with the chain's full row count so
+    // that draft rows keep their offsets for either draft kind.
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (draft_is_probs) {
+        if (tdt == SPEC_BF16) return launch_chain<SPEC_BF16, SPEC_F32, DK_PROBS>(P, st);
+        return launch_chain<SPEC_F32, SPEC_F32, DK_PROBS>(P, st);
+    }
+    if (tdt == SPEC_BF16 && ddt == SPEC_BF16) return launch_chain<SPEC_BF16, SPEC_BF16, DK_LOGITS>(P, st);
+    if (tdt == SPEC_BF16 && ddt == SPEC_F32) return launch_chain<SPEC_BF16, SPEC_F32, DK_LOGITS>(P, st);
+    if (tdt == SPEC_F32 && ddt == SPEC_BF16) return launch_chain<SPEC_F32, SPEC_BF16, DK_LOGITS>(P, st);
+    return launch_chain<SPEC_F32, SPEC_F32, DK_LOGITS>(P, st);
+}
+
+static spec_status tree_common(Params& P, int B, int N, int V, int max_depth,
+                               const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                               const int32_t* tokens, const int32_t* parents,
+                               int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted) {
+    if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
+    if (N < 1 || N > SPEC_MAX_NODES) return fail(SPEC_ERR_INVALID_ARG, "N = %d outside [1, %d]", N, SPEC_MAX_NODES);
+    if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
+    if (max_depth < 0 || max_depth > SPEC_MAX_DEPTH)
+        return fail(SPEC_ERR_INVALID_ARG, "max_depth = %d outside [0, %d]", max_depth, SPEC_MAX_DEPTH);
+    if (B == 0) return SPEC_OK;
+    spec_status s = check_rows("target_logits", target_logits, tdt, t_row_stride, V);
+    if (s != SPEC_OK) return s;
+    if (!tokens || !parents || !out_accept_index || !out_tokens || !out_num_accepted)
+        return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    P.B = B; P.N = N; P.V = V; P.max_depth = max_depth;
+    P.R = N; P.rows_tgt = N;
+    const int CH = tdt == SPEC_BF16 ? chunk_elems<SPEC_BF16>() : chunk_elems<SPEC_F32>();
+    P.nch = (V + CH - 1) / CH;
+    P.tgt = static_cast<const char*>(target_logits);
+    P.tstride = t_row_stride * (tdt == SPEC_F32 ? 4 : 2);
+    P.tokens = tokens; P.parents = parents;
+    P.out_accept_index = out_accept_index; P.out_tokens = out_tokens; P.out_num_accepted = out_num_accepted;
+    return SPEC_OK;
+}
+
+spec_status spec_verify_tree_greedy(int B, int N, int V, int max_depth,
+                                    const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                    const int32_t* tokens, const int32_t* parents,
+                                    int32_t* out_accept_index, int32_t* out_tokens,
+                                    int32_t* out_num_accepted,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    Params P{};
+    spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
+                                out_accept_index, out_tokens, out_num_accepted);
+    if (s != SPEC_OK || B == 0) return s;
+    const Layout L = make_layout(SPEC_ENTRY_TREE_GREEDY, B, N, V);
+    s = check_ws(workspace, workspace_bytes, L);
+    if (s != SPEC_OK) return s;
+    bind_ws(P, workspace, L);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (tdt == SPEC_BF16) return launch_tree<MODE_GREEDY, SPEC_BF16>(P, st);
+    return launch_tree<MODE_GREEDY, SPEC_F32>(P, st);
+}
+
+spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
+                                    const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                    const int32_t* tokens, const int32_t* parents,
+                                    const float* temperature, const float* coins, const float* final_u,
+                                    const float* draft_probs, int64_t dp_row_stride,
+                                    float threshold_single, float threshold_acc,
+                                    int32_t* out_accept_index, int32_t* out_tokens,
+                                    int32_t* out_num_accepted, float* diag,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    Params P{};
+    spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
+                                out_accept_index, out_tokens, out_num_accepted);
+    if (s != SPEC_OK || B == 0) return s;
+    if (!temperature || !coins || !final_u) return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!(threshold_single > 0.f) || !(threshold_acc > 0.f))
+        return fail(SPEC_ERR_INVALID_ARG, "thresholds must be > 0");
+    if (draft_probs) {
+        s = check_rows("draft_probs", draft_probs, SPEC_F32, dp_row_stride, V);
+        if (s != SPEC_OK) return s;
+    }
+    const Layout L = make_layout(SPEC_ENTRY_TREE_SAMPLE, B, N, V);
+    s = check_ws(workspace, workspace_bytes, L);
+    if (s != SPEC_OK) return s;
+    bind_ws(P, workspace, L);
+    P.temperature = temperature; P.coins = coins; P.final_u = final_u;
+    P.draft_probs = draft_probs; P.dpstride = dp_row_stride * 4;
+    P.th_single = threshold_single; P.th_acc = threshold_acc;
+    P.diag = diag;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (tdt == SPEC_BF16) return launch_tree<MODE_SAMPLE, SPEC_BF16>(P, st);
+    return launch_tree<MODE_SAMPLE, SPEC_F32>(P, st);
+}
+
+}  // extern "C"

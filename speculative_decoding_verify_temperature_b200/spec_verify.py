@@ -1,0 +1,238 @@
+"""Python binding of libspecverify: the C ABI of ``include/spec_verify.h`` with the
+same names, taking torch CUDA tensors.  Argument marshalling only -- every step
+of the verify path runs in the library's sm_100a kernels; there is no CPU
+fallback, and a missing library raises.
+
+Tensor conventions: logits/probabilities are ``[B, R, S]`` with unit stride in
+the last dim and ``stride(0) == R * stride(1)`` (rows equally spaced); the row
+stride passed to the library is ``stride(1)``.  Outputs are allocated with
+``torch.empty`` when not given.  All calls run on ``torch.cuda.current_stream()``
+unless a stream is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspecverify.so")
+
+SPEC_OK, SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA = 0, 1, 2, 3
+SPEC_ERR_DEVICE_INPUT, SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE = 4, 5, 6
+SPEC_F32, SPEC_BF16 = 0, 1
+SPEC_ENTRY_CHAIN, SPEC_ENTRY_TREE_GREEDY, SPEC_ENTRY_TREE_SAMPLE = 0, 1, 2
+
+_lib = None
+
+
+class SpecError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        detail = lib().spec_last_error_detail().decode()
+        msg = lib().spec_status_string(status).decode()
+        super().__init__(f"{where}: {msg} ({status}){': ' + detail if detail else ''}")
+
+
+def lib():
+    """Load libspecverify.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m speculative_decoding_verify_temperature_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.spec_verify_chain.restype = i32
+        L.spec_verify_chain.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
+                                        P, P, P, P, P, P, P, P, sz, P]
+        L.spec_verify_tree_greedy.restype = i32
+        L.spec_verify_tree_greedy.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, sz, P]
+        L.spec_verify_tree_sample.restype = i32
+        L.spec_verify_tree_sample.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
+                                              f32, f32, P, P, P, P, P, sz, P]
+        L.spec_workspace_bytes.restype = sz
+        L.spec_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.spec_workspace_init.restype = i32
+        L.spec_workspace_init.argtypes = [P, sz, P]
+        L.spec_read_device_status.restype = i32
+        L.spec_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
+        L.spec_status_string.restype = ctypes.c_char_p
+        L.spec_status_string.argtypes = [i32]
+        L.spec_last_error_detail.restype = ctypes.c_char_p
+        L.spec_last_error_detail.argtypes = []
+        L.spec_profile_events.restype = i32
+        L.spec_profile_events.argtypes = [P, P]
+        _lib = L
+    return _lib
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SPEC_BF16
+    if t.dtype == torch.float32:
+        return SPEC_F32
+    raise TypeError(f"logits must be bf16 or f32, got {t.dtype}")
+
+
+def _rows(t: torch.Tensor, name: str) -> int:
+    """Row stride (elements) of a [B, R, S] tensor whose rows are equally spaced.
+    Strides of size-1 dims carry no information and are ignored."""
+    if t.dim() != 3 or (t.shape[2] > 1 and t.stride(2) != 1):
+        raise ValueError(f"{name} must be [B, R, S] with unit stride in the last dim")
+    B, R, S = t.shape
+    if R > 1:
+        rs = t.stride(1)
+    elif B > 1:
+        rs = t.stride(0)
+    else:
+        q = 16 // t.element_size()
+        rs = -(-S // q) * q
+    if B > 1 and R > 1 and t.stride(0) != R * rs:
+        raise ValueError(f"{name}: rows must be equally spaced (stride(0) == R * stride(1))")
+    return rs
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != SPEC_OK:
+        raise SpecError(status, where)
+
+
+def spec_workspace_bytes(entry: int, B: int, rows: int, V: int) -> int:
+    return int(lib().spec_workspace_bytes(entry, B, rows, V))
+
+
+def spec_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _check(lib().spec_workspace_init(_p(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)), "spec_workspace_init")
+
+
+def spec_read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().spec_read_device_status(_p(workspace), ctypes.byref(v), _stream(stream)),
+           "spec_read_device_status")
+    return v.value
+
+
+def spec_profile_events(start=None, stop=None) -> None:
+    """Record ``start``/``stop`` (torch.cuda.Event) around the row kernel of later
+    calls on this thread; ``spec_profile_events()`` switches it off."""
+    for ev in (start, stop):
+        if ev is not None and not ev.cuda_event:
+            ev.record()                        # torch creates the CUDA event on first record
+    a = None if start is None else ctypes.c_void_p(start.cuda_event)
+    b = None if stop is None else ctypes.c_void_p(stop.cuda_event)
+    _check(lib().spec_profile_events(a, b), "spec_profile_events")
+
+
+class Workspace:
+    """Caller-owned scratch for one entry point and shape, zero-filled on creation
+    (and re-created whenever the shape changes)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.key = None
+        self.buf = None
+
+    def get(self, entry: int, B: int, rows: int, V: int, stream=None) -> torch.Tensor:
+        key = (entry, B, rows, V)
+        if key != self.key:
+            n = spec_workspace_bytes(entry, B, rows, V)
+            if n == 0:
+                raise ValueError(f"no workspace size for {key}")
+            self.buf = torch.empty(n, dtype=torch.uint8, device=self.device)
+            spec_workspace_init(self.buf, stream)
+            self.key = key
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(workspace, entry, B, rows, V, device, stream):
+    if workspace is not None:
+        return workspace
+    w = _default_ws.setdefault((device, entry), Workspace(device))
+    return w.get(entry, B, rows, V, stream)
+
+
+def spec_verify_chain(target, draft, draft_tokens, temperature, coins, final_u, *,
+                      draft_is_probs: bool = False, V: int | None = None, out_tokens=None,
+                      out_num_accepted=None, diag=None, workspace=None, stream=None):
+    """Chain verify of one round.  Returns ``(out_tokens [B, gamma+1], out_num_accepted [B])``."""
+    B, R, S = target.shape
+    gamma = R - 1
+    V = S if V is None else int(V)
+    dev = target.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, gamma + 1), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = _ws(workspace, SPEC_ENTRY_CHAIN, B, gamma, V, dev, stream)
+    st = lib().spec_verify_chain(
+        B, gamma, V, _p(target), _dtype(target), _rows(target, "target"),
+        _p(draft), SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
+        _rows(draft, "draft"), _p(draft_tokens), _p(temperature), _p(coins), _p(final_u),
+        _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "spec_verify_chain")
+    return out_tokens, out_num_accepted
+
+
+def spec_verify_tree_greedy(target, tokens, parents, max_depth: int, *, V: int | None = None,
+                            out_accept_index=None, out_tokens=None, out_num_accepted=None,
+                            workspace=None, stream=None):
+    """Greedy tree verify.  Returns ``(accept_index, tokens, num_accepted)``."""
+    B, N, S = target.shape
+    V = S if V is None else int(V)
+    dev = target.device
+    W = max_depth + 1
+    if out_accept_index is None:
+        out_accept_index = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = _ws(workspace, SPEC_ENTRY_TREE_GREEDY, B, N, V, dev, stream)
+    st = lib().spec_verify_tree_greedy(
+        B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens),
+        _p(parents), _p(out_accept_index), _p(out_tokens), _p(out_num_accepted), _p(ws), ws.numel(),
+        _stream(stream))
+    _check(st, "spec_verify_tree_greedy")
+    return out_accept_index, out_tokens, out_num_accepted
+
+
+def spec_verify_tree_sample(target, tokens, parents, temperature, coins, final_u, max_depth: int, *,
+                            draft_probs=None, threshold_single: float = 1.0,
+                            threshold_acc: float = 1.0, V: int | None = None,
+                            out_accept_index=None, out_tokens=None, out_num_accepted=None,
+                            diag=None, workspace=None, stream=None):
+    """Target-only tree sampling.  Returns ``(accept_index, tokens, num_accepted)``."""
+    B, N, S = target.shape
+    V = S if V is None else int(V)
+    dev = target.device
+    W = max_depth + 1
+    if out_accept_index is None:
+        out_accept_index = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = _ws(workspace, SPEC_ENTRY_TREE_SAMPLE, B, N, V, dev, stream)
+    dstride = _rows(draft_probs, "draft_probs") if draft_probs is not None else 0
+    st = lib().spec_verify_tree_sample(
+        B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens),
+        _p(parents), _p(temperature), _p(coins), _p(final_u), _p(draft_probs), dstride,
+        float(threshold_single), float(threshold_acc), _p(out_accept_index), _p(out_tokens),
+        _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "spec_verify_tree_sample")
+    return out_accept_index, out_tokens, out_num_accepted

@@ -144,17 +144,17 @@ def _chain_cases(model: ToyModel, prefix, gamma: int):
     return cases
 
 
-def _run_chain_cases(model: ToyModel, cases):
+def _run_chain_cases(model: ToyModel, cases, runner=None):
     target = np.stack([c["target"] for c in cases])
     draft = np.stack([c["draft"] for c in cases])
     x = np.stack([c["x"] for c in cases])
     coins = np.stack([c["coins"] for c in cases])
     u = np.array([c["u"] for c in cases], np.float32)
     T = np.full(len(cases), model.T, np.float32)
-    return oracle.chain(target, draft, model.draft_kind == "probs", x, T, coins, u)
+    return (runner or oracle.chain)(target, draft, model.draft_kind == "probs", x, T, coins, u)
 
 
-def chain_bruteforce(V=3, gamma=2, K=3, seed=1, draft_kind="probs", tol=1e-12, T=1.0) -> dict:
+def chain_bruteforce(V=3, gamma=2, K=3, seed=1, draft_kind="probs", tol=1e-12, T=1.0, runner=None) -> dict:
     """Exact distribution of the first K tokens of repeated chain rounds."""
     model = ToyModel(V, seed, draft_kind, T=T)
     states = {(): 1.0}
@@ -165,7 +165,7 @@ def chain_bruteforce(V=3, gamma=2, K=3, seed=1, draft_kind="probs", tol=1e-12, T
             cs = _chain_cases(model, prefix, gamma)
             batch += cs
             owners += [(prefix, w)] * len(cs)
-        res = _run_chain_cases(model, batch)
+        res = _run_chain_cases(model, batch, runner)
         nxt = {}
         for i, (prefix, w) in enumerate(owners):
             k = int(res["num_accepted"][i])
@@ -186,12 +186,12 @@ def chain_bruteforce(V=3, gamma=2, K=3, seed=1, draft_kind="probs", tol=1e-12, T
     return dict(ok=err < tol, err=err)
 
 
-def chain_closed_form_exact(V=4, gamma=3, seed=2, draft_kind="probs", tol=1e-12) -> dict:
+def chain_closed_form_exact(V=4, gamma=3, seed=2, draft_kind="probs", tol=1e-12, runner=None) -> dict:
     """Exact E[tokens per round] with one (p, q) pair at every position versus
     (1 - beta^(gamma+1)) / (1 - beta)."""
     model = ToyModel(V, seed, draft_kind, iid=True)
     cases = _chain_cases(model, (), gamma)
-    res = _run_chain_cases(model, cases)
+    res = _run_chain_cases(model, cases, runner)
     w = np.array([c["weight"] for c in cases])
     tau = res["num_accepted"].astype(np.float64) + 1.0
     e_tau = float((w * tau).sum())
@@ -262,7 +262,7 @@ def _uniform24(rng, shape):
 
 
 def chain_chisquare(V=4, gamma=3, K=3, rounds=1_000_000, seed=3, draft_kind="probs",
-                    pmin=1e-3, T=1.0) -> dict:
+                    pmin=1e-3, T=1.0, runner=None) -> dict:
     model = ToyModel(V, seed, draft_kind, T=T)
     tab = _Tables(model, K - 1 + gamma)
     rng = np.random.default_rng(seed + 100)
@@ -285,7 +285,7 @@ def chain_chisquare(V=4, gamma=3, K=3, rounds=1_000_000, seed=3, draft_kind="pro
             x[:, i] = _sample_rows(tab.Q[cur], rng)
             cur = tab.child(cur, x[:, i])
         rows_t[:, gamma] = cur
-        res = oracle.chain(tab.PL[rows_t], tab.QR[rows_q], draft_kind == "probs", x,
+        res = (runner or oracle.chain)(tab.PL[rows_t], tab.QR[rows_q], draft_kind == "probs", x,
                            np.full(m, model.T, np.float32), _uniform24(rng, (m, gamma)),
                            _uniform24(rng, m))
         k = res["num_accepted"]
@@ -331,14 +331,14 @@ def _chisq(first, tab, V, K, pmin):
 
 
 def chain_closed_form_mc(V=4, gamma=3, rounds=1_000_000, seed=4, draft_kind="probs",
-                         nse=4.0) -> dict:
+                         nse=4.0, runner=None) -> dict:
     """Mean tau over simulated rounds with one (p, q) at every position versus the
     closed form, within ``nse`` standard errors."""
     model = ToyModel(V, seed, draft_kind, iid=True)
     (pl, p), (qr, q) = model.p(()), model.q(())
     rng = np.random.default_rng(seed + 7)
     x = np.stack([_sample_rows(np.broadcast_to(q, (rounds, V)), rng) for _ in range(gamma)], 1)
-    res = oracle.chain(np.broadcast_to(pl, (rounds, gamma + 1, V)),
+    res = (runner or oracle.chain)(np.broadcast_to(pl, (rounds, gamma + 1, V)),
                        np.broadcast_to(qr, (rounds, gamma, V)), draft_kind == "probs",
                        x.astype(np.int32), np.ones(rounds, np.float32),
                        _uniform24(rng, (rounds, gamma)), _uniform24(rng, rounds))
@@ -418,7 +418,7 @@ def _tree_cases(model: ToyModel, prefix, parents):
 
 
 def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
-                    draft_probs_zero=False, T=1.0) -> dict:
+                    draft_probs_zero=False, T=1.0, runner=None) -> dict:
     """Exact distribution of the first K tokens of repeated target-only tree rounds
     (thresholds 1) against the target's autoregressive distribution."""
     model = ToyModel(V, seed, T=T)
@@ -434,7 +434,7 @@ def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
             batch += cs
             owners += [(prefix, w)] * len(cs)
         m = len(batch)
-        res = oracle.tree_sample(np.stack([c["target"] for c in batch]),
+        res = (runner or oracle.tree_sample)(np.stack([c["target"] for c in batch]),
                                  np.stack([c["tokens"] for c in batch]),
                                  np.broadcast_to(parents, (m, N)), np.full(m, model.T, np.float32),
                                  np.stack([c["coins"] for c in batch]),
@@ -457,7 +457,7 @@ def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
     return dict(ok=err < tol, err=err)
 
 
-def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3) -> dict:
+def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3, runner=None) -> dict:
     """Simulated target-only tree rounds (thresholds 1) over a few tree shapes with
     random distinct sibling tokens; chi-square of the first K tokens."""
     shapes = shapes or [(-1, 0, 0, 1, 1, 2), (-1, 0, 1, 2), (-1, 0, 0, 0, 1, 2, 3, 4)]
@@ -502,7 +502,7 @@ def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3) -
             d = [0] * N
             for c in range(1, N):
                 d[c] = d[par[c]] + 1
-            res = oracle.tree_sample(tab.PL[nid], tokens, np.broadcast_to(par, (m, N)),
+            res = (runner or oracle.tree_sample)(tab.PL[nid], tokens, np.broadcast_to(par, (m, N)),
                                      np.ones(m, np.float32), _uniform24(rng, (m, N)),
                                      _uniform24(rng, m), max(d))
             k = res["num_accepted"]
@@ -529,7 +529,8 @@ def _toy_row(h: int, V: int, levels: int) -> np.ndarray:
     return (vals.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def greedy_equivalence(steps=10_000, V=16, levels=4, seed=7, max_nodes=12, max_depth=4) -> dict:
+def greedy_equivalence(steps=10_000, V=16, levels=4, seed=7, max_nodes=12, max_depth=4,
+                       runner=None) -> dict:
     """Speculative greedy over random trees versus plain argmax decoding of the same
     toy model (lowest index among equal maxima), token for token."""
     MOD = (1 << 61) - 1
@@ -574,8 +575,8 @@ def greedy_equivalence(steps=10_000, V=16, levels=4, seed=7, max_nodes=12, max_d
                 tokens[n] = int(rng.integers(V))
             hs[n] = hnext(hs[pa], tokens[n])
             rows[n] = row_f(hs[n])[0]
-        res = oracle.tree_greedy(np.stack(rows)[None], np.array([tokens]), np.array([parents]),
-                                 max(depth))
+        res = (runner or oracle.tree_greedy)(np.stack(rows)[None], np.array([tokens]),
+                                             np.array([parents]), max(depth))
         k = int(res["num_accepted"][0])
         if k < 0:
             return dict(ok=False, reason="invalid")
