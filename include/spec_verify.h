@@ -207,6 +207,42 @@ spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spec_verify_chain_noalloc -- spec_verify_chain without a caller workspace.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory where they verify: a plugin running
+ * inside an engine whose allocator owns all GPU memory, a decode loop that
+ * cannot afford the implicit device synchronisation of cudaMalloc/cudaFree,
+ * or a host thread without access to an allocator.  It allocates nothing and
+ * calls no allocating routine.
+ *
+ * Arguments, semantics, outputs and error behaviour are those of
+ * spec_verify_chain, minus workspace and workspace_bytes.  The scratch is a
+ * built-in device array of SPEC_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU
+ * loading the library holds until the process exits.  A shape whose scratch
+ * need (spec_workspace_bytes(SPEC_ENTRY_CHAIN, B, gamma, V)) exceeds it is
+ * rejected with SPEC_ERR_WORKSPACE before anything is enqueued.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ * - All calls share the one array, which keeps the previous call's contents;
+ *   each call first clears (cudaMemsetAsync on `stream`) the parts that must
+ *   start at zero.  Calls whose executions overlap on the GPU -- on different
+ *   streams, or from different host threads -- race on the array and give
+ *   undefined results: serialise them.
+ * - Device-side input errors are reported through out_num_accepted = -1; the
+ *   status word lives in the shared array and is not readable by the caller.
+ */
+#define SPEC_NOALLOC_SCRATCH_BYTES (16u << 20)
+spec_status spec_verify_chain_noalloc(int B, int gamma, int V,
+                                      const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                      const void* draft, spec_dtype ddt, int draft_is_probs,
+                                      int64_t d_row_stride,
+                                      const int32_t* draft_tokens, const float* temperature,
+                                      const float* coins, const float* final_u,
+                                      int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                      void* stream);
+
+/*
  * spec_workspace_bytes -- workspace size for one entry point and shape.
  * rows = gamma for SPEC_ENTRY_CHAIN (sized for draft logits, which also
  * covers draft probabilities), N for the tree entry points.  Returns 0 for

@@ -32,6 +32,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "spec_verify.h"
 
 namespace sv {
@@ -1428,3 +1430,77 @@ spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
 }
 
 }  // extern "C"
+
+// ============================================================================= no-allocation variant
+//
+// Some callers cannot allocate device memory at the point where they verify:
+// a plugin inside a serving engine whose own allocator owns every byte of the
+// GPU, code that must not pay the implicit device-wide synchronisation that
+// cudaMalloc/cudaFree can cause in a latency-critical decode loop, or a host
+// thread that holds no allocator at all.  For them spec_verify_chain_noalloc
+// runs the same kernels on a scratch area compiled into the library.
+
+// The scratch area: SPEC_NOALLOC_SCRATCH_BYTES on every GPU that loads this
+// library, held until the process exits.  In host code this name is only a
+// host-side stand-in; the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SPEC_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[256] = {};
+
+// Device address of the scratch area on the current device, looked up once per
+// device (with that device current) and cached.
+spec_status noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 256) return fail(SPEC_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(SPEC_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SPEC_OK;
+}
+
+}  // namespace
+
+extern "C" spec_status spec_verify_chain_noalloc(int B, int gamma, int V,
+                                                 const void* target_logits, spec_dtype tdt,
+                                                 int64_t t_row_stride,
+                                                 const void* draft, spec_dtype ddt, int draft_is_probs,
+                                                 int64_t d_row_stride,
+                                                 const int32_t* draft_tokens, const float* temperature,
+                                                 const float* coins, const float* final_u,
+                                                 int32_t* out_tokens, int32_t* out_num_accepted,
+                                                 float* diag, void* stream) {
+    g_detail[0] = 0;
+    if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
+    if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
+    if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
+    if (B == 0) return SPEC_OK;
+    const Layout L = make_layout(SPEC_ENTRY_CHAIN, B, gamma, V);
+    if (L.total > (size_t)SPEC_NOALLOC_SCRATCH_BYTES)
+        return fail(SPEC_ERR_WORKSPACE,
+                    "B=%d gamma=%d V=%d needs %zu bytes of scratch; the built-in scratch holds %zu "
+                    "(use spec_verify_chain with a caller workspace)",
+                    B, gamma, V, L.total, (size_t)SPEC_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    spec_status s = noalloc_scratch(&scratch);
+    if (s != SPEC_OK) return s;
+    // The area keeps whatever the previous call left there: clear the status
+    // word and the arrival counters (everything before the statistics), the
+    // only parts that must start at zero.
+    cudaError_t e = cudaMemsetAsync(scratch, 0, L.stats, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "cudaMemsetAsync(scratch): %s", cudaGetErrorString(e));
+    return spec_verify_chain(B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                             d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens,
+                             out_num_accepted, diag, scratch, (size_t)SPEC_NOALLOC_SCRATCH_BYTES, stream);
+}
+
