@@ -40,7 +40,8 @@ namespace sv {
 
 constexpr int NT = 128;               // threads per CTA
 constexpr int NWARP = NT / 32;
-constexpr int VPT = 8;                // 16-byte vectors per thread per chunk
+constexpr int VPT = 8;                // 16-byte vectors per thread per 16 KB chunk
+constexpr int SPC = NWARP;            // statistics per chunk (one per warp)
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1 or N)
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
@@ -57,6 +58,7 @@ template <int DT> __host__ __device__ constexpr int chunk_elems() { return NT * 
 struct Params {
     int B, V, R, nch, gamma, N, max_depth;
     int rows_tgt;                  // target rows per sequence
+    int nsl;                       // chain finalisation: CTAs (slices of chunks) per sequence
     const char* tgt;
     int64_t tstride;               // bytes between consecutive target rows
     const char* drf;
@@ -74,7 +76,7 @@ struct Params {
     int32_t* out_accept_index;
     int32_t* out_num_accepted;
     float* diag;
-    float2* stats;                 // [B][R][nch][NWARP]
+    float2* stats;                 // [B][R][nch][SPC]
     float2* stats2;                // [B][nch][NWARP]   (chain residual chunk sums)
     unsigned* cnt2;                // [B]               (chain residual arrivals)
     unsigned* status;
@@ -157,6 +159,12 @@ __device__ __forceinline__ float scale_of(float T) { return (float)(LOG2E / (dou
 
 __device__ __forceinline__ float2 ldcg2(const float2* p) { return __ldcg(p); }
 
+// Programmatic dependent launch: the statistics kernel lets the finalize
+// kernel be scheduled early; the finalize kernel waits for the statistics
+// kernel's completion (and memory) before reading anything it wrote.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void flag_input_error(const Params& P) {
     atomicOr(P.status, 1u << SPEC_ERR_DEVICE_INPUT);
 }
@@ -186,16 +194,12 @@ __device__ double block_excl_scan(double v, double* total) {
 
 // ----------------------------------------------------------------------------- row-chunk statistics
 
-// Per-thread online-softmax partial over NV 16-byte vectors starting at element
-// e_base: (max x, sum 2^(x - max)), x = l * s.  `bad` is set by a NaN or +inf.
+// Per-thread online-softmax partial of NV 16-byte vectors held in registers:
+// (max x, sum 2^(x - max)), x = l * s.  `bad` is set by a NaN or +inf.
 template <int DT, int NV>
-__device__ __forceinline__ void thread_softmax(const char* row, int V, int64_t e_base, float s,
-                                               float& mt, float& st, bool& bad) {
+__device__ __forceinline__ void thread_softmax_regs(const uint4 (&v)[NV], float s, float& mt, float& st,
+                                                    bool& bad) {
     constexpr int EPV = Tr<DT>::EPV;
-    const int tid = threadIdx.x;
-    uint4 v[NV];
-#pragma unroll
-    for (int k = 0; k < NV; ++k) v[k] = ld_vec<DT>(row, e_base + (int64_t)(k * NT + tid) * EPV, V);
     float lmax;
     bool b = false;
     if constexpr (DT == SPEC_BF16) {
@@ -239,6 +243,33 @@ __device__ __forceinline__ void thread_softmax(const char* row, int V, int64_t e
     bad |= b;
 }
 
+// NV 16-byte vectors of a row starting at element e_base (thread tid takes
+// vectors k*NT + tid); elements at or past V read as -inf.
+template <int DT, int NV>
+__device__ __forceinline__ void load_vecs(const char* row, int V, int64_t e_base, uint4 (&v)[NV]) {
+    constexpr int EPV = Tr<DT>::EPV;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) v[k] = ld_vec<DT>(row, e_base + (int64_t)(k * NT + threadIdx.x) * EPV, V);
+}
+
+template <int DT, int NV>
+__device__ __forceinline__ void thread_softmax(const char* row, int V, int64_t e_base, float s,
+                                               float& mt, float& st, bool& bad) {
+    uint4 v[NV];
+    load_vecs<DT, NV>(row, V, e_base, v);
+    thread_softmax_regs<DT, NV>(v, s, mt, st, bad);
+}
+
+// Warp combination of per-thread softmax partials into the warp's statistic.
+__device__ __forceinline__ float2 warp_softmax_stat(float mt, float st, bool bad) {
+    const float mw = warp_max(mt);
+    const bool anybad = __any_sync(FULL, bad);
+    float contrib = (mt == -INFINITY) ? 0.f : st * ex2(mt - mw);
+    float sw = warp_sum(contrib);
+    if (anybad) sw = nanf_();
+    return make_float2(mw, sw);
+}
+
 // Online-softmax statistic of chunk c of a row, CH elements per chunk (the
 // target's chunking; rows of another dtype are split into as many 16-byte
 // vectors as that takes).  Per warp: (max x, sum 2^(x - max)); NaN sum for a
@@ -261,23 +292,16 @@ __device__ __forceinline__ float2 chunk_softmax(const char* row, int V, int c, f
         if (m > -INFINITY) st = (mt > -INFINITY ? st * ex2(mt - m) : 0.f) + (m2 > -INFINITY ? s2 * ex2(m2 - m) : 0.f);
         mt = m;
     }
-    const float mw = warp_max(mt);
-    const bool anybad = __any_sync(FULL, bad);
-    float contrib = (mt == -INFINITY) ? 0.f : st * ex2(mt - mw);
-    float sw = warp_sum(contrib);
-    if (anybad) sw = nanf_();
-    return make_float2(mw, sw);
+    return warp_softmax_stat(mt, st, bad);
 }
 
-// (max value, lowest index) of one chunk per warp; value NaN if any NaN was seen.
+// (max value, lowest index) per warp of one chunk held in registers (vector
+// k of thread tid starts at element c*CH + (k*NT + tid)*EPV); value NaN if any
+// NaN was seen.
 template <int DT>
-__device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
+__device__ __forceinline__ float2 argmax_regs(const uint4 (&v)[VPT], int c) {
     constexpr int EPV = Tr<DT>::EPV, CH = chunk_elems<DT>();
     const int tid = threadIdx.x;
-    uint4 v[VPT];
-#pragma unroll
-    for (int k = 0; k < VPT; ++k)
-        v[k] = ld_vec<DT>(row, (int64_t)c * CH + (int64_t)(k * NT + tid) * EPV, V);
     float best = -INFINITY;
     int bestk = 0;
     uint4 bw = v[0];
@@ -317,6 +341,13 @@ __device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
     return make_float2(best, __int_as_float(idx));
 }
 
+template <int DT>
+__device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
+    uint4 v[VPT];
+    load_vecs<DT, VPT>(row, V, (int64_t)c * chunk_elems<DT>(), v);
+    return argmax_regs<DT>(v, c);
+}
+
 // ----------------------------------------------------------------------------- finaliser pieces
 
 struct FinShared {
@@ -328,6 +359,7 @@ struct FinShared {
     double pch[SPEC_MAX_NODES];
     int rej[SPEC_MAX_NODES];
     double M[MAXCH];
+    float wp[MAXCH][NWARP];
     uint32_t bitmap[(NT * VPT * 8) / 32];
     int ivals[8];
     double dvals[4];
@@ -336,7 +368,7 @@ struct FinShared {
 // Combine the per-warp softmax statistics of rows [0, R) into (m, Z, bad).
 __device__ void combine_softmax_rows(const Params& P, int b, int R, FinShared& sh) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int E = P.nch * NWARP;
+    const int E = P.nch * SPC;
     for (int r = warp; r < R; r += NWARP) {
         const float2* st = P.stats + ((size_t)b * P.R + r) * E;
         float m = -INFINITY;
@@ -552,7 +584,7 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
     return r;
 }
 
-// Inverse-CDF draw from the target row `row` (statistics st: nch*NWARP entries)
+// Inverse-CDF draw from the target row `row` (statistics st: nch*SPC entries)
 // with the tokens in excl[0..nexcl) removed.  Chunk masses come from the
 // statistics (fp64), excluded tokens are subtracted from their chunk, the
 // chunk holding u*S is rescanned.  *S_unnorm = remaining mass in units of
@@ -565,8 +597,8 @@ __device__ int sample_target_row(const char* row, int V, int nch, const float2* 
     for (int c = tid; c < nch; c += NT) {
         double M = 0.0;
 #pragma unroll
-        for (int w = 0; w < NWARP; ++w) {
-            float2 x = ldcg2(st + c * NWARP + w);
+        for (int w = 0; w < SPC; ++w) {
+            float2 x = ldcg2(st + c * SPC + w);
             if (x.x > -INFINITY) M += (double)x.y * (double)ex2(x.x - m);
         }
         sh.M[c] = M;
@@ -655,64 +687,84 @@ __device__ int tree_valid(const Params& P, int N, int V, int max_depth, FinShare
 
 // ----------------------------------------------------------------------------- finalisers
 
-// Chain decision for sequence b (rule 1), computed by thread 0 after the row
-// statistics were combined into sh.m / sh.z / sh.bad.  Writes sh.ivals[0] =
-// valid, sh.ivals[1] = k, sh.dvals[0] = s.  When `write` is set it also writes
-// the accepted tokens, the -1 tail (position k excluded), num_accepted and the
-// p/q diagnostics, and flags invalid sequences.
+// Chain decision for sequence b (rule 1), after the row statistics were
+// combined into sh.m / sh.z / sh.bad.  Threads 0..gamma-1 gather p_i(x_i) and
+// q_i(x_i) in parallel (fp64 exp2 in the units of the row statistics); thread
+// 0 then takes the decisions.  Leaves sh.ivals[0] = valid, sh.ivals[1] = k,
+// sh.dvals[0] = s.  When `write` is set it also writes the accepted tokens,
+// the -1 tail (position k excluded), num_accepted and the p/q diagnostics, and
+// flags invalid sequences.  Ends with __syncthreads.
 template <int TDT, int DDT, int DK>
 __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write) {
+    const int tid = threadIdx.x;
     const int gamma = P.gamma, V = P.V, W = gamma + 1;
     int32_t* toks = P.out_tokens + (size_t)b * W;
     float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
     const float T = P.temperature[b];
-    bool ok = temperature_ok(T);
-    for (int r = 0; r < P.R; ++r) ok &= !sh.bad[r];
     const int32_t* x = P.draft_tokens + (size_t)b * gamma;
-    for (int i = 0; i < gamma; ++i) ok &= (x[i] >= 0 && x[i] < V);
-    const float s = ok ? scale_of(T) : 0.f;
-    int k = gamma;
-    if (ok) {
-        // p_i(x_i), q_i(x_i) for every position (diagnostics), then rule 1.
-        double pr[SPEC_MAX_GAMMA], qr[SPEC_MAX_GAMMA];
-        for (int i = 0; i < gamma; ++i) {
-            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride;
-            const char* drow = P.drf + ((size_t)b * gamma + i) * P.dstride;
-            pr[i] = prob_d(ld_elem<TDT>(trow, x[i]), s, sh.m[i], sh.z[i]);
+    const bool tok = temperature_ok(T);
+    const float s = tok ? scale_of(T) : 0.f;
+    if (tid < gamma) {
+        const int xi = x[tid];
+        bool ok = xi >= 0 && xi < V;
+        double p = 0.0, q = 0.0;
+        if (ok && tok) {
+            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + tid) * P.tstride;
+            const char* drow = P.drf + ((size_t)b * gamma + tid) * P.dstride;
+            p = prob_d(ld_elem<TDT>(trow, xi), s, sh.m[tid], sh.z[tid]);
             if constexpr (DK == DK_PROBS) {
-                qr[i] = (double)__ldg(reinterpret_cast<const float*>(drow) + x[i]);
-                ok &= (qr[i] >= 0.0 && qr[i] <= 3.0e38);
+                q = (double)__ldg(reinterpret_cast<const float*>(drow) + xi);
+                ok &= (q >= 0.0 && q <= 3.0e38);
             } else {
-                qr[i] = prob_d(ld_elem<DDT>(drow, x[i]), s, sh.m[gamma + 1 + i], sh.z[gamma + 1 + i]);
+                q = prob_d(ld_elem<DDT>(drow, xi), s, sh.m[gamma + 1 + tid], sh.z[gamma + 1 + tid]);
             }
-            if (dg && write) { dg[i] = (float)pr[i]; dg[gamma + i] = (float)qr[i]; }
         }
-        for (int i = 0; i < gamma && ok; ++i) {
-            const double ratio = (qr[i] > 0.0) ? pr[i] / qr[i] : INFINITY;
-            if (!((double)P.coins[(size_t)b * gamma + i] <= ratio)) { k = i; break; }
+        sh.pch[tid] = p;
+        sh.pch[SPEC_MAX_GAMMA + tid] = q;
+        sh.rej[tid] = ok;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        bool ok = tok;
+        for (int r = 0; r < P.R; ++r) ok &= !sh.bad[r];
+        for (int i = 0; i < gamma; ++i) ok &= (sh.rej[i] != 0);
+        int k = gamma;
+        if (ok) {
+            for (int i = 0; i < gamma; ++i) {
+                const double pi = sh.pch[i], qi = sh.pch[SPEC_MAX_GAMMA + i];
+                const double ratio = (qi > 0.0) ? pi / qi : INFINITY;
+                if (!((double)P.coins[(size_t)b * gamma + i] <= ratio)) { k = i; break; }
+            }
+        }
+        sh.ivals[0] = ok;
+        sh.ivals[1] = k;
+        sh.dvals[0] = (double)s;
+        if (write) {
+            if (!ok) {
+                for (int i = 0; i < W; ++i) toks[i] = -1;
+                P.out_num_accepted[b] = -1;
+                if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
+                flag_input_error(P);
+            } else {
+                for (int i = 0; i < k; ++i) toks[i] = x[i];
+                for (int i = k + 1; i < W; ++i) toks[i] = -1;
+                P.out_num_accepted[b] = k;
+                if (dg)
+                    for (int i = 0; i < gamma; ++i) {
+                        dg[i] = (float)sh.pch[i];
+                        dg[gamma + i] = (float)sh.pch[SPEC_MAX_GAMMA + i];
+                    }
+            }
         }
     }
-    sh.ivals[0] = ok;
-    sh.ivals[1] = k;
-    sh.dvals[0] = (double)s;
-    if (!write) return;
-    if (!ok) {
-        for (int i = 0; i < W; ++i) toks[i] = -1;
-        P.out_num_accepted[b] = -1;
-        if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
-        flag_input_error(P);
-    } else {
-        for (int i = 0; i < k; ++i) toks[i] = x[i];
-        for (int i = k + 1; i < W; ++i) toks[i] = -1;
-        P.out_num_accepted[b] = k;
-    }
+    __syncthreads();
 }
 
 template <int TDT>
 __device__ void finalize_greedy(const Params& P, int b, FinShared& sh) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
-    const int E = P.nch * NWARP;
+    const int E = P.nch * SPC;
     // per-node argmax (lowest index among equal maxima)
     for (int r = warp; r < N; r += NWARP) {
         const float2* st = P.stats + ((size_t)b * P.R + r) * E;
@@ -858,7 +910,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
     int y;
     double S;
     if (!P.draft_probs) {
-        const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * NWARP;
+        const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
         double Su;
         y = sample_target_row<TDT>(row, V, P.nch, st, s, sh.m[cur], u, sh.rej, nrej, sh, &Su);
         S = Su / sh.z[cur];
@@ -927,7 +979,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
         }
         if (y < 0) {
             // empty residual (rounding only): draw from p_cur itself
-            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * NWARP;
+            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
             double Su;
             y = sample_target_row<TDT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
         }
@@ -943,58 +995,108 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
 // ----------------------------------------------------------------------------- kernels
 
 // Row statistics (the streaming kernel).  The B*R*nch work items (sequence-
-// major, then row, then chunk) are split into gridDim.x contiguous ranges,
-// one per CTA.  Each warp writes one statistic per item; nothing else is
-// shared, so the kernel has no atomics and no fences: the finalize kernel
-// that follows in stream order reads the statistics.
+// major, then row, then chunk; a chunk is 16 KB of one row) are split into
+// gridDim.x contiguous ranges, one per CTA; (b, r, c) advance incrementally.
+// Each thread loads its eight 16-byte vectors of a chunk at once; each warp
+// reduces its quarter to one statistic -- online softmax (max x, sum
+// 2^(x - max)) or (max, lowest index) -- and writes it.  Nothing else is
+// shared: no atomics, no fences; the finalize kernel that follows in stream
+// order reads the statistics.  Ten CTAs of four warps per SM keep enough
+// loads in flight and enough warps to hide the exp2 and ALU latency.
 template <int MODE, int TDT, int DDT>
 __global__ void __launch_bounds__(NT) k_stats(const Params P) {
+    constexpr int CH = chunk_elems<TDT>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_trigger();
     const int per_seq = P.R * P.nch;
     const long long total = (long long)P.B * per_seq;
     const long long lo = total * blockIdx.x / gridDim.x;
-    const long long hi = total * (blockIdx.x + 1) / gridDim.x;
-    for (long long item = lo; item < hi; ++item) {
-        const int b = (int)(item / per_seq);
-        const int rem = (int)(item - (long long)b * per_seq);
-        const int r = rem / P.nch, c = rem - r * P.nch;
+    const long long n = total * (blockIdx.x + 1) / gridDim.x - lo;
+    int b = (int)(lo / per_seq);
+    int r, c;
+    {
+        const int rem = (int)(lo - (long long)b * per_seq);
+        r = rem / P.nch;
+        c = rem - r * P.nch;
+    }
+    int sb = -1;
+    float s = 0.f;
+    for (long long j = 0; j < n; ++j) {
         float2 stat;
         if constexpr (MODE == MODE_GREEDY) {
             const char* row = P.tgt + ((size_t)b * P.R + r) * P.tstride;
             stat = chunk_argmax<TDT>(row, P.V, c);
         } else {
-            const float s = scale_of(__ldg(P.temperature + b));
+            if (b != sb) { sb = b; s = scale_of(__ldg(P.temperature + b)); }
             if (r < P.rows_tgt) {
                 const char* row = P.tgt + ((size_t)b * P.rows_tgt + r) * P.tstride;
-                stat = chunk_softmax<TDT, chunk_elems<TDT>()>(row, P.V, c, s);
+                stat = chunk_softmax<TDT, CH>(row, P.V, c, s);
             } else {
                 const char* row = P.drf + ((size_t)b * (P.R - P.rows_tgt) + (r - P.rows_tgt)) * P.dstride;
-                stat = chunk_softmax<DDT, chunk_elems<TDT>()>(row, P.V, c, s);
+                stat = chunk_softmax<DDT, CH>(row, P.V, c, s);
             }
         }
-        if (lane == 0) P.stats[(((size_t)b * P.R + r) * P.nch + c) * NWARP + warp] = stat;
+        if (lane == 0) P.stats[(((size_t)b * P.R + r) * P.nch + c) * SPC + warp] = stat;
+        if (++c == P.nch) {
+            c = 0;
+            if (++r == P.R) { r = 0; ++b; }
+        }
     }
 }
 
-// Chain finalisation, grid = B * nch: CTA (b, c) recomputes sequence b's
-// decision from the row statistics (cheap, identical in every CTA), then
-//  - k = gamma: CTA c = 0 draws the bonus token from p_gamma (rule 3);
-//  - k < gamma, one chunk per row: CTA 0 draws the correction directly;
-//  - k < gamma, several chunks: every CTA sums max(0, p_k - q_k) over its
-//    chunk; the last CTA of the sequence to arrive locates the chunk holding
-//    u*S and rescans it (rule 2).
+// Locate the chunk holding t among the chunk masses sh.M[0..nch) (skipping
+// empty chunks) and rescan it; retries past chunks whose rescan finds no
+// positive weight (possible only through rounding).  Returns -1 if none.
+template <int CH, class WF>
+__device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u, FinShared& sh) {
+    const int tid = threadIdx.x;
+    int y = -1;
+    for (int attempt = 0; attempt < nch && y < 0; ++attempt) {
+        if (tid == 0) {
+            double C = 0.0, before = 0.0;
+            int cs = -1;
+            for (int cc = 0; cc < nch; ++cc) {
+                if (sh.M[cc] <= 0.0) continue;
+                if (t < C + sh.M[cc]) { cs = cc; before = C; break; }
+                C += sh.M[cc];
+            }
+            if (cs < 0)
+                for (int cc = nch - 1; cc >= 0; --cc)
+                    if (sh.M[cc] > 0.0) { cs = cc; before = C - sh.M[cc]; break; }
+            sh.ivals[2] = cs;
+            sh.dvals[1] = before;
+        }
+        __syncthreads();
+        const int cs = sh.ivals[2];
+        if (cs < 0) break;
+        double tot;
+        y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+        if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+        __syncthreads();
+    }
+    return y;
+}
+
+// Chain finalisation, grid = B * nsl: CTA (b, slice) recomputes sequence b's
+// decision from the row statistics (cheap, identical in every CTA of b), then
+//  - k = gamma: slice 0 draws the bonus token from p_gamma (rule 3);
+//  - k < gamma: every slice sums max(0, p_k - q_k) over its chunks of row k;
+//    with one slice the CTA draws directly, otherwise the last CTA of the
+//    sequence to arrive locates the chunk holding u*S and rescans it (rule 2).
 template <int TDT, int DDT, int DK>
 __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     __shared__ FinShared sh;
     __shared__ int is_last;
     constexpr int CH = chunk_elems<TDT>();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x / P.nch, c = blockIdx.x - b * P.nch;
+    const int nsl = P.nsl, nch = P.nch;
+    const int b = blockIdx.x / nsl, sl = blockIdx.x - b * nsl;
+    const int c0 = (int)((long long)nch * sl / nsl), c1 = (int)((long long)nch * (sl + 1) / nsl);
     const int gamma = P.gamma, V = P.V;
+    pdl_wait();
     combine_softmax_rows(P, b, P.R, sh);
     __syncthreads();
-    if (tid == 0) chain_decide<TDT, DDT, DK>(P, b, sh, c == 0);
-    __syncthreads();
+    chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0);
     const int ok = sh.ivals[0], k = sh.ivals[1];
     const float s = (float)sh.dvals[0];
     if (!ok) return;
@@ -1003,10 +1105,10 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
     const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
     if (k == gamma) {
-        if (c != 0) return;
-        const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * NWARP;
+        if (sl != 0) return;
+        const float2* st = P.stats + ((size_t)b * P.R + gamma) * nch * SPC;
         double S;
-        int y = sample_target_row<TDT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        int y = sample_target_row<TDT>(trow, V, nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
         if (tid == 0) {
             toks[k] = y;
             if (dg) dg[2 * gamma] = 1.0f;
@@ -1018,85 +1120,62 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
     const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
     WChainRes<TDT, DDT, DK> wf{trow, drow, s, mp, izp, mq, izq, V};
-    const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * NWARP;
-    if (P.nch == 1) {
-        double S;
-        int y = rescan_chunk<CH>(wf, 0, V, -1.0, u, &S);
-        if (y < 0 || !(S > 0.0)) {
-            double S2;
-            y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &S2);
+    // chunk sums of max(0, p_k - q_k) for this slice's chunks
+    for (int c = c0; c < c1; ++c) {
+        const float ws = warp_sum(chunk_weight_partial<CH>(wf, c));
+        if (lane == 0) {
+            if (nsl == 1) sh.wp[c][warp] = ws;
+            else P.stats2[((size_t)b * nch + c) * NWARP + warp] = make_float2(ws, 0.f);
         }
-        if (tid == 0) {
-            toks[k] = y;
-            if (dg) dg[2 * gamma] = (float)S;
-        }
-        return;
     }
-    const float ws = warp_sum(chunk_weight_partial<CH>(wf, c));
-    if (lane == 0) {
-        P.stats2[((size_t)b * P.nch + c) * NWARP + warp] = make_float2(ws, 0.f);
-        __threadfence();
-    }
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(P.cnt2 + b, 1u);
-        is_last = (prev == (unsigned)P.nch - 1u);
-    }
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    for (int cc = tid; cc < P.nch; cc += NT) {
-        double M = 0.0;
+    if (nsl == 1) {
+        __syncthreads();
+        for (int c = tid; c < nch; c += NT) {
+            double M = 0.0;
 #pragma unroll
-        for (int w = 0; w < NWARP; ++w) M += (double)ldcg2(P.stats2 + ((size_t)b * P.nch + cc) * NWARP + w).x;
-        sh.M[cc] = M;
+            for (int w = 0; w < NWARP; ++w) M += (double)sh.wp[c][w];
+            sh.M[c] = M;
+        }
+    } else {
+        if (lane == 0) __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const unsigned prev = atomicAdd(P.cnt2 + b, 1u);
+            is_last = (prev == (unsigned)nsl - 1u);
+        }
+        __syncthreads();
+        if (!is_last) return;
+        __threadfence();
+        for (int c = tid; c < nch; c += NT) {
+            double M = 0.0;
+#pragma unroll
+            for (int w = 0; w < NWARP; ++w) M += (double)ldcg2(P.stats2 + ((size_t)b * nch + c) * NWARP + w).x;
+            sh.M[c] = M;
+        }
     }
     __syncthreads();
     if (tid == 0) {
         double S = 0.0;
-        for (int cc = 0; cc < P.nch; ++cc) S += sh.M[cc];
+        for (int c = 0; c < nch; ++c) S += sh.M[c];
         sh.dvals[0] = S;
     }
     __syncthreads();
     const double S = sh.dvals[0];
-    int y = -1;
-    if (S > 0.0) {
-        const double t = (double)u * S;
-        for (int attempt = 0; attempt < P.nch && y < 0; ++attempt) {
-            if (tid == 0) {
-                double C = 0.0, before = 0.0;
-                int cs = -1;
-                for (int cc = 0; cc < P.nch; ++cc) {
-                    if (sh.M[cc] <= 0.0) continue;
-                    if (t < C + sh.M[cc]) { cs = cc; before = C; break; }
-                    C += sh.M[cc];
-                }
-                if (cs < 0)
-                    for (int cc = P.nch - 1; cc >= 0; --cc)
-                        if (sh.M[cc] > 0.0) { cs = cc; before = C - sh.M[cc]; break; }
-                sh.ivals[2] = cs;
-                sh.dvals[1] = before;
-            }
-            __syncthreads();
-            const int cs = sh.ivals[2];
-            if (cs < 0) break;
-            double tot;
-            y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
-            if (y < 0 && tid == 0) sh.M[cs] = 0.0;
-            __syncthreads();
-        }
-    }
+    int y = (S > 0.0) ? draw_from_chunks<CH>(wf, nch, V, (double)u * S, u, sh) : -1;
     if (y < 0) {
         // empty residual (rounding only): draw from p_k
+        const float2* stk = P.stats + ((size_t)b * P.R + k) * nch * SPC;
         double Su;
-        y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+        y = sample_target_row<TDT>(trow, V, nch, stk, s, mp, u, nullptr, 0, sh, &Su);
     }
     if (tid == 0) {
         toks[k] = y;
         if (dg) dg[2 * gamma] = (float)S;
-        __threadfence();
-        P.cnt2[b] = 0u;
+        if (nsl > 1) {
+            __threadfence();
+            P.cnt2[b] = 0u;
+        }
     }
 }
 
@@ -1104,6 +1183,7 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
 template <int MODE, int TDT>
 __global__ void __launch_bounds__(NT) k_tree_final(const Params P) {
     __shared__ FinShared sh;
+    pdl_wait();
     if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT>(P, blockIdx.x, sh);
     else finalize_sample<TDT>(P, blockIdx.x, sh);
 }
@@ -1152,7 +1232,7 @@ Layout make_layout(int entry, int B, int rows, int V) {
     size_t off = 0;
     L.status = off; off = align256(off + 16);
     L.cnt2 = off; off = align256(off + sizeof(unsigned) * (size_t)B);
-    L.stats = off; off = align256(off + sizeof(float2) * (size_t)B * L.R * nch * NWARP);
+    L.stats = off; off = align256(off + sizeof(float2) * (size_t)B * L.R * nch * SPC);
     L.stats2 = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(float2) * (size_t)B * nch * NWARP);
     L.total = off;
@@ -1229,20 +1309,41 @@ spec_status launch_stats(const Params& P, cudaStream_t st) {
     return s;
 }
 
+// Launch a finalize kernel as a programmatic dependent of the statistics
+// kernel just enqueued on `st`.
+template <class K>
+spec_status launch_dependent(K kernel, unsigned grid, const Params& P, cudaStream_t st, const char* what) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, P);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return launched(what);
+}
+
 template <int TDT, int DDT, int DK>
-spec_status launch_chain(const Params& P, cudaStream_t st) {
-    spec_status s = launch_stats<MODE_CHAIN, TDT, DDT>(P, st);
+spec_status launch_chain(Params P, cudaStream_t st) {
+    // draft probabilities are read only by the finalize kernel
+    spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
-    k_chain_final<TDT, DDT, DK><<<(unsigned)(P.B * P.nch), NT, 0, st>>>(P);
-    return launched("k_chain_final");
+    // enough CTAs to cover the SMs twice, at most one per chunk
+    int nsl = (2 * num_sms() + P.B - 1) / P.B;
+    P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
+    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), P, st, "k_chain_final");
 }
 
 template <int MODE, int TDT>
 spec_status launch_tree(const Params& P, cudaStream_t st) {
     spec_status s = launch_stats<MODE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
-    k_tree_final<MODE, TDT><<<(unsigned)P.B, NT, 0, st>>>(P);
-    return launched("k_tree_final");
+    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, P, st, "k_tree_final");
 }
 
 }  // namespace
