@@ -55,6 +55,24 @@ def dist_env():
     return ws, rank, local
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def reduce_max_ms(ms: float, world: int, device=None) -> float:
+    """Max over ranks of a per-rank duration (the job ends when the slowest rank does)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(steps: int, world: int, max_ms: float) -> float:
+    """Whole-job verify rounds/s: every rank verifies one round per step."""
+    return world * steps / (max_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- workloads
 
 def make_inputs(wid: int, rnd: int, device, rank: int = 0):
@@ -362,11 +380,8 @@ def main():
         if ws_ > 1:
             dist.barrier()
     ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], device=dev)
-    if ws_ > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = ws_ * K / (ms_max / 1e3)
+    ms_max = reduce_max_ms(ms, ws_, dev)
+    value = job_value(K, ws_, ms_max)
 
     # --- dominant kernel duration: the library records an event pair around its
     # row-statistics kernel; the calls are captured in a CUDA graph so that host

@@ -165,6 +165,44 @@ __device__ __forceinline__ float2 ldcg2(const float2* p) { return __ldcg(p); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// mbarrier and 1-D bulk copy (TMA) helpers, used to stage a row pair in
+// shared memory.  Waits are bounded: WAIT_LIMIT tries and WAIT_NS.
+constexpr unsigned WAIT_LIMIT = 1u << 24;
+constexpr unsigned long long WAIT_NS = 1000000000ull;
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint32_t a, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(a), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(a), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
+    if (mbar_try(a, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (unsigned i = 0; i < WAIT_LIMIT; ++i) {
+        if (mbar_try(a, parity)) return true;
+        if (global_ns() - t0 > WAIT_NS) break;
+    }
+    return false;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+
 __device__ __forceinline__ void flag_input_error(const Params& P) {
     atomicOr(P.status, 1u << SPEC_ERR_DEVICE_INPUT);
 }
@@ -371,29 +409,29 @@ __device__ void combine_softmax_rows(const Params& P, int b, int R, FinShared& s
     const int E = P.nch * SPC;
     for (int r = warp; r < R; r += NWARP) {
         const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        // one pass: each lane keeps an online (max, sum) over its entries
         float m = -INFINITY;
+        double z = 0.0;
         bool bad = false;
 #pragma unroll 4
         for (int e = lane; e < E; e += 32) {
-            float2 x = ldcg2(st + e);
-            m = fmaxf(m, x.x);
+            const float2 x = ldcg2(st + e);
             bad |= (x.y != x.y);
-        }
-        m = warp_max(m);
-        bad = __any_sync(FULL, bad);
-        double z = 0.0;
-        if (m > -INFINITY && !bad) {
-#pragma unroll 4
-            for (int e = lane; e < E; e += 32) {
-                float2 x = ldcg2(st + e);
-                if (x.x > -INFINITY) z += (double)x.y * (double)ex2(x.x - m);
+            if (x.x > m) {
+                z = (m > -INFINITY ? z * (double)ex2(m - x.x) : 0.0) + (double)x.y;
+                m = x.x;
+            } else if (x.x > -INFINITY) {
+                z += (double)x.y * (double)ex2(x.x - m);
             }
         }
-        z = warp_sum_d(z);
+        const float mw = warp_max(m);
+        bad = __any_sync(FULL, bad);
+        double zw = (m > -INFINITY && mw < INFINITY) ? z * (double)ex2(m - mw) : 0.0;
+        zw = warp_sum_d(zw);
         if (lane == 0) {
-            sh.m[r] = m;
-            sh.z[r] = z;
-            sh.bad[r] = bad || !(m > -INFINITY) || !(m < INFINITY) || !(z > 0.0) || !(z < 1e300);
+            sh.m[r] = mw;
+            sh.z[r] = zw;
+            sh.bad[r] = bad || !(mw > -INFINITY) || !(mw < INFINITY) || !(zw > 0.0) || !(zw < 1e300);
         }
     }
 }
@@ -687,41 +725,66 @@ __device__ int tree_valid(const Params& P, int N, int V, int max_depth, FinShare
 
 // ----------------------------------------------------------------------------- finalisers
 
-// Chain decision for sequence b (rule 1), after the row statistics were
-// combined into sh.m / sh.z / sh.bad.  Threads 0..gamma-1 gather p_i(x_i) and
-// q_i(x_i) in parallel (fp64 exp2 in the units of the row statistics); thread
-// 0 then takes the decisions.  Leaves sh.ivals[0] = valid, sh.ivals[1] = k,
-// sh.dvals[0] = s.  When `write` is set it also writes the accepted tokens,
-// the -1 tail (position k excluded), num_accepted and the p/q diagnostics, and
-// flags invalid sequences.  Ends with __syncthreads.
+// Inputs of the chain decision that the statistics kernel does not write:
+// loaded by threads 0..gamma-1 before waiting for that kernel (programmatic
+// dependent launch), so their latency hides under its tail.
+struct ChainPrefetch {
+    int x;          // draft token of position tid
+    float l;        // target logit at x
+    float d;        // draft logit (or probability) at x
+    bool ok;        // x in [0, V)
+};
+
 template <int TDT, int DDT, int DK>
-__device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write) {
+__device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) {
+    ChainPrefetch f{0, 0.f, 0.f, false};
+    const int tid = threadIdx.x, gamma = P.gamma;
+    if (tid < gamma) {
+        f.x = P.draft_tokens[(size_t)b * gamma + tid];
+        f.ok = f.x >= 0 && f.x < P.V;
+        if (f.ok) {
+            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + tid) * P.tstride;
+            const char* drow = P.drf + ((size_t)b * gamma + tid) * P.dstride;
+            f.l = ld_elem<TDT>(trow, f.x);
+            if constexpr (DK == DK_PROBS) f.d = __ldg(reinterpret_cast<const float*>(drow) + f.x);
+            else f.d = ld_elem<DDT>(drow, f.x);
+        }
+    }
+    return f;
+}
+
+// Chain decision for sequence b (rule 1), after the row statistics were
+// combined into sh.m / sh.z / sh.bad.  Threads 0..gamma-1 turn their
+// prefetched logits into p_i(x_i) and q_i(x_i) (fp64 exp2 in the units of the
+// row statistics); thread 0 then takes the decisions.  Leaves sh.ivals[0] =
+// valid, sh.ivals[1] = k, sh.dvals[0] = s.  When `write` is set it also writes
+// the accepted tokens, the -1 tail (position k excluded), num_accepted and
+// the p/q diagnostics, and flags invalid sequences.  Ends with __syncthreads.
+template <int TDT, int DDT, int DK>
+__device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, const ChainPrefetch& f) {
     const int tid = threadIdx.x;
-    const int gamma = P.gamma, V = P.V, W = gamma + 1;
+    const int gamma = P.gamma, W = gamma + 1;
     int32_t* toks = P.out_tokens + (size_t)b * W;
     float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
     const float T = P.temperature[b];
-    const int32_t* x = P.draft_tokens + (size_t)b * gamma;
     const bool tok = temperature_ok(T);
     const float s = tok ? scale_of(T) : 0.f;
     if (tid < gamma) {
-        const int xi = x[tid];
-        bool ok = xi >= 0 && xi < V;
+        bool ok = f.ok;
         double p = 0.0, q = 0.0;
         if (ok && tok) {
-            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + tid) * P.tstride;
-            const char* drow = P.drf + ((size_t)b * gamma + tid) * P.dstride;
-            p = prob_d(ld_elem<TDT>(trow, xi), s, sh.m[tid], sh.z[tid]);
+            p = prob_d(f.l, s, sh.m[tid], sh.z[tid]);
             if constexpr (DK == DK_PROBS) {
-                q = (double)__ldg(reinterpret_cast<const float*>(drow) + xi);
+                q = (double)f.d;
                 ok &= (q >= 0.0 && q <= 3.0e38);
             } else {
-                q = prob_d(ld_elem<DDT>(drow, xi), s, sh.m[gamma + 1 + tid], sh.z[gamma + 1 + tid]);
+                q = prob_d(f.d, s, sh.m[gamma + 1 + tid], sh.z[gamma + 1 + tid]);
             }
         }
         sh.pch[tid] = p;
         sh.pch[SPEC_MAX_GAMMA + tid] = q;
         sh.rej[tid] = ok;
+        sh.tok[tid] = f.x;
     }
     __syncthreads();
     if (tid == 0) {
@@ -746,7 +809,7 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write) 
                 if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
                 flag_input_error(P);
             } else {
-                for (int i = 0; i < k; ++i) toks[i] = x[i];
+                for (int i = 0; i < k; ++i) toks[i] = sh.tok[i];
                 for (int i = k + 1; i < W; ++i) toks[i] = -1;
                 P.out_num_accepted[b] = k;
                 if (dg)
@@ -1093,10 +1156,11 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     const int b = blockIdx.x / nsl, sl = blockIdx.x - b * nsl;
     const int c0 = (int)((long long)nch * sl / nsl), c1 = (int)((long long)nch * (sl + 1) / nsl);
     const int gamma = P.gamma, V = P.V;
+    const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
     pdl_wait();
     combine_softmax_rows(P, b, P.R, sh);
     __syncthreads();
-    chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0);
+    chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
     const float s = (float)sh.dvals[0];
     if (!ok) return;
@@ -1176,6 +1240,192 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
             __threadfence();
             P.cnt2[b] = 0u;
         }
+    }
+}
+
+// Eight elements e0..e0+7 of a row staged in shared memory: elements below
+// `nstaged` come from the stage, the rest below V from global memory, the
+// rest are `fill`.
+template <int DT>
+__device__ __forceinline__ void ld8_staged(const unsigned char* stage, const char* row, int64_t e0, int nstaged,
+                                           int V, float fill, float (&x)[8]) {
+    if (e0 + 8 <= nstaged) {
+        if constexpr (DT == SPEC_BF16) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + e0 * 2);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = vec_elem<DT>(v, i);
+        } else {
+            const uint4 a = *reinterpret_cast<const uint4*>(stage + e0 * 4);
+            const uint4 b = *reinterpret_cast<const uint4*>(stage + e0 * 4 + 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { x[i] = vec_elem<DT>(a, i); x[4 + i] = vec_elem<DT>(b, i); }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t e = e0 + i;
+            if (e < nstaged) {
+                if constexpr (DT == SPEC_BF16)
+                    x[i] = __uint_as_float((uint32_t)reinterpret_cast<const unsigned short*>(stage)[e] << 16);
+                else
+                    x[i] = reinterpret_cast<const float*>(stage)[e];
+            } else {
+                x[i] = e < V ? ld_elem<DT>(row, e) : fill;
+            }
+        }
+    }
+}
+
+// max(0, p_j - q_j) read from a staged row pair.
+template <int TDT, int DDT, int DK> struct WChainResStaged {
+    const unsigned char* ts; const unsigned char* ds; const char* trow; const char* drow;
+    int nt, nd; float s, mp, izp, mq, izq; int V;
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8_staged<TDT>(ts, trow, e0, nt, V, -INFINITY, x);
+        if constexpr (DK == DK_PROBS) ld8_staged<SPEC_F32>(ds, drow, e0, nd, V, 0.f, d);
+        else ld8_staged<DDT>(ds, drow, e0, nd, V, -INFINITY, d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float p = ex2(fmaf(x[i], s, -mp)) * izp;
+            const float q = (DK == DK_PROBS) ? d[i] : ex2(fmaf(d[i], s, -mq)) * izq;
+            w[i] = fmaxf(0.f, p - q);
+        }
+    }
+};
+
+// Shared-memory bytes of the row-staged chain finalisation.
+__host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
+    const size_t bt = ((size_t)V * tesz) & ~(size_t)15, bd = ((size_t)V * desz) & ~(size_t)15;
+    return bt + bd + (size_t)((V + 7) / 8) * 4;
+}
+
+// Chain finalisation with the rejected row pair staged in shared memory, one
+// CTA per sequence (used when the pair fits and the batch fits in one wave).
+// The decision inputs are prefetched before waiting for the statistics
+// kernel; after the decision, target row k and draft row k arrive with two
+// 1-D bulk copies (TMA) on one mbarrier; max(0, p - q) is evaluated once per
+// element into 8-element group sums, the group sums are scanned block-wide in
+// fp64 in index order, and only the group holding u*S is recomputed to pick
+// the token.  The bonus token (k = gamma) is drawn as in the sliced kernel.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
+    __shared__ FinShared sh;
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int owner, found_g;
+    extern __shared__ __align__(128) unsigned char stage[];
+    constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
+    const int tid = threadIdx.x, b = blockIdx.x;
+    const int gamma = P.gamma, V = P.V;
+    const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
+    if (tid == 0) mbar_init(smem_u32(&bar), 1);
+    pdl_wait();
+    combine_softmax_rows(P, b, P.R, sh);
+    __syncthreads();
+    chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
+    const int ok = sh.ivals[0], k = sh.ivals[1];
+    const float s = (float)sh.dvals[0];
+    if (!ok) return;
+    const float u = P.final_u[b];
+    int32_t* toks = P.out_tokens + (size_t)b * (gamma + 1);
+    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
+    if (k == gamma) {
+        const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * SPC;
+        double S;
+        int y = sample_target_row<TDT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        if (tid == 0) {
+            toks[k] = y;
+            if (dg) dg[2 * gamma] = 1.0f;
+        }
+        return;
+    }
+    const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
+    const uint32_t bt = ((uint32_t)V * Tr<TDT>::ESZ) & ~15u, bd = ((uint32_t)V * DESZ) & ~15u;
+    unsigned char* ts = stage;
+    unsigned char* ds = stage + bt;
+    float* gs = reinterpret_cast<float*>(stage + bt + bd);
+    if (tid == 0) {
+        mbar_expect_tx(smem_u32(&bar), bt + bd);
+        if (bt) bulk_g2s(smem_u32(ts), trow, bt, smem_u32(&bar));
+        if (bd) bulk_g2s(smem_u32(ds), drow, bd, smem_u32(&bar));
+    }
+    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]);
+    const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
+    const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
+    WChainResStaged<TDT, DDT, DK> wf{ts, ds, trow, drow, (int)(bt / Tr<TDT>::ESZ), (int)(bd / DESZ),
+                                     s, mp, izp, mq, izq, V};
+    if (!mbar_wait(smem_u32(&bar), 0)) {
+        // the copy did not land in time: report, let it finish (bounded), give up on b
+        if (tid == 0) {
+            atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
+            mbar_wait(smem_u32(&bar), 0);
+            for (int i = 0; i <= gamma; ++i) toks[i] = -1;
+            P.out_num_accepted[b] = -1;
+        }
+        return;
+    }
+    // group sums of max(0, p_k - q_k), groups g = tid + i*NT (conflict-free)
+    const int G = (V + 7) / 8;
+    for (int g = tid; g < G; g += NT) {
+        float w[8];
+        wf.group((int64_t)g * 8, w);
+        gs[g] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+    }
+    __syncthreads();
+    // fp64 scan over contiguous ranges of groups, in index order
+    const int g0 = (int)((long long)G * tid / NT), g1 = (int)((long long)G * (tid + 1) / NT);
+    double seg = 0.0;
+    for (int g = g0; g < g1; ++g) seg += (double)gs[g];
+    if (tid == 0) { owner = -1; found_g = -1; }
+    double S;
+    const double excl = block_excl_scan(seg, &S);
+    const double t = (double)u * S;
+    if (seg > 0.0 && excl <= t) atomicMax(&owner, tid);
+    __syncthreads();
+    int y = -1;
+    if (S > 0.0) {
+        if (tid == owner) {
+            double acc = excl;
+            int gsel = -1, glast = -1;
+            double before = excl;
+            for (int g = g0; g < g1; ++g) {
+                const double v = (double)gs[g];
+                if (v > 0.0) {
+                    glast = g;
+                    before = acc;
+                    if (t < acc + v) { gsel = g; break; }
+                }
+                acc += v;
+            }
+            if (gsel < 0) gsel = glast;
+            float w[8];
+            wf.group((int64_t)gsel * 8, w);
+            const double loc = t - before;
+            double a = 0.0;
+            int pick = -1, last = -1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                a += (double)w[i];
+                if (w[i] > 0.f) {
+                    last = gsel * 8 + i;
+                    if (pick < 0 && loc < a) pick = gsel * 8 + i;
+                }
+            }
+            found_g = pick >= 0 ? pick : last;
+        }
+        __syncthreads();
+        y = found_g;
+    }
+    if (y < 0) {
+        // empty residual (rounding only): draw from p_k
+        const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * SPC;
+        double Su;
+        y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+    }
+    if (tid == 0) {
+        toks[k] = y;
+        if (dg) dg[2 * gamma] = (float)S;
     }
 }
 
@@ -1328,11 +1578,47 @@ spec_status launch_dependent(K kernel, unsigned grid, const Params& P, cudaStrea
     return launched(what);
 }
 
+// Dynamic shared memory available to the row-staged finalisation (0 if it
+// cannot be configured).
+template <int TDT, int DDT, int DK>
+size_t row_stage_capacity() {
+    auto kern = k_chain_final_row<TDT, DDT, DK>;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 0;
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    const long long cap = (long long)optin - (long long)fa.sharedSizeBytes - 1024;
+    if (cap <= 0) return 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap) != cudaSuccess) return 0;
+    return (size_t)cap;
+}
+
 template <int TDT, int DDT, int DK>
 spec_status launch_chain(Params P, cudaStream_t st) {
     // draft probabilities are read only by the finalize kernel
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
+    // Row-staged finalisation when the rejected row pair fits in shared memory
+    // and one CTA per sequence fits in a single wave.
+    static const size_t cap = row_stage_capacity<TDT, DDT, DK>();
+    const size_t need = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
+    if (P.nch > 1 && need <= cap && P.B <= num_sms()) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)P.B);
+        cfg.blockDim = dim3(NT);
+        cfg.dynamicSmemBytes = need;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, k_chain_final_row<TDT, DDT, DK>, P);
+        if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "k_chain_final_row launch: %s", cudaGetErrorString(e));
+        return launched("k_chain_final_row");
+    }
     // enough CTAs to cover the SMs twice, at most one per chunk
     int nsl = (2 * num_sms() + P.B - 1) / P.B;
     P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
