@@ -42,6 +42,7 @@ constexpr int NT = 128;               // threads per CTA
 constexpr int NWARP = NT / 32;
 constexpr int VPT = 8;                // 16-byte vectors per thread per 16 KB chunk
 constexpr int SPC = NWARP;            // statistics per chunk (one per warp)
+constexpr int STATS_CTAS_PER_SM = 10; // occupancy target of the statistics kernel
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1 or N)
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
@@ -59,6 +60,8 @@ struct Params {
     int B, V, R, nch, gamma, N, max_depth;
     int rows_tgt;                  // target rows per sequence
     int nsl;                       // chain finalisation: CTAs (slices of chunks) per sequence
+    int stage_cap;                 // finalize kernels: shared bytes for a sequence's statistics
+    int stage_off;                 // row-staged chain finalisation: offset of that area
     const char* tgt;
     int64_t tstride;               // bytes between consecutive target rows
     const char* drf;
@@ -201,6 +204,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+
+// Stage sequence b's statistics block (R rows of nch*SPC float2, contiguous)
+// in shared memory with one bulk copy when it fits in `cap` bytes; returns
+// where to read it (shared memory, or global memory when it does not fit or
+// the bounded wait ran out).  All threads of the CTA must call it.
+__device__ const float2* stage_stats(const Params& P, int b, int R, unsigned char* buf, size_t cap,
+                                     uint64_t* bar) {
+    const size_t bytes = (size_t)R * P.nch * SPC * sizeof(float2);
+    const float2* src = P.stats + (size_t)b * P.R * P.nch * SPC;
+    if (bytes > cap || buf == nullptr) return src;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(bar), 1);
+        mbar_expect_tx(smem_u32(bar), (uint32_t)bytes);
+        bulk_g2s(smem_u32(buf), src, (uint32_t)bytes, smem_u32(bar));
+    }
+    __syncthreads();
+    if (mbar_wait(smem_u32(bar), 0)) return reinterpret_cast<const float2*>(buf);
+    // the copy did not land in time: report, let it land (bounded), read global
+    if (threadIdx.x == 0) atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
+    mbar_wait(smem_u32(bar), 0);
+    return src;
 }
 
 __device__ __forceinline__ void flag_input_error(const Params& P) {
@@ -404,18 +429,20 @@ struct FinShared {
 };
 
 // Combine the per-warp softmax statistics of rows [0, R) into (m, Z, bad).
-__device__ void combine_softmax_rows(const Params& P, int b, int R, FinShared& sh) {
+// `blk` is sequence b's statistics block ([R][nch][SPC]), in shared memory
+// when staged, else in global memory (written by the previous kernel).
+__device__ void combine_softmax_rows(const Params& P, const float2* blk, int R, FinShared& sh) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = P.nch * SPC;
     for (int r = warp; r < R; r += NWARP) {
-        const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        const float2* st = blk + (size_t)r * E;
         // one pass: each lane keeps an online (max, sum) over its entries
         float m = -INFINITY;
         double z = 0.0;
         bool bad = false;
 #pragma unroll 4
         for (int e = lane; e < E; e += 32) {
-            const float2 x = ldcg2(st + e);
+            const float2 x = st[e];
             bad |= (x.y != x.y);
             if (x.x > m) {
                 z = (m > -INFINITY ? z * (double)ex2(m - x.x) : 0.0) + (double)x.y;
@@ -466,32 +493,70 @@ template <int DT> __device__ __forceinline__ void ld8(const char* row, int64_t e
     }
 }
 
+// Eight consecutive elements of a row held as raw 16-byte vectors (one for
+// bf16, two for f32): loaded without bounds checks when the whole group lies
+// inside the row, so that several groups' loads can be in flight at once.
+template <int DT> struct Raw8 {
+    uint4 v[DT == SPEC_BF16 ? 1 : 2];
+};
+template <int DT> __device__ __forceinline__ void load_raw8(const char* row, int64_t e0, Raw8<DT>& r) {
+    if constexpr (DT == SPEC_BF16) {
+        r.v[0] = ld_stream(row + e0 * 2);
+    } else {
+        r.v[0] = ld_stream(row + e0 * 4);
+        r.v[1] = ld_stream(row + e0 * 4 + 16);
+    }
+}
+template <int DT> __device__ __forceinline__ void raw8_f32(const Raw8<DT>& r, float (&x)[8]) {
+    if constexpr (DT == SPEC_BF16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = vec_elem<DT>(r.v[0], i);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { x[i] = vec_elem<DT>(r.v[0], i); x[4 + i] = vec_elem<DT>(r.v[1], i); }
+    }
+}
+
 __device__ __forceinline__ bool excluded(const uint32_t* bitmap, int base, int64_t j) {
     const int o = (int)(j - base);
     return (bitmap[o >> 5] >> (o & 31)) & 1u;
 }
 
 // Weight functors of the inverse-CDF draws.  group(e0, w) gives the (f32)
-// weights of elements e0..e0+7 (0 past V); chunk sums and rescans both use it.
+// weights of elements e0..e0+7 (0 past V); for groups wholly inside the row
+// the same weights come from load(e0, raw) followed by weights(e0, raw, w).
+// Chunk sums and rescans both use them, so the arithmetic is identical.
 template <int TDT> struct WTarget {          // 2^(x_j - m), excluded tokens 0
     const char* row; float s, m; const uint32_t* bitmap; int base; int V;
-    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
-        float x[8];
-        ld8<TDT>(row, e0, V, -INFINITY, x);
+    struct Raw { Raw8<TDT> t; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const { load_raw8<TDT>(row, e0, r.t); }
+    __device__ __forceinline__ void finish(int64_t e0, const float (&x)[8], float (&w)[8]) const {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             w[i] = ex2(fmaf(x[i], s, -m));
             if (bitmap && e0 + i < V && excluded(bitmap, base, e0 + i)) w[i] = 0.f;
         }
     }
+    __device__ __forceinline__ void weights(int64_t e0, const Raw& r, float (&w)[8]) const {
+        float x[8];
+        raw8_f32<TDT>(r.t, x);
+        finish(e0, x, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8];
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+        finish(e0, x, w);
+    }
 };
 template <int TDT, int DDT, int DK> struct WChainRes {   // max(0, p_j - q_j)
+    static constexpr int QDT = DK == DK_PROBS ? SPEC_F32 : DDT;
     const char* trow; const char* drow; float s, mp, izp, mq, izq; int V;
-    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
-        float x[8], d[8];
-        ld8<TDT>(trow, e0, V, -INFINITY, x);
-        if constexpr (DK == DK_PROBS) ld8<SPEC_F32>(drow, e0, V, 0.f, d);
-        else ld8<DDT>(drow, e0, V, -INFINITY, d);
+    struct Raw { Raw8<TDT> t; Raw8<QDT> d; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const {
+        load_raw8<TDT>(trow, e0, r.t);
+        load_raw8<QDT>(drow, e0, r.d);
+    }
+    __device__ __forceinline__ void finish(const float (&x)[8], const float (&d)[8], float (&w)[8]) const {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float p = ex2(fmaf(x[i], s, -mp)) * izp;
@@ -499,36 +564,93 @@ template <int TDT, int DDT, int DK> struct WChainRes {   // max(0, p_j - q_j)
             w[i] = fmaxf(0.f, p - q);
         }
     }
+    __device__ __forceinline__ void weights(int64_t, const Raw& r, float (&w)[8]) const {
+        float x[8], d[8];
+        raw8_f32<TDT>(r.t, x);
+        raw8_f32<QDT>(r.d, d);
+        finish(x, d, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8<TDT>(trow, e0, V, -INFINITY, x);
+        if constexpr (DK == DK_PROBS) ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        else ld8<DDT>(drow, e0, V, -INFINITY, d);
+        finish(x, d, w);
+    }
 };
 template <int TDT> struct WTreeRes {         // relu(p_j - d_j), excluded tokens 0
     const char* row; const char* drow; float s, m, iz; const uint32_t* bitmap; int base; int V;
-    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
-        float x[8], d[8];
-        ld8<TDT>(row, e0, V, -INFINITY, x);
-        ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+    struct Raw { Raw8<TDT> t; Raw8<SPEC_F32> d; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const {
+        load_raw8<TDT>(row, e0, r.t);
+        load_raw8<SPEC_F32>(drow, e0, r.d);
+    }
+    __device__ __forceinline__ void finish(int64_t e0, const float (&x)[8], const float (&d)[8],
+                                           float (&w)[8]) const {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             w[i] = fmaxf(0.f, ex2(fmaf(x[i], s, -m)) * iz - d[i]);
             if (bitmap && e0 + i < V && excluded(bitmap, base, e0 + i)) w[i] = 0.f;
         }
     }
+    __device__ __forceinline__ void weights(int64_t e0, const Raw& r, float (&w)[8]) const {
+        float x[8], d[8];
+        raw8_f32<TDT>(r.t, x);
+        raw8_f32<SPEC_F32>(r.d, d);
+        finish(e0, x, d, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+        ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        finish(e0, x, d, w);
+    }
 };
 
-// Sum of the weights of chunk c, per thread (groups g = k*NT + tid, coalesced).
+// Group sums of the GPT groups this thread owns in chunk c (groups
+// g = k*NT + tid, coalesced).  For a chunk wholly inside the row, four groups'
+// loads are issued before any of them is used.
+template <int CH, class WF>
+__device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs)[CH / 8 / NT]) {
+    constexpr int GPT = CH / 8 / NT;
+    constexpr int BATCH = GPT < 4 ? GPT : 4;
+    const int64_t c0 = (int64_t)c * CH;
+    if (c0 + CH <= wf.V) {
+#pragma unroll
+        for (int k0 = 0; k0 < GPT; k0 += BATCH) {
+            typename WF::Raw raw[BATCH];
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) wf.load(c0 + (int64_t)((k0 + i) * NT + threadIdx.x) * 8, raw[i]);
+#pragma unroll
+            for (int i = 0; i < BATCH; ++i) {
+                float w[8];
+                wf.weights(c0 + (int64_t)((k0 + i) * NT + threadIdx.x) * 8, raw[i], w);
+                gs[k0 + i] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < GPT; ++k) {
+            gs[k] = 0.f;
+            const int64_t e0 = c0 + (int64_t)(k * NT + threadIdx.x) * 8;
+            if (e0 < wf.V) {
+                float w[8];
+                wf.group(e0, w);
+                gs[k] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+            }
+        }
+    }
+}
+
+// Sum of the weights of chunk c over this thread's groups.
 template <int CH, class WF>
 __device__ __forceinline__ float chunk_weight_partial(const WF& wf, int c) {
     constexpr int GPT = CH / 8 / NT;
+    float gs[GPT];
+    chunk_group_sums<CH>(wf, c, gs);
     float acc = 0.f;
 #pragma unroll
-    for (int k = 0; k < GPT; ++k) {
-        const int64_t e0 = (int64_t)c * CH + (int64_t)(k * NT + threadIdx.x) * 8;
-        if (e0 < wf.V) {
-            float w[8];
-            wf.group(e0, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc += w[i];
-        }
-    }
+    for (int k = 0; k < GPT; ++k) acc += gs[k];
     return acc;
 }
 
@@ -546,17 +668,7 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
     __shared__ int owner, found;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float gs[GPT];
-#pragma unroll
-    for (int k = 0; k < GPT; ++k) {
-        gs[k] = 0.f;
-        const int64_t e0 = (int64_t)c * CH + (int64_t)(k * NT + tid) * 8;
-        if (e0 < V) {
-            float w[8];
-            wf.group(e0, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) gs[k] += w[i];
-        }
-    }
+    chunk_group_sums<CH>(wf, c, gs);
     double inc[GPT];
 #pragma unroll
     for (int k = 0; k < GPT; ++k) {
@@ -824,18 +936,18 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
 }
 
 template <int TDT>
-__device__ void finalize_greedy(const Params& P, int b, FinShared& sh) {
+__device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
     const int E = P.nch * SPC;
     // per-node argmax (lowest index among equal maxima)
     for (int r = warp; r < N; r += NWARP) {
-        const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        const float2* st = blk + (size_t)r * E;
         float best = -INFINITY;
         int idx = 0x7fffffff;
         bool bad = false;
         for (int e = lane; e < E; e += 32) {
-            float2 x = ldcg2(st + e);
+            const float2 x = st[e];
             int xi = __float_as_int(x.y);
             if (x.x != x.x) bad = true;
             else if (x.x > best || (x.x == best && xi < idx)) { best = x.x; idx = xi; }
@@ -894,10 +1006,10 @@ __device__ void finalize_greedy(const Params& P, int b, FinShared& sh) {
 }
 
 template <int TDT>
-__device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
+__device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
-    combine_softmax_rows(P, b, N, sh);
+    combine_softmax_rows(P, blk, N, sh);
     for (int n = tid; n < N; n += NT) {
         sh.par[n] = P.parents[(size_t)b * N + n];
         sh.tok[n] = P.tokens[(size_t)b * N + n];
@@ -1059,15 +1171,16 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh) {
 
 // Row statistics (the streaming kernel).  The B*R*nch work items (sequence-
 // major, then row, then chunk; a chunk is 16 KB of one row) are split into
-// gridDim.x contiguous ranges, one per CTA; (b, r, c) advance incrementally.
-// Each thread loads its eight 16-byte vectors of a chunk at once; each warp
-// reduces its quarter to one statistic -- online softmax (max x, sum
-// 2^(x - max)) or (max, lowest index) -- and writes it.  Nothing else is
-// shared: no atomics, no fences; the finalize kernel that follows in stream
-// order reads the statistics.  Ten CTAs of four warps per SM keep enough
-// loads in flight and enough warps to hide the exp2 and ALU latency.
+// gridDim.x contiguous ranges of equal length (within one), one per CTA;
+// (b, r, c) advance incrementally.  Each thread loads its eight 16-byte
+// vectors of a chunk at once; each warp reduces its quarter to one statistic
+// -- online softmax (max x, sum 2^(x - max)) or (max, lowest index) -- and
+// writes it.  Nothing else is shared: no atomics, no fences; the finalize
+// kernel that follows in stream order reads the statistics.  Ten CTAs of four
+// warps per SM (at most 51 registers) keep enough loads in flight and enough
+// warps to hide the exp2 and ALU latency.
 template <int MODE, int TDT, int DDT>
-__global__ void __launch_bounds__(NT) k_stats(const Params P) {
+__global__ void __launch_bounds__(NT, STATS_CTAS_PER_SM) k_stats(const Params P) {
     constexpr int CH = chunk_elems<TDT>();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_trigger();
@@ -1150,6 +1263,8 @@ template <int TDT, int DDT, int DK>
 __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     __shared__ FinShared sh;
     __shared__ int is_last;
+    __shared__ __align__(8) uint64_t sbar;
+    extern __shared__ __align__(128) unsigned char dyn[];
     constexpr int CH = chunk_elems<TDT>();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nsl = P.nsl, nch = P.nch;
@@ -1158,7 +1273,8 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     const int gamma = P.gamma, V = P.V;
     const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
     pdl_wait();
-    combine_softmax_rows(P, b, P.R, sh);
+    const float2* blk = stage_stats(P, b, P.R, dyn, P.stage_cap, &sbar);
+    combine_softmax_rows(P, blk, P.R, sh);
     __syncthreads();
     chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
@@ -1294,10 +1410,11 @@ template <int TDT, int DDT, int DK> struct WChainResStaged {
     }
 };
 
-// Shared-memory bytes of the row-staged chain finalisation.
+// Shared-memory bytes of the row-staged chain finalisation: the row pair,
+// the group sums, then (16-byte aligned) the statistics area.
 __host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
     const size_t bt = ((size_t)V * tesz) & ~(size_t)15, bd = ((size_t)V * desz) & ~(size_t)15;
-    return bt + bd + (size_t)((V + 7) / 8) * 4;
+    return (bt + bd + (size_t)((V + 7) / 8) * 4 + 15) & ~(size_t)15;
 }
 
 // Chain finalisation with the rejected row pair staged in shared memory, one
@@ -1311,16 +1428,17 @@ __host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
 template <int TDT, int DDT, int DK>
 __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
     __shared__ FinShared sh;
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t bar, sbar;
     __shared__ int owner, found_g;
     extern __shared__ __align__(128) unsigned char stage[];
     constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
     const int tid = threadIdx.x, b = blockIdx.x;
     const int gamma = P.gamma, V = P.V;
     const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
-    if (tid == 0) mbar_init(smem_u32(&bar), 1);
     pdl_wait();
-    combine_softmax_rows(P, b, P.R, sh);
+    const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
+    if (tid == 0) mbar_init(smem_u32(&bar), 1);
+    combine_softmax_rows(P, blk, P.R, sh);
     __syncthreads();
     chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
@@ -1433,9 +1551,12 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
 template <int MODE, int TDT>
 __global__ void __launch_bounds__(NT) k_tree_final(const Params P) {
     __shared__ FinShared sh;
+    __shared__ __align__(8) uint64_t sbar;
+    extern __shared__ __align__(128) unsigned char dyn[];
     pdl_wait();
-    if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT>(P, blockIdx.x, sh);
-    else finalize_sample<TDT>(P, blockIdx.x, sh);
+    const float2* blk = stage_stats(P, blockIdx.x, P.N, dyn, P.stage_cap, &sbar);
+    if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT>(P, blockIdx.x, sh, blk);
+    else finalize_sample<TDT>(P, blockIdx.x, sh, blk);
 }
 
 }  // namespace sv
@@ -1549,8 +1670,16 @@ spec_status launch_stats(const Params& P, cudaStream_t st) {
     auto kern = k_stats<MODE, TDT, DDT>;
     static const int occ = blocks_per_sm(kern);
     const long long items = (long long)P.B * P.R * P.nch;
-    long long grid = (long long)num_sms() * occ;
-    if (grid > items) grid = items;
+    // Up to 4 CTAs per resident slot when every CTA would own many chunks (the
+    // extra CTAs start as others retire, which keeps the CTAs out of
+    // lockstep); then as few CTAs as give every CTA the same number of chunks
+    // (within one), so that no CTA trails the rest by a whole chunk.
+    const long long resident = (long long)num_sms() * occ;
+    long long mult = items / (8 * resident);
+    mult = mult < 1 ? 1 : (mult > 4 ? 4 : mult);
+    const long long slots = resident * mult;
+    const long long per_cta = (items + slots - 1) / slots;
+    const long long grid = (items + per_cta - 1) / per_cta;
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
     kern<<<(unsigned)grid, NT, 0, st>>>(P);
     spec_status s = launched("k_stats");
@@ -1559,14 +1688,25 @@ spec_status launch_stats(const Params& P, cudaStream_t st) {
     return s;
 }
 
+// Shared memory for staging a sequence's statistics in the finalize kernels.
+constexpr int STAGE_STATS_MAX = 96 * 1024;
+
+// Allow a finalize kernel STAGE_STATS_MAX bytes of dynamic shared memory (once).
+template <class K>
+bool allow_stage(K kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, STAGE_STATS_MAX) ==
+           cudaSuccess;
+}
+
 // Launch a finalize kernel as a programmatic dependent of the statistics
 // kernel just enqueued on `st`.
 template <class K>
-spec_status launch_dependent(K kernel, unsigned grid, const Params& P, cudaStream_t st, const char* what) {
+spec_status launch_dependent(K kernel, unsigned grid, size_t smem, const Params& P, cudaStream_t st,
+                             const char* what) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1578,8 +1718,14 @@ spec_status launch_dependent(K kernel, unsigned grid, const Params& P, cudaStrea
     return launched(what);
 }
 
-// Dynamic shared memory available to the row-staged finalisation (0 if it
-// cannot be configured).
+// Bytes of one sequence's statistics block, or 0 when it is not staged.
+inline int stats_stage_bytes(const Params& P, int rows, size_t limit) {
+    const size_t bytes = (size_t)rows * P.nch * SPC * sizeof(float2);
+    return bytes <= limit ? (int)bytes : 0;
+}
+
+// Dynamic shared memory available to the row-staged chain finalisation (0 if
+// it cannot be configured).
 template <int TDT, int DDT, int DK>
 size_t row_stage_capacity() {
     auto kern = k_chain_final_row<TDT, DDT, DK>;
@@ -1600,36 +1746,32 @@ spec_status launch_chain(Params P, cudaStream_t st) {
     // draft probabilities are read only by the finalize kernel
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
-    // Row-staged finalisation when the rejected row pair fits in shared memory
-    // and one CTA per sequence fits in a single wave.
+    // Row-staged finalisation when the rejected row pair (and the statistics)
+    // fit in shared memory and one CTA per sequence fits in a single wave.
     static const size_t cap = row_stage_capacity<TDT, DDT, DK>();
-    const size_t need = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
-    if (P.nch > 1 && need <= cap && P.B <= num_sms()) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)P.B);
-        cfg.blockDim = dim3(NT);
-        cfg.dynamicSmemBytes = need;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, k_chain_final_row<TDT, DDT, DK>, P);
-        if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "k_chain_final_row launch: %s", cudaGetErrorString(e));
-        return launched("k_chain_final_row");
+    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
+    if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
+        P.stage_off = (int)pair;
+        P.stage_cap = stats_stage_bytes(P, P.R, cap - pair);
+        return launch_dependent(k_chain_final_row<TDT, DDT, DK>, (unsigned)P.B, pair + P.stage_cap, P, st,
+                                "k_chain_final_row");
     }
+    static const bool big = allow_stage(k_chain_final<TDT, DDT, DK>);
+    P.stage_cap = stats_stage_bytes(P, P.R, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     // enough CTAs to cover the SMs twice, at most one per chunk
     int nsl = (2 * num_sms() + P.B - 1) / P.B;
     P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
-    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), P, st, "k_chain_final");
+    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), P.stage_cap, P, st,
+                            "k_chain_final");
 }
 
 template <int MODE, int TDT>
-spec_status launch_tree(const Params& P, cudaStream_t st) {
+spec_status launch_tree(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
-    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, P, st, "k_tree_final");
+    static const bool big = allow_stage(k_tree_final<MODE, TDT>);
+    P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
+    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, P.stage_cap, P, st, "k_tree_final");
 }
 
 }  // namespace
