@@ -43,6 +43,7 @@ constexpr int NWARP = NT / 32;
 constexpr int VPT = 8;                // 16-byte vectors per thread per 16 KB chunk
 constexpr int SPC = NWARP;            // statistics per chunk (one per warp)
 constexpr int STATS_CTAS_PER_SM = 10; // occupancy target of the statistics kernel
+constexpr int SEQ_BT = 512;           // threads of the one-CTA-per-sequence finalize kernels
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1 or N)
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
@@ -232,9 +233,12 @@ __device__ __forceinline__ void flag_input_error(const Params& P) {
     atomicOr(P.status, 1u << SPEC_ERR_DEVICE_INPUT);
 }
 
-// Block-wide exclusive scan of one double per thread; *total receives the sum.
+// Block-wide exclusive scan of one double per thread (BT threads); *total
+// receives the sum.
+template <int BT>
 __device__ double block_excl_scan(double v, double* total) {
-    __shared__ double wsum[NWARP];
+    constexpr int BW = BT / 32;
+    __shared__ double wsum[BW];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     double inc = v;
 #pragma unroll
@@ -246,7 +250,7 @@ __device__ double block_excl_scan(double v, double* total) {
     __syncthreads();
     double before = 0.0, tot = 0.0;
 #pragma unroll
-    for (int w = 0; w < NWARP; ++w) {
+    for (int w = 0; w < BW; ++w) {
         if (w < warp) before += wsum[w];
         tot += wsum[w];
     }
@@ -431,10 +435,11 @@ struct FinShared {
 // Combine the per-warp softmax statistics of rows [0, R) into (m, Z, bad).
 // `blk` is sequence b's statistics block ([R][nch][SPC]), in shared memory
 // when staged, else in global memory (written by the previous kernel).
+template <int BT>
 __device__ void combine_softmax_rows(const Params& P, const float2* blk, int R, FinShared& sh) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int E = P.nch * SPC;
-    for (int r = warp; r < R; r += NWARP) {
+    for (int r = warp; r < R; r += BT / 32) {
         const float2* st = blk + (size_t)r * E;
         // one pass: each lane keeps an online (max, sum) over its entries
         float m = -INFINITY;
@@ -610,9 +615,9 @@ template <int TDT> struct WTreeRes {         // relu(p_j - d_j), excluded tokens
 // Group sums of the GPT groups this thread owns in chunk c (groups
 // g = k*NT + tid, coalesced).  For a chunk wholly inside the row, four groups'
 // loads are issued before any of them is used.
-template <int CH, class WF>
-__device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs)[CH / 8 / NT]) {
-    constexpr int GPT = CH / 8 / NT;
+template <int CH, int BT, class WF>
+__device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs)[CH / 8 / BT]) {
+    constexpr int GPT = CH / 8 / BT;
     constexpr int BATCH = GPT < 4 ? GPT : 4;
     const int64_t c0 = (int64_t)c * CH;
     if (c0 + CH <= wf.V) {
@@ -620,11 +625,11 @@ __device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs
         for (int k0 = 0; k0 < GPT; k0 += BATCH) {
             typename WF::Raw raw[BATCH];
 #pragma unroll
-            for (int i = 0; i < BATCH; ++i) wf.load(c0 + (int64_t)((k0 + i) * NT + threadIdx.x) * 8, raw[i]);
+            for (int i = 0; i < BATCH; ++i) wf.load(c0 + (int64_t)((k0 + i) * BT + threadIdx.x) * 8, raw[i]);
 #pragma unroll
             for (int i = 0; i < BATCH; ++i) {
                 float w[8];
-                wf.weights(c0 + (int64_t)((k0 + i) * NT + threadIdx.x) * 8, raw[i], w);
+                wf.weights(c0 + (int64_t)((k0 + i) * BT + threadIdx.x) * 8, raw[i], w);
                 gs[k0 + i] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
             }
         }
@@ -632,7 +637,7 @@ __device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs
 #pragma unroll
         for (int k = 0; k < GPT; ++k) {
             gs[k] = 0.f;
-            const int64_t e0 = c0 + (int64_t)(k * NT + threadIdx.x) * 8;
+            const int64_t e0 = c0 + (int64_t)(k * BT + threadIdx.x) * 8;
             if (e0 < wf.V) {
                 float w[8];
                 wf.group(e0, w);
@@ -643,11 +648,11 @@ __device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs
 }
 
 // Sum of the weights of chunk c over this thread's groups.
-template <int CH, class WF>
+template <int CH, int BT, class WF>
 __device__ __forceinline__ float chunk_weight_partial(const WF& wf, int c) {
-    constexpr int GPT = CH / 8 / NT;
+    constexpr int GPT = CH / 8 / BT;
     float gs[GPT];
-    chunk_group_sums<CH>(wf, c, gs);
+    chunk_group_sums<CH, BT>(wf, c, gs);
     float acc = 0.f;
 #pragma unroll
     for (int k = 0; k < GPT; ++k) acc += gs[k];
@@ -661,14 +666,15 @@ __device__ __forceinline__ float chunk_weight_partial(const WF& wf, int c) {
 // If t_loc < 0, t_loc = u * (chunk total) (single-chunk rows).  Returns the
 // drawn index, or -1 when the chunk has no positive weight; *chunk_total gets
 // the chunk's sum.
-template <int CH, class WF>
+template <int CH, int BT, class WF>
 __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, double* chunk_total) {
-    constexpr int GPT = CH / 8 / NT;
-    __shared__ double wt[GPT][NWARP];
+    constexpr int GPT = CH / 8 / BT;
+    constexpr int BW = BT / 32;
+    __shared__ double wt[GPT][BW];
     __shared__ int owner, found;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float gs[GPT];
-    chunk_group_sums<CH>(wf, c, gs);
+    chunk_group_sums<CH, BT>(wf, c, gs);
     double inc[GPT];
 #pragma unroll
     for (int k = 0; k < GPT; ++k) {
@@ -686,7 +692,7 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
 #pragma unroll
     for (int k = 0; k < GPT; ++k)
 #pragma unroll
-        for (int w = 0; w < NWARP; ++w) total += wt[k][w];
+        for (int w = 0; w < BW; ++w) total += wt[k][w];
     if (chunk_total) *chunk_total = total;
     if (t_loc < 0.0) t_loc = (double)u * total;
     double base = 0.0;
@@ -694,19 +700,19 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
     for (int k = 0; k < GPT; ++k) {
         double before = base;
 #pragma unroll
-        for (int w = 0; w < NWARP; ++w) if (w < warp) before += wt[k][w];
+        for (int w = 0; w < BW; ++w) if (w < warp) before += wt[k][w];
         const double excl = before + inc[k] - (double)gs[k];
-        if (gs[k] > 0.f && excl <= t_loc) atomicMax(&owner, k * NT + tid);
+        if (gs[k] > 0.f && excl <= t_loc) atomicMax(&owner, k * BT + tid);
 #pragma unroll
-        for (int w = 0; w < NWARP; ++w) base += wt[k][w];
+        for (int w = 0; w < BW; ++w) base += wt[k][w];
     }
     __syncthreads();
     const int og = owner;
-    if (og >= 0 && (og % NT) == tid) {
-        const int k = og / NT;
+    if (og >= 0 && (og % BT) == tid) {
+        const int k = og / BT;
         double before = 0.0;
         for (int kk = 0; kk < k; ++kk)
-            for (int w = 0; w < NWARP; ++w) before += wt[kk][w];
+            for (int w = 0; w < BW; ++w) before += wt[kk][w];
         for (int w = 0; w < warp; ++w) before += wt[k][w];
         double excl = 0.0;
 #pragma unroll
@@ -739,12 +745,12 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
 // statistics (fp64), excluded tokens are subtracted from their chunk, the
 // chunk holding u*S is rescanned.  *S_unnorm = remaining mass in units of
 // 2^(x - m).  Returns the token (or -1 if nothing is left).
-template <int TDT>
+template <int TDT, int BT>
 __device__ int sample_target_row(const char* row, int V, int nch, const float2* st, float s, float m,
                                  float u, const int* excl, int nexcl, FinShared& sh, double* S_unnorm) {
     constexpr int CH = chunk_elems<TDT>();
     const int tid = threadIdx.x;
-    for (int c = tid; c < nch; c += NT) {
+    for (int c = tid; c < nch; c += BT) {
         double M = 0.0;
 #pragma unroll
         for (int w = 0; w < SPC; ++w) {
@@ -794,16 +800,16 @@ __device__ int sample_target_row(const char* row, int V, int nch, const float2* 
         __syncthreads();
         const int cs = sh.ivals[0];
         if (cs < 0) break;
-        for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+        for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
         __syncthreads();
-        for (int i = tid; i < nexcl; i += NT) {
+        for (int i = tid; i < nexcl; i += BT) {
             int o = excl[i] - cs * CH;
             if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
         }
         __syncthreads();
         WTarget<TDT> wf{row, s, m, nexcl ? sh.bitmap : nullptr, cs * CH, V};
         double tot;
-        result = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+        result = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
         if (result >= 0) break;
         if (tid == 0) sh.M[cs] = 0.0;         // nothing positive there after all: skip it
         __syncthreads();
@@ -812,18 +818,19 @@ __device__ int sample_target_row(const char* row, int V, int nch, const float2* 
 }
 
 // Validate a tree held in sh.par / sh.tok (N nodes); returns 1 if well formed.
+template <int BT>
 __device__ int tree_valid(const Params& P, int N, int V, int max_depth, FinShared& sh) {
     __shared__ int ok;
     if (threadIdx.x == 0) ok = 1;
     __syncthreads();
-    for (int n = threadIdx.x; n < N; n += NT) {
+    for (int n = threadIdx.x; n < N; n += BT) {
         int pa = sh.par[n];
         bool good = (n == 0) ? (pa == -1) : (pa >= 0 && pa < n && sh.tok[n] >= 0 && sh.tok[n] < V);
         if (!good) ok = 0;
     }
     __syncthreads();
     if (ok) {
-        for (int n = threadIdx.x; n < N; n += NT) {
+        for (int n = threadIdx.x; n < N; n += BT) {
             int d = 0, a = n;
             while (a > 0 && d <= max_depth) { a = sh.par[a]; ++d; }
             if (d > max_depth) ok = 0;
@@ -935,13 +942,13 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
     __syncthreads();
 }
 
-template <int TDT>
+template <int TDT, int BT>
 __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
     const int E = P.nch * SPC;
     // per-node argmax (lowest index among equal maxima)
-    for (int r = warp; r < N; r += NWARP) {
+    for (int r = warp; r < N; r += BT / 32) {
         const float2* st = blk + (size_t)r * E;
         float best = -INFINITY;
         int idx = 0x7fffffff;
@@ -961,12 +968,12 @@ __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const flo
         bad = __any_sync(FULL, bad);
         if (lane == 0) { sh.rej[r] = idx; sh.bad[r] = bad; }
     }
-    for (int n = tid; n < N; n += NT) {
+    for (int n = tid; n < N; n += BT) {
         sh.par[n] = P.parents[(size_t)b * N + n];
         sh.tok[n] = P.tokens[(size_t)b * N + n];
     }
     __syncthreads();
-    int ok = tree_valid(P, N, V, P.max_depth, sh);
+    int ok = tree_valid<BT>(P, N, V, P.max_depth, sh);
     if (tid == 0) {
         for (int r = 0; r < N; ++r) ok &= !sh.bad[r];
         sh.ivals[0] = ok;
@@ -976,7 +983,7 @@ __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const flo
     int32_t* ai = P.out_accept_index + (size_t)b * W;
     int32_t* ot = P.out_tokens + (size_t)b * W;
     if (!ok) {
-        for (int i = tid; i < W; i += NT) { ai[i] = -1; ot[i] = -1; }
+        for (int i = tid; i < W; i += BT) { ai[i] = -1; ot[i] = -1; }
         if (tid == 0) { P.out_num_accepted[b] = -1; flag_input_error(P); }
         return;
     }
@@ -1005,17 +1012,17 @@ __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const flo
     }
 }
 
-template <int TDT>
+template <int TDT, int BT>
 __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
-    combine_softmax_rows(P, blk, N, sh);
-    for (int n = tid; n < N; n += NT) {
+    combine_softmax_rows<BT>(P, blk, N, sh);
+    for (int n = tid; n < N; n += BT) {
         sh.par[n] = P.parents[(size_t)b * N + n];
         sh.tok[n] = P.tokens[(size_t)b * N + n];
     }
     __syncthreads();
-    int ok = tree_valid(P, N, V, P.max_depth, sh);
+    int ok = tree_valid<BT>(P, N, V, P.max_depth, sh);
     const float T = P.temperature[b];
     if (tid == 0) {
         ok &= temperature_ok(T);
@@ -1028,14 +1035,14 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     int32_t* ot = P.out_tokens + (size_t)b * W;
     float* dg = P.diag ? P.diag + (size_t)b * (N + 1) : nullptr;
     if (!ok) {
-        for (int i = tid; i < W; i += NT) { ai[i] = -1; ot[i] = -1; }
-        if (dg) for (int i = tid; i < N + 1; i += NT) dg[i] = nanf_();
+        for (int i = tid; i < W; i += BT) { ai[i] = -1; ot[i] = -1; }
+        if (dg) for (int i = tid; i < N + 1; i += BT) dg[i] = nanf_();
         if (tid == 0) { P.out_num_accepted[b] = -1; flag_input_error(P); }
         return;
     }
     const float s = scale_of(T);
     // p_parent(n)(tokens[n]) for every non-root node
-    for (int n = tid; n < N; n += NT) {
+    for (int n = tid; n < N; n += BT) {
         double pc = 0.0;
         if (n > 0) {
             int pa = sh.par[n];
@@ -1087,7 +1094,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     if (!P.draft_probs) {
         const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
         double Su;
-        y = sample_target_row<TDT>(row, V, P.nch, st, s, sh.m[cur], u, sh.rej, nrej, sh, &Su);
+        y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, sh.m[cur], u, sh.rej, nrej, sh, &Su);
         S = Su / sh.z[cur];
     } else {
         // relu(p_cur - d_cur) over the whole row: chunk sums, then one rescan.
@@ -1095,19 +1102,17 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * N + cur) * P.dpstride;
         const float m = sh.m[cur], iz = (float)(1.0 / sh.z[cur]);
         for (int c = 0; c < P.nch; ++c) {
-            for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+            for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
             __syncthreads();
-            for (int i = tid; i < nrej; i += NT) {
+            for (int i = tid; i < nrej; i += BT) {
                 int o = sh.rej[i] - c * CH;
                 if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
             }
             __syncthreads();
             WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, c * CH, V};
-            double part = (double)chunk_weight_partial<CH>(wf, c);
-            part = warp_sum_d(part);
-            if (lane == 0) sh.dvals[warp % 4] = part;     // NWARP == 4
-            __syncthreads();
-            if (tid == 0) sh.M[c] = sh.dvals[0] + sh.dvals[1] + sh.dvals[2] + sh.dvals[3];
+            double tot;
+            block_excl_scan<BT>((double)chunk_weight_partial<CH, BT>(wf, c), &tot);
+            if (tid == 0) sh.M[c] = tot;
             __syncthreads();
         }
         if (tid == 0) {
@@ -1138,16 +1143,16 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
                 __syncthreads();
                 const int cs = sh.ivals[4];
                 if (cs < 0) break;
-                for (int w = tid; w < CH / 32; w += NT) sh.bitmap[w] = 0u;
+                for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
                 __syncthreads();
-                for (int i = tid; i < nrej; i += NT) {
+                for (int i = tid; i < nrej; i += BT) {
                     int o = sh.rej[i] - cs * CH;
                     if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
                 }
                 __syncthreads();
                 WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, cs * CH, V};
                 double tot;
-                y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+                y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
                 if (y < 0 && tid == 0) sh.M[cs] = 0.0;
                 __syncthreads();
             }
@@ -1156,7 +1161,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
             // empty residual (rounding only): draw from p_cur itself
             const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
             double Su;
-            y = sample_target_row<TDT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
+            y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
         }
     }
     if (tid == 0) {
@@ -1223,7 +1228,7 @@ __global__ void __launch_bounds__(NT, STATS_CTAS_PER_SM) k_stats(const Params P)
 // Locate the chunk holding t among the chunk masses sh.M[0..nch) (skipping
 // empty chunks) and rescan it; retries past chunks whose rescan finds no
 // positive weight (possible only through rounding).  Returns -1 if none.
-template <int CH, class WF>
+template <int CH, int BT, class WF>
 __device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u, FinShared& sh) {
     const int tid = threadIdx.x;
     int y = -1;
@@ -1246,7 +1251,7 @@ __device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u,
         const int cs = sh.ivals[2];
         if (cs < 0) break;
         double tot;
-        y = rescan_chunk<CH>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+        y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
         if (y < 0 && tid == 0) sh.M[cs] = 0.0;
         __syncthreads();
     }
@@ -1274,7 +1279,7 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
     pdl_wait();
     const float2* blk = stage_stats(P, b, P.R, dyn, P.stage_cap, &sbar);
-    combine_softmax_rows(P, blk, P.R, sh);
+    combine_softmax_rows<NT>(P, blk, P.R, sh);
     __syncthreads();
     chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
@@ -1288,7 +1293,7 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
         if (sl != 0) return;
         const float2* st = P.stats + ((size_t)b * P.R + gamma) * nch * SPC;
         double S;
-        int y = sample_target_row<TDT>(trow, V, nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        int y = sample_target_row<TDT, NT>(trow, V, nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
         if (tid == 0) {
             toks[k] = y;
             if (dg) dg[2 * gamma] = 1.0f;
@@ -1302,7 +1307,7 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     WChainRes<TDT, DDT, DK> wf{trow, drow, s, mp, izp, mq, izq, V};
     // chunk sums of max(0, p_k - q_k) for this slice's chunks
     for (int c = c0; c < c1; ++c) {
-        const float ws = warp_sum(chunk_weight_partial<CH>(wf, c));
+        const float ws = warp_sum(chunk_weight_partial<CH, NT>(wf, c));
         if (lane == 0) {
             if (nsl == 1) sh.wp[c][warp] = ws;
             else P.stats2[((size_t)b * nch + c) * NWARP + warp] = make_float2(ws, 0.f);
@@ -1342,12 +1347,12 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     }
     __syncthreads();
     const double S = sh.dvals[0];
-    int y = (S > 0.0) ? draw_from_chunks<CH>(wf, nch, V, (double)u * S, u, sh) : -1;
+    int y = (S > 0.0) ? draw_from_chunks<CH, NT>(wf, nch, V, (double)u * S, u, sh) : -1;
     if (y < 0) {
         // empty residual (rounding only): draw from p_k
         const float2* stk = P.stats + ((size_t)b * P.R + k) * nch * SPC;
         double Su;
-        y = sample_target_row<TDT>(trow, V, nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+        y = sample_target_row<TDT, NT>(trow, V, nch, stk, s, mp, u, nullptr, 0, sh, &Su);
     }
     if (tid == 0) {
         toks[k] = y;
@@ -1426,7 +1431,7 @@ __host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
 // fp64 in index order, and only the group holding u*S is recomputed to pick
 // the token.  The bonus token (k = gamma) is drawn as in the sliced kernel.
 template <int TDT, int DDT, int DK>
-__global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
+__global__ void __launch_bounds__(SEQ_BT) k_chain_final_row(const Params P) {
     __shared__ FinShared sh;
     __shared__ __align__(8) uint64_t bar, sbar;
     __shared__ int owner, found_g;
@@ -1438,7 +1443,7 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
     pdl_wait();
     const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
     if (tid == 0) mbar_init(smem_u32(&bar), 1);
-    combine_softmax_rows(P, blk, P.R, sh);
+    combine_softmax_rows<SEQ_BT>(P, blk, P.R, sh);
     __syncthreads();
     chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
@@ -1451,7 +1456,7 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
     if (k == gamma) {
         const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * SPC;
         double S;
-        int y = sample_target_row<TDT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        int y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
         if (tid == 0) {
             toks[k] = y;
             if (dg) dg[2 * gamma] = 1.0f;
@@ -1485,19 +1490,19 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
     }
     // group sums of max(0, p_k - q_k), groups g = tid + i*NT (conflict-free)
     const int G = (V + 7) / 8;
-    for (int g = tid; g < G; g += NT) {
+    for (int g = tid; g < G; g += SEQ_BT) {
         float w[8];
         wf.group((int64_t)g * 8, w);
         gs[g] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
     }
     __syncthreads();
     // fp64 scan over contiguous ranges of groups, in index order
-    const int g0 = (int)((long long)G * tid / NT), g1 = (int)((long long)G * (tid + 1) / NT);
+    const int g0 = (int)((long long)G * tid / SEQ_BT), g1 = (int)((long long)G * (tid + 1) / SEQ_BT);
     double seg = 0.0;
     for (int g = g0; g < g1; ++g) seg += (double)gs[g];
     if (tid == 0) { owner = -1; found_g = -1; }
     double S;
-    const double excl = block_excl_scan(seg, &S);
+    const double excl = block_excl_scan<SEQ_BT>(seg, &S);
     const double t = (double)u * S;
     if (seg > 0.0 && excl <= t) atomicMax(&owner, tid);
     __syncthreads();
@@ -1539,7 +1544,7 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
         // empty residual (rounding only): draw from p_k
         const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * SPC;
         double Su;
-        y = sample_target_row<TDT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+        y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
     }
     if (tid == 0) {
         toks[k] = y;
@@ -1549,14 +1554,14 @@ __global__ void __launch_bounds__(NT) k_chain_final_row(const Params P) {
 
 // Tree finalisation, one CTA per sequence.
 template <int MODE, int TDT>
-__global__ void __launch_bounds__(NT) k_tree_final(const Params P) {
+__global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     __shared__ FinShared sh;
     __shared__ __align__(8) uint64_t sbar;
     extern __shared__ __align__(128) unsigned char dyn[];
     pdl_wait();
     const float2* blk = stage_stats(P, blockIdx.x, P.N, dyn, P.stage_cap, &sbar);
-    if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT>(P, blockIdx.x, sh, blk);
-    else finalize_sample<TDT>(P, blockIdx.x, sh, blk);
+    if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
+    else finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
 }
 
 }  // namespace sv
@@ -1701,11 +1706,11 @@ bool allow_stage(K kernel) {
 // Launch a finalize kernel as a programmatic dependent of the statistics
 // kernel just enqueued on `st`.
 template <class K>
-spec_status launch_dependent(K kernel, unsigned grid, size_t smem, const Params& P, cudaStream_t st,
-                             const char* what) {
+spec_status launch_dependent(K kernel, unsigned grid, unsigned block, size_t smem, const Params& P,
+                             cudaStream_t st, const char* what) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -1753,15 +1758,15 @@ spec_status launch_chain(Params P, cudaStream_t st) {
     if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
         P.stage_off = (int)pair;
         P.stage_cap = stats_stage_bytes(P, P.R, cap - pair);
-        return launch_dependent(k_chain_final_row<TDT, DDT, DK>, (unsigned)P.B, pair + P.stage_cap, P, st,
-                                "k_chain_final_row");
+        return launch_dependent(k_chain_final_row<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, pair + P.stage_cap, P,
+                                st, "k_chain_final_row");
     }
     static const bool big = allow_stage(k_chain_final<TDT, DDT, DK>);
     P.stage_cap = stats_stage_bytes(P, P.R, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     // enough CTAs to cover the SMs twice, at most one per chunk
     int nsl = (2 * num_sms() + P.B - 1) / P.B;
     P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
-    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), P.stage_cap, P, st,
+    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), NT, P.stage_cap, P, st,
                             "k_chain_final");
 }
 
@@ -1771,7 +1776,7 @@ spec_status launch_tree(Params P, cudaStream_t st) {
     if (s != SPEC_OK) return s;
     static const bool big = allow_stage(k_tree_final<MODE, TDT>);
     P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
-    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, P.stage_cap, P, st, "k_tree_final");
+    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st, "k_tree_final");
 }
 
 }  // namespace
