@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lazy-steps", type=int, default=400,
+                    help="steps of the row-on-demand (lazy) entry point timed beside the dense one (0: skip)")
     return ap.parse_args()
 
 
@@ -112,8 +114,8 @@ def describe(wid: int, inp) -> dict:
 class Runner:
     """Calls the verify entry point of a workload through the Python binding."""
 
-    def __init__(self, wid, inp, ws):
-        self.wid, self.inp, self.ws = wid, inp, ws
+    def __init__(self, wid, inp, ws, lazy=False):
+        self.wid, self.inp, self.ws, self.sfx = wid, inp, ws, "_lazy" if lazy else ""
         import torch
         B = inp.B
         dev = inp.target.device
@@ -130,15 +132,15 @@ class Runner:
         from speculative_decoding_verify_temperature_b200 import spec_verify as sv
         i = self.inp
         if self.wid in (0, 1, 4):
-            sv.spec_verify_chain(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
+            getattr(sv, "spec_verify_chain" + self.sfx)(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                  draft_is_probs=i.draft_is_probs, V=i.V, out_tokens=self.out[0],
                                  out_num_accepted=self.out[1], workspace=self.ws)
         elif self.wid == 2:
-            sv.spec_verify_tree_greedy(i.target, i.tokens, i.parents, i.max_depth, V=i.V,
+            getattr(sv, "spec_verify_tree_greedy" + self.sfx)(i.target, i.tokens, i.parents, i.max_depth, V=i.V,
                                        out_accept_index=self.out[0], out_tokens=self.out[1],
                                        out_num_accepted=self.out[2], workspace=self.ws)
         else:
-            sv.spec_verify_tree_sample(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
+            getattr(sv, "spec_verify_tree_sample" + self.sfx)(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
                                        i.max_depth, draft_probs=i.draft_probs, V=i.V,
                                        out_accept_index=self.out[0], out_tokens=self.out[1],
                                        out_num_accepted=self.out[2], workspace=self.ws)
@@ -150,6 +152,28 @@ class Runner:
 def kernels_per_step(wid, inp) -> int:
     """Launches per verify call: the row-statistics kernel and the finalize kernel."""
     return 2
+
+
+def lazy_kernels_per_step(wid, inp) -> int:
+    """Launches per lazy call: a statistics and a decision kernel per level (the
+    chain's last level has no decision), then the final draw (none for greedy)."""
+    if wid in (0, 1, 4):
+        return 2 * inp.gamma + 2
+    return 2 * (inp.max_depth + 1) + (1 if wid == 3 else 0)
+
+
+def lazy_bytes_read(wid, inp, num_accepted) -> int:
+    """Logit bytes the lazy walk streams for one round with these outcomes: chain
+    target rows 0..k (row gamma after a full accept) plus draft-logit rows 0..k
+    below gamma; trees the row of every node on the accepted path."""
+    k = num_accepted.clamp_min(0).long()
+    row_t = inp.V * inp.target.element_size()
+    if wid in (0, 1, 4):
+        n = int((k + 1).sum()) * row_t
+        if not inp.draft_is_probs:
+            n += int((k + 1).clamp_max(inp.gamma).sum()) * inp.V * inp.draft.element_size()
+        return n
+    return int((k + 1).sum()) * row_t
 
 
 def workspace_for(wid, inp):
@@ -429,6 +453,9 @@ def main():
     # --- end to end through the binding with host buffers
     e2e = run_e2e(wid, first, ws, args.e2e_steps, dev)
 
+    # --- the row-on-demand entry point on the same input sets
+    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 else None
+
     cfg = describe(wid, first)
     cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",
                l2=(f"{nsets} rotating input sets of {nbytes / 1e6:.1f} MB ({nsets * nbytes / 1e6:.0f} MB > 126 MB L2)"
@@ -442,7 +469,7 @@ def main():
         "round_hbm_gbs": round(round_gbs, 1),
         "draft_tokens_verified_per_s": round(value * draft_per_round, 1),
         "accepted_tokens_per_s": round(value * B * mean_tau, 1), "mean_tau": round(mean_tau, 4),
-        "e2e": e2e, "gpu_launches": K * kps, "clocks": sampler.summary(),
+        "e2e": e2e, "gpu_launches": K * kps, "clocks": sampler.summary(), "lazy": lazy,
     }
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wid, first, args.cpu_seconds)
@@ -454,6 +481,46 @@ def main():
         dist.barrier()
         del graph, singles
         dist.destroy_process_group()
+
+
+def run_lazy(wid, sets, ws, steps, alg, world, dev):
+    """Time the lazy entry point (whole rotations of the input sets in one CUDA
+    graph, CUDA events, max over ranks) and count the logit bytes it reads."""
+    import torch
+    runners = [Runner(wid, s, ws, lazy=True) for s in sets]
+    for _ in range(3):
+        for r in runners:
+            r()
+    torch.cuda.synchronize()
+    read = 0
+    for r, s in zip(runners, sets):
+        read += lazy_bytes_read(wid, s, r.num_accepted())
+    read /= len(sets)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for r in runners:
+            r()
+    reps = max(1, steps // len(runners))
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max_ms(e0.elapsed_time(e1), world, dev)
+    n = reps * len(runners)
+    del graph
+    return {"entry": "spec_verify_*_lazy (row-on-demand level walk)", "steps": n,
+            "ms_per_step": round(ms / n, 6), "value": round(job_value(n, world, ms), 2), "unit": "rounds/s",
+            "gpu_launches_per_step": lazy_kernels_per_step(wid, sets[0]),
+            "logit_bytes_read_per_step": int(read), "fraction_of_dense_bytes": round(read / alg, 4),
+            "achieved_gbs_on_bytes_read": round(read / (ms / n / 1e3) / 1e9, 1)}
 
 
 def run_e2e(wid, inp, ws, steps, dev):

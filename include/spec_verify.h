@@ -243,6 +243,59 @@ spec_status spec_verify_chain_noalloc(int B, int gamma, int V,
                                       void* stream);
 
 /*
+ * Lazy (row-on-demand) variants: spec_verify_chain_lazy,
+ * spec_verify_tree_greedy_lazy, spec_verify_tree_sample_lazy.
+ * [origins] "Speculative Decoding" (rules 1-3 look at position i only after
+ * positions 0..i-1 were accepted) and "SpecInfer" / "In SGLang" (the tree
+ * walk only ever reads the rows of the nodes it visits); [atlas] §0 (verify
+ * time is a cost the round pays whatever is accepted).
+ *
+ * Same arguments, workspace size (same `entry` as the dense function),
+ * outputs and error reporting as the function without the suffix; for valid
+ * inputs out_tokens, out_num_accepted and out_accept_index are bit-identical
+ * to it.  Instead of reading every row, they walk level by level on the
+ * device -- the rows the still-active sequences need, then one decision per
+ * active sequence -- and read about (accepted tokens + 1) rows (chain: row
+ * pairs) per sequence.  Costs and differences:
+ * - 2 kernel launches per level (gamma+1 levels for the chain, max_depth+1
+ *   for trees, launched whether or not a sequence is still active) plus the
+ *   final draw: worth it when rows are large and rejections come early.
+ * - Rows that are never read are not validated: a non-finite logit in a row
+ *   past the stopping point, or an invalid drafted token past the first
+ *   rejection, does not make the sequence invalid.  Tree structure and
+ *   temperature are always validated.
+ * - diag: only evaluated entries are written; the rest hold NaN (chain:
+ *   positions after the first rejection; tree sampling: children of nodes
+ *   the walk did not visit).  Evaluated entries equal the dense ones.
+ */
+spec_status spec_verify_chain_lazy(int B, int gamma, int V,
+                                   const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                   const void* draft, spec_dtype ddt, int draft_is_probs,
+                                   int64_t d_row_stride,
+                                   const int32_t* draft_tokens, const float* temperature,
+                                   const float* coins, const float* final_u,
+                                   int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_verify_tree_greedy_lazy(int B, int N, int V, int max_depth,
+                                         const void* target_logits, spec_dtype tdt,
+                                         int64_t t_row_stride,
+                                         const int32_t* tokens, const int32_t* parents,
+                                         int32_t* out_accept_index, int32_t* out_tokens,
+                                         int32_t* out_num_accepted,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_verify_tree_sample_lazy(int B, int N, int V, int max_depth,
+                                         const void* target_logits, spec_dtype tdt,
+                                         int64_t t_row_stride,
+                                         const int32_t* tokens, const int32_t* parents,
+                                         const float* temperature, const float* coins,
+                                         const float* final_u,
+                                         const float* draft_probs, int64_t dp_row_stride,
+                                         float threshold_single, float threshold_acc,
+                                         int32_t* out_accept_index, int32_t* out_tokens,
+                                         int32_t* out_num_accepted, float* diag,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_workspace_bytes -- workspace size for one entry point and shape.
  * rows = gamma for SPEC_ENTRY_CHAIN (sized for draft logits, which also
  * covers draft probabilities), N for the tree entry points.  Returns 0 for
@@ -265,7 +318,8 @@ spec_status spec_read_device_status(void* workspace, int* status_out, void* stre
  * later verify call on this host thread records `start_event` on its stream
  * just before launching its row-statistics kernel (the kernel that streams
  * every logit row, which dominates each call) and `stop_event` just after it,
- * so cudaEventElapsedTime gives that kernel's duration.  Both are
+ * so cudaEventElapsedTime gives that kernel's duration (for the lazy
+ * variants: the whole level walk and final draw).  Both are
  * cudaEvent_t handles owned by the caller; NULL, NULL switches the hook off.
  * Inside stream capture the records become external event nodes.
  */

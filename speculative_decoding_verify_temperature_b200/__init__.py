@@ -11,8 +11,11 @@ from .spec_verify import (  # noqa: F401
     spec_profile_events,
     spec_read_device_status,
     spec_verify_chain,
+    spec_verify_chain_lazy,
     spec_verify_tree_greedy,
+    spec_verify_tree_greedy_lazy,
     spec_verify_tree_sample,
+    spec_verify_tree_sample_lazy,
     spec_workspace_bytes,
     spec_workspace_init,
 )

@@ -57,6 +57,20 @@ template <> struct Tr<SPEC_BF16> { static constexpr int EPV = 8; static constexp
 template <> struct Tr<SPEC_F32> { static constexpr int EPV = 4; static constexpr int ESZ = 4; };
 template <int DT> __host__ __device__ constexpr int chunk_elems() { return NT * VPT * Tr<DT>::EPV; }
 
+// Per-sequence state of lazy (row-on-demand) verification.
+struct LazySeq {
+    int cur;       // chain: last position decided; trees: current node
+    int k;         // accepted draft tokens so far
+    int state;     // LZ_ACTIVE, LZ_DRAW (last token still to draw), LZ_DONE, LZ_INVALID
+    int nrej;      // trees: rejected children of cur
+    float s;       // log2(e) / T
+    float m, mq;   // combined statistics of the last decided row (chain: target, draft)
+    int pad;
+    double z, zq;
+};
+enum { LZ_ACTIVE = 0, LZ_DRAW = 1, LZ_DONE = 2, LZ_INVALID = 3 };
+constexpr int LZ_MAX_LEVELS = SPEC_MAX_DEPTH + 1;
+
 struct Params {
     int B, V, R, nch, gamma, N, max_depth;
     int rows_tgt;                  // target rows per sequence
@@ -84,6 +98,13 @@ struct Params {
     float2* stats2;                // [B][nch][NWARP]   (chain residual chunk sums)
     unsigned* cnt2;                // [B]               (chain residual arrivals)
     unsigned* status;
+    // lazy (row-on-demand) verification
+    struct LazySeq* lz_seq;        // [B]
+    int* lz_rej;                   // [B][rej_cap]      (trees: rejected children tokens)
+    int rej_cap;
+    int* lz_list;                  // [2][B]            (active sequences of a level, ping-pong)
+    unsigned* lz_count;            // [LZ_MAX_LEVELS + 1] (active count of each level; zero at rest)
+    int level;
 };
 
 // ----------------------------------------------------------------------------- small helpers
@@ -435,12 +456,12 @@ struct FinShared {
 // Combine the per-warp softmax statistics of rows [0, R) into (m, Z, bad).
 // `blk` is sequence b's statistics block ([R][nch][SPC]), in shared memory
 // when staged, else in global memory (written by the previous kernel).
-template <int BT>
-__device__ void combine_softmax_rows(const Params& P, const float2* blk, int R, FinShared& sh) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int E = P.nch * SPC;
-    for (int r = warp; r < R; r += BT / 32) {
-        const float2* st = blk + (size_t)r * E;
+// One row's statistics (E entries at st) combined by one warp: max m and sum
+// Z (fp64) in every lane; returns whether the row is unusable (NaN/+inf
+// logit, all -inf, Z not positive and finite).
+__device__ __forceinline__ bool warp_combine(const float2* st, int E, float& m_out, double& z_out) {
+    const int lane = threadIdx.x & 31;
+    {
         // one pass: each lane keeps an online (max, sum) over its entries
         float m = -INFINITY;
         double z = 0.0;
@@ -460,12 +481,29 @@ __device__ void combine_softmax_rows(const Params& P, const float2* blk, int R, 
         bad = __any_sync(FULL, bad);
         double zw = (m > -INFINITY && mw < INFINITY) ? z * (double)ex2(m - mw) : 0.0;
         zw = warp_sum_d(zw);
-        if (lane == 0) {
-            sh.m[r] = mw;
-            sh.z[r] = zw;
-            sh.bad[r] = bad || !(mw > -INFINITY) || !(mw < INFINITY) || !(zw > 0.0) || !(zw < 1e300);
-        }
+        m_out = mw;
+        z_out = zw;
+        return bad || !(mw > -INFINITY) || !(mw < INFINITY) || !(zw > 0.0) || !(zw < 1e300);
     }
+}
+
+// warp_combine of one row into sh slot `slot` (written by lane 0).
+__device__ __forceinline__ void combine_row(const float2* st, int E, FinShared& sh, int slot) {
+    float m;
+    double z;
+    const bool bad = warp_combine(st, E, m, z);
+    if ((threadIdx.x & 31) == 0) {
+        sh.m[slot] = m;
+        sh.z[slot] = z;
+        sh.bad[slot] = bad;
+    }
+}
+
+template <int BT>
+__device__ void combine_softmax_rows(const Params& P, const float2* blk, int R, FinShared& sh) {
+    const int warp = threadIdx.x >> 5;
+    const int E = P.nch * SPC;
+    for (int r = warp; r < R; r += BT / 32) combine_row(blk + (size_t)r * E, E, sh, r);
 }
 
 // p(x) of one element, fp64 exp2, in the units of the row statistics.
@@ -942,32 +980,94 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
     __syncthreads();
 }
 
+// Start of the lazy chain finalisation for sequence b: the decision comes from
+// the level walk.  A sequence still active after position gamma - 1 takes the
+// bonus draw from row gamma, whose statistics are combined here.  Leaves the
+// same shared state as chain_decide (sh.ivals[0] = valid, sh.ivals[1] = k,
+// sh.dvals[0] = s, the statistics of rows k and gamma + 1 + k); when `write`
+// is set also writes the accepted tokens, the -1 tail, num_accepted, NaN for
+// the diagnostics of positions never evaluated, and flags invalid sequences.
+// Ends with __syncthreads.
+__device__ void chain_lazy_state(const Params& P, int b, FinShared& sh, bool write) {
+    const int tid = threadIdx.x, gamma = P.gamma, W = gamma + 1;
+    if (tid < 32) {
+        const LazySeq L = P.lz_seq[b];
+        int ok = L.state == LZ_DRAW || (L.state == LZ_ACTIVE && L.k == gamma);
+        float m = L.m;
+        double z = L.z;
+        if (ok && L.state == LZ_ACTIVE) {
+            const int E = P.nch * SPC;
+            ok = !warp_combine(P.stats + ((size_t)b * P.R + gamma) * E, E, m, z);
+            if (!ok && tid == 0) flag_input_error(P);
+        }
+        if (tid == 0) {
+            const int k = ok ? L.k : 0;
+            sh.ivals[0] = ok;
+            sh.ivals[1] = k;
+            sh.dvals[0] = (double)L.s;
+            sh.m[k] = m;
+            sh.z[k] = z;
+            if (k < gamma) {
+                sh.m[gamma + 1 + k] = L.mq;
+                sh.z[gamma + 1 + k] = L.zq;
+            }
+            if (write) {
+                int32_t* toks = P.out_tokens + (size_t)b * W;
+                float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+                if (!ok) {
+                    for (int i = 0; i < W; ++i) toks[i] = -1;
+                    P.out_num_accepted[b] = -1;
+                    if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
+                } else {
+                    for (int i = 0; i < k; ++i) toks[i] = P.draft_tokens[(size_t)b * gamma + i];
+                    for (int i = k + 1; i < W; ++i) toks[i] = -1;
+                    P.out_num_accepted[b] = k;
+                    if (dg)
+                        for (int i = k + 1; i < gamma; ++i) { dg[i] = nanf_(); dg[gamma + i] = nanf_(); }
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// One row's argmax statistics (E entries at st) combined by one warp: the
+// maximum's lowest index in every lane; returns whether a NaN was seen.
+__device__ __forceinline__ bool warp_argmax(const float2* st, int E, int& idx_out) {
+    const int lane = threadIdx.x & 31;
+    float best = -INFINITY;
+    int idx = 0x7fffffff;
+    bool bad = false;
+    for (int e = lane; e < E; e += 32) {
+        const float2 x = st[e];
+        int xi = __float_as_int(x.y);
+        if (x.x != x.x) bad = true;
+        else if (x.x > best || (x.x == best && xi < idx)) { best = x.x; idx = xi; }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        float ov = __shfl_xor_sync(FULL, best, o);
+        int oi = __shfl_xor_sync(FULL, idx, o);
+        if (ov > best || (ov == best && oi < idx)) { best = ov; idx = oi; }
+    }
+    idx_out = idx;
+    return __any_sync(FULL, bad);
+}
+
+// warp_argmax of one row: index to sh.rej[slot], NaN flag to sh.bad[slot].
+__device__ __forceinline__ void argmax_row(const float2* st, int E, FinShared& sh, int slot) {
+    int idx;
+    const bool bad = warp_argmax(st, E, idx);
+    if ((threadIdx.x & 31) == 0) { sh.rej[slot] = idx; sh.bad[slot] = bad; }
+}
+
 template <int TDT, int BT>
 __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
     const int E = P.nch * SPC;
     // per-node argmax (lowest index among equal maxima)
-    for (int r = warp; r < N; r += BT / 32) {
-        const float2* st = blk + (size_t)r * E;
-        float best = -INFINITY;
-        int idx = 0x7fffffff;
-        bool bad = false;
-        for (int e = lane; e < E; e += 32) {
-            const float2 x = st[e];
-            int xi = __float_as_int(x.y);
-            if (x.x != x.x) bad = true;
-            else if (x.x > best || (x.x == best && xi < idx)) { best = x.x; idx = xi; }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            float ov = __shfl_xor_sync(FULL, best, o);
-            int oi = __shfl_xor_sync(FULL, idx, o);
-            if (ov > best || (ov == best && oi < idx)) { best = ov; idx = oi; }
-        }
-        bad = __any_sync(FULL, bad);
-        if (lane == 0) { sh.rej[r] = idx; sh.bad[r] = bad; }
-    }
+    for (int r = warp; r < N; r += BT / 32) argmax_row(blk + (size_t)r * E, E, sh, r);
     for (int n = tid; n < N; n += BT) {
         sh.par[n] = P.parents[(size_t)b * N + n];
         sh.tok[n] = P.tokens[(size_t)b * N + n];
@@ -1010,6 +1110,96 @@ __device__ void finalize_greedy(const Params& P, int b, FinShared& sh, const flo
             P.out_num_accepted[b] = k;
         }
     }
+}
+
+// Last token of a target-only tree walk ending at node `cur`: drawn with
+// final_u[b] from relu(p_cur - d_cur), d_cur = the draft_probs row of cur
+// (zeros when draft_probs is NULL) with the rejected children's tokens
+// rej[0..nrej) overwritten by their target probabilities.  (mc, zc) are the
+// statistics of row cur.  *S_out receives the mass of relu(p_cur - d_cur).
+template <int TDT, int BT>
+__device__ int tree_final_draw(const Params& P, int b, int cur, const int* rej, int nrej, float s, float mc,
+                               double zc, FinShared& sh, double* S_out) {
+    const int tid = threadIdx.x, N = P.N, V = P.V;
+    const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
+    const float u = P.final_u[b];
+    int y;
+    double S;
+    if (!P.draft_probs) {
+        const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
+        double Su;
+        y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, mc, u, rej, nrej, sh, &Su);
+        S = Su / zc;
+    } else {
+        // relu(p_cur - d_cur) over the whole row: chunk sums, then one rescan.
+        constexpr int CH = chunk_elems<TDT>();
+        const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * N + cur) * P.dpstride;
+        const float m = mc, iz = (float)(1.0 / zc);
+        for (int c = 0; c < P.nch; ++c) {
+            for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
+            __syncthreads();
+            for (int i = tid; i < nrej; i += BT) {
+                int o = rej[i] - c * CH;
+                if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+            }
+            __syncthreads();
+            WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, c * CH, V};
+            double tot;
+            block_excl_scan<BT>((double)chunk_weight_partial<CH, BT>(wf, c), &tot);
+            if (tid == 0) sh.M[c] = tot;
+            __syncthreads();
+        }
+        if (tid == 0) {
+            double tot = 0.0;
+            for (int c = 0; c < P.nch; ++c) tot += sh.M[c];
+            sh.dvals[0] = tot;
+        }
+        __syncthreads();
+        S = sh.dvals[0];
+        y = -1;
+        if (S > 0.0) {
+            const double t = (double)u * S;
+            for (int attempt = 0; attempt < P.nch && y < 0; ++attempt) {
+                if (tid == 0) {
+                    double C = 0.0, before = 0.0;
+                    int cs = -1;
+                    for (int c = 0; c < P.nch; ++c) {
+                        if (sh.M[c] <= 0.0) continue;
+                        if (t < C + sh.M[c]) { cs = c; before = C; break; }
+                        C += sh.M[c];
+                    }
+                    if (cs < 0)
+                        for (int c = P.nch - 1; c >= 0; --c)
+                            if (sh.M[c] > 0.0) { cs = c; before = C - sh.M[c]; break; }
+                    sh.ivals[4] = cs;
+                    sh.dvals[1] = before;
+                }
+                __syncthreads();
+                const int cs = sh.ivals[4];
+                if (cs < 0) break;
+                for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
+                __syncthreads();
+                for (int i = tid; i < nrej; i += BT) {
+                    int o = rej[i] - cs * CH;
+                    if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+                }
+                __syncthreads();
+                WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, cs * CH, V};
+                double tot;
+                y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+                if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+                __syncthreads();
+            }
+        }
+        if (y < 0) {
+            // empty residual (rounding only): draw from p_cur itself
+            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
+            double Su;
+            y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
+        }
+    }
+    *S_out = S;
+    return y;
 }
 
 template <int TDT, int BT>
@@ -1087,83 +1277,8 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     }
     __syncthreads();
     const int cur = sh.ivals[1], k = sh.ivals[2], nrej = sh.ivals[3];
-    const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
-    const float u = P.final_u[b];
-    int y;
     double S;
-    if (!P.draft_probs) {
-        const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
-        double Su;
-        y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, sh.m[cur], u, sh.rej, nrej, sh, &Su);
-        S = Su / sh.z[cur];
-    } else {
-        // relu(p_cur - d_cur) over the whole row: chunk sums, then one rescan.
-        constexpr int CH = chunk_elems<TDT>();
-        const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * N + cur) * P.dpstride;
-        const float m = sh.m[cur], iz = (float)(1.0 / sh.z[cur]);
-        for (int c = 0; c < P.nch; ++c) {
-            for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
-            __syncthreads();
-            for (int i = tid; i < nrej; i += BT) {
-                int o = sh.rej[i] - c * CH;
-                if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
-            }
-            __syncthreads();
-            WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, c * CH, V};
-            double tot;
-            block_excl_scan<BT>((double)chunk_weight_partial<CH, BT>(wf, c), &tot);
-            if (tid == 0) sh.M[c] = tot;
-            __syncthreads();
-        }
-        if (tid == 0) {
-            double tot = 0.0;
-            for (int c = 0; c < P.nch; ++c) tot += sh.M[c];
-            sh.dvals[0] = tot;
-        }
-        __syncthreads();
-        S = sh.dvals[0];
-        y = -1;
-        if (S > 0.0) {
-            const double t = (double)u * S;
-            for (int attempt = 0; attempt < P.nch && y < 0; ++attempt) {
-                if (tid == 0) {
-                    double C = 0.0, before = 0.0;
-                    int cs = -1;
-                    for (int c = 0; c < P.nch; ++c) {
-                        if (sh.M[c] <= 0.0) continue;
-                        if (t < C + sh.M[c]) { cs = c; before = C; break; }
-                        C += sh.M[c];
-                    }
-                    if (cs < 0)
-                        for (int c = P.nch - 1; c >= 0; --c)
-                            if (sh.M[c] > 0.0) { cs = c; before = C - sh.M[c]; break; }
-                    sh.ivals[4] = cs;
-                    sh.dvals[1] = before;
-                }
-                __syncthreads();
-                const int cs = sh.ivals[4];
-                if (cs < 0) break;
-                for (int w = tid; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
-                __syncthreads();
-                for (int i = tid; i < nrej; i += BT) {
-                    int o = sh.rej[i] - cs * CH;
-                    if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
-                }
-                __syncthreads();
-                WTreeRes<TDT> wf{row, drow, s, m, iz, sh.bitmap, cs * CH, V};
-                double tot;
-                y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
-                if (y < 0 && tid == 0) sh.M[cs] = 0.0;
-                __syncthreads();
-            }
-        }
-        if (y < 0) {
-            // empty residual (rounding only): draw from p_cur itself
-            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
-            double Su;
-            y = sample_target_row<TDT, BT>(row, V, P.nch, st, s, m, u, nullptr, 0, sh, &Su);
-        }
-    }
+    const int y = tree_final_draw<TDT, BT>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur], sh, &S);
     if (tid == 0) {
         ot[k] = y;
         for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
@@ -1264,7 +1379,7 @@ __device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u,
 //  - k < gamma: every slice sums max(0, p_k - q_k) over its chunks of row k;
 //    with one slice the CTA draws directly, otherwise the last CTA of the
 //    sequence to arrive locates the chunk holding u*S and rescans it (rule 2).
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool LZ>
 __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     __shared__ FinShared sh;
     __shared__ int is_last;
@@ -1276,12 +1391,17 @@ __global__ void __launch_bounds__(NT) k_chain_final(const Params P) {
     const int b = blockIdx.x / nsl, sl = blockIdx.x - b * nsl;
     const int c0 = (int)((long long)nch * sl / nsl), c1 = (int)((long long)nch * (sl + 1) / nsl);
     const int gamma = P.gamma, V = P.V;
-    const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
-    pdl_wait();
-    const float2* blk = stage_stats(P, b, P.R, dyn, P.stage_cap, &sbar);
-    combine_softmax_rows<NT>(P, blk, P.R, sh);
-    __syncthreads();
-    chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0, pf);
+    if constexpr (LZ) {
+        pdl_wait();
+        chain_lazy_state(P, b, sh, sl == 0);
+    } else {
+        const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
+        pdl_wait();
+        const float2* blk = stage_stats(P, b, P.R, dyn, P.stage_cap, &sbar);
+        combine_softmax_rows<NT>(P, blk, P.R, sh);
+        __syncthreads();
+        chain_decide<TDT, DDT, DK>(P, b, sh, sl == 0, pf);
+    }
     const int ok = sh.ivals[0], k = sh.ivals[1];
     const float s = (float)sh.dvals[0];
     if (!ok) return;
@@ -1430,7 +1550,7 @@ __host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
 // element into 8-element group sums, the group sums are scanned block-wide in
 // fp64 in index order, and only the group holding u*S is recomputed to pick
 // the token.  The bonus token (k = gamma) is drawn as in the sliced kernel.
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool LZ>
 __global__ void __launch_bounds__(SEQ_BT) k_chain_final_row(const Params P) {
     __shared__ FinShared sh;
     __shared__ __align__(8) uint64_t bar, sbar;
@@ -1439,13 +1559,19 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_row(const Params P) {
     constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
     const int tid = threadIdx.x, b = blockIdx.x;
     const int gamma = P.gamma, V = P.V;
-    const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
-    pdl_wait();
-    const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
-    if (tid == 0) mbar_init(smem_u32(&bar), 1);
-    combine_softmax_rows<SEQ_BT>(P, blk, P.R, sh);
-    __syncthreads();
-    chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
+    if constexpr (LZ) {
+        pdl_wait();
+        if (tid == 0) mbar_init(smem_u32(&bar), 1);
+        chain_lazy_state(P, b, sh, true);
+    } else {
+        const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
+        pdl_wait();
+        const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
+        if (tid == 0) mbar_init(smem_u32(&bar), 1);
+        combine_softmax_rows<SEQ_BT>(P, blk, P.R, sh);
+        __syncthreads();
+        chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
+    }
     const int ok = sh.ivals[0], k = sh.ivals[1];
     const float s = (float)sh.dvals[0];
     if (!ok) return;
@@ -1564,6 +1690,328 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     else finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
 }
 
+// ============================================================================= lazy (row-on-demand) verification
+//
+// The verify rules need only some rows: the chain reads the target row (and
+// draft row) of position i only if positions 0..i-1 were all accepted, and a
+// tree walk reads the row of each node it visits.  The lazy entry points walk
+// level by level -- statistics of the rows the active sequences need, then
+// one decision per active sequence -- so a round reads about (accepted + 1)
+// rows per sequence instead of all of them.  Each level is two programmatic
+// dependent launches; the list of sequences still active at a level lives in
+// the workspace, so the host never synchronises.  The row statistics have the
+// dense path's layout and arithmetic, so every decision and draw is bit-for-
+// bit the dense one; rows that are never read are not validated either.
+
+// Sequence j of the current level's active list (level 0: every sequence).
+__device__ __forceinline__ int lz_count_of(const Params& P) {
+    return P.level == 0 ? P.B : (int)__ldcg(P.lz_count + P.level);
+}
+__device__ __forceinline__ int lz_seq_of(const Params& P, int j) {
+    return P.level == 0 ? j : __ldcg(P.lz_list + (P.level & 1) * P.B + j);
+}
+// Append sequence b to the next level's active list.
+__device__ __forceinline__ void lz_push(const Params& P, int b) {
+    const unsigned j = atomicAdd(P.lz_count + P.level + 1, 1u);
+    P.lz_list[((P.level + 1) & 1) * P.B + j] = b;
+}
+
+// Row statistics of the rows the active sequences need at this level: chain
+// position `level` (target row, and the draft row when the draft is given as
+// logits and level < gamma), or the current node of a tree walk.  Work items
+// are (active sequence, row, chunk), split into contiguous ranges as in
+// k_stats; the statistics land where the dense path puts them.  Level 0 also
+// clears the per-level active counts.
+template <int MODE, int TDT, int DDT>
+__global__ void __launch_bounds__(NT, STATS_CTAS_PER_SM) k_lz_stats(const Params P) {
+    constexpr int CH = chunk_elems<TDT>();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    pdl_trigger();
+    pdl_wait();
+    const int level = P.level;
+    if (level == 0 && blockIdx.x == 0 && threadIdx.x <= LZ_MAX_LEVELS) P.lz_count[threadIdx.x] = 0u;
+    const int nact = lz_count_of(P);
+    const int rpl = (MODE == MODE_CHAIN && P.R > P.rows_tgt && level < P.gamma) ? 2 : 1;
+    const int per_seq = rpl * P.nch;
+    const long long total = (long long)nact * per_seq;
+    const long long lo = total * blockIdx.x / gridDim.x;
+    const long long n = total * (blockIdx.x + 1) / gridDim.x - lo;
+    if (n <= 0) return;
+    int j = (int)(lo / per_seq);
+    int r, c;
+    {
+        const int rem = (int)(lo - (long long)j * per_seq);
+        r = rem / P.nch;
+        c = rem - r * P.nch;
+    }
+    int jb = -1, b = 0, node = 0;
+    float s = 0.f;
+    for (long long i = 0; i < n; ++i) {
+        if (j != jb) {
+            jb = j;
+            b = lz_seq_of(P, j);
+            if constexpr (MODE != MODE_GREEDY) s = scale_of(__ldg(P.temperature + b));
+            if constexpr (MODE != MODE_CHAIN) node = level == 0 ? 0 : __ldcg(&P.lz_seq[b].cur);
+        }
+        float2 stat;
+        int srow;
+        if constexpr (MODE == MODE_GREEDY) {
+            srow = node;
+            stat = chunk_argmax<TDT>(P.tgt + ((size_t)b * P.R + node) * P.tstride, P.V, c);
+        } else if constexpr (MODE == MODE_SAMPLE) {
+            srow = node;
+            stat = chunk_softmax<TDT, CH>(P.tgt + ((size_t)b * P.R + node) * P.tstride, P.V, c, s);
+        } else {
+            if (r == 0) {
+                srow = level;
+                stat = chunk_softmax<TDT, CH>(P.tgt + ((size_t)b * P.rows_tgt + level) * P.tstride, P.V, c, s);
+            } else {
+                srow = P.rows_tgt + level;
+                stat = chunk_softmax<DDT, CH>(P.drf + ((size_t)b * P.gamma + level) * P.dstride, P.V, c, s);
+            }
+        }
+        if (lane == 0) P.stats[(((size_t)b * P.R + srow) * P.nch + c) * SPC + warp] = stat;
+        if (++c == P.nch) {
+            c = 0;
+            if (++r == rpl) { r = 0; ++j; }
+        }
+    }
+}
+
+// Chain decision at position `level` < gamma, one warp per active sequence:
+// combine the row statistics, gather p(x) and q(x) at the drafted token, test
+// coin <= p/q.  Accepted sequences move to the next level; a rejection leaves
+// the sequence for the final kernel (residual at this position).  The
+// temperature is checked at level 0; a bad row or token marks the sequence
+// invalid.  Writes the p/q diagnostics of this position.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(NT) k_lz_decide_chain(const Params P) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * NWARP + (threadIdx.x >> 5);
+    if (j >= lz_count_of(P)) return;
+    const int b = lz_seq_of(P, j);
+    const int level = P.level, gamma = P.gamma, E = P.nch * SPC;
+    bool ok = true;
+    float s;
+    if (level == 0) {
+        const float T = P.temperature[b];
+        ok = temperature_ok(T);
+        s = ok ? scale_of(T) : 0.f;
+    } else {
+        s = __ldcg(&P.lz_seq[b].s);
+    }
+    float m, mq = 0.f;
+    double z, zq = 0.0;
+    ok &= !warp_combine(P.stats + ((size_t)b * P.R + level) * E, E, m, z);
+    if constexpr (DK != DK_PROBS) ok &= !warp_combine(P.stats + ((size_t)b * P.R + gamma + 1 + level) * E, E, mq, zq);
+    if (lane != 0) return;
+    const int x = P.draft_tokens[(size_t)b * gamma + level];
+    ok &= (x >= 0 && x < P.V);
+    double p = 0.0, q = 0.0;
+    if (ok) {
+        p = prob_d(ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, x), s, m, z);
+        const char* drow = P.drf + ((size_t)b * gamma + level) * P.dstride;
+        if constexpr (DK == DK_PROBS) {
+            q = (double)__ldg(reinterpret_cast<const float*>(drow) + x);
+            ok &= (q >= 0.0 && q <= 3.0e38);
+        } else {
+            q = prob_d(ld_elem<DDT>(drow, x), s, mq, zq);
+        }
+    }
+    LazySeq L;
+    L.cur = level; L.nrej = 0; L.pad = 0;
+    L.s = s; L.m = m; L.mq = mq; L.z = z; L.zq = zq;
+    if (!ok) {
+        L.state = LZ_INVALID;
+        L.k = -1;
+        flag_input_error(P);
+    } else {
+        if (P.diag) {
+            float* dg = P.diag + (size_t)b * (2 * gamma + 1);
+            dg[level] = (float)p;
+            dg[gamma + level] = (float)q;
+        }
+        const double ratio = (q > 0.0) ? p / q : INFINITY;
+        if ((double)P.coins[(size_t)b * gamma + level] <= ratio) {
+            L.state = LZ_ACTIVE;
+            L.k = level + 1;
+            lz_push(P, b);
+        } else {
+            L.state = LZ_DRAW;
+            L.k = level;
+        }
+    }
+    P.lz_seq[b] = L;
+}
+
+// Is sequence b's tree well formed (parents[0] = -1, 0 <= parents[n] < n,
+// tokens in [0, V), depth <= max_depth)?  One warp.
+__device__ bool warp_tree_valid(const Params& P, int b) {
+    const int lane = threadIdx.x & 31, N = P.N;
+    const int32_t* par = P.parents + (size_t)b * N;
+    const int32_t* tok = P.tokens + (size_t)b * N;
+    bool good = true;
+    for (int n = lane; n < N; n += 32) {
+        const int pa = par[n];
+        good &= (n == 0) ? (pa == -1) : (pa >= 0 && pa < n && tok[n] >= 0 && tok[n] < P.V);
+    }
+    good = __all_sync(FULL, good);
+    if (good) {
+        for (int n = lane; n < N; n += 32) {
+            int d = 0, a = n;
+            while (a > 0 && d <= P.max_depth) { a = par[a]; ++d; }
+            good &= d <= P.max_depth;
+        }
+        good = __all_sync(FULL, good);
+    }
+    return good;
+}
+
+// Tree walk at depth `level`, one warp per active sequence at node cur.
+// Greedy: the first child of cur whose token is the argmax of row cur is
+// accepted, else the walk ends with that argmax as the bonus token (written
+// here: greedy needs no final kernel).  Sampling: the children of cur are
+// tried in node order with the coin of cur against prob_acc / threshold_acc
+// or p >= threshold_single; rejected children's tokens are kept for the final
+// draw.  Level 0 validates the tree (and the temperature).  Diagnostics hold
+// p_cur(token) for the children of visited nodes, NaN for the other nodes.
+template <int MODE, int TDT>
+__global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int j = blockIdx.x * NWARP + (threadIdx.x >> 5);
+    if (j >= lz_count_of(P)) return;
+    const int b = lz_seq_of(P, j);
+    const int level = P.level, N = P.N, W = P.max_depth + 1, E = P.nch * SPC;
+    int32_t* ai = P.out_accept_index + (size_t)b * W;
+    int32_t* ot = P.out_tokens + (size_t)b * W;
+    float* dg = (MODE == MODE_SAMPLE && P.diag) ? P.diag + (size_t)b * (N + 1) : nullptr;
+    const int32_t* par = P.parents + (size_t)b * N;
+    const int32_t* tok = P.tokens + (size_t)b * N;
+    LazySeq L;
+    bool ok = true;
+    if (level == 0) {
+        ok = warp_tree_valid(P, b);
+        L.cur = 0; L.k = 0; L.s = 0.f;
+        if constexpr (MODE == MODE_SAMPLE) {
+            const float T = P.temperature[b];
+            ok &= temperature_ok(T);
+            L.s = ok ? scale_of(T) : 0.f;
+        }
+        if (ok) {
+            if (lane == 0) ai[0] = 0;
+            if (dg) for (int n = lane; n < N; n += 32) dg[n] = n == 0 ? 0.f : nanf_();
+            __syncwarp();
+        }
+    } else {
+        L = P.lz_seq[b];
+    }
+    const int cur = L.cur, k = L.k;
+    const float2* st = P.stats + ((size_t)b * P.R + cur) * E;
+    int next = -1, nrej = 0;
+    int g = 0;
+    float m = 0.f;
+    double z = 0.0;
+    if (ok) {
+        if constexpr (MODE == MODE_GREEDY) {
+            ok = !warp_argmax(st, E, g);
+            if (ok)
+                for (int base = cur + 1; base < N && next < 0; base += 32) {
+                    const int c = base + lane;
+                    const unsigned hit = __ballot_sync(FULL, c < N && par[c] == cur && tok[c] == g);
+                    if (hit) next = base + __ffs(hit) - 1;
+                }
+        } else {
+            ok = !warp_combine(st, E, m, z);
+            if (ok) {
+                const char* trow = P.tgt + ((size_t)b * N + cur) * P.tstride;
+                const double coin = (double)P.coins[(size_t)b * N + cur];
+                const double ths = (double)P.th_single, tha = (double)P.th_acc;
+                int* rej = P.lz_rej + (size_t)b * P.rej_cap;
+                double acc = 0.0;
+                for (int base = cur + 1; base < N; base += 32) {
+                    const int c = base + lane;
+                    const bool child = c < N && par[c] == cur;
+                    double pc = 0.0;
+                    int t = 0;
+                    if (child) {
+                        t = tok[c];
+                        pc = prob_d(ld_elem<TDT>(trow, t), L.s, m, z);
+                        if (dg) dg[c] = (float)pc;
+                    }
+                    unsigned msk = __ballot_sync(FULL, child);
+                    while (msk && next < 0) {
+                        const int l = __ffs(msk) - 1;
+                        msk &= msk - 1;
+                        const double p = __shfl_sync(FULL, pc, l);
+                        const int tl = __shfl_sync(FULL, t, l);
+                        acc += p;
+                        if (coin <= acc / tha || p >= ths) next = base + l;
+                        else {
+                            if (lane == 0) rej[nrej] = tl;
+                            ++nrej;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (lane != 0) return;
+    if (!ok) {
+        for (int i = 0; i < W; ++i) { ai[i] = -1; ot[i] = -1; }
+        P.out_num_accepted[b] = -1;
+        if (dg) for (int i = 0; i <= N; ++i) dg[i] = nanf_();
+        flag_input_error(P);
+        L.state = LZ_INVALID;
+    } else if (next >= 0) {
+        ot[k] = tok[next];
+        ai[k + 1] = next;
+        L.cur = next;
+        L.k = k + 1;
+        L.state = LZ_ACTIVE;
+        lz_push(P, b);
+    } else if constexpr (MODE == MODE_GREEDY) {
+        ot[k] = g;
+        for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+        P.out_num_accepted[b] = k;
+        L.state = LZ_DONE;
+    } else {
+        L.state = LZ_DRAW;
+        L.nrej = nrej;
+        L.m = m;
+        L.z = z;
+    }
+    P.lz_seq[b] = L;
+}
+
+// Last token of a lazy target-only tree walk, one CTA per sequence (those
+// left in LZ_DRAW): tree_final_draw at the node where the walk stopped, with
+// the rejected children's tokens it kept.
+template <int TDT>
+__global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
+    __shared__ FinShared sh;
+    pdl_wait();
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const LazySeq L = P.lz_seq[b];
+    if (L.state != LZ_DRAW) return;
+    const int W = P.max_depth + 1;
+    for (int i = tid; i < L.nrej; i += SEQ_BT) sh.rej[i] = P.lz_rej[(size_t)b * P.rej_cap + i];
+    __syncthreads();
+    double S;
+    const int y = tree_final_draw<TDT, SEQ_BT>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, sh, &S);
+    if (tid == 0) {
+        int32_t* ai = P.out_accept_index + (size_t)b * W;
+        int32_t* ot = P.out_tokens + (size_t)b * W;
+        ot[L.k] = y;
+        for (int i = L.k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+        P.out_num_accepted[b] = L.k;
+        if (P.diag) P.diag[(size_t)b * (P.N + 1) + P.N] = (float)S;
+    }
+}
+
 }  // namespace sv
 
 // ============================================================================= host side
@@ -1594,7 +2042,8 @@ spec_status fail(spec_status st, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, cnt2, stats, stats2, total;
+    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, total;
+    int rej_cap;
     int R, nch_max;
 };
 
@@ -1611,6 +2060,12 @@ Layout make_layout(int entry, int B, int rows, int V) {
     L.stats = off; off = align256(off + sizeof(float2) * (size_t)B * L.R * nch * SPC);
     L.stats2 = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(float2) * (size_t)B * nch * NWARP);
+    // lazy (row-on-demand) verification state
+    L.lz_seq = off; off = align256(off + sizeof(LazySeq) * (size_t)B);
+    L.rej_cap = (entry == SPEC_ENTRY_CHAIN) ? 1 : rows;
+    L.lz_rej = off; off = align256(off + sizeof(int) * (size_t)B * L.rej_cap);
+    L.lz_list = off; off = align256(off + sizeof(int) * 2 * (size_t)B);
+    L.lz_count = off; off = align256(off + sizeof(unsigned) * (LZ_MAX_LEVELS + 1));
     L.total = off;
     return L;
 }
@@ -1662,6 +2117,11 @@ void bind_ws(Params& P, void* ws, const Layout& L) {
     P.cnt2 = reinterpret_cast<unsigned*>(w + L.cnt2);
     P.stats = reinterpret_cast<float2*>(w + L.stats);
     P.stats2 = reinterpret_cast<float2*>(w + L.stats2);
+    P.lz_seq = reinterpret_cast<LazySeq*>(w + L.lz_seq);
+    P.lz_rej = reinterpret_cast<int*>(w + L.lz_rej);
+    P.rej_cap = L.rej_cap;
+    P.lz_list = reinterpret_cast<int*>(w + L.lz_list);
+    P.lz_count = reinterpret_cast<unsigned*>(w + L.lz_count);
 }
 
 spec_status launched(const char* what) {
@@ -1670,23 +2130,27 @@ spec_status launched(const char* what) {
     return SPEC_OK;
 }
 
-template <int MODE, int TDT, int DDT>
-spec_status launch_stats(const Params& P, cudaStream_t st) {
-    auto kern = k_stats<MODE, TDT, DDT>;
-    static const int occ = blocks_per_sm(kern);
-    const long long items = (long long)P.B * P.R * P.nch;
-    // Up to 4 CTAs per resident slot when every CTA would own many chunks (the
-    // extra CTAs start as others retire, which keeps the CTAs out of
-    // lockstep); then as few CTAs as give every CTA the same number of chunks
-    // (within one), so that no CTA trails the rest by a whole chunk.
+// Grid of a statistics kernel over `items` chunks with `occ` resident CTAs
+// per SM.  Up to 4 CTAs per resident slot when every CTA would own many
+// chunks (the extra CTAs start as others retire, which keeps the CTAs out of
+// lockstep); then as few CTAs as give every CTA the same number of chunks
+// (within one), so that no CTA trails the rest by a whole chunk.
+unsigned stats_grid(long long items, int occ) {
     const long long resident = (long long)num_sms() * occ;
     long long mult = items / (8 * resident);
     mult = mult < 1 ? 1 : (mult > 4 ? 4 : mult);
     const long long slots = resident * mult;
     const long long per_cta = (items + slots - 1) / slots;
-    const long long grid = (items + per_cta - 1) / per_cta;
+    return (unsigned)((items + per_cta - 1) / per_cta);
+}
+
+template <int MODE, int TDT, int DDT>
+spec_status launch_stats(const Params& P, cudaStream_t st) {
+    auto kern = k_stats<MODE, TDT, DDT>;
+    static const int occ = blocks_per_sm(kern);
+    const unsigned grid = stats_grid((long long)P.B * P.R * P.nch, occ);
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
-    kern<<<(unsigned)grid, NT, 0, st>>>(P);
+    kern<<<grid, NT, 0, st>>>(P);
     spec_status s = launched("k_stats");
     if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
         return fail(SPEC_ERR_CUDA, "profile event");
@@ -1731,9 +2195,9 @@ inline int stats_stage_bytes(const Params& P, int rows, size_t limit) {
 
 // Dynamic shared memory available to the row-staged chain finalisation (0 if
 // it cannot be configured).
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool LZ>
 size_t row_stage_capacity() {
-    auto kern = k_chain_final_row<TDT, DDT, DK>;
+    auto kern = k_chain_final_row<TDT, DDT, DK, LZ>;
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 0;
     int dev = 0, optin = 0;
@@ -1746,28 +2210,35 @@ size_t row_stage_capacity() {
     return (size_t)cap;
 }
 
+// Chain finalisation after the statistics (dense, LZ = false) or after the
+// lazy level walk (LZ = true, which stages no statistics).
+template <int TDT, int DDT, int DK, bool LZ>
+spec_status launch_chain_final(Params P, cudaStream_t st) {
+    // Row-staged finalisation when the rejected row pair (and the statistics)
+    // fit in shared memory and one CTA per sequence fits in a single wave.
+    static const size_t cap = row_stage_capacity<TDT, DDT, DK, LZ>();
+    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
+    if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
+        P.stage_off = (int)pair;
+        P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, cap - pair);
+        return launch_dependent(k_chain_final_row<TDT, DDT, DK, LZ>, (unsigned)P.B, SEQ_BT, pair + P.stage_cap, P,
+                                st, "k_chain_final_row");
+    }
+    static const bool big = allow_stage(k_chain_final<TDT, DDT, DK, LZ>);
+    P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
+    // enough CTAs to cover the SMs twice, at most one per chunk
+    int nsl = (2 * num_sms() + P.B - 1) / P.B;
+    P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
+    return launch_dependent(k_chain_final<TDT, DDT, DK, LZ>, (unsigned)(P.B * P.nsl), NT, P.stage_cap, P, st,
+                            "k_chain_final");
+}
+
 template <int TDT, int DDT, int DK>
 spec_status launch_chain(Params P, cudaStream_t st) {
     // draft probabilities are read only by the finalize kernel
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
-    // Row-staged finalisation when the rejected row pair (and the statistics)
-    // fit in shared memory and one CTA per sequence fits in a single wave.
-    static const size_t cap = row_stage_capacity<TDT, DDT, DK>();
-    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
-    if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
-        P.stage_off = (int)pair;
-        P.stage_cap = stats_stage_bytes(P, P.R, cap - pair);
-        return launch_dependent(k_chain_final_row<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, pair + P.stage_cap, P,
-                                st, "k_chain_final_row");
-    }
-    static const bool big = allow_stage(k_chain_final<TDT, DDT, DK>);
-    P.stage_cap = stats_stage_bytes(P, P.R, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
-    // enough CTAs to cover the SMs twice, at most one per chunk
-    int nsl = (2 * num_sms() + P.B - 1) / P.B;
-    P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
-    return launch_dependent(k_chain_final<TDT, DDT, DK>, (unsigned)(P.B * P.nsl), NT, P.stage_cap, P, st,
-                            "k_chain_final");
+    return launch_chain_final<TDT, DDT, DK, false>(P, st);
 }
 
 template <int MODE, int TDT>
@@ -1777,6 +2248,62 @@ spec_status launch_tree(Params P, cudaStream_t st) {
     static const bool big = allow_stage(k_tree_final<MODE, TDT>);
     P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st, "k_tree_final");
+}
+
+// One level of the lazy walk: the statistics kernel (the first one as an
+// ordinary launch, so the walk starts after all earlier work on the stream),
+// then the decision kernel (none after the chain's bonus row).
+template <class KS, class KD>
+spec_status launch_level(KS ks, unsigned sgrid, KD kd, unsigned dgrid, Params& P, int level, cudaStream_t st) {
+    P.level = level;
+    spec_status s;
+    if (level == 0) {
+        ks<<<sgrid, NT, 0, st>>>(P);
+        s = launched("k_lz_stats");
+    } else {
+        s = launch_dependent(ks, sgrid, NT, 0, P, st, "k_lz_stats");
+    }
+    if (s != SPEC_OK || kd == nullptr) return s;
+    return launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
+}
+
+template <int TDT, int DDT, int DK>
+spec_status launch_chain_lazy(Params P, cudaStream_t st) {
+    auto ks = k_lz_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>;
+    auto kd = k_lz_decide_chain<TDT, DDT, DK>;
+    static const int occ = blocks_per_sm(ks);
+    const int rpl = P.R > P.rows_tgt ? 2 : 1;
+    const unsigned sgrid = stats_grid((long long)P.B * rpl * P.nch, occ);
+    const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    for (int level = 0; level <= P.gamma; ++level) {
+        spec_status s = launch_level(ks, sgrid, level < P.gamma ? kd : nullptr, dgrid, P, level, st);
+        if (s != SPEC_OK) return s;
+    }
+    spec_status s = launch_chain_final<TDT, DDT, DK, true>(P, st);
+    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
+        return fail(SPEC_ERR_CUDA, "profile event");
+    return s;
+}
+
+template <int MODE, int TDT>
+spec_status launch_tree_lazy(Params P, cudaStream_t st) {
+    auto ks = k_lz_stats<MODE, TDT, TDT>;
+    auto kd = k_lz_decide_tree<MODE, TDT>;
+    static const int occ = blocks_per_sm(ks);
+    const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
+    const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    for (int level = 0; level <= P.max_depth; ++level) {
+        spec_status s = launch_level(ks, sgrid, kd, dgrid, P, level, st);
+        if (s != SPEC_OK) return s;
+    }
+    spec_status s = SPEC_OK;
+    if constexpr (MODE == MODE_SAMPLE)
+        s = launch_dependent(k_lz_tree_final<TDT>, (unsigned)P.B, SEQ_BT, 0, P, st, "k_lz_tree_final");
+    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
+        return fail(SPEC_ERR_CUDA, "profile event");
+    return s;
 }
 
 }  // namespace
@@ -1835,14 +2362,16 @@ spec_status spec_profile_events(void* start_event, void* stop_event) {
     return SPEC_OK;
 }
 
-spec_status spec_verify_chain(int B, int gamma, int V,
-                              const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
-                              const void* draft, spec_dtype ddt, int draft_is_probs,
-                              int64_t d_row_stride,
-                              const int32_t* draft_tokens, const float* temperature,
-                              const float* coins, const float* final_u,
-                              int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+static spec_status chain_entry(bool lazy, int B, int gamma, int V,
+                               const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                               const void* draft, spec_dtype ddt, int draft_is_probs,
+                               int64_t d_row_stride,
+                               const int32_t* draft_tokens, const float* temperature,
+                               const float* coins, const float* final_u,
+                               int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                               void* workspace, size_t workspace_bytes, void* stream) {
     g_detail[0] = 0;
     if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
     if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
@@ -1874,14 +2403,16 @@ spec_status spec_verify_chain(int B, int gamma, int V,
     // The statistics of a row are laid out with the chain's full row count so
     // that draft rows keep their offsets for either draft kind.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+#define SPEC_CHAIN(T, D, K) return lazy ? launch_chain_lazy<T, D, K>(P, st) : launch_chain<T, D, K>(P, st)
     if (draft_is_probs) {
-        if (tdt == SPEC_BF16) return launch_chain<SPEC_BF16, SPEC_F32, DK_PROBS>(P, st);
-        return launch_chain<SPEC_F32, SPEC_F32, DK_PROBS>(P, st);
+        if (tdt == SPEC_BF16) SPEC_CHAIN(SPEC_BF16, SPEC_F32, DK_PROBS);
+        SPEC_CHAIN(SPEC_F32, SPEC_F32, DK_PROBS);
     }
-    if (tdt == SPEC_BF16 && ddt == SPEC_BF16) return launch_chain<SPEC_BF16, SPEC_BF16, DK_LOGITS>(P, st);
-    if (tdt == SPEC_BF16 && ddt == SPEC_F32) return launch_chain<SPEC_BF16, SPEC_F32, DK_LOGITS>(P, st);
-    if (tdt == SPEC_F32 && ddt == SPEC_BF16) return launch_chain<SPEC_F32, SPEC_BF16, DK_LOGITS>(P, st);
-    return launch_chain<SPEC_F32, SPEC_F32, DK_LOGITS>(P, st);
+    if (tdt == SPEC_BF16 && ddt == SPEC_BF16) SPEC_CHAIN(SPEC_BF16, SPEC_BF16, DK_LOGITS);
+    if (tdt == SPEC_BF16 && ddt == SPEC_F32) SPEC_CHAIN(SPEC_BF16, SPEC_F32, DK_LOGITS);
+    if (tdt == SPEC_F32 && ddt == SPEC_BF16) SPEC_CHAIN(SPEC_F32, SPEC_BF16, DK_LOGITS);
+    SPEC_CHAIN(SPEC_F32, SPEC_F32, DK_LOGITS);
+#undef SPEC_CHAIN
 }
 
 static spec_status tree_common(Params& P, int B, int N, int V, int max_depth,
@@ -1909,12 +2440,12 @@ static spec_status tree_common(Params& P, int B, int N, int V, int max_depth,
     return SPEC_OK;
 }
 
-spec_status spec_verify_tree_greedy(int B, int N, int V, int max_depth,
-                                    const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
-                                    const int32_t* tokens, const int32_t* parents,
-                                    int32_t* out_accept_index, int32_t* out_tokens,
-                                    int32_t* out_num_accepted,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
+static spec_status greedy_entry(bool lazy, int B, int N, int V, int max_depth,
+                                const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                const int32_t* tokens, const int32_t* parents,
+                                int32_t* out_accept_index, int32_t* out_tokens,
+                                int32_t* out_num_accepted,
+                                void* workspace, size_t workspace_bytes, void* stream) {
     g_detail[0] = 0;
     Params P{};
     spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
@@ -1925,19 +2456,23 @@ spec_status spec_verify_tree_greedy(int B, int N, int V, int max_depth,
     if (s != SPEC_OK) return s;
     bind_ws(P, workspace, L);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (lazy) {
+        if (tdt == SPEC_BF16) return launch_tree_lazy<MODE_GREEDY, SPEC_BF16>(P, st);
+        return launch_tree_lazy<MODE_GREEDY, SPEC_F32>(P, st);
+    }
     if (tdt == SPEC_BF16) return launch_tree<MODE_GREEDY, SPEC_BF16>(P, st);
     return launch_tree<MODE_GREEDY, SPEC_F32>(P, st);
 }
 
-spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
-                                    const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
-                                    const int32_t* tokens, const int32_t* parents,
-                                    const float* temperature, const float* coins, const float* final_u,
-                                    const float* draft_probs, int64_t dp_row_stride,
-                                    float threshold_single, float threshold_acc,
-                                    int32_t* out_accept_index, int32_t* out_tokens,
-                                    int32_t* out_num_accepted, float* diag,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
+static spec_status sample_entry(bool lazy, int B, int N, int V, int max_depth,
+                                const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                const int32_t* tokens, const int32_t* parents,
+                                const float* temperature, const float* coins, const float* final_u,
+                                const float* draft_probs, int64_t dp_row_stride,
+                                float threshold_single, float threshold_acc,
+                                int32_t* out_accept_index, int32_t* out_tokens,
+                                int32_t* out_num_accepted, float* diag,
+                                void* workspace, size_t workspace_bytes, void* stream) {
     g_detail[0] = 0;
     Params P{};
     spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
@@ -1959,9 +2494,52 @@ spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
     P.th_single = threshold_single; P.th_acc = threshold_acc;
     P.diag = diag;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (lazy) {
+        if (tdt == SPEC_BF16) return launch_tree_lazy<MODE_SAMPLE, SPEC_BF16>(P, st);
+        return launch_tree_lazy<MODE_SAMPLE, SPEC_F32>(P, st);
+    }
     if (tdt == SPEC_BF16) return launch_tree<MODE_SAMPLE, SPEC_BF16>(P, st);
     return launch_tree<MODE_SAMPLE, SPEC_F32>(P, st);
 }
+
+#define SPEC_CHAIN_ARGS_DECL                                                                         \
+    int B, int gamma, int V, const void* target_logits, spec_dtype tdt, int64_t t_row_stride,      \
+        const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,               \
+        const int32_t* draft_tokens, const float* temperature, const float* coins,                 \
+        const float* final_u, int32_t* out_tokens, int32_t* out_num_accepted, float* diag,         \
+        void* workspace, size_t workspace_bytes, void* stream
+#define SPEC_CHAIN_ARGS                                                                              \
+    B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs, d_row_stride,        \
+        draft_tokens, temperature, coins, final_u, out_tokens, out_num_accepted, diag, workspace,   \
+        workspace_bytes, stream
+#define SPEC_GREEDY_ARGS_DECL                                                                        \
+    int B, int N, int V, int max_depth, const void* target_logits, spec_dtype tdt,                 \
+        int64_t t_row_stride, const int32_t* tokens, const int32_t* parents,                       \
+        int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,                 \
+        void* workspace, size_t workspace_bytes, void* stream
+#define SPEC_GREEDY_ARGS                                                                             \
+    B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, out_accept_index,        \
+        out_tokens, out_num_accepted, workspace, workspace_bytes, stream
+#define SPEC_SAMPLE_ARGS_DECL                                                                        \
+    int B, int N, int V, int max_depth, const void* target_logits, spec_dtype tdt,                 \
+        int64_t t_row_stride, const int32_t* tokens, const int32_t* parents,                       \
+        const float* temperature, const float* coins, const float* final_u,                        \
+        const float* draft_probs, int64_t dp_row_stride, float threshold_single,                   \
+        float threshold_acc, int32_t* out_accept_index, int32_t* out_tokens,                       \
+        int32_t* out_num_accepted, float* diag, void* workspace, size_t workspace_bytes, void* stream
+#define SPEC_SAMPLE_ARGS                                                                             \
+    B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature, coins,      \
+        final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc, out_accept_index,     \
+        out_tokens, out_num_accepted, diag, workspace, workspace_bytes, stream
+
+extern "C" {
+
+spec_status spec_verify_chain(SPEC_CHAIN_ARGS_DECL) { return chain_entry(false, SPEC_CHAIN_ARGS); }
+spec_status spec_verify_chain_lazy(SPEC_CHAIN_ARGS_DECL) { return chain_entry(true, SPEC_CHAIN_ARGS); }
+spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(false, SPEC_GREEDY_ARGS); }
+spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(true, SPEC_GREEDY_ARGS); }
+spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(false, SPEC_SAMPLE_ARGS); }
+spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(true, SPEC_SAMPLE_ARGS); }
 
 }  // extern "C"
 

@@ -44,14 +44,17 @@ def lib():
                                "`python -m speculative_decoding_verify_temperature_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
-        L.spec_verify_chain.restype = i32
-        L.spec_verify_chain.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
-                                        P, P, P, P, P, P, P, P, sz, P]
-        L.spec_verify_tree_greedy.restype = i32
-        L.spec_verify_tree_greedy.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, sz, P]
-        L.spec_verify_tree_sample.restype = i32
-        L.spec_verify_tree_sample.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
-                                              f32, f32, P, P, P, P, P, sz, P]
+        for sfx in ("", "_lazy"):
+            f = getattr(L, "spec_verify_chain" + sfx)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64, P, P, P, P, P, P, P, P, sz, P]
+            f = getattr(L, "spec_verify_tree_greedy" + sfx)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, sz, P]
+            f = getattr(L, "spec_verify_tree_sample" + sfx)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
+                          f32, f32, P, P, P, P, P, sz, P]
         L.spec_workspace_bytes.restype = sz
         L.spec_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.spec_workspace_init.restype = i32
@@ -168,7 +171,8 @@ def _ws(workspace, entry, B, rows, V, device, stream):
 
 def spec_verify_chain(target, draft, draft_tokens, temperature, coins, final_u, *,
                       draft_is_probs: bool = False, V: int | None = None, out_tokens=None,
-                      out_num_accepted=None, diag=None, workspace=None, stream=None):
+                      out_num_accepted=None, diag=None, workspace=None, stream=None,
+                      _name: str = "spec_verify_chain"):
     """Chain verify of one round.  Returns ``(out_tokens [B, gamma+1], out_num_accepted [B])``."""
     B, R, S = target.shape
     gamma = R - 1
@@ -179,18 +183,18 @@ def spec_verify_chain(target, draft, draft_tokens, temperature, coins, final_u, 
     if out_num_accepted is None:
         out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
     ws = _ws(workspace, SPEC_ENTRY_CHAIN, B, gamma, V, dev, stream)
-    st = lib().spec_verify_chain(
+    st = getattr(lib(), _name)(
         B, gamma, V, _p(target), _dtype(target), _rows(target, "target"),
         _p(draft), SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
         _rows(draft, "draft"), _p(draft_tokens), _p(temperature), _p(coins), _p(final_u),
         _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
-    _check(st, "spec_verify_chain")
+    _check(st, _name)
     return out_tokens, out_num_accepted
 
 
 def spec_verify_tree_greedy(target, tokens, parents, max_depth: int, *, V: int | None = None,
                             out_accept_index=None, out_tokens=None, out_num_accepted=None,
-                            workspace=None, stream=None):
+                            workspace=None, stream=None, _name: str = "spec_verify_tree_greedy"):
     """Greedy tree verify.  Returns ``(accept_index, tokens, num_accepted)``."""
     B, N, S = target.shape
     V = S if V is None else int(V)
@@ -203,11 +207,11 @@ def spec_verify_tree_greedy(target, tokens, parents, max_depth: int, *, V: int |
     if out_num_accepted is None:
         out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
     ws = _ws(workspace, SPEC_ENTRY_TREE_GREEDY, B, N, V, dev, stream)
-    st = lib().spec_verify_tree_greedy(
+    st = getattr(lib(), _name)(
         B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens),
         _p(parents), _p(out_accept_index), _p(out_tokens), _p(out_num_accepted), _p(ws), ws.numel(),
         _stream(stream))
-    _check(st, "spec_verify_tree_greedy")
+    _check(st, _name)
     return out_accept_index, out_tokens, out_num_accepted
 
 
@@ -215,7 +219,7 @@ def spec_verify_tree_sample(target, tokens, parents, temperature, coins, final_u
                             draft_probs=None, threshold_single: float = 1.0,
                             threshold_acc: float = 1.0, V: int | None = None,
                             out_accept_index=None, out_tokens=None, out_num_accepted=None,
-                            diag=None, workspace=None, stream=None):
+                            diag=None, workspace=None, stream=None, _name: str = "spec_verify_tree_sample"):
     """Target-only tree sampling.  Returns ``(accept_index, tokens, num_accepted)``."""
     B, N, S = target.shape
     V = S if V is None else int(V)
@@ -229,10 +233,29 @@ def spec_verify_tree_sample(target, tokens, parents, temperature, coins, final_u
         out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
     ws = _ws(workspace, SPEC_ENTRY_TREE_SAMPLE, B, N, V, dev, stream)
     dstride = _rows(draft_probs, "draft_probs") if draft_probs is not None else 0
-    st = lib().spec_verify_tree_sample(
+    st = getattr(lib(), _name)(
         B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens),
         _p(parents), _p(temperature), _p(coins), _p(final_u), _p(draft_probs), dstride,
         float(threshold_single), float(threshold_acc), _p(out_accept_index), _p(out_tokens),
         _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
-    _check(st, "spec_verify_tree_sample")
+    _check(st, _name)
     return out_accept_index, out_tokens, out_num_accepted
+
+
+def spec_verify_chain_lazy(*args, **kw):
+    """Row-on-demand chain verify: the arguments and results of ``spec_verify_chain``
+    (bit-identical for valid inputs); ``diag`` entries of positions after the first
+    rejection are NaN."""
+    return spec_verify_chain(*args, _name="spec_verify_chain_lazy", **kw)
+
+
+def spec_verify_tree_greedy_lazy(*args, **kw):
+    """Row-on-demand greedy tree verify: the arguments and results of
+    ``spec_verify_tree_greedy``."""
+    return spec_verify_tree_greedy(*args, _name="spec_verify_tree_greedy_lazy", **kw)
+
+
+def spec_verify_tree_sample_lazy(*args, **kw):
+    """Row-on-demand target-only tree sampling: the arguments and results of
+    ``spec_verify_tree_sample``; ``diag`` holds NaN for children of unvisited nodes."""
+    return spec_verify_tree_sample(*args, _name="spec_verify_tree_sample_lazy", **kw)

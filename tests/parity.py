@@ -47,13 +47,17 @@ def oracle_chain(inp, rows=None, nthreads=0):
                         to_np(inp.coins[sel]), to_np(inp.final_u[sel]), V=inp.V, nthreads=nthreads)
 
 
-def gpu_chain(inp, workspace=None):
-    from speculative_decoding_verify_temperature_b200 import spec_verify_chain
+def _fn(name, lazy):
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    return getattr(sv, name + ("_lazy" if lazy else ""))
+
+
+def gpu_chain(inp, workspace=None, lazy=False):
     B, g = inp.B, inp.gamma
     diag = torch.full((B, 2 * g + 1), float("nan"), device=inp.target.device)
-    toks, na = spec_verify_chain(inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins,
-                                 inp.final_u, draft_is_probs=inp.draft_is_probs, V=inp.V, diag=diag,
-                                 workspace=workspace)
+    toks, na = _fn("spec_verify_chain", lazy)(
+        inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins, inp.final_u,
+        draft_is_probs=inp.draft_is_probs, V=inp.V, diag=diag, workspace=workspace)
     torch.cuda.synchronize()
     d = diag.cpu().numpy().astype(np.float64)
     return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy(),
@@ -95,10 +99,9 @@ def oracle_greedy(inp, rows=None, nthreads=0):
                               inp.max_depth, V=inp.V, nthreads=nthreads)
 
 
-def gpu_greedy(inp, workspace=None):
-    from speculative_decoding_verify_temperature_b200 import spec_verify_tree_greedy
-    ai, ot, na = spec_verify_tree_greedy(inp.target, inp.tokens, inp.parents, inp.max_depth, V=inp.V,
-                                         workspace=workspace)
+def gpu_greedy(inp, workspace=None, lazy=False):
+    ai, ot, na = _fn("spec_verify_tree_greedy", lazy)(inp.target, inp.tokens, inp.parents, inp.max_depth,
+                                                      V=inp.V, workspace=workspace)
     torch.cuda.synchronize()
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy())
 
@@ -112,14 +115,13 @@ def oracle_sample(inp, rows=None, nthreads=0, threshold_single=1.0, threshold_ac
                               threshold_acc=threshold_acc, V=inp.V, nthreads=nthreads)
 
 
-def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0):
-    from speculative_decoding_verify_temperature_b200 import spec_verify_tree_sample
+def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, lazy=False):
     B, N = inp.B, inp.N
     diag = torch.full((B, N + 1), float("nan"), device=inp.target.device)
-    ai, ot, na = spec_verify_tree_sample(inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins,
-                                         inp.final_u, inp.max_depth, draft_probs=inp.draft_probs,
-                                         threshold_single=threshold_single, threshold_acc=threshold_acc,
-                                         V=inp.V, diag=diag, workspace=workspace)
+    ai, ot, na = _fn("spec_verify_tree_sample", lazy)(
+        inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
+        draft_probs=inp.draft_probs, threshold_single=threshold_single, threshold_acc=threshold_acc,
+        V=inp.V, diag=diag, workspace=workspace)
     torch.cuda.synchronize()
     d = diag.cpu().numpy().astype(np.float64)
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy(),
@@ -149,11 +151,11 @@ def compare_tree(g, o, rows=None, sample=False):
 # ----------------------------------------------------------------------------- runners with the oracle's signature
 
 def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, coins, final_u, V=None,
-                     nthreads=0):
+                     nthreads=0, lazy=False):
     """Same call signature and result keys as ``oracle.chain`` (numpy in, numpy out),
     executed by the CUDA library.  Used to run the oracle's statistical pins
     through the GPU path."""
-    from speculative_decoding_verify_temperature_b200 import spec_verify_chain
+    spec_verify_chain = _fn("spec_verify_chain", lazy)
     dev = torch.device("cuda")
 
     def t(a):
@@ -174,8 +176,8 @@ def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, c
 
 
 def gpu_tree_sample_runner(target, tokens, parents, temperature, coins, final_u, max_depth, draft_probs=None,
-                           threshold_single=1.0, threshold_acc=1.0, V=None, nthreads=0):
-    from speculative_decoding_verify_temperature_b200 import spec_verify_tree_sample
+                           threshold_single=1.0, threshold_acc=1.0, V=None, nthreads=0, lazy=False):
+    spec_verify_tree_sample = _fn("spec_verify_tree_sample", lazy)
     dev = torch.device("cuda")
 
     def t(a):
@@ -197,8 +199,8 @@ def gpu_tree_sample_runner(target, tokens, parents, temperature, coins, final_u,
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy())
 
 
-def gpu_tree_greedy_runner(target, tokens, parents, max_depth, V=None, nthreads=0):
-    from speculative_decoding_verify_temperature_b200 import spec_verify_tree_greedy
+def gpu_tree_greedy_runner(target, tokens, parents, max_depth, V=None, nthreads=0, lazy=False):
+    spec_verify_tree_greedy = _fn("spec_verify_tree_greedy", lazy)
     dev = torch.device("cuda")
 
     def t(a):
