@@ -40,7 +40,9 @@
  *   with f32 accumulation (fp64 across chunks); T is per sequence.
  * - Uniforms (coins, final_u) are caller-supplied f32 values in [0, 1).
  *   Every random choice of a call is a deterministic function of them: the
- *   same inputs give bit-identical outputs.
+ *   same inputs give bit-identical outputs.  A coin of exactly 0 passes
+ *   coin <= ratio even when the ratio is 0, i.e. it accepts a token the
+ *   target gives probability 0; draw coins from (0, 1) to exclude that.
  * - Inverse-CDF draws scan the vocabulary in index order 0..V-1 and pick
  *   the smallest j with u * S < C_j (C = running sum of the weights, S the
  *   total): zero-weight tokens are never drawn.

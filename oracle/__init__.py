@@ -58,6 +58,9 @@ def lib():
         L.oracle_tree_sample.restype = None
         L.oracle_tree_sample.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                                          f32, f32, P, P, P, P, P, P, P, i32]
+        L.oracle_tree_mss.restype = None
+        L.oracle_tree_mss.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
+                                      P, P, P, P, P, P, P, i32]
         L.oracle_softmax_row.restype = i32
         L.oracle_softmax_row.argtypes = [P, i32, i32, f64, P]
         L.oracle_inverse_cdf.restype = i32
@@ -187,6 +190,41 @@ def tree_sample(target, tokens, parents, temperature, coins, final_u, max_depth:
                              _ptr(out["accept_index"]), _ptr(out["tokens"]),
                              _ptr(out["num_accepted"]), _ptr(out["pchild"]), _ptr(out["S"]),
                              _ptr(out["dmargin"]), _ptr(out["cmargin"]), int(nthreads))
+    return out
+
+
+def tree_mss(target, tokens, parents, temperature, coins, final_u, max_depth: int, draft_probs,
+             V=None, nthreads: int = 0) -> dict:
+    """Tree verification with a draft distribution (SpecInfer multi-step speculative
+    sampling).  ``coins`` is ``[B, N]`` (coin of the tested child), ``draft_probs``
+    f32 ``[B, N, dstride]`` (row n = the distribution n's children were drawn from)."""
+    target = _c(target)
+    B, N, ts = target.shape
+    V = ts if V is None else int(V)
+    tokens = _c(tokens, np.int32).reshape(B, N)
+    parents = _c(parents, np.int32).reshape(B, N)
+    temperature = _c(temperature, np.float32).reshape(B)
+    coins = _c(coins, np.float32).reshape(B, N)
+    final_u = _c(final_u, np.float32).reshape(B)
+    draft_probs = _c(draft_probs, np.float32)
+    W = max_depth + 1
+    out = dict(
+        accept_index=np.empty((B, W), np.int32),
+        tokens=np.empty((B, W), np.int32),
+        num_accepted=np.empty(B, np.int32),
+        ptest=np.empty((B, N), np.float64),
+        S=np.empty(B, np.float64),
+        dmargin=np.empty(B, np.float64),
+        cmargin=np.empty(B, np.float64),
+    )
+    if B == 0:
+        return out
+    lib().oracle_tree_mss(B, N, V, max_depth, _ptr(target), _dtype_code(target), ts,
+                          _ptr(tokens), _ptr(parents), _ptr(temperature), _ptr(coins),
+                          _ptr(final_u), _ptr(draft_probs), draft_probs.shape[2],
+                          _ptr(out["accept_index"]), _ptr(out["tokens"]),
+                          _ptr(out["num_accepted"]), _ptr(out["ptest"]), _ptr(out["S"]),
+                          _ptr(out["dmargin"]), _ptr(out["cmargin"]), int(nthreads))
     return out
 
 

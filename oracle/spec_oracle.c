@@ -491,6 +491,132 @@ void oracle_tree_sample(int B, int N, int V, int max_depth,
     }
 }
 
+/*
+ * Tree verification with a draft distribution: SpecInfer's multi-step
+ * speculative sampling ([origins] "SpecInfer", the MSS bullet: after a child
+ * is rejected the target distribution becomes the residual
+ * norm(max(0, p - q)) and the next sibling is tried; the output keeps the
+ * target distribution).
+ *   cur = root.  p = softmax(target row cur / T); q = draft_probs row cur,
+ *   the distribution the children of cur were drawn from.  Children c_1..c_m
+ *   in increasing node index: child c is accepted iff
+ *   coins[c] <= p(tok_c) / q(tok_c) (ratio +inf when q(tok_c) = 0); on
+ *   acceptance cur = c and the walk continues one level down with that
+ *   node's p and q; on rejection p <- max(0, p - q) / S, S = sum of
+ *   max(0, p - q) (p is kept when S is not positive: rounding only), and the
+ *   next sibling is tried.  When no child of cur is accepted, or cur is a
+ *   leaf, the last token is drawn with final_u from the current p.
+ * coins[b*N + c] is the uniform of the test of child c (coins[b*N] unused).
+ * draft_probs rows start at element (b*N+n)*dp_row_stride.  A drafted
+ * token's q(tok_c) must be finite and >= 0, else the sequence is invalid.
+ * Outputs as oracle_tree_greedy; out_ptest[b*N+c] = p(tok_c) at the test of
+ * child c (NaN for children never tested); out_S[b] = the last residual mass
+ * S at the final node (1 when it had no rejection); margins as oracle_chain.
+ */
+void oracle_tree_mss(int B, int N, int V, int max_depth,
+                     const void* target, int tdt, int64_t t_row_stride,
+                     const int32_t* tokens, const int32_t* parents,
+                     const float* temperature, const float* coins, const float* final_u,
+                     const float* draft_probs, int64_t dp_row_stride,
+                     int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,
+                     double* out_ptest, double* out_S, double* out_dmargin, double* out_cmargin,
+                     int nthreads) {
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel
+#endif
+    {
+        double* P = (double*)malloc(sizeof(double) * (size_t)V * (size_t)N);
+        double* p = (double*)malloc(sizeof(double) * (size_t)V);
+        double* p0 = (double*)malloc(sizeof(double) * (size_t)V);
+        int* depth = (int*)malloc(sizeof(int) * (size_t)N);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int b = 0; b < B; ++b) {
+            const int32_t* tk = tokens + (int64_t)b * N;
+            const int32_t* pa = parents + (int64_t)b * N;
+            int32_t* ai = out_accept_index + (int64_t)b * (max_depth + 1);
+            int32_t* ot = out_tokens + (int64_t)b * (max_depth + 1);
+            double* pt = out_ptest ? out_ptest + (int64_t)b * N : NULL;
+            double T = (double)temperature[b];
+            int bad = !temperature_ok(T) || !tree_ok(N, V, max_depth, tk, pa, depth);
+            for (int n = 0; n < N && !bad; ++n) {
+                const char* row = (const char*)target +
+                    ((int64_t)b * N + n) * t_row_stride * (tdt == OR_F32 ? 4 : 2);
+                if (softmax_T(row, tdt, V, T, P + (int64_t)n * V)) bad = 1;
+            }
+            fill_i32(ai, max_depth + 1, -1);
+            fill_i32(ot, max_depth + 1, -1);
+            if (pt) for (int n = 0; n < N; ++n) pt[n] = NAN;
+            double dmargin = INFINITY, S_last = 1.0;
+            int cur = 0, k = 0;
+            if (!bad) {
+                ai[0] = 0;
+                for (;;) {
+                    const float* q = draft_probs + ((int64_t)b * N + cur) * dp_row_stride;
+                    for (int j = 0; j < V; ++j) p[j] = p0[j] = P[(int64_t)cur * V + j];
+                    S_last = 1.0;
+                    int next = -1;
+                    for (int c = cur + 1; c < N && !bad; ++c) {
+                        if (pa[c] != cur) continue;
+                        const double qx = (double)q[tk[c]];
+                        if (!(qx >= 0.0 && qx <= 0x1.fffffep127)) { bad = 1; break; }
+                        const double px = p[tk[c]];
+                        if (pt) pt[c] = px;
+                        const double ratio = qx > 0.0 ? px / qx : INFINITY;
+                        const double u = (double)coins[(int64_t)b * N + (g_mutation == 15 ? cur : c)];
+                        const double m = fabs(u - ratio);
+                        if (m < dmargin) dmargin = m;
+                        if (u <= ratio) { next = c; break; }
+                        if (g_mutation == 13) continue;                 /* residual never taken */
+                        const double* base = (g_mutation == 14) ? p0 : p; /* residual of the first p */
+                        double S = 0.0;
+                        for (int j = 0; j < V; ++j) {
+                            const double d = base[j] - (double)q[j];
+                            S += d > 0.0 ? d : 0.0;
+                        }
+                        if (!(S <= 0x1.fffffffffffffp1023)) { bad = 1; break; }   /* NaN or inf */
+                        if (S > 0.0) {
+                            for (int j = 0; j < V; ++j) {
+                                const double d = base[j] - (double)q[j];
+                                p[j] = (d > 0.0 ? d : 0.0) / S;
+                            }
+                            S_last = S;
+                        }
+                    }
+                    if (bad || next < 0) break;
+                    ot[k] = tk[next];
+                    ++k;
+                    ai[k] = next;
+                    cur = next;
+                }
+            }
+            if (bad) {
+                fill_i32(ai, max_depth + 1, -1);
+                fill_i32(ot, max_depth + 1, -1);
+                out_num_accepted[b] = -1;
+                if (pt) for (int n = 0; n < N; ++n) pt[n] = NAN;
+                if (out_S) out_S[b] = NAN;
+                if (out_dmargin) out_dmargin[b] = INFINITY;
+                if (out_cmargin) out_cmargin[b] = INFINITY;
+                continue;
+            }
+            double S1, cm = INFINITY;
+            const int y = inverse_cdf(p, V, (double)final_u[b], &S1, &cm);
+            ot[k] = y;
+            out_num_accepted[b] = k;
+            if (out_S) out_S[b] = S_last;
+            if (out_dmargin) out_dmargin[b] = dmargin;
+            if (out_cmargin) out_cmargin[b] = cm;
+        }
+        free(P);
+        free(p);
+        free(p0);
+        free(depth);
+    }
+}
+
 /* Exposed for the pins: the temperature softmax of one row, and the
  * inverse-CDF draw, exactly as the verify functions above use them. */
 int oracle_softmax_row(const void* row, int dtype, int V, double T, double* p) {

@@ -258,7 +258,10 @@ def _sample_rows(probs: np.ndarray, rng) -> np.ndarray:
 
 
 def _uniform24(rng, shape):
-    return (rng.integers(0, 1 << 24, size=shape) * 2.0 ** -24).astype(np.float32)
+    """Uniforms k * 2^-24, k in [1, 2^24): exact in f32, and never 0 -- with u = 0
+    the rule u <= p(x)/q(x) would accept a token whose target probability is 0
+    (an event of probability 0 for a continuous uniform, 2^-24 on this grid)."""
+    return (rng.integers(1, 1 << 24, size=shape) * 2.0 ** -24).astype(np.float32)
 
 
 def chain_chisquare(V=4, gamma=3, K=3, rounds=1_000_000, seed=3, draft_kind="probs",
@@ -505,6 +508,157 @@ def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3, r
             res = (runner or oracle.tree_sample)(tab.PL[nid], tokens, np.broadcast_to(par, (m, N)),
                                      np.ones(m, np.float32), _uniform24(rng, (m, N)),
                                      _uniform24(rng, m), max(d))
+            k = res["num_accepted"]
+            if (k < 0).any():
+                return dict(ok=False, p=0.0)
+            for j in range(max(d) + 1):
+                sel = k >= j
+                idx = sub[sel]
+                tok = res["tokens"][sel, j]
+                put = ntok[idx] < K
+                first[idx[put], ntok[idx[put]]] = tok[put]
+                ntok[idx[put]] += 1
+                ids[idx] = tab.child(ids[idx], tok)
+        active = active[ntok[active] < K]
+    return _chisq(first, tab, V, K, pmin)
+
+
+# ----------------------------------------------------------------------------- trees with a draft distribution (MSS)
+
+def _mss_cases(model: ToyModel, prefix, parents):
+    """Every way one round of multi-step speculative sampling can go on a fixed
+    tree shape: the children's tokens drawn independently from the draft
+    distribution at their parent (weight = product of q), then every cell of
+    the coins' and final uniform's breakpoint partition, with its probability
+    under the rule (accept child with min(1, p/q), else p <- norm(max(0, p - q))
+    and try the next sibling; at the end draw from p)."""
+    V = model.V
+    N = len(parents)
+    children = {}
+    for n in range(1, N):
+        children.setdefault(int(parents[n]), []).append(n)
+    cases = []
+    for toks in itertools.product(range(V), repeat=N - 1):
+        tokens = np.zeros(N, np.int32)
+        tokens[1:] = toks
+        path = _paths(parents, tokens)
+        wq = 1.0
+        for n in range(1, N):
+            wq *= model.q(prefix + path[parents[n]])[1][tokens[n]]
+        if wq == 0.0:
+            continue
+        target = np.stack([model.p(prefix + path[n])[0] for n in range(N)])
+        draft = np.stack([model.q(prefix + path[n])[0] for n in range(N)]).astype(np.float32)
+
+        def visit(cur, weight, coins):
+            p = model.p(prefix + path[cur])[1].copy()
+            q = model.q(prefix + path[cur])[1]
+            for c in children.get(cur, []):
+                x = tokens[c]
+                a = min(1.0, p[x] / q[x])
+                if a > 0:
+                    visit(c, weight * a, coins | {c: a / 2})
+                if a >= 1.0:
+                    return
+                weight *= 1.0 - a
+                coins = coins | {c: (1.0 + a) / 2}
+                r = np.maximum(0.0, p - q)
+                p = r / r.sum()
+            C = np.cumsum(p)
+            for j in range(V):
+                if p[j] > 0:
+                    cv = np.full(N, 0.5, np.float32)
+                    for node, val in coins.items():
+                        cv[node] = val
+                    cases.append(dict(weight=wq * weight * p[j], target=target, draft=draft, tokens=tokens,
+                                      coins=cv, u=np.float32(C[j] - p[j] / 2)))
+
+        visit(0, 1.0, {})
+    return cases
+
+
+def tree_mss_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 0, 1, 1), tol=1e-12, T=1.0,
+                        runner=None) -> dict:
+    """Exact distribution of the first K tokens of repeated multi-step speculative
+    sampling rounds (children drawn from q) against the target's autoregressive
+    distribution ([origins] "SpecInfer": MSS keeps the target distribution)."""
+    model = ToyModel(V, seed, "probs", T=T)
+    parents = np.array(parents, np.int32)
+    N = len(parents)
+    depth = max(len(p) for p in _paths(parents, np.zeros(N, np.int32)))
+    states = {(): 1.0}
+    dist = {}
+    while states:
+        batch, owners = [], []
+        for prefix, w in states.items():
+            cs = _mss_cases(model, prefix, parents)
+            batch += cs
+            owners += [(prefix, w)] * len(cs)
+        m = len(batch)
+        res = (runner or oracle.tree_mss)(np.stack([c["target"] for c in batch]),
+                                          np.stack([c["tokens"] for c in batch]),
+                                          np.broadcast_to(parents, (m, N)), np.full(m, model.T, np.float32),
+                                          np.stack([c["coins"] for c in batch]),
+                                          np.array([c["u"] for c in batch], np.float32), depth,
+                                          np.stack([c["draft"] for c in batch]))
+        nxt = {}
+        for i, (prefix, w) in enumerate(owners):
+            k = int(res["num_accepted"][i])
+            if k < 0:
+                return dict(ok=False, err=float("inf"))
+            h = prefix + tuple(int(t) for t in res["tokens"][i, :k + 1])
+            ww = w * batch[i]["weight"]
+            if len(h) >= K:
+                dist[h[:K]] = dist.get(h[:K], 0.0) + ww
+            else:
+                nxt[h] = nxt.get(h, 0.0) + ww
+        states = nxt
+    want = _product_distribution(model, K)
+    err = max(abs(dist.get(s, 0.0) - pv) for s, pv in want.items())
+    err = max(err, sum(v for s, v in dist.items() if s not in want))
+    return dict(ok=err < tol, err=err)
+
+
+def tree_mss_chisquare(V=4, K=3, rounds=1_000_000, seed=16, shapes=None, pmin=1e-3, runner=None) -> dict:
+    """Simulated multi-step speculative sampling rounds over a few tree shapes whose
+    children are drawn independently from the draft distribution at their parent
+    (duplicate siblings included); chi-square of the first K tokens."""
+    shapes = shapes or [(-1, 0, 0, 0, 1, 1), (-1, 0, 1, 2), (-1, 0, 0, 1, 1, 2, 2, 3)]
+    model = ToyModel(V, seed, "probs")
+    maxd = 0
+    for sh in shapes:
+        d = [0] * len(sh)
+        for n in range(1, len(sh)):
+            d[n] = d[sh[n]] + 1
+        maxd = max(maxd, max(d))
+    tab = _Tables(model, K - 1 + maxd)
+    rng = np.random.default_rng(seed + 13)
+    n = rounds
+    ids = np.zeros(n, np.int64)
+    ntok = np.zeros(n, np.int64)
+    first = np.zeros((n, K), np.int64)
+    active = np.arange(n)
+    while active.size:
+        pick = rng.integers(0, len(shapes), active.size)
+        for si, shape in enumerate(shapes):
+            sub = active[pick == si]
+            if sub.size == 0:
+                continue
+            m = sub.size
+            par = np.array(shape, np.int32)
+            N = len(par)
+            tokens = np.zeros((m, N), np.int32)
+            nid = np.zeros((m, N), np.int64)
+            nid[:, 0] = ids[sub]
+            for c in range(1, N):
+                tokens[:, c] = _sample_rows(tab.Q[nid[:, par[c]]], rng)
+                nid[:, c] = tab.child(nid[:, par[c]], tokens[:, c])
+            d = [0] * N
+            for c in range(1, N):
+                d[c] = d[par[c]] + 1
+            res = (runner or oracle.tree_mss)(tab.PL[nid], tokens, np.broadcast_to(par, (m, N)),
+                                              np.ones(m, np.float32), _uniform24(rng, (m, N)),
+                                              _uniform24(rng, m), max(d), tab.QR[nid])
             k = res["num_accepted"]
             if (k < 0).any():
                 return dict(ok=False, p=0.0)

@@ -45,6 +45,20 @@ def test_tree_bruteforce_lossless(parents, V, K, seed, T, zeros):
     assert r["ok"], r
 
 
+@pytest.mark.parametrize("parents,V,K,seed,T", [
+    ((-1, 0, 0, 0, 1, 1), 3, 3, 5, 1.0),
+    ((-1, 0, 0, 1, 2, 2), 3, 2, 7, 0.7),
+    ((-1, 0, 0, 0, 1, 1), 4, 2, 3, 1.0),              # three siblings, V=4: second residuals matter
+    ((-1, 0, 1, 2), 4, 2, 9, 1.3),                     # chain-shaped tree
+    ((-1,), 3, 2, 35, 1.0),                            # root only: plain sampling
+])
+def test_tree_mss_bruteforce_lossless(parents, V, K, seed, T):
+    """Multi-step speculative sampling with the children drawn from q keeps the
+    target distribution exactly ([origins] "SpecInfer", MSS bullet)."""
+    r = pins.tree_mss_bruteforce(V=V, K=K, seed=seed, parents=parents, T=T)
+    assert r["ok"], r
+
+
 # ----------------------------------------------------------------------------- closed form
 
 @pytest.mark.parametrize("seed,kind", [(2, "probs"), (3, "logits"), (12, "probs")])
@@ -75,6 +89,12 @@ def test_chain_chisquare(seed, kind, T):
 @pytest.mark.parametrize("seed", [6, 16])
 def test_tree_chisquare(seed):
     r = pins.tree_chisquare(rounds=1_000_000, seed=seed)
+    assert r["ok"], r
+
+
+@pytest.mark.parametrize("seed", [16, 17])
+def test_tree_mss_chisquare(seed):
+    r = pins.tree_mss_chisquare(rounds=1_000_000, seed=seed)
     assert r["ok"], r
 
 
@@ -258,6 +278,58 @@ def test_cross_identity_tree_chain_onehot():
         assert list(rc["tokens"][0, :k + 1]) == list(rt["tokens"][0, :k + 1]), trial
 
 
+def test_cross_identity_mss_chain_tree_equals_chain():
+    """Multi-step speculative sampling on a chain-shaped tree is chain verify with
+    draft probabilities: one child per node, so the rejection of that child is
+    rule 2 (draw from norm(max(0, p - q))) and reaching the leaf is rule 3."""
+    rng = np.random.default_rng(14)
+    for trial in range(300):
+        V = int(rng.integers(2, 40))
+        gamma = int(rng.integers(1, 7))
+        T = float(rng.choice([0.5, 1.0, 1.7]))
+        t = rng.normal(0, 2, (1, gamma + 1, V)).astype(np.float32)
+        q = special.softmax(rng.normal(0, 2, (1, gamma, V)), axis=-1).astype(np.float32)
+        x = np.array([[rng.choice(V, p=q[0, i] / q[0, i].sum()) for i in range(gamma)]], np.int32)
+        coins = (rng.integers(0, 1 << 24, (1, gamma)) * 2.0 ** -24).astype(np.float32)
+        fu = rng.random(1).astype(np.float32)
+        rc = oracle.chain(t, q, True, x, np.array([T]), coins, fu)
+        tokens = np.concatenate([[0], x[0]]).astype(np.int32)[None]
+        parents = np.arange(-1, gamma, dtype=np.int32)[None]
+        tc = np.concatenate([[0.5], coins[0]]).astype(np.float32)[None]     # coin of child n = coins[n-1]
+        qt = np.concatenate([q, np.full((1, 1, V), 1.0 / V, np.float32)], axis=1)
+        rt = oracle.tree_mss(t, tokens, parents, np.array([T]), tc, fu, gamma, qt)
+        if min(rc["dmargin"][0], rt["dmargin"][0], rc["cmargin"][0], rt["cmargin"][0]) < 1e-9:
+            continue
+        assert rc["num_accepted"][0] == rt["num_accepted"][0], trial
+        k = rc["num_accepted"][0]
+        assert list(rc["tokens"][0, :k + 1]) == list(rt["tokens"][0, :k + 1]), trial
+        if k < gamma:
+            assert abs(rc["S"][0] - rt["S"][0]) <= 1e-12 * max(1.0, rc["S"][0]), trial
+
+
+def test_mss_invalid_inputs_and_diagnostics():
+    rng = np.random.default_rng(15)
+    V, N = 12, 4
+    t = rng.normal(0, 1, (4, N, V)).astype(np.float32)
+    q = special.softmax(rng.normal(0, 1, (4, N, V)), axis=-1).astype(np.float32)
+    tok = np.array([[0, 3, 5, 7]] * 4, np.int32)
+    par = np.array([[-1, 0, 0, 1]] * 4, np.int32)
+    T = np.array([1.0, np.nan, 1.0, 1.0], np.float32)
+    par[2, 2] = 3                                          # parent after child
+    q[3, 0, 3] = -0.5                                      # a drafted token's q(x) < 0
+    coins = np.full((4, N), 0.999, np.float32)             # reject every child
+    r = oracle.tree_mss(t, tok, par, T, coins, np.full(4, 0.5, np.float32), 2, q)
+    assert list(r["num_accepted"]) == [0, -1, -1, -1]
+    assert (r["tokens"][1:] == -1).all() and np.isnan(r["ptest"][1:]).all()
+    # sequence 0: both root children tested (p(x) recorded), node 3 never tested
+    p0 = special.softmax(t[0, 0].astype(np.float64))
+    assert abs(r["ptest"][0, 1] - p0[3]) < 1e-12
+    p1 = np.maximum(0, p0 - q[0, 0].astype(np.float64))
+    p1 /= p1.sum()
+    assert abs(r["ptest"][0, 2] - p1[5]) < 1e-12
+    assert np.isnan(r["ptest"][0, 3]) and np.isnan(r["ptest"][0, 0])
+
+
 def test_thresholds_literal():
     """threshold_single = 0 accepts the first child at every level (p >= 0);
     a tiny threshold_acc accepts the first child with positive probability."""
@@ -314,6 +386,10 @@ MUTATIONS = {
     10: ("rejected children not removed", lambda: pins.tree_bruteforce()),
     11: ("logits multiplied by T", lambda: pins.chain_bruteforce(T=0.6)),
     12: ("draft logits without T", lambda: pins.chain_bruteforce(draft_kind="logits", seed=11, T=0.7)),
+    13: ("MSS: p not replaced by the residual after a rejection", lambda: pins.tree_mss_bruteforce()),
+    14: ("MSS: every residual taken from the node's first p",
+         lambda: pins.tree_mss_bruteforce(V=4, K=2, seed=3, parents=(-1, 0, 0, 0, 1, 1))),
+    15: ("MSS: children tested with their parent's coin", lambda: pins.tree_mss_bruteforce()),
 }
 
 
