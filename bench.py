@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -89,6 +89,8 @@ def make_inputs(wid: int, rnd: int, device, rank: int = 0):
         return wl.tree_config2(r, device)
     if wid == 3:
         return wl.tree_config3(r, device)
+    if wid == 5:
+        return wl.tree_config5(r, device)
     return wl.chain_config4(r, device)
 
 
@@ -135,6 +137,10 @@ class Runner:
             getattr(sv, "spec_verify_chain" + self.sfx)(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                  draft_is_probs=i.draft_is_probs, V=i.V, out_tokens=self.out[0],
                                  out_num_accepted=self.out[1], workspace=self.ws)
+        elif self.wid == 5:
+            getattr(sv, "spec_verify_tree_mss" + self.sfx)(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u, i.max_depth,
+                                    i.draft_probs, V=i.V, out_accept_index=self.out[0], out_tokens=self.out[1],
+                                    out_num_accepted=self.out[2], workspace=self.ws)
         elif self.wid == 2:
             getattr(sv, "spec_verify_tree_greedy" + self.sfx)(i.target, i.tokens, i.parents, i.max_depth, V=i.V,
                                        out_accept_index=self.out[0], out_tokens=self.out[1],
@@ -159,7 +165,7 @@ def lazy_kernels_per_step(wid, inp) -> int:
     chain's last level has no decision), then the final draw (none for greedy)."""
     if wid in (0, 1, 4):
         return 2 * inp.gamma + 2
-    return 2 * (inp.max_depth + 1) + (1 if wid == 3 else 0)
+    return 2 * (inp.max_depth + 1) + (1 if wid == 3 else 0)      # workload 5 draws inside its last level
 
 
 def lazy_bytes_read(wid, inp, num_accepted) -> int:
@@ -181,7 +187,7 @@ def workspace_for(wid, inp):
     ws = sv.Workspace(inp.target.device)
     if wid in (0, 1, 4):
         return ws.get(sv.SPEC_ENTRY_CHAIN, inp.B, inp.gamma, inp.V)
-    e = sv.SPEC_ENTRY_TREE_GREEDY if wid == 2 else sv.SPEC_ENTRY_TREE_SAMPLE
+    e = {2: sv.SPEC_ENTRY_TREE_GREEDY, 3: sv.SPEC_ENTRY_TREE_SAMPLE, 5: sv.SPEC_ENTRY_TREE_MSS}[wid]
     return ws.get(e, inp.B, inp.N, inp.V)
 
 
@@ -269,11 +275,11 @@ def cpu_baseline(wid, inp, seconds, nthreads=None):
     # Copy the inputs to host once; the oracle reads the same bytes the GPU reads.
     n = 0
     fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain,
-          2: parity.oracle_greedy, 3: parity.oracle_sample}[wid]
+          2: parity.oracle_greedy, 3: parity.oracle_sample, 5: parity.oracle_mss}[wid]
     B = inp.B
     # Large workloads: a bounded sample of whole sequences per "round" of work,
     # scaled to full rounds below.
-    per = B if wid in (0, 1) else max(1, min(B, {2: 8, 3: 4, 4: 16}[wid]))
+    per = B if wid in (0, 1) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4}[wid]))
     rows = None if per == B else list(range(per))
     elapsed = 0.0
     while n == 0 or elapsed < seconds:

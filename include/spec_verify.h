@@ -86,7 +86,8 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 typedef enum {
     SPEC_ENTRY_CHAIN = 0,
     SPEC_ENTRY_TREE_GREEDY = 1,
-    SPEC_ENTRY_TREE_SAMPLE = 2
+    SPEC_ENTRY_TREE_SAMPLE = 2,
+    SPEC_ENTRY_TREE_MSS = 3
 } spec_entry;
 
 /*
@@ -207,6 +208,67 @@ spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
                                     int32_t* out_accept_index, int32_t* out_tokens,
                                     int32_t* out_num_accepted, float* diag,
                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * spec_verify_tree_mss -- tree verification with a draft distribution
+ * (multi-step speculative sampling).  [origins] "SpecInfer", MSS bullet:
+ * after a child is rejected the target distribution is replaced by the
+ * residual norm(max(0, p - q)) and the next sibling is tried; the emitted
+ * tokens keep the target distribution when the children of every node were
+ * drawn independently from that node's draft distribution.
+ *
+ * p = softmax(target row cur / T_b) and q = draft_probs row cur, starting at
+ * the root.  The children of cur are tested in increasing node index: child
+ * c is accepted iff coins[b,c] <= p(tokens[b,c]) / q(tokens[b,c]) (ratio +inf
+ * when q = 0); on acceptance the walk moves to c (fresh p and q of c); on
+ * rejection p <- max(0, p - q) / S, S = sum_j max(0, p_j - q_j) (p is kept
+ * when S is not positive: rounding only), and the next sibling is tried.
+ * When no child of cur is accepted, or cur is a leaf, the last token is
+ * drawn with final_u[b] from the current p.
+ *
+ * Arguments as spec_verify_tree_greedy, plus:
+ * temperature    [B] f32.
+ * coins          [B, N] f32: coins[b,c] is the uniform of the test of child
+ *                c (coins[b,0] is not read).  Note the difference from
+ *                spec_verify_tree_sample, whose coins belong to the visited
+ *                parent.
+ * final_u        [B] f32.
+ * draft_probs    [B, N, dp_row_stride] f32, required: row n is the draft
+ *                distribution from which the children of node n were drawn.
+ *                Only the rows of visited nodes are read; the drafted
+ *                tokens' entries must be finite and >= 0 (else the sequence
+ *                is invalid).  Never written.
+ * diag           nullable, [B, N+1] f32: p(tokens[b,c]) at the test of child
+ *                c (NaN for children never tested, and at n = 0), then the
+ *                last residual mass S at the final node (1 without one).
+ * workspace      >= spec_workspace_bytes(SPEC_ENTRY_TREE_MSS, B, N, V).
+ * Each rejection costs one extra pass over the (target, q) row pair of the
+ * node.
+ *
+ * spec_verify_tree_mss_lazy: the same call, walking level by level and
+ * reading only the rows of the visited nodes (see the lazy variants below):
+ * outputs bit-identical for valid inputs; rows never read are not validated.
+ */
+spec_status spec_verify_tree_mss(int B, int N, int V, int max_depth,
+                                 const void* target_logits, spec_dtype tdt,
+                                 int64_t t_row_stride,
+                                 const int32_t* tokens, const int32_t* parents,
+                                 const float* temperature, const float* coins,
+                                 const float* final_u,
+                                 const float* draft_probs, int64_t dp_row_stride,
+                                 int32_t* out_accept_index, int32_t* out_tokens,
+                                 int32_t* out_num_accepted, float* diag,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_verify_tree_mss_lazy(int B, int N, int V, int max_depth,
+                                      const void* target_logits, spec_dtype tdt,
+                                      int64_t t_row_stride,
+                                      const int32_t* tokens, const int32_t* parents,
+                                      const float* temperature, const float* coins,
+                                      const float* final_u,
+                                      const float* draft_probs, int64_t dp_row_stride,
+                                      int32_t* out_accept_index, int32_t* out_tokens,
+                                      int32_t* out_num_accepted, float* diag,
+                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * spec_verify_chain_noalloc -- spec_verify_chain without a caller workspace.

@@ -14,6 +14,8 @@ from .spec_verify import (  # noqa: F401
     spec_verify_chain_lazy,
     spec_verify_tree_greedy,
     spec_verify_tree_greedy_lazy,
+    spec_verify_tree_mss,
+    spec_verify_tree_mss_lazy,
     spec_verify_tree_sample,
     spec_verify_tree_sample_lazy,
     spec_workspace_bytes,

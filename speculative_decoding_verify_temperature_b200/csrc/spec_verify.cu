@@ -49,7 +49,7 @@ constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
 constexpr double LOG2E = 1.4426950408889634073599246810019;
 
-enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2 };
+enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2, MODE_MSS = 3 };
 enum { DK_NONE = 0, DK_LOGITS = 1, DK_PROBS = 2 };
 
 template <int DT> struct Tr;
@@ -650,6 +650,38 @@ template <int TDT> struct WTreeRes {         // relu(p_j - d_j), excluded tokens
     }
 };
 
+// Multi-step residual weights at one tree node.  After j rejections the
+// target distribution is p_j = max(0, p_0 - c_j q) / F(c_j), where
+// F(c) = sum_v max(0, p_0(v) - c q(v)), c_0 = 0 and c_{j+1} = c_j + F(c_j):
+// the residual of max(0, p_0 - c q) / F(c) against q is max(0, p_0 - (c +
+// F(c)) q) / F(c) wherever it is positive, and 0 where p_0 <= c q.  The
+// weight here is max(0, p_0 - c q) with p_0 = 2^(x s - m) / Z; its sum is
+// F(c).
+template <int TDT> struct WMss {
+    const char* row; const char* drow; float s, m, iz, c; int V;
+    struct Raw { Raw8<TDT> t; Raw8<SPEC_F32> d; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const {
+        load_raw8<TDT>(row, e0, r.t);
+        load_raw8<SPEC_F32>(drow, e0, r.d);
+    }
+    __device__ __forceinline__ void finish(const float (&x)[8], const float (&d)[8], float (&w)[8]) const {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = fmaxf(0.f, fmaf(-c, d[i], ex2(fmaf(x[i], s, -m)) * iz));
+    }
+    __device__ __forceinline__ void weights(int64_t, const Raw& r, float (&w)[8]) const {
+        float x[8], d[8];
+        raw8_f32<TDT>(r.t, x);
+        raw8_f32<SPEC_F32>(r.d, d);
+        finish(x, d, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8];
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+        ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        finish(x, d, w);
+    }
+};
+
 // Group sums of the GPT groups this thread owns in chunk c (groups
 // g = k*NT + tid, coalesced).  For a chunk wholly inside the row, four groups'
 // loads are issued before any of them is used.
@@ -695,6 +727,40 @@ __device__ __forceinline__ float chunk_weight_partial(const WF& wf, int c) {
 #pragma unroll
     for (int k = 0; k < GPT; ++k) acc += gs[k];
     return acc;
+}
+
+// Per-warp sums of the weights of every chunk of a row: wpw[c * BT/32 + warp]
+// (f32).  Whole chunks inside the row go three at a time, the loads of all
+// three issued before any weight is formed; no block-wide barrier per chunk.
+template <int CH, int BT, class WF>
+__device__ void row_warp_sums(const WF& wf, int nch, float* wpw) {
+    constexpr int GPT = CH / 8 / BT, NWB = BT / 32, CB = 3;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int c = 0;
+    for (; c + CB <= nch && (int64_t)(c + CB) * CH <= wf.V; c += CB) {
+        typename WF::Raw raw[CB][GPT];
+#pragma unroll
+        for (int j = 0; j < CB; ++j)
+#pragma unroll
+            for (int k = 0; k < GPT; ++k)
+                wf.load((int64_t)(c + j) * CH + (int64_t)(k * BT + threadIdx.x) * 8, raw[j][k]);
+#pragma unroll
+        for (int j = 0; j < CB; ++j) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < GPT; ++k) {
+                float w[8];
+                wf.weights((int64_t)(c + j) * CH + (int64_t)(k * BT + threadIdx.x) * 8, raw[j][k], w);
+                acc += ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) wpw[(c + j) * NWB + warp] = acc;
+        }
+    }
+    for (; c < nch; ++c) {
+        const float acc = warp_sum(chunk_weight_partial<CH, BT>(wf, c));
+        if (lane == 0) wpw[c * NWB + warp] = acc;
+    }
 }
 
 // Inverse-CDF rescan of chunk c: the chunk is read as coalesced 8-element
@@ -889,14 +955,16 @@ struct ChainPrefetch {
     int x;          // draft token of position tid
     float l;        // target logit at x
     float d;        // draft logit (or probability) at x
+    float coin;     // coins[b, tid]
     bool ok;        // x in [0, V)
 };
 
 template <int TDT, int DDT, int DK>
 __device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) {
-    ChainPrefetch f{0, 0.f, 0.f, false};
+    ChainPrefetch f{0, 0.f, 0.f, 0.f, false};
     const int tid = threadIdx.x, gamma = P.gamma;
     if (tid < gamma) {
+        f.coin = P.coins[(size_t)b * gamma + tid];
         f.x = P.draft_tokens[(size_t)b * gamma + tid];
         f.ok = f.x >= 0 && f.x < P.V;
         if (f.ok) {
@@ -940,6 +1008,7 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
         }
         sh.pch[tid] = p;
         sh.pch[SPEC_MAX_GAMMA + tid] = q;
+        sh.pch[2 * SPEC_MAX_GAMMA + tid] = (double)f.coin;
         sh.rej[tid] = ok;
         sh.tok[tid] = f.x;
     }
@@ -953,7 +1022,7 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
             for (int i = 0; i < gamma; ++i) {
                 const double pi = sh.pch[i], qi = sh.pch[SPEC_MAX_GAMMA + i];
                 const double ratio = (qi > 0.0) ? pi / qi : INFINITY;
-                if (!((double)P.coins[(size_t)b * gamma + i] <= ratio)) { k = i; break; }
+                if (!(sh.pch[2 * SPEC_MAX_GAMMA + i] <= ratio)) { k = i; break; }
             }
         }
         sh.ivals[0] = ok;
@@ -1287,6 +1356,212 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     }
 }
 
+// Locate the chunk holding t among the chunk masses sh.M[0..nch) (skipping
+// empty chunks) and rescan it; retries past chunks whose rescan finds no
+// positive weight (possible only through rounding).  Returns -1 if none.
+template <int CH, int BT, class WF>
+__device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u, FinShared& sh) {
+    const int tid = threadIdx.x;
+    int y = -1;
+    for (int attempt = 0; attempt < nch && y < 0; ++attempt) {
+        if (tid == 0) {
+            double C = 0.0, before = 0.0;
+            int cs = -1;
+            for (int cc = 0; cc < nch; ++cc) {
+                if (sh.M[cc] <= 0.0) continue;
+                if (t < C + sh.M[cc]) { cs = cc; before = C; break; }
+                C += sh.M[cc];
+            }
+            if (cs < 0)
+                for (int cc = nch - 1; cc >= 0; --cc)
+                    if (sh.M[cc] > 0.0) { cs = cc; before = C - sh.M[cc]; break; }
+            sh.ivals[2] = cs;
+            sh.dvals[1] = before;
+        }
+        __syncthreads();
+        const int cs = sh.ivals[2];
+        if (cs < 0) break;
+        double tot;
+        y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+        if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+        __syncthreads();
+    }
+    return y;
+}
+
+// Chunk masses sh.M[0..nch) of the weights wf over a row (per-warp sums in
+// wpw, then fp64 per chunk in warp order); returns their total (fp64, chunk
+// order).  All threads of the CTA call it.
+template <int CH, int BT, class WF>
+__device__ double row_chunk_masses(const WF& wf, int nch, float* wpw, FinShared& sh) {
+    constexpr int NWB = BT / 32;
+    row_warp_sums<CH, BT>(wf, nch, wpw);
+    __syncthreads();
+    for (int c = threadIdx.x; c < nch; c += BT) {
+        double M = 0.0;
+#pragma unroll
+        for (int w = 0; w < NWB; ++w) M += (double)wpw[c * NWB + w];
+        sh.M[c] = M;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double S = 0.0;
+        for (int c = 0; c < nch; ++c) S += sh.M[c];
+        sh.dvals[0] = S;
+    }
+    __syncthreads();
+    const double S = sh.dvals[0];
+    __syncthreads();
+    return S;
+}
+
+// State of the multi-step sampling walk at one node: p_j = max(0, p_0 - c q)
+// / D, D = F(c) (see WMss), after `steps` residual steps; `have_M` when sh.M
+// holds the chunk masses of max(0, p_0 - c q); S = the last residual mass
+// S_j = D_j / D_{j-1} (1 before any).  Uniform across the CTA.
+struct MssState {
+    double c, D, S;
+    int steps;
+    bool have_M;
+};
+
+// Multi-step speculative sampling at node cur of sequence b ([origins]
+// "SpecInfer", MSS bullet), all threads of the CTA: the children of cur
+// (sh.par / sh.tok) are tested in node order, child c with coins[b, c]
+// against p_j(x) / q(x), p_j(x) = max(0, p_0(x) - c q(x)) / D in fp64 from the
+// gathered logit; a rejection costs one pass over the (target, q) row pair
+// for the next F.  Returns the accepted child, -1 when none is (st then
+// describes the p of the final draw), -2 for an invalid drafted q(x) or a
+// non-finite residual mass.  Writes p_j(x) of each test to dg[c].
+template <int TDT, int BT>
+__device__ int mss_node(const Params& P, int b, int cur, float s, float m, double z, float* dg, float* wpw,
+                        FinShared& sh, MssState& st) {
+    constexpr int CH = chunk_elems<TDT>();
+    const int tid = threadIdx.x, N = P.N;
+    const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
+    const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * N + cur) * P.dpstride;
+    st = MssState{0.0, 1.0, 1.0, 0, false};
+    for (int c = cur + 1; c < N; ++c) {
+        if (sh.par[c] != cur) continue;
+        if (tid == 0) {
+            const int x = sh.tok[c];
+            const double qx = (double)__ldg(reinterpret_cast<const float*>(drow) + x);
+            int verdict = -1;                         // -1 invalid, 0 reject, 1 accept
+            if (qx >= 0.0 && qx <= 3.4028234663852886e38) {
+                const double p = fmax(0.0, prob_d(ld_elem<TDT>(row, x), s, m, z) - st.c * qx) / st.D;
+                if (dg) dg[c] = (float)p;
+                const double ratio = qx > 0.0 ? p / qx : INFINITY;
+                verdict = ((double)P.coins[(size_t)b * N + c] <= ratio) ? 1 : 0;
+            }
+            sh.ivals[1] = verdict;
+        }
+        __syncthreads();
+        const int verdict = sh.ivals[1];
+        __syncthreads();
+        if (verdict < 0) return -2;
+        if (verdict > 0) return c;
+        const double cn = st.c + st.D;
+        WMss<TDT> wf{row, drow, s, m, (float)(1.0 / z), (float)cn, P.V};
+        const double F = row_chunk_masses<CH, BT>(wf, P.nch, wpw, sh);
+        if (!(F <= 1.7976931348623157e308)) return -2;          // inf or NaN
+        st.have_M = F > 0.0;
+        if (st.have_M) {                                        // else p stays (rounding only)
+            st.S = F / st.D;
+            st.c = cn;
+            st.D = F;
+            ++st.steps;
+        }
+    }
+    return -1;
+}
+
+// The last token of a multi-step sampling walk that stopped at node cur: drawn
+// with final_u from the current p (the row statistics when no residual step
+// was taken, else the chunk masses of max(0, p_0 - c q) and one chunk rescan).
+template <int TDT, int BT>
+__device__ int mss_draw(const Params& P, int b, int cur, float s, float m, double z, float* wpw, FinShared& sh,
+                        const MssState& st) {
+    constexpr int CH = chunk_elems<TDT>();
+    const int nch = P.nch;
+    const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
+    const float u = P.final_u[b];
+    int y = -1;
+    if (st.steps > 0) {
+        const char* drow = reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * P.N + cur) * P.dpstride;
+        WMss<TDT> wf{row, drow, s, m, (float)(1.0 / z), (float)st.c, P.V};
+        if (!st.have_M) row_chunk_masses<CH, BT>(wf, nch, wpw, sh);
+        double tot = 0.0;
+        for (int c = 0; c < nch; ++c) tot += sh.M[c];
+        if (tot > 0.0) y = draw_from_chunks<CH, BT>(wf, nch, P.V, (double)u * tot, u, sh);
+    }
+    if (y < 0) {
+        const float2* stt = P.stats + ((size_t)b * P.R + cur) * nch * SPC;
+        double Su;
+        y = sample_target_row<TDT, BT>(row, P.V, nch, stt, s, m, u, nullptr, 0, sh, &Su);
+    }
+    return y;
+}
+
+// Tree verification with a draft distribution, one CTA per sequence: combine
+// every node's statistics, validate, then walk with mss_node and draw with
+// mss_draw.
+template <int TDT, int BT>
+__device__ void finalize_mss(const Params& P, int b, FinShared& sh, const float2* blk, float* wpw) {
+    const int tid = threadIdx.x;
+    const int N = P.N, V = P.V, W = P.max_depth + 1;
+    combine_softmax_rows<BT>(P, blk, N, sh);
+    for (int n = tid; n < N; n += BT) {
+        sh.par[n] = P.parents[(size_t)b * N + n];
+        sh.tok[n] = P.tokens[(size_t)b * N + n];
+    }
+    __syncthreads();
+    int ok = tree_valid<BT>(P, N, V, P.max_depth, sh);
+    const float T = P.temperature[b];
+    if (tid == 0) {
+        ok &= temperature_ok(T);
+        for (int r = 0; r < N; ++r) ok &= !sh.bad[r];
+        sh.ivals[0] = ok;
+    }
+    __syncthreads();
+    ok = sh.ivals[0];
+    int32_t* ai = P.out_accept_index + (size_t)b * W;
+    int32_t* ot = P.out_tokens + (size_t)b * W;
+    float* dg = P.diag ? P.diag + (size_t)b * (N + 1) : nullptr;
+    if (dg) for (int i = tid; i <= N; i += BT) dg[i] = nanf_();
+    __syncthreads();
+    const float s = ok ? scale_of(T) : 0.f;
+    int cur = 0, k = 0;
+    MssState st{0.0, 1.0, 1.0, 0, false};
+    if (ok) {
+        if (tid == 0) ai[0] = 0;
+        for (;;) {
+            const int next = mss_node<TDT, BT>(P, b, cur, s, sh.m[cur], sh.z[cur], dg, wpw, sh, st);
+            if (next == -2) ok = 0;
+            if (next < 0) break;
+            if (tid == 0) {
+                ot[k] = sh.tok[next];
+                ai[k + 1] = next;
+            }
+            ++k;
+            cur = next;
+        }
+    }
+    if (!ok) {
+        for (int i = tid; i < W; i += BT) { ai[i] = -1; ot[i] = -1; }
+        __syncthreads();
+        if (dg) for (int i = tid; i <= N; i += BT) dg[i] = nanf_();
+        if (tid == 0) { P.out_num_accepted[b] = -1; flag_input_error(P); }
+        return;
+    }
+    const int y = mss_draw<TDT, BT>(P, b, cur, s, sh.m[cur], sh.z[cur], wpw, sh, st);
+    if (tid == 0) {
+        ot[k] = y;
+        for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+        P.out_num_accepted[b] = k;
+        if (dg) dg[N] = (float)st.S;
+    }
+}
+
 // ----------------------------------------------------------------------------- kernels
 
 // Row statistics (the streaming kernel).  The B*R*nch work items (sequence-
@@ -1338,39 +1613,6 @@ __global__ void __launch_bounds__(NT, STATS_CTAS_PER_SM) k_stats(const Params P)
             if (++r == P.R) { r = 0; ++b; }
         }
     }
-}
-
-// Locate the chunk holding t among the chunk masses sh.M[0..nch) (skipping
-// empty chunks) and rescan it; retries past chunks whose rescan finds no
-// positive weight (possible only through rounding).  Returns -1 if none.
-template <int CH, int BT, class WF>
-__device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u, FinShared& sh) {
-    const int tid = threadIdx.x;
-    int y = -1;
-    for (int attempt = 0; attempt < nch && y < 0; ++attempt) {
-        if (tid == 0) {
-            double C = 0.0, before = 0.0;
-            int cs = -1;
-            for (int cc = 0; cc < nch; ++cc) {
-                if (sh.M[cc] <= 0.0) continue;
-                if (t < C + sh.M[cc]) { cs = cc; before = C; break; }
-                C += sh.M[cc];
-            }
-            if (cs < 0)
-                for (int cc = nch - 1; cc >= 0; --cc)
-                    if (sh.M[cc] > 0.0) { cs = cc; before = C - sh.M[cc]; break; }
-            sh.ivals[2] = cs;
-            sh.dvals[1] = before;
-        }
-        __syncthreads();
-        const int cs = sh.ivals[2];
-        if (cs < 0) break;
-        double tot;
-        y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
-        if (y < 0 && tid == 0) sh.M[cs] = 0.0;
-        __syncthreads();
-    }
-    return y;
 }
 
 // Chain finalisation, grid = B * nsl: CTA (b, slice) recomputes sequence b's
@@ -1687,7 +1929,8 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     pdl_wait();
     const float2* blk = stage_stats(P, blockIdx.x, P.N, dyn, P.stage_cap, &sbar);
     if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
-    else finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
+    else if constexpr (MODE == MODE_SAMPLE) finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
+    else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
 
 // ============================================================================= lazy (row-on-demand) verification
@@ -1987,6 +2230,100 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
     P.lz_seq[b] = L;
 }
 
+// Lazy multi-step sampling walk, one CTA per active sequence at this level:
+// level 0 validates the tree and the temperature; the current node's row is
+// combined from its statistics; mss_node tests its children.  An accepted
+// child moves the sequence to the next level; otherwise the last token is
+// drawn here (mss_draw) and the sequence is done.
+template <int TDT>
+__global__ void __launch_bounds__(SEQ_BT) k_lz_decide_mss(const Params P) {
+    __shared__ FinShared sh;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    pdl_trigger();
+    pdl_wait();
+    if ((int)blockIdx.x >= lz_count_of(P)) return;
+    const int b = lz_seq_of(P, blockIdx.x);
+    const int tid = threadIdx.x, N = P.N, W = P.max_depth + 1, level = P.level;
+    int32_t* ai = P.out_accept_index + (size_t)b * W;
+    int32_t* ot = P.out_tokens + (size_t)b * W;
+    float* dg = P.diag ? P.diag + (size_t)b * (N + 1) : nullptr;
+    float* wpw = reinterpret_cast<float*>(dyn);
+    for (int n = tid; n < N; n += SEQ_BT) {
+        sh.par[n] = P.parents[(size_t)b * N + n];
+        sh.tok[n] = P.tokens[(size_t)b * N + n];
+    }
+    __syncthreads();
+    LazySeq L;
+    int ok = 1;
+    if (level == 0) {
+        ok = tree_valid<SEQ_BT>(P, N, P.V, P.max_depth, sh);
+        const float T = P.temperature[b];
+        ok &= temperature_ok(T);
+        L.cur = 0; L.k = 0; L.nrej = 0; L.pad = 0;
+        L.s = ok ? scale_of(T) : 0.f;
+        L.mq = 0.f; L.zq = 0.0;
+        if (ok) {
+            if (tid == 0) ai[0] = 0;
+            if (dg) for (int i = tid; i <= N; i += SEQ_BT) dg[i] = nanf_();
+            __syncthreads();
+        }
+    } else {
+        L = P.lz_seq[b];
+    }
+    if (ok) {
+        if (tid < 32) {
+            const int E = P.nch * SPC;
+            float m;
+            double z;
+            const bool bad = warp_combine(P.stats + ((size_t)b * P.R + L.cur) * E, E, m, z);
+            if (tid == 0) { sh.m[0] = m; sh.z[0] = z; sh.ivals[0] = !bad; }
+        }
+        __syncthreads();
+        ok = sh.ivals[0];
+        __syncthreads();
+    }
+    if (ok) {
+        L.m = sh.m[0];
+        L.z = sh.z[0];
+        MssState st;
+        const int next = mss_node<TDT, SEQ_BT>(P, b, L.cur, L.s, L.m, L.z, dg, wpw, sh, st);
+        if (next == -2) {
+            ok = 0;
+        } else if (next >= 0) {
+            if (tid == 0) {
+                ot[L.k] = sh.tok[next];
+                ai[L.k + 1] = next;
+                L.cur = next;
+                L.k += 1;
+                L.state = LZ_ACTIVE;
+                lz_push(P, b);
+                P.lz_seq[b] = L;
+            }
+        } else {
+            const int y = mss_draw<TDT, SEQ_BT>(P, b, L.cur, L.s, L.m, L.z, wpw, sh, st);
+            if (tid == 0) {
+                ot[L.k] = y;
+                for (int i = L.k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+                P.out_num_accepted[b] = L.k;
+                if (dg) dg[N] = (float)st.S;
+                L.state = LZ_DONE;
+                P.lz_seq[b] = L;
+            }
+        }
+    }
+    if (!ok) {
+        for (int i = tid; i < W; i += SEQ_BT) { ai[i] = -1; ot[i] = -1; }
+        __syncthreads();
+        if (dg) for (int i = tid; i <= N; i += SEQ_BT) dg[i] = nanf_();
+        if (tid == 0) {
+            P.out_num_accepted[b] = -1;
+            flag_input_error(P);
+            L.state = LZ_INVALID;
+            P.lz_seq[b] = L;
+        }
+    }
+}
+
 // Last token of a lazy target-only tree walk, one CTA per sequence (those
 // left in LZ_DRAW): tree_final_draw at the node where the walk stopped, with
 // the rejected children's tokens it kept.
@@ -2243,18 +2580,28 @@ spec_status launch_chain(Params P, cudaStream_t st) {
 
 template <int MODE, int TDT>
 spec_status launch_tree(Params P, cudaStream_t st) {
-    spec_status s = launch_stats<MODE, TDT, TDT>(P, st);
+    // the multi-step sampling walk uses the same softmax statistics as target-only sampling
+    spec_status s = launch_stats<MODE == MODE_MSS ? MODE_SAMPLE : MODE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
     static const bool big = allow_stage(k_tree_final<MODE, TDT>);
     P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
-    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st, "k_tree_final");
+    size_t smem = P.stage_cap;
+    if (MODE == MODE_MSS) {
+        // per-warp chunk sums of the residual passes after the statistics stage
+        const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+        P.stage_cap = stats_stage_bytes(P, P.N, (big ? STAGE_STATS_MAX : 48 * 1024 - 1024) - wpw);
+        P.stage_off = (P.stage_cap + 15) & ~15;
+        smem = P.stage_off + wpw;
+    }
+    return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, SEQ_BT, smem, P, st, "k_tree_final");
 }
 
 // One level of the lazy walk: the statistics kernel (the first one as an
 // ordinary launch, so the walk starts after all earlier work on the stream),
 // then the decision kernel (none after the chain's bonus row).
 template <class KS, class KD>
-spec_status launch_level(KS ks, unsigned sgrid, KD kd, unsigned dgrid, Params& P, int level, cudaStream_t st) {
+spec_status launch_level(KS ks, unsigned sgrid, KD kd, unsigned dgrid, Params& P, int level, cudaStream_t st,
+                         unsigned dblock = NT, size_t dsmem = 0) {
     P.level = level;
     spec_status s;
     if (level == 0) {
@@ -2264,7 +2611,7 @@ spec_status launch_level(KS ks, unsigned sgrid, KD kd, unsigned dgrid, Params& P
         s = launch_dependent(ks, sgrid, NT, 0, P, st, "k_lz_stats");
     }
     if (s != SPEC_OK || kd == nullptr) return s;
-    return launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
+    return launch_dependent(kd, dgrid, dblock, dsmem, P, st, "k_lz_decide");
 }
 
 template <int TDT, int DDT, int DK>
@@ -2284,6 +2631,22 @@ spec_status launch_chain_lazy(Params P, cudaStream_t st) {
     if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
         return fail(SPEC_ERR_CUDA, "profile event");
     return s;
+}
+
+template <int TDT>
+spec_status launch_mss_lazy(Params P, cudaStream_t st) {
+    auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
+    auto kd = k_lz_decide_mss<TDT>;
+    static const int occ = blocks_per_sm(ks);
+    const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    for (int level = 0; level <= P.max_depth; ++level) {
+        spec_status s = launch_level(ks, sgrid, kd, (unsigned)P.B, P, level, st, SEQ_BT, wpw);
+        if (s != SPEC_OK) return s;
+    }
+    if (g_prof_stop && record(g_prof_stop, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    return SPEC_OK;
 }
 
 template <int MODE, int TDT>
@@ -2314,7 +2677,7 @@ size_t spec_workspace_bytes(int entry, int B, int rows, int V) {
     if (B < 0 || V < 1 || V > SPEC_MAX_V) return 0;
     if (entry == SPEC_ENTRY_CHAIN) {
         if (rows < 1 || rows > SPEC_MAX_GAMMA) return 0;
-    } else if (entry == SPEC_ENTRY_TREE_GREEDY || entry == SPEC_ENTRY_TREE_SAMPLE) {
+    } else if (entry == SPEC_ENTRY_TREE_GREEDY || entry == SPEC_ENTRY_TREE_SAMPLE || entry == SPEC_ENTRY_TREE_MSS) {
         if (rows < 1 || rows > SPEC_MAX_NODES) return 0;
     } else {
         return 0;
@@ -2502,6 +2865,38 @@ static spec_status sample_entry(bool lazy, int B, int N, int V, int max_depth,
     return launch_tree<MODE_SAMPLE, SPEC_F32>(P, st);
 }
 
+static spec_status mss_entry(bool lazy, int B, int N, int V, int max_depth,
+                             const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                             const int32_t* tokens, const int32_t* parents,
+                             const float* temperature, const float* coins, const float* final_u,
+                             const float* draft_probs, int64_t dp_row_stride,
+                             int32_t* out_accept_index, int32_t* out_tokens,
+                             int32_t* out_num_accepted, float* diag,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    Params P{};
+    spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
+                                out_accept_index, out_tokens, out_num_accepted);
+    if (s != SPEC_OK || B == 0) return s;
+    if (!temperature || !coins || !final_u) return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    s = check_rows("draft_probs", draft_probs, SPEC_F32, dp_row_stride, V);
+    if (s != SPEC_OK) return s;
+    const Layout L = make_layout(SPEC_ENTRY_TREE_MSS, B, N, V);
+    s = check_ws(workspace, workspace_bytes, L);
+    if (s != SPEC_OK) return s;
+    bind_ws(P, workspace, L);
+    P.temperature = temperature; P.coins = coins; P.final_u = final_u;
+    P.draft_probs = draft_probs; P.dpstride = dp_row_stride * 4;
+    P.diag = diag;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (lazy) {
+        if (tdt == SPEC_BF16) return launch_mss_lazy<SPEC_BF16>(P, st);
+        return launch_mss_lazy<SPEC_F32>(P, st);
+    }
+    if (tdt == SPEC_BF16) return launch_tree<MODE_MSS, SPEC_BF16>(P, st);
+    return launch_tree<MODE_MSS, SPEC_F32>(P, st);
+}
+
 #define SPEC_CHAIN_ARGS_DECL                                                                         \
     int B, int gamma, int V, const void* target_logits, spec_dtype tdt, int64_t t_row_stride,      \
         const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,               \
@@ -2540,6 +2935,21 @@ spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry
 spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(true, SPEC_GREEDY_ARGS); }
 spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(false, SPEC_SAMPLE_ARGS); }
 spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(true, SPEC_SAMPLE_ARGS); }
+
+#define SPEC_MSS_ARGS_DECL                                                                           \
+    int B, int N, int V, int max_depth, const void* target_logits, spec_dtype tdt,                 \
+        int64_t t_row_stride, const int32_t* tokens, const int32_t* parents,                       \
+        const float* temperature, const float* coins, const float* final_u,                        \
+        const float* draft_probs, int64_t dp_row_stride, int32_t* out_accept_index,                \
+        int32_t* out_tokens, int32_t* out_num_accepted, float* diag, void* workspace,              \
+        size_t workspace_bytes, void* stream
+#define SPEC_MSS_ARGS                                                                                \
+    B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature, coins,      \
+        final_u, draft_probs, dp_row_stride, out_accept_index, out_tokens, out_num_accepted, diag,  \
+        workspace, workspace_bytes, stream
+
+spec_status spec_verify_tree_mss(SPEC_MSS_ARGS_DECL) { return mss_entry(false, SPEC_MSS_ARGS); }
+spec_status spec_verify_tree_mss_lazy(SPEC_MSS_ARGS_DECL) { return mss_entry(true, SPEC_MSS_ARGS); }
 
 }  // extern "C"
 

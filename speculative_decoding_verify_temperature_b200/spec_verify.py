@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libspecverify.so")
 SPEC_OK, SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA = 0, 1, 2, 3
 SPEC_ERR_DEVICE_INPUT, SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE = 4, 5, 6
 SPEC_F32, SPEC_BF16 = 0, 1
-SPEC_ENTRY_CHAIN, SPEC_ENTRY_TREE_GREEDY, SPEC_ENTRY_TREE_SAMPLE = 0, 1, 2
+SPEC_ENTRY_CHAIN, SPEC_ENTRY_TREE_GREEDY, SPEC_ENTRY_TREE_SAMPLE, SPEC_ENTRY_TREE_MSS = 0, 1, 2, 3
 
 _lib = None
 
@@ -55,6 +55,10 @@ def lib():
             f.restype = i32
             f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                           f32, f32, P, P, P, P, P, sz, P]
+        for name in ("spec_verify_tree_mss", "spec_verify_tree_mss_lazy"):
+            f = getattr(L, name)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64, P, P, P, P, P, sz, P]
         L.spec_workspace_bytes.restype = sz
         L.spec_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.spec_workspace_init.restype = i32
@@ -259,3 +263,38 @@ def spec_verify_tree_sample_lazy(*args, **kw):
     """Row-on-demand target-only tree sampling: the arguments and results of
     ``spec_verify_tree_sample``; ``diag`` holds NaN for children of unvisited nodes."""
     return spec_verify_tree_sample(*args, _name="spec_verify_tree_sample_lazy", **kw)
+
+
+def spec_verify_tree_mss(target, tokens, parents, temperature, coins, final_u, max_depth: int, draft_probs, *,
+                         V: int | None = None, out_accept_index=None, out_tokens=None, out_num_accepted=None,
+                         diag=None, workspace=None, stream=None, _name: str = "spec_verify_tree_mss"):
+    """Tree verification with a draft distribution (multi-step speculative sampling).
+    ``coins`` ``[B, N]`` holds the uniform of each child's test; ``draft_probs`` f32
+    ``[B, N, S]`` row n is the distribution node n's children were drawn from.
+    Returns ``(accept_index, tokens, num_accepted)``."""
+    B, N, S = target.shape
+    V = S if V is None else int(V)
+    dev = target.device
+    W = max_depth + 1
+    if out_accept_index is None:
+        out_accept_index = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_tokens is None:
+        out_tokens = torch.empty((B, W), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    if draft_probs.dtype != torch.float32:
+        raise TypeError("draft_probs must be float32")
+    ws = _ws(workspace, SPEC_ENTRY_TREE_MSS, B, N, V, dev, stream)
+    st = getattr(lib(), _name)(
+        B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens), _p(parents),
+        _p(temperature), _p(coins), _p(final_u), _p(draft_probs), _rows(draft_probs, "draft_probs"),
+        _p(out_accept_index), _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(),
+        _stream(stream))
+    _check(st, _name)
+    return out_accept_index, out_tokens, out_num_accepted
+
+
+def spec_verify_tree_mss_lazy(*args, **kw):
+    """Row-on-demand multi-step speculative sampling: the arguments and results of
+    ``spec_verify_tree_mss``, reading only the rows of the visited nodes."""
+    return spec_verify_tree_mss(*args, _name="spec_verify_tree_mss_lazy", **kw)

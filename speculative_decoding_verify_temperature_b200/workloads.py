@@ -356,6 +356,61 @@ def tree_sample_inputs(B: int, V: int, *, seed: int, device="cpu", parents_fn=No
     return TreeInputs(target, tokens, parents, temp, coins, final_u, md, V, dp)
 
 
+def tree_mss_inputs(B: int, V: int, *, seed: int, device="cpu", parents_fn=None,
+                    level_sizes=(4, 8, 8, 6, 5), max_children: int = 4,
+                    target_sigma: float = 3.0, zipf: bool = True, temperature: float = 0.8,
+                    draft_noise: float = 1.0, target_dtype=torch.bfloat16,
+                    stride: int | None = None, max_depth: int | None = None) -> TreeInputs:
+    """Inputs of tree verification with a draft distribution: logits
+    N(0, sigma^2) [+ log-Zipf bias]; the draft distribution of every node is
+    q_n = softmax((logits_n + N(0, draft_noise^2)) / T) in f32 (a drafter that
+    samples at the target's temperature), and the children of node n carry
+    tokens drawn independently from q_n, with replacement (duplicate siblings
+    possible), as multi-step speculative sampling assumes."""
+    g = make_gen(seed, device)
+    gc = make_gen(seed ^ 0x7EE, "cpu")
+    par = [parents_fn(gc) if parents_fn else level_tree(level_sizes, max_children, gc) for _ in range(B)]
+    N = len(par[0])
+    assert all(len(p) == N for p in par)
+    md = max(tree_depth(p) for p in par) if max_depth is None else max_depth
+    lg = torch.randn((B, N, V), generator=g, device=device, dtype=torch.float32) * target_sigma
+    if zipf:
+        lg += zipf_bias(V, g, device).view(1, 1, V)
+    target = padded((B, N), V, stride, target_dtype, device)
+    target[:, :, :V] = lg.to(target_dtype)
+    del lg
+    dp = padded((B, N), V, -(-V // 4) * 4, torch.float32, device)        # 16-byte aligned f32 rows
+    step = max(1, (1 << 26) // max(1, N * V))
+    for b0 in range(0, B, step):
+        b1 = min(B, b0 + step)
+        noisy = target[b0:b1, :, :V].to(torch.float32) + draft_noise * torch.randn(
+            (b1 - b0, N, V), generator=g, device=device, dtype=torch.float32)
+        dp[b0:b1, :, :V] = torch.softmax(noisy / temperature, dim=-1)
+        del noisy
+    parents = torch.tensor(par, dtype=torch.int32, device=device)
+    tokens = torch.zeros((B, N), dtype=torch.int32, device=device)
+    for b in range(B):
+        children = {}
+        for n in range(1, N):
+            children.setdefault(par[b][n], []).append(n)
+        for n, ch in children.items():
+            draw = torch.multinomial(dp[b, n, :V], len(ch), replacement=True, generator=g)
+            tokens[b, ch] = draw.to(torch.int32)
+    temp = torch.full((B,), float(temperature), dtype=torch.float32, device=device)
+    coins = uniforms((B, N), g, device)
+    final_u = uniforms((B,), g, device)
+    return TreeInputs(target, tokens, parents, temp, coins, final_u, md, V, dp)
+
+
+def tree_config5(rnd: int = 0, device="cpu") -> TreeInputs:
+    """Tree verification with a draft distribution (multi-step speculative
+    sampling): the tree and target of the B=128, 32-node, V=151936 workload
+    (bf16 logits N(0, 3^2) + log-Zipf(1.1), T = 0.8) plus f32 draft
+    distributions softmax((logits + N(0, 1)) / T) per node, children drawn from
+    them."""
+    return tree_mss_inputs(128, 151936, seed=round_seed(5, rnd), device=device)
+
+
 def tree_config2(rnd: int = 0, device="cpu") -> TreeInputs:
     """Greedy tree: B=32, 64 nodes (root + levels 8,11,11,11,11,11; at most 8
     children), V=128256, bf16 logits N(0, 3^2), draft token = parent argmax
@@ -376,6 +431,7 @@ WORKLOADS = {
     2: "greedy tree B=32 N=64 V=128256 bf16",
     3: "target-only tree B=128 N=32 V=151936 bf16, T=0.8, draft_probs NULL",
     4: "chain B=512 gamma=7 V=129280 bf16 target + f32 draft probs, T=1",
+    5: "multi-step speculative sampling tree B=128 N=32 V=151936 bf16 + f32 draft distributions, T=0.8",
 }
 
 
@@ -392,6 +448,8 @@ def algorithmic_bytes(workload_id: int) -> int:
         return 128 * 32 * 151936 * 2
     if workload_id == 4:
         return 512 * 8 * 129280 * 2
+    if workload_id == 5:
+        return 128 * 32 * 151936 * 2
     raise ValueError(workload_id)
 
 

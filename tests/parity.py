@@ -148,6 +148,50 @@ def compare_tree(g, o, rows=None, sample=False):
     return int(flags.sum()), int(bad.sum()), dict(bad_rows=np.nonzero(bad)[0][:10].tolist())
 
 
+# ----------------------------------------------------------------------------- trees with a draft distribution
+
+def oracle_mss(inp, rows=None, nthreads=0):
+    sel = _sel(inp.target, rows)
+    return oracle.tree_mss(to_np(inp.target[sel]), to_np(inp.tokens[sel]), to_np(inp.parents[sel]),
+                           to_np(inp.temperature[sel]), to_np(inp.coins[sel]), to_np(inp.final_u[sel]),
+                           inp.max_depth, to_np(inp.draft_probs[sel]), V=inp.V, nthreads=nthreads)
+
+
+def gpu_mss(inp, workspace=None, lazy=False):
+    B, N = inp.B, inp.N
+    diag = torch.full((B, N + 1), -7.0, device=inp.target.device)
+    ai, ot, na = _fn("spec_verify_tree_mss", lazy)(inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins,
+                                         inp.final_u, inp.max_depth, inp.draft_probs, V=inp.V, diag=diag,
+                                         workspace=workspace)
+    torch.cuda.synchronize()
+    d = diag.cpu().numpy().astype(np.float64)
+    return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy(),
+                ptest=d[:, :N], S=d[:, N])
+
+
+def compare_mss(g, o, rows=None):
+    """Walk outputs bit-exact except on oracle-flagged near-ties; p(x) at every test
+    within RTOL (and NaN exactly where the oracle tested nothing); the final
+    residual mass within RTOL on matching, unflagged sequences."""
+    sel = _rows_np(rows)
+    gk, gt, ga = g["num_accepted"][sel], g["tokens"][sel], g["accept_index"][sel]
+    flags = (o["dmargin"] < TIE_TOL) | (o["cmargin"] < TIE_TOL)
+    same = (gk == o["num_accepted"]) & (gt == o["tokens"]).all(axis=1) & (ga == o["accept_index"]).all(axis=1)
+    bad = ~same & ~flags
+    valid = o["num_accepted"] >= 0
+    ok_rows = valid & same & ~flags
+    gp = g["ptest"][sel]
+    if ok_rows.any():
+        tested = ~np.isnan(o["ptest"][ok_rows])
+        assert (np.isnan(gp[ok_rows]) == ~tested).all(), "tested children differ"
+        np.testing.assert_allclose(gp[ok_rows][tested], o["ptest"][ok_rows][tested], rtol=RTOL, atol=1e-12)
+        np.testing.assert_allclose(g["S"][sel][ok_rows], o["S"][ok_rows], rtol=RTOL, atol=1e-12)
+    inval = ~valid
+    assert (gk[inval] == -1).all() and (gt[inval] == -1).all()
+    assert np.isnan(gp[inval]).all()
+    return int(flags.sum()), int(bad.sum()), dict(bad_rows=np.nonzero(bad)[0][:10].tolist())
+
+
 # ----------------------------------------------------------------------------- runners with the oracle's signature
 
 def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, coins, final_u, V=None,
@@ -226,3 +270,26 @@ def _pad_rows(x: torch.Tensor) -> torch.Tensor:
     out = torch.zeros((B, R, S), dtype=x.dtype, device=x.device)
     out[:, :, :V] = x
     return out
+
+
+def gpu_tree_mss_runner(target, tokens, parents, temperature, coins, final_u, max_depth, draft_probs, V=None,
+                        nthreads=0, lazy=False):
+    """``oracle.tree_mss``'s signature, executed by the CUDA library."""
+    spec_verify_tree_mss = _fn("spec_verify_tree_mss", lazy)
+    dev = torch.device("cuda")
+
+    def t(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    B, N, S = target.shape
+    V = S if V is None else V
+    ai, ot, na = spec_verify_tree_mss(_pad_rows(t(target)), t(np.asarray(tokens, np.int32)),
+                                         t(np.asarray(parents, np.int32)),
+                                         t(np.asarray(temperature, np.float32).reshape(B)),
+                                         t(np.asarray(coins, np.float32)),
+                                         t(np.asarray(final_u, np.float32).reshape(B)), max_depth,
+                                         _pad_rows(t(np.asarray(draft_probs, np.float32))), V=V)
+    return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy())
