@@ -58,6 +58,11 @@ def lib():
         L.oracle_tree_sample.restype = None
         L.oracle_tree_sample.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                                          f32, f32, P, P, P, P, P, P, P, i32]
+        L.oracle_chain_filtered.restype = None
+        L.oracle_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
+                                            P, P, P, P, P, P, P, P, P, P, P, P, P, P, i32]
+        L.oracle_filter_row.restype = i32
+        L.oracle_filter_row.argtypes = [P, i32, i32, f64, i32, f64, P, P]
         L.oracle_tree_mss.restype = None
         L.oracle_tree_mss.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                                       P, P, P, P, P, P, P, i32]
@@ -94,10 +99,11 @@ def _ptr(a):
 
 
 def chain(target, draft, draft_is_probs, draft_tokens, temperature, coins, final_u, V=None,
-          nthreads: int = 0) -> dict:
+          nthreads: int = 0, top_k=None, top_p=None) -> dict:
     """Chain verify (acceptance rules 1-3).  ``target`` is ``[B, gamma+1, stride]``,
     ``draft`` ``[B, gamma, dstride]`` (logits, or f32 probabilities when
-    ``draft_is_probs``)."""
+    ``draft_is_probs``).  With ``top_k`` / ``top_p`` (per sequence, ``[B]``) the
+    target rows and draft-logit rows are top-k / top-p filtered first."""
     target = _c(target)
     draft = _c(draft)
     B, R, ts = target.shape
@@ -121,14 +127,39 @@ def chain(target, draft, draft_is_probs, draft_tokens, temperature, coins, final
     )
     if B == 0:
         return out
-    lib().oracle_chain(B, gamma, V, _ptr(target), _dtype_code(target), ts,
-                       _ptr(draft), F32 if draft_is_probs else _dtype_code(draft),
-                       int(bool(draft_is_probs)), ds,
-                       _ptr(draft_tokens), _ptr(temperature), _ptr(coins), _ptr(final_u),
-                       _ptr(out["tokens"]), _ptr(out["num_accepted"]), _ptr(out["px"]),
-                       _ptr(out["qx"]), _ptr(out["S"]), _ptr(out["dmargin"]),
-                       _ptr(out["cmargin"]), int(nthreads))
+    if top_k is None and top_p is None:
+        lib().oracle_chain(B, gamma, V, _ptr(target), _dtype_code(target), ts,
+                           _ptr(draft), F32 if draft_is_probs else _dtype_code(draft),
+                           int(bool(draft_is_probs)), ds,
+                           _ptr(draft_tokens), _ptr(temperature), _ptr(coins), _ptr(final_u),
+                           _ptr(out["tokens"]), _ptr(out["num_accepted"]), _ptr(out["px"]),
+                           _ptr(out["qx"]), _ptr(out["S"]), _ptr(out["dmargin"]),
+                           _ptr(out["cmargin"]), int(nthreads))
+        return out
+    tk = _c(np.zeros(B, np.int32) if top_k is None else top_k, np.int32).reshape(B)
+    tp = _c(np.ones(B, np.float32) if top_p is None else top_p, np.float32).reshape(B)
+    out["fmargin"] = np.empty(B, np.float64)
+    lib().oracle_chain_filtered(B, gamma, V, _ptr(target), _dtype_code(target), ts,
+                                _ptr(draft), F32 if draft_is_probs else _dtype_code(draft),
+                                int(bool(draft_is_probs)), ds,
+                                _ptr(draft_tokens), _ptr(temperature), _ptr(coins), _ptr(final_u),
+                                _ptr(tk), _ptr(tp),
+                                _ptr(out["tokens"]), _ptr(out["num_accepted"]), _ptr(out["px"]),
+                                _ptr(out["qx"]), _ptr(out["S"]), _ptr(out["dmargin"]),
+                                _ptr(out["cmargin"]), _ptr(out["fmargin"]), int(nthreads))
     return out
+
+
+def filter_row(row: np.ndarray, T: float, top_k: int, top_p: float, V=None):
+    """The oracle's top-k / top-p filtered temperature softmax of one row:
+    ``(p, margin)``, or ``None`` for an invalid row or filter."""
+    row = _c(row)
+    V = row.shape[-1] if V is None else int(V)
+    p = np.empty(V, np.float64)
+    m = np.empty(1, np.float64)
+    r = lib().oracle_filter_row(_ptr(row), _dtype_code(row), V, float(np.float32(T)), int(top_k), float(top_p),
+                                _ptr(p), _ptr(m))
+    return None if r else (p, float(m[0]))
 
 
 def tree_greedy(target, tokens, parents, max_depth: int, V=None, nthreads: int = 0) -> dict:

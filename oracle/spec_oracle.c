@@ -132,6 +132,81 @@ static void fill_i32(int32_t* a, int n, int32_t v) { for (int i = 0; i < n; ++i)
 static int temperature_ok(double T) { return T >= 0x1p-126 && T <= 0x1.fffffep127; }
 
 /*
+ * Top-k / top-p filtering of one temperature-softmax row.  The pages name
+ * top-k and top-p next to temperature as the sampling strategies a verify
+ * step must stay unbiased under ([kevins] "draft / verify / accept",
+ * greedy vs sampling paragraph; "production limits": a wider top-p lowers
+ * acceptance) without defining them; the textbook definitions, in the order
+ * temperature -> top-k -> top-p:
+ *   top-k (0 < top_k < V): keep the tokens whose logit is >= the top_k-th
+ *     largest logit (every token tied with it is kept);
+ *   top-p (0 < top_p < 1): within the top-k set, with the distribution
+ *     renormalised on it, keep the smallest set of whole groups of equal
+ *     logits, taken from the largest down, whose mass reaches top_p;
+ *   the kept tokens' probabilities are renormalised, the rest are 0.
+ * p holds softmax(row / T) on entry and the filtered distribution on exit.
+ * *margin receives |cumulative mass - top_p| at the two masses around the
+ * top-p crossing (relative to the renormalised distribution; +inf when
+ * top-p is off).  Returns 0, or -1 for an out-of-range top_k or top_p.
+ */
+typedef struct { double v; int j; } vj_t;
+static int cmp_vj_desc(const void* a, const void* b) {
+    const vj_t* x = (const vj_t*)a;
+    const vj_t* y = (const vj_t*)b;
+    if (x->v > y->v) return -1;
+    if (x->v < y->v) return 1;
+    return x->j - y->j;
+}
+static int filter_probs(const void* row, int dtype, int V, double* p, int top_k, double top_p, vj_t* sorted,
+                        double* margin) {
+    *margin = INFINITY;
+    if (top_k < 0 || !(top_p > 0.0 && top_p <= 1.0)) return -1;
+    if ((top_k == 0 || top_k >= V) && top_p == 1.0) return 0;
+    for (int j = 0; j < V; ++j) {
+        sorted[j].v = widen(row, dtype, j);
+        sorted[j].j = j;
+    }
+    qsort(sorted, (size_t)V, sizeof(vj_t), cmp_vj_desc);
+    /* top-k: every token whose logit is >= the top_k-th largest */
+    int nA = V;
+    if (top_k > 0 && top_k < V) {
+        int kk = (g_mutation == 16) ? top_k - 1 : top_k;          /* keeps one group too few */
+        if (kk < 1) kk = 1;
+        const double th = sorted[kk - 1].v;
+        nA = kk;
+        while (nA < V && sorted[nA].v >= th) ++nA;
+    }
+    double ZA = 0.0;
+    for (int i = 0; i < nA; ++i) ZA += p[sorted[i].j];
+    /* top-p: whole groups of equal logits from the top until the mass reaches top_p */
+    int nB = nA;
+    if (top_p < 1.0) {
+        double cum = 0.0;
+        int i = 0;
+        while (i < nA) {
+            int e = i;
+            double g = 0.0;
+            while (e < nA && sorted[e].v == sorted[i].v) g += p[sorted[e++].j];
+            const double before = cum;
+            cum += g / ZA;
+            if (cum >= top_p) {
+                const double m1 = fabs(before - top_p), m2 = fabs(cum - top_p);
+                *margin = m1 < m2 ? m1 : m2;
+                nB = (g_mutation == 17 && i > 0) ? i : e;           /* drops the crossing group */
+                break;
+            }
+            i = e;
+        }
+    }
+    double ZB = 0.0;
+    for (int i = 0; i < nB; ++i) ZB += p[sorted[i].j];
+    for (int i = 0; i < nB; ++i) sorted[i].v = p[sorted[i].j];   /* the kept probabilities */
+    for (int j = 0; j < V; ++j) p[j] = 0.0;
+    for (int i = 0; i < nB; ++i) p[sorted[i].j] = sorted[i].v / ZB;  /* ZB > 0: the maximum is kept */
+    return 0;
+}
+
+/*
  * Chain verify, one call = one round for B independent sequences.
  *
  * [origins] "Speculative Decoding: sampling can be lossless", acceptance
@@ -154,14 +229,16 @@ static int temperature_ok(double T) { return T >= 0x1p-126 && T <= 0x1.fffffep12
  * out_dmargin[b] = min over the evaluated decisions of |coin - ratio|;
  * out_cmargin[b] = inverse-CDF margin.
  */
-void oracle_chain(int B, int gamma, int V,
-                  const void* target, int tdt, int64_t t_row_stride,
-                  const void* draft, int ddt, int draft_is_probs, int64_t d_row_stride,
-                  const int32_t* draft_tokens, const float* temperature,
-                  const float* coins, const float* final_u,
-                  int32_t* out_tokens, int32_t* out_num_accepted,
-                  double* out_px, double* out_qx, double* out_S,
-                  double* out_dmargin, double* out_cmargin, int nthreads) {
+static void chain_impl(int B, int gamma, int V,
+                       const void* target, int tdt, int64_t t_row_stride,
+                       const void* draft, int ddt, int draft_is_probs, int64_t d_row_stride,
+                       const int32_t* draft_tokens, const float* temperature,
+                       const float* coins, const float* final_u,
+                       const int32_t* top_k, const float* top_p,
+                       int32_t* out_tokens, int32_t* out_num_accepted,
+                       double* out_px, double* out_qx, double* out_S,
+                       double* out_dmargin, double* out_cmargin, double* out_fmargin, int nthreads) {
+    const int filtered = top_k != NULL || top_p != NULL;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel
@@ -170,6 +247,7 @@ void oracle_chain(int B, int gamma, int V,
         double* P = (double*)malloc(sizeof(double) * (size_t)V * (size_t)(gamma + 1));
         double* Q = (double*)malloc(sizeof(double) * (size_t)V * (size_t)gamma);
         double* w = (double*)malloc(sizeof(double) * (size_t)V);
+        vj_t* sorted = filtered ? (vj_t*)malloc(sizeof(vj_t) * (size_t)V) : NULL;
 #ifdef _OPENMP
 #pragma omp for schedule(dynamic, 1)
 #endif
@@ -178,10 +256,17 @@ void oracle_chain(int B, int gamma, int V,
             const int32_t* x = draft_tokens + (int64_t)b * gamma;
             double T = (double)temperature[b];
             int bad = !temperature_ok(T);
+            const int K = top_k ? top_k[b] : 0;
+            const double Pp = top_p ? (double)top_p[b] : 1.0;
+            double fmargin = INFINITY, fm;
             for (int i = 0; i <= gamma && !bad; ++i) {
                 const char* row = (const char*)target +
                     ((int64_t)b * (gamma + 1) + i) * t_row_stride * (tdt == OR_F32 ? 4 : 2);
                 if (softmax_T(row, tdt, V, T, P + (int64_t)i * V)) bad = 1;
+                else if (filtered) {
+                    if (filter_probs(row, tdt, V, P + (int64_t)i * V, K, Pp, sorted, &fm)) bad = 1;
+                    if (fm < fmargin) fmargin = fm;
+                }
             }
             for (int i = 0; i < gamma && !bad; ++i) {
                 const char* row = (const char*)draft +
@@ -191,10 +276,14 @@ void oracle_chain(int B, int gamma, int V,
                     for (int j = 0; j < V; ++j) q[j] = widen(row, OR_F32, j);
                 } else if (softmax_T(row, ddt, V, g_mutation == 12 ? 1.0 : T, q)) {
                     bad = 1;
+                } else if (filtered && g_mutation != 18) {              /* 18: draft left unfiltered */
+                    if (filter_probs(row, ddt, V, q, K, Pp, sorted, &fm)) bad = 1;
+                    if (fm < fmargin) fmargin = fm;
                 }
                 if (x[i] < 0 || x[i] >= V) bad = 1;
                 else if (isnan(q[x[i]]) || q[x[i]] < 0.0) bad = 1;
             }
+            if (out_fmargin) out_fmargin[b] = bad ? INFINITY : fmargin;
             if (bad) {
                 fill_i32(toks, gamma + 1, -1);
                 out_num_accepted[b] = -1;
@@ -260,7 +349,56 @@ void oracle_chain(int B, int gamma, int V,
         free(P);
         free(Q);
         free(w);
+        free(sorted);
     }
+}
+
+void oracle_chain(int B, int gamma, int V,
+                  const void* target, int tdt, int64_t t_row_stride,
+                  const void* draft, int ddt, int draft_is_probs, int64_t d_row_stride,
+                  const int32_t* draft_tokens, const float* temperature,
+                  const float* coins, const float* final_u,
+                  int32_t* out_tokens, int32_t* out_num_accepted,
+                  double* out_px, double* out_qx, double* out_S,
+                  double* out_dmargin, double* out_cmargin, int nthreads) {
+    chain_impl(B, gamma, V, target, tdt, t_row_stride, draft, ddt, draft_is_probs, d_row_stride,
+               draft_tokens, temperature, coins, final_u, NULL, NULL, out_tokens, out_num_accepted,
+               out_px, out_qx, out_S, out_dmargin, out_cmargin, NULL, nthreads);
+}
+
+/*
+ * Chain verify with top-k / top-p filtering (filter_probs) of every target
+ * row and, when the draft is given as logits, every draft row, with the
+ * sequence's top_k[b] (0 = off) and top_p[b] (1 = off); draft probabilities
+ * are used as given.  Rules 1-3 then run on the filtered distributions, so
+ * the emitted tokens follow the filtered target distribution.  top_k < 0 or
+ * top_p outside (0, 1] makes the sequence invalid.  out_fmargin[b] = the
+ * smallest top-p crossing margin over the sequence's rows.
+ */
+void oracle_chain_filtered(int B, int gamma, int V,
+                           const void* target, int tdt, int64_t t_row_stride,
+                           const void* draft, int ddt, int draft_is_probs, int64_t d_row_stride,
+                           const int32_t* draft_tokens, const float* temperature,
+                           const float* coins, const float* final_u,
+                           const int32_t* top_k, const float* top_p,
+                           int32_t* out_tokens, int32_t* out_num_accepted,
+                           double* out_px, double* out_qx, double* out_S,
+                           double* out_dmargin, double* out_cmargin, double* out_fmargin, int nthreads) {
+    chain_impl(B, gamma, V, target, tdt, t_row_stride, draft, ddt, draft_is_probs, d_row_stride,
+               draft_tokens, temperature, coins, final_u, top_k, top_p, out_tokens, out_num_accepted,
+               out_px, out_qx, out_S, out_dmargin, out_cmargin, out_fmargin, nthreads);
+}
+
+/* The filtered distribution of one row, as the verify above uses it (for the pins). */
+int oracle_filter_row(const void* row, int dtype, int V, double T, int top_k, double top_p, double* p,
+                      double* margin) {
+    if (softmax_T(row, dtype, V, T, p)) return -1;
+    vj_t* sorted = (vj_t*)malloc(sizeof(vj_t) * (size_t)V);
+    double m = INFINITY;
+    const int r = filter_probs(row, dtype, V, p, top_k, top_p, sorted, &m);
+    free(sorted);
+    if (margin) *margin = m;
+    return r;
 }
 
 /*

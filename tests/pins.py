@@ -523,6 +523,159 @@ def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3, r
     return _chisq(first, tab, V, K, pmin)
 
 
+# ----------------------------------------------------------------------------- top-k / top-p filtering
+
+def filter_definition(logits, T, top_k, top_p):
+    """Filtered distribution from the definitions in threshold form (independent of
+    the oracle's sort-and-accumulate): theta_k = the largest logit value t with
+    #{l >= t} >= top_k; theta_p = the largest value t >= theta_k whose set
+    {l >= t} carries, under softmax(l/T) renormalised on {l >= theta_k}, a mass
+    >= top_p; keep {l >= max(theta_k, theta_p)} and renormalise."""
+    l = np.asarray(logits, np.float64)
+    V = l.size
+    p = special.softmax(l / T)
+    vals = np.unique(l)[::-1]                                     # every distinct value, -inf included
+    th_k = -np.inf
+    if 0 < top_k < V:
+        th_k = max(t for t in vals if (l >= t).sum() >= top_k)
+    A = l >= th_k
+    pa = np.where(A, p, 0.0)
+    pa /= pa.sum()
+    th = th_k
+    if top_p < 1.0:
+        th = max(t for t in vals if t >= th_k and pa[l >= t].sum() >= top_p)
+    keep = l >= th
+    out = np.where(keep, p, 0.0)
+    return out / out.sum(), keep
+
+
+class FilteredModel:
+    """A ToyModel seen through top-k / top-p: p() and q() return the raw row given
+    to the verify step and the filtered distribution the drafts are drawn from
+    and the output must follow (draft probabilities are filtered by the caller
+    and handed over as they are)."""
+
+    def __init__(self, model: ToyModel, top_k: int, top_p: float):
+        self.m, self.top_k, self.top_p = model, top_k, top_p
+        self.V, self.T, self.draft_kind = model.V, model.T, model.draft_kind
+
+    def p(self, prefix):
+        logits, _ = self.m.p(prefix)
+        return logits, filter_definition(logits.astype(np.float64), self.T, self.top_k, self.top_p)[0]
+
+    def q(self, prefix):
+        row, probs = self.m.q(prefix)
+        if self.draft_kind == "probs":
+            f = filter_definition(np.log(np.maximum(probs, 1e-300)) + np.where(probs > 0, 0, -np.inf), 1.0,
+                                  self.top_k, self.top_p)[0]
+            return f.astype(np.float32), f.astype(np.float32).astype(np.float64)
+        return row, filter_definition(row.astype(np.float64), self.T, self.top_k, self.top_p)[0]
+
+
+def chain_filtered_bruteforce(V=4, gamma=2, K=2, seed=1, draft_kind="logits", T=1.0, top_k=3, top_p=0.8,
+                              tol=1e-12, runner=None) -> dict:
+    """Exact distribution of the first K tokens of repeated chain rounds under
+    top-k / top-p filtering against the filtered target's autoregressive
+    distribution (the rules keep whatever target distribution they are given)."""
+    model = FilteredModel(ToyModel(V, seed, draft_kind, T=T), top_k, top_p)
+    states = {(): 1.0}
+    dist = {}
+    fmin = np.inf
+    while states:
+        batch, owners = [], []
+        for prefix, w in states.items():
+            cs = _chain_cases(model, prefix, gamma)
+            batch += cs
+            owners += [(prefix, w)] * len(cs)
+        n = len(batch)
+        res = (runner or oracle.chain)(np.stack([c["target"] for c in batch]), np.stack([c["draft"] for c in batch]),
+                                       draft_kind == "probs", np.stack([c["x"] for c in batch]),
+                                       np.full(n, model.T, np.float32), np.stack([c["coins"] for c in batch]),
+                                       np.array([c["u"] for c in batch], np.float32),
+                                       top_k=np.full(n, top_k, np.int32), top_p=np.full(n, top_p, np.float32))
+        if "fmargin" in res:
+            fmin = min(fmin, float(res["fmargin"].min()))
+        nxt = {}
+        for i, (prefix, w) in enumerate(owners):
+            k = int(res["num_accepted"][i])
+            if k < 0:
+                return dict(ok=False, err=float("inf"), reason="flagged valid input")
+            h = prefix + tuple(int(t) for t in res["tokens"][i, :k + 1])
+            ww = w * batch[i]["weight"]
+            if len(h) >= K:
+                dist[h[:K]] = dist.get(h[:K], 0.0) + ww
+            else:
+                nxt[h] = nxt.get(h, 0.0) + ww
+        states = nxt
+    want = _product_distribution(model, K)
+    err = max(abs(dist.get(s, 0.0) - pv) for s, pv in want.items())
+    err = max(err, sum(v for s, v in dist.items() if s not in want))
+    return dict(ok=err < tol and fmin > 1e-9, err=err, fmargin=fmin)
+
+
+def filter_properties(trials=400, seed=3) -> dict:
+    """The oracle's filter against the defining properties on random rows (ties,
+    signed zeros, -inf entries, bf16 and f32): kept values dominate dropped
+    ones; top-k keeps >= top_k tokens with < top_k strictly above its smallest
+    kept value; top-p keeps whole groups of equal logits, reaches top_p and
+    would fall short without its smallest kept group; kept probabilities are
+    scipy's softmax on the kept set; off switches give scipy's softmax."""
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for t in range(trials):
+        V = int(rng.integers(1, 60))
+        kind = rng.integers(3)
+        if kind == 0:
+            l = rng.integers(-3, 4, V).astype(np.float32)            # many ties
+            l[rng.random(V) < 0.1] = -0.0
+        elif kind == 1:
+            l = rng.normal(0, 2, V).astype(np.float32)
+        else:
+            l = (rng.normal(0, 2, V).astype(np.float32).view(np.uint32) >> 16 << 16).view(np.float32)
+        if V > 2 and rng.random() < 0.2:
+            l[rng.integers(V)] = -np.inf
+        if not np.isfinite(l).any():
+            l[0] = 0.0
+        T = float(np.float32(rng.choice([0.5, 1.0, 1.7])))
+        K = int(rng.choice([0, 1, 2, 5, V, V + 3]))
+        P = float(np.float32(rng.choice([1.0, 0.3, 0.7, 0.95, 1e-6])))
+        row = l if rng.random() < 0.5 else (l.view(np.uint32) >> 16).astype(np.uint16)
+        lv = l if row.dtype == np.float32 else (row.astype(np.uint32) << 16).view(np.float32)
+        res = oracle.filter_row(row, T, K, P)
+        if res is None:
+            return dict(ok=False, trial=t, reason="valid filter rejected")
+        p, margin = res
+        lv64 = lv.astype(np.float64)
+        keep = p > 0
+        base = special.softmax(lv64 / T)
+        if (K == 0 or K >= V) and P >= 1.0:
+            worst = max(worst, float(np.abs(p - base).max()))
+            continue
+        if not keep.any() or (keep.any() and (~keep).any() and lv64[keep].min() < lv64[~keep].max()):
+            return dict(ok=False, trial=t, reason="a dropped value exceeds a kept one")
+        lo = lv64[keep].min()
+        if (~keep & (lv64 == lo)).any():
+            return dict(ok=False, trial=t, reason="a group of equal values was split")
+        if 0 < K < V:
+            if keep.sum() < K and P >= 1.0:
+                return dict(ok=False, trial=t, reason="top-k kept too few")
+            if (lv64 > lo).sum() >= K:
+                return dict(ok=False, trial=t, reason="top-k kept too many")
+        if P < 1.0:
+            A = lv64 >= (np.sort(lv64)[::-1][K - 1] if 0 < K < V else -np.inf)
+            pa = np.where(A, base, 0.0)
+            pa /= pa.sum()
+            if margin > 1e-9:
+                if pa[keep].sum() < P:
+                    return dict(ok=False, trial=t, reason="top-p mass short of top_p")
+                if pa[keep & (lv64 > lo)].sum() >= P:
+                    return dict(ok=False, trial=t, reason="top-p set not minimal")
+        want = np.where(keep, base, 0.0)
+        want /= want.sum()
+        worst = max(worst, float(np.abs(p - want).max()))
+    return dict(ok=worst < 1e-12, worst=worst)
+
+
 # ----------------------------------------------------------------------------- trees with a draft distribution (MSS)
 
 def _mss_cases(model: ToyModel, prefix, parents):

@@ -59,6 +59,64 @@ def test_tree_mss_bruteforce_lossless(parents, V, K, seed, T):
     assert r["ok"], r
 
 
+# ----------------------------------------------------------------------------- top-k / top-p
+
+def test_filter_properties():
+    """The oracle's top-k / top-p filter satisfies the defining properties on
+    random rows with ties, signed zeros and -inf entries."""
+    r = pins.filter_properties(trials=600)
+    assert r["ok"], r
+
+
+def test_filter_special_cases():
+    l = np.array([0.5, 2.0, -1.0, 1.5, 2.0, 0.0], np.float32)
+    base = special.softmax(l.astype(np.float64) / float(np.float32(0.8)))   # T is taken as its f32 value
+    p, m = oracle.filter_row(l, 0.8, 0, 1.0)
+    np.testing.assert_allclose(p, base, rtol=0, atol=1e-15)          # both off: the softmax
+    p, m = oracle.filter_row(l, 0.8, len(l) + 5, 1.0)
+    np.testing.assert_allclose(p, base, rtol=0, atol=1e-15)          # top_k >= V: off
+    p, m = oracle.filter_row(l, 0.8, 1, 1.0)
+    np.testing.assert_allclose(p, [0, 0.5, 0, 0, 0.5, 0], atol=1e-15)   # top-1 keeps both tied maxima
+    p, m = oracle.filter_row(l, 0.8, 0, 1e-6)
+    np.testing.assert_allclose(p, [0, 0.5, 0, 0, 0.5, 0], atol=1e-15)   # tiny top_p: the top group
+    p, m = oracle.filter_row(l, 0.8, 3, 1.0)                          # 2, 2, 1.5
+    want = np.where(l >= 1.5, base, 0)
+    np.testing.assert_allclose(p, want / want.sum(), atol=1e-15)
+    assert oracle.filter_row(l, 0.8, -1, 1.0) is None
+    assert oracle.filter_row(l, 0.8, 0, 0.0) is None
+    assert oracle.filter_row(l, 0.8, 0, 1.5) is None
+
+
+def test_chain_filter_off_is_plain_chain():
+    """top_k = 0 and top_p = 1 for every sequence: the filtered chain equals the
+    plain chain bit for bit."""
+    rng = np.random.default_rng(31)
+    B, gamma, V = 40, 3, 50
+    t = rng.normal(0, 2, (B, gamma + 1, V)).astype(np.float32)
+    d = rng.normal(0, 2, (B, gamma, V)).astype(np.float32)
+    x = rng.integers(0, V, (B, gamma)).astype(np.int32)
+    T = np.full(B, 0.9, np.float32)
+    c = rng.random((B, gamma)).astype(np.float32)
+    u = rng.random(B).astype(np.float32)
+    a = oracle.chain(t, d, False, x, T, c, u)
+    b = oracle.chain(t, d, False, x, T, c, u, top_k=np.zeros(B, np.int32), top_p=np.ones(B, np.float32))
+    for key in ("tokens", "num_accepted", "px", "qx", "S"):
+        np.testing.assert_array_equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),
+    dict(draft_kind="probs", seed=2, top_k=2, top_p=0.9, tol=1e-7),   # filtered q rounded to f32
+    dict(V=4, gamma=2, seed=5, T=0.7, top_k=0, top_p=0.61),
+    dict(V=5, gamma=1, seed=6, top_k=2, top_p=1.0),
+    dict(V=3, gamma=3, K=3, seed=8, top_k=2, top_p=0.77),
+])
+def test_chain_filtered_bruteforce_lossless(kw):
+    """The rules keep the (filtered) target distribution exactly."""
+    r = pins.chain_filtered_bruteforce(**kw)
+    assert r["ok"], r
+
+
 # ----------------------------------------------------------------------------- closed form
 
 @pytest.mark.parametrize("seed,kind", [(2, "probs"), (3, "logits"), (12, "probs")])
@@ -390,6 +448,9 @@ MUTATIONS = {
     14: ("MSS: every residual taken from the node's first p",
          lambda: pins.tree_mss_bruteforce(V=4, K=2, seed=3, parents=(-1, 0, 0, 0, 1, 1))),
     15: ("MSS: children tested with their parent's coin", lambda: pins.tree_mss_bruteforce()),
+    16: ("top-k keeps one group too few", lambda: pins.filter_properties()),
+    17: ("top-p drops the group that reaches top_p", lambda: pins.filter_properties()),
+    18: ("draft logits left unfiltered", lambda: pins.chain_filtered_bruteforce()),
 }
 
 
