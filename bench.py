@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -91,6 +91,8 @@ def make_inputs(wid: int, rnd: int, device, rank: int = 0):
         return wl.tree_config3(r, device)
     if wid == 5:
         return wl.tree_config5(r, device)
+    if wid == 6:
+        return wl.chain_config6(r, device)
     return wl.chain_config4(r, device)
 
 
@@ -105,7 +107,7 @@ def input_bytes(inp) -> int:
 def describe(wid: int, inp) -> dict:
     from speculative_decoding_verify_temperature_b200 import workloads as wl
     d = {"workload": wl.WORKLOADS[wid], "global_batch": inp.B}
-    if wid in (0, 1, 4):
+    if wid in (0, 1, 4, 6):
         d.update(gamma=inp.gamma, V=inp.V, target_dtype=str(inp.target.dtype).split(".")[-1],
                  draft="f32 probabilities" if inp.draft_is_probs else str(inp.draft.dtype).split(".")[-1] + " logits")
     else:
@@ -121,7 +123,7 @@ class Runner:
         import torch
         B = inp.B
         dev = inp.target.device
-        if wid in (0, 1, 4):
+        if wid in (0, 1, 4, 6):
             self.out = (torch.empty((B, inp.gamma + 1), dtype=torch.int32, device=dev),
                         torch.empty((B,), dtype=torch.int32, device=dev))
         else:
@@ -133,7 +135,11 @@ class Runner:
     def __call__(self):
         from speculative_decoding_verify_temperature_b200 import spec_verify as sv
         i = self.inp
-        if self.wid in (0, 1, 4):
+        if self.wid == 6:
+            sv.spec_verify_chain_filtered(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
+                                          i.meta["top_k"], i.meta["top_p"], draft_is_probs=i.draft_is_probs, V=i.V,
+                                          out_tokens=self.out[0], out_num_accepted=self.out[1], workspace=self.ws)
+        elif self.wid in (0, 1, 4):
             getattr(sv, "spec_verify_chain" + self.sfx)(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                  draft_is_probs=i.draft_is_probs, V=i.V, out_tokens=self.out[0],
                                  out_num_accepted=self.out[1], workspace=self.ws)
@@ -156,8 +162,9 @@ class Runner:
 
 
 def kernels_per_step(wid, inp) -> int:
-    """Launches per verify call: the row-statistics kernel and the finalize kernel."""
-    return 2
+    """Launches per verify call: the row-statistics kernel and the finalize kernel
+    (and the filter kernel between them for the filtered chain)."""
+    return 3 if wid == 6 else 2
 
 
 def lazy_kernels_per_step(wid, inp) -> int:
@@ -185,7 +192,7 @@ def lazy_bytes_read(wid, inp, num_accepted) -> int:
 def workspace_for(wid, inp):
     from speculative_decoding_verify_temperature_b200 import spec_verify as sv
     ws = sv.Workspace(inp.target.device)
-    if wid in (0, 1, 4):
+    if wid in (0, 1, 4, 6):
         return ws.get(sv.SPEC_ENTRY_CHAIN, inp.B, inp.gamma, inp.V)
     e = {2: sv.SPEC_ENTRY_TREE_GREEDY, 3: sv.SPEC_ENTRY_TREE_SAMPLE, 5: sv.SPEC_ENTRY_TREE_MSS}[wid]
     return ws.get(e, inp.B, inp.N, inp.V)
@@ -194,7 +201,7 @@ def workspace_for(wid, inp):
 def algorithmic_bytes(wid, inp) -> int:
     """Bytes of logits / probabilities the row kernel must read once per round."""
     b = inp.target[:, :, :inp.V].numel() * inp.target.element_size()
-    if wid in (0, 1):
+    if wid in (0, 1, 6):
         b += inp.draft[:, :, :inp.V].numel() * inp.draft.element_size()
     return b
 
@@ -275,11 +282,13 @@ def cpu_baseline(wid, inp, seconds, nthreads=None):
     # Copy the inputs to host once; the oracle reads the same bytes the GPU reads.
     n = 0
     fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain,
-          2: parity.oracle_greedy, 3: parity.oracle_sample, 5: parity.oracle_mss}[wid]
+          2: parity.oracle_greedy, 3: parity.oracle_sample, 5: parity.oracle_mss,
+          6: lambda i, r, nthreads: parity.oracle_chain_filtered(i, i.meta["top_k"], i.meta["top_p"], r,
+                                                                 nthreads=nthreads)}[wid]
     B = inp.B
     # Large workloads: a bounded sample of whole sequences per "round" of work,
     # scaled to full rounds below.
-    per = B if wid in (0, 1) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4}[wid]))
+    per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4}[wid]))
     rows = None if per == B else list(range(per))
     elapsed = 0.0
     while n == 0 or elapsed < seconds:
@@ -454,13 +463,14 @@ def main():
     acc = torch.cat(acc)
     mean_tau = float((acc + 1).mean())
     B = first.B
-    draft_per_round = B * (first.gamma if wid in (0, 1, 4) else first.N - 1)
+    draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6) else first.N - 1)
 
     # --- end to end through the binding with host buffers
     e2e = run_e2e(wid, first, ws, args.e2e_steps, dev)
 
     # --- the row-on-demand entry point on the same input sets
-    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 else None
+    # (the filtered chain has no row-on-demand variant)
+    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid != 6 else None
 
     cfg = describe(wid, first)
     cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",
@@ -534,11 +544,18 @@ def run_e2e(wid, inp, ws, steps, dev):
     pinned host memory, verifies, and copies the outputs back."""
     import torch
     host = {k: v.detach().cpu().pin_memory() for k, v in vars(inp).items() if isinstance(v, torch.Tensor)}
+    meta = getattr(inp, "meta", None) or {}
+    host.update({"meta." + k: v.detach().cpu().pin_memory() for k, v in meta.items() if isinstance(v, torch.Tensor)})
     dev_bufs = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     import copy
     dinp = copy.copy(inp)
+    if meta:
+        dinp.meta = dict(meta)
     for k, v in dev_bufs.items():
-        setattr(dinp, k, v)
+        if k.startswith("meta."):
+            dinp.meta[k[5:]] = v
+        else:
+            setattr(dinp, k, v)
     runner = Runner(wid, dinp, ws)
     out_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in runner.out]
     h2d = sum(v.numel() * v.element_size() for v in host.values())

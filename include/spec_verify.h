@@ -135,6 +135,47 @@ spec_status spec_verify_chain(int B, int gamma, int V,
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spec_verify_chain_filtered -- spec_verify_chain under top-k / top-p
+ * filtered temperature sampling.  [kevins] "draft / verify / accept" (real
+ * serving samples with temperature, top-p and top-k, and verify must stay
+ * unbiased under them) and "production limits" (a wider top-p lowers
+ * acceptance); the pages do not define the filters, so the textbook ones:
+ *   p'_i = softmax(target row i / T_b) restricted to the kept tokens and
+ *   renormalised, where the kept tokens are: top-k (0 < top_k[b] < V) the
+ *   tokens whose logit is >= the top_k-th largest logit (ties kept); then
+ *   top-p (0 < top_p[b] < 1) the smallest set of whole groups of equal
+ *   logits, from the largest down, whose share of the top-k set's mass
+ *   reaches top_p[b].
+ * Draft logits are filtered the same way (the drafter sampled from its own
+ * filtered distribution); draft probabilities are used as given.  Rules 1-3
+ * then run on p' and q' exactly as in spec_verify_chain, so the emitted
+ * tokens follow the filtered target distribution.
+ *
+ * Arguments as spec_verify_chain, plus:
+ * top_k          [B] int32, nullable (NULL or 0 = no top-k); < 0 makes the
+ *                sequence invalid.
+ * top_p          [B] f32, nullable (NULL or 1 = no top-p); outside (0, 1]
+ *                makes the sequence invalid.  At least one of the two must
+ *                be non-NULL.
+ * diag           p'_i(x_i), q'_i(x_i), then the final mass S as in
+ *                spec_verify_chain.
+ * workspace      >= spec_workspace_bytes(SPEC_ENTRY_CHAIN, B, gamma, V).
+ * Cost: per filtered row, one CTA walks the row 2-4 times (bf16; 4-8 for f32)
+ * to find its thresholds by radix descent (16-bit / 32-bit order keys, 8 bits
+ * per pass; counts for top-k, fixed-point masses in 2^-40 units for top-p),
+ * and the correction or bonus is drawn over the whole filtered row.
+ */
+spec_status spec_verify_chain_filtered(int B, int gamma, int V,
+                                       const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                       const void* draft, spec_dtype ddt, int draft_is_probs,
+                                       int64_t d_row_stride,
+                                       const int32_t* draft_tokens, const float* temperature,
+                                       const float* coins, const float* final_u,
+                                       const int32_t* top_k, const float* top_p,
+                                       int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_verify_tree_greedy -- greedy verify of a draft token tree.
  * [origins] "In SGLang" (greedy goes through verify_tree_greedy) and
  * "Blockwise Parallel Decoding" (verify keeps the longest prefix equal to

@@ -11,6 +11,7 @@ from .spec_verify import (  # noqa: F401
     spec_profile_events,
     spec_read_device_status,
     spec_verify_chain,
+    spec_verify_chain_filtered,
     spec_verify_chain_lazy,
     spec_verify_tree_greedy,
     spec_verify_tree_greedy_lazy,

@@ -105,6 +105,19 @@ struct Params {
     int* lz_list;                  // [2][B]            (active sequences of a level, ping-pong)
     unsigned* lz_count;            // [LZ_MAX_LEVELS + 1] (active count of each level; zero at rest)
     int level;
+    // top-k / top-p filtering (chain)
+    const int32_t* top_k;          // [B], nullable (0 = off)
+    const float* top_p;            // [B], nullable (1 = off)
+    struct FiltRec* filt;          // [B][R]            (per-row threshold and kept mass)
+};
+
+// Top-k / top-p filter of one row: keep logits >= theta; Z = the kept mass in
+// units of 2^(x - m) (the row's statistics units).  on = 0: no filter (theta
+// -inf, the statistics' Z applies); on = -1: invalid filter parameters.
+struct FiltRec {
+    float theta;
+    int on;
+    double Z;
 };
 
 // ----------------------------------------------------------------------------- small helpers
@@ -449,6 +462,7 @@ struct FinShared {
     double M[MAXCH];
     float wp[MAXCH][NWARP];
     uint32_t bitmap[(NT * VPT * 8) / 32];
+    float th[MAXR];
     int ivals[8];
     double dvals[4];
 };
@@ -985,7 +999,7 @@ __device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) 
 // valid, sh.ivals[1] = k, sh.dvals[0] = s.  When `write` is set it also writes
 // the accepted tokens, the -1 tail (position k excluded), num_accepted and
 // the p/q diagnostics, and flags invalid sequences.  Ends with __syncthreads.
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool FILT = false>
 __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, const ChainPrefetch& f) {
     const int tid = threadIdx.x;
     const int gamma = P.gamma, W = gamma + 1;
@@ -999,11 +1013,13 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
         double p = 0.0, q = 0.0;
         if (ok && tok) {
             p = prob_d(f.l, s, sh.m[tid], sh.z[tid]);
+            if (FILT && f.l < sh.th[tid]) p = 0.0;               // filtered out
             if constexpr (DK == DK_PROBS) {
                 q = (double)f.d;
                 ok &= (q >= 0.0 && q <= 3.0e38);
             } else {
                 q = prob_d(f.d, s, sh.m[gamma + 1 + tid], sh.z[gamma + 1 + tid]);
+                if (FILT && f.d < sh.th[gamma + 1 + tid]) q = 0.0;
             }
         }
         sh.pch[tid] = p;
@@ -1933,6 +1949,482 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
 
+// ============================================================================= top-k / top-p filtering
+//
+// The filtered target distribution keeps the logits >= theta: theta_k = the
+// top_k-th largest logit (ties kept), then, within that set, theta_p = the
+// largest logit whose set {l >= theta_p} carries a top_p share of the set's
+// mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds come from a radix
+// descent over order-preserving keys of the logits (16 bits for bf16, 32 for
+// f32, -0 folded onto +0), 8 bits per pass over the row: counts for top-k,
+// fixed-point masses (2^-40 units, integer atomics, so the sums do not depend
+// on the order of the additions) for top-p and Z'.
+
+constexpr int FILT_BT = 1024;
+constexpr double FIX_ONE = 1099511627776.0;      // 2^40
+
+template <int DT> __device__ __forceinline__ uint32_t order_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;                                   // -0 sorts with +0
+    const uint32_t k = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return DT == SPEC_BF16 ? (k >> 16) : k;
+}
+template <int DT> __device__ __forceinline__ float key_value(uint32_t k) {
+    if constexpr (DT == SPEC_BF16) {
+        const uint32_t b = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+        return __uint_as_float(b << 16);
+    } else {
+        return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+    }
+}
+
+// Digits of the order keys, most significant first: 12 + 4 bits for bf16,
+// 12 + 12 + 8 for f32.  The wide first digit (sign, exponent and the top
+// mantissa bits) spreads a row's values over many buckets, so the shared
+// histogram updates rarely collide.
+template <int DT> struct FiltDigits;
+template <> struct FiltDigits<SPEC_BF16> {
+    static constexpr int NL = 2;
+    __host__ __device__ static constexpr int width(int l) { return l == 0 ? 12 : 4; }
+    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 4 : 0; }
+};
+template <> struct FiltDigits<SPEC_F32> {
+    static constexpr int NL = 3;
+    __host__ __device__ static constexpr int width(int l) { return l == 2 ? 8 : 12; }
+    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 20 : (l == 1 ? 8 : 0); }
+};
+// Shared bytes of the per-level histograms (counts u32 + masses u64 per bucket).
+template <int DT> __host__ __device__ constexpr size_t filt_hist_bytes() {
+    size_t n = 0;
+    for (int l = 0; l < FiltDigits<DT>::NL; ++l) n += ((size_t)1 << FiltDigits<DT>::width(l)) * 12;
+    return n;
+}
+
+struct FiltShared {
+    unsigned long long red[FILT_BT / 32];
+    unsigned long long at, above;
+    int sel;
+};
+
+// Level l's histograms inside the dynamic area.
+template <int DT> struct FiltHist {
+    unsigned char* base;
+    __device__ unsigned long long* mass(int l) const {
+        size_t off = 0;
+        for (int k = 0; k < l; ++k) off += ((size_t)1 << FiltDigits<DT>::width(k)) * 12;
+        return reinterpret_cast<unsigned long long*>(base + off);
+    }
+    __device__ unsigned* cnt(int l) const {
+        return reinterpret_cast<unsigned*>(mass(l) + ((size_t)1 << FiltDigits<DT>::width(l)));
+    }
+};
+
+// One pass over a row: histograms of digit `level` (counts and fixed-point
+// masses of 2^(x s - m)) of the keys whose higher digits equal `prefix` (all
+// keys at level 0).  Integer atomics: the sums do not depend on their order.
+template <int DT>
+__device__ void filt_pass(const char* row, int V, float s, float m, int level, uint32_t prefix, const FiltHist<DT>& h) {
+    using D = FiltDigits<DT>;
+    constexpr int EPV = Tr<DT>::EPV;
+    const int nb = 1 << D::width(level), sh = D::shift(level);
+    const int psh = sh + D::width(level);
+    unsigned* cnt = h.cnt(level);
+    unsigned long long* mass = h.mass(level);
+    for (int d = threadIdx.x; d < nb; d += FILT_BT) { cnt[d] = 0u; mass[d] = 0ull; }
+    __syncthreads();
+    const int nv = (V + EPV - 1) / EPV;
+    for (int vi = threadIdx.x; vi < nv; vi += FILT_BT) {
+        const uint4 v = ld_vec<DT>(row, (int64_t)vi * EPV, V);
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) {
+            if (vi * EPV + i >= V) break;
+            const float x = vec_elem<DT>(v, i);
+            const uint32_t key = order_key<DT>(x);
+            if (level > 0 && (key >> psh) != prefix) continue;
+            const uint32_t d = (key >> sh) & (uint32_t)(nb - 1);
+            atomicAdd(&cnt[d], 1u);
+            atomicAdd(&mass[d], (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE));
+        }
+    }
+    __syncthreads();
+}
+
+// Scan buckets [dlo, nb) from the top for the first bucket d whose running
+// total base + (buckets above d) + w[d] reaches target; every thread owns a
+// run of buckets, a block-wide u64 scan gives each run its start.  Returns d,
+// or -1 when the range never reaches the target.  fs.above = base + the
+// buckets of the range strictly above d (the whole range when -1), fs.at =
+// fs.above + w[d].  All threads call it.
+template <class T>
+__device__ int filt_scan(const T* w, int nb, int dlo, unsigned long long base, double target, FiltShared& fs) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = nb - dlo;
+    const int per = (n + FILT_BT - 1) / FILT_BT;
+    const int hi = nb - tid * per, lo = max(dlo, hi - per);     // buckets [lo, hi), this thread's run
+    unsigned long long own = 0ull;
+    for (int d = hi - 1; d >= lo; --d) own += (unsigned long long)w[d];
+    unsigned long long inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long v = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += v;
+    }
+    if (lane == 31) fs.red[warp] = inc;
+    if (tid == 0) fs.sel = -1;
+    __syncthreads();
+    unsigned long long excl = base;
+    for (int k = 0; k < warp; ++k) excl += fs.red[k];
+    excl += inc - own;
+    if (hi > lo && (double)excl < target && (double)(excl + own) >= target) {
+        unsigned long long cum = excl;
+        for (int d = hi - 1; d >= lo; --d) {
+            if ((double)(cum + (unsigned long long)w[d]) >= target) {
+                fs.sel = d;
+                fs.above = cum;
+                fs.at = cum + (unsigned long long)w[d];
+                break;
+            }
+            cum += (unsigned long long)w[d];
+        }
+    }
+    __syncthreads();
+    const int d = fs.sel;
+    if (d < 0 && tid == 0) {
+        unsigned long long t = base;
+        for (int k = 0; k < FILT_BT / 32; ++k) t += fs.red[k];
+        fs.above = t;
+        fs.at = t;
+    }
+    __syncthreads();
+    return d;
+}
+
+// Threshold and kept mass of one row (one CTA).
+//  top-k: walk the digits of the top_k-th largest key (filt_scan over the
+//    counts, one pass per digit); every pass keeps the masses, so the mass of
+//    the kept set {key >= path} is the masses strictly above the path at
+//    each level plus the path's key.
+//  top-p: within the kept set, scan from the top -- the buckets strictly
+//    above the path at each level, then the path's key -- for the bucket
+//    where the mass reaches top_p * (kept mass); a whole key ends the search,
+//    another bucket is refined digit by digit with more passes (every key in
+//    it lies above the top-k key).
+//  top-p alone: one pass of the first digit over every key; the crossing
+//    bucket is refined the same way.
+template <int DT>
+__device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
+                              const FiltHist<DT>& h) {
+    using D = FiltDigits<DT>;
+    constexpr int NL = D::NL;
+    FiltRec r{-INFINITY, 0, 0.0};
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    if (!use_k && !use_p) return r;
+    int path[NL];
+    uint32_t prefix = 0;
+    unsigned long long cabove = 0ull, mabove = 0ull;           // counts / masses strictly above the path
+    const int nl = use_k ? NL : 1;
+    for (int level = 0; level < nl; ++level) {
+        filt_pass<DT>(row, V, s, m, level, prefix, h);
+        const int nb = 1 << D::width(level);
+        if (use_k) {
+            path[level] = filt_scan(h.cnt(level), nb, 0, cabove, (double)K, fs);
+            cabove = fs.above;
+        } else {
+            path[level] = 0;                                   // top-p alone: every key is kept
+        }
+        filt_scan(h.mass(level), nb, path[level] + 1, 0ull, INFINITY, fs);   // masses above the path digit
+        mabove += fs.above;
+        prefix = (prefix << D::width(level)) | (uint32_t)path[level];
+    }
+    const unsigned long long mk = mabove + h.mass(nl - 1)[path[nl - 1]];
+    uint32_t key = prefix;
+    unsigned long long z = mk;
+    if (use_p) {
+        const double target = (double)Pp * (double)mk;
+        unsigned long long base = 0ull;
+        int cl = -1, cd = 0;
+        for (int l = 0; l < nl && cl < 0; ++l) {                // buckets strictly above the path digit
+            const int d = filt_scan(h.mass(l), 1 << D::width(l), path[l] + 1, base, target, fs);
+            if (d >= 0) { cl = l; cd = d; z = fs.at; }
+            base = fs.above;
+        }
+        if (cl < 0) {                                          // the path's own bucket
+            cl = nl - 1;
+            cd = path[nl - 1];
+            z = base + h.mass(cl)[cd];
+        }
+        uint32_t pre = 0;
+        for (int l = 0; l < cl; ++l) pre = (pre << D::width(l)) | (uint32_t)path[l];
+        pre = (pre << D::width(cl)) | (uint32_t)cd;
+        if (!(use_k && cl == NL - 1)) {                        // not a whole key: refine
+            for (int level = cl + 1; level < NL; ++level) {
+                filt_pass<DT>(row, V, s, m, level, pre, h);
+                int d = filt_scan(h.mass(level), 1 << D::width(level), 0, base, target, fs);
+                if (d < 0) d = 0;                              // rounding only
+                base = fs.above;
+                z = fs.at;
+                pre = (pre << D::width(level)) | (uint32_t)d;
+            }
+        }
+        key = pre;
+    }
+    r.theta = key_value<DT>(key);
+    r.on = 1;
+    r.Z = (double)z / FIX_ONE;
+    return r;
+}
+
+// bf16 rows: an exact histogram of the row's values (65536 order keys, two
+// 16-bit counters per 32-bit word, 132 KB of shared memory) from one pass;
+// every mass then follows exactly as count * fixed(2^(v s - m)) per value,
+// the same fixed-point numbers the radix path adds element by element.  One
+// spare word after every 32 puts the runs that the scans give consecutive
+// threads (32 words apart) in consecutive banks.
+constexpr size_t VH_WORDS = 32768 + 32768 / 32;
+constexpr size_t VH_BYTES = VH_WORDS * 4;
+
+__device__ __forceinline__ uint32_t vh_word(uint32_t k) {
+    const uint32_t i = k >> 1;
+    return i + (i >> 5);
+}
+__device__ __forceinline__ unsigned vh_count(const uint32_t* w, uint32_t k) {
+    return (w[vh_word(k)] >> ((k & 1u) * 16u)) & 0xFFFFu;
+}
+__device__ __forceinline__ unsigned long long vh_weight(const uint32_t* w, uint32_t k, bool mass, float s, float m) {
+    const unsigned c = vh_count(w, k);
+    if (!mass || c == 0u) return c;
+    return (unsigned long long)c *
+           (unsigned long long)(ex2(fmaf(key_value<SPEC_BF16>(k), s, -m)) * (float)FIX_ONE);
+}
+
+// The largest key t >= lo whose weight W(keys >= t) reaches target (counts or
+// masses); a negative target means -target times W(keys >= lo).  Returns -1
+// when the keys >= lo never reach it.  fs.at = W(keys >= t) (W(keys >= lo)
+// when -1); fs.above = W(keys >= lo).  Each thread owns a run of 65536 /
+// FILT_BT keys, a block-wide u64 scan orders the runs.  All threads call it.
+__device__ int vh_scan(const uint32_t* w, uint32_t lo, bool mass, float s, float m, double target, FiltShared& fs) {
+    constexpr int PER = 65536 / FILT_BT;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hi = 65536 - tid * PER, lt = max((int)lo, hi - PER);
+    unsigned long long own = 0ull;
+    for (int k = hi - 1; k >= lt; --k) own += vh_weight(w, (uint32_t)k, mass, s, m);
+    unsigned long long inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long v = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += v;
+    }
+    if (lane == 31) fs.red[warp] = inc;
+    if (tid == 0) fs.sel = -1;
+    __syncthreads();
+    unsigned long long excl = 0ull, total = 0ull;
+    for (int k = 0; k < FILT_BT / 32; ++k) {
+        if (k < warp) excl += fs.red[k];
+        total += fs.red[k];
+    }
+    excl += inc - own;
+    if (target < 0.0) target = -target * (double)total;
+    if (hi > lt && (double)excl < target && (double)(excl + own) >= target) {
+        unsigned long long cum = excl;
+        for (int k = hi - 1; k >= lt; --k) {
+            cum += vh_weight(w, (uint32_t)k, mass, s, m);
+            if ((double)cum >= target) { fs.sel = k; fs.at = cum; break; }
+        }
+    }
+    __syncthreads();
+    const int t = fs.sel;
+    if (tid == 0) {
+        fs.above = total;
+        if (t < 0) fs.at = total;
+    }
+    __syncthreads();
+    return t;
+}
+
+// Threshold and kept mass of a bf16 row from its value histogram.  Returns
+// false when a value occurs 65536 times or more (a 16-bit counter wrapped:
+// possible only for V > 65535); the caller then takes the radix path.
+__device__ bool filter_row_vh(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
+                              uint32_t* w, FiltRec* out) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < (int)VH_WORDS; i += FILT_BT) w[i] = 0u;
+    __syncthreads();
+    const int nv = (V + 7) / 8;
+    for (int vi = tid; vi < nv; vi += FILT_BT) {
+        const uint4 v = ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (vi * 8 + i >= V) break;
+            const uint32_t k = order_key<SPEC_BF16>(vec_elem<SPEC_BF16>(v, i));
+            atomicAdd(&w[vh_word(k)], 1u << ((k & 1u) * 16u));
+        }
+    }
+    __syncthreads();
+    if (V > 65535) {                                   // a wrapped counter loses 65535 from the total
+        vh_scan(w, 0u, false, s, m, INFINITY, fs);
+        if (fs.at != (unsigned long long)V) return false;
+    }
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    uint32_t t = 0u;
+    if (use_k) t = (uint32_t)vh_scan(w, 0u, false, s, m, (double)K, fs);
+    // one mass scan: the top-k set's (or the row's) mass, and where top_p of it is reached
+    const int tp = vh_scan(w, t, true, s, m, use_p ? -(double)Pp : INFINITY, fs);
+    unsigned long long z = fs.at;
+    if (use_p && tp >= 0) t = (uint32_t)tp;
+    out->theta = key_value<SPEC_BF16>(t);
+    out->on = 1;
+    out->Z = (double)z / FIX_ONE;
+    return true;
+}
+
+// Filter thresholds of every row of a chain round, one CTA per (sequence,
+// row): target rows 0..gamma, then the draft-logit rows.  Needs the rows'
+// maxima from the statistics (waits for them); the finalize kernel that
+// follows reads the records.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
+    __shared__ FiltShared fs;
+    __shared__ float msh;
+    __shared__ int bad;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    pdl_trigger();
+    pdl_wait();
+    const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
+    const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
+    FiltRec* out = P.filt + (size_t)b * P.R + r;
+    const int K = P.top_k ? P.top_k[b] : 0;
+    const float Pp = P.top_p ? P.top_p[b] : 1.f;
+    const float T = P.temperature[b];
+    if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
+        return;
+    }
+    if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const int E = P.nch * SPC;
+    if (threadIdx.x < 32) {
+        float m;
+        double z;
+        const bool bd = warp_combine(P.stats + ((size_t)b * P.R + r) * E, E, m, z);
+        if (threadIdx.x == 0) { msh = m; bad = bd; }
+    }
+    __syncthreads();
+    if (bad) {                                   // the decision marks the sequence invalid
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const float s = scale_of(T), m = msh;
+    FiltRec rec;
+    if (r <= P.gamma) {
+        const char* row = P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride;
+        if (TDT != SPEC_BF16 || !filter_row_vh(row, P.V, s, m, K, Pp, fs, reinterpret_cast<uint32_t*>(dyn), &rec))
+            rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
+    } else {
+        const char* row = P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
+        if (DDT != SPEC_BF16 || !filter_row_vh(row, P.V, s, m, K, Pp, fs, reinterpret_cast<uint32_t*>(dyn), &rec))
+            rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
+    }
+    if (threadIdx.x == 0) *out = rec;
+}
+
+// max(0, p' - q') of a filtered target row and a filtered draft row (QK =
+// DK_LOGITS), a draft probability row (DK_PROBS), or no draft (DK_NONE: p').
+template <int TDT, int QDT, int QK> struct WFilt {
+    const char* trow; const char* drow; float s, mp, izp, thp, mq, izq, thq; int V;
+    struct Raw { Raw8<TDT> t; Raw8<QDT> d; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const {
+        load_raw8<TDT>(trow, e0, r.t);
+        if constexpr (QK != DK_NONE) load_raw8<QDT>(drow, e0, r.d);
+    }
+    __device__ __forceinline__ void finish(const float (&x)[8], const float (&d)[8], float (&w)[8]) const {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float p = x[i] >= thp ? ex2(fmaf(x[i], s, -mp)) * izp : 0.f;
+            float q = 0.f;
+            if constexpr (QK == DK_PROBS) q = d[i];
+            if constexpr (QK == DK_LOGITS) q = d[i] >= thq ? ex2(fmaf(d[i], s, -mq)) * izq : 0.f;
+            w[i] = fmaxf(0.f, p - q);
+        }
+    }
+    __device__ __forceinline__ void weights(int64_t, const Raw& r, float (&w)[8]) const {
+        float x[8], d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        raw8_f32<TDT>(r.t, x);
+        if constexpr (QK != DK_NONE) raw8_f32<QDT>(r.d, d);
+        finish(x, d, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        ld8<TDT>(trow, e0, V, -INFINITY, x);
+        if constexpr (QK == DK_PROBS) ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        if constexpr (QK == DK_LOGITS) ld8<QDT>(drow, e0, V, -INFINITY, d);
+        finish(x, d, w);
+    }
+};
+
+// Inverse-CDF draw over a whole row with the weights wf (chunk masses, one
+// chunk rescanned); *S receives the total.  -1 when the total is not positive.
+template <int CH, int BT, class WF>
+__device__ int draw_row(const WF& wf, int nch, float u, float* wpw, FinShared& sh, double* S) {
+    *S = row_chunk_masses<CH, BT>(wf, nch, wpw, sh);
+    return *S > 0.0 ? draw_from_chunks<CH, BT>(wf, nch, wf.V, (double)u * *S, u, sh) : -1;
+}
+
+// Filtered chain finalisation, one CTA per sequence: the decision of
+// chain_decide on the filtered distributions (p' and q' from each row's
+// statistics, threshold and kept mass), then the correction from
+// max(0, p'_k - q'_k) or the bonus from p'_gamma over the whole row.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
+    __shared__ FinShared sh;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    constexpr int CH = chunk_elems<TDT>();
+    constexpr int QDT = DK == DK_PROBS ? SPEC_F32 : DDT;
+    const int tid = threadIdx.x, b = blockIdx.x;
+    const int gamma = P.gamma, V = P.V;
+    float* wpw = reinterpret_cast<float*>(dyn);
+    const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
+    pdl_wait();
+    combine_softmax_rows<SEQ_BT>(P, P.stats + (size_t)b * P.R * P.nch * SPC, P.R, sh);
+    __syncthreads();
+    const int rows = (DK == DK_LOGITS) ? 2 * gamma + 1 : gamma + 1;
+    for (int r = tid; r < rows; r += SEQ_BT) {
+        const FiltRec f = P.filt[(size_t)b * P.R + r];
+        sh.th[r] = f.theta;
+        if (f.on > 0) sh.z[r] = f.Z;
+        if (f.on < 0) sh.bad[r] = 1;                 // invalid top_k / top_p
+    }
+    __syncthreads();
+    chain_decide<TDT, DDT, DK, true>(P, b, sh, true, pf);
+    const int ok = sh.ivals[0], k = sh.ivals[1];
+    const float s = (float)sh.dvals[0];
+    if (!ok) return;
+    const float u = P.final_u[b];
+    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
+    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]), thp = sh.th[k];
+    double S;
+    int y = -1;
+    if (k < gamma) {
+        const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
+        const int rq = gamma + 1 + k;
+        WFilt<TDT, QDT, DK> wf{trow, drow, s, mp, izp, thp, DK == DK_LOGITS ? sh.m[rq] : 0.f,
+                               DK == DK_LOGITS ? (float)(1.0 / sh.z[rq]) : 0.f,
+                               DK == DK_LOGITS ? sh.th[rq] : -INFINITY, V};
+        y = draw_row<CH, SEQ_BT>(wf, P.nch, u, wpw, sh, &S);
+    }
+    if (y < 0) {                                     // bonus, or an empty residual (rounding only)
+        WFilt<TDT, QDT, DK_NONE> wp{trow, nullptr, s, mp, izp, thp, 0.f, 0.f, -INFINITY, V};
+        double S0;
+        y = draw_row<CH, SEQ_BT>(wp, P.nch, u, wpw, sh, &S0);
+        if (k == gamma) S = 1.0;
+    }
+    if (tid == 0) {
+        P.out_tokens[(size_t)b * (gamma + 1) + k] = y;
+        if (P.diag) P.diag[(size_t)b * (2 * gamma + 1) + 2 * gamma] = (float)S;
+    }
+}
+
 // ============================================================================= lazy (row-on-demand) verification
 //
 // The verify rules need only some rows: the chain reads the target row (and
@@ -2379,7 +2871,7 @@ spec_status fail(spec_status st, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, total;
+    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, total;
     int rej_cap;
     int R, nch_max;
 };
@@ -2403,6 +2895,9 @@ Layout make_layout(int entry, int B, int rows, int V) {
     L.lz_rej = off; off = align256(off + sizeof(int) * (size_t)B * L.rej_cap);
     L.lz_list = off; off = align256(off + sizeof(int) * 2 * (size_t)B);
     L.lz_count = off; off = align256(off + sizeof(unsigned) * (LZ_MAX_LEVELS + 1));
+    // top-k / top-p filter records of the chain's rows
+    L.filt = off;
+    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(FiltRec) * (size_t)B * L.R);
     L.total = off;
     return L;
 }
@@ -2459,6 +2954,7 @@ void bind_ws(Params& P, void* ws, const Layout& L) {
     P.rej_cap = L.rej_cap;
     P.lz_list = reinterpret_cast<int*>(w + L.lz_list);
     P.lz_count = reinterpret_cast<unsigned*>(w + L.lz_count);
+    P.filt = reinterpret_cast<FiltRec*>(w + L.filt);
 }
 
 spec_status launched(const char* what) {
@@ -2568,6 +3064,26 @@ spec_status launch_chain_final(Params P, cudaStream_t st) {
     P.nsl = nsl < 1 ? 1 : (nsl > P.nch ? P.nch : nsl);
     return launch_dependent(k_chain_final<TDT, DDT, DK, LZ>, (unsigned)(P.B * P.nsl), NT, P.stage_cap, P, st,
                             "k_chain_final");
+}
+
+// Filtered chain: statistics, per-row filter thresholds, filtered finalisation.
+template <int TDT, int DDT, int DK>
+spec_status launch_chain_filtered(Params P, cudaStream_t st) {
+    spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
+    if (s != SPEC_OK) return s;
+    const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
+    constexpr size_t hr = filt_hist_bytes<TDT>() > filt_hist_bytes<DDT>() ? filt_hist_bytes<TDT>()
+                                                                            : filt_hist_bytes<DDT>();
+    constexpr size_t hist = (TDT == SPEC_BF16 || DDT == SPEC_BF16) && VH_BYTES > hr ? VH_BYTES : hr;
+    static const bool attr = cudaFuncSetAttribute(k_filter<TDT, DDT, DK>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) ==
+                             cudaSuccess;
+    if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
+    s = launch_dependent(k_filter<TDT, DDT, DK>, (unsigned)(P.B * rows), FILT_BT, hist, P, st, "k_filter");
+    if (s != SPEC_OK) return s;
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    return launch_dependent(k_chain_final_filt<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, wpw, P, st,
+                            "k_chain_final_filt");
 }
 
 template <int TDT, int DDT, int DK>
@@ -2727,14 +3243,15 @@ spec_status spec_profile_events(void* start_event, void* stop_event) {
 
 }  // extern "C"
 
-static spec_status chain_entry(bool lazy, int B, int gamma, int V,
+static spec_status chain_entry(int mode, int B, int gamma, int V,
                                const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
                                const void* draft, spec_dtype ddt, int draft_is_probs,
                                int64_t d_row_stride,
                                const int32_t* draft_tokens, const float* temperature,
                                const float* coins, const float* final_u,
                                int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               void* workspace, size_t workspace_bytes, void* stream,
+                               const int32_t* top_k = nullptr, const float* top_p = nullptr) {
     g_detail[0] = 0;
     if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
     if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
@@ -2762,11 +3279,14 @@ static spec_status chain_entry(bool lazy, int B, int gamma, int V,
     P.dstride = d_row_stride * (ddt == SPEC_F32 ? 4 : 2);
     P.draft_tokens = draft_tokens; P.temperature = temperature; P.coins = coins; P.final_u = final_u;
     P.out_tokens = out_tokens; P.out_num_accepted = out_num_accepted; P.diag = diag;
+    P.top_k = top_k; P.top_p = top_p;
     bind_ws(P, workspace, L);
     // The statistics of a row are laid out with the chain's full row count so
     // that draft rows keep their offsets for either draft kind.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-#define SPEC_CHAIN(T, D, K) return lazy ? launch_chain_lazy<T, D, K>(P, st) : launch_chain<T, D, K>(P, st)
+#define SPEC_CHAIN(T, D, K)                                                                          \
+    return mode == 1 ? launch_chain_lazy<T, D, K>(P, st)                                             \
+                     : (mode == 2 ? launch_chain_filtered<T, D, K>(P, st) : launch_chain<T, D, K>(P, st))
     if (draft_is_probs) {
         if (tdt == SPEC_BF16) SPEC_CHAIN(SPEC_BF16, SPEC_F32, DK_PROBS);
         SPEC_CHAIN(SPEC_F32, SPEC_F32, DK_PROBS);
@@ -2929,8 +3449,23 @@ static spec_status mss_entry(bool lazy, int B, int N, int V, int max_depth,
 
 extern "C" {
 
-spec_status spec_verify_chain(SPEC_CHAIN_ARGS_DECL) { return chain_entry(false, SPEC_CHAIN_ARGS); }
-spec_status spec_verify_chain_lazy(SPEC_CHAIN_ARGS_DECL) { return chain_entry(true, SPEC_CHAIN_ARGS); }
+spec_status spec_verify_chain(SPEC_CHAIN_ARGS_DECL) { return chain_entry(0, SPEC_CHAIN_ARGS); }
+spec_status spec_verify_chain_lazy(SPEC_CHAIN_ARGS_DECL) { return chain_entry(1, SPEC_CHAIN_ARGS); }
+
+spec_status spec_verify_chain_filtered(int B, int gamma, int V,
+                                       const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                       const void* draft, spec_dtype ddt, int draft_is_probs,
+                                       int64_t d_row_stride,
+                                       const int32_t* draft_tokens, const float* temperature,
+                                       const float* coins, const float* final_u,
+                                       const int32_t* top_k, const float* top_p,
+                                       int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+    if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
+    return chain_entry(2, B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                       d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens, out_num_accepted,
+                       diag, workspace, workspace_bytes, stream, top_k, top_p);
+}
 spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(false, SPEC_GREEDY_ARGS); }
 spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(true, SPEC_GREEDY_ARGS); }
 spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(false, SPEC_SAMPLE_ARGS); }

@@ -59,6 +59,9 @@ def lib():
             f = getattr(L, name)
             f.restype = i32
             f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64, P, P, P, P, P, sz, P]
+        L.spec_verify_chain_filtered.restype = i32
+        L.spec_verify_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
+                                                 P, P, P, P, P, P, P, P, P, P, sz, P]
         L.spec_workspace_bytes.restype = sz
         L.spec_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.spec_workspace_init.restype = i32
@@ -298,3 +301,33 @@ def spec_verify_tree_mss_lazy(*args, **kw):
     """Row-on-demand multi-step speculative sampling: the arguments and results of
     ``spec_verify_tree_mss``, reading only the rows of the visited nodes."""
     return spec_verify_tree_mss(*args, _name="spec_verify_tree_mss_lazy", **kw)
+
+
+def spec_verify_chain_filtered(target, draft, draft_tokens, temperature, coins, final_u, top_k=None, top_p=None, *,
+                               draft_is_probs: bool = False, V: int | None = None, out_tokens=None,
+                               out_num_accepted=None, diag=None, workspace=None, stream=None):
+    """Chain verify under top-k / top-p filtered temperature sampling; ``top_k`` int32
+    ``[B]`` (0 = off) and ``top_p`` f32 ``[B]`` (1 = off), either may be None (not
+    both).  Returns ``(out_tokens [B, gamma+1], out_num_accepted [B])``."""
+    B, R, S = target.shape
+    gamma = R - 1
+    V = S if V is None else int(V)
+    dev = target.device
+    if top_k is None and top_p is None:
+        raise ValueError("give top_k, top_p or both")
+    if out_tokens is None:
+        out_tokens = torch.empty((B, gamma + 1), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    if top_k is not None and top_k.dtype != torch.int32:
+        raise TypeError("top_k must be int32")
+    if top_p is not None and top_p.dtype != torch.float32:
+        raise TypeError("top_p must be float32")
+    ws = _ws(workspace, SPEC_ENTRY_CHAIN, B, gamma, V, dev, stream)
+    st = lib().spec_verify_chain_filtered(
+        B, gamma, V, _p(target), _dtype(target), _rows(target, "target"),
+        _p(draft), SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
+        _rows(draft, "draft"), _p(draft_tokens), _p(temperature), _p(coins), _p(final_u), _p(top_k), _p(top_p),
+        _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "spec_verify_chain_filtered")
+    return out_tokens, out_num_accepted

@@ -180,6 +180,19 @@ def chain_config1(rnd: int = 0, device="cpu") -> ChainInputs:
                         target_sigma=3.0, draft_noise=1.0, temperatures=(0.6, 1.0))
 
 
+def chain_config6(rnd: int = 0, device="cpu") -> ChainInputs:
+    """The B=64, gamma=5, V=32000 chain workload under serving-style filters:
+    per sequence top_k drawn from {0 (off), 20, 50} and top_p from {1 (off), 0.9,
+    0.95}, in ``meta["top_k"]`` (int32 [B]) and ``meta["top_p"]`` (f32 [B])."""
+    inp = chain_config1(rnd, device)
+    g = make_gen(round_seed(6, rnd), device)
+    ks = torch.tensor([0, 20, 50], dtype=torch.int32, device=device)
+    ps = torch.tensor([1.0, 0.9, 0.95], dtype=torch.float32, device=device)
+    inp.meta["top_k"] = ks[torch.randint(0, 3, (inp.B,), generator=g, device=device)].contiguous()
+    inp.meta["top_p"] = ps[torch.randint(0, 3, (inp.B,), generator=g, device=device)].contiguous()
+    return inp
+
+
 def chain_config4(rnd: int = 0, device="cpu") -> ChainInputs:
     """B=512, gamma=7, V=129280, bf16 target N(0, 3^2), f32 draft probabilities
     softmax(target + N(0, 1.5^2)) at T = 1, T = 1."""
@@ -432,6 +445,7 @@ WORKLOADS = {
     3: "target-only tree B=128 N=32 V=151936 bf16, T=0.8, draft_probs NULL",
     4: "chain B=512 gamma=7 V=129280 bf16 target + f32 draft probs, T=1",
     5: "multi-step speculative sampling tree B=128 N=32 V=151936 bf16 + f32 draft distributions, T=0.8",
+    6: "chain B=64 gamma=5 V=32000 bf16 target+draft logits, T in {0.6,1.0}, top-k in {0,20,50}, top-p in {1,0.9,0.95}",
 }
 
 
@@ -450,6 +464,8 @@ def algorithmic_bytes(workload_id: int) -> int:
         return 512 * 8 * 129280 * 2
     if workload_id == 5:
         return 128 * 32 * 151936 * 2
+    if workload_id == 6:
+        return 64 * (6 + 5) * 32000 * 2
     raise ValueError(workload_id)
 
 

@@ -64,9 +64,37 @@ def gpu_chain(inp, workspace=None, lazy=False):
                 px=d[:, :g], qx=d[:, g:2 * g], S=d[:, 2 * g])
 
 
+def oracle_chain_filtered(inp, top_k, top_p, rows=None, nthreads=0):
+    sel = _sel(inp.target, rows)
+    tk = None if top_k is None else to_np(top_k[sel])
+    tp = None if top_p is None else to_np(top_p[sel])
+    if tk is None:
+        tk = np.zeros(len(to_np(inp.temperature[sel])), np.int32)
+    return oracle.chain(to_np(inp.target[sel]), to_np(inp.draft[sel]), inp.draft_is_probs,
+                        to_np(inp.draft_tokens[sel]), to_np(inp.temperature[sel]),
+                        to_np(inp.coins[sel]), to_np(inp.final_u[sel]), V=inp.V, nthreads=nthreads,
+                        top_k=tk, top_p=tp)
+
+
+def gpu_chain_filtered(inp, top_k, top_p, workspace=None):
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    B, g = inp.B, inp.gamma
+    diag = torch.full((B, 2 * g + 1), float("nan"), device=inp.target.device)
+    toks, na = sv.spec_verify_chain_filtered(inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins,
+                                             inp.final_u, top_k, top_p, draft_is_probs=inp.draft_is_probs,
+                                             V=inp.V, diag=diag, workspace=workspace)
+    torch.cuda.synchronize()
+    d = diag.cpu().numpy().astype(np.float64)
+    return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy(),
+                px=d[:, :g], qx=d[:, g:2 * g], S=d[:, 2 * g])
+
+
 def chain_flags(o, gamma):
     k = o["num_accepted"]
-    return (o["dmargin"] < TIE_TOL) | (o["cmargin"] < TIE_TOL) | ((k >= 0) & (k < gamma) & (o["S"] < TIE_TOL))
+    f = (o["dmargin"] < TIE_TOL) | (o["cmargin"] < TIE_TOL) | ((k >= 0) & (k < gamma) & (o["S"] < TIE_TOL))
+    if "fmargin" in o:                         # a top-p set decided within the tolerance
+        f |= o["fmargin"] < TIE_TOL
+    return f
 
 
 def compare_chain(g, o, gamma, rows=None):
@@ -195,7 +223,7 @@ def compare_mss(g, o, rows=None):
 # ----------------------------------------------------------------------------- runners with the oracle's signature
 
 def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, coins, final_u, V=None,
-                     nthreads=0, lazy=False):
+                     nthreads=0, lazy=False, top_k=None, top_p=None):
     """Same call signature and result keys as ``oracle.chain`` (numpy in, numpy out),
     executed by the CUDA library.  Used to run the oracle's statistical pins
     through the GPU path."""
@@ -212,10 +240,15 @@ def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, c
     dr = _pad_rows(t(draft))
     B, R, S = target.shape
     V = S if V is None else V
-    toks, na = spec_verify_chain(tg, dr, t(np.asarray(draft_tokens, np.int32)),
-                                 t(np.asarray(temperature, np.float32).reshape(B)),
-                                 t(np.asarray(coins, np.float32)), t(np.asarray(final_u, np.float32).reshape(B)),
-                                 draft_is_probs=draft_is_probs, V=V)
+    args = (tg, dr, t(np.asarray(draft_tokens, np.int32)), t(np.asarray(temperature, np.float32).reshape(B)),
+            t(np.asarray(coins, np.float32)), t(np.asarray(final_u, np.float32).reshape(B)))
+    if top_k is not None or top_p is not None:
+        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+        tk = None if top_k is None else t(np.asarray(top_k, np.int32).reshape(B))
+        tp = None if top_p is None else t(np.asarray(top_p, np.float32).reshape(B))
+        toks, na = sv.spec_verify_chain_filtered(*args, tk, tp, draft_is_probs=draft_is_probs, V=V)
+    else:
+        toks, na = spec_verify_chain(*args, draft_is_probs=draft_is_probs, V=V)
     return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy())
 
 
