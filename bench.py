@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -93,6 +93,8 @@ def make_inputs(wid: int, rnd: int, device, rank: int = 0):
         return wl.tree_config5(r, device)
     if wid == 6:
         return wl.chain_config6(r, device)
+    if wid == 7:
+        return wl.chain_config4(r, device)
     return wl.chain_config4(r, device)
 
 
@@ -104,10 +106,23 @@ def input_bytes(inp) -> int:
     return n
 
 
+VP_WORLD = 8          # vocabulary shards of the vocabulary-parallel workload
+
+
+def vp_cuts(V: int, world: int = VP_WORLD):
+    return [V * r // world for r in range(world + 1)]
+
+
 def describe(wid: int, inp) -> dict:
     from speculative_decoding_verify_temperature_b200 import workloads as wl
+    if wid == 7:
+        return {"workload": f"vocabulary-parallel chain: {wl.WORKLOADS[4]}, split over {VP_WORLD} vocabulary shards; "
+                            "timed: one rank's five device steps (shard 0); the three exchanges are prepared "
+                            "once and not timed (one GPU)",
+                "global_batch": inp.B, "gamma": inp.gamma, "V": inp.V, "shards": VP_WORLD,
+                "V_shard": vp_cuts(inp.V)[1], "target_dtype": "bfloat16", "draft": "f32 probabilities"}
     d = {"workload": wl.WORKLOADS[wid], "global_batch": inp.B}
-    if wid in (0, 1, 4, 6):
+    if wid in (0, 1, 4, 6, 7):
         d.update(gamma=inp.gamma, V=inp.V, target_dtype=str(inp.target.dtype).split(".")[-1],
                  draft="f32 probabilities" if inp.draft_is_probs else str(inp.draft.dtype).split(".")[-1] + " logits")
     else:
@@ -120,10 +135,12 @@ class Runner:
 
     def __init__(self, wid, inp, ws, lazy=False):
         self.wid, self.inp, self.ws, self.sfx = wid, inp, ws, "_lazy" if lazy else ""
+        if wid == 7:
+            self._vp_setup()
         import torch
         B = inp.B
         dev = inp.target.device
-        if wid in (0, 1, 4, 6):
+        if wid in (0, 1, 4, 6, 7):
             self.out = (torch.empty((B, inp.gamma + 1), dtype=torch.int32, device=dev),
                         torch.empty((B,), dtype=torch.int32, device=dev))
         else:
@@ -132,10 +149,59 @@ class Runner:
                         torch.empty((B, W), dtype=torch.int32, device=dev),
                         torch.empty((B,), dtype=torch.int32, device=dev))
 
+    def _vp_setup(self):
+        """Shard 0's columns of every row, and the exchanged buffers of a round
+        over all shards (computed once, as the other ranks would have)."""
+        import torch
+        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+        i = self.inp
+        cuts = vp_cuts(i.V)
+
+        def shard(x, a, b):
+            q = 16 // x.element_size()
+            out = torch.zeros((x.shape[0], x.shape[1], -(-(b - a) // q) * q), dtype=x.dtype, device=x.device)
+            out[:, :, :b - a] = x[:, :, a:b]
+            return out
+
+        shards = [(shard(i.target, cuts[r], cuts[r + 1]), shard(i.draft, cuts[r], cuts[r + 1]), cuts[r],
+                   cuts[r + 1] - cuts[r]) for r in range(VP_WORLD)]
+        wss = [sv.Workspace(i.target.device).get(sv.SPEC_ENTRY_CHAIN, i.B, i.gamma, vs) for (_, _, _, vs) in shards]
+        recs = [sv.spec_vp_chain_stats(t, d, i.draft_tokens, i.temperature, vocab_offset=a, draft_is_probs=True,
+                                       V_shard=vs, workspace=wss[r]) for r, (t, d, a, vs) in enumerate(shards)]
+        self.rec_all = torch.stack(recs)
+        for r, (t, d, a, vs) in enumerate(shards):
+            sv.spec_vp_chain_decide(self.rec_all, i.draft_tokens, i.temperature, i.coins, V=i.V, V_shard=vs,
+                                    draft_is_probs=True, workspace=wss[r])
+        self.mass_all = torch.stack([sv.spec_vp_chain_residual(t, d, self.rec_all, rank=r, draft_is_probs=True,
+                                                               V_shard=vs, workspace=wss[r])
+                                     for r, (t, d, a, vs) in enumerate(shards)])
+        toks = [sv.spec_vp_chain_sample(t, d, i.final_u, self.rec_all, self.mass_all, vocab_offset=a, rank=r,
+                                        draft_is_probs=True, V_shard=vs, workspace=wss[r])
+                for r, (t, d, a, vs) in enumerate(shards)]
+        self.tok = torch.stack(toks).max(dim=0).values
+        self.t0, self.d0, _, self.vs0 = shards[0]
+        self.ws = wss[0]
+        self.rec0 = torch.empty_like(recs[0])
+        self.mass0 = torch.empty_like(self.mass_all[0])
+        self.tok0 = torch.empty_like(self.tok)
+        del shards, recs, toks
+
     def __call__(self):
         from speculative_decoding_verify_temperature_b200 import spec_verify as sv
         i = self.inp
-        if self.wid == 6:
+        if self.wid == 7:
+            # rank 0 of the vocabulary-parallel round; exchanged buffers from the setup
+            sv.spec_vp_chain_stats(self.t0, self.d0, i.draft_tokens, i.temperature, vocab_offset=0, draft_is_probs=True,
+                                   V_shard=self.vs0, rec_out=self.rec0, workspace=self.ws)
+            sv.spec_vp_chain_decide(self.rec_all, i.draft_tokens, i.temperature, i.coins, V=i.V, V_shard=self.vs0,
+                                    draft_is_probs=True, out_tokens=self.out[0], out_num_accepted=self.out[1],
+                                    workspace=self.ws)
+            sv.spec_vp_chain_residual(self.t0, self.d0, self.rec_all, rank=0, draft_is_probs=True, V_shard=self.vs0,
+                                      mass_out=self.mass0, workspace=self.ws)
+            sv.spec_vp_chain_sample(self.t0, self.d0, i.final_u, self.rec_all, self.mass_all, vocab_offset=0, rank=0,
+                                    draft_is_probs=True, V_shard=self.vs0, tok_out=self.tok0, workspace=self.ws)
+            sv.spec_vp_chain_finish(self.tok, self.out[0], V_shard=self.vs0, workspace=self.ws)
+        elif self.wid == 6:
             sv.spec_verify_chain_filtered(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                           i.meta["top_k"], i.meta["top_p"], draft_is_probs=i.draft_is_probs, V=i.V,
                                           out_tokens=self.out[0], out_num_accepted=self.out[1], workspace=self.ws)
@@ -163,8 +229,9 @@ class Runner:
 
 def kernels_per_step(wid, inp) -> int:
     """Launches per verify call: the row-statistics kernel and the finalize kernel
-    (and the filter kernel between them for the filtered chain)."""
-    return 3 if wid == 6 else 2
+    (and the filter kernel between them for the filtered chain; six for one rank
+    of the vocabulary-parallel round)."""
+    return {6: 3, 7: 6}.get(wid, 2)
 
 
 def lazy_kernels_per_step(wid, inp) -> int:
@@ -194,12 +261,16 @@ def workspace_for(wid, inp):
     ws = sv.Workspace(inp.target.device)
     if wid in (0, 1, 4, 6):
         return ws.get(sv.SPEC_ENTRY_CHAIN, inp.B, inp.gamma, inp.V)
+    if wid == 7:
+        return None                           # each rank's workspace is set up by the runner
     e = {2: sv.SPEC_ENTRY_TREE_GREEDY, 3: sv.SPEC_ENTRY_TREE_SAMPLE, 5: sv.SPEC_ENTRY_TREE_MSS}[wid]
     return ws.get(e, inp.B, inp.N, inp.V)
 
 
 def algorithmic_bytes(wid, inp) -> int:
     """Bytes of logits / probabilities the row kernel must read once per round."""
+    if wid == 7:                              # rank 0's shard of the target rows
+        return inp.B * (inp.gamma + 1) * vp_cuts(inp.V)[1] * inp.target.element_size()
     b = inp.target[:, :, :inp.V].numel() * inp.target.element_size()
     if wid in (0, 1, 6):
         b += inp.draft[:, :, :inp.V].numel() * inp.draft.element_size()
@@ -281,14 +352,14 @@ def cpu_baseline(wid, inp, seconds, nthreads=None):
     cores = nthreads or len(os.sched_getaffinity(0))
     # Copy the inputs to host once; the oracle reads the same bytes the GPU reads.
     n = 0
-    fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain,
+    fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain, 7: parity.oracle_chain,
           2: parity.oracle_greedy, 3: parity.oracle_sample, 5: parity.oracle_mss,
           6: lambda i, r, nthreads: parity.oracle_chain_filtered(i, i.meta["top_k"], i.meta["top_p"], r,
                                                                  nthreads=nthreads)}[wid]
     B = inp.B
     # Large workloads: a bounded sample of whole sequences per "round" of work,
     # scaled to full rounds below.
-    per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4}[wid]))
+    per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4, 7: 16}[wid]))
     rows = None if per == B else list(range(per))
     elapsed = 0.0
     while n == 0 or elapsed < seconds:
@@ -463,14 +534,15 @@ def main():
     acc = torch.cat(acc)
     mean_tau = float((acc + 1).mean())
     B = first.B
-    draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6) else first.N - 1)
+    draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6, 7) else first.N - 1)
 
     # --- end to end through the binding with host buffers
-    e2e = run_e2e(wid, first, ws, args.e2e_steps, dev)
+    e2e = run_e2e(wid, first, ws, args.e2e_steps, dev) if wid != 7 else {
+        "value": None, "unit": "rounds/s", "note": "one rank of a vocabulary-parallel round: no single-GPU host path"}
 
     # --- the row-on-demand entry point on the same input sets
     # (the filtered chain has no row-on-demand variant)
-    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid != 6 else None
+    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid < 6 else None
 
     cfg = describe(wid, first)
     cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",

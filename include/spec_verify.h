@@ -401,6 +401,59 @@ spec_status spec_verify_tree_sample_lazy(int B, int N, int V, int max_depth,
                                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Vocabulary-parallel chain verify: the target (and draft) logits of every
+ * row are sharded along the vocabulary over the `world` ranks of a tensor-
+ * parallel group; rank r holds columns [vocab_offset_r, vocab_offset_r +
+ * V_shard_r) and the shards tile [0, V).  The pages assume one device holds
+ * whole rows ([origins] "Speculative Decoding" rules 1-3); these calls split
+ * the same rules into per-shard steps joined by three small exchanges that
+ * the caller performs (NCCL all-gather / all-reduce), giving the tokens and
+ * counts of spec_verify_chain up to rounding (shard sums are combined in
+ * rank order):
+ *   1. spec_vp_chain_stats on every rank -> rec_out [B, 2*gamma+1] records of
+ *      spec_vp_record_bytes() bytes; all-gather into rec_all [world, B, ...]
+ *      in rank order;
+ *   2. spec_vp_chain_decide on every rank (identical results): accepted
+ *      tokens, out_num_accepted, p/q diagnostics, and the per-sequence state
+ *      the next steps read from the workspace;
+ *   3. spec_vp_chain_residual -> mass_out [B] f64, the shard's part of the
+ *      mass of the last token's distribution; all-gather into mass_all
+ *      [world, B];
+ *   4. spec_vp_chain_sample -> tok_out [B] int32: the global token id on the
+ *      rank whose shard holds u*S, -1 elsewhere; all-reduce MAX;
+ *   5. spec_vp_chain_finish writes the reduced token at position k of
+ *      out_tokens.
+ * Each rank uses one workspace of spec_workspace_bytes(SPEC_ENTRY_CHAIN, B,
+ * gamma, V_shard) for all five steps of a round (V_shard of that rank).
+ * Argument conventions otherwise as spec_verify_chain (rows of the shard,
+ * strides in elements); draft_tokens are global ids in [0, V).
+ */
+size_t spec_vp_record_bytes(void);
+spec_status spec_vp_chain_stats(int B, int gamma, int V_shard, int vocab_offset,
+                                const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                const int32_t* draft_tokens, const float* temperature, void* rec_out,
+                                void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_vp_chain_decide(int B, int gamma, int V, int V_shard, int world, const void* rec_all,
+                                 int draft_is_probs,
+                                 const int32_t* draft_tokens, const float* temperature, const float* coins,
+                                 int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_vp_chain_residual(int B, int gamma, int V_shard, int world, int rank,
+                                   const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                   const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                   const void* rec_all, double* mass_out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_vp_chain_sample(int B, int gamma, int V_shard, int vocab_offset, int world, int rank,
+                                 const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                 const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                 const float* final_u, const void* rec_all, const double* mass_all,
+                                 int32_t* tok_out, float* diag,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+spec_status spec_vp_chain_finish(int B, int gamma, int V_shard, const int32_t* tok, int32_t* out_tokens,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_workspace_bytes -- workspace size for one entry point and shape.
  * rows = gamma for SPEC_ENTRY_CHAIN (sized for draft logits, which also
  * covers draft probabilities), N for the tree entry points.  Returns 0 for

@@ -13,6 +13,7 @@ from .spec_verify import (  # noqa: F401
     spec_verify_chain,
     spec_verify_chain_filtered,
     spec_verify_chain_lazy,
+    spec_verify_chain_vocab_parallel,
     spec_verify_tree_greedy,
     spec_verify_tree_greedy_lazy,
     spec_verify_tree_mss,

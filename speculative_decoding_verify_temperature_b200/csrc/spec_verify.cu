@@ -2425,6 +2425,298 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
     }
 }
 
+// ============================================================================= vocabulary-parallel chain verify
+//
+// The target (and draft) logits are sharded along the vocabulary over the
+// ranks of a tensor-parallel group; rank r holds columns [off_r, off_r + Vs)
+// of every row.  A round takes three small exchanges between four kernel
+// steps (the collectives themselves are the caller's, e.g. NCCL):
+//   stats    per row and shard: (m_r, Z_r) in the base-2 units of the
+//            statistics, and the drafted token's logit (or draft
+//            probability) when the token falls in the shard  -> all-gather
+//   decide   every rank combines the shards' rows in rank order (m = max m_r,
+//            Z = sum Z_r 2^(m_r - m), fp64) and takes the same decisions
+//   residual the shard's mass of max(0, p_k - q_k) (or of p_gamma for the
+//            bonus, from the statistics alone)                  -> all-gather
+//   sample   every rank locates the shard holding u * S; that shard draws
+//            inside itself, the others give -1                  -> all-reduce max
+//   finish   the token goes to position k.
+
+struct ShardRec {
+    float m;          // max x of the shard's row (base-2 units), -inf if none
+    float val;        // logit (or draft probability) at the drafted token, if in this shard
+    double Z;         // sum 2^(x - m) over the shard's row
+    int has;          // the drafted token lies in this shard
+    int bad;          // NaN / +inf in the shard's row
+};
+
+// Per-sequence result of the decision, kept in the workspace for the
+// residual and sample steps.
+struct VpState {
+    int k;            // accepted drafts; -1 invalid
+    float s;          // log2(e) / T
+    float mp, mq;     // global maxima of target row k and draft row k
+    double zp, zq;    // global sums of target row k and draft row k
+};
+
+// stats: one warp per (sequence, row) of the shard, from k_stats' chunk
+// statistics; rows 0..gamma target, gamma+1.. draft logits; with draft
+// probabilities the draft "rows" only carry q(x).
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(NT) k_vp_rows(const Params P, ShardRec* out, int off) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * NWARP + (threadIdx.x >> 5);
+    const int R2 = 2 * P.gamma + 1;
+    if (gw >= P.B * R2) return;
+    const int b = gw / R2, r = gw - b * R2, gamma = P.gamma;
+    ShardRec rec{-INFINITY, 0.f, 0.0, 0, 0};
+    const int E = P.nch * SPC;
+    if (r <= gamma || DK == DK_LOGITS) {
+        const bool bd = warp_combine(P.stats + ((size_t)b * P.R + r) * E, E, rec.m, rec.Z);
+        // an all -inf shard row is legal (the other shards hold the mass); NaN / +inf is not
+        const float2* st = P.stats + ((size_t)b * P.R + r) * E;
+        bool nan = false;
+        for (int e = lane; e < E; e += 32) nan |= (st[e].y != st[e].y);
+        rec.bad = __any_sync(FULL, nan) ? 1 : 0;
+        if (!(rec.m > -INFINITY)) { rec.m = -INFINITY; rec.Z = 0.0; }
+        (void)bd;
+    }
+    if (lane == 0) {
+        const int i = r <= gamma ? r : r - gamma - 1;
+        if (i < gamma) {
+            const int x = P.draft_tokens[(size_t)b * gamma + i] - off;
+            if (x >= 0 && x < P.V) {
+                rec.has = 1;
+                if (r <= gamma) {
+                    rec.val = ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride, x);
+                } else {
+                    const char* drow = P.drf + ((size_t)b * gamma + i) * P.dstride;
+                    rec.val = (DK == DK_PROBS) ? __ldg(reinterpret_cast<const float*>(drow) + x) : ld_elem<DDT>(drow, x);
+                }
+            }
+        }
+        out[(size_t)b * R2 + r] = rec;
+    }
+}
+
+// Global (m, Z) of row r of sequence b from all shards, in rank order.
+__device__ __forceinline__ void vp_combine(const ShardRec* all, int world, int B, int R2, int b, int r, float* m,
+                                           double* Z, bool* bad) {
+    float mm = -INFINITY;
+    bool bd = false;
+    for (int w = 0; w < world; ++w) {
+        const ShardRec& x = all[((size_t)w * B + b) * R2 + r];
+        mm = fmaxf(mm, x.m);
+        bd |= x.bad != 0;
+    }
+    double z = 0.0;
+    for (int w = 0; w < world; ++w) {
+        const ShardRec& x = all[((size_t)w * B + b) * R2 + r];
+        if (x.m > -INFINITY) z += x.Z * exp2((double)x.m - (double)mm);
+    }
+    *m = mm;
+    *Z = z;
+    *bad = bd || !(mm > -INFINITY) || !(mm < INFINITY) || !(z > 0.0) || !(z < 1e300);
+}
+
+// decide: one warp per sequence, identical on every rank (rule 1).  Lanes
+// combine the rows over the shards (one row each, ranks in order) into
+// shared memory; lane 0 then takes the decisions.
+template <int DK>
+__global__ void __launch_bounds__(NT) k_vp_decide(const Params P, const ShardRec* all, int world, VpState* vs) {
+    constexpr int MR = 2 * SPEC_MAX_GAMMA + 1;
+    __shared__ float sm_m[NWARP][MR], sm_v[NWARP][MR];
+    __shared__ double sm_z[NWARP][MR];
+    __shared__ int sm_ok[NWARP][MR];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int b = blockIdx.x * NWARP + warp;
+    if (b >= P.B) return;
+    const int gamma = P.gamma, R2 = 2 * gamma + 1;
+    for (int r = lane; r < R2; r += 32) {
+        float m;
+        double Z;
+        bool bad;
+        const bool probs_row = DK == DK_PROBS && r > gamma;
+        if (probs_row) { m = 0.f; Z = 1.0; bad = false; }
+        else vp_combine(all, world, P.B, R2, b, r, &m, &Z, &bad);
+        int owners = 0;
+        float v = 0.f;
+        for (int w = 0; w < world; ++w) {
+            const ShardRec& x = all[((size_t)w * P.B + b) * R2 + r];
+            if (x.has) { ++owners; v = x.val; }
+        }
+        const int i = r <= gamma ? r : r - gamma - 1;
+        sm_m[warp][r] = m;
+        sm_z[warp][r] = Z;
+        sm_v[warp][r] = v;
+        sm_ok[warp][r] = !bad && (i >= gamma || owners == 1);
+    }
+    __syncwarp();
+    if (lane != 0) return;
+    const float T = P.temperature[b];
+    bool ok = temperature_ok(T);
+    const float s = ok ? scale_of(T) : 0.f;
+    int32_t* toks = P.out_tokens + (size_t)b * (gamma + 1);
+    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+    double px[SPEC_MAX_GAMMA], qx[SPEC_MAX_GAMMA];
+    for (int r = 0; r < R2 && ok; ++r) ok &= sm_ok[warp][r] != 0;
+    for (int i = 0; i < gamma && ok; ++i) {
+        const int x = P.draft_tokens[(size_t)b * gamma + i];
+        ok &= (x >= 0 && x < P.V);
+        px[i] = exp2((double)sm_v[warp][i] * (double)s - (double)sm_m[warp][i]) / sm_z[warp][i];
+        if constexpr (DK == DK_PROBS) {
+            qx[i] = (double)sm_v[warp][gamma + 1 + i];
+            ok &= (qx[i] >= 0.0 && qx[i] <= 3.0e38);
+        } else {
+            qx[i] = exp2((double)sm_v[warp][gamma + 1 + i] * (double)s - (double)sm_m[warp][gamma + 1 + i]) /
+                    sm_z[warp][gamma + 1 + i];
+        }
+    }
+    VpState st{-1, s, 0.f, 0.f, 0.0, 0.0};
+    if (!ok) {
+        for (int i = 0; i <= gamma; ++i) toks[i] = -1;
+        P.out_num_accepted[b] = -1;
+        if (dg) for (int i = 0; i < 2 * gamma + 1; ++i) dg[i] = nanf_();
+        flag_input_error(P);
+        vs[b] = st;
+        return;
+    }
+    int k = gamma;
+    for (int i = 0; i < gamma; ++i) {
+        const double ratio = qx[i] > 0.0 ? px[i] / qx[i] : INFINITY;
+        if (!((double)P.coins[(size_t)b * gamma + i] <= ratio)) { k = i; break; }
+    }
+    for (int i = 0; i < k; ++i) toks[i] = P.draft_tokens[(size_t)b * gamma + i];
+    for (int i = k; i <= gamma; ++i) toks[i] = -1;
+    P.out_num_accepted[b] = k;
+    if (dg)
+        for (int i = 0; i < gamma; ++i) { dg[i] = (float)px[i]; dg[gamma + i] = (float)qx[i]; }
+    st.k = k;
+    st.mp = sm_m[warp][k];
+    st.zp = sm_z[warp][k];
+    if (DK == DK_LOGITS && k < gamma) {
+        st.mq = sm_m[warp][gamma + 1 + k];
+        st.zq = sm_z[warp][gamma + 1 + k];
+    }
+    vs[b] = st;
+}
+
+// residual: the shard's part of the mass the last token is drawn from, one
+// CTA per sequence -- sum over the shard of max(0, p_k - q_k) (k < gamma), or
+// Z_r 2^(m_r - m) of row gamma (the bonus; no pass over the row).
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(SEQ_BT) k_vp_residual(const Params P, const ShardRec* all, int rank,
+                                                         const VpState* vs, double* mass) {
+    __shared__ FinShared sh;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    constexpr int CH = chunk_elems<TDT>();
+    const int b = blockIdx.x, gamma = P.gamma, R2 = 2 * gamma + 1;
+    const VpState st = vs[b];
+    double M = 0.0;
+    if (st.k >= 0 && st.k < gamma) {
+        const char* trow = P.tgt + ((size_t)b * (gamma + 1) + st.k) * P.tstride;
+        const char* drow = P.drf + ((size_t)b * gamma + st.k) * P.dstride;
+        WChainRes<TDT, DDT, DK> wf{trow, drow, st.s, st.mp, (float)(1.0 / st.zp), st.mq,
+                                   DK == DK_PROBS ? 0.f : (float)(1.0 / st.zq), P.V};
+        M = row_chunk_masses<CH, SEQ_BT>(wf, P.nch, reinterpret_cast<float*>(dyn), sh);
+    } else if (st.k == gamma) {
+        const ShardRec& x = all[((size_t)rank * P.B + b) * R2 + gamma];
+        M = x.m > -INFINITY ? x.Z * exp2((double)x.m - (double)st.mp) : 0.0;
+    }
+    if (threadIdx.x == 0) mass[b] = M;
+}
+
+// The shard holding u * S among per-shard masses (smallest r with u*S below
+// the running total, skipping empty shards; rounding past the end goes to
+// the last non-empty one), or -1 when the total is not positive.
+__device__ __forceinline__ int vp_owner(const double* ms, int world, int B, int b, double u, double* t_local,
+                                        double* S) {
+    double tot = 0.0;
+    for (int w = 0; w < world; ++w) tot += ms[(size_t)w * B + b];
+    *S = tot;
+    if (!(tot > 0.0)) return -1;
+    const double t = u * tot;
+    double c = 0.0;
+    int last = -1;
+    double before_last = 0.0;
+    for (int w = 0; w < world; ++w) {
+        const double x = ms[(size_t)w * B + b];
+        if (x > 0.0) {
+            if (t < c + x) { *t_local = t - c; return w; }
+            last = w;
+            before_last = c;
+        }
+        c += x;
+    }
+    *t_local = t - before_last;
+    return last;
+}
+
+// sample: one CTA per sequence; every rank finds the owner shard from the
+// gathered masses, the owner draws inside its shard (chunk masses of the same
+// weights, one chunk rescanned) and writes the global token id, the others
+// write -1.  An empty residual (rounding only) draws from p_k instead, with
+// the shards' masses of p_k taken from the statistics.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(SEQ_BT) k_vp_sample(const Params P, const ShardRec* all, int world, int rank,
+                                                       int off, const VpState* vs, const double* mass_all,
+                                                       int32_t* tok) {
+    __shared__ FinShared sh;
+    __shared__ double pk[64];
+    extern __shared__ __align__(128) unsigned char dyn[];
+    constexpr int CH = chunk_elems<TDT>();
+    const int b = blockIdx.x, gamma = P.gamma, R2 = 2 * gamma + 1;
+    const VpState st = vs[b];
+    if (st.k < 0) {
+        if (threadIdx.x == 0) tok[b] = -1;
+        return;
+    }
+    const double u = (double)P.final_u[b];
+    double tl = 0.0, S = 0.0;
+    int owner = vp_owner(mass_all, world, P.B, b, u, &tl, &S);
+    bool from_p = st.k == gamma;
+    if (owner < 0 && st.k < gamma) {                 // empty residual: draw from p_k
+        for (int w = threadIdx.x; w < world; w += SEQ_BT) {
+            const ShardRec& x = all[((size_t)w * P.B + b) * R2 + st.k];
+            pk[w] = x.m > -INFINITY ? x.Z * exp2((double)x.m - (double)st.mp) : 0.0;
+        }
+        __syncthreads();
+        double Sp;
+        owner = vp_owner(pk, world, 1, 0, u, &tl, &Sp);
+        from_p = true;
+    }
+    int y = -1;
+    if (owner == rank) {
+        const char* trow = P.tgt + ((size_t)b * (gamma + 1) + st.k) * P.tstride;
+        float* wpw = reinterpret_cast<float*>(dyn);
+        if (from_p) {
+            WTarget<TDT> wf{trow, st.s, st.mp, nullptr, 0, P.V};
+            row_chunk_masses<CH, SEQ_BT>(wf, P.nch, wpw, sh);
+            y = draw_from_chunks<CH, SEQ_BT>(wf, P.nch, P.V, tl, (float)u, sh);
+        } else {
+            const char* drow = P.drf + ((size_t)b * gamma + st.k) * P.dstride;
+            WChainRes<TDT, DDT, DK> wf{trow, drow, st.s, st.mp, (float)(1.0 / st.zp), st.mq,
+                                       DK == DK_PROBS ? 0.f : (float)(1.0 / st.zq), P.V};
+            row_chunk_masses<CH, SEQ_BT>(wf, P.nch, wpw, sh);
+            y = draw_from_chunks<CH, SEQ_BT>(wf, P.nch, P.V, tl, (float)u, sh);
+        }
+        if (y >= 0) y += off;
+    }
+    if (threadIdx.x == 0) {
+        tok[b] = y;
+        if (P.diag) P.diag[(size_t)b * (2 * gamma + 1) + 2 * gamma] = st.k == gamma ? 1.f : (float)S;
+    }
+}
+
+// finish: the reduced token goes to position k.
+__global__ void k_vp_finish(const Params P, const VpState* vs, const int32_t* tok) {
+    const int b = blockIdx.x * NT + threadIdx.x;
+    if (b >= P.B) return;
+    const int k = vs[b].k;
+    if (k >= 0) P.out_tokens[(size_t)b * (P.gamma + 1) + k] = tok[b];
+}
+
 // ============================================================================= lazy (row-on-demand) verification
 //
 // The verify rules need only some rows: the chain reads the target row (and
@@ -2871,7 +3163,7 @@ spec_status fail(spec_status st, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, total;
+    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, vp, total;
     int rej_cap;
     int R, nch_max;
 };
@@ -2898,6 +3190,9 @@ Layout make_layout(int entry, int B, int rows, int V) {
     // top-k / top-p filter records of the chain's rows
     L.filt = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(FiltRec) * (size_t)B * L.R);
+    // vocabulary-parallel chain: the decision's per-sequence state
+    L.vp = off;
+    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(VpState) * (size_t)B);
     L.total = off;
     return L;
 }
@@ -3485,6 +3780,206 @@ spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) { return sample_
 
 spec_status spec_verify_tree_mss(SPEC_MSS_ARGS_DECL) { return mss_entry(false, SPEC_MSS_ARGS); }
 spec_status spec_verify_tree_mss_lazy(SPEC_MSS_ARGS_DECL) { return mss_entry(true, SPEC_MSS_ARGS); }
+
+}  // extern "C"
+
+// ============================================================================= vocabulary-parallel chain entries
+
+namespace {
+
+// Common checks and Params of a shard step (V = the shard's width, or the full
+// vocabulary for the decision).  target == NULL skips the row checks.
+spec_status vp_params(Params& P, int B, int gamma, int V, const void* target, spec_dtype tdt, int64_t ts,
+                      const void* draft, spec_dtype ddt, int draft_is_probs, int64_t ds, void* workspace,
+                      size_t wsb, VpState** vs) {
+    if (B < 1) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 1", B);
+    if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
+    if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
+    spec_status s = SPEC_OK;
+    if (target) {
+        s = check_rows("target_logits", target, tdt, ts, V);
+        if (s != SPEC_OK) return s;
+        if (draft_is_probs && ddt != SPEC_F32) return fail(SPEC_ERR_INVALID_ARG, "draft probabilities must be SPEC_F32");
+        s = check_rows("draft", draft, ddt, ds, V);
+        if (s != SPEC_OK) return s;
+    }
+    const Layout L = make_layout(SPEC_ENTRY_CHAIN, B, gamma, V);
+    s = check_ws(workspace, wsb, L);
+    if (s != SPEC_OK) return s;
+    P.B = B; P.V = V; P.gamma = gamma;
+    P.rows_tgt = gamma + 1;
+    P.R = draft_is_probs ? gamma + 1 : 2 * gamma + 1;
+    const int CH = tdt == SPEC_BF16 ? chunk_elems<SPEC_BF16>() : chunk_elems<SPEC_F32>();
+    P.nch = (V + CH - 1) / CH;
+    P.tgt = static_cast<const char*>(target);
+    P.tstride = ts * (tdt == SPEC_F32 ? 4 : 2);
+    P.drf = static_cast<const char*>(draft);
+    P.dstride = ds * (ddt == SPEC_F32 ? 4 : 2);
+    bind_ws(P, workspace, L);
+    *vs = reinterpret_cast<VpState*>(static_cast<char*>(workspace) + L.vp);
+    return SPEC_OK;
+}
+
+template <int TDT, int DDT, int DK>
+spec_status vp_stats_launch(Params P, ShardRec* rec, int off, cudaStream_t st) {
+    spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
+    if (s != SPEC_OK) return s;
+    const unsigned grid = (unsigned)(((long long)P.B * (2 * P.gamma + 1) + NWARP - 1) / NWARP);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_vp_rows<TDT, DDT, DK>, P, rec, off);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "k_vp_rows launch: %s", cudaGetErrorString(e));
+    return launched("k_vp_rows");
+}
+
+template <int TDT, int DDT, int DK>
+spec_status vp_residual_launch(Params P, const ShardRec* all, int rank, const VpState* vs, double* mass,
+                               cudaStream_t st) {
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    k_vp_residual<TDT, DDT, DK><<<(unsigned)P.B, SEQ_BT, wpw, st>>>(P, all, rank, vs, mass);
+    return launched("k_vp_residual");
+}
+
+template <int TDT, int DDT, int DK>
+spec_status vp_sample_launch(Params P, const ShardRec* all, int world, int rank, int off, const VpState* vs,
+                             const double* mass_all, int32_t* tok, cudaStream_t st) {
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    k_vp_sample<TDT, DDT, DK><<<(unsigned)P.B, SEQ_BT, wpw, st>>>(P, all, world, rank, off, vs, mass_all, tok);
+    return launched("k_vp_sample");
+}
+
+#define SPEC_VP_DISPATCH(CALL)                                                                       \
+    do {                                                                                             \
+        if (draft_is_probs) {                                                                        \
+            if (tdt == SPEC_BF16) return CALL(SPEC_BF16, SPEC_F32, DK_PROBS);                        \
+            return CALL(SPEC_F32, SPEC_F32, DK_PROBS);                                               \
+        }                                                                                            \
+        if (tdt == SPEC_BF16 && ddt == SPEC_BF16) return CALL(SPEC_BF16, SPEC_BF16, DK_LOGITS);      \
+        if (tdt == SPEC_BF16 && ddt == SPEC_F32) return CALL(SPEC_BF16, SPEC_F32, DK_LOGITS);        \
+        if (tdt == SPEC_F32 && ddt == SPEC_BF16) return CALL(SPEC_F32, SPEC_BF16, DK_LOGITS);        \
+        return CALL(SPEC_F32, SPEC_F32, DK_LOGITS);                                                  \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t spec_vp_record_bytes(void) { return sizeof(ShardRec); }
+
+spec_status spec_vp_chain_stats(int B, int gamma, int V_shard, int vocab_offset,
+                                const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                const int32_t* draft_tokens, const float* temperature, void* rec_out,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (!target_logits || !draft_tokens || !temperature || !rec_out)
+        return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (vocab_offset < 0) return fail(SPEC_ERR_INVALID_ARG, "vocab_offset < 0");
+    Params P{};
+    VpState* vs;
+    spec_status s = vp_params(P, B, gamma, V_shard, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                              d_row_stride, workspace, workspace_bytes, &vs);
+    if (s != SPEC_OK) return s;
+    P.draft_tokens = draft_tokens;
+    P.temperature = temperature;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    ShardRec* rec = static_cast<ShardRec*>(rec_out);
+#define SPEC_VP_STATS(T, D, K) vp_stats_launch<T, D, K>(P, rec, vocab_offset, st)
+    SPEC_VP_DISPATCH(SPEC_VP_STATS);
+#undef SPEC_VP_STATS
+}
+
+spec_status spec_vp_chain_decide(int B, int gamma, int V, int V_shard, int world, const void* rec_all,
+                                 int draft_is_probs,
+                                 const int32_t* draft_tokens, const float* temperature, const float* coins,
+                                 int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (world < 1 || world > 64) return fail(SPEC_ERR_INVALID_ARG, "world = %d outside [1, 64]", world);
+    if (!rec_all || !draft_tokens || !temperature || !coins || !out_tokens || !out_num_accepted)
+        return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
+    Params P{};
+    VpState* vs;
+    spec_status s = vp_params(P, B, gamma, V_shard, nullptr, SPEC_BF16, 0, nullptr, SPEC_BF16, draft_is_probs, 0,
+                              workspace, workspace_bytes, &vs);
+    if (s != SPEC_OK) return s;
+    P.V = V;                                     // drafted tokens range over the whole vocabulary
+    P.draft_tokens = draft_tokens; P.temperature = temperature; P.coins = coins;
+    P.out_tokens = out_tokens; P.out_num_accepted = out_num_accepted; P.diag = diag;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = (unsigned)((B + NWARP - 1) / NWARP);
+    if (draft_is_probs) k_vp_decide<DK_PROBS><<<grid, NT, 0, st>>>(P, static_cast<const ShardRec*>(rec_all), world, vs);
+    else k_vp_decide<DK_LOGITS><<<grid, NT, 0, st>>>(P, static_cast<const ShardRec*>(rec_all), world, vs);
+    return launched("k_vp_decide");
+}
+
+spec_status spec_vp_chain_residual(int B, int gamma, int V_shard, int world, int rank,
+                                   const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                   const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                   const void* rec_all, double* mass_out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (world < 1 || world > 64 || rank < 0 || rank >= world)
+        return fail(SPEC_ERR_INVALID_ARG, "rank %d / world %d", rank, world);
+    if (!target_logits || !rec_all || !mass_out) return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    Params P{};
+    VpState* vs;
+    spec_status s = vp_params(P, B, gamma, V_shard, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                              d_row_stride, workspace, workspace_bytes, &vs);
+    if (s != SPEC_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ShardRec* all = static_cast<const ShardRec*>(rec_all);
+#define SPEC_VP_RES(T, D, K) vp_residual_launch<T, D, K>(P, all, rank, vs, mass_out, st)
+    SPEC_VP_DISPATCH(SPEC_VP_RES);
+#undef SPEC_VP_RES
+}
+
+spec_status spec_vp_chain_sample(int B, int gamma, int V_shard, int vocab_offset, int world, int rank,
+                                 const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                 const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
+                                 const float* final_u, const void* rec_all, const double* mass_all,
+                                 int32_t* tok_out, float* diag,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (world < 1 || world > 64 || rank < 0 || rank >= world)
+        return fail(SPEC_ERR_INVALID_ARG, "rank %d / world %d", rank, world);
+    if (!target_logits || !final_u || !rec_all || !mass_all || !tok_out)
+        return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    Params P{};
+    VpState* vs;
+    spec_status s = vp_params(P, B, gamma, V_shard, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                              d_row_stride, workspace, workspace_bytes, &vs);
+    if (s != SPEC_OK) return s;
+    P.final_u = final_u;
+    P.diag = diag;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ShardRec* all = static_cast<const ShardRec*>(rec_all);
+#define SPEC_VP_SAMPLE(T, D, K) vp_sample_launch<T, D, K>(P, all, world, rank, vocab_offset, vs, mass_all, tok_out, st)
+    SPEC_VP_DISPATCH(SPEC_VP_SAMPLE);
+#undef SPEC_VP_SAMPLE
+}
+
+spec_status spec_vp_chain_finish(int B, int gamma, int V_shard, const int32_t* tok, int32_t* out_tokens,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (!tok || !out_tokens) return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    Params P{};
+    VpState* vs;
+    spec_status s = vp_params(P, B, gamma, V_shard, nullptr, SPEC_BF16, 0, nullptr, SPEC_BF16, 0, 0, workspace,
+                              workspace_bytes, &vs);
+    if (s != SPEC_OK) return s;
+    P.out_tokens = out_tokens;
+    k_vp_finish<<<(unsigned)((B + NT - 1) / NT), NT, 0, static_cast<cudaStream_t>(stream)>>>(P, vs, tok);
+    return launched("k_vp_finish");
+}
 
 }  // extern "C"
 

@@ -62,6 +62,19 @@ def lib():
         L.spec_verify_chain_filtered.restype = i32
         L.spec_verify_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
                                                  P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.spec_vp_record_bytes.restype = sz
+        L.spec_vp_record_bytes.argtypes = []
+        L.spec_vp_chain_stats.restype = i32
+        L.spec_vp_chain_stats.argtypes = [i32, i32, i32, i32, P, i32, i64, P, i32, i32, i64, P, P, P, P, sz, P]
+        L.spec_vp_chain_decide.restype = i32
+        L.spec_vp_chain_decide.argtypes = [i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, P, P, sz, P]
+        L.spec_vp_chain_residual.restype = i32
+        L.spec_vp_chain_residual.argtypes = [i32, i32, i32, i32, i32, P, i32, i64, P, i32, i32, i64, P, P, P, sz, P]
+        L.spec_vp_chain_sample.restype = i32
+        L.spec_vp_chain_sample.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, i64, P, i32, i32, i64,
+                                           P, P, P, P, P, P, sz, P]
+        L.spec_vp_chain_finish.restype = i32
+        L.spec_vp_chain_finish.argtypes = [i32, i32, i32, P, P, P, sz, P]
         L.spec_workspace_bytes.restype = sz
         L.spec_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.spec_workspace_init.restype = i32
@@ -331,3 +344,158 @@ def spec_verify_chain_filtered(target, draft, draft_tokens, temperature, coins, 
         _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
     _check(st, "spec_verify_chain_filtered")
     return out_tokens, out_num_accepted
+
+
+
+# ----------------------------------------------------------------------------- vocabulary-parallel chain
+
+def spec_vp_record_bytes() -> int:
+    return int(lib().spec_vp_record_bytes())
+
+
+def _vp_ws(workspace, B, gamma, Vs, dev, stream):
+    return _ws(workspace, SPEC_ENTRY_CHAIN, B, gamma, Vs, dev, stream)
+
+
+def spec_vp_chain_stats(target, draft, draft_tokens, temperature, *, vocab_offset: int, draft_is_probs=False,
+                        V_shard=None, rec_out=None, workspace=None, stream=None):
+    """Step 1 on one rank: per-row shard statistics, ``uint8 [B, 2*gamma+1, record]``."""
+    B, R, S = target.shape
+    gamma = R - 1
+    Vs = S if V_shard is None else int(V_shard)
+    if rec_out is None:
+        rec_out = torch.empty((B, 2 * gamma + 1, spec_vp_record_bytes()), dtype=torch.uint8, device=target.device)
+    ws = _vp_ws(workspace, B, gamma, Vs, target.device, stream)
+    st = lib().spec_vp_chain_stats(B, gamma, Vs, int(vocab_offset), _p(target), _dtype(target), _rows(target, "target"),
+                                   _p(draft), SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
+                                   _rows(draft, "draft"), _p(draft_tokens), _p(temperature), _p(rec_out), _p(ws),
+                                   ws.numel(), _stream(stream))
+    _check(st, "spec_vp_chain_stats")
+    return rec_out
+
+
+def spec_vp_chain_decide(rec_all, draft_tokens, temperature, coins, *, V: int, V_shard: int, draft_is_probs=False,
+                         out_tokens=None, out_num_accepted=None, diag=None, workspace=None, stream=None):
+    """Step 2 (identical on every rank): ``(out_tokens, out_num_accepted)`` with the
+    last token still -1."""
+    world, B, R2, _ = rec_all.shape
+    gamma = (R2 - 1) // 2
+    dev = rec_all.device
+    if out_tokens is None:
+        out_tokens = torch.empty((B, gamma + 1), dtype=torch.int32, device=dev)
+    if out_num_accepted is None:
+        out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = _vp_ws(workspace, B, gamma, int(V_shard), dev, stream)
+    st = lib().spec_vp_chain_decide(B, gamma, int(V), int(V_shard), world, _p(rec_all), int(bool(draft_is_probs)),
+                                    _p(draft_tokens), _p(temperature), _p(coins), _p(out_tokens),
+                                    _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "spec_vp_chain_decide")
+    return out_tokens, out_num_accepted
+
+
+def spec_vp_chain_residual(target, draft, rec_all, *, rank: int, draft_is_probs=False, V_shard=None,
+                           mass_out=None, workspace=None, stream=None):
+    """Step 3 on one rank: the shard's part of the last distribution's mass, f64 ``[B]``."""
+    B, R, S = target.shape
+    gamma = R - 1
+    Vs = S if V_shard is None else int(V_shard)
+    world = rec_all.shape[0]
+    if mass_out is None:
+        mass_out = torch.empty((B,), dtype=torch.float64, device=target.device)
+    ws = _vp_ws(workspace, B, gamma, Vs, target.device, stream)
+    st = lib().spec_vp_chain_residual(B, gamma, Vs, world, int(rank), _p(target), _dtype(target),
+                                      _rows(target, "target"), _p(draft),
+                                      SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
+                                      _rows(draft, "draft"), _p(rec_all), _p(mass_out), _p(ws), ws.numel(),
+                                      _stream(stream))
+    _check(st, "spec_vp_chain_residual")
+    return mass_out
+
+
+def spec_vp_chain_sample(target, draft, final_u, rec_all, mass_all, *, vocab_offset: int, rank: int,
+                         draft_is_probs=False, V_shard=None, tok_out=None, diag=None, workspace=None, stream=None):
+    """Step 4 on one rank: int32 ``[B]``, the global token id where this shard holds
+    u*S, else -1."""
+    B, R, S = target.shape
+    gamma = R - 1
+    Vs = S if V_shard is None else int(V_shard)
+    world = rec_all.shape[0]
+    if tok_out is None:
+        tok_out = torch.empty((B,), dtype=torch.int32, device=target.device)
+    ws = _vp_ws(workspace, B, gamma, Vs, target.device, stream)
+    st = lib().spec_vp_chain_sample(B, gamma, Vs, int(vocab_offset), world, int(rank), _p(target), _dtype(target),
+                                    _rows(target, "target"), _p(draft),
+                                    SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
+                                    _rows(draft, "draft"), _p(final_u), _p(rec_all), _p(mass_all), _p(tok_out),
+                                    _p(diag), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "spec_vp_chain_sample")
+    return tok_out
+
+
+def spec_vp_chain_finish(tok, out_tokens, *, V_shard: int, workspace=None, stream=None):
+    """Step 5: the reduced token into position k of ``out_tokens``."""
+    B, W = out_tokens.shape
+    ws = _vp_ws(workspace, B, W - 1, int(V_shard), out_tokens.device, stream)
+    st = lib().spec_vp_chain_finish(B, W - 1, int(V_shard), _p(tok), _p(out_tokens), _p(ws), ws.numel(),
+                                    _stream(stream))
+    _check(st, "spec_vp_chain_finish")
+    return out_tokens
+
+
+class TorchExchange:
+    """The three exchanges of a vocabulary-parallel round over a torch.distributed
+    process group (NCCL on GPUs)."""
+
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.dist, self.group = dist, group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+
+    def all_gather(self, t):
+        parts = [torch.empty_like(t) for _ in range(self.world)]
+        self.dist.all_gather(parts, t.contiguous(), group=self.group)
+        return torch.stack(parts)
+
+    def all_reduce_max(self, t):
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX, group=self.group)
+        return t
+
+
+def spec_verify_chain_vocab_parallel(target, draft, draft_tokens, temperature, coins, final_u, *, vocab_offset: int,
+                                     V: int, draft_is_probs=False, exchange=None, ops=None, out_tokens=None,
+                                     out_num_accepted=None, diag=None, workspace=None, stream=None):
+    """One chain round with the vocabulary sharded over the ranks of ``exchange``
+    (default: the torch.distributed world).  ``target`` / ``draft`` are this
+    rank's shard ``[B, R, V_shard]``; the others are replicated.  Returns
+    ``(out_tokens [B, gamma+1], out_num_accepted [B])`` on every rank.  ``ops``
+    replaces the five device steps (tests of the exchange logic only)."""
+    ex = exchange or TorchExchange()
+    o = ops or _VP_OPS
+    Vs = target.shape[2]
+    rec = o.stats(target, draft, draft_tokens, temperature, vocab_offset=vocab_offset, draft_is_probs=draft_is_probs,
+                  V_shard=Vs, workspace=workspace, stream=stream)
+    rec_all = ex.all_gather(rec)
+    out_tokens, out_num_accepted = o.decide(rec_all, draft_tokens, temperature, coins, V=V, V_shard=Vs,
+                                            draft_is_probs=draft_is_probs, out_tokens=out_tokens,
+                                            out_num_accepted=out_num_accepted, diag=diag, workspace=workspace,
+                                            stream=stream)
+    mass = o.residual(target, draft, rec_all, rank=ex.rank, draft_is_probs=draft_is_probs, V_shard=Vs,
+                      workspace=workspace, stream=stream)
+    mass_all = ex.all_gather(mass)
+    tok = o.sample(target, draft, final_u, rec_all, mass_all, vocab_offset=vocab_offset, rank=ex.rank,
+                   draft_is_probs=draft_is_probs, V_shard=Vs, diag=diag, workspace=workspace, stream=stream)
+    tok = ex.all_reduce_max(tok)
+    o.finish(tok, out_tokens, V_shard=Vs, workspace=workspace, stream=stream)
+    return out_tokens, out_num_accepted
+
+
+class _VpOps:
+    stats = staticmethod(spec_vp_chain_stats)
+    decide = staticmethod(spec_vp_chain_decide)
+    residual = staticmethod(spec_vp_chain_residual)
+    sample = staticmethod(spec_vp_chain_sample)
+    finish = staticmethod(spec_vp_chain_finish)
+
+
+_VP_OPS = _VpOps()

@@ -75,3 +75,60 @@ def test_two_gloo_ranks_shard_the_batch_and_take_the_slowest_time():
     # max over ranks, whole-job rounds/s
     assert all(g[2] == 2.0 for g in got)
     assert all(abs(g[3] - 2 * 100 / 2e-3) < 1e-6 for g in got)
+
+
+
+def _vp_rank(rank, world, port, cuts, out):
+    """One rank of a vocabulary-parallel chain round: the orchestration of
+    spec_verify_chain_vocab_parallel over gloo, with CPU stand-ins for the
+    device steps."""
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    from speculative_decoding_verify_temperature_b200 import workloads as wl
+    import vp_fakes
+    inp = wl.chain_inputs(24, 4, 300, seed=5, device="cpu", target_dtype=__import__("torch").float32,
+                          draft_dtype=__import__("torch").float32, zipf=True, temperatures=(0.6, 1.0))
+    a, b = cuts[rank], cuts[rank + 1]
+    toks, k = sv.spec_verify_chain_vocab_parallel(
+        inp.target[:, :, a:b].contiguous(), inp.draft[:, :, a:b].contiguous(), inp.draft_tokens, inp.temperature,
+        inp.coins, inp.final_u, vocab_offset=a, V=300, exchange=sv.TorchExchange(), ops=vp_fakes.FakeVpOps())
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, toks.numpy(), k.numpy()))
+
+
+def test_two_gloo_ranks_vocab_parallel_round_matches_oracle():
+    """Two ranks each hold part of every row's vocabulary; the three exchanges
+    (all-gather of row statistics, all-gather of residual masses, all-reduce of
+    the token) give both ranks the oracle's tokens for the whole rows."""
+    world, cuts = 2, [0, 172, 300]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_vp_rank, args=(r, world, port, cuts, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q.get(timeout=240) for _ in range(world)], key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    import sys
+    import torch
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity
+    from speculative_decoding_verify_temperature_b200 import workloads as wl
+    inp = wl.chain_inputs(24, 4, 300, seed=5, device="cpu", target_dtype=torch.float32, draft_dtype=torch.float32,
+                          zipf=True, temperatures=(0.6, 1.0))
+    o = parity.oracle_chain(inp)
+    flags = parity.chain_flags(o, inp.gamma)
+    for r in range(world):
+        same = (got[r][2] == o["num_accepted"]) & (got[r][1] == o["tokens"]).all(axis=1)
+        assert (same | flags).all()
+        assert np.array_equal(got[r][1], got[0][1])
