@@ -1936,6 +1936,195 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_row(const Params P) {
     }
 }
 
+// Thread-block cluster helpers (a pair of CTAs per sequence).
+__device__ __forceinline__ unsigned cluster_rank() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ double peer_ld_f64(const double* p, unsigned peer) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(peer));
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(remote) : "memory");
+    return v;
+}
+__device__ __forceinline__ int peer_ld_s32(const int* p, unsigned peer) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(peer));
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// Chain finalisation by a cluster of two CTAs per sequence: both take the
+// decision (identical); the rejected row pair is split at a group boundary,
+// each CTA stages its half with two bulk copies, forms the 8-element group
+// sums of max(0, p_k - q_k) and scans them; the two half masses meet through
+// distributed shared memory (two cluster barriers, which every CTA of the pair
+// reaches on every path: the decision is the same in both); the CTA whose
+// half holds u*S draws inside it.  The bonus token is drawn by the first CTA
+// as in the one-CTA kernel.
+template <int TDT, int DDT, int DK, bool LZ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SEQ_BT) k_chain_final_pair(const Params P) {
+    __shared__ FinShared sh;
+    __shared__ __align__(8) uint64_t bar, sbar;
+    __shared__ int owner, found_g, s_fail;
+    __shared__ double s_half;
+    extern __shared__ __align__(128) unsigned char stage[];
+    constexpr int TESZ = Tr<TDT>::ESZ;
+    constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
+    const unsigned rank = cluster_rank();
+    const int tid = threadIdx.x, b = blockIdx.x >> 1;
+    const int gamma = P.gamma, V = P.V;
+    if constexpr (LZ) {
+        pdl_wait();
+        if (tid == 0) mbar_init(smem_u32(&bar), 1);
+        chain_lazy_state(P, b, sh, rank == 0);
+    } else {
+        const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
+        pdl_wait();
+        const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
+        if (tid == 0) mbar_init(smem_u32(&bar), 1);
+        combine_softmax_rows<SEQ_BT>(P, blk, P.R, sh);
+        __syncthreads();
+        chain_decide<TDT, DDT, DK>(P, b, sh, rank == 0, pf);
+    }
+    const int ok = sh.ivals[0], k = sh.ivals[1];
+    const float s = (float)sh.dvals[0];
+    if (!ok) return;                                  // the same in both CTAs of the pair
+    const float u = P.final_u[b];
+    int32_t* toks = P.out_tokens + (size_t)b * (gamma + 1);
+    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
+    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
+    if (k == gamma) {                                 // the same in both CTAs of the pair
+        if (rank != 0) return;
+        const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * SPC;
+        double S;
+        const int y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
+        if (tid == 0) {
+            toks[k] = y;
+            if (dg) dg[2 * gamma] = 1.0f;
+        }
+        return;
+    }
+    const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
+    // this CTA's half: groups [0, G0) or [G0, G), G0 = ceil(G / 2)
+    const int G = (V + 7) / 8, G0 = (G + 1) / 2;
+    const int lo = rank == 0 ? 0 : 8 * G0;
+    const int Vh = rank == 0 ? min(V, 8 * G0) : max(0, V - 8 * G0);
+    const char* th = trow + (size_t)lo * TESZ;
+    const char* dh = drow + (size_t)lo * DESZ;
+    const uint32_t bt = ((uint32_t)Vh * TESZ) & ~15u, bd = ((uint32_t)Vh * DESZ) & ~15u;
+    unsigned char* ts = stage;
+    unsigned char* ds = stage + bt;
+    float* gs = reinterpret_cast<float*>(stage + bt + bd);
+    if (tid == 0) {
+        mbar_expect_tx(smem_u32(&bar), bt + bd);
+        if (bt) bulk_g2s(smem_u32(ts), th, bt, smem_u32(&bar));
+        if (bd) bulk_g2s(smem_u32(ds), dh, bd, smem_u32(&bar));
+    }
+    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]);
+    const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
+    const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
+    WChainResStaged<TDT, DDT, DK> wf{ts, ds, th, dh, (int)(bt / TESZ), (int)(bd / DESZ), s, mp, izp, mq, izq, Vh};
+    const bool copied = mbar_wait(smem_u32(&bar), 0);
+    if (!copied && tid == 0) {
+        atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
+        mbar_wait(smem_u32(&bar), 0);                 // let the copy land (bounded)
+    }
+    const int Gh = (Vh + 7) / 8;
+    if (copied)
+        for (int g = tid; g < Gh; g += SEQ_BT) {
+            float w[8];
+            wf.group((int64_t)g * 8, w);
+            gs[g] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+        }
+    __syncthreads();
+    const int g0 = (int)((long long)Gh * tid / SEQ_BT), g1 = (int)((long long)Gh * (tid + 1) / SEQ_BT);
+    double seg = 0.0;
+    if (copied)
+        for (int g = g0; g < g1; ++g) seg += (double)gs[g];
+    if (tid == 0) { owner = -1; found_g = -1; }
+    double Sh;
+    const double excl = block_excl_scan<SEQ_BT>(seg, &Sh);
+    if (tid == 0) { s_half = Sh; s_fail = copied ? 0 : 1; }
+    cluster_sync_all();                               // both halves' masses are written
+    const double Sp = peer_ld_f64(&s_half, rank ^ 1u);
+    const int fail = (copied ? 0 : 1) | peer_ld_s32(&s_fail, rank ^ 1u);
+    cluster_sync_all();                               // nothing reads the peer's shared memory after this
+    if (fail) {
+        if (rank == 0 && tid == 0) {
+            for (int i = 0; i <= gamma; ++i) toks[i] = -1;
+            P.out_num_accepted[b] = -1;
+        }
+        return;
+    }
+    const double S0 = rank == 0 ? Sh : Sp, S1 = rank == 0 ? Sp : Sh;
+    const double S = S0 + S1;                         // the same sum in both CTAs
+    const double t = (double)u * S;
+    if (!(S > 0.0)) {                                 // empty residual (rounding only): draw from p_k
+        if (rank != 0) return;
+        const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * SPC;
+        double Su;
+        const int y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+        if (tid == 0) {
+            toks[k] = y;
+            if (dg) dg[2 * gamma] = (float)S;
+        }
+        return;
+    }
+    // the half holding t (rounding past the end goes to the last half with mass)
+    const unsigned own = (S0 > 0.0 && (t < S0 || !(S1 > 0.0))) ? 0u : 1u;
+    if (rank != own) return;
+    const double tl = own == 0 ? t : t - S0;
+    if (seg > 0.0 && excl <= tl) atomicMax(&owner, tid);
+    __syncthreads();
+    if (tid == owner) {
+        double acc = excl;
+        int gsel = -1, glast = -1;
+        double before = excl;
+        for (int g = g0; g < g1; ++g) {
+            const double v = (double)gs[g];
+            if (v > 0.0) {
+                glast = g;
+                before = acc;
+                if (tl < acc + v) { gsel = g; break; }
+            }
+            acc += v;
+        }
+        if (gsel < 0) gsel = glast;
+        float w[8];
+        wf.group((int64_t)gsel * 8, w);
+        const double loc = tl - before;
+        double a = 0.0;
+        int pick = -1, last = -1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a += (double)w[i];
+            if (w[i] > 0.f) {
+                last = gsel * 8 + i;
+                if (pick < 0 && loc < a) pick = gsel * 8 + i;
+            }
+        }
+        found_g = pick >= 0 ? pick : last;
+    }
+    __syncthreads();
+    int y = found_g >= 0 ? lo + found_g : -1;
+    if (y < 0) {                                      // nothing positive found (rounding only): draw from p_k
+        const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * SPC;
+        double Su;
+        y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
+    }
+    if (tid == 0) {
+        toks[k] = y;
+        if (dg) dg[2 * gamma] = (float)S;
+    }
+}
+
 // Tree finalisation, one CTA per sequence.
 template <int MODE, int TDT>
 __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
@@ -3321,11 +3510,10 @@ inline int stats_stage_bytes(const Params& P, int rows, size_t limit) {
     return bytes <= limit ? (int)bytes : 0;
 }
 
-// Dynamic shared memory available to the row-staged chain finalisation (0 if
-// it cannot be configured).
-template <int TDT, int DDT, int DK, bool LZ>
-size_t row_stage_capacity() {
-    auto kern = k_chain_final_row<TDT, DDT, DK, LZ>;
+// Dynamic shared memory available to a row-staged chain finalisation kernel
+// (0 if it cannot be configured).
+template <class K>
+size_t stage_capacity(K kern) {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return 0;
     int dev = 0, optin = 0;
@@ -3342,10 +3530,21 @@ size_t row_stage_capacity() {
 // lazy level walk (LZ = true, which stages no statistics).
 template <int TDT, int DDT, int DK, bool LZ>
 spec_status launch_chain_final(Params P, cudaStream_t st) {
-    // Row-staged finalisation when the rejected row pair (and the statistics)
-    // fit in shared memory and one CTA per sequence fits in a single wave.
-    static const size_t cap = row_stage_capacity<TDT, DDT, DK, LZ>();
-    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DK == DK_PROBS ? 4 : Tr<DDT>::ESZ);
+    constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
+    // A pair of CTAs per sequence (a cluster) when each half of the rejected
+    // row pair fits in shared memory and the pairs fit in a single wave; else
+    // one CTA per sequence with the whole pair staged; else the sliced kernel.
+    static const size_t cap2 = stage_capacity(k_chain_final_pair<TDT, DDT, DK, LZ>);
+    const int G = (P.V + 7) / 8;
+    const size_t half = staged_bytes(min(P.V, 8 * ((G + 1) / 2)), Tr<TDT>::ESZ, DESZ);
+    if (P.nch > 1 && half <= cap2 && P.B <= num_sms()) {
+        P.stage_off = (int)half;
+        P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, cap2 - half);
+        return launch_dependent(k_chain_final_pair<TDT, DDT, DK, LZ>, (unsigned)(2 * P.B), SEQ_BT,
+                                half + P.stage_cap, P, st, "k_chain_final_pair");
+    }
+    static const size_t cap = stage_capacity(k_chain_final_row<TDT, DDT, DK, LZ>);
+    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DESZ);
     if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
         P.stage_off = (int)pair;
         P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, cap - pair);
