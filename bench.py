@@ -522,7 +522,8 @@ def main():
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profile_traffic(wid),
                 "kernel": "k_stats (streams every logit row once)",
                 "kernel_ms": round(k_avg_ms, 5), "algorithmic_bytes_per_launch": alg,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"}
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+                "frac_of_nominal_8000_gbs": round(achieved / 8000.0, 4)}
     round_gbs = alg / (ms_max / K / 1e3) / 1e9
 
     # --- acceptance statistics of the benchmarked rounds
@@ -561,6 +562,8 @@ def main():
     }
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wid, first, args.cpu_seconds)
+        one = cpu_baseline(wid, first, args.cpu_seconds / 4, nthreads=1)
+        line["cpu_baseline"]["value_1thread"] = one["value"]
     elif rank == 0:
         line["cpu_baseline"] = None
     if rank == 0:

@@ -2191,7 +2191,9 @@ template <int DT> __host__ __device__ constexpr size_t filt_hist_bytes() {
 
 struct FiltShared {
     unsigned long long red[FILT_BT / 32];
-    unsigned long long at, above;
+    unsigned redc[FILT_BT / 32];
+    unsigned long long at, above, tm;
+    unsigned tc;
     int sel;
 };
 
@@ -2364,102 +2366,212 @@ __device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, f
 }
 
 // bf16 rows: an exact histogram of the row's values (65536 order keys, two
-// 16-bit counters per 32-bit word, 132 KB of shared memory) from one pass;
+// 16-bit counters per 32-bit word, 128 KB of shared memory) from one pass;
 // every mass then follows exactly as count * fixed(2^(v s - m)) per value,
-// the same fixed-point numbers the radix path adds element by element.  One
-// spare word after every 32 puts the runs that the scans give consecutive
-// threads (32 words apart) in consecutive banks.
-constexpr size_t VH_WORDS = 32768 + 32768 / 32;
-constexpr size_t VH_BYTES = VH_WORDS * 4;
+// the same fixed-point numbers the radix path adds element by element.
+//
+// A row has at most V distinct values, so most of the 32768 words are empty.
+// Thread t reads the 32 words of key block 1023 - t (16-byte loads, the four
+// quads of a block stored XOR-swizzled by the block index so that eight
+// consecutive threads hit eight distinct bank groups), and a block-wide scan
+// packs the indices of the non-empty words into a list in descending key
+// order.  The counts and masses are then summed over equal slices of that
+// list, so the exp2 work is spread evenly whatever the values' spread, and
+// one more scan orders the slices: the top-k key is where the running count
+// reaches top_k, the top-p key where the running mass reaches top_p times the
+// mass kept by top-k.
+constexpr int VH_WORDS = 32768;
+constexpr size_t VH_BYTES = (size_t)VH_WORDS * 4 + (size_t)VH_WORDS * 2;   // counters + word list
 
-__device__ __forceinline__ uint32_t vh_word(uint32_t k) {
-    const uint32_t i = k >> 1;
-    return i + (i >> 5);
+// Physical word of logical word i (= key >> 1): block i >> 5, quad
+// ((i >> 2) & 7) ^ (block & 7), lane i & 3.
+__device__ __forceinline__ uint32_t vh_phys(uint32_t i) { return i ^ ((i >> 3) & 0x1Cu); }
+
+// Order keys of the two bf16 values packed in x (low half = lower index), as
+// order_key does for one value: -0 folded onto +0, negative values
+// complemented, the sign bit of the others set.
+__device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
+    x &= ~__vcmpeq2(x, 0x80008000u);
+    return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
 }
-__device__ __forceinline__ unsigned vh_count(const uint32_t* w, uint32_t k) {
-    return (w[vh_word(k)] >> ((k & 1u) * 16u)) & 0xFFFFu;
+__device__ __forceinline__ void vh_count1(uint32_t* w, uint32_t k) {
+    atomicAdd(&w[vh_phys(k >> 1)], (k & 1u) ? 0x10000u : 1u);
 }
-__device__ __forceinline__ unsigned long long vh_weight(const uint32_t* w, uint32_t k, bool mass, float s, float m) {
-    const unsigned c = vh_count(w, k);
-    if (!mass || c == 0u) return c;
+__device__ __forceinline__ unsigned long long vh_mass(unsigned c, uint32_t k, float s, float m) {
+    if (c == 0u) return 0ull;
     return (unsigned long long)c *
            (unsigned long long)(ex2(fmaf(key_value<SPEC_BF16>(k), s, -m)) * (float)FIX_ONE);
 }
 
-// The largest key t >= lo whose weight W(keys >= t) reaches target (counts or
-// masses); a negative target means -target times W(keys >= lo).  Returns -1
-// when the keys >= lo never reach it.  fs.at = W(keys >= t) (W(keys >= lo)
-// when -1); fs.above = W(keys >= lo).  Each thread owns a run of 65536 /
-// FILT_BT keys, a block-wide u64 scan orders the runs.  All threads call it.
-__device__ int vh_scan(const uint32_t* w, uint32_t lo, bool mass, float s, float m, double target, FiltShared& fs) {
-    constexpr int PER = 65536 / FILT_BT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int hi = 65536 - tid * PER, lt = max((int)lo, hi - PER);
-    unsigned long long own = 0ull;
-    for (int k = hi - 1; k >= lt; --k) own += vh_weight(w, (uint32_t)k, mass, s, m);
-    unsigned long long inc = own;
+// Exclusive block-wide scan, in thread order, of a u32 and a u64; the totals
+// go to *ta / *tb.  All threads call it.
+__device__ void vh_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
+                         unsigned long long* tb, FiltShared& fs) {
+    static_assert(FILT_BT == 1024, "one warp scans the 32 warp totals");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned ia = a;
+    unsigned long long ib = b;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long v = __shfl_up_sync(FULL, inc, o);
-        if (lane >= o) inc += v;
+        const unsigned va = __shfl_up_sync(FULL, ia, o);
+        const unsigned long long vb = __shfl_up_sync(FULL, ib, o);
+        if (lane >= o) { ia += va; ib += vb; }
     }
-    if (lane == 31) fs.red[warp] = inc;
-    if (tid == 0) fs.sel = -1;
+    if (lane == 31) { fs.redc[warp] = ia; fs.red[warp] = ib; }
     __syncthreads();
-    unsigned long long excl = 0ull, total = 0ull;
-    for (int k = 0; k < FILT_BT / 32; ++k) {
-        if (k < warp) excl += fs.red[k];
-        total += fs.red[k];
-    }
-    excl += inc - own;
-    if (target < 0.0) target = -target * (double)total;
-    if (hi > lt && (double)excl < target && (double)(excl + own) >= target) {
-        unsigned long long cum = excl;
-        for (int k = hi - 1; k >= lt; --k) {
-            cum += vh_weight(w, (uint32_t)k, mass, s, m);
-            if ((double)cum >= target) { fs.sel = k; fs.at = cum; break; }
+    if (warp == 0) {
+        const unsigned xa = fs.redc[lane];
+        const unsigned long long xb = fs.red[lane];
+        unsigned sa = xa;
+        unsigned long long sb = xb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned va = __shfl_up_sync(FULL, sa, o);
+            const unsigned long long vb = __shfl_up_sync(FULL, sb, o);
+            if (lane >= o) { sa += va; sb += vb; }
         }
+        fs.redc[lane] = sa - xa;
+        fs.red[lane] = sb - xb;
+        if (lane == 31) { fs.tc = sa; fs.tm = sb; }
     }
     __syncthreads();
-    const int t = fs.sel;
-    if (tid == 0) {
-        fs.above = total;
-        if (t < 0) fs.at = total;
-    }
-    __syncthreads();
-    return t;
+    *ea = fs.redc[warp] + ia - a;
+    *eb = fs.red[warp] + ib - b;
+    *ta = fs.tc;
+    *tb = fs.tm;
+    __syncthreads();                                   // fs is free again
 }
 
-// Threshold and kept mass of a bf16 row from its value histogram.  Returns
-// false when a value occurs 65536 times or more (a 16-bit counter wrapped:
-// possible only for V > 65535); the caller then takes the radix path.
-__device__ bool filter_row_vh(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
-                              uint32_t* w, FiltRec* out) {
+// The value histogram of a bf16 row and its list of non-empty words (from the
+// logits alone, before the statistics are needed).  Returns the list length.
+// All threads call it.
+__device__ int vh_build(const char* row, int V, FiltShared& fs, uint32_t* w) {
     const int tid = threadIdx.x;
-    for (int i = tid; i < (int)VH_WORDS; i += FILT_BT) w[i] = 0u;
-    __syncthreads();
+    uint4* w4 = reinterpret_cast<uint4*>(w);
+    unsigned short* list = reinterpret_cast<unsigned short*>(w + VH_WORDS);
+    // histogram: four 16-byte loads per thread in flight (the first four
+    // while the counters are cleared), then the updates
     const int nv = (V + 7) / 8;
-    for (int vi = tid; vi < nv; vi += FILT_BT) {
-        const uint4 v = ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V);
+    uint4 v[4];
+    auto load4 = [&](int v0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (vi * 8 + i >= V) break;
-            const uint32_t k = order_key<SPEC_BF16>(vec_elem<SPEC_BF16>(v, i));
-            atomicAdd(&w[vh_word(k)], 1u << ((k & 1u) * 16u));
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * FILT_BT;
+            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    load4(tid);
+    for (int i = tid; i < VH_WORDS / 4; i += FILT_BT) w4[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int v0 = tid;;) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * FILT_BT;
+            if (vi >= nv) break;
+            const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            const int lim = V - vi * 8;                   // elements of this vector inside the row
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t k2 = vh_keys2(xs[c]);
+                if (2 * c < lim) vh_count1(w, k2 & 0xFFFFu);
+                if (2 * c + 1 < lim) vh_count1(w, k2 >> 16);
+            }
+        }
+        v0 += 4 * FILT_BT;
+        if (v0 >= nv) break;
+        load4(v0);
+    }
+    __syncthreads();
+    // non-empty words of this thread's block, highest first
+    const uint32_t blk = (uint32_t)(VH_WORDS / 32 - 1 - tid);
+    uint32_t mask = 0u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint4 x = w4[blk * 8 + (q ^ (blk & 7u))];
+        mask |= (x.x ? 1u : 0u) << (4 * q) | (x.y ? 1u : 0u) << (4 * q + 1) | (x.z ? 1u : 0u) << (4 * q + 2) |
+                (x.w ? 1u : 0u) << (4 * q + 3);
+    }
+    unsigned off, n;
+    unsigned long long d0, d1;
+    vh_scan2((unsigned)__popc(mask), 0ull, &off, &d0, &n, &d1, fs);
+    while (mask) {
+        const int j = 31 - __clz(mask);
+        list[off++] = (unsigned short)(blk * 32 + j);
+        mask &= ~(1u << j);
+    }
+    __syncthreads();
+    return (int)n;
+}
+
+// Threshold and kept mass of a bf16 row from its value histogram and word
+// list (vh_build).  Returns false when a value occurs 65536 times or more (a
+// 16-bit counter wrapped: possible only for V > 65535); the caller then takes
+// the radix path.  All threads call it.
+__device__ bool vh_select(int V, int n, float s, float m, int K, float Pp, FiltShared& fs, const uint32_t* w,
+                          FiltRec* out) {
+    const int tid = threadIdx.x;
+    const unsigned short* list = reinterpret_cast<const unsigned short*>(w + VH_WORDS);
+    // counts and masses of this thread's slice of the list
+    const int e0 = (int)((long long)n * tid / FILT_BT), e1 = (int)((long long)n * (tid + 1) / FILT_BT);
+    unsigned cs = 0u;
+    unsigned long long ms = 0ull;
+    for (int e = e0; e < e1; ++e) {
+        const uint32_t i = list[e];
+        const uint32_t x = w[vh_phys(i)];
+        cs += (x >> 16) + (x & 0xFFFFu);
+        ms += vh_mass(x >> 16, 2 * i + 1, s, m) + vh_mass(x & 0xFFFFu, 2 * i, s, m);
+    }
+    unsigned c0, ctot;
+    unsigned long long m0, mtot;
+    vh_scan2(cs, ms, &c0, &m0, &ctot, &mtot, fs);
+    if (V > 65535 && ctot != (unsigned)V) return false;   // a counter wrapped (the same in every thread)
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    // top-k: the first key (from the top) where the running count reaches K
+    if (tid == 0) { fs.sel = 0; fs.at = mtot; }          // top-p alone: every key is kept
+    __syncthreads();
+    if (use_k && c0 < (unsigned)K && c0 + cs >= (unsigned)K) {
+        unsigned c = c0;
+        unsigned long long mm = m0;
+        for (int e = e0; e < e1; ++e) {
+            const uint32_t i = list[e];
+            const uint32_t x = w[vh_phys(i)];
+            const unsigned ch = x >> 16, cl = x & 0xFFFFu;
+            c += ch;
+            mm += vh_mass(ch, 2 * i + 1, s, m);
+            if (c >= (unsigned)K) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
+            c += cl;
+            mm += vh_mass(cl, 2 * i, s, m);
+            if (c >= (unsigned)K) { fs.sel = (int)(2 * i); fs.at = mm; break; }
         }
     }
     __syncthreads();
-    if (V > 65535) {                                   // a wrapped counter loses 65535 from the total
-        vh_scan(w, 0u, false, s, m, INFINITY, fs);
-        if (fs.at != (unsigned long long)V) return false;
+    uint32_t t = (uint32_t)fs.sel;
+    const unsigned long long zk = fs.at;
+    unsigned long long z = zk;
+    if (use_p) {
+        // the first key where the running mass reaches top_p of the kept mass
+        // (a key >= the top-k key, since the running mass there is zk)
+        const double target = (double)Pp * (double)zk;
+        __syncthreads();
+        if (tid == 0) fs.sel = -1;
+        __syncthreads();
+        if ((double)m0 < target && (double)(m0 + ms) >= target) {
+            unsigned long long mm = m0;
+            for (int e = e0; e < e1; ++e) {
+                const uint32_t i = list[e];
+                const uint32_t x = w[vh_phys(i)];
+                mm += vh_mass(x >> 16, 2 * i + 1, s, m);
+                if ((double)mm >= target) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
+                mm += vh_mass(x & 0xFFFFu, 2 * i, s, m);
+                if ((double)mm >= target) { fs.sel = (int)(2 * i); fs.at = mm; break; }
+            }
+        }
+        __syncthreads();
+        if (fs.sel >= 0) {
+            t = (uint32_t)fs.sel;
+            z = fs.at;
+        }
     }
-    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
-    uint32_t t = 0u;
-    if (use_k) t = (uint32_t)vh_scan(w, 0u, false, s, m, (double)K, fs);
-    // one mass scan: the top-k set's (or the row's) mass, and where top_p of it is reached
-    const int tp = vh_scan(w, t, true, s, m, use_p ? -(double)Pp : INFINITY, fs);
-    unsigned long long z = fs.at;
-    if (use_p && tp >= 0) t = (uint32_t)tp;
     out->theta = key_value<SPEC_BF16>(t);
     out->on = 1;
     out->Z = (double)z / FIX_ONE;
@@ -2467,9 +2579,11 @@ __device__ bool filter_row_vh(const char* row, int V, float s, float m, int K, f
 }
 
 // Filter thresholds of every row of a chain round, one CTA per (sequence,
-// row): target rows 0..gamma, then the draft-logit rows.  Needs the rows'
-// maxima from the statistics (waits for them); the finalize kernel that
-// follows reads the records.
+// row): target rows 0..gamma, then the draft-logit rows.  A bf16 row's value
+// histogram needs only the logits, so it is built before waiting for the
+// statistics (the rows' maxima, which the masses are relative to).  Every CTA
+// waits before it exits, so the finalize kernel that follows (and reads the
+// records and the statistics) waits for the statistics through this kernel.
 template <int TDT, int DDT, int DK>
 __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     __shared__ FiltShared fs;
@@ -2477,7 +2591,6 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
     pdl_trigger();
-    pdl_wait();
     const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
     const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
     FiltRec* out = P.filt + (size_t)b * P.R + r;
@@ -2485,13 +2598,22 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     const float Pp = P.top_p ? P.top_p[b] : 1.f;
     const float T = P.temperature[b];
     if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
+        pdl_wait();
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
         return;
     }
     if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
+        pdl_wait();
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
+    const bool tgt = r <= P.gamma;
+    const char* row = tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
+                          : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
+    const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
+    uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
+    const int n = vh ? vh_build(row, P.V, fs, w) : 0;
+    pdl_wait();
     const int E = P.nch * SPC;
     if (threadIdx.x < 32) {
         float m;
@@ -2506,14 +2628,9 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     }
     const float s = scale_of(T), m = msh;
     FiltRec rec;
-    if (r <= P.gamma) {
-        const char* row = P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride;
-        if (TDT != SPEC_BF16 || !filter_row_vh(row, P.V, s, m, K, Pp, fs, reinterpret_cast<uint32_t*>(dyn), &rec))
-            rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
-    } else {
-        const char* row = P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
-        if (DDT != SPEC_BF16 || !filter_row_vh(row, P.V, s, m, K, Pp, fs, reinterpret_cast<uint32_t*>(dyn), &rec))
-            rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
+    if (!vh || !vh_select(P.V, n, s, m, K, Pp, fs, w, &rec)) {
+        if (tgt) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
+        else rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
     }
     if (threadIdx.x == 0) *out = rec;
 }
@@ -3461,6 +3578,28 @@ unsigned stats_grid(long long items, int occ) {
     return (unsigned)((items + per_cta - 1) / per_cta);
 }
 
+// Launch a kernel as a programmatic dependent of the kernel enqueued before it
+// on `st` (the statistics kernel, a filter or level kernel): it may start
+// while that kernel drains and waits for it (griddepcontrol.wait) before
+// reading what that kernel writes.
+template <class K>
+spec_status launch_dependent(K kernel, unsigned grid, unsigned block, size_t smem, const Params& P,
+                             cudaStream_t st, const char* what) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, P);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return launched(what);
+}
+
 template <int MODE, int TDT, int DDT>
 spec_status launch_stats(const Params& P, cudaStream_t st) {
     auto kern = k_stats<MODE, TDT, DDT>;
@@ -3484,25 +3623,6 @@ bool allow_stage(K kernel) {
            cudaSuccess;
 }
 
-// Launch a finalize kernel as a programmatic dependent of the statistics
-// kernel just enqueued on `st`.
-template <class K>
-spec_status launch_dependent(K kernel, unsigned grid, unsigned block, size_t smem, const Params& P,
-                             cudaStream_t st, const char* what) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, P);
-    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
-    return launched(what);
-}
 
 // Bytes of one sequence's statistics block, or 0 when it is not staged.
 inline int stats_stage_bytes(const Params& P, int rows, size_t limit) {
