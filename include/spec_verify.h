@@ -417,8 +417,8 @@ spec_status spec_verify_tree_sample_lazy(int B, int N, int V, int max_depth,
  *      tokens, out_num_accepted, p/q diagnostics, and the per-sequence state
  *      the next steps read from the workspace;
  *   3. spec_vp_chain_residual -> mass_out [B] f64, the shard's part of the
- *      mass of the last token's distribution; all-gather into mass_all
- *      [world, B];
+ *      mass of the last token's distribution (its chunk masses stay in the
+ *      workspace for step 4); all-gather into mass_all [world, B];
  *   4. spec_vp_chain_sample -> tok_out [B] int32: the global token id on the
  *      rank whose shard holds u*S, -1 elsewhere; all-reduce MAX;
  *   5. spec_vp_chain_finish writes the reduced token at position k of

@@ -109,6 +109,7 @@ struct Params {
     const int32_t* top_k;          // [B], nullable (0 = off)
     const float* top_p;            // [B], nullable (1 = off)
     struct FiltRec* filt;          // [B][R]            (per-row threshold and kept mass)
+    double* vp_cm;                 // [B][nch]          (vocabulary-parallel: chunk masses of the shard's residual)
 };
 
 // Top-k / top-p filter of one row: keep logits >= theta; Z = the kept mass in
@@ -2806,20 +2807,65 @@ __global__ void __launch_bounds__(NT) k_vp_rows(const Params P, ShardRec* out, i
     }
 }
 
-// Global (m, Z) of row r of sequence b from all shards, in rank order.
-__device__ __forceinline__ void vp_combine(const ShardRec* all, int world, int B, int R2, int b, int r, float* m,
-                                           double* Z, bool* bad) {
-    float mm = -INFINITY;
+// Shards' records are read VP_WB at a time into registers, so that their
+// loads are in flight together rather than one per loop iteration.
+constexpr int VP_WB = 8;
+
+// Threads of the per-sequence residual and sampling kernels (four CTAs per SM).
+constexpr int VP_BT = 256;
+
+// Global (m, Z) of row r of sequence b from all shards, in rank order, and
+// how many shards hold the drafted token (with its value).  `softmax` false
+// (a draft probability row): only the owners.
+__device__ __forceinline__ void vp_combine(const ShardRec* all, int world, int B, int R2, int b, int r, bool softmax,
+                                           float* m, double* Z, bool* bad, int* owners, float* val) {
+    const size_t stride = (size_t)B * R2;
+    const ShardRec* base = all + (size_t)b * R2 + r;
+    float mm = -INFINITY, v = 0.f;
     bool bd = false;
-    for (int w = 0; w < world; ++w) {
-        const ShardRec& x = all[((size_t)w * B + b) * R2 + r];
-        mm = fmaxf(mm, x.m);
-        bd |= x.bad != 0;
+    int own = 0;
+    for (int w0 = 0; w0 < world; w0 += VP_WB) {
+        float xm[VP_WB], xv[VP_WB];
+        int xb[VP_WB], xh[VP_WB];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) {
+                const ShardRec* x = base + (size_t)(w0 + j) * stride;
+                xm[j] = x->m;
+                xv[j] = x->val;
+                xb[j] = x->bad;
+                xh[j] = x->has;
+            }
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) {
+                mm = fmaxf(mm, xm[j]);
+                bd |= xb[j] != 0;
+                if (xh[j]) { ++own; v = xv[j]; }
+            }
+    }
+    *owners = own;
+    *val = v;
+    if (!softmax) {
+        *m = 0.f;
+        *Z = 1.0;
+        *bad = false;
+        return;
     }
     double z = 0.0;
-    for (int w = 0; w < world; ++w) {
-        const ShardRec& x = all[((size_t)w * B + b) * R2 + r];
-        if (x.m > -INFINITY) z += x.Z * exp2((double)x.m - (double)mm);
+    for (int w0 = 0; w0 < world; w0 += VP_WB) {
+        float xm[VP_WB];
+        double xz[VP_WB];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) {
+                const ShardRec* x = base + (size_t)(w0 + j) * stride;
+                xm[j] = x->m;
+                xz[j] = x->Z;
+            }
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world && xm[j] > -INFINITY) z += xz[j] * exp2((double)xm[j] - (double)mm);
     }
     *m = mm;
     *Z = z;
@@ -2840,18 +2886,11 @@ __global__ void __launch_bounds__(NT) k_vp_decide(const Params P, const ShardRec
     if (b >= P.B) return;
     const int gamma = P.gamma, R2 = 2 * gamma + 1;
     for (int r = lane; r < R2; r += 32) {
-        float m;
+        float m, v;
         double Z;
         bool bad;
-        const bool probs_row = DK == DK_PROBS && r > gamma;
-        if (probs_row) { m = 0.f; Z = 1.0; bad = false; }
-        else vp_combine(all, world, P.B, R2, b, r, &m, &Z, &bad);
-        int owners = 0;
-        float v = 0.f;
-        for (int w = 0; w < world; ++w) {
-            const ShardRec& x = all[((size_t)w * P.B + b) * R2 + r];
-            if (x.has) { ++owners; v = x.val; }
-        }
+        int owners;
+        vp_combine(all, world, P.B, R2, b, r, !(DK == DK_PROBS && r > gamma), &m, &Z, &bad, &owners, &v);
         const int i = r <= gamma ? r : r - gamma - 1;
         sm_m[warp][r] = m;
         sm_z[warp][r] = Z;
@@ -2912,7 +2951,7 @@ __global__ void __launch_bounds__(NT) k_vp_decide(const Params P, const ShardRec
 // CTA per sequence -- sum over the shard of max(0, p_k - q_k) (k < gamma), or
 // Z_r 2^(m_r - m) of row gamma (the bonus; no pass over the row).
 template <int TDT, int DDT, int DK>
-__global__ void __launch_bounds__(SEQ_BT) k_vp_residual(const Params P, const ShardRec* all, int rank,
+__global__ void __launch_bounds__(VP_BT, 4) k_vp_residual(const Params P, const ShardRec* all, int rank,
                                                          const VpState* vs, double* mass) {
     __shared__ FinShared sh;
     extern __shared__ __align__(128) unsigned char dyn[];
@@ -2925,7 +2964,8 @@ __global__ void __launch_bounds__(SEQ_BT) k_vp_residual(const Params P, const Sh
         const char* drow = P.drf + ((size_t)b * gamma + st.k) * P.dstride;
         WChainRes<TDT, DDT, DK> wf{trow, drow, st.s, st.mp, (float)(1.0 / st.zp), st.mq,
                                    DK == DK_PROBS ? 0.f : (float)(1.0 / st.zq), P.V};
-        M = row_chunk_masses<CH, SEQ_BT>(wf, P.nch, reinterpret_cast<float*>(dyn), sh);
+        M = row_chunk_masses<CH, VP_BT>(wf, P.nch, reinterpret_cast<float*>(dyn), sh);
+        for (int c = threadIdx.x; c < P.nch; c += VP_BT) P.vp_cm[(size_t)b * P.nch + c] = sh.M[c];
     } else if (st.k == gamma) {
         const ShardRec& x = all[((size_t)rank * P.B + b) * R2 + gamma];
         M = x.m > -INFINITY ? x.Z * exp2((double)x.m - (double)st.mp) : 0.0;
@@ -2939,21 +2979,36 @@ __global__ void __launch_bounds__(SEQ_BT) k_vp_residual(const Params P, const Sh
 __device__ __forceinline__ int vp_owner(const double* ms, int world, int B, int b, double u, double* t_local,
                                         double* S) {
     double tot = 0.0;
-    for (int w = 0; w < world; ++w) tot += ms[(size_t)w * B + b];
+    for (int w0 = 0; w0 < world; w0 += VP_WB) {
+        double x[VP_WB];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) x[j] = ms[(size_t)(w0 + j) * B + b];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) tot += x[j];
+    }
     *S = tot;
     if (!(tot > 0.0)) return -1;
     const double t = u * tot;
     double c = 0.0;
     int last = -1;
     double before_last = 0.0;
-    for (int w = 0; w < world; ++w) {
-        const double x = ms[(size_t)w * B + b];
-        if (x > 0.0) {
-            if (t < c + x) { *t_local = t - c; return w; }
-            last = w;
-            before_last = c;
-        }
-        c += x;
+    for (int w0 = 0; w0 < world; w0 += VP_WB) {
+        double x[VP_WB];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) x[j] = ms[(size_t)(w0 + j) * B + b];
+#pragma unroll
+        for (int j = 0; j < VP_WB; ++j)
+            if (w0 + j < world) {
+                if (x[j] > 0.0) {
+                    if (t < c + x[j]) { *t_local = t - c; return w0 + j; }
+                    last = w0 + j;
+                    before_last = c;
+                }
+                c += x[j];
+            }
     }
     *t_local = t - before_last;
     return last;
@@ -2965,7 +3020,7 @@ __device__ __forceinline__ int vp_owner(const double* ms, int world, int B, int 
 // write -1.  An empty residual (rounding only) draws from p_k instead, with
 // the shards' masses of p_k taken from the statistics.
 template <int TDT, int DDT, int DK>
-__global__ void __launch_bounds__(SEQ_BT) k_vp_sample(const Params P, const ShardRec* all, int world, int rank,
+__global__ void __launch_bounds__(VP_BT, 4) k_vp_sample(const Params P, const ShardRec* all, int world, int rank,
                                                        int off, const VpState* vs, const double* mass_all,
                                                        int32_t* tok) {
     __shared__ FinShared sh;
@@ -2983,7 +3038,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_vp_sample(const Params P, const Shar
     int owner = vp_owner(mass_all, world, P.B, b, u, &tl, &S);
     bool from_p = st.k == gamma;
     if (owner < 0 && st.k < gamma) {                 // empty residual: draw from p_k
-        for (int w = threadIdx.x; w < world; w += SEQ_BT) {
+        for (int w = threadIdx.x; w < world; w += VP_BT) {
             const ShardRec& x = all[((size_t)w * P.B + b) * R2 + st.k];
             pk[w] = x.m > -INFINITY ? x.Z * exp2((double)x.m - (double)st.mp) : 0.0;
         }
@@ -2998,14 +3053,16 @@ __global__ void __launch_bounds__(SEQ_BT) k_vp_sample(const Params P, const Shar
         float* wpw = reinterpret_cast<float*>(dyn);
         if (from_p) {
             WTarget<TDT> wf{trow, st.s, st.mp, nullptr, 0, P.V};
-            row_chunk_masses<CH, SEQ_BT>(wf, P.nch, wpw, sh);
-            y = draw_from_chunks<CH, SEQ_BT>(wf, P.nch, P.V, tl, (float)u, sh);
+            row_chunk_masses<CH, VP_BT>(wf, P.nch, wpw, sh);
+            y = draw_from_chunks<CH, VP_BT>(wf, P.nch, P.V, tl, (float)u, sh);
         } else {
             const char* drow = P.drf + ((size_t)b * gamma + st.k) * P.dstride;
             WChainRes<TDT, DDT, DK> wf{trow, drow, st.s, st.mp, (float)(1.0 / st.zp), st.mq,
                                        DK == DK_PROBS ? 0.f : (float)(1.0 / st.zq), P.V};
-            row_chunk_masses<CH, SEQ_BT>(wf, P.nch, wpw, sh);
-            y = draw_from_chunks<CH, SEQ_BT>(wf, P.nch, P.V, tl, (float)u, sh);
+            // the chunk masses k_vp_residual computed over the same weights
+            for (int c = threadIdx.x; c < P.nch; c += VP_BT) sh.M[c] = P.vp_cm[(size_t)b * P.nch + c];
+            __syncthreads();
+            y = draw_from_chunks<CH, VP_BT>(wf, P.nch, P.V, tl, (float)u, sh);
         }
         if (y >= 0) y += off;
     }
@@ -3469,7 +3526,7 @@ spec_status fail(spec_status st, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, vp, total;
+    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, vp, vpcm, total;
     int rej_cap;
     int R, nch_max;
 };
@@ -3499,6 +3556,9 @@ Layout make_layout(int entry, int B, int rows, int V) {
     // vocabulary-parallel chain: the decision's per-sequence state
     L.vp = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(VpState) * (size_t)B);
+    // ... and the chunk masses of the shard's residual (reused by the draw)
+    L.vpcm = off;
+    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(double) * (size_t)B * nch);
     L.total = off;
     return L;
 }
@@ -3556,6 +3616,7 @@ void bind_ws(Params& P, void* ws, const Layout& L) {
     P.lz_list = reinterpret_cast<int*>(w + L.lz_list);
     P.lz_count = reinterpret_cast<unsigned*>(w + L.lz_count);
     P.filt = reinterpret_cast<FiltRec*>(w + L.filt);
+    P.vp_cm = reinterpret_cast<double*>(w + L.vpcm);
 }
 
 spec_status launched(const char* what) {
@@ -4161,16 +4222,16 @@ spec_status vp_stats_launch(Params P, ShardRec* rec, int off, cudaStream_t st) {
 template <int TDT, int DDT, int DK>
 spec_status vp_residual_launch(Params P, const ShardRec* all, int rank, const VpState* vs, double* mass,
                                cudaStream_t st) {
-    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
-    k_vp_residual<TDT, DDT, DK><<<(unsigned)P.B, SEQ_BT, wpw, st>>>(P, all, rank, vs, mass);
+    const size_t wpw = (size_t)P.nch * (VP_BT / 32) * sizeof(float);
+    k_vp_residual<TDT, DDT, DK><<<(unsigned)P.B, VP_BT, wpw, st>>>(P, all, rank, vs, mass);
     return launched("k_vp_residual");
 }
 
 template <int TDT, int DDT, int DK>
 spec_status vp_sample_launch(Params P, const ShardRec* all, int world, int rank, int off, const VpState* vs,
                              const double* mass_all, int32_t* tok, cudaStream_t st) {
-    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
-    k_vp_sample<TDT, DDT, DK><<<(unsigned)P.B, SEQ_BT, wpw, st>>>(P, all, world, rank, off, vs, mass_all, tok);
+    const size_t wpw = (size_t)P.nch * (VP_BT / 32) * sizeof(float);
+    k_vp_sample<TDT, DDT, DK><<<(unsigned)P.B, VP_BT, wpw, st>>>(P, all, world, rank, off, vs, mass_all, tok);
     return launched("k_vp_sample");
 }
 
