@@ -362,15 +362,46 @@ def cpu_baseline(wid, inp, seconds, nthreads=None):
     per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4, 7: 16}[wid]))
     rows = None if per == B else list(range(per))
     elapsed = 0.0
+    out = None
     while n == 0 or elapsed < seconds:
         t1 = time.perf_counter()
-        fn(inp, rows, nthreads=cores)
+        out = fn(inp, rows, nthreads=cores)
         elapsed += time.perf_counter() - t1
         n += 1
     rounds = n * per / B
-    return {"value": rounds / elapsed, "unit": "rounds/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x {per} of {B} sequences of one round (whole sequences), fp64 C oracle, "
-                      f"OpenMP over sequences, {elapsed:.1f} s of CPU time; rounds/s scaled by {per}/{B}"}
+    res = {"value": rounds / elapsed, "unit": "rounds/s", "cores": cores, "kind": "oracle",
+           "sample": f"{n} x {per} of {B} sequences of one round (whole sequences), fp64 C oracle, "
+                     f"OpenMP over sequences, {elapsed:.1f} s of CPU time; rounds/s scaled by {per}/{B}"}
+    return res, out, rows
+
+
+def sample_parity(wid, inp, o, rows, ws):
+    """The CUDA path's result on the sequences the oracle baseline computed
+    (the same bytes): identical accepted lengths and tokens except on the
+    sequences the oracle flags as near-ties, diagnostics within 1e-5."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity
+    if wid == 7:
+        return {"checked": False, "why": "one rank of a vocabulary-parallel round; parity of the sharded path "
+                                         "is in the GPU tests (all shards emulated on one GPU)"}
+    n = inp.B if rows is None else len(rows)
+    try:
+        if wid in (0, 1, 4):
+            fl, bad, _ = parity.compare_chain(parity.gpu_chain(inp, workspace=ws), o, inp.gamma, rows)
+        elif wid == 6:
+            g = parity.gpu_chain_filtered(inp, inp.meta["top_k"], inp.meta["top_p"], workspace=ws)
+            fl, bad, _ = parity.compare_chain(g, o, inp.gamma, rows)
+        elif wid == 2:
+            fl, bad, _ = parity.compare_tree(parity.gpu_greedy(inp, workspace=ws), o, rows)
+        elif wid == 3:
+            fl, bad, _ = parity.compare_tree(parity.gpu_sample(inp, workspace=ws), o, rows, sample=True)
+        else:
+            fl, bad, _ = parity.compare_mss(parity.gpu_mss(inp, workspace=ws), o, rows)
+        diag = True
+    except AssertionError as e:
+        return {"checked": True, "sequences": n, "diagnostics_within_tolerance": False, "error": str(e)[:200]}
+    return {"checked": True, "sequences": n, "identical_or_flagged": n - bad, "flagged_near_ties": fl,
+            "mismatches": bad, "diagnostics_within_tolerance": diag}
 
 
 # ----------------------------------------------------------------------------- main
@@ -405,7 +436,7 @@ def run_reference(args, ws_, rank):
     inp = make_inputs(args.workload, 0, dev)
     steps = max(1, args.steps)
     # each step is a bounded sample of the workload (see cpu_baseline)
-    cb = cpu_baseline(args.workload, inp, seconds=min(60.0, max(5.0, 0.02 * steps)))
+    cb, _, _ = cpu_baseline(args.workload, inp, seconds=min(60.0, max(5.0, 0.02 * steps)))
     cfg = describe(args.workload, inp)
     line = {"impl": "reference", "metric": "verify rounds/s", "value": cb["value"], "unit": "rounds/s",
             "n_gpus": ws_, "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
@@ -561,9 +592,11 @@ def main():
         "e2e": e2e, "gpu_launches": K * kps, "clocks": sampler.summary(), "lazy": lazy,
     }
     if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wid, first, args.cpu_seconds)
-        one = cpu_baseline(wid, first, args.cpu_seconds / 4, nthreads=1)
-        line["cpu_baseline"]["value_1thread"] = one["value"]
+        cb, o, rows = cpu_baseline(wid, first, args.cpu_seconds)
+        one, _, _ = cpu_baseline(wid, first, args.cpu_seconds / 4, nthreads=1)
+        cb["value_1thread"] = one["value"]
+        cb["parity"] = sample_parity(wid, first, o, rows, ws)
+        line["cpu_baseline"] = cb
     elif rank == 0:
         line["cpu_baseline"] = None
     if rank == 0:
