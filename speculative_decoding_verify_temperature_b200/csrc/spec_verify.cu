@@ -719,14 +719,29 @@ __device__ __forceinline__ void chunk_group_sums(const WF& wf, int c, float (&gs
             }
         }
     } else {
+        // the row's last chunk: whole groups two at a time, the one group
+        // that straddles V (and the groups past it) bounds-checked
+        constexpr int PB = GPT < 2 ? GPT : 2;
 #pragma unroll
-        for (int k = 0; k < GPT; ++k) {
-            gs[k] = 0.f;
-            const int64_t e0 = c0 + (int64_t)(k * BT + threadIdx.x) * 8;
-            if (e0 < wf.V) {
+        for (int k0 = 0; k0 < GPT; k0 += PB) {
+            typename WF::Raw raw[PB];
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const int64_t e0 = c0 + (int64_t)((k0 + i) * BT + threadIdx.x) * 8;
+                if (e0 + 8 <= wf.V) wf.load(e0, raw[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < PB; ++i) {
+                const int64_t e0 = c0 + (int64_t)((k0 + i) * BT + threadIdx.x) * 8;
                 float w[8];
-                wf.group(e0, w);
-                gs[k] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+                gs[k0 + i] = 0.f;
+                if (e0 + 8 <= wf.V) {
+                    wf.weights(e0, raw[i], w);
+                    gs[k0 + i] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+                } else if (e0 < wf.V) {
+                    wf.group(e0, w);
+                    gs[k0 + i] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+                }
             }
         }
     }
@@ -2811,7 +2826,9 @@ __global__ void __launch_bounds__(NT) k_vp_rows(const Params P, ShardRec* out, i
 // loads are in flight together rather than one per loop iteration.
 constexpr int VP_WB = 8;
 
-// Threads of the per-sequence residual and sampling kernels (four CTAs per SM).
+// Threads of the per-sequence residual and sampling kernels (the residual
+// kernel four CTAs per SM; the sampling kernel, where only the owner shard's
+// CTAs draw, two with more registers).
 constexpr int VP_BT = 256;
 
 // Global (m, Z) of row r of sequence b from all shards, in rank order, and
@@ -3020,7 +3037,7 @@ __device__ __forceinline__ int vp_owner(const double* ms, int world, int B, int 
 // write -1.  An empty residual (rounding only) draws from p_k instead, with
 // the shards' masses of p_k taken from the statistics.
 template <int TDT, int DDT, int DK>
-__global__ void __launch_bounds__(VP_BT, 4) k_vp_sample(const Params P, const ShardRec* all, int world, int rank,
+__global__ void __launch_bounds__(VP_BT, 2) k_vp_sample(const Params P, const ShardRec* all, int world, int rank,
                                                        int off, const VpState* vs, const double* mass_all,
                                                        int32_t* tok) {
     __shared__ FinShared sh;
