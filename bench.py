@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -406,14 +407,24 @@ def sample_parity(wid, inp, o, rows, ws):
 
 # ----------------------------------------------------------------------------- main
 
+def kernel_source_hash(text: str) -> str:
+    """First 16 hex digits of the SHA-256 of the kernel source with its comments
+    and white space removed (a change to the code changes it, a change to a
+    comment does not)."""
+    code = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    code = re.sub(r"//[^\n]*", "", code)
+    code = re.sub(r"\s+", "", code)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def profile_traffic(wid):
     """Per-launch DRAM traffic of the row kernel from a committed ncu summary,
-    valid only while the kernel source is unchanged."""
+    valid only while the kernel source's code is unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     src = os.path.join(ROOT, "speculative_decoding_verify_temperature_b200", "csrc", "spec_verify.cu")
     try:
         rec = json.load(open(path)).get(str(wid))
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        h = kernel_source_hash(open(src, encoding="utf-8").read())
         if rec and rec.get("source_sha256_16") == h:
             return rec.get("dram_bytes_per_launch")
     except Exception:

@@ -2159,11 +2159,13 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
 // The filtered target distribution keeps the logits >= theta: theta_k = the
 // top_k-th largest logit (ties kept), then, within that set, theta_p = the
 // largest logit whose set {l >= theta_p} carries a top_p share of the set's
-// mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds come from a radix
-// descent over order-preserving keys of the logits (16 bits for bf16, 32 for
-// f32, -0 folded onto +0), 8 bits per pass over the row: counts for top-k,
-// fixed-point masses (2^-40 units, integer atomics, so the sums do not depend
-// on the order of the additions) for top-p and Z'.
+// mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds are found over
+// order-preserving keys of the logits (-0 folded onto +0): for bf16 rows an
+// exact histogram of the 65536 possible keys (vh_build / vh_select), for f32
+// rows (and a bf16 row whose histogram counter would wrap) a radix descent of
+// 12 + 12 + 8 bit digits (filter_row).  Counts decide top-k; masses are fixed
+// point (2^-40 units, integer sums, so they do not depend on the order of the
+// additions) and decide top-p and Z'.
 
 constexpr int FILT_BT = 1024;
 constexpr double FIX_ONE = 1099511627776.0;      // 2^40
