@@ -1,6 +1,6 @@
 // spec_verify.cu -- sm_100a kernels and C ABI of libspecverify (see include/spec_verify.h).
 //
-// Data path (one call = one verify round over B sequences, two launches):
+// Data path (one call = one verify round over B sequences):
 //
 //   k_stats     streams every logit row once.  The (sequence, row, chunk) work
 //               items -- a chunk is 128 threads x 8 x 16-byte vectors = 16 KB
@@ -9,18 +9,28 @@
 //               statistic: online softmax (max m, sum 2^(x - m), x = l*log2e/T)
 //               for the sampling entry points, (max value, lowest index) for
 //               greedy.  No atomics, no fences: the next kernel in stream order
-//               reads the statistics.
+//               (a programmatic dependent) reads the statistics.
 //
-//   k_chain_final / k_tree_final   per-sequence finalisation: combine the
-//               statistics per row (fp64 across chunks), gather the drafted
-//               tokens' probabilities, take the accept/reject decisions or walk
-//               the tree, and draw the last token by inverse CDF -- the chunk
-//               holding u*S is located from chunk masses, then rescanned with
-//               coalesced 8-element groups and a block-wide fp64 prefix scan.
-//               The chain residual max(0, p_k - q_k) over several chunks is
-//               summed by one CTA per chunk; the last to arrive (atomicAdd after
-//               __threadfence, no spin-wait) draws and resets its counter, so
-//               workspaces need no per-call memset.
+//   finalisation, one dependent launch per call:
+//     k_chain_final_pair  chain, a cluster of two CTAs per sequence: both take
+//               the decision, each stages half of the rejected row pair with
+//               bulk copies and scans its residual mass; the halves meet
+//               through distributed shared memory and one CTA draws.
+//     k_chain_final_row   chain, one CTA per sequence, the row pair staged.
+//     k_chain_final       chain, one CTA per (sequence, slice of chunks); the
+//               last to arrive (atomicAdd after __threadfence, no spin-wait)
+//               draws and resets its counter.
+//     k_tree_final        trees: greedy walk, target-only sibling walk, or
+//               multi-step speculative sampling with draft distributions.
+//   The last token is drawn by inverse CDF: the chunk holding u*S is located
+//   from chunk masses, then rescanned with coalesced 8-element groups and a
+//   block-wide fp64 prefix scan.
+//
+//   Variants on the same statistics:
+//     k_filter + k_chain_final_filt     top-k / top-p filtered chain verify.
+//     k_lz_*                            row-on-demand (lazy) level walk.
+//     k_vp_*                            vocabulary-parallel chain verify: the
+//               per-shard device steps between the callers' collectives.
 //
 // Nothing here is a dense contraction, so no tensor cores: the path is a
 // streaming reduction bounded by HBM bandwidth, with the exp2 unit (MUFU, 16
