@@ -580,7 +580,7 @@ def main():
     draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6, 7) else first.N - 1)
 
     # --- end to end through the binding with host buffers
-    e2e = run_e2e(wid, first, ws, args.e2e_steps, dev) if wid != 7 else {
+    e2e = run_e2e(wid, first, ws, args.e2e_steps, dev, ws_) if wid != 7 else {
         "value": None, "unit": "rounds/s", "note": "one rank of a vocabulary-parallel round: no single-GPU host path"}
 
     # --- the row-on-demand entry point on the same input sets
@@ -658,9 +658,11 @@ def run_lazy(wid, sets, ws, steps, alg, world, dev):
             "achieved_gbs_on_bytes_read": round(read / (ms / n / 1e3) / 1e9, 1)}
 
 
-def run_e2e(wid, inp, ws, steps, dev):
+def run_e2e(wid, inp, ws, steps, dev, world=1):
     """Same metric through the binding: every step copies this round's inputs from
-    pinned host memory, verifies, and copies the outputs back."""
+    pinned host memory, verifies, and copies the outputs back.  With several
+    ranks, the whole job's rounds/s over the slowest rank's time, and the bytes
+    all ranks copy per step."""
     import torch
     host = {k: v.detach().cpu().pin_memory() for k, v in vars(inp).items() if isinstance(v, torch.Tensor)}
     meta = getattr(inp, "meta", None) or {}
@@ -691,15 +693,17 @@ def run_e2e(wid, inp, ws, steps, dev):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    return {"value": round(steps / (ms / 1e3), 2), "unit": "rounds/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps}
+    ms = reduce_max_ms(e0.elapsed_time(e1), world, dev)
+    return {"value": round(job_value(steps, world, ms), 2), "unit": "rounds/s", "h2d_bytes_per_step": h2d * world,
+            "d2h_bytes_per_step": d2h * world, "steps": steps}
 
 
 if __name__ == "__main__":
