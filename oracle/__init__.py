@@ -58,6 +58,9 @@ def lib():
         L.oracle_tree_sample.restype = None
         L.oracle_tree_sample.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                                          f32, f32, P, P, P, P, P, P, P, i32]
+        L.oracle_tree_sample_filtered.restype = None
+        L.oracle_tree_sample_filtered.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
+                                                  f32, f32, P, P, P, P, P, P, P, P, P, P, i32]
         L.oracle_chain_filtered.restype = None
         L.oracle_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
                                             P, P, P, P, P, P, P, P, P, P, P, P, P, P, i32]
@@ -187,9 +190,11 @@ def tree_greedy(target, tokens, parents, max_depth: int, V=None, nthreads: int =
 
 def tree_sample(target, tokens, parents, temperature, coins, final_u, max_depth: int,
                 draft_probs=None, threshold_single: float = 1.0, threshold_acc: float = 1.0,
-                V=None, nthreads: int = 0) -> dict:
+                V=None, nthreads: int = 0, top_k=None, top_p=None) -> dict:
     """Target-only tree sampling.  ``coins`` is ``[B, N]`` (coin of the visited node),
-    ``draft_probs`` ``None`` (zeros) or f32 ``[B, N, dstride]``."""
+    ``draft_probs`` ``None`` (zeros) or f32 ``[B, N, dstride]``.  With ``top_k`` /
+    ``top_p`` (per sequence, ``[B]``) every node's target row is top-k / top-p
+    filtered first (the result then has ``fmargin``)."""
     target = _c(target)
     B, N, ts = target.shape
     V = ts if V is None else int(V)
@@ -214,13 +219,26 @@ def tree_sample(target, tokens, parents, temperature, coins, final_u, max_depth:
     )
     if B == 0:
         return out
-    lib().oracle_tree_sample(B, N, V, max_depth, _ptr(target), _dtype_code(target), ts,
-                             _ptr(tokens), _ptr(parents), _ptr(temperature), _ptr(coins),
-                             _ptr(final_u), _ptr(draft_probs), dstride,
-                             float(threshold_single), float(threshold_acc),
-                             _ptr(out["accept_index"]), _ptr(out["tokens"]),
-                             _ptr(out["num_accepted"]), _ptr(out["pchild"]), _ptr(out["S"]),
-                             _ptr(out["dmargin"]), _ptr(out["cmargin"]), int(nthreads))
+    if top_k is None and top_p is None:
+        lib().oracle_tree_sample(B, N, V, max_depth, _ptr(target), _dtype_code(target), ts,
+                                 _ptr(tokens), _ptr(parents), _ptr(temperature), _ptr(coins),
+                                 _ptr(final_u), _ptr(draft_probs), dstride,
+                                 float(threshold_single), float(threshold_acc),
+                                 _ptr(out["accept_index"]), _ptr(out["tokens"]),
+                                 _ptr(out["num_accepted"]), _ptr(out["pchild"]), _ptr(out["S"]),
+                                 _ptr(out["dmargin"]), _ptr(out["cmargin"]), int(nthreads))
+        return out
+    tk = _c(np.zeros(B, np.int32) if top_k is None else top_k, np.int32).reshape(B)
+    tp = _c(np.ones(B, np.float32) if top_p is None else top_p, np.float32).reshape(B)
+    out["fmargin"] = np.empty(B, np.float64)
+    lib().oracle_tree_sample_filtered(B, N, V, max_depth, _ptr(target), _dtype_code(target), ts,
+                                      _ptr(tokens), _ptr(parents), _ptr(temperature), _ptr(coins),
+                                      _ptr(final_u), _ptr(draft_probs), dstride,
+                                      float(threshold_single), float(threshold_acc), _ptr(tk), _ptr(tp),
+                                      _ptr(out["accept_index"]), _ptr(out["tokens"]),
+                                      _ptr(out["num_accepted"]), _ptr(out["pchild"]), _ptr(out["S"]),
+                                      _ptr(out["dmargin"]), _ptr(out["cmargin"]), _ptr(out["fmargin"]),
+                                      int(nthreads))
     return out
 
 

@@ -519,15 +519,17 @@ void oracle_tree_greedy(int B, int N, int V, int max_depth,
  * Outputs as oracle_tree_greedy; out_pchild[b*N+n] = p_parent(n)(tokens[n])
  * for n >= 1 and 0 for the root; margins as oracle_chain.
  */
-void oracle_tree_sample(int B, int N, int V, int max_depth,
-                        const void* target, int tdt, int64_t t_row_stride,
-                        const int32_t* tokens, const int32_t* parents,
-                        const float* temperature, const float* coins, const float* final_u,
-                        const float* draft_probs, int64_t dp_row_stride,
-                        float threshold_single, float threshold_acc,
-                        int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,
-                        double* out_pchild, double* out_S, double* out_dmargin,
-                        double* out_cmargin, int nthreads) {
+static void tree_sample_impl(int B, int N, int V, int max_depth,
+                             const void* target, int tdt, int64_t t_row_stride,
+                             const int32_t* tokens, const int32_t* parents,
+                             const float* temperature, const float* coins, const float* final_u,
+                             const float* draft_probs, int64_t dp_row_stride,
+                             float threshold_single, float threshold_acc,
+                             const int32_t* top_k, const float* top_p,
+                             int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,
+                             double* out_pchild, double* out_S, double* out_dmargin,
+                             double* out_cmargin, double* out_fmargin, int nthreads) {
+    const int filtered = top_k != NULL || top_p != NULL;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel
@@ -538,6 +540,7 @@ void oracle_tree_sample(int B, int N, int V, int max_depth,
         double* w = (double*)malloc(sizeof(double) * (size_t)V);
         int* depth = (int*)malloc(sizeof(int) * (size_t)N);
         int* rej = (int*)malloc(sizeof(int) * (size_t)N);
+        vj_t* sorted = filtered ? (vj_t*)malloc(sizeof(vj_t) * (size_t)V) : NULL;
 #ifdef _OPENMP
 #pragma omp for schedule(dynamic, 1)
 #endif
@@ -548,11 +551,19 @@ void oracle_tree_sample(int B, int N, int V, int max_depth,
             int32_t* ot = out_tokens + (int64_t)b * (max_depth + 1);
             double T = (double)temperature[b];
             int bad = !temperature_ok(T) || !tree_ok(N, V, max_depth, tk, pa, depth);
+            const int K = top_k ? top_k[b] : 0;
+            const double Pp = top_p ? (double)top_p[b] : 1.0;
+            double fmargin = INFINITY, fm;
             for (int n = 0; n < N && !bad; ++n) {
                 const char* row = (const char*)target +
                     ((int64_t)b * N + n) * t_row_stride * (tdt == OR_F32 ? 4 : 2);
                 if (softmax_T(row, tdt, V, T, P + (int64_t)n * V)) bad = 1;
+                else if (filtered && g_mutation != 19) {              /* 19: tree rows left unfiltered */
+                    if (filter_probs(row, tdt, V, P + (int64_t)n * V, K, Pp, sorted, &fm)) bad = 1;
+                    if (fm < fmargin) fmargin = fm;
+                }
             }
+            if (out_fmargin) out_fmargin[b] = bad ? INFINITY : fmargin;
             fill_i32(ai, max_depth + 1, -1);
             fill_i32(ot, max_depth + 1, -1);
             if (bad) {
@@ -626,7 +637,46 @@ void oracle_tree_sample(int B, int N, int V, int max_depth,
         free(w);
         free(depth);
         free(rej);
+        free(sorted);
     }
+}
+
+void oracle_tree_sample(int B, int N, int V, int max_depth,
+                        const void* target, int tdt, int64_t t_row_stride,
+                        const int32_t* tokens, const int32_t* parents,
+                        const float* temperature, const float* coins, const float* final_u,
+                        const float* draft_probs, int64_t dp_row_stride,
+                        float threshold_single, float threshold_acc,
+                        int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,
+                        double* out_pchild, double* out_S, double* out_dmargin,
+                        double* out_cmargin, int nthreads) {
+    tree_sample_impl(B, N, V, max_depth, target, tdt, t_row_stride, tokens, parents, temperature, coins,
+                     final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc, NULL, NULL,
+                     out_accept_index, out_tokens, out_num_accepted, out_pchild, out_S, out_dmargin,
+                     out_cmargin, NULL, nthreads);
+}
+
+/*
+ * Target-only tree sampling under top-k / top-p filtering: every node's
+ * target row is filtered (filter_probs, the sequence's top_k[b] / top_p[b])
+ * before the walk above uses it, so prob_acc, the thresholds and the final
+ * relu(p_cur - d_cur) all see the filtered distribution; draft_probs rows are
+ * used as given.  out_fmargin[b] = the smallest top-p margin over the rows.
+ */
+void oracle_tree_sample_filtered(int B, int N, int V, int max_depth,
+                                 const void* target, int tdt, int64_t t_row_stride,
+                                 const int32_t* tokens, const int32_t* parents,
+                                 const float* temperature, const float* coins, const float* final_u,
+                                 const float* draft_probs, int64_t dp_row_stride,
+                                 float threshold_single, float threshold_acc,
+                                 const int32_t* top_k, const float* top_p,
+                                 int32_t* out_accept_index, int32_t* out_tokens, int32_t* out_num_accepted,
+                                 double* out_pchild, double* out_S, double* out_dmargin,
+                                 double* out_cmargin, double* out_fmargin, int nthreads) {
+    tree_sample_impl(B, N, V, max_depth, target, tdt, t_row_stride, tokens, parents, temperature, coins,
+                     final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc, top_k, top_p,
+                     out_accept_index, out_tokens, out_num_accepted, out_pchild, out_S, out_dmargin,
+                     out_cmargin, out_fmargin, nthreads);
 }
 
 /*

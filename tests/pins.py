@@ -388,6 +388,8 @@ def _tree_cases(model: ToyModel, prefix, parents):
     N = len(parents)
     target = np.stack([model.p(prefix + path[n])[0] for n in range(N)])
     probs = [model.p(prefix + path[n])[1] for n in range(N)]
+    # p_parent(n)(token_n): what the walk must use for node n
+    pch = np.array([0.0] + [probs[parents[n]][tokens[n]] for n in range(1, N)])
     cases = []
 
     def visit(cur, weight, coins):
@@ -414,22 +416,28 @@ def _tree_cases(model: ToyModel, prefix, parents):
                 for node, val in cc.items():
                     cv[node] = val
                 cases.append(dict(weight=weight * rest * r[j] / S, target=target, tokens=tokens,
-                                  coins=cv, u=np.float32((C[j] - r[j] / 2) / S)))
+                                  coins=cv, u=np.float32((C[j] - r[j] / 2) / S), pch=pch))
 
     visit(0, 1.0, {})
     return cases
 
 
 def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
-                    draft_probs_zero=False, T=1.0, runner=None) -> dict:
+                    draft_probs_zero=False, T=1.0, runner=None, top_k=None, top_p=None) -> dict:
     """Exact distribution of the first K tokens of repeated target-only tree rounds
-    (thresholds 1) against the target's autoregressive distribution."""
+    (thresholds 1) against the target's autoregressive distribution -- with
+    ``top_k`` / ``top_p``, against the filtered target's (filter_definition), the
+    rows handed over unfiltered and the filter left to the verify step."""
+    filt = top_k is not None or top_p is not None
     model = ToyModel(V, seed, T=T)
+    if filt:
+        model = FilteredModel(model, 0 if top_k is None else top_k, 1.0 if top_p is None else top_p)
     parents = np.array(parents, np.int32)
     N = len(parents)
     depth = max(len(p) for p in _paths(parents, np.zeros(N, np.int32)))
     states = {(): 1.0}
     dist = {}
+    fmin, perr = np.inf, 0.0
     while states:
         batch, owners = [], []
         for prefix, w in states.items():
@@ -437,12 +445,20 @@ def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
             batch += cs
             owners += [(prefix, w)] * len(cs)
         m = len(batch)
+        fk = dict(top_k=np.full(m, model.top_k, np.int32), top_p=np.full(m, model.top_p, np.float32)) if filt \
+            else {}
         res = (runner or oracle.tree_sample)(np.stack([c["target"] for c in batch]),
                                  np.stack([c["tokens"] for c in batch]),
                                  np.broadcast_to(parents, (m, N)), np.full(m, model.T, np.float32),
                                  np.stack([c["coins"] for c in batch]),
                                  np.array([c["u"] for c in batch], np.float32), depth,
-                                 draft_probs=np.zeros((m, N, V), np.float32) if draft_probs_zero else None)
+                                 draft_probs=np.zeros((m, N, V), np.float32) if draft_probs_zero else None,
+                                 **fk)
+        if "fmargin" in res:
+            fmin = min(fmin, float(res["fmargin"].min()))
+        if filt:                   # the walk's child probabilities are the filtered ones (f32 logits: 1e-6)
+            perr = max(perr, float(np.abs(np.asarray(res["pchild"])[:, 1:]
+                                          - np.stack([c["pch"] for c in batch])[:, 1:]).max()))
         nxt = {}
         for i, (prefix, w) in enumerate(owners):
             k = int(res["num_accepted"][i])
@@ -457,7 +473,8 @@ def tree_bruteforce(V=3, K=3, seed=5, parents=(-1, 0, 0, 1, 1, 2, 3), tol=1e-12,
         states = nxt
     want = _product_distribution(model, K)
     err = max(abs(dist.get(s, 0.0) - pv) for s, pv in want.items())
-    return dict(ok=err < tol, err=err)
+    err = max(err, sum(v for s, v in dist.items() if s not in want))
+    return dict(ok=err < tol and fmin > 1e-9 and perr < 1e-6, err=err, fmargin=fmin, pchild_err=perr)
 
 
 def tree_chisquare(V=4, K=3, rounds=1_000_000, seed=6, shapes=None, pmin=1e-3, runner=None) -> dict:
@@ -557,7 +574,7 @@ class FilteredModel:
 
     def __init__(self, model: ToyModel, top_k: int, top_p: float):
         self.m, self.top_k, self.top_p = model, top_k, top_p
-        self.V, self.T, self.draft_kind = model.V, model.T, model.draft_kind
+        self.V, self.T, self.draft_kind, self.seed = model.V, model.T, model.draft_kind, model.seed
 
     def p(self, prefix):
         logits, _ = self.m.p(prefix)

@@ -429,6 +429,65 @@ def test_invalid_inputs_mark_sequence():
     assert (g["num_accepted"] == -1).all()
 
 
+# ----------------------------------------------------------------------------- filtered tree sampling
+
+def test_tree_filter_off_is_plain_tree():
+    """Target-only tree sampling with both filters off (top_k 0, top_p 1) is the
+    unfiltered walk bit for bit, with and without draft probabilities."""
+    rng = np.random.default_rng(21)
+    B, V = 6, 40
+    parents = np.array([[-1, 0, 0, 1, 1, 2, 4, 4]] * B, np.int32)
+    N = parents.shape[1]
+    tokens = rng.integers(0, V, (B, N)).astype(np.int32)
+    t = rng.normal(0, 2, (B, N, V)).astype(np.float32)
+    coins = pins._uniform24(rng, (B, N))
+    fu = pins._uniform24(rng, (B,))
+    T = np.full(B, 0.8, np.float32)
+    for dp in (None, rng.dirichlet(np.ones(V), (B, N)).astype(np.float32)):
+        a = oracle.tree_sample(t, tokens, parents, T, coins, fu, 3, draft_probs=dp)
+        b = oracle.tree_sample(t, tokens, parents, T, coins, fu, 3, draft_probs=dp,
+                               top_k=np.zeros(B, np.int32), top_p=np.ones(B, np.float32))
+        for key in ("accept_index", "tokens", "num_accepted", "pchild", "S"):
+            np.testing.assert_array_equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(top_k=2, top_p=None),
+    dict(top_k=None, top_p=0.7),
+    dict(top_k=3, top_p=0.8, V=4, K=2, seed=3, parents=(-1, 0, 0, 1, 2)),
+    dict(top_k=2, top_p=0.9, T=0.7, seed=8, draft_probs_zero=True),
+])
+def test_tree_filtered_bruteforce_lossless(kw):
+    """Filtered target-only tree rounds emit the filtered target's
+    autoregressive distribution exactly ([origins] "In SGLang": the walk keeps
+    whatever target distribution it is given; the filters follow the
+    threshold-form definition written separately in the harness)."""
+    r = pins.tree_bruteforce(**kw)
+    assert r["ok"], (kw, r)
+
+
+def test_tree_topk1_sampling_is_greedy():
+    """top_k = 1 on rows without ties makes every filtered row one-hot at its
+    argmax: a child is accepted iff it carries its parent's argmax, and the last
+    token is the argmax, which is greedy tree verification."""
+    rng = np.random.default_rng(22)
+    B, V = 40, 12
+    parents = np.array([[-1, 0, 0, 0, 1, 1, 2, 3, 5, 5]] * B, np.int32)
+    N = parents.shape[1]
+    t = rng.normal(0, 2, (B, N, V)).astype(np.float32)             # continuous: no ties
+    am = t.argmax(axis=2)
+    tokens = rng.integers(0, V, (B, N)).astype(np.int32)
+    hit = rng.random((B, N)) < 0.6                                   # many children match their parent's argmax
+    for n in range(1, N):
+        tokens[hit[:, n], n] = am[hit[:, n], parents[0, n]]
+    g = oracle.tree_greedy(t, tokens, parents, 3)
+    s = oracle.tree_sample(t, tokens, parents, np.full(B, 0.9, np.float32), pins._uniform24(rng, (B, N)),
+                           pins._uniform24(rng, (B,)), 3, top_k=np.ones(B, np.int32))
+    np.testing.assert_array_equal(s["num_accepted"], g["num_accepted"])
+    np.testing.assert_array_equal(s["accept_index"], g["accept_index"])
+    np.testing.assert_array_equal(s["tokens"], g["tokens"])
+
+
 # ----------------------------------------------------------------------------- the pins bite
 
 MUTATIONS = {
@@ -451,6 +510,8 @@ MUTATIONS = {
     16: ("top-k keeps one group too few", lambda: pins.filter_properties()),
     17: ("top-p drops the group that reaches top_p", lambda: pins.filter_properties()),
     18: ("draft logits left unfiltered", lambda: pins.chain_filtered_bruteforce()),
+    19: ("tree rows left unfiltered", lambda: pins.tree_bruteforce(V=4, K=2, seed=3, top_k=2, top_p=0.8,
+                                                                    parents=(-1, 0, 0, 1, 2))),
 }
 
 
