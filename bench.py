@@ -41,7 +41,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
+    ap.add_argument("--workload", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7, 8])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -94,6 +94,8 @@ def make_inputs(wid: int, rnd: int, device, rank: int = 0):
         return wl.tree_config5(r, device)
     if wid == 6:
         return wl.chain_config6(r, device)
+    if wid == 8:
+        return wl.tree_config8(r, device)
     if wid == 7:
         return wl.chain_config4(r, device)
     return wl.chain_config4(r, device)
@@ -202,6 +204,12 @@ class Runner:
             sv.spec_vp_chain_sample(self.t0, self.d0, i.final_u, self.rec_all, self.mass_all, vocab_offset=0, rank=0,
                                     draft_is_probs=True, V_shard=self.vs0, tok_out=self.tok0, workspace=self.ws)
             sv.spec_vp_chain_finish(self.tok, self.out[0], V_shard=self.vs0, workspace=self.ws)
+        elif self.wid == 8:
+            sv.spec_verify_tree_sample_filtered(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
+                                                i.max_depth, i.meta["top_k"], i.meta["top_p"],
+                                                draft_probs=i.draft_probs, V=i.V, out_accept_index=self.out[0],
+                                                out_tokens=self.out[1], out_num_accepted=self.out[2],
+                                                workspace=self.ws)
         elif self.wid == 6:
             sv.spec_verify_chain_filtered(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                           i.meta["top_k"], i.meta["top_p"], draft_is_probs=i.draft_is_probs, V=i.V,
@@ -230,9 +238,9 @@ class Runner:
 
 def kernels_per_step(wid, inp) -> int:
     """Launches per verify call: the row-statistics kernel and the finalize kernel
-    (and the filter kernel between them for the filtered chain; six for one rank
-    of the vocabulary-parallel round)."""
-    return {6: 3, 7: 6}.get(wid, 2)
+    (and the filter kernel between them for the filtered chain and tree; six for
+    one rank of the vocabulary-parallel round)."""
+    return {6: 3, 7: 6, 8: 3}.get(wid, 2)
 
 
 def lazy_kernels_per_step(wid, inp) -> int:
@@ -264,7 +272,8 @@ def workspace_for(wid, inp):
         return ws.get(sv.SPEC_ENTRY_CHAIN, inp.B, inp.gamma, inp.V)
     if wid == 7:
         return None                           # each rank's workspace is set up by the runner
-    e = {2: sv.SPEC_ENTRY_TREE_GREEDY, 3: sv.SPEC_ENTRY_TREE_SAMPLE, 5: sv.SPEC_ENTRY_TREE_MSS}[wid]
+    e = {2: sv.SPEC_ENTRY_TREE_GREEDY, 3: sv.SPEC_ENTRY_TREE_SAMPLE, 5: sv.SPEC_ENTRY_TREE_MSS,
+         8: sv.SPEC_ENTRY_TREE_SAMPLE}[wid]
     return ws.get(e, inp.B, inp.N, inp.V)
 
 
@@ -355,12 +364,14 @@ def cpu_baseline(wid, inp, seconds, nthreads=None):
     n = 0
     fn = {0: parity.oracle_chain, 1: parity.oracle_chain, 4: parity.oracle_chain, 7: parity.oracle_chain,
           2: parity.oracle_greedy, 3: parity.oracle_sample, 5: parity.oracle_mss,
+          8: lambda i, r, nthreads: parity.oracle_sample(i, r, nthreads=nthreads, top_k=i.meta["top_k"],
+                                                        top_p=i.meta["top_p"]),
           6: lambda i, r, nthreads: parity.oracle_chain_filtered(i, i.meta["top_k"], i.meta["top_p"], r,
                                                                  nthreads=nthreads)}[wid]
     B = inp.B
     # Large workloads: a bounded sample of whole sequences per "round" of work,
     # scaled to full rounds below.
-    per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4, 7: 16}[wid]))
+    per = B if wid in (0, 1, 6) else max(1, min(B, {2: 8, 3: 4, 4: 16, 5: 4, 7: 16, 8: 4}[wid]))
     rows = None if per == B else list(range(per))
     elapsed = 0.0
     out = None
@@ -396,6 +407,9 @@ def sample_parity(wid, inp, o, rows, ws):
             fl, bad, _ = parity.compare_tree(parity.gpu_greedy(inp, workspace=ws), o, rows)
         elif wid == 3:
             fl, bad, _ = parity.compare_tree(parity.gpu_sample(inp, workspace=ws), o, rows, sample=True)
+        elif wid == 8:
+            g = parity.gpu_sample(inp, workspace=ws, top_k=inp.meta["top_k"], top_p=inp.meta["top_p"])
+            fl, bad, _ = parity.compare_tree(g, o, rows, sample=True)
         else:
             fl, bad, _ = parity.compare_mss(parity.gpu_mss(inp, workspace=ws), o, rows)
         diag = True

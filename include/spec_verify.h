@@ -251,6 +251,38 @@ spec_status spec_verify_tree_sample(int B, int N, int V, int max_depth,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spec_verify_tree_sample_filtered -- target-only tree sampling under
+ * top-k / top-p filtered temperature sampling ([kevins] "draft / verify /
+ * accept": serving samples with temperature, top-k and top-p).  Every
+ * node's target row is filtered as spec_verify_chain_filtered filters a
+ * target row (top-k with ties kept, then top-p over whole groups of equal
+ * logits, renormalised), per sequence; the walk, prob_acc, the thresholds
+ * and the final relu(p'_cur - d_cur) then use the filtered distributions.
+ * draft_probs rows are used as given.  With both thresholds 1 the emitted
+ * tokens are distributed exactly as the filtered target's.
+ *
+ * Arguments as spec_verify_tree_sample, plus top_k [B] int32 and top_p [B]
+ * f32 as in spec_verify_chain_filtered (each nullable, not both; top_k < 0 or
+ * top_p outside (0, 1] makes that sequence invalid).  diag as
+ * spec_verify_tree_sample, with the filtered probabilities.  Same workspace
+ * as spec_verify_tree_sample.  Three launches: the statistics, the filter
+ * (one CTA of 1024 threads per node row, about 192 KB of shared memory for
+ * bf16 rows), the walk.
+ */
+spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth,
+                                             const void* target_logits, spec_dtype tdt,
+                                             int64_t t_row_stride,
+                                             const int32_t* tokens, const int32_t* parents,
+                                             const float* temperature, const float* coins,
+                                             const float* final_u,
+                                             const float* draft_probs, int64_t dp_row_stride,
+                                             float threshold_single, float threshold_acc,
+                                             const int32_t* top_k, const float* top_p,
+                                             int32_t* out_accept_index, int32_t* out_tokens,
+                                             int32_t* out_num_accepted, float* diag,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_verify_tree_mss -- tree verification with a draft distribution
  * (multi-step speculative sampling).  [origins] "SpecInfer", MSS bullet:
  * after a child is rejected the target distribution is replaced by the

@@ -595,9 +595,12 @@ static void tree_sample_impl(int B, int N, int V, int max_depth,
                     acc = (g_mutation == 9) ? pc : acc + pc;
                     double r = acc / th_a;
                     double m1 = fabs(u - r), m2 = fabs(pc - th_s);
-                    if (m1 < dmargin) dmargin = m1;
-                    if (m2 < dmargin) dmargin = m2;
-                    if (u <= r || pc >= th_s) { next = c; break; }
+                    /* accept iff (u <= r) or (pc >= th_s): an acceptance flips only if every
+                     * condition that holds can flip, a rejection if either can */
+                    const int a1 = u <= r, a2 = pc >= th_s;
+                    const double mm = (a1 || a2) ? fmax(a1 ? m1 : 0.0, a2 ? m2 : 0.0) : fmin(m1, m2);
+                    if (mm < dmargin) dmargin = mm;
+                    if (a1 || a2) { next = c; break; }
                     rej[nrej++] = tk[c];
                 }
                 if (next < 0) break;

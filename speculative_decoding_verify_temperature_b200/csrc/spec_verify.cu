@@ -59,7 +59,7 @@ constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
 constexpr double LOG2E = 1.4426950408889634073599246810019;
 
-enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2, MODE_MSS = 3 };
+enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2, MODE_MSS = 3, MODE_SAMPLE_FILT = 4 };
 enum { DK_NONE = 0, DK_LOGITS = 1, DK_PROBS = 2 };
 
 template <int DT> struct Tr;
@@ -671,6 +671,39 @@ template <int TDT> struct WTreeRes {         // relu(p_j - d_j), excluded tokens
         float x[8], d[8];
         ld8<TDT>(row, e0, V, -INFINITY, x);
         ld8<SPEC_F32>(drow, e0, V, 0.f, d);
+        finish(e0, x, d, w);
+    }
+};
+
+// relu(p'_j - d_j) of a filtered tree row: p' = [x >= th] 2^(x s - m) / Z'
+// (iz = 1 / Z'), d = the draft-probability row (HD) or zeros; excluded tokens
+// (the rejected children) 0.
+template <int TDT, bool HD> struct WTreeFilt {
+    const char* row; const char* drow; float s, m, iz, th; const uint32_t* bitmap; int base; int V;
+    struct Raw { Raw8<TDT> t; Raw8<SPEC_F32> d; };
+    __device__ __forceinline__ void load(int64_t e0, Raw& r) const {
+        load_raw8<TDT>(row, e0, r.t);
+        if constexpr (HD) load_raw8<SPEC_F32>(drow, e0, r.d);
+    }
+    __device__ __forceinline__ void finish(int64_t e0, const float (&x)[8], const float (&d)[8],
+                                           float (&w)[8]) const {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float p = x[i] >= th ? ex2(fmaf(x[i], s, -m)) * iz : 0.f;
+            w[i] = fmaxf(0.f, p - d[i]);
+            if (bitmap && e0 + i < V && excluded(bitmap, base, e0 + i)) w[i] = 0.f;
+        }
+    }
+    __device__ __forceinline__ void weights(int64_t e0, const Raw& r, float (&w)[8]) const {
+        float x[8], d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        raw8_f32<TDT>(r.t, x);
+        if constexpr (HD) raw8_f32<SPEC_F32>(r.d, d);
+        finish(e0, x, d, w);
+    }
+    __device__ __forceinline__ void group(int64_t e0, float (&w)[8]) const {
+        float x[8], d[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        ld8<TDT>(row, e0, V, -INFINITY, x);
+        if constexpr (HD) ld8<SPEC_F32>(drow, e0, V, 0.f, d);
         finish(e0, x, d, w);
     }
 };
@@ -1313,7 +1346,99 @@ __device__ int tree_final_draw(const Params& P, int b, int cur, const int* rej, 
     return y;
 }
 
-template <int TDT, int BT>
+// Bitmap (sh.bitmap) of the excluded tokens rej[0..nrej) that fall in chunk c.
+template <int CH, int BT>
+__device__ void excl_bitmap(const int* rej, int nrej, int c, FinShared& sh) {
+    for (int w = threadIdx.x; w < CH / 32; w += BT) sh.bitmap[w] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nrej; i += BT) {
+        const int o = rej[i] - c * CH;
+        if (o >= 0 && o < CH) atomicOr(&sh.bitmap[o >> 5], 1u << (o & 31));
+    }
+    __syncthreads();
+}
+
+// Inverse-CDF draw over a whole row with the weights wf (whose bitmap is
+// sh.bitmap) and the tokens rej[0..nrej) excluded: chunk masses (block sums
+// in fp64), the chunk holding u*S, one rescan.  *S_out = the total; -1 when
+// it is not positive.  All threads call it.
+template <int CH, int BT, class WF>
+__device__ int draw_excluding(WF wf, const int* rej, int nrej, int nch, int V, float u, FinShared& sh,
+                              double* S_out) {
+    const int tid = threadIdx.x;
+    for (int c = 0; c < nch; ++c) {
+        excl_bitmap<CH, BT>(rej, nrej, c, sh);
+        wf.base = c * CH;
+        double tot;
+        block_excl_scan<BT>((double)chunk_weight_partial<CH, BT>(wf, c), &tot);
+        if (tid == 0) sh.M[c] = tot;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        double tot = 0.0;
+        for (int c = 0; c < nch; ++c) tot += sh.M[c];
+        sh.dvals[0] = tot;
+    }
+    __syncthreads();
+    const double S = sh.dvals[0];
+    *S_out = S;
+    int y = -1;
+    if (S > 0.0) {
+        const double t = (double)u * S;
+        for (int attempt = 0; attempt < nch && y < 0; ++attempt) {
+            if (tid == 0) {
+                double C = 0.0, before = 0.0;
+                int cs = -1;
+                for (int c = 0; c < nch; ++c) {
+                    if (sh.M[c] <= 0.0) continue;
+                    if (t < C + sh.M[c]) { cs = c; before = C; break; }
+                    C += sh.M[c];
+                }
+                if (cs < 0)
+                    for (int c = nch - 1; c >= 0; --c)
+                        if (sh.M[c] > 0.0) { cs = c; before = C - sh.M[c]; break; }
+                sh.ivals[4] = cs;
+                sh.dvals[1] = before;
+            }
+            __syncthreads();
+            const int cs = sh.ivals[4];
+            if (cs < 0) break;
+            excl_bitmap<CH, BT>(rej, nrej, cs, sh);
+            wf.base = cs * CH;
+            double tot;
+            y = rescan_chunk<CH, BT>(wf, cs, V, fmax(0.0, t - sh.dvals[1]), u, &tot);
+            if (y < 0 && tid == 0) sh.M[cs] = 0.0;
+            __syncthreads();
+        }
+    }
+    return y;
+}
+
+// The last token of a filtered target-only walk that stopped at node cur:
+// drawn from relu(p'_cur - d_cur) with the rejected children removed
+// (d = draft_probs row, or zeros); an empty residual (rounding only) draws
+// from p'_cur itself.  *S_out = the residual's mass.
+template <int TDT, int BT, bool HD>
+__device__ int tree_filt_draw(const Params& P, int b, int cur, const int* rej, int nrej, float s, float m,
+                              double zc, float th, FinShared& sh, double* S_out) {
+    constexpr int CH = chunk_elems<TDT>();
+    const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
+    const char* drow = HD ? reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * P.N + cur) * P.dpstride
+                          : nullptr;
+    const float u = P.final_u[b], iz = (float)(1.0 / zc);
+    WTreeFilt<TDT, HD> wr{row, drow, s, m, iz, th, sh.bitmap, 0, P.V};
+    int y = draw_excluding<CH, BT>(wr, rej, nrej, P.nch, P.V, u, sh, S_out);
+    if (y < 0) {
+        WTreeFilt<TDT, false> wp{row, nullptr, s, m, iz, th, sh.bitmap, 0, P.V};
+        double S1;
+        y = draw_excluding<CH, BT>(wp, rej, 0, P.nch, P.V, u, sh, &S1);
+    }
+    return y;
+}
+
+// Target-only tree sampling, one CTA per sequence (FILT: on the top-k /
+// top-p filtered rows, from the records of k_filter).
+template <int TDT, int BT, bool FILT = false>
 __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
@@ -1323,6 +1448,16 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         sh.tok[n] = P.tokens[(size_t)b * N + n];
     }
     __syncthreads();
+    if constexpr (FILT) {
+        // each row's threshold and kept mass (same 2^(x s - m) units as z)
+        for (int n = tid; n < N; n += BT) {
+            const FiltRec f = P.filt[(size_t)b * P.R + n];
+            sh.th[n] = f.theta;
+            if (f.on > 0) sh.z[n] = f.Z;
+            if (f.on < 0) sh.bad[n] = 1;             // invalid top_k / top_p
+        }
+        __syncthreads();
+    }
     int ok = tree_valid<BT>(P, N, V, P.max_depth, sh);
     const float T = P.temperature[b];
     if (tid == 0) {
@@ -1342,13 +1477,14 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         return;
     }
     const float s = scale_of(T);
-    // p_parent(n)(tokens[n]) for every non-root node
+    // p_parent(n)(tokens[n]) for every non-root node (0 below the row's threshold)
     for (int n = tid; n < N; n += BT) {
         double pc = 0.0;
         if (n > 0) {
             int pa = sh.par[n];
             const char* row = P.tgt + ((size_t)b * N + pa) * P.tstride;
-            pc = prob_d(ld_elem<TDT>(row, sh.tok[n]), s, sh.m[pa], sh.z[pa]);
+            const float l = ld_elem<TDT>(row, sh.tok[n]);
+            if (!FILT || l >= sh.th[pa]) pc = prob_d(l, s, sh.m[pa], sh.z[pa]);
         }
         sh.pch[n] = pc;
         if (dg) dg[n] = (float)pc;
@@ -1389,7 +1525,15 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     __syncthreads();
     const int cur = sh.ivals[1], k = sh.ivals[2], nrej = sh.ivals[3];
     double S;
-    const int y = tree_final_draw<TDT, BT>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur], sh, &S);
+    int y;
+    if constexpr (FILT) {
+        y = P.draft_probs ? tree_filt_draw<TDT, BT, true>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur],
+                                                          sh.th[cur], sh, &S)
+                          : tree_filt_draw<TDT, BT, false>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur],
+                                                           sh.th[cur], sh, &S);
+    } else {
+        y = tree_final_draw<TDT, BT>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur], sh, &S);
+    }
     if (tid == 0) {
         ot[k] = y;
         for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
@@ -2161,6 +2305,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     const float2* blk = stage_stats(P, blockIdx.x, P.N, dyn, P.stage_cap, &sbar);
     if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
     else if constexpr (MODE == MODE_SAMPLE) finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
+    else if constexpr (MODE == MODE_SAMPLE_FILT) finalize_sample<TDT, SEQ_BT, true>(P, blockIdx.x, sh, blk);
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
 
@@ -2607,19 +2752,20 @@ __device__ bool vh_select(int V, int n, float s, float m, int K, float Pp, FiltS
 }
 
 // Filter thresholds of every row of a chain round, one CTA per (sequence,
-// row): target rows 0..gamma, then the draft-logit rows.  A bf16 row's value
+// row): target rows 0..gamma, then the draft-logit rows (TREE: the N node
+// rows of every tree).  A bf16 row's value
 // histogram needs only the logits, so it is built before waiting for the
 // statistics (the rows' maxima, which the masses are relative to).  Every CTA
 // waits before it exits, so the finalize kernel that follows (and reads the
 // records and the statistics) waits for the statistics through this kernel.
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool TREE = false>
 __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     __shared__ FiltShared fs;
     __shared__ float msh;
     __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
     pdl_trigger();
-    const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
+    const int rows = TREE ? P.N : ((DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1);
     const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
     FiltRec* out = P.filt + (size_t)b * P.R + r;
     const int K = P.top_k ? P.top_k[b] : 0;
@@ -2635,9 +2781,10 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
-    const bool tgt = r <= P.gamma;
-    const char* row = tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
-                          : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
+    const bool tgt = TREE || r <= P.gamma;
+    const char* row = TREE  ? P.tgt + ((size_t)b * P.N + r) * P.tstride
+                      : tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
+                            : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
     const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
     uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
     const int n = vh ? vh_build(row, P.V, fs, w) : 0;
@@ -3579,9 +3726,10 @@ Layout make_layout(int entry, int B, int rows, int V) {
     L.lz_rej = off; off = align256(off + sizeof(int) * (size_t)B * L.rej_cap);
     L.lz_list = off; off = align256(off + sizeof(int) * 2 * (size_t)B);
     L.lz_count = off; off = align256(off + sizeof(unsigned) * (LZ_MAX_LEVELS + 1));
-    // top-k / top-p filter records of the chain's rows
+    // top-k / top-p filter records of the chain's rows (or of every tree node's row)
     L.filt = off;
-    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(FiltRec) * (size_t)B * L.R);
+    if (entry == SPEC_ENTRY_CHAIN || entry == SPEC_ENTRY_TREE_SAMPLE)
+        off = align256(off + sizeof(FiltRec) * (size_t)B * L.R);
     // vocabulary-parallel chain: the decision's per-sequence state
     L.vp = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(VpState) * (size_t)B);
@@ -3814,6 +3962,27 @@ spec_status launch_tree(Params P, cudaStream_t st) {
         smem = P.stage_off + wpw;
     }
     return launch_dependent(k_tree_final<MODE, TDT>, (unsigned)P.B, SEQ_BT, smem, P, st, "k_tree_final");
+}
+
+// Filtered target-only tree sampling: statistics, per-node-row filter
+// thresholds, the filtered walk.
+template <int TDT>
+spec_status launch_tree_filtered(Params P, cudaStream_t st) {
+    spec_status s = launch_stats<MODE_SAMPLE, TDT, TDT>(P, st);
+    if (s != SPEC_OK) return s;
+    constexpr size_t hr = filt_hist_bytes<TDT>();
+    constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
+    static const bool attr = cudaFuncSetAttribute(k_filter<TDT, TDT, DK_NONE, true>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) ==
+                             cudaSuccess;
+    if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
+    s = launch_dependent(k_filter<TDT, TDT, DK_NONE, true>, (unsigned)(P.B * P.N), FILT_BT, hist, P, st,
+                         "k_filter");
+    if (s != SPEC_OK) return s;
+    static const bool big = allow_stage(k_tree_final<MODE_SAMPLE_FILT, TDT>);
+    P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
+    return launch_dependent(k_tree_final<MODE_SAMPLE_FILT, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st,
+                            "k_tree_final");
 }
 
 // One level of the lazy walk: the statistics kernel (the first one as an
@@ -4059,7 +4228,8 @@ static spec_status sample_entry(bool lazy, int B, int N, int V, int max_depth,
                                 float threshold_single, float threshold_acc,
                                 int32_t* out_accept_index, int32_t* out_tokens,
                                 int32_t* out_num_accepted, float* diag,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream,
+                                const int32_t* top_k = nullptr, const float* top_p = nullptr) {
     g_detail[0] = 0;
     Params P{};
     spec_status s = tree_common(P, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents,
@@ -4081,6 +4251,11 @@ static spec_status sample_entry(bool lazy, int B, int N, int V, int max_depth,
     P.th_single = threshold_single; P.th_acc = threshold_acc;
     P.diag = diag;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (top_k || top_p) {
+        P.top_k = top_k; P.top_p = top_p;
+        if (tdt == SPEC_BF16) return launch_tree_filtered<SPEC_BF16>(P, st);
+        return launch_tree_filtered<SPEC_F32>(P, st);
+    }
     if (lazy) {
         if (tdt == SPEC_BF16) return launch_tree_lazy<MODE_SAMPLE, SPEC_BF16>(P, st);
         return launch_tree_lazy<MODE_SAMPLE, SPEC_F32>(P, st);
@@ -4174,6 +4349,21 @@ spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry
 spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(true, SPEC_GREEDY_ARGS); }
 spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(false, SPEC_SAMPLE_ARGS); }
 spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(true, SPEC_SAMPLE_ARGS); }
+
+spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth, const void* target_logits,
+                                             spec_dtype tdt, int64_t t_row_stride, const int32_t* tokens,
+                                             const int32_t* parents, const float* temperature, const float* coins,
+                                             const float* final_u, const float* draft_probs,
+                                             int64_t dp_row_stride, float threshold_single, float threshold_acc,
+                                             const int32_t* top_k, const float* top_p, int32_t* out_accept_index,
+                                             int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+    if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
+    return sample_entry(false, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature,
+                        coins, final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc,
+                        out_accept_index, out_tokens, out_num_accepted, diag, workspace, workspace_bytes, stream,
+                        top_k, top_p);
+}
 
 #define SPEC_MSS_ARGS_DECL                                                                           \
     int B, int N, int V, int max_depth, const void* target_logits, spec_dtype tdt,                 \

@@ -271,6 +271,7 @@ class TreeInputs:
     max_depth: int
     V: int
     draft_probs: torch.Tensor | None = None
+    meta: dict = field(default_factory=dict)
 
     @property
     def B(self):
@@ -438,6 +439,20 @@ def tree_config3(rnd: int = 0, device="cpu") -> TreeInputs:
     return tree_sample_inputs(128, 151936, seed=round_seed(3, rnd), device=device)
 
 
+def tree_config8(rnd: int = 0, device="cpu") -> TreeInputs:
+    """The B=128, 32-node, V=151936 target-only tree workload under serving-style
+    filters: per sequence top_k drawn from {0 (off), 20, 50} and top_p from
+    {1 (off), 0.9, 0.95}, in ``meta["top_k"]`` (int32 [B]) and ``meta["top_p"]``
+    (f32 [B])."""
+    inp = tree_config3(rnd, device)
+    g = make_gen(round_seed(8, rnd), device)
+    ks = torch.tensor([0, 20, 50], dtype=torch.int32, device=device)
+    ps = torch.tensor([1.0, 0.9, 0.95], dtype=torch.float32, device=device)
+    inp.meta["top_k"] = ks[torch.randint(0, 3, (inp.B,), generator=g, device=device)].contiguous()
+    inp.meta["top_p"] = ps[torch.randint(0, 3, (inp.B,), generator=g, device=device)].contiguous()
+    return inp
+
+
 WORKLOADS = {
     0: "chain B=1 gamma=4 V=1000 f32 logits (1000 rounds)",
     1: "chain B=64 gamma=5 V=32000 bf16 target+draft logits, T in {0.6,1.0}",
@@ -446,6 +461,7 @@ WORKLOADS = {
     4: "chain B=512 gamma=7 V=129280 bf16 target + f32 draft probs, T=1",
     5: "multi-step speculative sampling tree B=128 N=32 V=151936 bf16 + f32 draft distributions, T=0.8",
     6: "chain B=64 gamma=5 V=32000 bf16 target+draft logits, T in {0.6,1.0}, top-k in {0,20,50}, top-p in {1,0.9,0.95}",
+    8: "target-only tree B=128 N=32 V=151936 bf16, T=0.8, draft_probs NULL, top-k in {0,20,50}, top-p in {1,0.9,0.95}",
 }
 
 
@@ -466,6 +482,8 @@ def algorithmic_bytes(workload_id: int) -> int:
         return 128 * 32 * 151936 * 2
     if workload_id == 6:
         return 64 * (6 + 5) * 32000 * 2
+    if workload_id == 8:
+        return 128 * 32 * 151936 * 2
     raise ValueError(workload_id)
 
 

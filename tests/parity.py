@@ -134,22 +134,31 @@ def gpu_greedy(inp, workspace=None, lazy=False):
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy())
 
 
-def oracle_sample(inp, rows=None, nthreads=0, threshold_single=1.0, threshold_acc=1.0):
+def oracle_sample(inp, rows=None, nthreads=0, threshold_single=1.0, threshold_acc=1.0, top_k=None, top_p=None):
     sel = _sel(inp.target, rows)
     dp = None if inp.draft_probs is None else to_np(inp.draft_probs[sel])
+    tk = None if top_k is None else to_np(top_k[sel])
+    tp = None if top_p is None else to_np(top_p[sel])
     return oracle.tree_sample(to_np(inp.target[sel]), to_np(inp.tokens[sel]), to_np(inp.parents[sel]),
                               to_np(inp.temperature[sel]), to_np(inp.coins[sel]), to_np(inp.final_u[sel]),
                               inp.max_depth, draft_probs=dp, threshold_single=threshold_single,
-                              threshold_acc=threshold_acc, V=inp.V, nthreads=nthreads)
+                              threshold_acc=threshold_acc, V=inp.V, nthreads=nthreads, top_k=tk, top_p=tp)
 
 
-def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, lazy=False):
+def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, lazy=False, top_k=None, top_p=None):
     B, N = inp.B, inp.N
     diag = torch.full((B, N + 1), float("nan"), device=inp.target.device)
-    ai, ot, na = _fn("spec_verify_tree_sample", lazy)(
-        inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
-        draft_probs=inp.draft_probs, threshold_single=threshold_single, threshold_acc=threshold_acc,
-        V=inp.V, diag=diag, workspace=workspace)
+    if top_k is not None or top_p is not None:
+        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+        ai, ot, na = sv.spec_verify_tree_sample_filtered(
+            inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
+            top_k, top_p, draft_probs=inp.draft_probs, threshold_single=threshold_single,
+            threshold_acc=threshold_acc, V=inp.V, diag=diag, workspace=workspace)
+    else:
+        ai, ot, na = _fn("spec_verify_tree_sample", lazy)(
+            inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
+            draft_probs=inp.draft_probs, threshold_single=threshold_single, threshold_acc=threshold_acc,
+            V=inp.V, diag=diag, workspace=workspace)
     torch.cuda.synchronize()
     d = diag.cpu().numpy().astype(np.float64)
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy(),
@@ -161,6 +170,8 @@ def compare_tree(g, o, rows=None, sample=False):
     gk, gt, ga = g["num_accepted"][sel], g["tokens"][sel], g["accept_index"][sel]
     if sample:
         flags = (o["dmargin"] < TIE_TOL) | (o["cmargin"] < TIE_TOL)
+        if "fmargin" in o:                     # a top-p set decided within the tolerance
+            flags |= o["fmargin"] < TIE_TOL
     else:
         flags = np.zeros(len(gk), bool)
     same = (gk == o["num_accepted"]) & (gt == o["tokens"]).all(axis=1) & (ga == o["accept_index"]).all(axis=1)
@@ -253,12 +264,13 @@ def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, c
 
 
 def gpu_tree_sample_runner(target, tokens, parents, temperature, coins, final_u, max_depth, draft_probs=None,
-                           threshold_single=1.0, threshold_acc=1.0, V=None, nthreads=0, lazy=False):
+                           threshold_single=1.0, threshold_acc=1.0, V=None, nthreads=0, lazy=False,
+                           top_k=None, top_p=None):
     spec_verify_tree_sample = _fn("spec_verify_tree_sample", lazy)
     dev = torch.device("cuda")
 
     def t(a):
-        a = np.ascontiguousarray(a)
+        a = np.array(a, order="C", copy=True)          # writable, whatever view it came as
         if a.dtype == np.uint16:
             return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(a).to(dev)
@@ -266,14 +278,22 @@ def gpu_tree_sample_runner(target, tokens, parents, temperature, coins, final_u,
     B, N, S = target.shape
     V = S if V is None else V
     dp = None if draft_probs is None else _pad_rows(t(draft_probs))
-    ai, ot, na = spec_verify_tree_sample(_pad_rows(t(target)), t(np.asarray(tokens, np.int32)),
-                                         t(np.asarray(parents, np.int32)),
-                                         t(np.asarray(temperature, np.float32).reshape(B)),
-                                         t(np.asarray(coins, np.float32)),
-                                         t(np.asarray(final_u, np.float32).reshape(B)), max_depth,
-                                         draft_probs=dp, threshold_single=threshold_single,
-                                         threshold_acc=threshold_acc, V=V)
-    return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy())
+    args = (_pad_rows(t(target)), t(np.asarray(tokens, np.int32)), t(np.asarray(parents, np.int32)),
+            t(np.asarray(temperature, np.float32).reshape(B)), t(np.asarray(coins, np.float32)),
+            t(np.asarray(final_u, np.float32).reshape(B)), max_depth)
+    diag = torch.full((B, N + 1), float("nan"), device=dev)
+    if top_k is not None or top_p is not None:
+        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+        ai, ot, na = sv.spec_verify_tree_sample_filtered(
+            *args, None if top_k is None else t(np.asarray(top_k, np.int32)),
+            None if top_p is None else t(np.asarray(top_p, np.float32)), draft_probs=dp,
+            threshold_single=threshold_single, threshold_acc=threshold_acc, V=V, diag=diag)
+    else:
+        ai, ot, na = spec_verify_tree_sample(*args, draft_probs=dp, threshold_single=threshold_single,
+                                             threshold_acc=threshold_acc, V=V, diag=diag)
+    d = diag.cpu().numpy().astype(np.float64)
+    return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy(),
+                pchild=d[:, :N])
 
 
 def gpu_tree_greedy_runner(target, tokens, parents, max_depth, V=None, nthreads=0, lazy=False):
