@@ -205,7 +205,7 @@ class Runner:
                                     draft_is_probs=True, V_shard=self.vs0, tok_out=self.tok0, workspace=self.ws)
             sv.spec_vp_chain_finish(self.tok, self.out[0], V_shard=self.vs0, workspace=self.ws)
         elif self.wid == 8:
-            sv.spec_verify_tree_sample_filtered(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
+            getattr(sv, "spec_verify_tree_sample_filtered" + self.sfx)(i.target, i.tokens, i.parents, i.temperature, i.coins, i.final_u,
                                                 i.max_depth, i.meta["top_k"], i.meta["top_p"],
                                                 draft_probs=i.draft_probs, V=i.V, out_accept_index=self.out[0],
                                                 out_tokens=self.out[1], out_num_accepted=self.out[2],
@@ -248,13 +248,16 @@ def lazy_kernels_per_step(wid, inp) -> int:
     chain's last level has no decision), then the final draw (none for greedy)."""
     if wid in (0, 1, 4):
         return 2 * inp.gamma + 2
+    if wid == 8:
+        return 3 * (inp.max_depth + 1) + 1                          # statistics, filter, decision per level
     return 2 * (inp.max_depth + 1) + (1 if wid == 3 else 0)      # workload 5 draws inside its last level
 
 
 def lazy_bytes_read(wid, inp, num_accepted) -> int:
     """Logit bytes the lazy walk streams for one round with these outcomes: chain
     target rows 0..k (row gamma after a full accept) plus draft-logit rows 0..k
-    below gamma; trees the row of every node on the accepted path."""
+    below gamma; trees the row of every node on the accepted path (read twice by
+    the filtered walk: statistics and filter)."""
     k = num_accepted.clamp_min(0).long()
     row_t = inp.V * inp.target.element_size()
     if wid in (0, 1, 4):
@@ -262,6 +265,8 @@ def lazy_bytes_read(wid, inp, num_accepted) -> int:
         if not inp.draft_is_probs:
             n += int((k + 1).clamp_max(inp.gamma).sum()) * inp.V * inp.draft.element_size()
         return n
+    if wid == 8:                              # each visited row is read by the statistics and by the filter
+        return 2 * int((k + 1).sum()) * row_t
     return int((k + 1).sum()) * row_t
 
 
@@ -599,7 +604,8 @@ def main():
 
     # --- the row-on-demand entry point on the same input sets
     # (the filtered chain has no row-on-demand variant)
-    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid < 6 else None
+    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid in (0, 1, 2, 3, 4, 5, 8) \
+        else None
 
     cfg = describe(wid, first)
     cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",

@@ -283,6 +283,27 @@ spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth,
                                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spec_verify_tree_sample_filtered_lazy -- the same results, filtering only
+ * the rows the walk reaches: per level the statistics and the filter record
+ * of each active sequence's current node, then the decisions (three
+ * dependent launches per level), then the draw.  Differences as the other
+ * _lazy entry points: diag holds NaN for the children of unvisited nodes,
+ * and rows that are never read are not validated.
+ */
+spec_status spec_verify_tree_sample_filtered_lazy(int B, int N, int V, int max_depth,
+                                                  const void* target_logits, spec_dtype tdt,
+                                                  int64_t t_row_stride,
+                                                  const int32_t* tokens, const int32_t* parents,
+                                                  const float* temperature, const float* coins,
+                                                  const float* final_u,
+                                                  const float* draft_probs, int64_t dp_row_stride,
+                                                  float threshold_single, float threshold_acc,
+                                                  const int32_t* top_k, const float* top_p,
+                                                  int32_t* out_accept_index, int32_t* out_tokens,
+                                                  int32_t* out_num_accepted, float* diag,
+                                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_verify_tree_mss -- tree verification with a draft distribution
  * (multi-step speculative sampling).  [origins] "SpecInfer", MSS bullet:
  * after a child is rejected the target distribution is replaced by the

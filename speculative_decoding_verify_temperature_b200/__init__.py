@@ -20,6 +20,7 @@ from .spec_verify import (  # noqa: F401
     spec_verify_tree_mss_lazy,
     spec_verify_tree_sample,
     spec_verify_tree_sample_filtered,
+    spec_verify_tree_sample_filtered_lazy,
     spec_verify_tree_sample_lazy,
     spec_workspace_bytes,
     spec_workspace_init,

@@ -75,7 +75,7 @@ struct LazySeq {
     int nrej;      // trees: rejected children of cur
     float s;       // log2(e) / T
     float m, mq;   // combined statistics of the last decided row (chain: target, draft)
-    int pad;
+    float th;      // filtered trees: threshold of cur's row (z is then its kept mass)
     double z, zq;
 };
 enum { LZ_ACTIVE = 0, LZ_DRAW = 1, LZ_DONE = 2, LZ_INVALID = 3 };
@@ -3387,7 +3387,7 @@ __global__ void __launch_bounds__(NT) k_lz_decide_chain(const Params P) {
         }
     }
     LazySeq L;
-    L.cur = level; L.nrej = 0; L.pad = 0;
+    L.cur = level; L.nrej = 0; L.th = -INFINITY;
     L.s = s; L.m = m; L.mq = mq; L.z = z; L.zq = zq;
     if (!ok) {
         L.state = LZ_INVALID;
@@ -3443,7 +3443,7 @@ __device__ bool warp_tree_valid(const Params& P, int b) {
 // or p >= threshold_single; rejected children's tokens are kept for the final
 // draw.  Level 0 validates the tree (and the temperature).  Diagnostics hold
 // p_cur(token) for the children of visited nodes, NaN for the other nodes.
-template <int MODE, int TDT>
+template <int MODE, int TDT, bool FILT = false>
 __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
     pdl_trigger();
     pdl_wait();
@@ -3492,6 +3492,14 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
                 }
         } else {
             ok = !warp_combine(st, E, m, z);
+            float th = -INFINITY;
+            if constexpr (FILT) {                      // cur's filter record (k_lz_filter_tree)
+                const FiltRec f = P.filt[(size_t)b * P.R + cur];
+                if (f.on < 0) ok = false;
+                if (f.on > 0) z = f.Z;
+                th = f.theta;
+                L.th = th;
+            }
             if (ok) {
                 const char* trow = P.tgt + ((size_t)b * N + cur) * P.tstride;
                 const double coin = (double)P.coins[(size_t)b * N + cur];
@@ -3505,7 +3513,8 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
                     int t = 0;
                     if (child) {
                         t = tok[c];
-                        pc = prob_d(ld_elem<TDT>(trow, t), L.s, m, z);
+                        const float l = ld_elem<TDT>(trow, t);
+                        if (!FILT || l >= th) pc = prob_d(l, L.s, m, z);
                         if (dg) dg[c] = (float)pc;
                     }
                     unsigned msk = __ballot_sync(FULL, child);
@@ -3553,6 +3562,53 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
     P.lz_seq[b] = L;
 }
 
+// Lazy filtered tree walk: the filter record of the current node's row of
+// every active sequence at this level (one CTA each, as k_filter), between
+// the level's statistics and its decisions.
+template <int TDT>
+__global__ void __launch_bounds__(FILT_BT) k_lz_filter_tree(const Params P) {
+    __shared__ FiltShared fs;
+    __shared__ float msh;
+    __shared__ int bad;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    pdl_trigger();
+    pdl_wait();
+    if ((int)blockIdx.x >= lz_count_of(P)) return;
+    const int b = lz_seq_of(P, blockIdx.x);
+    const int cur = P.level == 0 ? 0 : P.lz_seq[b].cur;
+    FiltRec* out = P.filt + (size_t)b * P.R + cur;
+    const int K = P.top_k ? P.top_k[b] : 0;
+    const float Pp = P.top_p ? P.top_p[b] : 1.f;
+    const float T = P.temperature[b];
+    if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
+        return;
+    }
+    if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const int E = P.nch * SPC;
+    if (threadIdx.x < 32) {
+        float m;
+        double z;
+        const bool bd = warp_combine(P.stats + ((size_t)b * P.R + cur) * E, E, m, z);
+        if (threadIdx.x == 0) { msh = m; bad = bd; }
+    }
+    __syncthreads();
+    if (bad) {                                   // the decision marks the sequence invalid
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
+    const float s = scale_of(T), m = msh;
+    uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
+    FiltRec rec;
+    if (TDT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, K, Pp, fs, w, &rec))
+        rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
+    if (threadIdx.x == 0) *out = rec;
+}
+
 // Lazy multi-step sampling walk, one CTA per active sequence at this level:
 // level 0 validates the tree and the temperature; the current node's row is
 // combined from its statistics; mss_node tests its children.  An accepted
@@ -3582,7 +3638,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_decide_mss(const Params P) {
         ok = tree_valid<SEQ_BT>(P, N, P.V, P.max_depth, sh);
         const float T = P.temperature[b];
         ok &= temperature_ok(T);
-        L.cur = 0; L.k = 0; L.nrej = 0; L.pad = 0;
+        L.cur = 0; L.k = 0; L.nrej = 0; L.th = -INFINITY;
         L.s = ok ? scale_of(T) : 0.f;
         L.mq = 0.f; L.zq = 0.0;
         if (ok) {
@@ -3650,7 +3706,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_decide_mss(const Params P) {
 // Last token of a lazy target-only tree walk, one CTA per sequence (those
 // left in LZ_DRAW): tree_final_draw at the node where the walk stopped, with
 // the rejected children's tokens it kept.
-template <int TDT>
+template <int TDT, bool FILT = false>
 __global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
     __shared__ FinShared sh;
     pdl_wait();
@@ -3661,7 +3717,14 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
     for (int i = tid; i < L.nrej; i += SEQ_BT) sh.rej[i] = P.lz_rej[(size_t)b * P.rej_cap + i];
     __syncthreads();
     double S;
-    const int y = tree_final_draw<TDT, SEQ_BT>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, sh, &S);
+    int y;
+    if constexpr (FILT) {
+        y = P.draft_probs ? tree_filt_draw<TDT, SEQ_BT, true>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, sh, &S)
+                          : tree_filt_draw<TDT, SEQ_BT, false>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, sh,
+                                                               &S);
+    } else {
+        y = tree_final_draw<TDT, SEQ_BT>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, sh, &S);
+    }
     if (tid == 0) {
         int32_t* ai = P.out_accept_index + (size_t)b * W;
         int32_t* ot = P.out_tokens + (size_t)b * W;
@@ -4058,6 +4121,36 @@ spec_status launch_tree_lazy(Params P, cudaStream_t st) {
     return s;
 }
 
+// Lazy filtered target-only tree sampling: per level the statistics of the
+// current nodes' rows, their filter records, the decisions; then the draw.
+template <int TDT>
+spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
+    auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
+    auto kf = k_lz_filter_tree<TDT>;
+    auto kd = k_lz_decide_tree<MODE_SAMPLE, TDT, true>;
+    static const int occ = blocks_per_sm(ks);
+    const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
+    const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
+    constexpr size_t hr = filt_hist_bytes<TDT>();
+    constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
+    static const bool attr =
+        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) == cudaSuccess;
+    if (!attr) return fail(SPEC_ERR_CUDA, "k_lz_filter_tree shared memory attribute");
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    for (int level = 0; level <= P.max_depth; ++level) {
+        spec_status s = launch_level(ks, sgrid, (void (*)(Params))nullptr, 0, P, level, st);
+        if (s != SPEC_OK) return s;
+        s = launch_dependent(kf, (unsigned)P.B, FILT_BT, hist, P, st, "k_lz_filter_tree");
+        if (s != SPEC_OK) return s;
+        s = launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
+        if (s != SPEC_OK) return s;
+    }
+    spec_status s = launch_dependent(k_lz_tree_final<TDT, true>, (unsigned)P.B, SEQ_BT, 0, P, st, "k_lz_tree_final");
+    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
+        return fail(SPEC_ERR_CUDA, "profile event");
+    return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -4253,6 +4346,10 @@ static spec_status sample_entry(bool lazy, int B, int N, int V, int max_depth,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (top_k || top_p) {
         P.top_k = top_k; P.top_p = top_p;
+        if (lazy) {
+            if (tdt == SPEC_BF16) return launch_tree_filtered_lazy<SPEC_BF16>(P, st);
+            return launch_tree_filtered_lazy<SPEC_F32>(P, st);
+        }
         if (tdt == SPEC_BF16) return launch_tree_filtered<SPEC_BF16>(P, st);
         return launch_tree_filtered<SPEC_F32>(P, st);
     }
@@ -4360,6 +4457,22 @@ spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth,
                                              void* workspace, size_t workspace_bytes, void* stream) {
     if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
     return sample_entry(false, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature,
+                        coins, final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc,
+                        out_accept_index, out_tokens, out_num_accepted, diag, workspace, workspace_bytes, stream,
+                        top_k, top_p);
+}
+
+spec_status spec_verify_tree_sample_filtered_lazy(int B, int N, int V, int max_depth, const void* target_logits,
+                                                  spec_dtype tdt, int64_t t_row_stride, const int32_t* tokens,
+                                                  const int32_t* parents, const float* temperature,
+                                                  const float* coins, const float* final_u, const float* draft_probs,
+                                                  int64_t dp_row_stride, float threshold_single,
+                                                  float threshold_acc, const int32_t* top_k, const float* top_p,
+                                                  int32_t* out_accept_index, int32_t* out_tokens,
+                                                  int32_t* out_num_accepted, float* diag, void* workspace,
+                                                  size_t workspace_bytes, void* stream) {
+    if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
+    return sample_entry(true, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature,
                         coins, final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc,
                         out_accept_index, out_tokens, out_num_accepted, diag, workspace, workspace_bytes, stream,
                         top_k, top_p);

@@ -59,9 +59,11 @@ def lib():
             f = getattr(L, name)
             f.restype = i32
             f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64, P, P, P, P, P, sz, P]
-        L.spec_verify_tree_sample_filtered.restype = i32
-        L.spec_verify_tree_sample_filtered.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
-                                                       f32, f32, P, P, P, P, P, P, P, sz, P]
+        for name in ("spec_verify_tree_sample_filtered", "spec_verify_tree_sample_filtered_lazy"):
+            f = getattr(L, name)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
+                          f32, f32, P, P, P, P, P, P, P, sz, P]
         L.spec_verify_chain_filtered.restype = i32
         L.spec_verify_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
                                                  P, P, P, P, P, P, P, P, P, P, sz, P]
@@ -269,7 +271,7 @@ def spec_verify_tree_sample_filtered(target, tokens, parents, temperature, coins
                                      top_k=None, top_p=None, *, draft_probs=None, threshold_single: float = 1.0,
                                      threshold_acc: float = 1.0, V: int | None = None, out_accept_index=None,
                                      out_tokens=None, out_num_accepted=None, diag=None, workspace=None,
-                                     stream=None):
+                                     stream=None, _name: str = "spec_verify_tree_sample_filtered"):
     """Target-only tree sampling on top-k / top-p filtered node rows; ``top_k`` int32
     ``[B]`` (0 = off) and ``top_p`` f32 ``[B]`` (1 = off), either may be None (not
     both).  Returns ``(accept_index, tokens, num_accepted)``."""
@@ -291,13 +293,20 @@ def spec_verify_tree_sample_filtered(target, tokens, parents, temperature, coins
         out_num_accepted = torch.empty((B,), dtype=torch.int32, device=dev)
     ws = _ws(workspace, SPEC_ENTRY_TREE_SAMPLE, B, N, V, dev, stream)
     dstride = _rows(draft_probs, "draft_probs") if draft_probs is not None else 0
-    st = lib().spec_verify_tree_sample_filtered(
+    st = getattr(lib(), _name)(
         B, N, V, max_depth, _p(target), _dtype(target), _rows(target, "target"), _p(tokens),
         _p(parents), _p(temperature), _p(coins), _p(final_u), _p(draft_probs), dstride,
         float(threshold_single), float(threshold_acc), _p(top_k), _p(top_p), _p(out_accept_index),
         _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
-    _check(st, "spec_verify_tree_sample_filtered")
+    _check(st, _name)
     return out_accept_index, out_tokens, out_num_accepted
+
+
+def spec_verify_tree_sample_filtered_lazy(*args, **kw):
+    """Row-on-demand filtered tree sampling: the arguments and results of
+    ``spec_verify_tree_sample_filtered``, filtering only the rows the walk reaches;
+    ``diag`` holds NaN for children of unvisited nodes."""
+    return spec_verify_tree_sample_filtered(*args, _name="spec_verify_tree_sample_filtered_lazy", **kw)
 
 
 def spec_verify_chain_lazy(*args, **kw):

@@ -149,8 +149,7 @@ def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, laz
     B, N = inp.B, inp.N
     diag = torch.full((B, N + 1), float("nan"), device=inp.target.device)
     if top_k is not None or top_p is not None:
-        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
-        ai, ot, na = sv.spec_verify_tree_sample_filtered(
+        ai, ot, na = _fn("spec_verify_tree_sample_filtered", lazy)(
             inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
             top_k, top_p, draft_probs=inp.draft_probs, threshold_single=threshold_single,
             threshold_acc=threshold_acc, V=inp.V, diag=diag, workspace=workspace)
@@ -283,8 +282,7 @@ def gpu_tree_sample_runner(target, tokens, parents, temperature, coins, final_u,
             t(np.asarray(final_u, np.float32).reshape(B)), max_depth)
     diag = torch.full((B, N + 1), float("nan"), device=dev)
     if top_k is not None or top_p is not None:
-        from speculative_decoding_verify_temperature_b200 import spec_verify as sv
-        ai, ot, na = sv.spec_verify_tree_sample_filtered(
+        ai, ot, na = _fn("spec_verify_tree_sample_filtered", lazy)(
             *args, None if top_k is None else t(np.asarray(top_k, np.int32)),
             None if top_p is None else t(np.asarray(top_p, np.float32)), draft_probs=dp,
             threshold_single=threshold_single, threshold_acc=threshold_acc, V=V, diag=diag)

@@ -143,3 +143,52 @@ def test_tree_filtered_workload3_shapes(cuda_device):
     inp = wl.tree_config3(0, "cuda")
     tk, tp = _params(inp.B, inp.V, 9)
     _check(inp, tk, tp, rows=np.arange(0, 128, 8))
+
+
+# ----------------------------------------------------------------------------- the lazy walk
+
+def _lazy_same(inp, tk, tp):
+    """Lazy == dense on tokens, accept indices and counts; child probabilities
+    equal where the lazy walk evaluated them (children of visited nodes), NaN
+    elsewhere; the final residual mass equal."""
+    d = parity.gpu_sample(inp, top_k=tk, top_p=tp)
+    z = parity.gpu_sample(inp, top_k=tk, top_p=tp, lazy=True)
+    for key in ("accept_index", "tokens", "num_accepted"):
+        np.testing.assert_array_equal(z[key], d[key])
+    par = inp.parents.cpu().numpy()
+    for b in range(inp.B):
+        if d["num_accepted"][b] < 0:
+            continue
+        visited = set(int(n) for n in d["accept_index"][b] if n >= 0)
+        ev = np.array([n > 0 and par[b, n] in visited for n in range(inp.N)])
+        np.testing.assert_array_equal(z["pchild"][b, ev], d["pchild"][b, ev])
+        assert np.isnan(z["pchild"][b, 1:][~ev[1:]]).all()
+        assert z["S"][b] == d["S"][b]
+    return z
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}V{c[1]}{str(c[2])[-4:]}{c[3]}{c[4]}")
+def test_tree_filtered_lazy_equals_dense(case, cuda_device):
+    B, V, dt, kind, dp, T, pad = case
+    for seed in range(2):
+        stride = -(-(V + pad) // _q(dt)) * _q(dt)
+        inp = wl.tree_sample_inputs(B, V, seed=8400 + seed, device="cuda", parents_fn=_parents_fn(kind),
+                                    target_dtype=dt, stride=stride, temperature=T, draft_probs=dp,
+                                    zipf=V > 100)
+        tk, tp = _params(B, V, 10 + seed)
+        _lazy_same(inp, tk, tp)
+        _lazy_same(inp, tk, None)
+
+
+def test_tree_filtered_lazy_workload3_shapes(cuda_device):
+    inp = wl.tree_config3(0, "cuda")
+    tk, tp = _params(inp.B, inp.V, 11)
+    _lazy_same(inp, tk, tp)
+
+
+@pytest.mark.parametrize("kw", [dict(top_k=2, top_p=None), dict(top_k=3, top_p=0.8, V=4, K=2, seed=3,
+                                                                 parents=(-1, 0, 0, 1, 2))])
+def test_tree_filtered_lazy_lossless_through_gpu(kw, cuda_device):
+    import functools
+    r = pins.tree_bruteforce(runner=functools.partial(parity.gpu_tree_sample_runner, lazy=True), **kw)
+    assert r["ok"], (kw, r)
