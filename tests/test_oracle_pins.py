@@ -488,6 +488,29 @@ def test_tree_topk1_sampling_is_greedy():
     np.testing.assert_array_equal(s["tokens"], g["tokens"])
 
 
+def test_tree_margin_of_two_condition_acceptance():
+    """A child is accepted when coin <= prob_acc/theta_acc or p >= theta_single.
+    An acceptance flips only if every condition that holds can flip: p = 1 exactly
+    at theta_single = 1 with a coin far below 1 is not a near-tie; a rejection
+    with the coin just above prob_acc is."""
+    V = 6
+    parents = np.array([[-1, 0]], np.int32)
+    t = np.full((1, 2, V), -np.inf, np.float32)
+    t[0, 0, 3] = 0.0                                      # the root row keeps one token: p = 1 exactly
+    t[0, 1, :] = 0.0
+    tokens = np.array([[0, 3]], np.int32)
+    r = oracle.tree_sample(t, tokens, parents, np.ones(1, np.float32), np.array([[0.25, 0.5]], np.float32),
+                           np.array([0.5], np.float32), 1)
+    assert r["num_accepted"][0] == 1 and r["pchild"][0, 1] == 1.0
+    assert r["dmargin"][0] >= 0.5                         # the coin settles it: 1 - 0.25
+    t2 = np.zeros((1, 2, V), np.float32)                  # uniform root row: p = 1/6 for every token
+    c = np.float32(1.0 / 6.0) + np.float32(2 ** -24)
+    r2 = oracle.tree_sample(t2, tokens, parents, np.ones(1, np.float32), np.array([[c, 0.5]], np.float32),
+                            np.array([0.5], np.float32), 1)
+    assert r2["num_accepted"][0] == 0                     # coin just above prob_acc: rejected
+    assert r2["dmargin"][0] < 1e-6                        # and flagged as a near-tie
+
+
 # ----------------------------------------------------------------------------- the pins bite
 
 MUTATIONS = {
