@@ -1,6 +1,6 @@
 """Benchmark of the speculative-decoding verify step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {0..4}] [--impl {ours,reference}]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload {0..8}] [--impl {ours,reference}]
 
 One step = one verify round (one C-ABI call) over the workload's whole batch.
 Default workload 1: chain speculative sampling, B=64, gamma=5, V=32000, bf16
@@ -10,13 +10,15 @@ with no exchange): weak scaling, time = max over ranks.
 
 Rank 0 prints ONE JSON line.  ``value`` is whole-job verify rounds/s with the
 inputs already in HBM (CUDA-graph replays, CUDA events); L2 is kept cold by
-rotating several input sets whose total exceeds the 126 MB L2 (workload 1) or
-by inputs larger than L2 (workloads 2-4).  ``e2e`` is the same metric through
+rotating several input sets whose total exceeds the 126 MB L2 (workloads 0-1)
+or by inputs larger than L2 (workloads 2-4).  ``e2e`` is the same metric through
 the Python binding with pinned host buffers copied in and results copied out
 every step.  ``roofline`` reports the row kernel (the dominant one) against
 the measured HBM copy bandwidth; ``cpu_baseline`` times the fp64 oracle on a
-bounded sample on the host cores.  ``--impl reference`` runs that oracle
-alone as the reference arm.
+bounded sample on the host cores.  The default run also measures each of the
+five benchmark configurations (workloads 0-4) the same way under
+``per_config``.  ``--impl reference`` runs that oracle alone as the reference
+arm.
 """
 from __future__ import annotations
 
@@ -48,6 +50,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lazy-steps", type=int, default=400,
                     help="steps of the row-on-demand (lazy) entry point timed beside the dense one (0: skip)")
+    ap.add_argument("--configs", default=None,
+                    help="comma-separated workloads measured under per_config (default: 0,1,2,3,4 when "
+                         "--workload is 1, none otherwise; 'none' skips)")
+    ap.add_argument("--config-cpu-seconds", type=float, default=3.0,
+                    help="oracle seconds per configuration under per_config")
     return ap.parse_args()
 
 
@@ -236,23 +243,6 @@ class Runner:
         return self.out[-1]
 
 
-def kernels_per_step(wid, inp) -> int:
-    """Launches per verify call: the row-statistics kernel and the finalize kernel
-    (and the filter kernel between them for the filtered chain and tree; six for
-    one rank of the vocabulary-parallel round)."""
-    return {6: 3, 7: 6, 8: 3}.get(wid, 2)
-
-
-def lazy_kernels_per_step(wid, inp) -> int:
-    """Launches per lazy call: a statistics and a decision kernel per level (the
-    chain's last level has no decision), then the final draw (none for greedy)."""
-    if wid in (0, 1, 4):
-        return 2 * inp.gamma + 2
-    if wid == 8:
-        return 3 * (inp.max_depth + 1) + 1                          # statistics, filter, decision per level
-    return 2 * (inp.max_depth + 1) + (1 if wid == 3 else 0)      # workload 5 draws inside its last level
-
-
 def lazy_bytes_read(wid, inp, num_accepted) -> int:
     """Logit bytes the lazy walk streams for one round with these outcomes: chain
     target rows 0..k (row gamma after a full accept) plus draft-logit rows 0..k
@@ -290,6 +280,29 @@ def algorithmic_bytes(wid, inp) -> int:
     if wid in (0, 1, 6):
         b += inp.draft[:, :, :inp.V].numel() * inp.draft.element_size()
     return b
+
+
+def round_bytes(wid, inp, num_accepted) -> int:
+    """Algorithmic bytes of one whole round with these outcomes: the row
+    kernel's bytes, plus, for a chain with draft probabilities, the gathered
+    q(x) of every drafted token and the full q row of every sequence that
+    rejects (the residual norm(max(0, p - q)) reads it once)."""
+    b = algorithmic_bytes(wid, inp)
+    if wid in (4, 7) and inp.draft_is_probs:
+        k = num_accepted
+        rejecting = int(((k >= 0) & (k < inp.gamma)).sum())
+        V = vp_cuts(inp.V)[1] if wid == 7 else inp.V
+        b += inp.B * inp.gamma * 4 + rejecting * V * 4
+    return b
+
+
+def accept_histogram(wid, inp, num_accepted) -> dict:
+    """Counts of the accepted lengths (draft tokens accepted per sequence and
+    round; -1 = invalid sequence) over the measured rounds."""
+    top = inp.gamma if wid in (0, 1, 4, 6, 7) else inp.max_depth
+    k = num_accepted.long().cpu()
+    h = {str(v): int((k == v).sum()) for v in range(-1, top + 1)}
+    return {key: n for key, n in h.items() if n or key != "-1"}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -458,22 +471,191 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0}, "fallback"
 
 
+def input_sets(wid, dev, rank=0):
+    """The workload's rotating input sets: enough of them that their total
+    exceeds twice the L2 (one set when a set alone is that large)."""
+    first = make_inputs(wid, 0, dev, rank)
+    nbytes = input_bytes(first)
+    nsets = 1 if nbytes > 2 * L2_BYTES else min(16, -(-2 * L2_BYTES // nbytes))
+    return [first] + [make_inputs(wid, r, dev, rank) for r in range(1, nsets)], nbytes
+
+
+def bench_config(wid, first, nsets, nbytes, world) -> dict:
+    """The `config` object of a bench line (the same for both arms)."""
+    cfg = describe(wid, first)
+    cfg.update(parallelism=f"batch-sharded x{world} (no collective)" if world > 1 else "single GPU",
+               l2=(f"{nsets} rotating input sets of {nbytes / 1e6:.1f} MB ({nsets * nbytes / 1e6:.0f} MB > 126 MB L2)"
+                   if nsets > 1 else f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2"))
+    return cfg
+
+
+CONFIG_STEPS = {0: 2000, 1: 2000, 2: 500, 3: 250, 4: 250}
+
+
+def measure(wid, dev, world, steps, warmup, local, rank=0):
+    """Time one workload: CUDA-graph replays of its rotating input sets (CUDA
+    events, max over ranks), the row kernel's own duration, the launches per
+    call, and the accepted lengths of the measured rounds."""
+    import torch
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    sets, nbytes = input_sets(wid, dev, rank)
+    first, nsets = sets[0], len(sets)
+    ws = workspace_for(wid, first)
+    runners = [Runner(wid, s, ws) for s in sets]
+    stream = torch.cuda.current_stream()
+    for i in range(max(3, warmup)):
+        runners[i % nsets]()
+    torch.cuda.synchronize()
+
+    # --- one CUDA graph per rotation of the input sets; the library counts the
+    # kernels it adds to the graph
+    n0 = sv.spec_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for r in runners:
+            r()
+    kps = (sv.spec_launch_count() - n0) // nsets
+    torch.cuda.synchronize()
+    singles = []
+    for r in runners:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            r()
+        singles.append(g)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+
+    K = steps
+    sampler = ClockSampler(local)
+    with sampler:
+        time.sleep(0.02)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sampler.mark = True
+        e0.record(stream)
+        full, rem = divmod(K, nsets)
+        for _ in range(full):
+            graph.replay()
+        for i in range(rem):
+            singles[i].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sampler.mark = False
+        if world > 1:
+            torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    ms_max = reduce_max_ms(ms, world, dev)
+    value = job_value(K, world, ms_max)
+    del graph, singles
+
+    # --- dominant kernel duration: the library records an event pair around its
+    # row kernel; the calls are captured in a CUDA graph so that host launch
+    # latency never shows up between the two events.
+    nk = max(nsets, min(256, K))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+    for a, b in evs:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    pg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pg):
+        for i in range(nk):
+            sv.spec_profile_events(*evs[i])
+            runners[i % nsets]()
+        sv.spec_profile_events()
+    kms = []
+    for _ in range(3):
+        pg.replay()
+        torch.cuda.synchronize()
+        kms += [a.elapsed_time(b) for a, b in evs]
+    del pg
+    k_avg_ms = sum(kms) / len(kms)
+
+    # --- acceptance statistics and whole-round bytes of the benchmarked rounds
+    torch.cuda.synchronize()
+    acc, rb = [], 0
+    for r, st in zip(runners, sets):
+        r()
+        k = r.num_accepted()
+        acc.append(k.clone())
+        rb += round_bytes(wid, st, k)
+    acc = torch.cat(acc)
+    return dict(wid=wid, sets=sets, first=first, nsets=nsets, nbytes=nbytes, ws=ws, runners=runners, K=K,
+                ms_max=ms_max, value=value, kps=kps, k_avg_ms=k_avg_ms, clocks=sampler.summary(),
+                alg=algorithmic_bytes(wid, first), round_bytes=rb / nsets,
+                mean_tau=float((acc.float() + 1).mean()), hist=accept_histogram(wid, first, acc))
+
+
+ROW_KERNEL = {
+    "fused": "k_chain_fused (streams every row pair once and takes the whole round's decisions)",
+    "stats": "k_stats (streams every logit row once)",
+}
+
+
+def roofline_of(m, peaks, peak_kind, row_kernel):
+    achieved = m["alg"] / (m["k_avg_ms"] / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profile_traffic(m["wid"]),
+            "kernel": ROW_KERNEL[row_kernel], "kernel_ms": round(m["k_avg_ms"], 5),
+            "algorithmic_bytes_per_launch": m["alg"],
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+            "frac_of_nominal_8000_gbs": round(achieved / 8000.0, 4)}
+
+
+def row_kernel_of(m) -> str:
+    """Which kernel the library's timing hook brackets for this workload: the
+    fused chain kernel is the only launch of its call."""
+    return "fused" if m["kps"] == 1 else "stats"
+
+
+def config_summary(m, peaks, peak_kind, cpu=None) -> dict:
+    """The per_config entry of one measured workload."""
+    step_s = m["ms_max"] / m["K"] / 1e3
+    d = {"workload": describe(m["wid"], m["first"])["workload"], "steps": m["K"],
+         "rounds_per_s": round(m["value"], 2), "step_us": round(step_s * 1e6, 3),
+         "gpu_launches_per_step": m["kps"],
+         "row_kernel": roofline_of(m, peaks, peak_kind, row_kernel_of(m)),
+         "round_algorithmic_bytes": int(m["round_bytes"]),
+         "round_hbm_gbs": round(m["round_bytes"] / step_s / 1e9, 1),
+         "round_frac": round(m["round_bytes"] / step_s / 1e9 / peaks["hbm_gbs"], 4),
+         "mean_tau": round(m["mean_tau"], 4), "accept_length_histogram": m["hist"],
+         "clocks": m["clocks"]}
+    if cpu is not None:
+        d["cpu_baseline"] = cpu
+    return d
+
+
 def run_reference(args, ws_, rank):
     import torch
     if rank != 0:
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = make_inputs(args.workload, 0, dev)
+    sets, nbytes = input_sets(args.workload, dev)
+    inp = sets[0]
     steps = max(1, args.steps)
     # each step is a bounded sample of the workload (see cpu_baseline)
     cb, _, _ = cpu_baseline(args.workload, inp, seconds=min(60.0, max(5.0, 0.02 * steps)))
-    cfg = describe(args.workload, inp)
+    cfg = bench_config(args.workload, inp, len(sets), nbytes, ws_)
     line = {"impl": "reference", "metric": "verify rounds/s", "value": cb["value"], "unit": "rounds/s",
             "n_gpus": ws_, "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": cfg, "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def config_list(args):
+    if args.configs is None:
+        return [0, 1, 2, 3, 4] if args.workload == 1 else []
+    if args.configs.strip().lower() in ("", "none"):
+        return []
+    return [int(c) for c in args.configs.split(",")]
 
 
 def main():
@@ -494,107 +676,13 @@ def main():
         return
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
     wid = args.workload
 
-    # --- inputs: enough rotating sets to keep L2 cold between steps
-    first = make_inputs(wid, 0, dev, rank)
-    nbytes = input_bytes(first)
-    nsets = 1 if nbytes > 2 * L2_BYTES else min(16, -(-2 * L2_BYTES // nbytes))
-    sets = [first] + [make_inputs(wid, r, dev, rank) for r in range(1, nsets)]
-    ws = workspace_for(wid, first)
-    runners = [Runner(wid, s, ws) for s in sets]
-    kps = kernels_per_step(wid, first)
-    stream = torch.cuda.current_stream()
-
-    for i in range(max(3, args.warmup)):
-        runners[i % nsets]()
-    torch.cuda.synchronize()
-
-    # --- one CUDA graph per rotation of the input sets
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for r in runners:
-            r()
-    torch.cuda.synchronize()
-    singles = []
-    for r in runners:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            r()
-        singles.append(g)
-    torch.cuda.synchronize()
-    graph.replay()
-    torch.cuda.synchronize()
-
-    K = args.steps
-    sampler = ClockSampler(local)
-    with sampler:
-        time.sleep(0.02)
-        for _ in range(3):
-            graph.replay()
-        torch.cuda.synchronize()
-        if ws_ > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        sampler.mark = True
-        e0.record(stream)
-        full, rem = divmod(K, nsets)
-        for _ in range(full):
-            graph.replay()
-        for i in range(rem):
-            singles[i].replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        sampler.mark = False
-        if ws_ > 1:
-            dist.barrier()
-    ms = e0.elapsed_time(e1)
-    ms_max = reduce_max_ms(ms, ws_, dev)
-    value = job_value(K, ws_, ms_max)
-
-    # --- dominant kernel duration: the library records an event pair around its
-    # row-statistics kernel; the calls are captured in a CUDA graph so that host
-    # launch latency never shows up between the two events.
-    nk = max(nsets, min(256, K))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
-    for a, b in evs:
-        a.record(stream)
-        b.record(stream)
-    torch.cuda.synchronize()
-    pg = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(pg):
-        for i in range(nk):
-            sv.spec_profile_events(*evs[i])
-            runners[i % nsets]()
-        sv.spec_profile_events()
-    kms = []
-    for _ in range(3):
-        pg.replay()
-        torch.cuda.synchronize()
-        kms += [a.elapsed_time(b) for a, b in evs]
-    del pg
-    k_avg_ms = sum(kms) / len(kms)
-    alg = algorithmic_bytes(wid, first)
+    m = measure(wid, dev, ws_, args.steps, args.warmup, local, rank)
+    first, sets, ws, K = m["first"], m["sets"], m["ws"], m["K"]
     peaks, peak_kind = measured_peaks()
-    achieved = alg / (k_avg_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profile_traffic(wid),
-                "kernel": "k_stats (streams every logit row once)",
-                "kernel_ms": round(k_avg_ms, 5), "algorithmic_bytes_per_launch": alg,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
-                "frac_of_nominal_8000_gbs": round(achieved / 8000.0, 4)}
-    round_gbs = alg / (ms_max / K / 1e3) / 1e9
-
-    # --- acceptance statistics of the benchmarked rounds
-    torch.cuda.synchronize()
-    acc = []
-    for r in runners:
-        r()
-        acc.append(r.num_accepted().float())
-    acc = torch.cat(acc)
-    mean_tau = float((acc + 1).mean())
+    roofline = roofline_of(m, peaks, peak_kind, row_kernel_of(m))
+    value, ms_max = m["value"], m["ms_max"]
     B = first.B
     draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6, 7) else first.N - 1)
 
@@ -604,25 +692,24 @@ def main():
 
     # --- the row-on-demand entry point on the same input sets
     # (the filtered chain has no row-on-demand variant)
-    lazy = run_lazy(wid, sets, ws, args.lazy_steps, alg, ws_, dev) if args.lazy_steps > 0 and wid in (0, 1, 2, 3, 4, 5, 8) \
-        else None
+    lazy = run_lazy(wid, sets, ws, args.lazy_steps, m["alg"], ws_, dev) \
+        if args.lazy_steps > 0 and wid in (0, 1, 2, 3, 4, 5, 8) else None
 
-    cfg = describe(wid, first)
-    cfg.update(parallelism=f"batch-sharded x{ws_} (no collective)" if ws_ > 1 else "single GPU",
-               l2=(f"{nsets} rotating input sets of {nbytes / 1e6:.1f} MB ({nsets * nbytes / 1e6:.0f} MB > 126 MB L2)"
-                   if nsets > 1 else f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2"),
-               timing="CUDA-graph replays, CUDA events, max over ranks")
+    cfg = bench_config(wid, first, m["nsets"], m["nbytes"], ws_)
     line = {
         "metric": "verify rounds/s", "value": round(value, 2), "unit": "rounds/s", "n_gpus": ws_,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+        "timing": "CUDA-graph replays, CUDA events, max over ranks",
         "roofline": roofline,
-        "round_hbm_gbs": round(round_gbs, 1),
+        "round_hbm_gbs": round(m["round_bytes"] / (ms_max / K / 1e3) / 1e9, 1),
         "draft_tokens_verified_per_s": round(value * draft_per_round, 1),
-        "accepted_tokens_per_s": round(value * B * mean_tau, 1), "mean_tau": round(mean_tau, 4),
-        "e2e": e2e, "gpu_launches": K * kps, "clocks": sampler.summary(), "lazy": lazy,
+        "accepted_tokens_per_s": round(value * B * m["mean_tau"], 1), "mean_tau": round(m["mean_tau"], 4),
+        "accept_length_histogram": m["hist"],
+        "e2e": e2e, "gpu_launches": K * m["kps"], "clocks": m["clocks"], "lazy": lazy,
     }
-    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
+    cpu_here = rank == 0 and ws_ == 1 and not args.no_cpu_baseline
+    if cpu_here:
         cb, o, rows = cpu_baseline(wid, first, args.cpu_seconds)
         one, _, _ = cpu_baseline(wid, first, args.cpu_seconds / 4, nthreads=1)
         cb["value_1thread"] = one["value"]
@@ -630,11 +717,27 @@ def main():
         line["cpu_baseline"] = cb
     elif rank == 0:
         line["cpu_baseline"] = None
+
+    # --- every benchmark configuration, measured the same way
+    per = {}
+    for c in config_list(args):
+        if c == wid:
+            per[str(c)] = config_summary(m, peaks, peak_kind, line.get("cpu_baseline"))
+            continue
+        mc = measure(c, dev, ws_, CONFIG_STEPS.get(c, 200), 10, local, rank)
+        cpu = None
+        if cpu_here:
+            cpu, o, rows = cpu_baseline(c, mc["first"], args.config_cpu_seconds)
+            cpu["parity"] = sample_parity(c, mc["first"], o, rows, mc["ws"])
+        per[str(c)] = config_summary(mc, peaks, peak_kind, cpu)
+        del mc
+        torch.cuda.empty_cache()
+    if per:
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_ > 1:
         dist.barrier()
-        del graph, singles
         dist.destroy_process_group()
 
 
@@ -651,10 +754,13 @@ def run_lazy(wid, sets, ws, steps, alg, world, dev):
     for r, s in zip(runners, sets):
         read += lazy_bytes_read(wid, s, r.num_accepted())
     read /= len(sets)
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    n0 = sv.spec_launch_count()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for r in runners:
             r()
+    launches = (sv.spec_launch_count() - n0) // len(runners)
     reps = max(1, steps // len(runners))
     for _ in range(2):
         graph.replay()
@@ -673,7 +779,7 @@ def run_lazy(wid, sets, ws, steps, alg, world, dev):
     del graph
     return {"entry": "spec_verify_*_lazy (row-on-demand level walk)", "steps": n,
             "ms_per_step": round(ms / n, 6), "value": round(job_value(n, world, ms), 2), "unit": "rounds/s",
-            "gpu_launches_per_step": lazy_kernels_per_step(wid, sets[0]),
+            "gpu_launches_per_step": launches,
             "logit_bytes_read_per_step": int(read), "fraction_of_dense_bytes": round(read / alg, 4),
             "achieved_gbs_on_bytes_read": round(read / (ms / n / 1e3) / 1e9, 1)}
 

@@ -78,7 +78,11 @@ typedef enum {
     SPEC_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     SPEC_ERR_DEVICE_INPUT = 4,  /* (status bit) a sequence had invalid device-side inputs */
     SPEC_ERR_TIMEOUT = 5,       /* (status bit) a bounded device-side wait gave up */
-    SPEC_ERR_WORKSPACE = 6      /* workspace too small or misaligned */
+    SPEC_ERR_WORKSPACE = 6,     /* workspace too small or misaligned */
+    SPEC_ERR_COPY_IN_FLIGHT = 7 /* (status bit) after a timeout, the wait that lets a CTA's own bulk
+                                   copy land gave up too: the copy may still have been writing that
+                                   CTA's shared memory when it went on (results of the call are
+                                   undefined) */
 } spec_status;
 
 typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
@@ -535,6 +539,28 @@ spec_status spec_read_device_status(void* workspace, int* status_out, void* stre
  * Inside stream capture the records become external event nodes.
  */
 spec_status spec_profile_events(void* start_event, void* stop_event);
+
+/*
+ * spec_debug_wait_budget -- testing hook for the device-side timeout path.
+ * The finalize kernels stage data in shared memory with bulk copies and wait
+ * for each copy with a bounded poll (by default 2^24 polls and 1 s); when the
+ * first wait gives up they OR (1 << SPEC_ERR_TIMEOUT) into the status word,
+ * wait again with the full budget so that the copy lands before the CTA goes
+ * on (else also (1 << SPEC_ERR_COPY_IN_FLIGHT)), and then read the staged
+ * statistics from global memory instead, or give up on the sequence (-1 in
+ * its outputs) when the staged row pair was lost.  tries = 0 makes every first
+ * wait give up at once while the copies land normally, which drives that
+ * path without making any copy late; tries < 0 restores the default.
+ * Applies to later calls on the calling host thread.  Not for production use.
+ */
+spec_status spec_debug_wait_budget(long long tries);
+
+/*
+ * spec_launch_count -- number of kernels this library has launched (or, inside
+ * stream capture, added to a graph) from the calling host thread since the
+ * process started.  The difference across a call is that call's launch count.
+ */
+unsigned long long spec_launch_count(void);
 
 /* spec_status_string -- static description of a status code. */
 const char* spec_status_string(spec_status status);

@@ -8,6 +8,8 @@ from .spec_verify import (  # noqa: F401
     SpecError,
     Workspace,
     lib,
+    spec_debug_wait_budget,
+    spec_launch_count,
     spec_profile_events,
     spec_read_device_status,
     spec_verify_chain,

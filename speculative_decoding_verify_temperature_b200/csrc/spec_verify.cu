@@ -16,7 +16,6 @@
 //               the decision, each stages half of the rejected row pair with
 //               bulk copies and scans its residual mass; the halves meet
 //               through distributed shared memory and one CTA draws.
-//     k_chain_final_row   chain, one CTA per sequence, the row pair staged.
 //     k_chain_final       chain, one CTA per (sequence, slice of chunks); the
 //               last to arrive (atomicAdd after __threadfence, no spin-wait)
 //               draws and resets its counter.
@@ -86,7 +85,7 @@ struct Params {
     int rows_tgt;                  // target rows per sequence
     int nsl;                       // chain finalisation: CTAs (slices of chunks) per sequence
     int stage_cap;                 // finalize kernels: shared bytes for a sequence's statistics
-    int stage_off;                 // row-staged chain finalisation: offset of that area
+    int stage_off;                 // pair-staged chain finalisation / MSS walk: offset of the area after the stage
     const char* tgt;
     int64_t tstride;               // bytes between consecutive target rows
     const char* drf;
@@ -108,6 +107,7 @@ struct Params {
     float2* stats2;                // [B][nch][NWARP]   (chain residual chunk sums)
     unsigned* cnt2;                // [B]               (chain residual arrivals)
     unsigned* status;
+    unsigned wait_tries;           // polls of the first wait for a CTA's own bulk copy (0: give up at once)
     // lazy (row-on-demand) verification
     struct LazySeq* lz_seq;        // [B]
     int* lz_rej;                   // [B][rej_cap]      (trees: rejected children tokens)
@@ -235,10 +235,12 @@ __device__ __forceinline__ unsigned long long global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
+// At most `tries` polls (0: give up at once, without polling) and WAIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, unsigned tries = WAIT_LIMIT) {
+    if (tries == 0) return false;
     if (mbar_try(a, parity)) return true;
     const unsigned long long t0 = global_ns();
-    for (unsigned i = 0; i < WAIT_LIMIT; ++i) {
+    for (unsigned i = 0; i < tries; ++i) {
         if (mbar_try(a, parity)) return true;
         if (global_ns() - t0 > WAIT_NS) break;
     }
@@ -250,6 +252,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+
+// A first bounded wait for a CTA's own bulk copy gave up: record it; if the
+// second (full-budget) wait that lets the copy land gave up too, record that
+// the copy may still have been writing this CTA's shared memory when the CTA
+// went on.
+__device__ __forceinline__ void copy_timed_out(const Params& P, bool landed) {
+    atomicOr(P.status, (1u << SPEC_ERR_TIMEOUT) | (landed ? 0u : (1u << SPEC_ERR_COPY_IN_FLIGHT)));
 }
 
 // Stage sequence b's statistics block (R rows of nch*SPC float2, contiguous)
@@ -267,10 +277,12 @@ __device__ const float2* stage_stats(const Params& P, int b, int R, unsigned cha
         bulk_g2s(smem_u32(buf), src, (uint32_t)bytes, smem_u32(bar));
     }
     __syncthreads();
-    if (mbar_wait(smem_u32(bar), 0)) return reinterpret_cast<const float2*>(buf);
-    // the copy did not land in time: report, let it land (bounded), read global
-    if (threadIdx.x == 0) atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
-    mbar_wait(smem_u32(bar), 0);
+    if (__syncthreads_and(mbar_wait(smem_u32(bar), 0, P.wait_tries)))
+        return reinterpret_cast<const float2*>(buf);
+    // the copy did not land in time (for some thread): report, let it land
+    // (bounded), read global memory
+    const bool landed = __syncthreads_and(mbar_wait(smem_u32(bar), 0)) != 0;
+    if (threadIdx.x == 0) copy_timed_out(P, landed);
     return src;
 }
 
@@ -1963,147 +1975,12 @@ template <int TDT, int DDT, int DK> struct WChainResStaged {
     }
 };
 
-// Shared-memory bytes of the row-staged chain finalisation: the row pair,
-// the group sums, then (16-byte aligned) the statistics area.
+// Shared-memory bytes of one CTA's part of a staged row pair (target part,
+// draft part, its group sums), rounded up to 16 bytes; the statistics area
+// follows.
 __host__ __device__ inline size_t staged_bytes(int V, int tesz, int desz) {
     const size_t bt = ((size_t)V * tesz) & ~(size_t)15, bd = ((size_t)V * desz) & ~(size_t)15;
     return (bt + bd + (size_t)((V + 7) / 8) * 4 + 15) & ~(size_t)15;
-}
-
-// Chain finalisation with the rejected row pair staged in shared memory, one
-// CTA per sequence (used when the pair fits and the batch fits in one wave).
-// The decision inputs are prefetched before waiting for the statistics
-// kernel; after the decision, target row k and draft row k arrive with two
-// 1-D bulk copies (TMA) on one mbarrier; max(0, p - q) is evaluated once per
-// element into 8-element group sums, the group sums are scanned block-wide in
-// fp64 in index order, and only the group holding u*S is recomputed to pick
-// the token.  The bonus token (k = gamma) is drawn as in the sliced kernel.
-template <int TDT, int DDT, int DK, bool LZ>
-__global__ void __launch_bounds__(SEQ_BT) k_chain_final_row(const Params P) {
-    __shared__ FinShared sh;
-    __shared__ __align__(8) uint64_t bar, sbar;
-    __shared__ int owner, found_g;
-    extern __shared__ __align__(128) unsigned char stage[];
-    constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
-    const int tid = threadIdx.x, b = blockIdx.x;
-    const int gamma = P.gamma, V = P.V;
-    if constexpr (LZ) {
-        pdl_wait();
-        if (tid == 0) mbar_init(smem_u32(&bar), 1);
-        chain_lazy_state(P, b, sh, true);
-    } else {
-        const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
-        pdl_wait();
-        const float2* blk = stage_stats(P, b, P.R, stage + P.stage_off, P.stage_cap, &sbar);
-        if (tid == 0) mbar_init(smem_u32(&bar), 1);
-        combine_softmax_rows<SEQ_BT>(P, blk, P.R, sh);
-        __syncthreads();
-        chain_decide<TDT, DDT, DK>(P, b, sh, true, pf);
-    }
-    const int ok = sh.ivals[0], k = sh.ivals[1];
-    const float s = (float)sh.dvals[0];
-    if (!ok) return;
-    const float u = P.final_u[b];
-    int32_t* toks = P.out_tokens + (size_t)b * (gamma + 1);
-    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
-    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
-    if (k == gamma) {
-        const float2* st = P.stats + ((size_t)b * P.R + gamma) * P.nch * SPC;
-        double S;
-        int y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, st, s, sh.m[gamma], u, nullptr, 0, sh, &S);
-        if (tid == 0) {
-            toks[k] = y;
-            if (dg) dg[2 * gamma] = 1.0f;
-        }
-        return;
-    }
-    const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
-    const uint32_t bt = ((uint32_t)V * Tr<TDT>::ESZ) & ~15u, bd = ((uint32_t)V * DESZ) & ~15u;
-    unsigned char* ts = stage;
-    unsigned char* ds = stage + bt;
-    float* gs = reinterpret_cast<float*>(stage + bt + bd);
-    if (tid == 0) {
-        mbar_expect_tx(smem_u32(&bar), bt + bd);
-        if (bt) bulk_g2s(smem_u32(ts), trow, bt, smem_u32(&bar));
-        if (bd) bulk_g2s(smem_u32(ds), drow, bd, smem_u32(&bar));
-    }
-    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]);
-    const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
-    const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
-    WChainResStaged<TDT, DDT, DK> wf{ts, ds, trow, drow, (int)(bt / Tr<TDT>::ESZ), (int)(bd / DESZ),
-                                     s, mp, izp, mq, izq, V};
-    if (!mbar_wait(smem_u32(&bar), 0)) {
-        // the copy did not land in time: report, let it finish (bounded), give up on b
-        if (tid == 0) {
-            atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
-            mbar_wait(smem_u32(&bar), 0);
-            for (int i = 0; i <= gamma; ++i) toks[i] = -1;
-            P.out_num_accepted[b] = -1;
-        }
-        return;
-    }
-    // group sums of max(0, p_k - q_k), groups g = tid + i*NT (conflict-free)
-    const int G = (V + 7) / 8;
-    for (int g = tid; g < G; g += SEQ_BT) {
-        float w[8];
-        wf.group((int64_t)g * 8, w);
-        gs[g] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
-    }
-    __syncthreads();
-    // fp64 scan over contiguous ranges of groups, in index order
-    const int g0 = (int)((long long)G * tid / SEQ_BT), g1 = (int)((long long)G * (tid + 1) / SEQ_BT);
-    double seg = 0.0;
-    for (int g = g0; g < g1; ++g) seg += (double)gs[g];
-    if (tid == 0) { owner = -1; found_g = -1; }
-    double S;
-    const double excl = block_excl_scan<SEQ_BT>(seg, &S);
-    const double t = (double)u * S;
-    if (seg > 0.0 && excl <= t) atomicMax(&owner, tid);
-    __syncthreads();
-    int y = -1;
-    if (S > 0.0) {
-        if (tid == owner) {
-            double acc = excl;
-            int gsel = -1, glast = -1;
-            double before = excl;
-            for (int g = g0; g < g1; ++g) {
-                const double v = (double)gs[g];
-                if (v > 0.0) {
-                    glast = g;
-                    before = acc;
-                    if (t < acc + v) { gsel = g; break; }
-                }
-                acc += v;
-            }
-            if (gsel < 0) gsel = glast;
-            float w[8];
-            wf.group((int64_t)gsel * 8, w);
-            const double loc = t - before;
-            double a = 0.0;
-            int pick = -1, last = -1;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                a += (double)w[i];
-                if (w[i] > 0.f) {
-                    last = gsel * 8 + i;
-                    if (pick < 0 && loc < a) pick = gsel * 8 + i;
-                }
-            }
-            found_g = pick >= 0 ? pick : last;
-        }
-        __syncthreads();
-        y = found_g;
-    }
-    if (y < 0) {
-        // empty residual (rounding only): draw from p_k
-        const float2* stk = P.stats + ((size_t)b * P.R + k) * P.nch * SPC;
-        double Su;
-        y = sample_target_row<TDT, SEQ_BT>(trow, V, P.nch, stk, s, mp, u, nullptr, 0, sh, &Su);
-    }
-    if (tid == 0) {
-        toks[k] = y;
-        if (dg) dg[2 * gamma] = (float)S;
-    }
 }
 
 // Thread-block cluster helpers (a pair of CTAs per sequence).
@@ -2201,11 +2078,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SEQ_BT) k_chain_fina
     const float mq = (DK == DK_PROBS) ? 0.f : sh.m[gamma + 1 + k];
     const float izq = (DK == DK_PROBS) ? 0.f : (float)(1.0 / sh.z[gamma + 1 + k]);
     WChainResStaged<TDT, DDT, DK> wf{ts, ds, th, dh, (int)(bt / TESZ), (int)(bd / DESZ), s, mp, izp, mq, izq, Vh};
-    const bool copied = mbar_wait(smem_u32(&bar), 0);
-    if (!copied && tid == 0) {
-        atomicOr(P.status, 1u << SPEC_ERR_TIMEOUT);
-        mbar_wait(smem_u32(&bar), 0);                 // let the copy land (bounded)
-    }
+    // the same verdict in every thread: a wait that gave up in any thread fails the copy
+    const bool copied = __syncthreads_and(mbar_wait(smem_u32(&bar), 0, P.wait_tries)) != 0;
+    if (!copied && tid == 0) copy_timed_out(P, mbar_wait(smem_u32(&bar), 0));   // let the copy land (bounded)
     const int Gh = (Vh + 7) / 8;
     if (copied)
         for (int g = tid; g < Gh; g += SEQ_BT) {
@@ -3745,6 +3620,8 @@ namespace {
 
 thread_local char g_detail[512];
 thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+thread_local unsigned g_wait_tries = WAIT_LIMIT;
+thread_local unsigned long long g_launches = 0;   // kernel launches issued by this host thread
 
 cudaError_t record(cudaEvent_t ev, cudaStream_t st) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -3803,16 +3680,41 @@ Layout make_layout(int entry, int B, int rows, int V) {
     return L;
 }
 
-int num_sms() {
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cache[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+constexpr int MAX_DEVICES = 64;
+
+// A value computed once per device ordinal (with that device current): kernel
+// attributes set with cudaFuncSetAttribute and occupancy queries apply to the
+// current device only, so a process that drives several GPUs needs each one's.
+template <class T>
+class PerDevice {
+  public:
+    template <class F>
+    T get(F make) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return make();
+        std::lock_guard<std::mutex> lock(mu_);
+        if (!set_[dev]) {
+            val_[dev] = make();
+            set_[dev] = true;
+        }
+        return val_[dev];
     }
-    return cache[dev];
+
+  private:
+    std::mutex mu_;
+    bool set_[MAX_DEVICES] = {};
+    T val_[MAX_DEVICES] = {};
+};
+
+int num_sms() {
+    static PerDevice<int> cache;
+    return cache.get([] {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        return n;
+    });
 }
 
 template <class K>
@@ -3846,6 +3748,7 @@ spec_status check_ws(void* ws, size_t bytes, const Layout& L) {
 
 void bind_ws(Params& P, void* ws, const Layout& L) {
     char* w = static_cast<char*>(ws);
+    P.wait_tries = g_wait_tries;
     P.status = reinterpret_cast<unsigned*>(w + L.status);
     P.cnt2 = reinterpret_cast<unsigned*>(w + L.cnt2);
     P.stats = reinterpret_cast<float2*>(w + L.stats);
@@ -3862,6 +3765,7 @@ void bind_ws(Params& P, void* ws, const Layout& L) {
 spec_status launched(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    ++g_launches;
     return SPEC_OK;
 }
 
@@ -3904,7 +3808,8 @@ spec_status launch_dependent(K kernel, unsigned grid, unsigned block, size_t sme
 template <int MODE, int TDT, int DDT>
 spec_status launch_stats(const Params& P, cudaStream_t st) {
     auto kern = k_stats<MODE, TDT, DDT>;
-    static const int occ = blocks_per_sm(kern);
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(kern); });
     const unsigned grid = stats_grid((long long)P.B * P.R * P.nch, occ);
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
     kern<<<grid, NT, 0, st>>>(P);
@@ -3917,11 +3822,16 @@ spec_status launch_stats(const Params& P, cudaStream_t st) {
 // Shared memory for staging a sequence's statistics in the finalize kernels.
 constexpr int STAGE_STATS_MAX = 96 * 1024;
 
-// Allow a finalize kernel STAGE_STATS_MAX bytes of dynamic shared memory (once).
+// Allow a kernel `bytes` of dynamic shared memory on the current device.
+template <class K>
+bool allow_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+// Allow a finalize kernel STAGE_STATS_MAX bytes of dynamic shared memory.
 template <class K>
 bool allow_stage(K kernel) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, STAGE_STATS_MAX) ==
-           cudaSuccess;
+    return allow_smem(kernel, STAGE_STATS_MAX);
 }
 
 
@@ -3931,7 +3841,7 @@ inline int stats_stage_bytes(const Params& P, int rows, size_t limit) {
     return bytes <= limit ? (int)bytes : 0;
 }
 
-// Dynamic shared memory available to a row-staged chain finalisation kernel
+// Dynamic shared memory available to a pair-staged chain finalisation kernel
 // (0 if it cannot be configured).
 template <class K>
 size_t stage_capacity(K kern) {
@@ -3954,8 +3864,9 @@ spec_status launch_chain_final(Params P, cudaStream_t st) {
     constexpr int DESZ = DK == DK_PROBS ? 4 : Tr<DDT>::ESZ;
     // A pair of CTAs per sequence (a cluster) when each half of the rejected
     // row pair fits in shared memory and the pairs fit in a single wave; else
-    // one CTA per sequence with the whole pair staged; else the sliced kernel.
-    static const size_t cap2 = stage_capacity(k_chain_final_pair<TDT, DDT, DK, LZ>);
+    // the sliced kernel.
+    static PerDevice<size_t> cap2_c;
+    const size_t cap2 = cap2_c.get([] { return stage_capacity(k_chain_final_pair<TDT, DDT, DK, LZ>); });
     const int G = (P.V + 7) / 8;
     const size_t half = staged_bytes(min(P.V, 8 * ((G + 1) / 2)), Tr<TDT>::ESZ, DESZ);
     if (P.nch > 1 && half <= cap2 && P.B <= num_sms()) {
@@ -3964,15 +3875,8 @@ spec_status launch_chain_final(Params P, cudaStream_t st) {
         return launch_dependent(k_chain_final_pair<TDT, DDT, DK, LZ>, (unsigned)(2 * P.B), SEQ_BT,
                                 half + P.stage_cap, P, st, "k_chain_final_pair");
     }
-    static const size_t cap = stage_capacity(k_chain_final_row<TDT, DDT, DK, LZ>);
-    const size_t pair = staged_bytes(P.V, Tr<TDT>::ESZ, DESZ);
-    if (P.nch > 1 && pair <= cap && P.B <= num_sms()) {
-        P.stage_off = (int)pair;
-        P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, cap - pair);
-        return launch_dependent(k_chain_final_row<TDT, DDT, DK, LZ>, (unsigned)P.B, SEQ_BT, pair + P.stage_cap, P,
-                                st, "k_chain_final_row");
-    }
-    static const bool big = allow_stage(k_chain_final<TDT, DDT, DK, LZ>);
+    static PerDevice<bool> big_c;
+    const bool big = big_c.get([] { return allow_stage(k_chain_final<TDT, DDT, DK, LZ>); });
     P.stage_cap = LZ ? 0 : stats_stage_bytes(P, P.R, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     // enough CTAs to cover the SMs twice, at most one per chunk
     int nsl = (2 * num_sms() + P.B - 1) / P.B;
@@ -3990,9 +3894,8 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     constexpr size_t hr = filt_hist_bytes<TDT>() > filt_hist_bytes<DDT>() ? filt_hist_bytes<TDT>()
                                                                             : filt_hist_bytes<DDT>();
     constexpr size_t hist = (TDT == SPEC_BF16 || DDT == SPEC_BF16) && VH_BYTES > hr ? VH_BYTES : hr;
-    static const bool attr = cudaFuncSetAttribute(k_filter<TDT, DDT, DK>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) ==
-                             cudaSuccess;
+    static PerDevice<bool> attr_c;
+    const bool attr = attr_c.get([] { return allow_smem(k_filter<TDT, DDT, DK>, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
     s = launch_dependent(k_filter<TDT, DDT, DK>, (unsigned)(P.B * rows), FILT_BT, hist, P, st, "k_filter");
     if (s != SPEC_OK) return s;
@@ -4014,7 +3917,8 @@ spec_status launch_tree(Params P, cudaStream_t st) {
     // the multi-step sampling walk uses the same softmax statistics as target-only sampling
     spec_status s = launch_stats<MODE == MODE_MSS ? MODE_SAMPLE : MODE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
-    static const bool big = allow_stage(k_tree_final<MODE, TDT>);
+    static PerDevice<bool> big_c;
+    const bool big = big_c.get([] { return allow_stage(k_tree_final<MODE, TDT>); });
     P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     size_t smem = P.stage_cap;
     if (MODE == MODE_MSS) {
@@ -4035,14 +3939,14 @@ spec_status launch_tree_filtered(Params P, cudaStream_t st) {
     if (s != SPEC_OK) return s;
     constexpr size_t hr = filt_hist_bytes<TDT>();
     constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
-    static const bool attr = cudaFuncSetAttribute(k_filter<TDT, TDT, DK_NONE, true>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) ==
-                             cudaSuccess;
+    static PerDevice<bool> attr_c;
+    const bool attr = attr_c.get([] { return allow_smem(k_filter<TDT, TDT, DK_NONE, true>, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
     s = launch_dependent(k_filter<TDT, TDT, DK_NONE, true>, (unsigned)(P.B * P.N), FILT_BT, hist, P, st,
                          "k_filter");
     if (s != SPEC_OK) return s;
-    static const bool big = allow_stage(k_tree_final<MODE_SAMPLE_FILT, TDT>);
+    static PerDevice<bool> big_c;
+    const bool big = big_c.get([] { return allow_stage(k_tree_final<MODE_SAMPLE_FILT, TDT>); });
     P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
     return launch_dependent(k_tree_final<MODE_SAMPLE_FILT, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st,
                             "k_tree_final");
@@ -4070,7 +3974,8 @@ template <int TDT, int DDT, int DK>
 spec_status launch_chain_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>;
     auto kd = k_lz_decide_chain<TDT, DDT, DK>;
-    static const int occ = blocks_per_sm(ks);
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const int rpl = P.R > P.rows_tgt ? 2 : 1;
     const unsigned sgrid = stats_grid((long long)P.B * rpl * P.nch, occ);
     const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
@@ -4089,7 +3994,8 @@ template <int TDT>
 spec_status launch_mss_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
     auto kd = k_lz_decide_mss<TDT>;
-    static const int occ = blocks_per_sm(ks);
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
     const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
@@ -4105,7 +4011,8 @@ template <int MODE, int TDT>
 spec_status launch_tree_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE, TDT, TDT>;
     auto kd = k_lz_decide_tree<MODE, TDT>;
-    static const int occ = blocks_per_sm(ks);
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
     const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
@@ -4128,13 +4035,14 @@ spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
     auto kf = k_lz_filter_tree<TDT>;
     auto kd = k_lz_decide_tree<MODE_SAMPLE, TDT, true>;
-    static const int occ = blocks_per_sm(ks);
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
     const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
     constexpr size_t hr = filt_hist_bytes<TDT>();
     constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
-    static const bool attr =
-        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist) == cudaSuccess;
+    static PerDevice<bool> attr_c;
+    const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_lz_filter_tree shared memory attribute");
     if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
     for (int level = 0; level <= P.max_depth; ++level) {
@@ -4195,11 +4103,19 @@ const char* spec_status_string(spec_status s) {
         case SPEC_ERR_DEVICE_INPUT: return "invalid device-side input in a sequence";
         case SPEC_ERR_TIMEOUT: return "device-side wait timed out";
         case SPEC_ERR_WORKSPACE: return "workspace too small or misaligned";
+        case SPEC_ERR_COPY_IN_FLIGHT: return "a timed-out bulk copy may still have been in flight when its CTA went on";
     }
     return "unknown status";
 }
 
 const char* spec_last_error_detail(void) { return g_detail; }
+
+unsigned long long spec_launch_count(void) { return g_launches; }
+
+spec_status spec_debug_wait_budget(long long tries) {
+    g_wait_tries = tries < 0 ? WAIT_LIMIT : (tries > (long long)WAIT_LIMIT ? WAIT_LIMIT : (unsigned)tries);
+    return SPEC_OK;
+}
 
 spec_status spec_profile_events(void* start_event, void* stop_event) {
     g_prof_start = static_cast<cudaEvent_t>(start_event);
@@ -4209,16 +4125,13 @@ spec_status spec_profile_events(void* start_event, void* stop_event) {
 
 }  // extern "C"
 
-static spec_status chain_entry(int mode, int B, int gamma, int V,
-                               const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
-                               const void* draft, spec_dtype ddt, int draft_is_probs,
-                               int64_t d_row_stride,
-                               const int32_t* draft_tokens, const float* temperature,
-                               const float* coins, const float* final_u,
-                               int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
-                               void* workspace, size_t workspace_bytes, void* stream,
-                               const int32_t* top_k = nullptr, const float* top_p = nullptr) {
-    g_detail[0] = 0;
+// Host-side argument checks of the chain entry points (everything except the
+// workspace); B == 0 passes.
+static spec_status chain_args(int B, int gamma, int V, const void* target_logits, spec_dtype tdt,
+                              int64_t t_row_stride, const void* draft, spec_dtype ddt, int draft_is_probs,
+                              int64_t d_row_stride, const int32_t* draft_tokens, const float* temperature,
+                              const float* coins, const float* final_u, const int32_t* out_tokens,
+                              const int32_t* out_num_accepted) {
     if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
     if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);
     if (V < 1 || V > SPEC_MAX_V) return fail(SPEC_ERR_INVALID_ARG, "V = %d outside [1, %d]", V, SPEC_MAX_V);
@@ -4230,6 +4143,23 @@ static spec_status chain_entry(int mode, int B, int gamma, int V,
     if (s != SPEC_OK) return s;
     if (!draft_tokens || !temperature || !coins || !final_u || !out_tokens || !out_num_accepted)
         return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
+    return SPEC_OK;
+}
+
+static spec_status chain_entry(int mode, int B, int gamma, int V,
+                               const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                               const void* draft, spec_dtype ddt, int draft_is_probs,
+                               int64_t d_row_stride,
+                               const int32_t* draft_tokens, const float* temperature,
+                               const float* coins, const float* final_u,
+                               int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                               void* workspace, size_t workspace_bytes, void* stream,
+                               const int32_t* top_k = nullptr, const float* top_p = nullptr) {
+    g_detail[0] = 0;
+    spec_status s = chain_args(B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                               d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens,
+                               out_num_accepted);
+    if (s != SPEC_OK || B == 0) return s;
     const Layout L = make_layout(SPEC_ENTRY_CHAIN, B, gamma, V);
     s = check_ws(workspace, workspace_bytes, L);
     if (s != SPEC_OK) return s;
@@ -4755,8 +4685,14 @@ extern "C" spec_status spec_verify_chain_noalloc(int B, int gamma, int V,
                     "B=%d gamma=%d V=%d needs %zu bytes of scratch; the built-in scratch holds %zu "
                     "(use spec_verify_chain with a caller workspace)",
                     B, gamma, V, L.total, (size_t)SPEC_NOALLOC_SCRATCH_BYTES);
+    // every other argument check runs before anything is enqueued on the
+    // shared array
+    spec_status s = chain_args(B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                               d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens,
+                               out_num_accepted);
+    if (s != SPEC_OK) return s;
     void* scratch = nullptr;
-    spec_status s = noalloc_scratch(&scratch);
+    s = noalloc_scratch(&scratch);
     if (s != SPEC_OK) return s;
     // The area keeps whatever the previous call left there: clear the status
     // word and the arrival counters (everything before the statistics), the

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspecverify.so")
 
 SPEC_OK, SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA = 0, 1, 2, 3
-SPEC_ERR_DEVICE_INPUT, SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE = 4, 5, 6
+SPEC_ERR_DEVICE_INPUT, SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE, SPEC_ERR_COPY_IN_FLIGHT = 4, 5, 6, 7
 SPEC_F32, SPEC_BF16 = 0, 1
 SPEC_ENTRY_CHAIN, SPEC_ENTRY_TREE_GREEDY, SPEC_ENTRY_TREE_SAMPLE, SPEC_ENTRY_TREE_MSS = 0, 1, 2, 3
 
@@ -92,6 +92,10 @@ def lib():
         L.spec_last_error_detail.argtypes = []
         L.spec_profile_events.restype = i32
         L.spec_profile_events.argtypes = [P, P]
+        L.spec_debug_wait_budget.restype = i32
+        L.spec_debug_wait_budget.argtypes = [ctypes.c_longlong]
+        L.spec_launch_count.restype = ctypes.c_ulonglong
+        L.spec_launch_count.argtypes = []
         _lib = L
     return _lib
 
@@ -161,6 +165,18 @@ def spec_profile_events(start=None, stop=None) -> None:
     a = None if start is None else ctypes.c_void_p(start.cuda_event)
     b = None if stop is None else ctypes.c_void_p(stop.cuda_event)
     _check(lib().spec_profile_events(a, b), "spec_profile_events")
+
+
+def spec_launch_count() -> int:
+    """Kernels launched (or captured) by the library from this host thread so far."""
+    return int(lib().spec_launch_count())
+
+
+def spec_debug_wait_budget(tries: int = -1) -> None:
+    """Testing hook: polls of the first wait for each bulk copy the finalize
+    kernels issue, for later calls on this thread (0 = give up at once and take
+    the timeout path; negative = the default budget)."""
+    _check(lib().spec_debug_wait_budget(int(tries)), "spec_debug_wait_budget")
 
 
 class Workspace:

@@ -38,8 +38,9 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     from speculative_decoding_verify_temperature_b200 import spec_verify as sv
-    for s in range(7):
+    for s in range(8):
         assert L.spec_status_string(s)
+        assert L.spec_status_string(s) != b"unknown status"
     assert L.spec_status_string(sv.SPEC_OK) == b"ok"
 
 
@@ -90,6 +91,31 @@ def test_chain_argument_errors_on_host(L):
     assert _chain(L, ws=None) == sv.SPEC_ERR_WORKSPACE
     assert _chain(L, ws=(1 << 24) + 64) == sv.SPEC_ERR_WORKSPACE      # not 256-aligned
     assert _chain(L, wsb=100) == sv.SPEC_ERR_WORKSPACE                 # too small
+
+
+def test_noalloc_rejects_arguments_before_any_cuda_call(L):
+    """The no-allocation chain entry point checks every argument before it
+    touches the device: here, with no GPU, a check that ran after a CUDA call
+    would come back as SPEC_ERR_CUDA instead (on a GPU it would already have
+    enqueued a clear of the shared scratch array)."""
+    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+    f = L.spec_verify_chain_noalloc
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f.restype = i32
+    f.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64, P, P, P, P, P, P, P, P]
+
+    def call(t=FAKE, tdt=1, ts=1000, d=FAKE, ddt=1, probs=0, ds=1000, x=FAKE, na=FAKE):
+        return f(2, 3, 1000, t, tdt, ts, d, ddt, probs, ds, x, FAKE, FAKE, FAKE, FAKE, na, None, None)
+
+    E = sv.SPEC_ERR_INVALID_ARG
+    assert call(t=None) == E
+    assert call(d=None) == E
+    assert call(x=None) == E
+    assert call(na=None) == E
+    assert call(tdt=5) == E
+    assert call(ts=1004) == E
+    assert call(d=FAKE + 2) == E
+    assert call(probs=1, ddt=1) == E
 
 
 def test_tree_argument_errors_on_host(L):

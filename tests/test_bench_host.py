@@ -33,7 +33,51 @@ def test_traffic_record_is_consistent():
         assert t == rec[str(w)]["dram_bytes_per_launch"]
 
 
-def test_job_value_and_launch_counts():
+def test_job_value():
     assert bench.job_value(100, 4, 10.0) == 4 * 100 / 0.01
-    assert bench.kernels_per_step(1, None) == 2 and bench.kernels_per_step(6, None) == 3
-    assert bench.kernels_per_step(7, None) == 6 and bench.kernels_per_step(8, None) == 3
+
+
+class _Inp:
+    def __init__(self, B, gamma, V, probs=True):
+        import torch
+        self.B, self.gamma, self.V, self.draft_is_probs = B, gamma, V, probs
+        self.target = torch.zeros((B, gamma + 1, V), dtype=torch.bfloat16)
+        self.draft = torch.zeros((B, gamma, V), dtype=torch.float32 if probs else torch.bfloat16)
+
+
+def test_round_bytes_count_the_rejected_q_rows():
+    """A chain round with draft probabilities reads every target row, the
+    gathered q(x) of each drafted token, and the full q row of each sequence
+    that rejects (k in [0, gamma)); -1 (invalid) and k = gamma read no q row."""
+    import torch
+    B, g, V = 6, 3, 40
+    inp = _Inp(B, g, V)
+    k = torch.tensor([0, 1, 3, 3, -1, 2], dtype=torch.int32)
+    target = B * (g + 1) * V * 2
+    assert bench.algorithmic_bytes(4, inp) == target
+    assert bench.round_bytes(4, inp, k) == target + B * g * 4 + 3 * V * 4
+    assert bench.round_bytes(4, inp, torch.full((B,), g, dtype=torch.int32)) == target + B * g * 4
+    logits = _Inp(B, g, V, probs=False)
+    both = B * (g + 1) * V * 2 + B * g * V * 2
+    assert bench.round_bytes(1, logits, k) == bench.algorithmic_bytes(1, logits) == both
+
+
+def test_accept_histogram():
+    import torch
+    inp = _Inp(4, 3, 10)
+    h = bench.accept_histogram(1, inp, torch.tensor([0, 3, 3, -1, 2], dtype=torch.int32))
+    assert h == {"-1": 1, "0": 1, "1": 0, "2": 1, "3": 2}
+    h = bench.accept_histogram(1, inp, torch.tensor([1, 1], dtype=torch.int32))
+    assert h == {"0": 0, "1": 2, "2": 0, "3": 0}
+
+
+def test_config_list_defaults():
+    class A:
+        workload, configs = 1, None
+    assert bench.config_list(A) == [0, 1, 2, 3, 4]
+    A.workload = 3
+    assert bench.config_list(A) == []
+    A.configs = "2,4"
+    assert bench.config_list(A) == [2, 4]
+    A.configs = "none"
+    assert bench.config_list(A) == []
