@@ -562,6 +562,18 @@ spec_status spec_debug_wait_budget(long long tries);
  */
 unsigned long long spec_launch_count(void);
 
+/*
+ * spec_debug_bounds_hits -- in a library compiled with -DSPEC_DEBUG_BOUNDS
+ * (libspecverify_debug.so), every data-driven index the kernels use -- a
+ * gathered token id, a parent link, a drawn chunk -- is range-checked on the
+ * device; a failed check is counted and the access skipped (a token gathered
+ * out of range reads as NaN, which invalidates its sequence).  This call
+ * synchronises the device, stores the count since the last call in *hits and
+ * clears it.  A library built without the flag returns SPEC_ERR_UNSUPPORTED
+ * (and *hits = 0).  The checks cost time; they are for debugging.
+ */
+spec_status spec_debug_bounds_hits(unsigned long long* hits);
+
 /* spec_status_string -- static description of a status code. */
 const char* spec_status_string(spec_status status);
 

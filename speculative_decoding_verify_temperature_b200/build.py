@@ -1,4 +1,5 @@
-"""Build libspecverify.so in-tree with nvcc for sm_100a."""
+"""Build libspecverify.so (and its bounds-checked twin libspecverify_debug.so)
+in-tree with nvcc for sm_100a."""
 from __future__ import annotations
 
 import os
@@ -10,6 +11,7 @@ ROOT = os.path.dirname(PKG)
 SRC = [os.path.join(PKG, "csrc", "spec_verify.cu")]
 HDR = os.path.join(ROOT, "include", "spec_verify.h")
 OUT = os.path.join(PKG, "libspecverify.so")
+OUT_DEBUG = os.path.join(PKG, "libspecverify_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -17,6 +19,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "-cudart", "static",
 ]
+DEBUG_FLAGS = ["-DSPEC_DEBUG_BOUNDS"]
 
 
 def nvcc() -> str:
@@ -24,22 +27,33 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(OUT):
+def stale(out: str = OUT) -> bool:
+    if not os.path.exists(out):
         return True
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return any(os.path.getmtime(p) > t for p in SRC + [HDR, __file__])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not (force or stale()):
-        return OUT
-    tmp = OUT + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *SRC, "-o", tmp]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, OUT)
+def _cmd(out: str, extra) -> list:
+    return [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), *SRC, "-o", out + ".tmp"]
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Compile the library (and, with ``debug``, the bounds-checked one) when a
+    source is newer than it; the two compile in parallel.  Returns the path of
+    the library."""
+    jobs = [(o, x) for o, x in [(OUT, []), (OUT_DEBUG, DEBUG_FLAGS)] if (o == OUT or debug) and (force or stale(o))]
+    procs = []
+    for out, extra in jobs:
+        cmd = _cmd(out, extra)
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        procs.append((out, subprocess.Popen(cmd)))
+    failed = [out for out, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(failed)})")
+    for out, _ in procs:
+        os.replace(out + ".tmp", out)
     return OUT
 
 

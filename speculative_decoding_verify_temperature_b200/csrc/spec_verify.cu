@@ -43,6 +43,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "spec_verify.h"
 
 namespace sv {
@@ -147,7 +149,24 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
     return v;
 }
 
-template <int DT> __device__ __forceinline__ float ld_elem(const char* row, int64_t j) {
+// Bounds checks of data-driven indices (token ids, parents, chunk indices),
+// compiled in with -DSPEC_DEBUG_BOUNDS: a failed check is counted in a device
+// counter (spec_debug_bounds_hits) and the access is skipped.  Without the
+// flag every check is the constant true.
+#ifdef SPEC_DEBUG_BOUNDS
+__device__ unsigned long long g_bounds_hits;
+__device__ __forceinline__ bool bounds_ok(bool c) {
+    if (!c) atomicAdd(&g_bounds_hits, 1ull);
+    return c;
+}
+#else
+__device__ __forceinline__ constexpr bool bounds_ok(bool) { return true; }
+#endif
+
+// Element j of a row of V elements (a NaN, counted, when a bounds-checked
+// build finds j outside [0, V)).
+template <int DT> __device__ __forceinline__ float ld_elem(const char* row, int64_t j, int64_t V) {
+    if (!bounds_ok(j >= 0 && j < V)) return __int_as_float(0x7fffffff);
     if constexpr (DT == SPEC_BF16) {
         unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(row) + j);
         return __uint_as_float((uint32_t)h << 16);
@@ -574,7 +593,7 @@ template <int DT> __device__ __forceinline__ void ld8(const char* row, int64_t e
             for (int i = 0; i < 8; ++i) x[i] = vec_elem<DT>(v, i);
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i) : fill;
+            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i, V) : fill;
         }
     } else {
         if (e0 + 8 <= V) {
@@ -583,7 +602,7 @@ template <int DT> __device__ __forceinline__ void ld8(const char* row, int64_t e
             for (int i = 0; i < 4; ++i) { x[i] = vec_elem<DT>(a, i); x[4 + i] = vec_elem<DT>(b, i); }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i) : fill;
+            for (int i = 0; i < 8; ++i) x[i] = (e0 + i < V) ? ld_elem<DT>(row, e0 + i, V) : fill;
         }
     }
 }
@@ -877,6 +896,7 @@ __device__ int rescan_chunk(const WF& wf, int c, int V, double t_loc, float u, d
     __shared__ double wt[GPT][BW];
     __shared__ int owner, found;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (!bounds_ok(c >= 0 && (int64_t)c * CH < V)) c = 0;
     float gs[GPT];
     chunk_group_sums<CH, BT>(wf, c, gs);
     double inc[GPT];
@@ -970,7 +990,8 @@ __device__ int sample_target_row(const char* row, int V, int nch, const float2* 
             bool dup = false;
             for (int j = 0; j < i; ++j) dup |= (excl[j] == t);
             if (dup) continue;
-            double e = exp2((double)ld_elem<TDT>(row, t) * (double)s - (double)m);
+            if (!bounds_ok(t >= 0 && t < V)) continue;
+            double e = exp2((double)ld_elem<TDT>(row, t, V) * (double)s - (double)m);
             double& M = sh.M[t / CH];
             M = fmax(0.0, M - e);
         }
@@ -1036,7 +1057,7 @@ __device__ int tree_valid(const Params& P, int N, int V, int max_depth, FinShare
     if (ok) {
         for (int n = threadIdx.x; n < N; n += BT) {
             int d = 0, a = n;
-            while (a > 0 && d <= max_depth) { a = sh.par[a]; ++d; }
+            while (a > 0 && d <= max_depth) { a = bounds_ok(a < N) ? sh.par[a] : 0; ++d; }
             if (d > max_depth) ok = 0;
         }
     }
@@ -1070,9 +1091,9 @@ __device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) 
         if (f.ok) {
             const char* trow = P.tgt + ((size_t)b * (gamma + 1) + tid) * P.tstride;
             const char* drow = P.drf + ((size_t)b * gamma + tid) * P.dstride;
-            f.l = ld_elem<TDT>(trow, f.x);
+            f.l = ld_elem<TDT>(trow, f.x, P.V);
             if constexpr (DK == DK_PROBS) f.d = __ldg(reinterpret_cast<const float*>(drow) + f.x);
-            else f.d = ld_elem<DDT>(drow, f.x);
+            else f.d = ld_elem<DDT>(drow, f.x, P.V);
         }
     }
     return f;
@@ -1510,7 +1531,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         if (n > 0) {
             int pa = sh.par[n];
             const char* row = P.tgt + ((size_t)b * N + pa) * P.tstride;
-            const float l = ld_elem<TDT>(row, sh.tok[n]);
+            const float l = ld_elem<TDT>(row, sh.tok[n], P.V);
             if (!FILT || l >= sh.th[pa]) pc = prob_d(l, s, sh.m[pa], sh.z[pa]);
         }
         sh.pch[n] = pc;
@@ -1661,7 +1682,7 @@ __device__ int mss_node(const Params& P, int b, int cur, float s, float m, doubl
             const double qx = (double)__ldg(reinterpret_cast<const float*>(drow) + x);
             int verdict = -1;                         // -1 invalid, 0 reject, 1 accept
             if (qx >= 0.0 && qx <= 3.4028234663852886e38) {
-                const double p = fmax(0.0, prob_d(ld_elem<TDT>(row, x), s, m, z) - st.c * qx) / st.D;
+                const double p = fmax(0.0, prob_d(ld_elem<TDT>(row, x, P.V), s, m, z) - st.c * qx) / st.D;
                 if (dg) dg[c] = (float)p;
                 const double ratio = qx > 0.0 ? p / qx : INFINITY;
                 verdict = ((double)P.coins[(size_t)b * N + c] <= ratio) ? 1 : 0;
@@ -1966,7 +1987,7 @@ __device__ __forceinline__ void ld8_staged(const unsigned char* stage, const cha
                 else
                     x[i] = reinterpret_cast<const float*>(stage)[e];
             } else {
-                x[i] = e < V ? ld_elem<DT>(row, e) : fill;
+                x[i] = e < V ? ld_elem<DT>(row, e, V) : fill;
             }
         }
     }
@@ -2444,8 +2465,8 @@ __global__ void __launch_bounds__(NT, FUSED_CTAS_PER_SM) k_chain_fused(const Par
         coin = P.coins[(size_t)b * gamma + i];
         xok = x >= 0 && x < V;
         if (xok) {
-            lx = ld_elem<DT>(trow, x);
-            dx = ld_elem<DT>(drow, x);
+            lx = ld_elem<DT>(trow, x, V);
+            dx = ld_elem<DT>(drow, x, V);
         }
     }
     cp_async_wait_all();
@@ -2519,6 +2540,7 @@ __global__ void __launch_bounds__(NT, FUSED_CTAS_PER_SM) k_chain_fused(const Par
         t = (double)u * fused_target_masses(xst, nch, mp, Mt);
         cs = mass_crossing(Mt, nch, t, &before);
     }
+    if (!bounds_ok(cs < nch)) cs = -1;
     const int writer = cs >= 0 ? cs : 0;
     if ((int)c != writer) return;                 // no CTA reads another's shared memory after the barriers
     int y = -1;
@@ -2622,7 +2644,8 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
 // largest logit whose set {l >= theta_p} carries a top_p share of the set's
 // mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds are found over
 // order-preserving keys of the logits (-0 folded onto +0): for bf16 rows an
-// exact histogram of the 65536 possible keys (vh_build / vh_select), for f32
+// exact count histogram of a window of keys below the row's maximum
+// (wfilter_row), for f32
 // rows (and a bf16 row whose histogram counter would wrap) a radix descent of
 // 12 + 12 + 8 bit digits (filter_row).  Counts decide top-k; masses are fixed
 // point (2^-40 units, integer sums, so they do not depend on the order of the
@@ -2844,28 +2867,6 @@ __device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, f
     return r;
 }
 
-// bf16 rows: an exact histogram of the row's values (65536 order keys, two
-// 16-bit counters per 32-bit word, 128 KB of shared memory) from one pass;
-// every mass then follows exactly as count * fixed(2^(v s - m)) per value,
-// the same fixed-point numbers the radix path adds element by element.
-//
-// A row has at most V distinct values, so most of the 32768 words are empty.
-// Thread t reads the 32 words of key block 1023 - t (16-byte loads, the four
-// quads of a block stored XOR-swizzled by the block index so that eight
-// consecutive threads hit eight distinct bank groups), and a block-wide scan
-// packs the indices of the non-empty words into a list in descending key
-// order.  The counts and masses are then summed over equal slices of that
-// list, so the exp2 work is spread evenly whatever the values' spread, and
-// one more scan orders the slices: the top-k key is where the running count
-// reaches top_k, the top-p key where the running mass reaches top_p times the
-// mass kept by top-k.
-constexpr int VH_WORDS = 32768;
-constexpr size_t VH_BYTES = (size_t)VH_WORDS * 4 + (size_t)VH_WORDS * 2;   // counters + word list
-
-// Physical word of logical word i (= key >> 1): block i >> 5, quad
-// ((i >> 2) & 7) ^ (block & 7), lane i & 3.
-__device__ __forceinline__ uint32_t vh_phys(uint32_t i) { return i ^ ((i >> 3) & 0x1Cu); }
-
 // Order keys of the two bf16 values packed in x (low half = lower index), as
 // order_key does for one value: -0 folded onto +0, negative values
 // complemented, the sign bit of the others set.
@@ -2873,20 +2874,39 @@ __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
     x &= ~__vcmpeq2(x, 0x80008000u);
     return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
 }
-__device__ __forceinline__ void vh_count1(uint32_t* w, uint32_t k) {
-    atomicAdd(&w[vh_phys(k >> 1)], (k & 1u) ? 0x10000u : 1u);
-}
-__device__ __forceinline__ unsigned long long vh_mass(unsigned c, uint32_t k, float s, float m) {
-    if (c == 0u) return 0ull;
-    return (unsigned long long)c *
-           (unsigned long long)(ex2(fmaf(key_value<SPEC_BF16>(k), s, -m)) * (float)FIX_ONE);
+
+// bf16 rows, windowed: an exact count histogram of WF_KEYS consecutive order
+// keys (u32 counters, 32 KB) from the row's largest key down, plus exact
+// integer totals -- counts and fixed-point masses, count * fixed(2^(v s - m))
+// per value -- of the elements above and below the window.  Every key's
+// mass is count * fixed(2^(v s - m)), so the running counts and masses from
+// the top, and with them the top-k key, the kept mass and the top-p key, are
+// the integers of the full value histogram.  A threshold that falls outside
+// the window moves it (up to the row's true maximum, or down below it) and
+// the row is counted again; the first window holds both thresholds unless the
+// kept set reaches far below the maximum.
+constexpr int WF_KEYS = 8192;
+constexpr size_t WF_BYTES = (size_t)WF_KEYS * 4;
+
+struct WinShared {
+    unsigned long long red[32];
+    unsigned redc[32];
+    unsigned long long am, bm, tm;        // masses above / below the window, window total
+    unsigned ac, bc, tc, amax;            // counts above / below, window total, largest key above
+    int sel;
+    unsigned long long at;
+};
+
+__device__ __forceinline__ unsigned long long fix_mass(float x, float s, float m) {
+    return (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE);
 }
 
-// Exclusive block-wide scan, in thread order, of a u32 and a u64; the totals
-// go to *ta / *tb.  All threads call it.
-__device__ void vh_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
-                         unsigned long long* tb, FiltShared& fs) {
-    static_assert(FILT_BT == 1024, "one warp scans the 32 warp totals");
+// Block-wide exclusive scan, in thread order, of a u32 and a u64 (BT threads,
+// BT / 32 <= 32 warps); the totals go to *ta / *tb.  All threads call it.
+template <int BT>
+__device__ void wf_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
+                         unsigned long long* tb, WinShared& ws) {
+    constexpr int NW = BT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned ia = a;
     unsigned long long ib = b;
@@ -2896,11 +2916,11 @@ __device__ void vh_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigne
         const unsigned long long vb = __shfl_up_sync(FULL, ib, o);
         if (lane >= o) { ia += va; ib += vb; }
     }
-    if (lane == 31) { fs.redc[warp] = ia; fs.red[warp] = ib; }
+    if (lane == 31) { ws.redc[warp] = ia; ws.red[warp] = ib; }
     __syncthreads();
     if (warp == 0) {
-        const unsigned xa = fs.redc[lane];
-        const unsigned long long xb = fs.red[lane];
+        const unsigned xa = lane < NW ? ws.redc[lane] : 0u;
+        const unsigned long long xb = lane < NW ? ws.red[lane] : 0ull;
         unsigned sa = xa;
         unsigned long long sb = xb;
 #pragma unroll
@@ -2909,164 +2929,191 @@ __device__ void vh_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigne
             const unsigned long long vb = __shfl_up_sync(FULL, sb, o);
             if (lane >= o) { sa += va; sb += vb; }
         }
-        fs.redc[lane] = sa - xa;
-        fs.red[lane] = sb - xb;
-        if (lane == 31) { fs.tc = sa; fs.tm = sb; }
+        if (lane < NW) { ws.redc[lane] = sa - xa; ws.red[lane] = sb - xb; }
+        if (lane == 31) { ws.tc = sa; ws.tm = sb; }
     }
     __syncthreads();
-    *ea = fs.redc[warp] + ia - a;
-    *eb = fs.red[warp] + ib - b;
-    *ta = fs.tc;
-    *tb = fs.tm;
-    __syncthreads();                                   // fs is free again
+    *ea = ws.redc[warp] + ia - a;
+    *eb = ws.red[warp] + ib - b;
+    *ta = ws.tc;
+    *tb = ws.tm;
+    __syncthreads();
 }
 
-// The value histogram of a bf16 row and its list of non-empty words (from the
-// logits alone, before the statistics are needed).  Returns the list length.
-// All threads call it.
-__device__ int vh_build(const char* row, int V, FiltShared& fs, uint32_t* w) {
+// One pass over a bf16 row: the window [khi - WF_KEYS + 1, khi] counted per
+// key in win[khi - key]; the rest summed into ws.ac/am/amax (above) and
+// ws.bc/bm (below).  All threads call it.
+template <int BT>
+__device__ void wf_pass(const char* row, int V, float s, float m, uint32_t khi, uint32_t* win, WinShared& ws) {
     const int tid = threadIdx.x;
-    uint4* w4 = reinterpret_cast<uint4*>(w);
-    unsigned short* list = reinterpret_cast<unsigned short*>(w + VH_WORDS);
-    // histogram: four 16-byte loads per thread in flight (the first four
-    // while the counters are cleared), then the updates
+    const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
+    for (int i = tid; i < WF_KEYS / 4; i += BT) reinterpret_cast<uint4*>(win)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid == 0) { ws.ac = 0u; ws.bc = 0u; ws.am = 0ull; ws.bm = 0ull; ws.amax = 0u; }
+    __syncthreads();
+    unsigned ac = 0u, bc = 0u, amax = 0u;
+    unsigned long long am = 0ull, bm = 0ull;
     const int nv = (V + 7) / 8;
-    uint4 v[4];
-    auto load4 = [&](int v0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int vi = v0 + q * FILT_BT;
-            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
+    auto one = [&](uint32_t k) {
+        if (k > khi) {
+            ++ac;
+            amax = max(amax, k);
+            am += fix_mass(key_value<SPEC_BF16>(k), s, m);
+        } else if (k >= klo) {
+            atomicAdd(&win[khi - k], 1u);
+        } else {
+            ++bc;
+            bm += fix_mass(key_value<SPEC_BF16>(k), s, m);
         }
     };
-    load4(tid);
-    for (int i = tid; i < VH_WORDS / 4; i += FILT_BT) w4[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
-    for (int v0 = tid;;) {
+    for (int v0 = tid; v0 < nv; v0 += 4 * BT) {
+        uint4 v[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int vi = v0 + q * FILT_BT;
+            const int vi = v0 + q * BT;
+            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * BT;
             if (vi >= nv) break;
             const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-            const int lim = V - vi * 8;                   // elements of this vector inside the row
+            const int lim = V - vi * 8;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const uint32_t k2 = vh_keys2(xs[c]);
-                if (2 * c < lim) vh_count1(w, k2 & 0xFFFFu);
-                if (2 * c + 1 < lim) vh_count1(w, k2 >> 16);
+                if (2 * c < lim) one(k2 & 0xFFFFu);
+                if (2 * c + 1 < lim) one(k2 >> 16);
             }
         }
-        v0 += 4 * FILT_BT;
-        if (v0 >= nv) break;
-        load4(v0);
     }
-    __syncthreads();
-    // non-empty words of this thread's block, highest first
-    const uint32_t blk = (uint32_t)(VH_WORDS / 32 - 1 - tid);
-    uint32_t mask = 0u;
+    // fold the per-thread totals (integers: any order gives the same sums)
+    ac = __reduce_add_sync(FULL, ac);
+    bc = __reduce_add_sync(FULL, bc);
+    amax = __reduce_max_sync(FULL, amax);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const uint4 x = w4[blk * 8 + (q ^ (blk & 7u))];
-        mask |= (x.x ? 1u : 0u) << (4 * q) | (x.y ? 1u : 0u) << (4 * q + 1) | (x.z ? 1u : 0u) << (4 * q + 2) |
-                (x.w ? 1u : 0u) << (4 * q + 3);
+    for (int o = 16; o; o >>= 1) {
+        am += __shfl_xor_sync(FULL, am, o);
+        bm += __shfl_xor_sync(FULL, bm, o);
     }
-    unsigned off, n;
-    unsigned long long d0, d1;
-    vh_scan2((unsigned)__popc(mask), 0ull, &off, &d0, &n, &d1, fs);
-    while (mask) {
-        const int j = 31 - __clz(mask);
-        list[off++] = (unsigned short)(blk * 32 + j);
-        mask &= ~(1u << j);
+    if ((tid & 31) == 0) {
+        atomicAdd(&ws.ac, ac);
+        atomicAdd(&ws.bc, bc);
+        atomicMax(&ws.amax, amax);
+        atomicAdd(&ws.am, am);
+        atomicAdd(&ws.bm, bm);
     }
     __syncthreads();
-    return (int)n;
 }
 
-// Threshold and kept mass of a bf16 row from its value histogram and word
-// list (vh_build).  Returns false when a value occurs 65536 times or more (a
-// 16-bit counter wrapped: possible only for V > 65535); the caller then takes
-// the radix path.  All threads call it.
-__device__ bool vh_select(int V, int n, float s, float m, int K, float Pp, FiltShared& fs, const uint32_t* w,
-                          FiltRec* out) {
+// Threshold and kept mass of one bf16 row (the record filter_row gives).  The
+// first window starts just above the key of the row's maximum estimated from
+// the statistics (m / s).  All threads call it.
+template <int BT>
+__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, uint32_t* win,
+                               WinShared& ws) {
+    constexpr int RUN = WF_KEYS / BT;                 // window keys per thread
+    static_assert(RUN * BT == WF_KEYS, "window split");
     const int tid = threadIdx.x;
-    const unsigned short* list = reinterpret_cast<const unsigned short*>(w + VH_WORDS);
-    // counts and masses of this thread's slice of the list
-    const int e0 = (int)((long long)n * tid / FILT_BT), e1 = (int)((long long)n * (tid + 1) / FILT_BT);
-    unsigned cs = 0u;
-    unsigned long long ms = 0ull;
-    for (int e = e0; e < e1; ++e) {
-        const uint32_t i = list[e];
-        const uint32_t x = w[vh_phys(i)];
-        cs += (x >> 16) + (x & 0xFFFFu);
-        ms += vh_mass(x >> 16, 2 * i + 1, s, m) + vh_mass(x & 0xFFFFu, 2 * i, s, m);
-    }
-    unsigned c0, ctot;
-    unsigned long long m0, mtot;
-    vh_scan2(cs, ms, &c0, &m0, &ctot, &mtot, fs);
-    if (V > 65535 && ctot != (unsigned)V) return false;   // a counter wrapped (the same in every thread)
+    FiltRec r{-INFINITY, 0, 0.0};
     const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
-    // top-k: the first key (from the top) where the running count reaches K
-    if (tid == 0) { fs.sel = 0; fs.at = mtot; }          // top-p alone: every key is kept
-    __syncthreads();
-    if (use_k && c0 < (unsigned)K && c0 + cs >= (unsigned)K) {
-        unsigned c = c0;
-        unsigned long long mm = m0;
-        for (int e = e0; e < e1; ++e) {
-            const uint32_t i = list[e];
-            const uint32_t x = w[vh_phys(i)];
-            const unsigned ch = x >> 16, cl = x & 0xFFFFu;
-            c += ch;
-            mm += vh_mass(ch, 2 * i + 1, s, m);
-            if (c >= (unsigned)K) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
-            c += cl;
-            mm += vh_mass(cl, 2 * i, s, m);
-            if (c >= (unsigned)K) { fs.sel = (int)(2 * i); fs.at = mm; break; }
+    if (!use_k && !use_p) return r;
+    // the row's largest value is about m / s (m = its value times s, rounded)
+    uint32_t khi = min(0xFFFFu, order_key<SPEC_BF16>(__bfloat162float(__float2bfloat16_rn(m / s))) + 4u);
+    bool rk = !use_k;                                 // top-k resolved
+    uint32_t tk = 0u, tp = 0u;
+    unsigned long long zk = 0ull, z = 0ull;
+    for (int it = 0; it < 2 * (65536 / WF_KEYS) + 2; ++it) {
+        wf_pass<BT>(row, V, s, m, khi, win, ws);
+        const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
+        const unsigned ac = ws.ac, amax = ws.amax;
+        const unsigned long long am = ws.am, bm = ws.bm;
+        // this thread's run of window indices [j0, j0 + RUN): keys khi - j
+        const int j0 = tid * RUN;
+        unsigned rc = 0u;
+        unsigned long long rm = 0ull;
+#pragma unroll 4
+        for (int j = j0; j < j0 + RUN; ++j) {
+            const unsigned c = win[j];
+            if (c) {
+                rc += c;
+                rm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+            }
         }
-    }
-    __syncthreads();
-    uint32_t t = (uint32_t)fs.sel;
-    const unsigned long long zk = fs.at;
-    unsigned long long z = zk;
-    if (use_p) {
-        // the first key where the running mass reaches top_p of the kept mass
-        // (a key >= the top-k key, since the running mass there is zk)
+        unsigned c0, ctot;
+        unsigned long long m0, mtot;
+        wf_scan2<BT>(rc, rm, &c0, &m0, &ctot, &mtot, ws);
+        c0 += ac;
+        m0 += am;
+        if (!use_k) zk = am + mtot + bm;
+        if (!rk) {
+            if ((unsigned)K <= ac) { khi = amax; continue; }                 // above the window
+            if ((unsigned)K > ac + ctot) {                                   // below the window
+                if (klo == 0u) break;                                        // (cannot happen: K < V)
+                khi = klo - 1u;
+                continue;
+            }
+            if (tid == 0) ws.sel = -1;
+            __syncthreads();
+            if (c0 < (unsigned)K && c0 + rc >= (unsigned)K) {
+                unsigned c = c0;
+                unsigned long long mm = m0;
+                for (int j = j0; j < j0 + RUN; ++j) {
+                    const unsigned cj = win[j];
+                    c += cj;
+                    if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+                    if (c >= (unsigned)K) { ws.sel = j; ws.at = mm; break; }
+                }
+            }
+            __syncthreads();
+            tk = khi - (uint32_t)ws.sel;
+            zk = ws.at;
+            rk = true;
+            __syncthreads();
+        }
+        if (!use_p) { tp = tk; z = zk; break; }
         const double target = (double)Pp * (double)zk;
+        if ((double)am >= target) { khi = amax; continue; }                 // above the window
+        if ((double)(am + mtot) < target) {                                 // below (top-p alone)
+            if (klo == 0u) break;                                            // (cannot happen: target <= total)
+            khi = klo - 1u;
+            continue;
+        }
+        if (tid == 0) ws.sel = -1;
         __syncthreads();
-        if (tid == 0) fs.sel = -1;
-        __syncthreads();
-        if ((double)m0 < target && (double)(m0 + ms) >= target) {
+        if ((double)m0 < target && (double)(m0 + rm) >= target) {
             unsigned long long mm = m0;
-            for (int e = e0; e < e1; ++e) {
-                const uint32_t i = list[e];
-                const uint32_t x = w[vh_phys(i)];
-                mm += vh_mass(x >> 16, 2 * i + 1, s, m);
-                if ((double)mm >= target) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
-                mm += vh_mass(x & 0xFFFFu, 2 * i, s, m);
-                if ((double)mm >= target) { fs.sel = (int)(2 * i); fs.at = mm; break; }
+            for (int j = j0; j < j0 + RUN; ++j) {
+                const unsigned cj = win[j];
+                if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+                if (cj && (double)mm >= target) { ws.sel = j; ws.at = mm; break; }
             }
         }
         __syncthreads();
-        if (fs.sel >= 0) {
-            t = (uint32_t)fs.sel;
-            z = fs.at;
-        }
+        tp = khi - (uint32_t)ws.sel;
+        z = ws.at;
+        __syncthreads();
+        break;
     }
-    out->theta = key_value<SPEC_BF16>(t);
-    out->on = 1;
-    out->Z = (double)z / FIX_ONE;
-    return true;
+    r.theta = key_value<SPEC_BF16>(tp);
+    r.on = 1;
+    r.Z = (double)z / FIX_ONE;
+    return r;
 }
 
 // Filter thresholds of every row of a chain round, one CTA per (sequence,
 // row): target rows 0..gamma, then the draft-logit rows (TREE: the N node
-// rows of every tree).  A bf16 row's value
-// histogram needs only the logits, so it is built before waiting for the
-// statistics (the rows' maxima, which the masses are relative to).  Every CTA
-// waits before it exits, so the finalize kernel that follows (and reads the
-// records and the statistics) waits for the statistics through this kernel.
-template <int TDT, int DDT, int DK, bool TREE = false>
-__global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
+// rows of every tree).  bf16 rows take the windowed histogram (wfilter_row),
+// f32 rows the radix descent (filter_row, which needs FILT_BT threads); a
+// launch whose rows are all bf16 runs WF_BT threads per CTA and 32 KB of
+// shared memory, so several rows share an SM.  Every CTA waits for the
+// statistics before it exits, so the finalize kernel that follows (and reads
+// the records and the statistics) waits for them through this kernel.
+constexpr int WF_BT = 256;
+
+template <int TDT, int DDT, int DK, bool TREE, int BT>
+__global__ void __launch_bounds__(BT) k_filter(const Params P) {
     __shared__ FiltShared fs;
+    __shared__ WinShared ws;
     __shared__ float msh;
     __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
@@ -3077,13 +3124,12 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     const int K = P.top_k ? P.top_k[b] : 0;
     const float Pp = P.top_p ? P.top_p[b] : 1.f;
     const float T = P.temperature[b];
+    pdl_wait();
     if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
-        pdl_wait();
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
         return;
     }
     if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
-        pdl_wait();
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
@@ -3091,10 +3137,6 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
     const char* row = TREE  ? P.tgt + ((size_t)b * P.N + r) * P.tstride
                       : tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
                             : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
-    const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
-    uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
-    const int n = vh ? vh_build(row, P.V, fs, w) : 0;
-    pdl_wait();
     const int E = P.nch * SPC;
     if (threadIdx.x < 32) {
         float m;
@@ -3108,8 +3150,10 @@ __global__ void __launch_bounds__(FILT_BT) k_filter(const Params P) {
         return;
     }
     const float s = scale_of(T), m = msh;
-    FiltRec rec;
-    if (!vh || !vh_select(P.V, n, s, m, K, Pp, fs, w, &rec)) {
+    FiltRec rec{-INFINITY, 0, 0.0};
+    if ((tgt ? TDT : DDT) == SPEC_BF16) {
+        rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, reinterpret_cast<uint32_t*>(dyn), ws);
+    } else if constexpr (BT == FILT_BT) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
     }
@@ -3276,10 +3320,10 @@ __global__ void __launch_bounds__(NT) k_vp_rows(const Params P, ShardRec* out, i
             if (x >= 0 && x < P.V) {
                 rec.has = 1;
                 if (r <= gamma) {
-                    rec.val = ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride, x);
+                    rec.val = ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride, x, P.V);
                 } else {
                     const char* drow = P.drf + ((size_t)b * gamma + i) * P.dstride;
-                    rec.val = (DK == DK_PROBS) ? __ldg(reinterpret_cast<const float*>(drow) + x) : ld_elem<DDT>(drow, x);
+                    rec.val = (DK == DK_PROBS) ? __ldg(reinterpret_cast<const float*>(drow) + x) : ld_elem<DDT>(drow, x, P.V);
                 }
             }
         }
@@ -3683,13 +3727,13 @@ __global__ void __launch_bounds__(NT) k_lz_decide_chain(const Params P) {
     ok &= (x >= 0 && x < P.V);
     double p = 0.0, q = 0.0;
     if (ok) {
-        p = prob_d(ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, x), s, m, z);
+        p = prob_d(ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, x, P.V), s, m, z);
         const char* drow = P.drf + ((size_t)b * gamma + level) * P.dstride;
         if constexpr (DK == DK_PROBS) {
             q = (double)__ldg(reinterpret_cast<const float*>(drow) + x);
             ok &= (q >= 0.0 && q <= 3.0e38);
         } else {
-            q = prob_d(ld_elem<DDT>(drow, x), s, mq, zq);
+            q = prob_d(ld_elem<DDT>(drow, x, P.V), s, mq, zq);
         }
     }
     LazySeq L;
@@ -3733,7 +3777,7 @@ __device__ bool warp_tree_valid(const Params& P, int b) {
     if (good) {
         for (int n = lane; n < N; n += 32) {
             int d = 0, a = n;
-            while (a > 0 && d <= P.max_depth) { a = par[a]; ++d; }
+            while (a > 0 && d <= P.max_depth) { a = bounds_ok(a < N) ? par[a] : 0; ++d; }
             good &= d <= P.max_depth;
         }
         good = __all_sync(FULL, good);
@@ -3819,7 +3863,7 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
                     int t = 0;
                     if (child) {
                         t = tok[c];
-                        const float l = ld_elem<TDT>(trow, t);
+                        const float l = ld_elem<TDT>(trow, t, P.V);
                         if (!FILT || l >= th) pc = prob_d(l, L.s, m, z);
                         if (dg) dg[c] = (float)pc;
                     }
@@ -3871,9 +3915,10 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
 // Lazy filtered tree walk: the filter record of the current node's row of
 // every active sequence at this level (one CTA each, as k_filter), between
 // the level's statistics and its decisions.
-template <int TDT>
-__global__ void __launch_bounds__(FILT_BT) k_lz_filter_tree(const Params P) {
+template <int TDT, int BT>
+__global__ void __launch_bounds__(BT) k_lz_filter_tree(const Params P) {
     __shared__ FiltShared fs;
+    __shared__ WinShared ws;
     __shared__ float msh;
     __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
@@ -3908,10 +3953,9 @@ __global__ void __launch_bounds__(FILT_BT) k_lz_filter_tree(const Params P) {
     }
     const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
     const float s = scale_of(T), m = msh;
-    uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
-    FiltRec rec;
-    if (TDT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, K, Pp, fs, w, &rec))
-        rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
+    FiltRec rec{-INFINITY, 0, 0.0};
+    if constexpr (TDT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, reinterpret_cast<uint32_t*>(dyn), ws);
+    else if constexpr (BT == FILT_BT) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
     if (threadIdx.x == 0) *out = rec;
 }
 
@@ -4050,6 +4094,15 @@ using namespace sv;
 namespace {
 
 thread_local char g_detail[512];
+
+// An NVTX range around one C-ABI call (visible in Nsight Systems timelines;
+// a no-op without a tool attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
 thread_local unsigned g_wait_tries = WAIT_LIMIT;
 thread_local unsigned long long g_launches = 0;   // kernel launches issued by this host thread
@@ -4326,13 +4379,17 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
     const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
-    constexpr size_t hr = filt_hist_bytes<TDT>() > filt_hist_bytes<DDT>() ? filt_hist_bytes<TDT>()
-                                                                            : filt_hist_bytes<DDT>();
-    constexpr size_t hist = (TDT == SPEC_BF16 || DDT == SPEC_BF16) && VH_BYTES > hr ? VH_BYTES : hr;
+    // all rows bf16: windowed histograms, WF_BT threads; else FILT_BT threads
+    // and room for an f32 row's radix histograms
+    constexpr bool all_bf16 = TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16);
+    constexpr int bt = all_bf16 ? WF_BT : FILT_BT;
+    constexpr size_t hist = all_bf16 ? WF_BYTES
+                                     : (filt_hist_bytes<SPEC_F32>() > WF_BYTES ? filt_hist_bytes<SPEC_F32>() : WF_BYTES);
+    auto kf = k_filter<TDT, DDT, DK, false, bt>;
     static PerDevice<bool> attr_c;
-    const bool attr = attr_c.get([] { return allow_smem(k_filter<TDT, DDT, DK>, hist); });
+    const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
-    s = launch_dependent(k_filter<TDT, DDT, DK>, (unsigned)(P.B * rows), FILT_BT, hist, P, st, "k_filter");
+    s = launch_dependent(kf, (unsigned)(P.B * rows), bt, hist, P, st, "k_filter");
     if (s != SPEC_OK) return s;
     const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
     return launch_dependent(k_chain_final_filt<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, wpw, P, st,
@@ -4401,13 +4458,13 @@ template <int TDT>
 spec_status launch_tree_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_SAMPLE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
-    constexpr size_t hr = filt_hist_bytes<TDT>();
-    constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
+    constexpr int bt = TDT == SPEC_BF16 ? WF_BT : FILT_BT;
+    constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
+    auto kf = k_filter<TDT, TDT, DK_NONE, true, bt>;
     static PerDevice<bool> attr_c;
-    const bool attr = attr_c.get([] { return allow_smem(k_filter<TDT, TDT, DK_NONE, true>, hist); });
+    const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
-    s = launch_dependent(k_filter<TDT, TDT, DK_NONE, true>, (unsigned)(P.B * P.N), FILT_BT, hist, P, st,
-                         "k_filter");
+    s = launch_dependent(kf, (unsigned)(P.B * P.N), bt, hist, P, st, "k_filter");
     if (s != SPEC_OK) return s;
     static PerDevice<bool> big_c;
     const bool big = big_c.get([] { return allow_stage(k_tree_final<MODE_SAMPLE_FILT, TDT>); });
@@ -4497,14 +4554,14 @@ spec_status launch_tree_lazy(Params P, cudaStream_t st) {
 template <int TDT>
 spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
-    auto kf = k_lz_filter_tree<TDT>;
+    constexpr int fbt = TDT == SPEC_BF16 ? WF_BT : FILT_BT;
+    auto kf = k_lz_filter_tree<TDT, fbt>;
     auto kd = k_lz_decide_tree<MODE_SAMPLE, TDT, true>;
     static PerDevice<int> occ_c;
     const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
     const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
-    constexpr size_t hr = filt_hist_bytes<TDT>();
-    constexpr size_t hist = TDT == SPEC_BF16 && VH_BYTES > hr ? VH_BYTES : hr;
+    constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_lz_filter_tree shared memory attribute");
@@ -4512,7 +4569,7 @@ spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
     for (int level = 0; level <= P.max_depth; ++level) {
         spec_status s = launch_level(ks, sgrid, (void (*)(Params))nullptr, 0, P, level, st);
         if (s != SPEC_OK) return s;
-        s = launch_dependent(kf, (unsigned)P.B, FILT_BT, hist, P, st, "k_lz_filter_tree");
+        s = launch_dependent(kf, (unsigned)P.B, fbt, hist, P, st, "k_lz_filter_tree");
         if (s != SPEC_OK) return s;
         s = launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
         if (s != SPEC_OK) return s;
@@ -4575,6 +4632,21 @@ const char* spec_status_string(spec_status s) {
 const char* spec_last_error_detail(void) { return g_detail; }
 
 unsigned long long spec_launch_count(void) { return g_launches; }
+
+spec_status spec_debug_bounds_hits(unsigned long long* hits) {
+    if (!hits) return fail(SPEC_ERR_INVALID_ARG, "hits is NULL");
+#ifdef SPEC_DEBUG_BOUNDS
+    unsigned long long zero = 0ull;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(hits, g_bounds_hits, sizeof *hits);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_bounds_hits, &zero, sizeof zero);
+    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "bounds counter: %s", cudaGetErrorString(e));
+    return SPEC_OK;
+#else
+    *hits = 0ull;
+    return fail(SPEC_ERR_UNSUPPORTED, "this build has no bounds checks (compile with -DSPEC_DEBUG_BOUNDS)");
+#endif
+}
 
 spec_status spec_debug_wait_budget(long long tries) {
     g_wait_tries = tries < 0 ? WAIT_LIMIT : (tries > (long long)WAIT_LIMIT ? WAIT_LIMIT : (unsigned)tries);
@@ -4819,8 +4891,14 @@ static spec_status mss_entry(bool lazy, int B, int N, int V, int max_depth,
 
 extern "C" {
 
-spec_status spec_verify_chain(SPEC_CHAIN_ARGS_DECL) { return chain_entry(0, SPEC_CHAIN_ARGS); }
-spec_status spec_verify_chain_lazy(SPEC_CHAIN_ARGS_DECL) { return chain_entry(1, SPEC_CHAIN_ARGS); }
+spec_status spec_verify_chain(SPEC_CHAIN_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_chain");
+    return chain_entry(0, SPEC_CHAIN_ARGS);
+}
+spec_status spec_verify_chain_lazy(SPEC_CHAIN_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_chain_lazy");
+    return chain_entry(1, SPEC_CHAIN_ARGS);
+}
 
 spec_status spec_verify_chain_filtered(int B, int gamma, int V,
                                        const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
@@ -4831,15 +4909,28 @@ spec_status spec_verify_chain_filtered(int B, int gamma, int V,
                                        const int32_t* top_k, const float* top_p,
                                        int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
                                        void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_verify_chain_filtered");
     if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
     return chain_entry(2, B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
                        d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens, out_num_accepted,
                        diag, workspace, workspace_bytes, stream, top_k, top_p);
 }
-spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(false, SPEC_GREEDY_ARGS); }
-spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) { return greedy_entry(true, SPEC_GREEDY_ARGS); }
-spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(false, SPEC_SAMPLE_ARGS); }
-spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) { return sample_entry(true, SPEC_SAMPLE_ARGS); }
+spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_greedy");
+    return greedy_entry(false, SPEC_GREEDY_ARGS);
+}
+spec_status spec_verify_tree_greedy_lazy(SPEC_GREEDY_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_greedy_lazy");
+    return greedy_entry(true, SPEC_GREEDY_ARGS);
+}
+spec_status spec_verify_tree_sample(SPEC_SAMPLE_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_sample");
+    return sample_entry(false, SPEC_SAMPLE_ARGS);
+}
+spec_status spec_verify_tree_sample_lazy(SPEC_SAMPLE_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_sample_lazy");
+    return sample_entry(true, SPEC_SAMPLE_ARGS);
+}
 
 spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth, const void* target_logits,
                                              spec_dtype tdt, int64_t t_row_stride, const int32_t* tokens,
@@ -4849,6 +4940,7 @@ spec_status spec_verify_tree_sample_filtered(int B, int N, int V, int max_depth,
                                              const int32_t* top_k, const float* top_p, int32_t* out_accept_index,
                                              int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
                                              void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_verify_tree_sample_filtered");
     if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
     return sample_entry(false, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature,
                         coins, final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc,
@@ -4865,6 +4957,7 @@ spec_status spec_verify_tree_sample_filtered_lazy(int B, int N, int V, int max_d
                                                   int32_t* out_accept_index, int32_t* out_tokens,
                                                   int32_t* out_num_accepted, float* diag, void* workspace,
                                                   size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_verify_tree_sample_filtered_lazy");
     if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
     return sample_entry(true, B, N, V, max_depth, target_logits, tdt, t_row_stride, tokens, parents, temperature,
                         coins, final_u, draft_probs, dp_row_stride, threshold_single, threshold_acc,
@@ -4884,8 +4977,14 @@ spec_status spec_verify_tree_sample_filtered_lazy(int B, int N, int V, int max_d
         final_u, draft_probs, dp_row_stride, out_accept_index, out_tokens, out_num_accepted, diag,  \
         workspace, workspace_bytes, stream
 
-spec_status spec_verify_tree_mss(SPEC_MSS_ARGS_DECL) { return mss_entry(false, SPEC_MSS_ARGS); }
-spec_status spec_verify_tree_mss_lazy(SPEC_MSS_ARGS_DECL) { return mss_entry(true, SPEC_MSS_ARGS); }
+spec_status spec_verify_tree_mss(SPEC_MSS_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_mss");
+    return mss_entry(false, SPEC_MSS_ARGS);
+}
+spec_status spec_verify_tree_mss_lazy(SPEC_MSS_ARGS_DECL) {
+    NvtxRange nvtx("spec_verify_tree_mss_lazy");
+    return mss_entry(true, SPEC_MSS_ARGS);
+}
 
 }  // extern "C"
 
@@ -4984,6 +5083,7 @@ spec_status spec_vp_chain_stats(int B, int gamma, int V_shard, int vocab_offset,
                                 const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
                                 const int32_t* draft_tokens, const float* temperature, void* rec_out,
                                 void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_vp_chain_stats");
     g_detail[0] = 0;
     if (!target_logits || !draft_tokens || !temperature || !rec_out)
         return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
@@ -5007,6 +5107,7 @@ spec_status spec_vp_chain_decide(int B, int gamma, int V, int V_shard, int world
                                  const int32_t* draft_tokens, const float* temperature, const float* coins,
                                  int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
                                  void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_vp_chain_decide");
     g_detail[0] = 0;
     if (world < 1 || world > 64) return fail(SPEC_ERR_INVALID_ARG, "world = %d outside [1, 64]", world);
     if (!rec_all || !draft_tokens || !temperature || !coins || !out_tokens || !out_num_accepted)
@@ -5032,6 +5133,7 @@ spec_status spec_vp_chain_residual(int B, int gamma, int V_shard, int world, int
                                    const void* draft, spec_dtype ddt, int draft_is_probs, int64_t d_row_stride,
                                    const void* rec_all, double* mass_out,
                                    void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_vp_chain_residual");
     g_detail[0] = 0;
     if (world < 1 || world > 64 || rank < 0 || rank >= world)
         return fail(SPEC_ERR_INVALID_ARG, "rank %d / world %d", rank, world);
@@ -5054,6 +5156,7 @@ spec_status spec_vp_chain_sample(int B, int gamma, int V_shard, int vocab_offset
                                  const float* final_u, const void* rec_all, const double* mass_all,
                                  int32_t* tok_out, float* diag,
                                  void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_vp_chain_sample");
     g_detail[0] = 0;
     if (world < 1 || world > 64 || rank < 0 || rank >= world)
         return fail(SPEC_ERR_INVALID_ARG, "rank %d / world %d", rank, world);
@@ -5075,6 +5178,7 @@ spec_status spec_vp_chain_sample(int B, int gamma, int V_shard, int vocab_offset
 
 spec_status spec_vp_chain_finish(int B, int gamma, int V_shard, const int32_t* tok, int32_t* out_tokens,
                                  void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_vp_chain_finish");
     g_detail[0] = 0;
     if (!tok || !out_tokens) return fail(SPEC_ERR_INVALID_ARG, "a required pointer is NULL");
     Params P{};
@@ -5138,6 +5242,7 @@ extern "C" spec_status spec_verify_chain_noalloc(int B, int gamma, int V,
                                                  const float* coins, const float* final_u,
                                                  int32_t* out_tokens, int32_t* out_num_accepted,
                                                  float* diag, void* stream) {
+    NvtxRange nvtx("spec_verify_chain_noalloc");
     g_detail[0] = 0;
     if (B < 0) return fail(SPEC_ERR_INVALID_ARG, "B = %d < 0", B);
     if (gamma < 1 || gamma > SPEC_MAX_GAMMA) return fail(SPEC_ERR_INVALID_ARG, "gamma = %d outside [1, %d]", gamma, SPEC_MAX_GAMMA);

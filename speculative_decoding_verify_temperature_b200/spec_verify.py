@@ -17,7 +17,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libspecverify.so")
+# SPEC_VERIFY_LIB selects another build of the library, e.g. the bounds-checked
+# libspecverify_debug.so next to this file.
+LIB_PATH = os.environ.get("SPEC_VERIFY_LIB") or os.path.join(_HERE, "libspecverify.so")
 
 SPEC_OK, SPEC_ERR_INVALID_ARG, SPEC_ERR_UNSUPPORTED, SPEC_ERR_CUDA = 0, 1, 2, 3
 SPEC_ERR_DEVICE_INPUT, SPEC_ERR_TIMEOUT, SPEC_ERR_WORKSPACE, SPEC_ERR_COPY_IN_FLIGHT = 4, 5, 6, 7
@@ -96,6 +98,8 @@ def lib():
         L.spec_debug_wait_budget.argtypes = [ctypes.c_longlong]
         L.spec_launch_count.restype = ctypes.c_ulonglong
         L.spec_launch_count.argtypes = []
+        L.spec_debug_bounds_hits.restype = i32
+        L.spec_debug_bounds_hits.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
         _lib = L
     return _lib
 
@@ -170,6 +174,17 @@ def spec_profile_events(start=None, stop=None) -> None:
 def spec_launch_count() -> int:
     """Kernels launched (or captured) by the library from this host thread so far."""
     return int(lib().spec_launch_count())
+
+
+def spec_debug_bounds_hits() -> int | None:
+    """Failed device-side bounds checks since the last call (synchronises the
+    device), or None when the loaded library was built without them."""
+    v = ctypes.c_ulonglong(0)
+    st = lib().spec_debug_bounds_hits(ctypes.byref(v))
+    if st == SPEC_ERR_UNSUPPORTED:
+        return None
+    _check(st, "spec_debug_bounds_hits")
+    return int(v.value)
 
 
 def spec_debug_wait_budget(tries: int = -1) -> None:

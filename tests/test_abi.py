@@ -36,6 +36,18 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, n), f"{n} declared in spec_verify.h but not exported"
 
 
+def test_bounds_checks_only_in_the_debug_build(L):
+    """The release library reports that it has no bounds checks; the debug
+    library exports every declared symbol too."""
+    from speculative_decoding_verify_temperature_b200 import build, spec_verify as sv
+    v = ctypes.c_ulonglong(7)
+    L.spec_debug_bounds_hits.restype = ctypes.c_int
+    assert L.spec_debug_bounds_hits(ctypes.byref(v)) == sv.SPEC_ERR_UNSUPPORTED and v.value == 0
+    D = ctypes.CDLL(build.OUT_DEBUG)
+    for n in declared_functions():
+        assert hasattr(D, n), f"{n} missing from the debug library"
+
+
 def test_status_strings(L):
     from speculative_decoding_verify_temperature_b200 import spec_verify as sv
     for s in range(8):

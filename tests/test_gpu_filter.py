@@ -112,14 +112,31 @@ def test_filtered_invalid_parameters(cuda_device):
                                       inp.final_u)
 
 
-def test_filtered_value_histogram_overflow_fallback(cuda_device):
-    """bf16 rows longer than 65535 where one value repeats more than 65535 times:
-    the value-histogram counter wraps, the kernel detects it and takes the radix
-    path; results still match the oracle.  Also a long row without repeats."""
+def test_filtered_value_repeated_beyond_16_bits(cuda_device):
+    """bf16 rows longer than 65535 where one value repeats more than 65535 times
+    (the window's counters are 32-bit); results match the oracle.  Also a long
+    row without repeats."""
     B, gamma, V = 3, 2, 70000
     inp = wl.chain_inputs(B, gamma, V, seed=77, device="cuda", zipf=True, stride=70000, dstride=70000)
     inp.target[0, :, :V - 40] = 0.0                     # value 0 repeated 69960 times per row
     inp.draft[0, :, :V - 40] = 0.0
     tk = torch.tensor([5, 0, 100], dtype=torch.int32, device="cuda")
     tp = torch.tensor([0.9, 0.8, 1.0], dtype=torch.float32, device="cuda")
+    _check(inp, tk, tp)
+
+
+def test_filtered_thresholds_far_below_the_maximum(cuda_device):
+    """Flat rows (logits spread over [-40, 40], T = 30, so bf16 values of both
+    signs and every magnitude carry mass) where the top-p threshold and a top_k
+    close to V lie far below the row's maximum: the windowed histogram has to
+    move its window down (and count the row again) before it finds them."""
+    B, gamma, V = 12, 2, 40000
+    inp = wl.chain_inputs(B, gamma, V, seed=78, device="cuda", temperatures=(30.0,))
+    g = torch.Generator(device="cuda").manual_seed(5)
+    flat = (torch.rand((B, gamma + 1, V), generator=g, device="cuda") * 80.0 - 40.0)
+    inp.target[:, :, :V] = flat.to(torch.bfloat16)
+    inp.draft[:, :, :V] = (flat[:, :gamma] + torch.randn((B, gamma, V), generator=g, device="cuda")).to(torch.bfloat16)
+    tk = torch.tensor([0, V - 3, 30000, 0, 0, 25000, 1, 0, V - 1, 0, 12000, 0], dtype=torch.int32, device="cuda")
+    tp = torch.tensor([0.99, 1.0, 0.9, 0.5, 0.999, 1.0, 0.9, 0.2, 0.95, 0.75, 1.0, 0.97], dtype=torch.float32,
+                      device="cuda")
     _check(inp, tk, tp)
