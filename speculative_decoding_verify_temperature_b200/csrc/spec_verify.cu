@@ -60,7 +60,8 @@ constexpr int MAXR = 256;             // max statistic rows per sequence (2*16+1
 constexpr int MAXCH = SPEC_MAX_V / (NT * VPT * 4);   // max chunks per row (f32 rows)
 constexpr double LOG2E = 1.4426950408889634073599246810019;
 
-enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2, MODE_MSS = 3, MODE_SAMPLE_FILT = 4 };
+enum { MODE_CHAIN = 0, MODE_GREEDY = 1, MODE_SAMPLE = 2, MODE_MSS = 3, MODE_SAMPLE_FILT = 4,
+       MODE_SAMPLE_FILT_OD = 5 };
 enum { DK_NONE = 0, DK_LOGITS = 1, DK_PROBS = 2 };
 
 template <int DT> struct Tr;
@@ -504,6 +505,469 @@ __device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
     uint4 v[VPT];
     load_vecs<DT, VPT>(row, V, (int64_t)c * chunk_elems<DT>(), v);
     return argmax_regs<DT>(v, c);
+}
+
+// ============================================================================= top-k / top-p filtering
+//
+// The filtered target distribution keeps the logits >= theta: theta_k = the
+// top_k-th largest logit (ties kept), then, within that set, theta_p = the
+// largest logit whose set {l >= theta_p} carries a top_p share of the set's
+// mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds are found over
+// order-preserving keys of the logits (-0 folded onto +0): for bf16 rows an
+// exact count histogram of a window of keys below the row's maximum
+// (wfilter_row), for f32
+// rows (and a bf16 row whose histogram counter would wrap) a radix descent of
+// 12 + 12 + 8 bit digits (filter_row).  Counts decide top-k; masses are fixed
+// point (2^-40 units, integer sums, so they do not depend on the order of the
+// additions) and decide top-p and Z'.
+
+constexpr int FILT_BT = 1024;
+constexpr double FIX_ONE = 1099511627776.0;      // 2^40
+
+template <int DT> __device__ __forceinline__ uint32_t order_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;                                   // -0 sorts with +0
+    const uint32_t k = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return DT == SPEC_BF16 ? (k >> 16) : k;
+}
+template <int DT> __device__ __forceinline__ float key_value(uint32_t k) {
+    if constexpr (DT == SPEC_BF16) {
+        const uint32_t b = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
+        return __uint_as_float(b << 16);
+    } else {
+        return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+    }
+}
+
+// Digits of the order keys, most significant first: 12 + 4 bits for bf16,
+// 12 + 12 + 8 for f32.  The wide first digit (sign, exponent and the top
+// mantissa bits) spreads a row's values over many buckets, so the shared
+// histogram updates rarely collide.
+template <int DT> struct FiltDigits;
+template <> struct FiltDigits<SPEC_BF16> {
+    static constexpr int NL = 2;
+    __host__ __device__ static constexpr int width(int l) { return l == 0 ? 12 : 4; }
+    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 4 : 0; }
+};
+template <> struct FiltDigits<SPEC_F32> {
+    static constexpr int NL = 3;
+    __host__ __device__ static constexpr int width(int l) { return l == 2 ? 8 : 12; }
+    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 20 : (l == 1 ? 8 : 0); }
+};
+// Shared bytes of the per-level histograms (counts u32 + masses u64 per bucket).
+template <int DT> __host__ __device__ constexpr size_t filt_hist_bytes() {
+    size_t n = 0;
+    for (int l = 0; l < FiltDigits<DT>::NL; ++l) n += ((size_t)1 << FiltDigits<DT>::width(l)) * 12;
+    return n;
+}
+
+struct FiltShared {
+    unsigned long long red[FILT_BT / 32];
+    unsigned redc[FILT_BT / 32];
+    unsigned long long at, above, tm;
+    unsigned tc;
+    int sel;
+};
+
+// Level l's histograms inside the dynamic area.
+template <int DT> struct FiltHist {
+    unsigned char* base;
+    __device__ unsigned long long* mass(int l) const {
+        size_t off = 0;
+        for (int k = 0; k < l; ++k) off += ((size_t)1 << FiltDigits<DT>::width(k)) * 12;
+        return reinterpret_cast<unsigned long long*>(base + off);
+    }
+    __device__ unsigned* cnt(int l) const {
+        return reinterpret_cast<unsigned*>(mass(l) + ((size_t)1 << FiltDigits<DT>::width(l)));
+    }
+};
+
+// One pass over a row: histograms of digit `level` (counts and fixed-point
+// masses of 2^(x s - m)) of the keys whose higher digits equal `prefix` (all
+// keys at level 0).  Integer atomics: the sums do not depend on their order.
+template <int DT>
+__device__ void filt_pass(const char* row, int V, float s, float m, int level, uint32_t prefix, const FiltHist<DT>& h) {
+    using D = FiltDigits<DT>;
+    constexpr int EPV = Tr<DT>::EPV;
+    const int nb = 1 << D::width(level), sh = D::shift(level);
+    const int psh = sh + D::width(level);
+    unsigned* cnt = h.cnt(level);
+    unsigned long long* mass = h.mass(level);
+    for (int d = threadIdx.x; d < nb; d += FILT_BT) { cnt[d] = 0u; mass[d] = 0ull; }
+    __syncthreads();
+    const int nv = (V + EPV - 1) / EPV;
+    for (int vi = threadIdx.x; vi < nv; vi += FILT_BT) {
+        const uint4 v = ld_vec<DT>(row, (int64_t)vi * EPV, V);
+#pragma unroll
+        for (int i = 0; i < EPV; ++i) {
+            if (vi * EPV + i >= V) break;
+            const float x = vec_elem<DT>(v, i);
+            const uint32_t key = order_key<DT>(x);
+            if (level > 0 && (key >> psh) != prefix) continue;
+            const uint32_t d = (key >> sh) & (uint32_t)(nb - 1);
+            atomicAdd(&cnt[d], 1u);
+            atomicAdd(&mass[d], (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE));
+        }
+    }
+    __syncthreads();
+}
+
+// Scan buckets [dlo, nb) from the top for the first bucket d whose running
+// total base + (buckets above d) + w[d] reaches target; every thread owns a
+// run of buckets, a block-wide u64 scan gives each run its start.  Returns d,
+// or -1 when the range never reaches the target.  fs.above = base + the
+// buckets of the range strictly above d (the whole range when -1), fs.at =
+// fs.above + w[d].  All threads call it.
+template <class T>
+__device__ int filt_scan(const T* w, int nb, int dlo, unsigned long long base, double target, FiltShared& fs) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = nb - dlo;
+    const int per = (n + FILT_BT - 1) / FILT_BT;
+    const int hi = nb - tid * per, lo = max(dlo, hi - per);     // buckets [lo, hi), this thread's run
+    unsigned long long own = 0ull;
+    for (int d = hi - 1; d >= lo; --d) own += (unsigned long long)w[d];
+    unsigned long long inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long v = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += v;
+    }
+    if (lane == 31) fs.red[warp] = inc;
+    if (tid == 0) fs.sel = -1;
+    __syncthreads();
+    unsigned long long excl = base;
+    for (int k = 0; k < warp; ++k) excl += fs.red[k];
+    excl += inc - own;
+    if (hi > lo && (double)excl < target && (double)(excl + own) >= target) {
+        unsigned long long cum = excl;
+        for (int d = hi - 1; d >= lo; --d) {
+            if ((double)(cum + (unsigned long long)w[d]) >= target) {
+                fs.sel = d;
+                fs.above = cum;
+                fs.at = cum + (unsigned long long)w[d];
+                break;
+            }
+            cum += (unsigned long long)w[d];
+        }
+    }
+    __syncthreads();
+    const int d = fs.sel;
+    if (d < 0 && tid == 0) {
+        unsigned long long t = base;
+        for (int k = 0; k < FILT_BT / 32; ++k) t += fs.red[k];
+        fs.above = t;
+        fs.at = t;
+    }
+    __syncthreads();
+    return d;
+}
+
+// Threshold and kept mass of one row (one CTA).
+//  top-k: walk the digits of the top_k-th largest key (filt_scan over the
+//    counts, one pass per digit); every pass keeps the masses, so the mass of
+//    the kept set {key >= path} is the masses strictly above the path at
+//    each level plus the path's key.
+//  top-p: within the kept set, scan from the top -- the buckets strictly
+//    above the path at each level, then the path's key -- for the bucket
+//    where the mass reaches top_p * (kept mass); a whole key ends the search,
+//    another bucket is refined digit by digit with more passes (every key in
+//    it lies above the top-k key).
+//  top-p alone: one pass of the first digit over every key; the crossing
+//    bucket is refined the same way.
+template <int DT>
+__device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
+                              const FiltHist<DT>& h) {
+    using D = FiltDigits<DT>;
+    constexpr int NL = D::NL;
+    FiltRec r{-INFINITY, 0, 0.0};
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    if (!use_k && !use_p) return r;
+    int path[NL];
+    uint32_t prefix = 0;
+    unsigned long long cabove = 0ull, mabove = 0ull;           // counts / masses strictly above the path
+    const int nl = use_k ? NL : 1;
+    for (int level = 0; level < nl; ++level) {
+        filt_pass<DT>(row, V, s, m, level, prefix, h);
+        const int nb = 1 << D::width(level);
+        if (use_k) {
+            path[level] = filt_scan(h.cnt(level), nb, 0, cabove, (double)K, fs);
+            cabove = fs.above;
+        } else {
+            path[level] = 0;                                   // top-p alone: every key is kept
+        }
+        filt_scan(h.mass(level), nb, path[level] + 1, 0ull, INFINITY, fs);   // masses above the path digit
+        mabove += fs.above;
+        prefix = (prefix << D::width(level)) | (uint32_t)path[level];
+    }
+    const unsigned long long mk = mabove + h.mass(nl - 1)[path[nl - 1]];
+    uint32_t key = prefix;
+    unsigned long long z = mk;
+    if (use_p) {
+        const double target = (double)Pp * (double)mk;
+        unsigned long long base = 0ull;
+        int cl = -1, cd = 0;
+        for (int l = 0; l < nl && cl < 0; ++l) {                // buckets strictly above the path digit
+            const int d = filt_scan(h.mass(l), 1 << D::width(l), path[l] + 1, base, target, fs);
+            if (d >= 0) { cl = l; cd = d; z = fs.at; }
+            base = fs.above;
+        }
+        if (cl < 0) {                                          // the path's own bucket
+            cl = nl - 1;
+            cd = path[nl - 1];
+            z = base + h.mass(cl)[cd];
+        }
+        uint32_t pre = 0;
+        for (int l = 0; l < cl; ++l) pre = (pre << D::width(l)) | (uint32_t)path[l];
+        pre = (pre << D::width(cl)) | (uint32_t)cd;
+        if (!(use_k && cl == NL - 1)) {                        // not a whole key: refine
+            for (int level = cl + 1; level < NL; ++level) {
+                filt_pass<DT>(row, V, s, m, level, pre, h);
+                int d = filt_scan(h.mass(level), 1 << D::width(level), 0, base, target, fs);
+                if (d < 0) d = 0;                              // rounding only
+                base = fs.above;
+                z = fs.at;
+                pre = (pre << D::width(level)) | (uint32_t)d;
+            }
+        }
+        key = pre;
+    }
+    r.theta = key_value<DT>(key);
+    r.on = 1;
+    r.Z = (double)z / FIX_ONE;
+    return r;
+}
+
+// Order keys of the two bf16 values packed in x (low half = lower index), as
+// order_key does for one value: -0 folded onto +0, negative values
+// complemented, the sign bit of the others set.
+__device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
+    x &= ~__vcmpeq2(x, 0x80008000u);
+    return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
+}
+
+// bf16 rows, windowed: an exact count histogram of WF_KEYS consecutive order
+// keys (u32 counters, 32 KB) from the row's largest key down, plus exact
+// integer totals -- counts and fixed-point masses, count * fixed(2^(v s - m))
+// per value -- of the elements above and below the window.  Every key's
+// mass is count * fixed(2^(v s - m)), so the running counts and masses from
+// the top, and with them the top-k key, the kept mass and the top-p key, are
+// the integers of the full value histogram.  A threshold that falls outside
+// the window moves it (up to the row's true maximum, or down below it) and
+// the row is counted again; the first window holds both thresholds unless the
+// kept set reaches far below the maximum.
+constexpr int WF_KEYS = 8192;
+constexpr size_t WF_BYTES = (size_t)WF_KEYS * 4;
+
+struct WinShared {
+    unsigned long long red[32];
+    unsigned redc[32];
+    unsigned long long am, bm, tm;        // masses above / below the window, window total
+    unsigned ac, bc, tc, amax;            // counts above / below, window total, largest key above
+    int sel;
+    unsigned long long at;
+};
+
+__device__ __forceinline__ unsigned long long fix_mass(float x, float s, float m) {
+    return (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE);
+}
+
+// Block-wide exclusive scan, in thread order, of a u32 and a u64 (BT threads,
+// BT / 32 <= 32 warps); the totals go to *ta / *tb.  All threads call it.
+template <int BT>
+__device__ void wf_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
+                         unsigned long long* tb, WinShared& ws) {
+    constexpr int NW = BT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned ia = a;
+    unsigned long long ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned va = __shfl_up_sync(FULL, ia, o);
+        const unsigned long long vb = __shfl_up_sync(FULL, ib, o);
+        if (lane >= o) { ia += va; ib += vb; }
+    }
+    if (lane == 31) { ws.redc[warp] = ia; ws.red[warp] = ib; }
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned xa = lane < NW ? ws.redc[lane] : 0u;
+        const unsigned long long xb = lane < NW ? ws.red[lane] : 0ull;
+        unsigned sa = xa;
+        unsigned long long sb = xb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned va = __shfl_up_sync(FULL, sa, o);
+            const unsigned long long vb = __shfl_up_sync(FULL, sb, o);
+            if (lane >= o) { sa += va; sb += vb; }
+        }
+        if (lane < NW) { ws.redc[lane] = sa - xa; ws.red[lane] = sb - xb; }
+        if (lane == 31) { ws.tc = sa; ws.tm = sb; }
+    }
+    __syncthreads();
+    *ea = ws.redc[warp] + ia - a;
+    *eb = ws.red[warp] + ib - b;
+    *ta = ws.tc;
+    *tb = ws.tm;
+    __syncthreads();
+}
+
+// One pass over a bf16 row: the window [khi - WF_KEYS + 1, khi] counted per
+// key in win[khi - key]; the rest summed into ws.ac/am/amax (above) and
+// ws.bc/bm (below).  All threads call it.
+template <int BT>
+__device__ void wf_pass(const char* row, int V, float s, float m, uint32_t khi, uint32_t* win, WinShared& ws) {
+    const int tid = threadIdx.x;
+    const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
+    for (int i = tid; i < WF_KEYS / 4; i += BT) reinterpret_cast<uint4*>(win)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (tid == 0) { ws.ac = 0u; ws.bc = 0u; ws.am = 0ull; ws.bm = 0ull; ws.amax = 0u; }
+    __syncthreads();
+    unsigned ac = 0u, bc = 0u, amax = 0u;
+    unsigned long long am = 0ull, bm = 0ull;
+    const int nv = (V + 7) / 8;
+    auto one = [&](uint32_t k) {
+        if (k > khi) {
+            ++ac;
+            amax = max(amax, k);
+            am += fix_mass(key_value<SPEC_BF16>(k), s, m);
+        } else if (k >= klo) {
+            atomicAdd(&win[khi - k], 1u);
+        } else {
+            ++bc;
+            bm += fix_mass(key_value<SPEC_BF16>(k), s, m);
+        }
+    };
+    for (int v0 = tid; v0 < nv; v0 += 4 * BT) {
+        uint4 v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * BT;
+            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * BT;
+            if (vi >= nv) break;
+            const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            const int lim = V - vi * 8;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t k2 = vh_keys2(xs[c]);
+                if (2 * c < lim) one(k2 & 0xFFFFu);
+                if (2 * c + 1 < lim) one(k2 >> 16);
+            }
+        }
+    }
+    // fold the per-thread totals (integers: any order gives the same sums)
+    ac = __reduce_add_sync(FULL, ac);
+    bc = __reduce_add_sync(FULL, bc);
+    amax = __reduce_max_sync(FULL, amax);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        am += __shfl_xor_sync(FULL, am, o);
+        bm += __shfl_xor_sync(FULL, bm, o);
+    }
+    if ((tid & 31) == 0) {
+        atomicAdd(&ws.ac, ac);
+        atomicAdd(&ws.bc, bc);
+        atomicMax(&ws.amax, amax);
+        atomicAdd(&ws.am, am);
+        atomicAdd(&ws.bm, bm);
+    }
+    __syncthreads();
+}
+
+// Threshold and kept mass of one bf16 row (the record filter_row gives).  The
+// first window starts just above the key of the row's maximum estimated from
+// the statistics (m / s).  All threads call it.
+template <int BT>
+__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, uint32_t* win,
+                               WinShared& ws) {
+    constexpr int RUN = WF_KEYS / BT;                 // window keys per thread
+    static_assert(RUN * BT == WF_KEYS, "window split");
+    const int tid = threadIdx.x;
+    FiltRec r{-INFINITY, 0, 0.0};
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    if (!use_k && !use_p) return r;
+    // the row's largest value is about m / s (m = its value times s, rounded)
+    uint32_t khi = min(0xFFFFu, order_key<SPEC_BF16>(__bfloat162float(__float2bfloat16_rn(m / s))) + 4u);
+    bool rk = !use_k;                                 // top-k resolved
+    uint32_t tk = 0u, tp = 0u;
+    unsigned long long zk = 0ull, z = 0ull;
+    for (int it = 0; it < 2 * (65536 / WF_KEYS) + 2; ++it) {
+        wf_pass<BT>(row, V, s, m, khi, win, ws);
+        const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
+        const unsigned ac = ws.ac, amax = ws.amax;
+        const unsigned long long am = ws.am, bm = ws.bm;
+        // this thread's run of window indices [j0, j0 + RUN): keys khi - j
+        const int j0 = tid * RUN;
+        unsigned rc = 0u;
+        unsigned long long rm = 0ull;
+#pragma unroll 4
+        for (int j = j0; j < j0 + RUN; ++j) {
+            const unsigned c = win[j];
+            if (c) {
+                rc += c;
+                rm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+            }
+        }
+        unsigned c0, ctot;
+        unsigned long long m0, mtot;
+        wf_scan2<BT>(rc, rm, &c0, &m0, &ctot, &mtot, ws);
+        c0 += ac;
+        m0 += am;
+        if (!use_k) zk = am + mtot + bm;
+        if (!rk) {
+            if ((unsigned)K <= ac) { khi = amax; continue; }                 // above the window
+            if ((unsigned)K > ac + ctot) {                                   // below the window
+                if (klo == 0u) break;                                        // (cannot happen: K < V)
+                khi = klo - 1u;
+                continue;
+            }
+            if (tid == 0) ws.sel = -1;
+            __syncthreads();
+            if (c0 < (unsigned)K && c0 + rc >= (unsigned)K) {
+                unsigned c = c0;
+                unsigned long long mm = m0;
+                for (int j = j0; j < j0 + RUN; ++j) {
+                    const unsigned cj = win[j];
+                    c += cj;
+                    if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+                    if (c >= (unsigned)K) { ws.sel = j; ws.at = mm; break; }
+                }
+            }
+            __syncthreads();
+            tk = khi - (uint32_t)ws.sel;
+            zk = ws.at;
+            rk = true;
+            __syncthreads();
+        }
+        if (!use_p) { tp = tk; z = zk; break; }
+        const double target = (double)Pp * (double)zk;
+        if ((double)am >= target) { khi = amax; continue; }                 // above the window
+        if ((double)(am + mtot) < target) {                                 // below (top-p alone)
+            if (klo == 0u) break;                                            // (cannot happen: target <= total)
+            khi = klo - 1u;
+            continue;
+        }
+        if (tid == 0) ws.sel = -1;
+        __syncthreads();
+        if ((double)m0 < target && (double)(m0 + rm) >= target) {
+            unsigned long long mm = m0;
+            for (int j = j0; j < j0 + RUN; ++j) {
+                const unsigned cj = win[j];
+                if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+                if (cj && (double)mm >= target) { ws.sel = j; ws.at = mm; break; }
+            }
+        }
+        __syncthreads();
+        tp = khi - (uint32_t)ws.sel;
+        z = ws.at;
+        __syncthreads();
+        break;
+    }
+    r.theta = key_value<SPEC_BF16>(tp);
+    r.on = 1;
+    r.Z = (double)z / FIX_ONE;
+    return r;
 }
 
 // ----------------------------------------------------------------------------- finaliser pieces
@@ -1486,8 +1950,14 @@ __device__ int tree_filt_draw(const Params& P, int b, int cur, const int* rej, i
 
 // Target-only tree sampling, one CTA per sequence (FILT: on the top-k /
 // top-p filtered rows, from the records of k_filter).
-template <int TDT, int BT, bool FILT = false>
-__device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk) {
+// Target-only tree sampling for sequence b, one CTA.  FILT: under top-k /
+// top-p filtering, with each row's threshold and kept mass read from the
+// filter records (k_filter) -- or, OD (on demand, bf16 rows, no diagnostics),
+// computed here for the rows of the nodes the walk visits, one window
+// histogram each (win: WF_BYTES of shared memory).
+template <int TDT, int BT, bool FILT = false, bool OD = false>
+__device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk, uint32_t* win = nullptr,
+                                WinShared* ws = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
     combine_softmax_rows<BT>(P, blk, N, sh);
@@ -1496,7 +1966,9 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         sh.tok[n] = P.tokens[(size_t)b * N + n];
     }
     __syncthreads();
-    if constexpr (FILT) {
+    const int K = (FILT && OD && P.top_k) ? P.top_k[b] : 0;
+    const float Pp = (FILT && OD && P.top_p) ? P.top_p[b] : 1.f;
+    if constexpr (FILT && !OD) {
         // each row's threshold and kept mass (same 2^(x s - m) units as z)
         for (int n = tid; n < N; n += BT) {
             const FiltRec f = P.filt[(size_t)b * P.R + n];
@@ -1511,6 +1983,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     if (tid == 0) {
         ok &= temperature_ok(T);
         for (int r = 0; r < N; ++r) ok &= !sh.bad[r];
+        if (FILT && OD) ok &= (K >= 0 && Pp > 0.f && Pp <= 1.f);        // invalid top_k / top_p
         sh.ivals[0] = ok;
     }
     __syncthreads();
@@ -1525,6 +1998,67 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         return;
     }
     const float s = scale_of(T);
+    if constexpr (FILT && OD) {
+        // the walk, filtering the row of each node it visits
+        const double ths = (double)P.th_single, tha = (double)P.th_acc;
+        int cur = 0, k = 0, nrej = 0;
+        float thc;
+        double zc;
+        if (tid == 0) ai[0] = 0;
+        for (;;) {
+            const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
+            const FiltRec f = wfilter_row<BT>(row, V, s, sh.m[cur], K, Pp, win, *ws);
+            thc = f.theta;
+            zc = f.on > 0 ? f.Z : sh.z[cur];
+            for (int n = cur + 1 + tid; n < N; n += BT)
+                if (sh.par[n] == cur) {
+                    const float l = ld_elem<TDT>(row, sh.tok[n], V);
+                    sh.pch[n] = l >= thc ? prob_d(l, s, sh.m[cur], zc) : 0.0;
+                }
+            __syncthreads();
+            if (warp == 0) {
+                const double coin = (double)P.coins[(size_t)b * N + cur];
+                double acc = 0.0;
+                int next = -1;
+                nrej = 0;
+                for (int base = cur + 1; base < N && next < 0; base += 32) {
+                    const int c = base + lane;
+                    unsigned m = __ballot_sync(FULL, c < N && sh.par[c] == cur);
+                    if (lane == 0) {
+                        while (m && next < 0) {
+                            const int cc = base + __ffs(m) - 1;
+                            m &= m - 1;
+                            const double pc = sh.pch[cc];
+                            acc += pc;
+                            if (coin <= acc / tha || pc >= ths) next = cc;
+                            else sh.rej[nrej++] = sh.tok[cc];
+                        }
+                    }
+                    next = __shfl_sync(FULL, next, 0);
+                }
+                if (lane == 0) { sh.ivals[1] = next; sh.ivals[3] = nrej; }
+            }
+            __syncthreads();
+            const int next = sh.ivals[1];
+            nrej = sh.ivals[3];
+            __syncthreads();
+            if (next < 0) break;
+            if (tid == 0) { ot[k] = sh.tok[next]; ai[k + 1] = next; }
+            ++k;
+            cur = next;
+        }
+        double S;
+        const int y = P.draft_probs ? tree_filt_draw<TDT, BT, true>(P, b, cur, sh.rej, nrej, s, sh.m[cur], zc, thc,
+                                                                    sh, &S)
+                                    : tree_filt_draw<TDT, BT, false>(P, b, cur, sh.rej, nrej, s, sh.m[cur], zc, thc,
+                                                                     sh, &S);
+        if (tid == 0) {
+            ot[k] = y;
+            for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
+            P.out_num_accepted[b] = k;
+        }
+        return;
+    }
     // p_parent(n)(tokens[n]) for every non-root node (0 below the row's threshold)
     for (int n = tid; n < N; n += BT) {
         double pc = 0.0;
@@ -2634,470 +3168,12 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
     else if constexpr (MODE == MODE_SAMPLE) finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
     else if constexpr (MODE == MODE_SAMPLE_FILT) finalize_sample<TDT, SEQ_BT, true>(P, blockIdx.x, sh, blk);
+    else if constexpr (MODE == MODE_SAMPLE_FILT_OD) {
+        __shared__ WinShared ws;
+        finalize_sample<TDT, SEQ_BT, true, true>(P, blockIdx.x, sh, blk,
+                                                 reinterpret_cast<uint32_t*>(dyn + P.stage_off), &ws);
+    }
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
-}
-
-// ============================================================================= top-k / top-p filtering
-//
-// The filtered target distribution keeps the logits >= theta: theta_k = the
-// top_k-th largest logit (ties kept), then, within that set, theta_p = the
-// largest logit whose set {l >= theta_p} carries a top_p share of the set's
-// mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds are found over
-// order-preserving keys of the logits (-0 folded onto +0): for bf16 rows an
-// exact count histogram of a window of keys below the row's maximum
-// (wfilter_row), for f32
-// rows (and a bf16 row whose histogram counter would wrap) a radix descent of
-// 12 + 12 + 8 bit digits (filter_row).  Counts decide top-k; masses are fixed
-// point (2^-40 units, integer sums, so they do not depend on the order of the
-// additions) and decide top-p and Z'.
-
-constexpr int FILT_BT = 1024;
-constexpr double FIX_ONE = 1099511627776.0;      // 2^40
-
-template <int DT> __device__ __forceinline__ uint32_t order_key(float v) {
-    uint32_t b = __float_as_uint(v);
-    if (b == 0x80000000u) b = 0u;                                   // -0 sorts with +0
-    const uint32_t k = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return DT == SPEC_BF16 ? (k >> 16) : k;
-}
-template <int DT> __device__ __forceinline__ float key_value(uint32_t k) {
-    if constexpr (DT == SPEC_BF16) {
-        const uint32_t b = (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu);
-        return __uint_as_float(b << 16);
-    } else {
-        return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-    }
-}
-
-// Digits of the order keys, most significant first: 12 + 4 bits for bf16,
-// 12 + 12 + 8 for f32.  The wide first digit (sign, exponent and the top
-// mantissa bits) spreads a row's values over many buckets, so the shared
-// histogram updates rarely collide.
-template <int DT> struct FiltDigits;
-template <> struct FiltDigits<SPEC_BF16> {
-    static constexpr int NL = 2;
-    __host__ __device__ static constexpr int width(int l) { return l == 0 ? 12 : 4; }
-    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 4 : 0; }
-};
-template <> struct FiltDigits<SPEC_F32> {
-    static constexpr int NL = 3;
-    __host__ __device__ static constexpr int width(int l) { return l == 2 ? 8 : 12; }
-    __host__ __device__ static constexpr int shift(int l) { return l == 0 ? 20 : (l == 1 ? 8 : 0); }
-};
-// Shared bytes of the per-level histograms (counts u32 + masses u64 per bucket).
-template <int DT> __host__ __device__ constexpr size_t filt_hist_bytes() {
-    size_t n = 0;
-    for (int l = 0; l < FiltDigits<DT>::NL; ++l) n += ((size_t)1 << FiltDigits<DT>::width(l)) * 12;
-    return n;
-}
-
-struct FiltShared {
-    unsigned long long red[FILT_BT / 32];
-    unsigned redc[FILT_BT / 32];
-    unsigned long long at, above, tm;
-    unsigned tc;
-    int sel;
-};
-
-// Level l's histograms inside the dynamic area.
-template <int DT> struct FiltHist {
-    unsigned char* base;
-    __device__ unsigned long long* mass(int l) const {
-        size_t off = 0;
-        for (int k = 0; k < l; ++k) off += ((size_t)1 << FiltDigits<DT>::width(k)) * 12;
-        return reinterpret_cast<unsigned long long*>(base + off);
-    }
-    __device__ unsigned* cnt(int l) const {
-        return reinterpret_cast<unsigned*>(mass(l) + ((size_t)1 << FiltDigits<DT>::width(l)));
-    }
-};
-
-// One pass over a row: histograms of digit `level` (counts and fixed-point
-// masses of 2^(x s - m)) of the keys whose higher digits equal `prefix` (all
-// keys at level 0).  Integer atomics: the sums do not depend on their order.
-template <int DT>
-__device__ void filt_pass(const char* row, int V, float s, float m, int level, uint32_t prefix, const FiltHist<DT>& h) {
-    using D = FiltDigits<DT>;
-    constexpr int EPV = Tr<DT>::EPV;
-    const int nb = 1 << D::width(level), sh = D::shift(level);
-    const int psh = sh + D::width(level);
-    unsigned* cnt = h.cnt(level);
-    unsigned long long* mass = h.mass(level);
-    for (int d = threadIdx.x; d < nb; d += FILT_BT) { cnt[d] = 0u; mass[d] = 0ull; }
-    __syncthreads();
-    const int nv = (V + EPV - 1) / EPV;
-    for (int vi = threadIdx.x; vi < nv; vi += FILT_BT) {
-        const uint4 v = ld_vec<DT>(row, (int64_t)vi * EPV, V);
-#pragma unroll
-        for (int i = 0; i < EPV; ++i) {
-            if (vi * EPV + i >= V) break;
-            const float x = vec_elem<DT>(v, i);
-            const uint32_t key = order_key<DT>(x);
-            if (level > 0 && (key >> psh) != prefix) continue;
-            const uint32_t d = (key >> sh) & (uint32_t)(nb - 1);
-            atomicAdd(&cnt[d], 1u);
-            atomicAdd(&mass[d], (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE));
-        }
-    }
-    __syncthreads();
-}
-
-// Scan buckets [dlo, nb) from the top for the first bucket d whose running
-// total base + (buckets above d) + w[d] reaches target; every thread owns a
-// run of buckets, a block-wide u64 scan gives each run its start.  Returns d,
-// or -1 when the range never reaches the target.  fs.above = base + the
-// buckets of the range strictly above d (the whole range when -1), fs.at =
-// fs.above + w[d].  All threads call it.
-template <class T>
-__device__ int filt_scan(const T* w, int nb, int dlo, unsigned long long base, double target, FiltShared& fs) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = nb - dlo;
-    const int per = (n + FILT_BT - 1) / FILT_BT;
-    const int hi = nb - tid * per, lo = max(dlo, hi - per);     // buckets [lo, hi), this thread's run
-    unsigned long long own = 0ull;
-    for (int d = hi - 1; d >= lo; --d) own += (unsigned long long)w[d];
-    unsigned long long inc = own;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long v = __shfl_up_sync(FULL, inc, o);
-        if (lane >= o) inc += v;
-    }
-    if (lane == 31) fs.red[warp] = inc;
-    if (tid == 0) fs.sel = -1;
-    __syncthreads();
-    unsigned long long excl = base;
-    for (int k = 0; k < warp; ++k) excl += fs.red[k];
-    excl += inc - own;
-    if (hi > lo && (double)excl < target && (double)(excl + own) >= target) {
-        unsigned long long cum = excl;
-        for (int d = hi - 1; d >= lo; --d) {
-            if ((double)(cum + (unsigned long long)w[d]) >= target) {
-                fs.sel = d;
-                fs.above = cum;
-                fs.at = cum + (unsigned long long)w[d];
-                break;
-            }
-            cum += (unsigned long long)w[d];
-        }
-    }
-    __syncthreads();
-    const int d = fs.sel;
-    if (d < 0 && tid == 0) {
-        unsigned long long t = base;
-        for (int k = 0; k < FILT_BT / 32; ++k) t += fs.red[k];
-        fs.above = t;
-        fs.at = t;
-    }
-    __syncthreads();
-    return d;
-}
-
-// Threshold and kept mass of one row (one CTA).
-//  top-k: walk the digits of the top_k-th largest key (filt_scan over the
-//    counts, one pass per digit); every pass keeps the masses, so the mass of
-//    the kept set {key >= path} is the masses strictly above the path at
-//    each level plus the path's key.
-//  top-p: within the kept set, scan from the top -- the buckets strictly
-//    above the path at each level, then the path's key -- for the bucket
-//    where the mass reaches top_p * (kept mass); a whole key ends the search,
-//    another bucket is refined digit by digit with more passes (every key in
-//    it lies above the top-k key).
-//  top-p alone: one pass of the first digit over every key; the crossing
-//    bucket is refined the same way.
-template <int DT>
-__device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
-                              const FiltHist<DT>& h) {
-    using D = FiltDigits<DT>;
-    constexpr int NL = D::NL;
-    FiltRec r{-INFINITY, 0, 0.0};
-    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
-    if (!use_k && !use_p) return r;
-    int path[NL];
-    uint32_t prefix = 0;
-    unsigned long long cabove = 0ull, mabove = 0ull;           // counts / masses strictly above the path
-    const int nl = use_k ? NL : 1;
-    for (int level = 0; level < nl; ++level) {
-        filt_pass<DT>(row, V, s, m, level, prefix, h);
-        const int nb = 1 << D::width(level);
-        if (use_k) {
-            path[level] = filt_scan(h.cnt(level), nb, 0, cabove, (double)K, fs);
-            cabove = fs.above;
-        } else {
-            path[level] = 0;                                   // top-p alone: every key is kept
-        }
-        filt_scan(h.mass(level), nb, path[level] + 1, 0ull, INFINITY, fs);   // masses above the path digit
-        mabove += fs.above;
-        prefix = (prefix << D::width(level)) | (uint32_t)path[level];
-    }
-    const unsigned long long mk = mabove + h.mass(nl - 1)[path[nl - 1]];
-    uint32_t key = prefix;
-    unsigned long long z = mk;
-    if (use_p) {
-        const double target = (double)Pp * (double)mk;
-        unsigned long long base = 0ull;
-        int cl = -1, cd = 0;
-        for (int l = 0; l < nl && cl < 0; ++l) {                // buckets strictly above the path digit
-            const int d = filt_scan(h.mass(l), 1 << D::width(l), path[l] + 1, base, target, fs);
-            if (d >= 0) { cl = l; cd = d; z = fs.at; }
-            base = fs.above;
-        }
-        if (cl < 0) {                                          // the path's own bucket
-            cl = nl - 1;
-            cd = path[nl - 1];
-            z = base + h.mass(cl)[cd];
-        }
-        uint32_t pre = 0;
-        for (int l = 0; l < cl; ++l) pre = (pre << D::width(l)) | (uint32_t)path[l];
-        pre = (pre << D::width(cl)) | (uint32_t)cd;
-        if (!(use_k && cl == NL - 1)) {                        // not a whole key: refine
-            for (int level = cl + 1; level < NL; ++level) {
-                filt_pass<DT>(row, V, s, m, level, pre, h);
-                int d = filt_scan(h.mass(level), 1 << D::width(level), 0, base, target, fs);
-                if (d < 0) d = 0;                              // rounding only
-                base = fs.above;
-                z = fs.at;
-                pre = (pre << D::width(level)) | (uint32_t)d;
-            }
-        }
-        key = pre;
-    }
-    r.theta = key_value<DT>(key);
-    r.on = 1;
-    r.Z = (double)z / FIX_ONE;
-    return r;
-}
-
-// Order keys of the two bf16 values packed in x (low half = lower index), as
-// order_key does for one value: -0 folded onto +0, negative values
-// complemented, the sign bit of the others set.
-__device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
-    x &= ~__vcmpeq2(x, 0x80008000u);
-    return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
-}
-
-// bf16 rows, windowed: an exact count histogram of WF_KEYS consecutive order
-// keys (u32 counters, 32 KB) from the row's largest key down, plus exact
-// integer totals -- counts and fixed-point masses, count * fixed(2^(v s - m))
-// per value -- of the elements above and below the window.  Every key's
-// mass is count * fixed(2^(v s - m)), so the running counts and masses from
-// the top, and with them the top-k key, the kept mass and the top-p key, are
-// the integers of the full value histogram.  A threshold that falls outside
-// the window moves it (up to the row's true maximum, or down below it) and
-// the row is counted again; the first window holds both thresholds unless the
-// kept set reaches far below the maximum.
-constexpr int WF_KEYS = 8192;
-constexpr size_t WF_BYTES = (size_t)WF_KEYS * 4;
-
-struct WinShared {
-    unsigned long long red[32];
-    unsigned redc[32];
-    unsigned long long am, bm, tm;        // masses above / below the window, window total
-    unsigned ac, bc, tc, amax;            // counts above / below, window total, largest key above
-    int sel;
-    unsigned long long at;
-};
-
-__device__ __forceinline__ unsigned long long fix_mass(float x, float s, float m) {
-    return (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE);
-}
-
-// Block-wide exclusive scan, in thread order, of a u32 and a u64 (BT threads,
-// BT / 32 <= 32 warps); the totals go to *ta / *tb.  All threads call it.
-template <int BT>
-__device__ void wf_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
-                         unsigned long long* tb, WinShared& ws) {
-    constexpr int NW = BT / 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned ia = a;
-    unsigned long long ib = b;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned va = __shfl_up_sync(FULL, ia, o);
-        const unsigned long long vb = __shfl_up_sync(FULL, ib, o);
-        if (lane >= o) { ia += va; ib += vb; }
-    }
-    if (lane == 31) { ws.redc[warp] = ia; ws.red[warp] = ib; }
-    __syncthreads();
-    if (warp == 0) {
-        const unsigned xa = lane < NW ? ws.redc[lane] : 0u;
-        const unsigned long long xb = lane < NW ? ws.red[lane] : 0ull;
-        unsigned sa = xa;
-        unsigned long long sb = xb;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned va = __shfl_up_sync(FULL, sa, o);
-            const unsigned long long vb = __shfl_up_sync(FULL, sb, o);
-            if (lane >= o) { sa += va; sb += vb; }
-        }
-        if (lane < NW) { ws.redc[lane] = sa - xa; ws.red[lane] = sb - xb; }
-        if (lane == 31) { ws.tc = sa; ws.tm = sb; }
-    }
-    __syncthreads();
-    *ea = ws.redc[warp] + ia - a;
-    *eb = ws.red[warp] + ib - b;
-    *ta = ws.tc;
-    *tb = ws.tm;
-    __syncthreads();
-}
-
-// One pass over a bf16 row: the window [khi - WF_KEYS + 1, khi] counted per
-// key in win[khi - key]; the rest summed into ws.ac/am/amax (above) and
-// ws.bc/bm (below).  All threads call it.
-template <int BT>
-__device__ void wf_pass(const char* row, int V, float s, float m, uint32_t khi, uint32_t* win, WinShared& ws) {
-    const int tid = threadIdx.x;
-    const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
-    for (int i = tid; i < WF_KEYS / 4; i += BT) reinterpret_cast<uint4*>(win)[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (tid == 0) { ws.ac = 0u; ws.bc = 0u; ws.am = 0ull; ws.bm = 0ull; ws.amax = 0u; }
-    __syncthreads();
-    unsigned ac = 0u, bc = 0u, amax = 0u;
-    unsigned long long am = 0ull, bm = 0ull;
-    const int nv = (V + 7) / 8;
-    auto one = [&](uint32_t k) {
-        if (k > khi) {
-            ++ac;
-            amax = max(amax, k);
-            am += fix_mass(key_value<SPEC_BF16>(k), s, m);
-        } else if (k >= klo) {
-            atomicAdd(&win[khi - k], 1u);
-        } else {
-            ++bc;
-            bm += fix_mass(key_value<SPEC_BF16>(k), s, m);
-        }
-    };
-    for (int v0 = tid; v0 < nv; v0 += 4 * BT) {
-        uint4 v[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int vi = v0 + q * BT;
-            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int vi = v0 + q * BT;
-            if (vi >= nv) break;
-            const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-            const int lim = V - vi * 8;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t k2 = vh_keys2(xs[c]);
-                if (2 * c < lim) one(k2 & 0xFFFFu);
-                if (2 * c + 1 < lim) one(k2 >> 16);
-            }
-        }
-    }
-    // fold the per-thread totals (integers: any order gives the same sums)
-    ac = __reduce_add_sync(FULL, ac);
-    bc = __reduce_add_sync(FULL, bc);
-    amax = __reduce_max_sync(FULL, amax);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        am += __shfl_xor_sync(FULL, am, o);
-        bm += __shfl_xor_sync(FULL, bm, o);
-    }
-    if ((tid & 31) == 0) {
-        atomicAdd(&ws.ac, ac);
-        atomicAdd(&ws.bc, bc);
-        atomicMax(&ws.amax, amax);
-        atomicAdd(&ws.am, am);
-        atomicAdd(&ws.bm, bm);
-    }
-    __syncthreads();
-}
-
-// Threshold and kept mass of one bf16 row (the record filter_row gives).  The
-// first window starts just above the key of the row's maximum estimated from
-// the statistics (m / s).  All threads call it.
-template <int BT>
-__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, uint32_t* win,
-                               WinShared& ws) {
-    constexpr int RUN = WF_KEYS / BT;                 // window keys per thread
-    static_assert(RUN * BT == WF_KEYS, "window split");
-    const int tid = threadIdx.x;
-    FiltRec r{-INFINITY, 0, 0.0};
-    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
-    if (!use_k && !use_p) return r;
-    // the row's largest value is about m / s (m = its value times s, rounded)
-    uint32_t khi = min(0xFFFFu, order_key<SPEC_BF16>(__bfloat162float(__float2bfloat16_rn(m / s))) + 4u);
-    bool rk = !use_k;                                 // top-k resolved
-    uint32_t tk = 0u, tp = 0u;
-    unsigned long long zk = 0ull, z = 0ull;
-    for (int it = 0; it < 2 * (65536 / WF_KEYS) + 2; ++it) {
-        wf_pass<BT>(row, V, s, m, khi, win, ws);
-        const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
-        const unsigned ac = ws.ac, amax = ws.amax;
-        const unsigned long long am = ws.am, bm = ws.bm;
-        // this thread's run of window indices [j0, j0 + RUN): keys khi - j
-        const int j0 = tid * RUN;
-        unsigned rc = 0u;
-        unsigned long long rm = 0ull;
-#pragma unroll 4
-        for (int j = j0; j < j0 + RUN; ++j) {
-            const unsigned c = win[j];
-            if (c) {
-                rc += c;
-                rm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
-            }
-        }
-        unsigned c0, ctot;
-        unsigned long long m0, mtot;
-        wf_scan2<BT>(rc, rm, &c0, &m0, &ctot, &mtot, ws);
-        c0 += ac;
-        m0 += am;
-        if (!use_k) zk = am + mtot + bm;
-        if (!rk) {
-            if ((unsigned)K <= ac) { khi = amax; continue; }                 // above the window
-            if ((unsigned)K > ac + ctot) {                                   // below the window
-                if (klo == 0u) break;                                        // (cannot happen: K < V)
-                khi = klo - 1u;
-                continue;
-            }
-            if (tid == 0) ws.sel = -1;
-            __syncthreads();
-            if (c0 < (unsigned)K && c0 + rc >= (unsigned)K) {
-                unsigned c = c0;
-                unsigned long long mm = m0;
-                for (int j = j0; j < j0 + RUN; ++j) {
-                    const unsigned cj = win[j];
-                    c += cj;
-                    if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
-                    if (c >= (unsigned)K) { ws.sel = j; ws.at = mm; break; }
-                }
-            }
-            __syncthreads();
-            tk = khi - (uint32_t)ws.sel;
-            zk = ws.at;
-            rk = true;
-            __syncthreads();
-        }
-        if (!use_p) { tp = tk; z = zk; break; }
-        const double target = (double)Pp * (double)zk;
-        if ((double)am >= target) { khi = amax; continue; }                 // above the window
-        if ((double)(am + mtot) < target) {                                 // below (top-p alone)
-            if (klo == 0u) break;                                            // (cannot happen: target <= total)
-            khi = klo - 1u;
-            continue;
-        }
-        if (tid == 0) ws.sel = -1;
-        __syncthreads();
-        if ((double)m0 < target && (double)(m0 + rm) >= target) {
-            unsigned long long mm = m0;
-            for (int j = j0; j < j0 + RUN; ++j) {
-                const unsigned cj = win[j];
-                if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
-                if (cj && (double)mm >= target) { ws.sel = j; ws.at = mm; break; }
-            }
-        }
-        __syncthreads();
-        tp = khi - (uint32_t)ws.sel;
-        z = ws.at;
-        __syncthreads();
-        break;
-    }
-    r.theta = key_value<SPEC_BF16>(tp);
-    r.on = 1;
-    r.Z = (double)z / FIX_ONE;
-    return r;
 }
 
 // Filter thresholds of every row of a chain round, one CTA per (sequence,
@@ -3206,7 +3282,15 @@ __device__ int draw_row(const WF& wf, int nch, float u, float* wpw, FinShared& s
 // chain_decide on the filtered distributions (p' and q' from each row's
 // statistics, threshold and kept mass), then the correction from
 // max(0, p'_k - q'_k) or the bonus from p'_gamma over the whole row.
-template <int TDT, int DDT, int DK>
+//
+// OD (on demand: bf16 rows, no diagnostics): instead of reading every row's
+// filter record, the CTA filters the rows the decision reaches -- target row
+// i and draft row i for i = 0, 1, ... up to the first rejection, row gamma
+// after a full acceptance -- with one window histogram each (win, after the
+// per-warp sums in dynamic shared memory).  The decision then takes the same
+// steps as with every record present: it never looks past the first
+// rejection.
+template <int TDT, int DDT, int DK, bool OD = false>
 __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
     __shared__ FinShared sh;
     extern __shared__ __align__(128) unsigned char dyn[];
@@ -3220,13 +3304,72 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
     combine_softmax_rows<SEQ_BT>(P, P.stats + (size_t)b * P.R * P.nch * SPC, P.R, sh);
     __syncthreads();
     const int rows = (DK == DK_LOGITS) ? 2 * gamma + 1 : gamma + 1;
-    for (int r = tid; r < rows; r += SEQ_BT) {
-        const FiltRec f = P.filt[(size_t)b * P.R + r];
-        sh.th[r] = f.theta;
-        if (f.on > 0) sh.z[r] = f.Z;
-        if (f.on < 0) sh.bad[r] = 1;                 // invalid top_k / top_p
+    if constexpr (!OD) {
+        for (int r = tid; r < rows; r += SEQ_BT) {
+            const FiltRec f = P.filt[(size_t)b * P.R + r];
+            sh.th[r] = f.theta;
+            if (f.on > 0) sh.z[r] = f.Z;
+            if (f.on < 0) sh.bad[r] = 1;             // invalid top_k / top_p
+        }
+        __syncthreads();
+    } else {
+        __shared__ WinShared ws;
+        uint32_t* win = reinterpret_cast<uint32_t*>(dyn + P.stage_off);
+        const int K = P.top_k ? P.top_k[b] : 0;
+        const float Pp = P.top_p ? P.top_p[b] : 1.f;
+        const float T = P.temperature[b];
+        for (int r = tid; r < rows; r += SEQ_BT) sh.th[r] = -INFINITY;
+        if (tid < gamma) {                          // the prefetched decision inputs, for thread 0
+            sh.tok[tid] = pf.x;
+            sh.pch[tid] = pf.ok ? (double)pf.l : NAN;
+            sh.pch[SPEC_MAX_GAMMA + tid] = (double)pf.d;
+            sh.pch[2 * SPEC_MAX_GAMMA + tid] = (double)pf.coin;
+        }
+        __syncthreads();
+        bool go = temperature_ok(T) && K >= 0 && Pp > 0.f && Pp <= 1.f;
+        for (int r = 0; r < rows; ++r) go &= !sh.bad[r];
+        if (!(K >= 0 && Pp > 0.f && Pp <= 1.f) && tid == 0) sh.bad[0] = 1;   // invalid top_k / top_p
+        const float s = scale_of(T);
+        for (int i = 0; go && i <= gamma; ++i) {
+            // filter target row i, and draft-logit row i below gamma
+            for (int half = 0; half < ((DK == DK_LOGITS && i < gamma) ? 2 : 1); ++half) {
+                const int r = half ? gamma + 1 + i : i;
+                const char* row = half ? P.drf + ((size_t)b * gamma + i) * P.dstride
+                                       : P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride;
+                const FiltRec f = wfilter_row<SEQ_BT>(row, V, s, sh.m[r], K, Pp, win, ws);
+                if (tid == 0) {
+                    sh.th[r] = f.theta;
+                    if (f.on > 0) sh.z[r] = f.Z;
+                }
+                __syncthreads();
+            }
+            if (i == gamma) break;
+            // the accept test of position i, as chain_decide takes it
+            if (tid == 0) {
+                int go_on = 0;
+                const double l = sh.pch[i];
+                if (l == l) {
+                    double p = prob_d((float)l, s, sh.m[i], sh.z[i]);
+                    if ((float)l < sh.th[i]) p = 0.0;
+                    double q;
+                    if constexpr (DK == DK_PROBS) {
+                        q = sh.pch[SPEC_MAX_GAMMA + i];
+                    } else {
+                        const float d = (float)sh.pch[SPEC_MAX_GAMMA + i];
+                        q = prob_d(d, s, sh.m[gamma + 1 + i], sh.z[gamma + 1 + i]);
+                        if (d < sh.th[gamma + 1 + i]) q = 0.0;
+                    }
+                    const double ratio = (q > 0.0) ? p / q : INFINITY;
+                    go_on = sh.pch[2 * SPEC_MAX_GAMMA + i] <= ratio;
+                }
+                sh.ivals[4] = go_on;
+            }
+            __syncthreads();
+            go = sh.ivals[4] != 0;
+            __syncthreads();
+        }
+        __syncthreads();
     }
-    __syncthreads();
     chain_decide<TDT, DDT, DK, true>(P, b, sh, true, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
     const float s = (float)sh.dvals[0];
@@ -4389,9 +4532,22 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    if constexpr (all_bf16) {
+        // No diagnostics to fill: the finalisation filters only the rows the
+        // decision reaches.
+        if (P.diag == nullptr) {
+            P.stage_off = (int)((wpw + 127) & ~(size_t)127);
+            auto kod = k_chain_final_filt<TDT, DDT, DK, true>;
+            const size_t smem = (size_t)P.stage_off + WF_BYTES;
+            static PerDevice<bool> od_c;
+            const bool od = od_c.get([&] { return allow_smem(kod, STAGE_STATS_MAX); });
+            if (!od || smem > STAGE_STATS_MAX) return fail(SPEC_ERR_CUDA, "k_chain_final_filt shared memory");
+            return launch_dependent(kod, (unsigned)P.B, SEQ_BT, smem, P, st, "k_chain_final_filt");
+        }
+    }
     s = launch_dependent(kf, (unsigned)(P.B * rows), bt, hist, P, st, "k_filter");
     if (s != SPEC_OK) return s;
-    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
     return launch_dependent(k_chain_final_filt<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, wpw, P, st,
                             "k_chain_final_filt");
 }
@@ -4458,6 +4614,17 @@ template <int TDT>
 spec_status launch_tree_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_SAMPLE, TDT, TDT>(P, st);
     if (s != SPEC_OK) return s;
+    if constexpr (TDT == SPEC_BF16) {
+        // No diagnostics to fill: the walk filters only the rows it visits.
+        if (P.diag == nullptr) {
+            static PerDevice<bool> od_c;
+            const bool od = od_c.get([] { return allow_stage(k_tree_final<MODE_SAMPLE_FILT_OD, TDT>); });
+            P.stage_cap = stats_stage_bytes(P, P.N, (od ? STAGE_STATS_MAX : 48 * 1024 - 1024) - WF_BYTES);
+            P.stage_off = (P.stage_cap + 15) & ~15;
+            return launch_dependent(k_tree_final<MODE_SAMPLE_FILT_OD, TDT>, (unsigned)P.B, SEQ_BT,
+                                    (size_t)P.stage_off + WF_BYTES, P, st, "k_tree_final");
+        }
+    }
     constexpr int bt = TDT == SPEC_BF16 ? WF_BT : FILT_BT;
     constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_filter<TDT, TDT, DK_NONE, true, bt>;

@@ -76,15 +76,15 @@ def oracle_chain_filtered(inp, top_k, top_p, rows=None, nthreads=0):
                         top_k=tk, top_p=tp)
 
 
-def gpu_chain_filtered(inp, top_k, top_p, workspace=None):
+def gpu_chain_filtered(inp, top_k, top_p, workspace=None, with_diag=True):
     from speculative_decoding_verify_temperature_b200 import spec_verify as sv
     B, g = inp.B, inp.gamma
-    diag = torch.full((B, 2 * g + 1), float("nan"), device=inp.target.device)
+    diag = torch.full((B, 2 * g + 1), float("nan"), device=inp.target.device) if with_diag else None
     toks, na = sv.spec_verify_chain_filtered(inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins,
                                              inp.final_u, top_k, top_p, draft_is_probs=inp.draft_is_probs,
                                              V=inp.V, diag=diag, workspace=workspace)
     torch.cuda.synchronize()
-    d = diag.cpu().numpy().astype(np.float64)
+    d = diag.cpu().numpy().astype(np.float64) if with_diag else np.full((B, 2 * g + 1), np.nan)
     return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy(),
                 px=d[:, :g], qx=d[:, g:2 * g], S=d[:, 2 * g])
 
@@ -145,9 +145,10 @@ def oracle_sample(inp, rows=None, nthreads=0, threshold_single=1.0, threshold_ac
                               threshold_acc=threshold_acc, V=inp.V, nthreads=nthreads, top_k=tk, top_p=tp)
 
 
-def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, lazy=False, top_k=None, top_p=None):
+def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, lazy=False, top_k=None, top_p=None,
+               with_diag=True):
     B, N = inp.B, inp.N
-    diag = torch.full((B, N + 1), float("nan"), device=inp.target.device)
+    diag = torch.full((B, N + 1), float("nan"), device=inp.target.device) if with_diag else None
     if top_k is not None or top_p is not None:
         ai, ot, na = _fn("spec_verify_tree_sample_filtered", lazy)(
             inp.target, inp.tokens, inp.parents, inp.temperature, inp.coins, inp.final_u, inp.max_depth,
@@ -159,7 +160,7 @@ def gpu_sample(inp, workspace=None, threshold_single=1.0, threshold_acc=1.0, laz
             draft_probs=inp.draft_probs, threshold_single=threshold_single, threshold_acc=threshold_acc,
             V=inp.V, diag=diag, workspace=workspace)
     torch.cuda.synchronize()
-    d = diag.cpu().numpy().astype(np.float64)
+    d = diag.cpu().numpy().astype(np.float64) if with_diag else np.full((B, N + 1), np.nan)
     return dict(accept_index=ai.cpu().numpy(), tokens=ot.cpu().numpy(), num_accepted=na.cpu().numpy(),
                 pchild=d[:, :N], S=d[:, N])
 

@@ -28,6 +28,11 @@ def _check(inp, tk, tp, rows=None, max_flag_frac=0.2):
     n = len(o["num_accepted"])
     assert nbad == 0, f"{nbad} unflagged mismatches of {n}: {det}"
     assert nflag <= max_flag_frac * n + 1, f"too many near-ties: {nflag}/{n}"
+    # without diagnostics (bf16 rows) only the rows the decision reaches are
+    # filtered: the same records there, so the same decisions and tokens
+    d = parity.gpu_chain_filtered(inp, tk, tp, with_diag=False)
+    np.testing.assert_array_equal(d["num_accepted"], g["num_accepted"])
+    np.testing.assert_array_equal(d["tokens"], g["tokens"])
     return g, o
 
 

@@ -28,6 +28,11 @@ def _check(inp, tk, tp, rows=None, max_flag_frac=0.2, **th):
     n = len(o["num_accepted"])
     assert nbad == 0, f"{nbad} unflagged mismatches of {n}: {det}"
     assert nflag <= max_flag_frac * n + 1, f"too many near-ties: {nflag}/{n}"
+    # without diagnostics (bf16 rows) the walk filters only the rows it
+    # visits: the same records, so the same walk and tokens
+    d = parity.gpu_sample(inp, top_k=tk, top_p=tp, with_diag=False, **th)
+    for key in ("num_accepted", "tokens", "accept_index"):
+        np.testing.assert_array_equal(d[key], g[key])
     return g, o
 
 
