@@ -55,6 +55,8 @@ def parse():
                          "--workload is 1, none otherwise; 'none' skips)")
     ap.add_argument("--config-cpu-seconds", type=float, default=3.0,
                     help="oracle seconds per configuration under per_config")
+    ap.add_argument("--with-diag", action="store_true",
+                    help="pass diagnostics buffers (the filtered workloads then filter every row up front)")
     return ap.parse_args()
 
 
@@ -143,13 +145,18 @@ def describe(wid: int, inp) -> dict:
 class Runner:
     """Calls the verify entry point of a workload through the Python binding."""
 
-    def __init__(self, wid, inp, ws, lazy=False):
+    def __init__(self, wid, inp, ws, lazy=False, diag=False):
         self.wid, self.inp, self.ws, self.sfx = wid, inp, ws, "_lazy" if lazy else ""
         if wid == 7:
             self._vp_setup()
         import torch
         B = inp.B
         dev = inp.target.device
+        self.diag = None
+        if diag and wid == 6:
+            self.diag = torch.empty((B, 2 * inp.gamma + 1), dtype=torch.float32, device=dev)
+        if diag and wid == 8:
+            self.diag = torch.empty((B, inp.N + 1), dtype=torch.float32, device=dev)
         if wid in (0, 1, 4, 6, 7):
             self.out = (torch.empty((B, inp.gamma + 1), dtype=torch.int32, device=dev),
                         torch.empty((B,), dtype=torch.int32, device=dev))
@@ -216,11 +223,12 @@ class Runner:
                                                 i.max_depth, i.meta["top_k"], i.meta["top_p"],
                                                 draft_probs=i.draft_probs, V=i.V, out_accept_index=self.out[0],
                                                 out_tokens=self.out[1], out_num_accepted=self.out[2],
-                                                workspace=self.ws)
+                                                diag=self.diag, workspace=self.ws)
         elif self.wid == 6:
             sv.spec_verify_chain_filtered(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                           i.meta["top_k"], i.meta["top_p"], draft_is_probs=i.draft_is_probs, V=i.V,
-                                          out_tokens=self.out[0], out_num_accepted=self.out[1], workspace=self.ws)
+                                          out_tokens=self.out[0], out_num_accepted=self.out[1], diag=self.diag,
+                                          workspace=self.ws)
         elif self.wid in (0, 1, 4):
             getattr(sv, "spec_verify_chain" + self.sfx)(i.target, i.draft, i.draft_tokens, i.temperature, i.coins, i.final_u,
                                  draft_is_probs=i.draft_is_probs, V=i.V, out_tokens=self.out[0],
@@ -492,7 +500,7 @@ def bench_config(wid, first, nsets, nbytes, world) -> dict:
 CONFIG_STEPS = {0: 2000, 1: 2000, 2: 500, 3: 250, 4: 250}
 
 
-def measure(wid, dev, world, steps, warmup, local, rank=0):
+def measure(wid, dev, world, steps, warmup, local, rank=0, diag=False):
     """Time one workload: CUDA-graph replays of its rotating input sets (CUDA
     events, max over ranks), the row kernel's own duration, the launches per
     call, and the accepted lengths of the measured rounds."""
@@ -501,7 +509,7 @@ def measure(wid, dev, world, steps, warmup, local, rank=0):
     sets, nbytes = input_sets(wid, dev, rank)
     first, nsets = sets[0], len(sets)
     ws = workspace_for(wid, first)
-    runners = [Runner(wid, s, ws) for s in sets]
+    runners = [Runner(wid, s, ws, diag=diag) for s in sets]
     stream = torch.cuda.current_stream()
     for i in range(max(3, warmup)):
         runners[i % nsets]()
@@ -678,7 +686,7 @@ def main():
     dev = torch.device("cuda", local)
     wid = args.workload
 
-    m = measure(wid, dev, ws_, args.steps, args.warmup, local, rank)
+    m = measure(wid, dev, ws_, args.steps, args.warmup, local, rank, diag=args.with_diag)
     first, sets, ws, K = m["first"], m["sets"], m["ws"], m["K"]
     peaks, peak_kind = measured_peaks()
     roofline = roofline_of(m, peaks, peak_kind, row_kernel_of(m))
@@ -696,6 +704,8 @@ def main():
         if args.lazy_steps > 0 and wid in (0, 1, 2, 3, 4, 5, 8) else None
 
     cfg = bench_config(wid, first, m["nsets"], m["nbytes"], ws_)
+    if args.with_diag:
+        cfg["diagnostics"] = "requested"
     line = {
         "metric": "verify rounds/s", "value": round(value, 2), "unit": "rounds/s", "n_gpus": ws_,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,

@@ -123,7 +123,6 @@ struct Params {
     const float* top_p;            // [B], nullable (1 = off)
     struct FiltRec* filt;          // [B][R]            (per-row threshold and kept mass)
     double* vp_cm;                 // [B][nch]          (vocabulary-parallel: chunk masses of the shard's residual)
-    struct FusedRec* frec;         // [B][gamma+1]      (fused chain: one record per position)
 };
 
 // Top-k / top-p filter of one row: keep logits >= theta; Z = the kept mass in
@@ -421,7 +420,7 @@ __device__ __forceinline__ void thread_softmax(const char* row, int V, int64_t e
 __device__ __forceinline__ float2 warp_softmax_stat(float mt, float st, bool bad) {
     const float mw = warp_max(mt);
     const bool anybad = __any_sync(FULL, bad);
-    const double contrib = (mt == -INFINITY) ? 0.0 : (double)st * ex2d(mt, mw);
+    const double contrib = (mt == -INFINITY) ? 0.0 : (double)(st * ex2(mt - mw));
     float sw = (float)warp_sum_d(contrib);
     if (anybad) sw = nanf_();
     return make_float2(mw, sw);
@@ -2740,423 +2739,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SEQ_BT) k_chain_fina
     }
 }
 
-// ============================================================================= fused chain verification
-//
-// Chain verification with draft logits of the target's dtype, when a row spans
-// at most FUSED_MAXC chunks: one launch per call.  The CTAs of a cluster hold
-// one position's target row and draft row, one 16 KB chunk of each per CTA,
-// staged in shared memory by asynchronous copies (thread tid stages and reads
-// the vectors k*NT + tid, the layout of k_stats, so the per-warp statistics
-// are the same numbers):
-//   1. each CTA pushes its chunk's per-warp softmax statistics into every
-//      CTA of the cluster (distributed shared memory), cluster barrier;
-//   2. every CTA combines the row statistics (the warp_combine order of the
-//      two-kernel path, so m, Z and p(x), q(x) are bit-identical), and forms
-//      the group sums of max(0, p - q) over its chunk (rule 2), pushes its
-//      chunk mass, cluster barrier;
-//   3. the CTA whose chunk holds u*S draws the position's correction token
-//      from its stage -- for every position, whether or not it turns out to
-//      be the first rejection -- and writes the position's record; the bonus
-//      position draws from p_gamma the same way (rule 3);
-//   4. the last record of a sequence to arrive (a counter, __threadfence
-//      before atomicAdd, no spin-wait) finds the first rejection k (rule 1)
-//      and writes the sequence's outputs.
-// Every element is exponentiated twice (statistics, residual) instead of once
-// plus a second launch that re-reads the rejected row pair: the round ends
-// when the last chunk has been streamed and scanned, with no separate tail.
-constexpr int FUSED_MAXC = 8;            // largest cluster: 8 chunks per row
-constexpr int FUSED_CTAS_PER_SM = 6;     // 32 KB of stage each
-constexpr int FUSED_STAGE = 2 * NT * VPT * 16;   // target chunk + draft chunk, bytes
-
-struct __align__(16) FusedRec {
-    int tok;       // the position's draw: correction (i < gamma) or bonus (i = gamma)
-    int x;         // drafted token
-    int acc;       // coin <= p(x) / q(x)
-    int ok;        // rows usable, token in range, temperature valid
-    float p, q;    // p_i(x_i), q_i(x_i)
-    float S;       // mass the draw was taken from (residual mass; 1 for the bonus)
-    int pad;
-};
-
-__device__ __forceinline__ void peer_st_f2(float2* p, unsigned peer, float2 v) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(peer));
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(remote), "f"(v.x), "f"(v.y) : "memory");
-}
-__device__ __forceinline__ void peer_st_f64(double* p, unsigned peer, double v) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(peer));
-    asm volatile("st.shared::cluster.f64 [%0], %1;" :: "r"(remote), "d"(v) : "memory");
-}
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" :: "r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-// Stage the NT*VPT 16-byte vectors of chunk c of a row (vector k*NT + tid by
-// thread tid): asynchronous copies for vectors inside the row, elements at or
-// past V as -inf.
-template <int DT>
-__device__ __forceinline__ void fused_stage(uint4* dst, const char* row, int V, int c) {
-    constexpr int EPV = Tr<DT>::EPV, CH = chunk_elems<DT>();
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        const int v = k * NT + threadIdx.x;
-        const int64_t e0 = (int64_t)c * CH + (int64_t)v * EPV;
-        if (e0 + EPV <= V) cp_async16(dst + v, row + e0 * Tr<DT>::ESZ);
-        else dst[v] = ld_vec<DT>(row, e0, V);
-    }
-}
-
-// Weights of the EPV elements of one 16-byte vector: max(0, p - q) of the
-// position's row pair (RES), or 2^(x s - m) of the target row -- the f32
-// expressions of the two-kernel path's weight functors.
-template <int DT, bool RES>
-__device__ __forceinline__ void fused_weights(const uint4& t, const uint4& d, float s, float mp, float izp,
-                                              float mq, float izq, float (&w)[8]) {
-    constexpr int EPV = Tr<DT>::EPV;
-#pragma unroll
-    for (int e = 0; e < EPV; ++e) {
-        if constexpr (RES) {
-            const float p = ex2(fmaf(vec_elem<DT>(t, e), s, -mp)) * izp;
-            const float q = ex2(fmaf(vec_elem<DT>(d, e), s, -mq)) * izq;
-            w[e] = fmaxf(0.f, p - q);
-        } else {
-            w[e] = ex2(fmaf(vec_elem<DT>(t, e), s, -mp));
-        }
-    }
-}
-
-// Scan units of this thread's vectors: the sum of each 8-element group in
-// index order, held by the thread whose vector starts the group (bf16: one
-// group per vector; f32: a vector is half a group, the even lane holds the
-// group's sum and the odd lane 0).
-template <int DT, bool RES>
-__device__ __forceinline__ void fused_units(const uint4* st_t, const uint4* st_d, float s, float mp, float izp,
-                                            float mq, float izq, float (&unit)[VPT]) {
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        const int v = k * NT + threadIdx.x;
-        float w[8];
-        fused_weights<DT, RES>(st_t[v], RES ? st_d[v] : st_t[v], s, mp, izp, mq, izq, w);
-        if constexpr (DT == SPEC_BF16) {
-            unit[k] = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
-        } else {
-            const float h = (w[0] + w[1]) + (w[2] + w[3]);
-            const float o = __shfl_xor_sync(FULL, h, 1);
-            unit[k] = (threadIdx.x & 1) ? 0.f : h + o;
-        }
-    }
-}
-
-// Inverse-CDF pick inside this CTA's chunk c: the scan units are scanned
-// block-wide in fp64 in index order (the arithmetic of rescan_chunk), the last
-// positive unit starting at or below t_loc owns the draw, and its thread walks
-// the group's weights.  Returns the token (-1 if the chunk holds no positive
-// weight).  All threads of the CTA must call it.
-template <int DT, bool RES>
-__device__ int fused_pick(const uint4* st_t, const uint4* st_d, const float (&unit)[VPT], int c, double t_loc,
-                          float s, float mp, float izp, float mq, float izq) {
-    constexpr int EPV = Tr<DT>::EPV, CH = chunk_elems<DT>();
-    __shared__ double wt[VPT][NWARP];
-    __shared__ int owner, found;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    double inc[VPT];
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        inc[k] = (double)unit[k];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double n = __shfl_up_sync(FULL, inc[k], o);
-            if (lane >= o) inc[k] += n;
-        }
-        if (lane == 31) wt[k][warp] = inc[k];
-    }
-    if (tid == 0) { owner = -1; found = -1; }
-    __syncthreads();
-    double base = 0.0;
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        double before = base;
-#pragma unroll
-        for (int w = 0; w < NWARP; ++w) if (w < warp) before += wt[k][w];
-        const double excl = before + inc[k] - (double)unit[k];
-        if (unit[k] > 0.f && excl <= t_loc) atomicMax(&owner, k * NT + tid);
-#pragma unroll
-        for (int w = 0; w < NWARP; ++w) base += wt[k][w];
-    }
-    __syncthreads();
-    const int og = owner;
-    if (og >= 0) {
-        const int ko = og / NT, lo = og - ko * NT;
-        if ((lo >> 5) == warp) {                      // the owner's warp (f32: the owner's pair partner too)
-            float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            const int v = ko * NT + tid;
-            fused_weights<DT, RES>(st_t[v], RES ? st_d[v] : st_t[v], s, mp, izp, mq, izq, w);
-            double inc_o = 0.0;
-            float unit_o = 0.f;
-#pragma unroll
-            for (int k = 0; k < VPT; ++k)
-                if (k == ko) { inc_o = inc[k]; unit_o = unit[k]; }
-            if constexpr (DT == SPEC_F32) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) w[4 + e] = __shfl_down_sync(FULL, w[e], 1);
-            }
-            if (tid == lo) {
-                double before = 0.0;
-                for (int kk = 0; kk < ko; ++kk)
-                    for (int ww = 0; ww < NWARP; ++ww) before += wt[kk][ww];
-                for (int ww = 0; ww < warp; ++ww) before += wt[ko][ww];
-                const double excl = before + inc_o - (double)unit_o;
-                const int64_t e0 = (int64_t)c * CH + (int64_t)og * EPV;
-                const double loc = t_loc - excl;
-                double acc = 0.0;
-                int pick = -1, last = -1;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    acc += (double)w[i];
-                    if (w[i] > 0.f) {
-                        last = (int)(e0 + i);
-                        if (pick < 0 && loc < acc) pick = (int)(e0 + i);
-                    }
-                }
-                found = pick >= 0 ? pick : last;
-            }
-        }
-    }
-    __syncthreads();
-    const int r = found;
-    __syncthreads();
-    return r;
-}
-
-// Chunk masses of the target row from its per-warp statistics, in units of
-// 2^(x - m) (the arithmetic of sample_target_row); returns their sum.
-__device__ __forceinline__ double fused_target_masses(const float2* st, int nch, float m, double* M) {
-    double S = 0.0;
-    for (int c = 0; c < nch; ++c) {
-        double Mc = 0.0;
-#pragma unroll
-        for (int w = 0; w < SPC; ++w) {
-            const float2 x = st[c * SPC + w];
-            if (x.x > -INFINITY) Mc += (double)x.y * ex2d(x.x, m);
-        }
-        M[c] = Mc;
-    }
-    for (int c = 0; c < nch; ++c) S += M[c];
-    return S;
-}
-
-// The chunk holding t (the first chunk with mass whose running total passes
-// t; rounding past the end: the last chunk with mass), -1 if none has mass;
-// *before = the mass of the chunks before it.
-__device__ __forceinline__ int mass_crossing(const double* M, int n, double t, double* before) {
-    double C = 0.0;
-    for (int c = 0; c < n; ++c) {
-        if (M[c] <= 0.0) continue;
-        if (t < C + M[c]) { *before = C; return c; }
-        C += M[c];
-    }
-    for (int c = n - 1; c >= 0; --c)
-        if (M[c] > 0.0) { *before = C - M[c]; return c; }
-    *before = 0.0;
-    return -1;
-}
-
-template <int DT>
-__global__ void __launch_bounds__(NT, FUSED_CTAS_PER_SM) k_chain_fused(const Params P) {
-    constexpr int CH = chunk_elems<DT>();
-    extern __shared__ __align__(128) unsigned char dyn[];
-    __shared__ float2 xst[FUSED_MAXC * SPC];      // per-warp statistics of the target row, [chunk][warp]
-    __shared__ float2 xsd[FUSED_MAXC * SPC];      // ... of the draft row
-    __shared__ double xm[FUSED_MAXC];             // residual masses of the chunks
-    __shared__ double s_z[2], s_red[NWARP];
-    __shared__ float s_m[2];
-    __shared__ int s_bad[2], s_last;
-    uint4* st_t = reinterpret_cast<uint4*>(dyn);
-    uint4* st_d = st_t + NT * VPT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nch = P.nch, gamma = P.gamma, W = gamma + 1, V = P.V;
-    const unsigned c = cluster_rank();
-    const int pid = blockIdx.x / nch;             // b * (gamma + 1) + i
-    const int b = pid / W, i = pid - b * W;
-    const bool pair = i < gamma;
-    const char* trow = P.tgt + ((size_t)b * W + i) * P.tstride;
-    const char* drow = P.drf + ((size_t)b * gamma + (pair ? i : 0)) * P.dstride;
-    fused_stage<DT>(st_t, trow, V, (int)c);
-    if (pair) fused_stage<DT>(st_d, drow, V, (int)c);
-    // decision inputs (thread 0), loaded while the chunks stream in
-    const float T = __ldg(P.temperature + b);
-    const float s = scale_of(T);
-    const float u = __ldg(P.final_u + b);
-    int x = 0;
-    float lx = 0.f, dx = 0.f, coin = 0.f;
-    bool xok = false;
-    if (pair && tid == 0) {
-        x = P.draft_tokens[(size_t)b * gamma + i];
-        coin = P.coins[(size_t)b * gamma + i];
-        xok = x >= 0 && x < V;
-        if (xok) {
-            lx = ld_elem<DT>(trow, x, V);
-            dx = ld_elem<DT>(drow, x, V);
-        }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    {
-        uint4 v[VPT];
-        float mt, st;
-        bool bad = false;
-#pragma unroll
-        for (int k = 0; k < VPT; ++k) v[k] = st_t[k * NT + tid];
-        thread_softmax_regs<DT, VPT>(v, s, mt, st, bad);
-        const float2 ws = warp_softmax_stat(mt, st, bad);
-        float2 wd = make_float2(-INFINITY, 0.f);
-        if (pair) {
-            bool bd = false;
-#pragma unroll
-            for (int k = 0; k < VPT; ++k) v[k] = st_d[k * NT + tid];
-            thread_softmax_regs<DT, VPT>(v, s, mt, st, bd);
-            wd = warp_softmax_stat(mt, st, bd);
-        }
-        if (lane == 0)
-            for (int r = 0; r < nch; ++r) {
-                peer_st_f2(&xst[c * SPC + warp], (unsigned)r, ws);
-                if (pair) peer_st_f2(&xsd[c * SPC + warp], (unsigned)r, wd);
-            }
-    }
-    cluster_sync_all();                           // every CTA holds the position's row statistics
-    if (warp < (pair ? 2 : 1)) {
-        float m;
-        double z;
-        const bool bad = warp_combine(warp == 0 ? xst : xsd, nch * SPC, m, z);
-        if (lane == 0) { s_m[warp] = m; s_z[warp] = z; s_bad[warp] = bad; }
-    }
-    __syncthreads();
-    const float mp = s_m[0];
-    const double zp = s_z[0];
-    const float mq = pair ? s_m[1] : 0.f;
-    const double zq = pair ? s_z[1] : 1.0;
-    const float izp = (float)(1.0 / zp), izq = (float)(1.0 / zq);
-    float unit[VPT];
-    double S = 1.0;                               // the mass of the draw (diagnostic)
-    bool res = pair;                              // residual draw (else from the target row)
-    int cs = -1;
-    double before = 0.0, t = 0.0;
-    if (pair) {
-        fused_units<DT, true>(st_t, st_d, s, mp, izp, mq, izq, unit);
-        double mine = 0.0;
-#pragma unroll
-        for (int k = 0; k < VPT; ++k) mine += (double)unit[k];
-        mine = warp_sum_d(mine);
-        if (lane == 0) s_red[warp] = mine;
-        __syncthreads();
-        if (tid < nch) {
-            double Mc = 0.0;
-#pragma unroll
-            for (int w = 0; w < NWARP; ++w) Mc += s_red[w];
-            peer_st_f64(&xm[c], (unsigned)tid, Mc);
-        }
-        cluster_sync_all();                       // every CTA holds every chunk's residual mass
-        S = 0.0;
-        for (int q = 0; q < nch; ++q) S += xm[q];
-        if (S > 0.0) {
-            t = (double)u * S;
-            cs = mass_crossing(xm, nch, t, &before);
-        } else {
-            res = false;                          // empty residual (rounding only): draw from p_i
-        }
-    }
-    double Mt[FUSED_MAXC];                        // target-row chunk masses (every thread its own copy)
-    if (!res) {
-        t = (double)u * fused_target_masses(xst, nch, mp, Mt);
-        cs = mass_crossing(Mt, nch, t, &before);
-    }
-    if (!bounds_ok(cs < nch)) cs = -1;
-    const int writer = cs >= 0 ? cs : 0;
-    if ((int)c != writer) return;                 // no CTA reads another's shared memory after the barriers
-    int y = -1;
-    if (cs >= 0) {
-        if (res) {
-            y = fused_pick<DT, true>(st_t, st_d, unit, cs, fmax(0.0, t - before), s, mp, izp, mq, izq);
-        } else {
-            fused_units<DT, false>(st_t, st_d, s, mp, 1.f, 0.f, 0.f, unit);
-            y = fused_pick<DT, false>(st_t, st_d, unit, cs, fmax(0.0, t - before), s, mp, 1.f, 0.f, 0.f);
-            // The chunk's statistics promised mass its weights do not hold (f32
-            // underflow at the edge of the range): skip it and rescan the next
-            // chunk from global memory, as the two-kernel path does.  Every
-            // thread takes the same steps.
-            for (int attempt = 1; y < 0 && attempt < nch; ++attempt) {
-                Mt[cs] = 0.0;
-                cs = mass_crossing(Mt, nch, t, &before);
-                if (cs < 0) break;
-                WTarget<DT> wf{trow, s, mp, nullptr, cs * CH, V};
-                double tot;
-                y = rescan_chunk<CH, NT>(wf, cs, V, fmax(0.0, t - before), u, &tot);
-            }
-        }
-    }
-    if (tid == 0) {
-        FusedRec r;
-        r.tok = y;
-        r.x = x;
-        r.ok = temperature_ok(T) && !s_bad[0] && (!pair || (!s_bad[1] && xok));
-        r.acc = 1;
-        r.p = r.q = 0.f;
-        if (pair && r.ok) {
-            const double p = prob_d(lx, s, mp, zp), q = prob_d(dx, s, mq, zq);
-            const double ratio = (q > 0.0) ? p / q : INFINITY;
-            r.acc = (coin <= ratio) ? 1 : 0;
-            r.p = (float)p;
-            r.q = (float)q;
-        }
-        r.S = pair ? (float)S : 1.0f;
-        r.pad = 0;
-        P.frec[(size_t)b * W + i] = r;
-        __threadfence();
-        s_last = atomicAdd(P.cnt2 + b, 1u) == (unsigned)W - 1u;
-    }
-    __syncthreads();
-    if (!s_last || warp != 0) return;
-    // the last position of sequence b to arrive: first rejection, outputs
-    __threadfence();
-    FusedRec r{};
-    if (lane < W) {
-        const int4* src = reinterpret_cast<const int4*>(P.frec + (size_t)b * W + lane);
-        const int4 a = __ldcg(src), e = __ldcg(src + 1);
-        r.tok = a.x; r.x = a.y; r.acc = a.z; r.ok = a.w;
-        r.p = __int_as_float(e.x); r.q = __int_as_float(e.y); r.S = __int_as_float(e.z);
-    }
-    const bool all_ok = __all_sync(FULL, lane >= W || r.ok);
-    const unsigned rej = __ballot_sync(FULL, lane < gamma && !r.acc);
-    const int k = rej ? __ffs(rej) - 1 : gamma;
-    const int yk = __shfl_sync(FULL, r.tok, k);
-    const float Sk = __shfl_sync(FULL, r.S, k);
-    int32_t* toks = P.out_tokens + (size_t)b * W;
-    float* dg = P.diag ? P.diag + (size_t)b * (2 * gamma + 1) : nullptr;
-    if (!all_ok) {
-        if (lane < W) toks[lane] = -1;
-        if (dg) for (int j = lane; j < 2 * gamma + 1; j += 32) dg[j] = nanf_();
-        if (lane == 0) {
-            P.out_num_accepted[b] = -1;
-            flag_input_error(P);
-        }
-    } else {
-        if (lane < W) toks[lane] = lane < k ? r.x : (lane == k ? yk : -1);
-        if (dg && lane < gamma) {
-            dg[lane] = r.p;
-            dg[gamma + lane] = r.q;
-        }
-        if (lane == 0) {
-            P.out_num_accepted[b] = k;
-            if (dg) dg[2 * gamma] = k < gamma ? Sk : 1.0f;
-        }
-    }
-    if (lane == 0) P.cnt2[b] = 0u;               // at rest again for the next call
-}
-
 // Tree finalisation, one CTA per sequence.
 template <int MODE, int TDT>
 __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
@@ -4269,7 +3851,7 @@ spec_status fail(spec_status st, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, vp, vpcm, frec, total;
+    size_t status, cnt2, stats, stats2, lz_seq, lz_rej, lz_list, lz_count, filt, vp, vpcm, total;
     int rej_cap;
     int R, nch_max;
 };
@@ -4303,9 +3885,6 @@ Layout make_layout(int entry, int B, int rows, int V) {
     // ... and the chunk masses of the shard's residual (reused by the draw)
     L.vpcm = off;
     if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(double) * (size_t)B * nch);
-    // fused chain verification: one record per (sequence, position)
-    L.frec = off;
-    if (entry == SPEC_ENTRY_CHAIN) off = align256(off + sizeof(FusedRec) * (size_t)B * (rows + 1));
     L.total = off;
     return L;
 }
@@ -4390,7 +3969,6 @@ void bind_ws(Params& P, void* ws, const Layout& L) {
     P.lz_count = reinterpret_cast<unsigned*>(w + L.lz_count);
     P.filt = reinterpret_cast<FiltRec*>(w + L.filt);
     P.vp_cm = reinterpret_cast<double*>(w + L.vpcm);
-    P.frec = reinterpret_cast<FusedRec*>(w + L.frec);
 }
 
 spec_status launched(const char* what) {
@@ -4552,37 +4130,8 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
                             "k_chain_final_filt");
 }
 
-// Fused chain verification: one cluster of nch CTAs per (sequence, position).
-template <int DT>
-spec_status launch_chain_fused(const Params& P, cudaStream_t st) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((long long)P.B * (P.gamma + 1) * P.nch));
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = FUSED_STAGE;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)P.nch;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_chain_fused<DT>, P);
-    if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "k_chain_fused launch: %s", cudaGetErrorString(e));
-    spec_status s = launched("k_chain_fused");
-    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
-        return fail(SPEC_ERR_CUDA, "profile event");
-    return s;
-}
-
 template <int TDT, int DDT, int DK>
 spec_status launch_chain(Params P, cudaStream_t st) {
-    // Draft logits of the target's dtype with rows of at most FUSED_MAXC
-    // chunks: the whole round in one launch.
-    if constexpr (DK == DK_LOGITS && TDT == DDT) {
-        if (P.nch <= FUSED_MAXC) return launch_chain_fused<TDT>(P, st);
-    }
     // draft probabilities are read only by the finalize kernel
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;

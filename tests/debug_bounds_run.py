@@ -26,8 +26,10 @@ def main():
                 wl.chain_inputs(4, 2, 40000, seed=3, device="cuda", target_dtype=torch.float32,
                                 draft_dtype=torch.float32)]:
         o = parity.oracle_chain(inp)
-        bad += parity.compare_chain(parity.gpu_chain(inp), o, inp.gamma)[1]
-        bad += parity.compare_chain(parity.gpu_chain(inp, lazy=True), o, inp.gamma)[1]
+        d = parity.gpu_chain(inp)
+        bad += parity.compare_chain(d, o, inp.gamma)[1]
+        z = parity.gpu_chain(inp, lazy=True)             # diagnostics only where evaluated: compare tokens
+        bad += int((z["tokens"] != d["tokens"]).any(axis=1).sum() + (z["num_accepted"] != d["num_accepted"]).sum())
     inp = wl.chain_inputs(6, 3, 5000, seed=4, device="cuda", zipf=True)
     tk = torch.tensor([0, 20, 50, 0, 20, 50], dtype=torch.int32, device="cuda")
     tp = torch.tensor([0.9, 1.0, 0.95, 0.9, 1.0, 0.95], dtype=torch.float32, device="cuda")
@@ -38,8 +40,10 @@ def main():
     bad += parity.compare_tree(parity.gpu_greedy(inp), parity.oracle_greedy(inp))[1]
     inp = wl.tree_sample_inputs(4, 3000, seed=6, device="cuda")
     o = parity.oracle_sample(inp)
-    bad += parity.compare_tree(parity.gpu_sample(inp), o, sample=True)[1]
-    bad += parity.compare_tree(parity.gpu_sample(inp, lazy=True), o, sample=True)[1]
+    d = parity.gpu_sample(inp)
+    bad += parity.compare_tree(d, o, sample=True)[1]
+    z = parity.gpu_sample(inp, lazy=True)
+    bad += int((z["tokens"] != d["tokens"]).any(axis=1).sum() + (z["num_accepted"] != d["num_accepted"]).sum())
     tk = torch.tensor([0, 20, 50, 5], dtype=torch.int32, device="cuda")
     tp = torch.tensor([0.9, 1.0, 0.95, 0.5], dtype=torch.float32, device="cuda")
     bad += parity.compare_tree(parity.gpu_sample(inp, top_k=tk, top_p=tp),
