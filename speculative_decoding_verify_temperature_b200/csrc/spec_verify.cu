@@ -744,34 +744,50 @@ __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
     return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
 }
 
-// bf16 rows, windowed: an exact count histogram of WF_KEYS consecutive order
-// keys (u32 counters, 32 KB) from the row's largest key down, plus exact
-// integer totals -- counts and fixed-point masses, count * fixed(2^(v s - m))
-// per value -- of the elements above and below the window.  Every key's
-// mass is count * fixed(2^(v s - m)), so the running counts and masses from
-// the top, and with them the top-k key, the kept mass and the top-p key, are
-// the integers of the full value histogram.  A threshold that falls outside
-// the window moves it (up to the row's true maximum, or down below it) and
-// the row is counted again; the first window holds both thresholds unless the
-// kept set reaches far below the maximum.
-constexpr int WF_KEYS = 8192;
-constexpr size_t WF_BYTES = (size_t)WF_KEYS * 4;
+// bf16 rows, two passes and a sparse window.
+//  1. a count histogram of the order keys' top 12 bits (4096 buckets of 16
+//     keys) over the whole row;
+//  2. from it, per bucket, bounds on its mass (count times the fixed-point
+//     mass of its lowest and highest key, with a relative slack far above
+//     the exp2 unit's ulp); scanned from the top, the bounds give a bucket at
+//     or below both thresholds: the top-k bucket (counts are exact) and the
+//     first bucket whose lower-bound running mass reaches top_p times the
+//     upper bound of the kept mass;
+//  3. a second pass counts, per key, only the elements of the non-empty
+//     buckets from the top down to that bucket (16 counters per non-empty
+//     bucket, in descending key order); every other element adds its fixed-
+//     point mass to an exact total (the kept mass when top-k is off).
+// Every key's mass is then count * fixed(2^(v s - m)), as in a full value
+// histogram, so the running counts and masses from the top, the top-k key,
+// the kept mass and the top-p key are the same integers.  A window needing
+// more than WF_SLOTS counters is counted in segments, one more pass each.
+constexpr int WF_NB = 4096;                       // coarse buckets (key >> 4)
+constexpr int WF_SLOTS = 8192;                    // per-key counters of the window
+constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 56 KB
+constexpr unsigned short WF_NONE = 0xFFFFu;
 
 struct WinShared {
     unsigned long long red[32];
+    double rlo[32], rhi[32];
     unsigned redc[32];
-    unsigned long long am, bm, tm;        // masses above / below the window, window total
-    unsigned ac, bc, tc, amax;            // counts above / below, window total, largest key above
-    int sel;
+    unsigned long long tm, acc;
+    double tlo, thi, dv;
+    unsigned tc;
+    int pos_k, pos_p, nord, sel;
     unsigned long long at;
 };
 
 __device__ __forceinline__ unsigned long long fix_mass(float x, float s, float m) {
     return (unsigned long long)(ex2(fmaf(x, s, -m)) * (float)FIX_ONE);
 }
+// The same mass as a double, for bounds only (exponent clamped: a bucket's
+// top key may lie above the row's maximum).
+__device__ __forceinline__ double bound_mass(float x, float s, float m) {
+    return (double)ex2(fminf(fmaf(x, s, -m), 60.f)) * FIX_ONE;
+}
 
-// Block-wide exclusive scan, in thread order, of a u32 and a u64 (BT threads,
-// BT / 32 <= 32 warps); the totals go to *ta / *tb.  All threads call it.
+// Block-wide exclusive scan, in thread order, of a u32 and a u64 (BT / 32 <=
+// 32 warps); totals to *ta / *tb.  All threads call it.
 template <int BT>
 __device__ void wf_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
                          unsigned long long* tb, WinShared& ws) {
@@ -809,32 +825,53 @@ __device__ void wf_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigne
     __syncthreads();
 }
 
-// One pass over a bf16 row: the window [khi - WF_KEYS + 1, khi] counted per
-// key in win[khi - key]; the rest summed into ws.ac/am/amax (above) and
-// ws.bc/bm (below).  All threads call it.
+// Block-wide exclusive scan, in thread order, of a u32 and two doubles (the
+// bucket counts and mass bounds); totals to *tc, *tl, *th.
 template <int BT>
-__device__ void wf_pass(const char* row, int V, float s, float m, uint32_t khi, uint32_t* win, WinShared& ws) {
-    const int tid = threadIdx.x;
-    const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
-    for (int i = tid; i < WF_KEYS / 4; i += BT) reinterpret_cast<uint4*>(win)[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (tid == 0) { ws.ac = 0u; ws.bc = 0u; ws.am = 0ull; ws.bm = 0ull; ws.amax = 0u; }
+__device__ void wf_scan3(unsigned c, double l, double h, unsigned* ec, double* el, double* eh, unsigned* tc,
+                         double* tl, double* th, WinShared& ws) {
+    constexpr int NW = BT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned ic = c;
+    double il = l, ih = h;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned vc = __shfl_up_sync(FULL, ic, o);
+        const double vl = __shfl_up_sync(FULL, il, o), vh = __shfl_up_sync(FULL, ih, o);
+        if (lane >= o) { ic += vc; il += vl; ih += vh; }
+    }
+    if (lane == 31) { ws.redc[warp] = ic; ws.rlo[warp] = il; ws.rhi[warp] = ih; }
     __syncthreads();
-    unsigned ac = 0u, bc = 0u, amax = 0u;
-    unsigned long long am = 0ull, bm = 0ull;
-    const int nv = (V + 7) / 8;
-    auto one = [&](uint32_t k) {
-        if (k > khi) {
-            ++ac;
-            amax = max(amax, k);
-            am += fix_mass(key_value<SPEC_BF16>(k), s, m);
-        } else if (k >= klo) {
-            atomicAdd(&win[khi - k], 1u);
-        } else {
-            ++bc;
-            bm += fix_mass(key_value<SPEC_BF16>(k), s, m);
+    if (warp == 0) {
+        const unsigned xc = lane < NW ? ws.redc[lane] : 0u;
+        const double xl = lane < NW ? ws.rlo[lane] : 0.0, xh = lane < NW ? ws.rhi[lane] : 0.0;
+        unsigned sc = xc;
+        double sl = xl, sh = xh;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned vc = __shfl_up_sync(FULL, sc, o);
+            const double vl = __shfl_up_sync(FULL, sl, o), vh = __shfl_up_sync(FULL, sh, o);
+            if (lane >= o) { sc += vc; sl += vl; sh += vh; }
         }
-    };
-    for (int v0 = tid; v0 < nv; v0 += 4 * BT) {
+        if (lane < NW) { ws.redc[lane] = sc - xc; ws.rlo[lane] = sl - xl; ws.rhi[lane] = sh - xh; }
+        if (lane == 31) { ws.tc = sc; ws.tlo = sl; ws.thi = sh; }
+    }
+    __syncthreads();
+    *ec = ws.redc[warp] + ic - c;
+    *el = ws.rlo[warp] + il - l;
+    *eh = ws.rhi[warp] + ih - h;
+    *tc = ws.tc;
+    *tl = ws.tlo;
+    *th = ws.thi;
+    __syncthreads();
+}
+
+// Calls f(key) for every element of a bf16 row (BT threads, four 16-byte
+// loads in flight per thread).
+template <int BT, class F>
+__device__ __forceinline__ void wf_each_key(const char* row, int V, F f) {
+    const int nv = (V + 7) / 8;
+    for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * BT) {
         uint4 v[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -850,119 +887,197 @@ __device__ void wf_pass(const char* row, int V, float s, float m, uint32_t khi, 
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const uint32_t k2 = vh_keys2(xs[c]);
-                if (2 * c < lim) one(k2 & 0xFFFFu);
-                if (2 * c + 1 < lim) one(k2 >> 16);
+                if (2 * c < lim) f(k2 & 0xFFFFu);
+                if (2 * c + 1 < lim) f(k2 >> 16);
             }
         }
     }
-    // fold the per-thread totals (integers: any order gives the same sums)
-    ac = __reduce_add_sync(FULL, ac);
-    bc = __reduce_add_sync(FULL, bc);
-    amax = __reduce_max_sync(FULL, amax);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        am += __shfl_xor_sync(FULL, am, o);
-        bm += __shfl_xor_sync(FULL, bm, o);
-    }
-    if ((tid & 31) == 0) {
-        atomicAdd(&ws.ac, ac);
-        atomicAdd(&ws.bc, bc);
-        atomicMax(&ws.amax, amax);
-        atomicAdd(&ws.am, am);
-        atomicAdd(&ws.bm, bm);
-    }
-    __syncthreads();
 }
 
-// Threshold and kept mass of one bf16 row (the record filter_row gives).  The
-// first window starts just above the key of the row's maximum estimated from
-// the statistics (m / s).  All threads call it.
+// Threshold and kept mass of one bf16 row (the record filter_row gives).
+// smem: WF_BYTES of shared memory.  All threads call it.
 template <int BT>
-__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, uint32_t* win,
+__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, unsigned char* smem,
                                WinShared& ws) {
-    constexpr int RUN = WF_KEYS / BT;                 // window keys per thread
-    static_assert(RUN * BT == WF_KEYS, "window split");
+    constexpr int RB = WF_NB / BT;                    // coarse buckets per thread (descending positions)
+    constexpr int RS = WF_SLOTS / BT;                 // window counters per thread
+    static_assert(RB * BT == WF_NB && RS * BT == WF_SLOTS, "split");
     const int tid = threadIdx.x;
     FiltRec r{-INFINITY, 0, 0.0};
     const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
     if (!use_k && !use_p) return r;
-    // the row's largest value is about m / s (m = its value times s, rounded)
-    uint32_t khi = min(0xFFFFu, order_key<SPEC_BF16>(__bfloat162float(__float2bfloat16_rn(m / s))) + 4u);
-    bool rk = !use_k;                                 // top-k resolved
-    uint32_t tk = 0u, tp = 0u;
-    unsigned long long zk = 0ull, z = 0ull;
-    for (int it = 0; it < 2 * (65536 / WF_KEYS) + 2; ++it) {
-        wf_pass<BT>(row, V, s, m, khi, win, ws);
-        const uint32_t klo = khi >= (uint32_t)(WF_KEYS - 1) ? khi - (uint32_t)(WF_KEYS - 1) : 0u;
-        const unsigned ac = ws.ac, amax = ws.amax;
-        const unsigned long long am = ws.am, bm = ws.bm;
-        // this thread's run of window indices [j0, j0 + RUN): keys khi - j
-        const int j0 = tid * RUN;
-        unsigned rc = 0u;
-        unsigned long long rm = 0ull;
-#pragma unroll 4
-        for (int j = j0; j < j0 + RUN; ++j) {
-            const unsigned c = win[j];
-            if (c) {
-                rc += c;
-                rm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
+    uint32_t* coarse = reinterpret_cast<uint32_t*>(smem);                        // pass 1 counts
+    unsigned short* bucket_of = reinterpret_cast<unsigned short*>(smem);         // ordinal -> bucket (reuses coarse)
+    unsigned short* ord_of = reinterpret_cast<unsigned short*>(smem + (size_t)WF_NB * 4);   // bucket -> ordinal
+    uint32_t* slots = reinterpret_cast<uint32_t*>(smem + (size_t)WF_NB * 6);
+    // ---- pass 1: coarse counts
+    for (int i = tid; i < WF_NB / 4; i += BT) reinterpret_cast<uint4*>(coarse)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    wf_each_key<BT>(row, V, [&](uint32_t k) { atomicAdd(&coarse[k >> 4], 1u); });
+    __syncthreads();
+    // ---- choose the window: positions p = 0.. from the top bucket down
+    const int p0 = tid * RB;
+    unsigned cnt[RB];
+    unsigned rc = 0u;
+    double rl = 0.0, rh = 0.0;
+    constexpr double LO = 1.0 - 1e-5, HI = 1.0 + 1e-5;      // slack over the exp2 unit's rounding
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+        const uint32_t b = (uint32_t)(WF_NB - 1 - (p0 + j));
+        cnt[j] = coarse[b];
+        if (cnt[j]) {
+            rc += cnt[j];
+            rl += (double)cnt[j] * bound_mass(key_value<SPEC_BF16>(b << 4), s, m) * LO;
+            rh += (double)cnt[j] * bound_mass(key_value<SPEC_BF16>((b << 4) | 15u), s, m) * HI;
+        }
+    }
+    unsigned c0, ctot;
+    double l0, h0, ltot, htot;
+    wf_scan3<BT>(rc, rl, rh, &c0, &l0, &h0, &ctot, &ltot, &htot, ws);
+    if (tid == 0) { ws.pos_k = -1; ws.pos_p = WF_NB - 1; ws.dv = htot; }
+    __syncthreads();
+    if (use_k && c0 < (unsigned)K && c0 + rc >= (unsigned)K) {     // the top-k bucket (exact counts)
+        unsigned c = c0;
+        double h = h0;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            c += cnt[j];
+            if (cnt[j]) {
+                const uint32_t b = (uint32_t)(WF_NB - 1 - (p0 + j));
+                h += (double)cnt[j] * bound_mass(key_value<SPEC_BF16>((b << 4) | 15u), s, m) * HI;
+            }
+            if (c >= (unsigned)K) { ws.pos_k = p0 + j; ws.dv = h; break; }
+        }
+    }
+    __syncthreads();
+    const int pos_k = ws.pos_k;
+    const double target_hi = (double)Pp * ws.dv * HI;   // top_p of an upper bound of the kept mass
+    __syncthreads();
+    if (use_p && l0 < target_hi && l0 + rl >= target_hi) {
+        double l = l0;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            if (cnt[j]) {
+                const uint32_t b = (uint32_t)(WF_NB - 1 - (p0 + j));
+                l += (double)cnt[j] * bound_mass(key_value<SPEC_BF16>(b << 4), s, m) * LO;
+            }
+            if (l >= target_hi) { ws.pos_p = p0 + j; break; }
+        }
+    }
+    __syncthreads();
+    // window: positions [0, nb) -- down to the top-k bucket (the top-p key lies
+    // at or above the top-k key), else down to the top-p bound
+    const int nb = use_k ? pos_k + 1 : ws.pos_p + 1;
+    // ---- ordinals of the window's non-empty buckets, in descending order
+    unsigned ne = 0u;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) ne += (p0 + j < nb && cnt[j]) ? 1u : 0u;
+    unsigned o0, otot;
+    unsigned long long d0, d1;
+    wf_scan2<BT>(ne, 0ull, &o0, &d0, &otot, &d1, ws);      // (after its barriers nobody reads coarse)
+    {
+        unsigned o = o0;
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            const uint32_t b = (uint32_t)(WF_NB - 1 - (p0 + j));
+            if (p0 + j < nb && cnt[j]) {
+                ord_of[b] = (unsigned short)o;
+                bucket_of[o] = (unsigned short)b;
+                ++o;
+            } else {
+                ord_of[b] = WF_NONE;
             }
         }
-        unsigned c0, ctot;
-        unsigned long long m0, mtot;
-        wf_scan2<BT>(rc, rm, &c0, &m0, &ctot, &mtot, ws);
-        c0 += ac;
-        m0 += am;
-        if (!use_k) zk = am + mtot + bm;
-        if (!rk) {
-            if ((unsigned)K <= ac) { khi = amax; continue; }                 // above the window
-            if ((unsigned)K > ac + ctot) {                                   // below the window
-                if (klo == 0u) break;                                        // (cannot happen: K < V)
-                khi = klo - 1u;
-                continue;
+    }
+    __syncthreads();
+    const int nslot = (int)otot * 16;
+    // ---- pass 2, per segment of WF_SLOTS counters: per-key counts, exact totals
+    bool rk = !use_k, rp = !use_p;
+    uint32_t tk = 0x007Fu, tp = 0x007Fu;             // -inf: keep everything (never left so)
+    unsigned cb = 0u;                                  // count of the keys above this segment
+    unsigned long long mb = 0ull, zk = 0ull, z = 0ull, total = 0ull;
+    for (int seg = 0; seg * WF_SLOTS < max(nslot, 1) && !(rk && rp); ++seg) {
+        const int slo = seg * WF_SLOTS;
+        for (int i = tid; i < WF_SLOTS / 4; i += BT) reinterpret_cast<uint4*>(slots)[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (tid == 0) ws.acc = 0ull;
+        __syncthreads();
+        unsigned long long other = 0ull;               // fixed-point mass of the elements outside this segment
+        wf_each_key<BT>(row, V, [&](uint32_t k) {
+            const unsigned short o = ord_of[k >> 4];
+            const int sl = (int)o * 16 + (15 - (int)(k & 15u)) - slo;
+            if (o != WF_NONE && sl >= 0 && sl < WF_SLOTS) atomicAdd(&slots[sl], 1u);
+            else if (seg == 0 && !use_k) other += fix_mass(key_value<SPEC_BF16>(k), s, m);
+        });
+        if (seg == 0 && !use_k) {
+#pragma unroll
+            for (int o = 16; o; o >>= 1) other += __shfl_xor_sync(FULL, other, o);
+            if ((tid & 31) == 0) atomicAdd(&ws.acc, other);
+        }
+        __syncthreads();
+        // this segment's keys in descending order: thread runs of RS counters
+        const int s0 = tid * RS;
+        unsigned sc = 0u;
+        unsigned long long sm = 0ull;
+        for (int j = 0; j < RS; ++j) {
+            const unsigned c = slots[s0 + j];
+            if (c) {
+                const int g = slo + s0 + j;
+                const uint32_t key = ((uint32_t)bucket_of[g >> 4] << 4) | (uint32_t)(15 - (g & 15));
+                sc += c;
+                sm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(key), s, m);
             }
+        }
+        unsigned e0, etot;
+        unsigned long long f0, ftot;
+        wf_scan2<BT>(sc, sm, &e0, &f0, &etot, &ftot, ws);
+        e0 += cb;
+        f0 += mb;
+        if (seg == 0 && !use_k) { total = ws.acc + ftot; zk = total; }
+        auto find = [&](bool by_count, double target) {   // the thread whose run crosses the target
             if (tid == 0) ws.sel = -1;
             __syncthreads();
-            if (c0 < (unsigned)K && c0 + rc >= (unsigned)K) {
-                unsigned c = c0;
-                unsigned long long mm = m0;
-                for (int j = j0; j < j0 + RUN; ++j) {
-                    const unsigned cj = win[j];
+            const bool cross = by_count ? (e0 < (unsigned)K && e0 + sc >= (unsigned)K)
+                                        : ((double)f0 < target && (double)(f0 + sm) >= target);
+            if (cross) {
+                unsigned c = e0;
+                unsigned long long mm = f0;
+                for (int j = 0; j < RS; ++j) {
+                    const unsigned cj = slots[s0 + j];
+                    if (!cj) continue;
+                    const int g = slo + s0 + j;
+                    const uint32_t key = ((uint32_t)bucket_of[g >> 4] << 4) | (uint32_t)(15 - (g & 15));
                     c += cj;
-                    if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
-                    if (c >= (unsigned)K) { ws.sel = j; ws.at = mm; break; }
+                    mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(key), s, m);
+                    if (by_count ? c >= (unsigned)K : (double)mm >= target) {
+                        ws.sel = (int)key;
+                        ws.at = mm;
+                        break;
+                    }
                 }
             }
             __syncthreads();
-            tk = khi - (uint32_t)ws.sel;
+        };
+        if (!rk && cb + etot >= (unsigned)K) {               // the top-k key lies in this segment
+            find(true, 0.0);
+            tk = (uint32_t)ws.sel;
             zk = ws.at;
             rk = true;
             __syncthreads();
         }
-        if (!use_p) { tp = tk; z = zk; break; }
-        const double target = (double)Pp * (double)zk;
-        if ((double)am >= target) { khi = amax; continue; }                 // above the window
-        if ((double)(am + mtot) < target) {                                 // below (top-p alone)
-            if (klo == 0u) break;                                            // (cannot happen: target <= total)
-            khi = klo - 1u;
-            continue;
-        }
-        if (tid == 0) ws.sel = -1;
-        __syncthreads();
-        if ((double)m0 < target && (double)(m0 + rm) >= target) {
-            unsigned long long mm = m0;
-            for (int j = j0; j < j0 + RUN; ++j) {
-                const unsigned cj = win[j];
-                if (cj) mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(khi - (uint32_t)j), s, m);
-                if (cj && (double)mm >= target) { ws.sel = j; ws.at = mm; break; }
+        if (rk && !rp) {
+            const double target = (double)Pp * (double)zk;
+            if ((double)(mb + ftot) >= target) {            // the top-p key lies in this segment
+                find(false, target);
+                tp = (uint32_t)ws.sel;
+                z = ws.at;
+                rp = true;
+                __syncthreads();
             }
         }
-        __syncthreads();
-        tp = khi - (uint32_t)ws.sel;
-        z = ws.at;
-        __syncthreads();
-        break;
+        cb += etot;
+        mb += ftot;
     }
+    if (!use_p) { tp = tk; z = zk; }
     r.theta = key_value<SPEC_BF16>(tp);
     r.on = 1;
     r.Z = (double)z / FIX_ONE;
@@ -1955,7 +2070,7 @@ __device__ int tree_filt_draw(const Params& P, int b, int cur, const int* rej, i
 // computed here for the rows of the nodes the walk visits, one window
 // histogram each (win: WF_BYTES of shared memory).
 template <int TDT, int BT, bool FILT = false, bool OD = false>
-__device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk, uint32_t* win = nullptr,
+__device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk, unsigned char* win = nullptr,
                                 WinShared* ws = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = P.N, V = P.V, W = P.max_depth + 1;
@@ -2753,7 +2868,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     else if constexpr (MODE == MODE_SAMPLE_FILT_OD) {
         __shared__ WinShared ws;
         finalize_sample<TDT, SEQ_BT, true, true>(P, blockIdx.x, sh, blk,
-                                                 reinterpret_cast<uint32_t*>(dyn + P.stage_off), &ws);
+                                                 dyn + P.stage_off, &ws);
     }
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
@@ -2769,7 +2884,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
 constexpr int WF_BT = 256;
 
 template <int TDT, int DDT, int DK, bool TREE, int BT>
-__global__ void __launch_bounds__(BT) k_filter(const Params P) {
+__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Params P) {
     __shared__ FiltShared fs;
     __shared__ WinShared ws;
     __shared__ float msh;
@@ -2810,7 +2925,7 @@ __global__ void __launch_bounds__(BT) k_filter(const Params P) {
     const float s = scale_of(T), m = msh;
     FiltRec rec{-INFINITY, 0, 0.0};
     if ((tgt ? TDT : DDT) == SPEC_BF16) {
-        rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, reinterpret_cast<uint32_t*>(dyn), ws);
+        rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
     } else if constexpr (BT == FILT_BT) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
@@ -2896,7 +3011,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
         __syncthreads();
     } else {
         __shared__ WinShared ws;
-        uint32_t* win = reinterpret_cast<uint32_t*>(dyn + P.stage_off);
+        unsigned char* win = dyn + P.stage_off;
         const int K = P.top_k ? P.top_k[b] : 0;
         const float Pp = P.top_p ? P.top_p[b] : 1.f;
         const float T = P.temperature[b];
@@ -3641,7 +3756,7 @@ __global__ void __launch_bounds__(NT) k_lz_decide_tree(const Params P) {
 // every active sequence at this level (one CTA each, as k_filter), between
 // the level's statistics and its decisions.
 template <int TDT, int BT>
-__global__ void __launch_bounds__(BT) k_lz_filter_tree(const Params P) {
+__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_lz_filter_tree(const Params P) {
     __shared__ FiltShared fs;
     __shared__ WinShared ws;
     __shared__ float msh;
@@ -3679,7 +3794,7 @@ __global__ void __launch_bounds__(BT) k_lz_filter_tree(const Params P) {
     const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
     const float s = scale_of(T), m = msh;
     FiltRec rec{-INFINITY, 0, 0.0};
-    if constexpr (TDT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, reinterpret_cast<uint32_t*>(dyn), ws);
+    if constexpr (TDT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
     else if constexpr (BT == FILT_BT) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
     if (threadIdx.x == 0) *out = rec;
 }

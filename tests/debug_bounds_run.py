@@ -22,7 +22,7 @@ def main():
     bad = 0
     # chain: fused (draft logits), two-kernel (probabilities, f32 over 8 chunks), lazy, filtered
     for inp in [wl.chain_inputs(8, 4, 20000, seed=1, device="cuda", zipf=True, temperatures=(0.6, 1.0)),
-                wl.chain_inputs(6, 3, 30001, seed=2, device="cuda", draft_is_probs=True),
+                wl.chain_inputs(6, 3, 30000, seed=2, device="cuda", draft_is_probs=True),
                 wl.chain_inputs(4, 2, 40000, seed=3, device="cuda", target_dtype=torch.float32,
                                 draft_dtype=torch.float32)]:
         o = parity.oracle_chain(inp)
