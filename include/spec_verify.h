@@ -180,6 +180,25 @@ spec_status spec_verify_chain_filtered(int B, int gamma, int V,
                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * spec_verify_chain_filtered_lazy -- spec_verify_chain_filtered as a
+ * row-on-demand level walk (the lazy conventions below): per position the
+ * statistics and filter records of only the rows the still-active sequences
+ * reach (target row i, draft-logit row i; row gamma after a full acceptance),
+ * then one decision per active sequence; then the draw.  Same arguments,
+ * workspace size and outputs; rows never read are not validated and the
+ * diagnostics hold NaN where nothing was evaluated.
+ */
+spec_status spec_verify_chain_filtered_lazy(int B, int gamma, int V,
+                                       const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                       const void* draft, spec_dtype ddt, int draft_is_probs,
+                                       int64_t d_row_stride,
+                                       const int32_t* draft_tokens, const float* temperature,
+                                       const float* coins, const float* final_u,
+                                       const int32_t* top_k, const float* top_p,
+                                       int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * spec_verify_tree_greedy -- greedy verify of a draft token tree.
  * [origins] "In SGLang" (greedy goes through verify_tree_greedy) and
  * "Blockwise Parallel Decoding" (verify keeps the longest prefix equal to

@@ -14,6 +14,7 @@ from .spec_verify import (  # noqa: F401
     spec_read_device_status,
     spec_verify_chain,
     spec_verify_chain_filtered,
+    spec_verify_chain_filtered_lazy,
     spec_verify_chain_lazy,
     spec_verify_chain_vocab_parallel,
     spec_verify_tree_greedy,

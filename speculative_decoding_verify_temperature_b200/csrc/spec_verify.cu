@@ -2883,21 +2883,19 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
 // the records and the statistics) waits for them through this kernel.
 constexpr int WF_BT = 256;
 
-template <int TDT, int DDT, int DK, bool TREE, int BT>
-__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Params P) {
-    __shared__ FiltShared fs;
-    __shared__ WinShared ws;
+// The filter record of one row of sequence b (statistics row r, logits at
+// `row`, element type DT): invalid top_k / top_p give on = -1; filters off, a
+// bad temperature or an unusable row (the decision marks the sequence
+// invalid) give on = 0.  All threads of the CTA call it; thread 0 writes.
+template <int DT, int BT>
+__device__ void filter_one_row(const Params& P, int b, int r, const char* row, FiltShared& fs, WinShared& ws,
+                               unsigned char* dyn) {
     __shared__ float msh;
     __shared__ int bad;
-    extern __shared__ __align__(128) unsigned char dyn[];
-    pdl_trigger();
-    const int rows = TREE ? P.N : ((DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1);
-    const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
     FiltRec* out = P.filt + (size_t)b * P.R + r;
     const int K = P.top_k ? P.top_k[b] : 0;
     const float Pp = P.top_p ? P.top_p[b] : 1.f;
     const float T = P.temperature[b];
-    pdl_wait();
     if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
         return;
@@ -2906,10 +2904,6 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Para
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
-    const bool tgt = TREE || r <= P.gamma;
-    const char* row = TREE  ? P.tgt + ((size_t)b * P.N + r) * P.tstride
-                      : tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
-                            : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
     const int E = P.nch * SPC;
     if (threadIdx.x < 32) {
         float m;
@@ -2918,20 +2912,38 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Para
         if (threadIdx.x == 0) { msh = m; bad = bd; }
     }
     __syncthreads();
-    if (bad) {                                   // the decision marks the sequence invalid
+    const bool unusable = bad;
+    const float s = scale_of(T), m = msh;
+    __syncthreads();
+    if (unusable) {
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
-    const float s = scale_of(T), m = msh;
     FiltRec rec{-INFINITY, 0, 0.0};
-    if ((tgt ? TDT : DDT) == SPEC_BF16) {
-        rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
-    } else if constexpr (BT == FILT_BT) {
-        if (tgt) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
-        else rec = filter_row<DDT>(row, P.V, s, m, K, Pp, fs, FiltHist<DDT>{dyn});
-    }
+    if constexpr (DT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
+    else if constexpr (BT == FILT_BT) rec = filter_row<DT>(row, P.V, s, m, K, Pp, fs, FiltHist<DT>{dyn});
     if (threadIdx.x == 0) *out = rec;
 }
+
+template <int TDT, int DDT, int DK, bool TREE, int BT>
+__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Params P) {
+    __shared__ FiltShared fs;
+    __shared__ WinShared ws;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    pdl_trigger();
+    const int rows = TREE ? P.N : ((DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1);
+    const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
+    pdl_wait();
+    if (TREE || r <= P.gamma) {
+        const char* row = TREE ? P.tgt + ((size_t)b * P.N + r) * P.tstride
+                               : P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride;
+        filter_one_row<TDT, BT>(P, b, r, row, fs, ws, dyn);
+    } else {
+        filter_one_row<DDT, BT>(P, b, r, P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride, fs, ws,
+                                dyn);
+    }
+}
+
 
 // max(0, p' - q') of a filtered target row and a filtered draft row (QK =
 // DK_LOGITS), a draft probability row (DK_PROBS), or no draft (DK_NONE: p').
@@ -2980,6 +2992,41 @@ __device__ int draw_row(const WF& wf, int nch, float u, float* wpw, FinShared& s
 // statistics, threshold and kept mass), then the correction from
 // max(0, p'_k - q'_k) or the bonus from p'_gamma over the whole row.
 //
+// The last token of a filtered chain round for sequence b with k accepted:
+// the correction from max(0, p'_k - q'_k) or, for k = gamma (or an empty
+// residual), from p'_k, over the whole row (chunk masses, one chunk
+// rescanned), with sh.m / sh.z / sh.th holding rows k and gamma + 1 + k.
+// Writes out_tokens[b, k] and the S diagnostic.  All threads call it.
+template <int TDT, int DDT, int DK>
+__device__ void chain_filt_draw(const Params& P, int b, int k, float s, FinShared& sh, float* wpw) {
+    constexpr int CH = chunk_elems<TDT>();
+    constexpr int QDT = DK == DK_PROBS ? SPEC_F32 : DDT;
+    const int gamma = P.gamma, V = P.V;
+    const float u = P.final_u[b];
+    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
+    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]), thp = sh.th[k];
+    double S;
+    int y = -1;
+    if (k < gamma) {
+        const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
+        const int rq = gamma + 1 + k;
+        WFilt<TDT, QDT, DK> wf{trow, drow, s, mp, izp, thp, DK == DK_LOGITS ? sh.m[rq] : 0.f,
+                               DK == DK_LOGITS ? (float)(1.0 / sh.z[rq]) : 0.f,
+                               DK == DK_LOGITS ? sh.th[rq] : -INFINITY, V};
+        y = draw_row<CH, SEQ_BT>(wf, P.nch, u, wpw, sh, &S);
+    }
+    if (y < 0) {                                     // bonus, or an empty residual (rounding only)
+        WFilt<TDT, QDT, DK_NONE> wp{trow, nullptr, s, mp, izp, thp, 0.f, 0.f, -INFINITY, V};
+        double S0;
+        y = draw_row<CH, SEQ_BT>(wp, P.nch, u, wpw, sh, &S0);
+        if (k == gamma) S = 1.0;
+    }
+    if (threadIdx.x == 0) {
+        P.out_tokens[(size_t)b * (gamma + 1) + k] = y;
+        if (P.diag) P.diag[(size_t)b * (2 * gamma + 1) + 2 * gamma] = (float)S;
+    }
+}
+
 // OD (on demand: bf16 rows, no diagnostics): instead of reading every row's
 // filter record, the CTA filters the rows the decision reaches -- target row
 // i and draft row i for i = 0, 1, ... up to the first rejection, row gamma
@@ -3069,31 +3116,34 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
     }
     chain_decide<TDT, DDT, DK, true>(P, b, sh, true, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
-    const float s = (float)sh.dvals[0];
     if (!ok) return;
-    const float u = P.final_u[b];
-    const char* trow = P.tgt + ((size_t)b * (gamma + 1) + k) * P.tstride;
-    const float mp = sh.m[k], izp = (float)(1.0 / sh.z[k]), thp = sh.th[k];
-    double S;
-    int y = -1;
-    if (k < gamma) {
-        const char* drow = P.drf + ((size_t)b * gamma + k) * P.dstride;
-        const int rq = gamma + 1 + k;
-        WFilt<TDT, QDT, DK> wf{trow, drow, s, mp, izp, thp, DK == DK_LOGITS ? sh.m[rq] : 0.f,
-                               DK == DK_LOGITS ? (float)(1.0 / sh.z[rq]) : 0.f,
-                               DK == DK_LOGITS ? sh.th[rq] : -INFINITY, V};
-        y = draw_row<CH, SEQ_BT>(wf, P.nch, u, wpw, sh, &S);
+    chain_filt_draw<TDT, DDT, DK>(P, b, k, (float)sh.dvals[0], sh, wpw);
+}
+
+// Lazy filtered chain: the last token after the level walk, drawn as the
+// dense filtered finalisation draws it, from the filter records the walk
+// computed for the rows it reached.
+template <int TDT, int DDT, int DK>
+__global__ void __launch_bounds__(SEQ_BT) k_lz_chain_final_filt(const Params P) {
+    __shared__ FinShared sh;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    const int b = blockIdx.x, gamma = P.gamma;
+    pdl_wait();
+    chain_lazy_state(P, b, sh, true);
+    const int ok = sh.ivals[0], k = sh.ivals[1];
+    if (!ok) return;
+    if (threadIdx.x == 0) {
+        const FiltRec fp = P.filt[(size_t)b * P.R + k];
+        sh.th[k] = fp.theta;
+        if (fp.on > 0) sh.z[k] = fp.Z;
+        if (DK == DK_LOGITS && k < gamma) {
+            const FiltRec fq = P.filt[(size_t)b * P.R + gamma + 1 + k];
+            sh.th[gamma + 1 + k] = fq.theta;
+            if (fq.on > 0) sh.z[gamma + 1 + k] = fq.Z;
+        }
     }
-    if (y < 0) {                                     // bonus, or an empty residual (rounding only)
-        WFilt<TDT, QDT, DK_NONE> wp{trow, nullptr, s, mp, izp, thp, 0.f, 0.f, -INFINITY, V};
-        double S0;
-        y = draw_row<CH, SEQ_BT>(wp, P.nch, u, wpw, sh, &S0);
-        if (k == gamma) S = 1.0;
-    }
-    if (tid == 0) {
-        P.out_tokens[(size_t)b * (gamma + 1) + k] = y;
-        if (P.diag) P.diag[(size_t)b * (2 * gamma + 1) + 2 * gamma] = (float)S;
-    }
+    __syncthreads();
+    chain_filt_draw<TDT, DDT, DK>(P, b, k, (float)sh.dvals[0], sh, reinterpret_cast<float*>(dyn));
 }
 
 // ============================================================================= vocabulary-parallel chain verify
@@ -3540,7 +3590,7 @@ __global__ void __launch_bounds__(NT, STATS_CTAS_PER_SM) k_lz_stats(const Params
 // the sequence for the final kernel (residual at this position).  The
 // temperature is checked at level 0; a bad row or token marks the sequence
 // invalid.  Writes the p/q diagnostics of this position.
-template <int TDT, int DDT, int DK>
+template <int TDT, int DDT, int DK, bool FILT = false>
 __global__ void __launch_bounds__(NT) k_lz_decide_chain(const Params P) {
     pdl_trigger();
     pdl_wait();
@@ -3565,15 +3615,30 @@ __global__ void __launch_bounds__(NT) k_lz_decide_chain(const Params P) {
     if (lane != 0) return;
     const int x = P.draft_tokens[(size_t)b * gamma + level];
     ok &= (x >= 0 && x < P.V);
+    float th = -INFINITY, thq = -INFINITY;
+    if constexpr (FILT) {                       // the rows' filter records (this level's filter kernel)
+        const FiltRec fp = P.filt[(size_t)b * P.R + level];
+        ok &= fp.on >= 0;
+        th = fp.theta;
+        if (fp.on > 0) z = fp.Z;
+        if constexpr (DK == DK_LOGITS) {
+            const FiltRec fq = P.filt[(size_t)b * P.R + gamma + 1 + level];
+            ok &= fq.on >= 0;
+            thq = fq.theta;
+            if (fq.on > 0) zq = fq.Z;
+        }
+    }
     double p = 0.0, q = 0.0;
     if (ok) {
-        p = prob_d(ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, x, P.V), s, m, z);
+        const float l = ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, x, P.V);
+        p = (l >= th) ? prob_d(l, s, m, z) : 0.0;
         const char* drow = P.drf + ((size_t)b * gamma + level) * P.dstride;
         if constexpr (DK == DK_PROBS) {
             q = (double)__ldg(reinterpret_cast<const float*>(drow) + x);
             ok &= (q >= 0.0 && q <= 3.0e38);
         } else {
-            q = prob_d(ld_elem<DDT>(drow, x, P.V), s, mq, zq);
+            const float d = ld_elem<DDT>(drow, x, P.V);
+            q = (d >= thq) ? prob_d(d, s, mq, zq) : 0.0;
         }
     }
     LazySeq L;
@@ -3797,6 +3862,26 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_lz_filter_tree(co
     if constexpr (TDT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
     else if constexpr (BT == FILT_BT) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
     if (threadIdx.x == 0) *out = rec;
+}
+
+// Lazy filtered chain, one CTA per still-active sequence: the filter records
+// of target row `level` and, for draft logits below gamma, draft row `level`.
+template <int TDT, int DDT, int DK, int BT>
+__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_lz_filter_chain(const Params P) {
+    __shared__ FiltShared fs;
+    __shared__ WinShared ws;
+    extern __shared__ __align__(128) unsigned char dyn[];
+    pdl_trigger();
+    pdl_wait();
+    if ((int)blockIdx.x >= lz_count_of(P)) return;
+    const int b = lz_seq_of(P, blockIdx.x);
+    const int level = P.level, gamma = P.gamma;
+    filter_one_row<TDT, BT>(P, b, level, P.tgt + ((size_t)b * (gamma + 1) + level) * P.tstride, fs, ws, dyn);
+    if (DK == DK_LOGITS && level < gamma) {
+        __syncthreads();
+        filter_one_row<DDT, BT>(P, b, gamma + 1 + level, P.drf + ((size_t)b * gamma + level) * P.dstride, fs, ws,
+                                dyn);
+    }
 }
 
 // Lazy multi-step sampling walk, one CTA per active sequence at this level:
@@ -4342,6 +4427,44 @@ spec_status launch_chain_lazy(Params P, cudaStream_t st) {
     return s;
 }
 
+// Lazy filtered chain: per level the statistics of the rows the still-active
+// sequences reach, their filter records, the decisions; then the draw.
+template <int TDT, int DDT, int DK>
+spec_status launch_chain_filtered_lazy(Params P, cudaStream_t st) {
+    auto ks = k_lz_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>;
+    auto kd = k_lz_decide_chain<TDT, DDT, DK, true>;
+    constexpr bool all_bf16 = TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16);
+    constexpr int fbt = all_bf16 ? WF_BT : FILT_BT;
+    constexpr size_t hist = all_bf16 ? WF_BYTES
+                                     : (filt_hist_bytes<SPEC_F32>() > WF_BYTES ? filt_hist_bytes<SPEC_F32>() : WF_BYTES);
+    auto kf = k_lz_filter_chain<TDT, DDT, DK, fbt>;
+    static PerDevice<bool> attr_c;
+    const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
+    if (!attr) return fail(SPEC_ERR_CUDA, "k_lz_filter_chain shared memory attribute");
+    static PerDevice<int> occ_c;
+    const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
+    const int rpl = P.R > P.rows_tgt ? 2 : 1;
+    const unsigned sgrid = stats_grid((long long)P.B * rpl * P.nch, occ);
+    const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
+    if (g_prof_start && record(g_prof_start, st) != cudaSuccess) return fail(SPEC_ERR_CUDA, "profile event");
+    for (int level = 0; level <= P.gamma; ++level) {
+        spec_status s = launch_level(ks, sgrid, (void (*)(Params))nullptr, 0, P, level, st);
+        if (s != SPEC_OK) return s;
+        s = launch_dependent(kf, (unsigned)P.B, fbt, hist, P, st, "k_lz_filter_chain");
+        if (s != SPEC_OK) return s;
+        if (level < P.gamma) {
+            s = launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
+            if (s != SPEC_OK) return s;
+        }
+    }
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    spec_status s = launch_dependent(k_lz_chain_final_filt<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, wpw, P, st,
+                                     "k_lz_chain_final_filt");
+    if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
+        return fail(SPEC_ERR_CUDA, "profile event");
+    return s;
+}
+
 template <int TDT>
 spec_status launch_mss_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
@@ -4548,8 +4671,10 @@ static spec_status chain_entry(int mode, int B, int gamma, int V,
     // that draft rows keep their offsets for either draft kind.
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 #define SPEC_CHAIN(T, D, K)                                                                          \
-    return mode == 1 ? launch_chain_lazy<T, D, K>(P, st)                                             \
-                     : (mode == 2 ? launch_chain_filtered<T, D, K>(P, st) : launch_chain<T, D, K>(P, st))
+    return mode == 1   ? launch_chain_lazy<T, D, K>(P, st)                                           \
+           : mode == 2 ? launch_chain_filtered<T, D, K>(P, st)                                       \
+           : mode == 3 ? launch_chain_filtered_lazy<T, D, K>(P, st)                                  \
+                       : launch_chain<T, D, K>(P, st)
     if (draft_is_probs) {
         if (tdt == SPEC_BF16) SPEC_CHAIN(SPEC_BF16, SPEC_F32, DK_PROBS);
         SPEC_CHAIN(SPEC_F32, SPEC_F32, DK_PROBS);
@@ -4746,6 +4871,22 @@ spec_status spec_verify_chain_filtered(int B, int gamma, int V,
                        d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens, out_num_accepted,
                        diag, workspace, workspace_bytes, stream, top_k, top_p);
 }
+spec_status spec_verify_chain_filtered_lazy(int B, int gamma, int V,
+                                            const void* target_logits, spec_dtype tdt, int64_t t_row_stride,
+                                            const void* draft, spec_dtype ddt, int draft_is_probs,
+                                            int64_t d_row_stride,
+                                            const int32_t* draft_tokens, const float* temperature,
+                                            const float* coins, const float* final_u,
+                                            const int32_t* top_k, const float* top_p,
+                                            int32_t* out_tokens, int32_t* out_num_accepted, float* diag,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+    NvtxRange nvtx("spec_verify_chain_filtered_lazy");
+    if (!top_k && !top_p) return fail(SPEC_ERR_INVALID_ARG, "top_k and top_p are both NULL");
+    return chain_entry(3, B, gamma, V, target_logits, tdt, t_row_stride, draft, ddt, draft_is_probs,
+                       d_row_stride, draft_tokens, temperature, coins, final_u, out_tokens, out_num_accepted,
+                       diag, workspace, workspace_bytes, stream, top_k, top_p);
+}
+
 spec_status spec_verify_tree_greedy(SPEC_GREEDY_ARGS_DECL) {
     NvtxRange nvtx("spec_verify_tree_greedy");
     return greedy_entry(false, SPEC_GREEDY_ARGS);

@@ -66,9 +66,10 @@ def lib():
             f.restype = i32
             f.argtypes = [i32, i32, i32, i32, P, i32, i64, P, P, P, P, P, P, i64,
                           f32, f32, P, P, P, P, P, P, P, sz, P]
-        L.spec_verify_chain_filtered.restype = i32
-        L.spec_verify_chain_filtered.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64,
-                                                 P, P, P, P, P, P, P, P, P, P, sz, P]
+        for name in ("spec_verify_chain_filtered", "spec_verify_chain_filtered_lazy"):
+            f = getattr(L, name)
+            f.restype = i32
+            f.argtypes = [i32, i32, i32, P, i32, i64, P, i32, i32, i64, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.spec_vp_record_bytes.restype = sz
         L.spec_vp_record_bytes.argtypes = []
         L.spec_vp_chain_stats.restype = i32
@@ -396,7 +397,8 @@ def spec_verify_tree_mss_lazy(*args, **kw):
 
 def spec_verify_chain_filtered(target, draft, draft_tokens, temperature, coins, final_u, top_k=None, top_p=None, *,
                                draft_is_probs: bool = False, V: int | None = None, out_tokens=None,
-                               out_num_accepted=None, diag=None, workspace=None, stream=None):
+                               out_num_accepted=None, diag=None, workspace=None, stream=None,
+                               _name: str = "spec_verify_chain_filtered"):
     """Chain verify under top-k / top-p filtered temperature sampling; ``top_k`` int32
     ``[B]`` (0 = off) and ``top_p`` f32 ``[B]`` (1 = off), either may be None (not
     both).  Returns ``(out_tokens [B, gamma+1], out_num_accepted [B])``."""
@@ -415,13 +417,20 @@ def spec_verify_chain_filtered(target, draft, draft_tokens, temperature, coins, 
     if top_p is not None and top_p.dtype != torch.float32:
         raise TypeError("top_p must be float32")
     ws = _ws(workspace, SPEC_ENTRY_CHAIN, B, gamma, V, dev, stream)
-    st = lib().spec_verify_chain_filtered(
+    st = getattr(lib(), _name)(
         B, gamma, V, _p(target), _dtype(target), _rows(target, "target"),
         _p(draft), SPEC_F32 if draft_is_probs else _dtype(draft), int(bool(draft_is_probs)),
         _rows(draft, "draft"), _p(draft_tokens), _p(temperature), _p(coins), _p(final_u), _p(top_k), _p(top_p),
         _p(out_tokens), _p(out_num_accepted), _p(diag), _p(ws), ws.numel(), _stream(stream))
-    _check(st, "spec_verify_chain_filtered")
+    _check(st, _name)
     return out_tokens, out_num_accepted
+
+
+def spec_verify_chain_filtered_lazy(*args, **kw):
+    """spec_verify_chain_filtered as a row-on-demand level walk: only the rows the
+    decisions reach get statistics and filter records; same outputs for valid
+    inputs (diagnostics only where evaluated)."""
+    return spec_verify_chain_filtered(*args, _name="spec_verify_chain_filtered_lazy", **kw)
 
 
 

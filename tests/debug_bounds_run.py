@@ -33,8 +33,10 @@ def main():
     inp = wl.chain_inputs(6, 3, 5000, seed=4, device="cuda", zipf=True)
     tk = torch.tensor([0, 20, 50, 0, 20, 50], dtype=torch.int32, device="cuda")
     tp = torch.tensor([0.9, 1.0, 0.95, 0.9, 1.0, 0.95], dtype=torch.float32, device="cuda")
-    bad += parity.compare_chain(parity.gpu_chain_filtered(inp, tk, tp), parity.oracle_chain_filtered(inp, tk, tp),
-                                inp.gamma)[1]
+    d = parity.gpu_chain_filtered(inp, tk, tp)
+    bad += parity.compare_chain(d, parity.oracle_chain_filtered(inp, tk, tp), inp.gamma)[1]
+    z = parity.gpu_chain_filtered(inp, tk, tp, lazy=True)
+    bad += int((z["tokens"] != d["tokens"]).any(axis=1).sum())
     # trees: greedy, target-only sampling (dense and lazy, filtered), multi-step sampling
     inp = wl.tree_greedy_inputs(4, 3000, seed=5, device="cuda")
     bad += parity.compare_tree(parity.gpu_greedy(inp), parity.oracle_greedy(inp))[1]

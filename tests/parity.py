@@ -76,13 +76,13 @@ def oracle_chain_filtered(inp, top_k, top_p, rows=None, nthreads=0):
                         top_k=tk, top_p=tp)
 
 
-def gpu_chain_filtered(inp, top_k, top_p, workspace=None, with_diag=True):
-    from speculative_decoding_verify_temperature_b200 import spec_verify as sv
+def gpu_chain_filtered(inp, top_k, top_p, workspace=None, with_diag=True, lazy=False):
     B, g = inp.B, inp.gamma
     diag = torch.full((B, 2 * g + 1), float("nan"), device=inp.target.device) if with_diag else None
-    toks, na = sv.spec_verify_chain_filtered(inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins,
-                                             inp.final_u, top_k, top_p, draft_is_probs=inp.draft_is_probs,
-                                             V=inp.V, diag=diag, workspace=workspace)
+    toks, na = _fn("spec_verify_chain_filtered", lazy)(inp.target, inp.draft, inp.draft_tokens, inp.temperature,
+                                                       inp.coins, inp.final_u, top_k, top_p,
+                                                       draft_is_probs=inp.draft_is_probs, V=inp.V, diag=diag,
+                                                       workspace=workspace)
     torch.cuda.synchronize()
     d = diag.cpu().numpy().astype(np.float64) if with_diag else np.full((B, 2 * g + 1), np.nan)
     return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy(),
@@ -257,7 +257,7 @@ def gpu_chain_runner(target, draft, draft_is_probs, draft_tokens, temperature, c
         from speculative_decoding_verify_temperature_b200 import spec_verify as sv
         tk = None if top_k is None else t(np.asarray(top_k, np.int32).reshape(B))
         tp = None if top_p is None else t(np.asarray(top_p, np.float32).reshape(B))
-        toks, na = sv.spec_verify_chain_filtered(*args, tk, tp, draft_is_probs=draft_is_probs, V=V)
+        toks, na = _fn("spec_verify_chain_filtered", lazy)(*args, tk, tp, draft_is_probs=draft_is_probs, V=V)
     else:
         toks, na = spec_verify_chain(*args, draft_is_probs=draft_is_probs, V=V)
     return dict(tokens=toks.cpu().numpy(), num_accepted=na.cpu().numpy())

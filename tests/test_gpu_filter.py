@@ -1,5 +1,7 @@
 """GPU parity of spec_verify_chain_filtered (chain verify under top-k / top-p
 filtered temperature sampling) against the fp64 oracle, through the C ABI."""
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -33,6 +35,19 @@ def _check(inp, tk, tp, rows=None, max_flag_frac=0.2):
     d = parity.gpu_chain_filtered(inp, tk, tp, with_diag=False)
     np.testing.assert_array_equal(d["num_accepted"], g["num_accepted"])
     np.testing.assert_array_equal(d["tokens"], g["tokens"])
+    # the row-on-demand walk: the same records for the rows it reaches, the
+    # same outputs; diagnostics where it evaluated them, NaN after
+    z = parity.gpu_chain_filtered(inp, tk, tp, lazy=True)
+    np.testing.assert_array_equal(z["num_accepted"], g["num_accepted"])
+    np.testing.assert_array_equal(z["tokens"], g["tokens"])
+    for b, k in enumerate(g["num_accepted"]):
+        if k < 0:
+            continue
+        ev = min(k + 1, inp.gamma)
+        np.testing.assert_array_equal(z["px"][b, :ev], g["px"][b, :ev])
+        np.testing.assert_array_equal(z["qx"][b, :ev], g["qx"][b, :ev])
+        assert np.isnan(z["px"][b, ev:]).all()
+        assert z["S"][b] == g["S"][b]
     return g, o
 
 
@@ -91,11 +106,13 @@ def test_filtered_workload1_shape(cuda_device):
         _check(inp, tk, tp)
 
 
-def test_filtered_lossless_through_gpu(cuda_device):
+@pytest.mark.parametrize("lazy", [False, True])
+def test_filtered_lossless_through_gpu(lazy, cuda_device):
+    run = functools.partial(parity.gpu_chain_runner, lazy=lazy)
     for kw in [dict(), dict(V=4, gamma=2, seed=5, T=0.7, top_k=0, top_p=0.61),
                dict(V=3, gamma=3, K=3, seed=8, top_k=2, top_p=0.77),
                dict(draft_kind="probs", seed=2, top_k=2, top_p=0.9, tol=1e-7)]:
-        r = pins.chain_filtered_bruteforce(runner=parity.gpu_chain_runner, **kw)
+        r = pins.chain_filtered_bruteforce(runner=run, **kw)
         assert r["ok"], (kw, r)
 
 
@@ -112,6 +129,8 @@ def test_filtered_invalid_parameters(cuda_device):
     assert sv.spec_read_device_status(buf) & (1 << sv.SPEC_ERR_DEVICE_INPUT)
     o = parity.oracle_chain_filtered(inp, tk, tp)
     assert list(o["num_accepted"][1:5]) == [-1] * 4
+    z = parity.gpu_chain_filtered(inp, tk, tp, lazy=True)
+    assert list(z["num_accepted"][1:5]) == [-1] * 4 and z["num_accepted"][0] >= 0
     with pytest.raises(ValueError):
         sv.spec_verify_chain_filtered(inp.target, inp.draft, inp.draft_tokens, inp.temperature, inp.coins,
                                       inp.final_u)
