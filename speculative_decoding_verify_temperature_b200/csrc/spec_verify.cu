@@ -755,12 +755,14 @@ __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
 //     upper bound of the kept mass;
 //  3. a second pass counts, per key, only the elements of the non-empty
 //     buckets from the top down to that bucket (16 counters per non-empty
-//     bucket, in descending key order); every other element adds its fixed-
-//     point mass to an exact total (the kept mass when top-k is off).
-// Every key's mass is then count * fixed(2^(v s - m)), as in a full value
-// histogram, so the running counts and masses from the top, the top-k key,
-// the kept mass and the top-p key are the same integers.  A window needing
-// more than WF_SLOTS counters is counted in segments, one more pass each.
+//     bucket, in descending key order).
+// Every key's mass is count * fixed(2^(v s - m)), so the running counts and
+// masses from the top, the top-k key and the kept mass are exact integers,
+// independent of the order of the additions.  With top-k off the mass the
+// top-p share is taken of is the whole row's, zrow (the row statistics' sum,
+// fp64 across chunks, relative error ~2e-7): top-p decisions that close to a
+// boundary are the near-ties the oracle flags.  A window needing more than
+// WF_SLOTS counters is counted in segments, one more pass each.
 constexpr int WF_NB = 4096;                       // coarse buckets (key >> 4)
 constexpr int WF_SLOTS = 8192;                    // per-key counters of the window
 constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 56 KB
@@ -897,8 +899,8 @@ __device__ __forceinline__ void wf_each_key(const char* row, int V, F f) {
 // Threshold and kept mass of one bf16 row (the record filter_row gives).
 // smem: WF_BYTES of shared memory.  All threads call it.
 template <int BT>
-__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, float Pp, unsigned char* smem,
-                               WinShared& ws) {
+__device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp,
+                               unsigned char* smem, WinShared& ws) {
     constexpr int RB = WF_NB / BT;                    // coarse buckets per thread (descending positions)
     constexpr int RS = WF_SLOTS / BT;                 // window counters per thread
     static_assert(RB * BT == WF_NB && RS * BT == WF_SLOTS, "split");
@@ -934,7 +936,8 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, 
     unsigned c0, ctot;
     double l0, h0, ltot, htot;
     wf_scan3<BT>(rc, rl, rh, &c0, &l0, &h0, &ctot, &ltot, &htot, ws);
-    if (tid == 0) { ws.pos_k = -1; ws.pos_p = WF_NB - 1; ws.dv = htot; }
+    const double zfix = zrow * FIX_ONE;                 // the row's mass in fixed-point units
+    if (tid == 0) { ws.pos_k = -1; ws.pos_p = WF_NB - 1; ws.dv = zfix; }
     __syncthreads();
     if (use_k && c0 < (unsigned)K && c0 + rc >= (unsigned)K) {     // the top-k bucket (exact counts)
         unsigned c = c0;
@@ -995,30 +998,23 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, 
     bool rk = !use_k, rp = !use_p;
     uint32_t tk = 0x007Fu, tp = 0x007Fu;             // -inf: keep everything (never left so)
     unsigned cb = 0u;                                  // count of the keys above this segment
-    unsigned long long mb = 0ull, zk = 0ull, z = 0ull, total = 0ull;
+    unsigned long long mb = 0ull, zk = 0ull, z = 0ull;
+    if (!use_k) zk = (unsigned long long)zfix;
     for (int seg = 0; seg * WF_SLOTS < max(nslot, 1) && !(rk && rp); ++seg) {
-        const int slo = seg * WF_SLOTS;
-        for (int i = tid; i < WF_SLOTS / 4; i += BT) reinterpret_cast<uint4*>(slots)[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (tid == 0) ws.acc = 0ull;
+        const int slo = seg * WF_SLOTS, used = min(WF_SLOTS, nslot - slo);
+        for (int i = tid; i < (used + 3) / 4; i += BT) reinterpret_cast<uint4*>(slots)[i] = make_uint4(0u, 0u, 0u, 0u);
         __syncthreads();
-        unsigned long long other = 0ull;               // fixed-point mass of the elements outside this segment
         wf_each_key<BT>(row, V, [&](uint32_t k) {
             const unsigned short o = ord_of[k >> 4];
             const int sl = (int)o * 16 + (15 - (int)(k & 15u)) - slo;
             if (o != WF_NONE && sl >= 0 && sl < WF_SLOTS) atomicAdd(&slots[sl], 1u);
-            else if (seg == 0 && !use_k) other += fix_mass(key_value<SPEC_BF16>(k), s, m);
         });
-        if (seg == 0 && !use_k) {
-#pragma unroll
-            for (int o = 16; o; o >>= 1) other += __shfl_xor_sync(FULL, other, o);
-            if ((tid & 31) == 0) atomicAdd(&ws.acc, other);
-        }
         __syncthreads();
         // this segment's keys in descending order: thread runs of RS counters
         const int s0 = tid * RS;
         unsigned sc = 0u;
         unsigned long long sm = 0ull;
-        for (int j = 0; j < RS; ++j) {
+        for (int j = 0; j < RS && s0 + j < used; ++j) {
             const unsigned c = slots[s0 + j];
             if (c) {
                 const int g = slo + s0 + j;
@@ -1032,7 +1028,6 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, 
         wf_scan2<BT>(sc, sm, &e0, &f0, &etot, &ftot, ws);
         e0 += cb;
         f0 += mb;
-        if (seg == 0 && !use_k) { total = ws.acc + ftot; zk = total; }
         auto find = [&](bool by_count, double target) {   // the thread whose run crosses the target
             if (tid == 0) ws.sel = -1;
             __syncthreads();
@@ -1041,7 +1036,7 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, int K, 
             if (cross) {
                 unsigned c = e0;
                 unsigned long long mm = f0;
-                for (int j = 0; j < RS; ++j) {
+                for (int j = 0; j < RS && s0 + j < used; ++j) {
                     const unsigned cj = slots[s0 + j];
                     if (!cj) continue;
                     const int g = slo + s0 + j;
@@ -2121,7 +2116,7 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         if (tid == 0) ai[0] = 0;
         for (;;) {
             const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
-            const FiltRec f = wfilter_row<BT>(row, V, s, sh.m[cur], K, Pp, win, *ws);
+            const FiltRec f = wfilter_row<BT>(row, V, s, sh.m[cur], sh.z[cur], K, Pp, win, *ws);
             thc = f.theta;
             zc = f.on > 0 ? f.Z : sh.z[cur];
             for (int n = cur + 1 + tid; n < N; n += BT)
@@ -2891,6 +2886,7 @@ template <int DT, int BT>
 __device__ void filter_one_row(const Params& P, int b, int r, const char* row, FiltShared& fs, WinShared& ws,
                                unsigned char* dyn) {
     __shared__ float msh;
+    __shared__ double zsh_;
     __shared__ int bad;
     FiltRec* out = P.filt + (size_t)b * P.R + r;
     const int K = P.top_k ? P.top_k[b] : 0;
@@ -2909,18 +2905,19 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
         float m;
         double z;
         const bool bd = warp_combine(P.stats + ((size_t)b * P.R + r) * E, E, m, z);
-        if (threadIdx.x == 0) { msh = m; bad = bd; }
+        if (threadIdx.x == 0) { msh = m; zsh_ = z; bad = bd; }
     }
     __syncthreads();
     const bool unusable = bad;
     const float s = scale_of(T), m = msh;
+    const double zsh = zsh_;
     __syncthreads();
     if (unusable) {
         if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
         return;
     }
     FiltRec rec{-INFINITY, 0, 0.0};
-    if constexpr (DT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
+    if constexpr (DT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, zsh, K, Pp, dyn, ws);
     else if constexpr (BT == FILT_BT) rec = filter_row<DT>(row, P.V, s, m, K, Pp, fs, FiltHist<DT>{dyn});
     if (threadIdx.x == 0) *out = rec;
 }
@@ -3080,7 +3077,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
                 const int r = half ? gamma + 1 + i : i;
                 const char* row = half ? P.drf + ((size_t)b * gamma + i) * P.dstride
                                        : P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride;
-                const FiltRec f = wfilter_row<SEQ_BT>(row, V, s, sh.m[r], K, Pp, win, ws);
+                const FiltRec f = wfilter_row<SEQ_BT>(row, V, s, sh.m[r], sh.z[r], K, Pp, win, ws);
                 if (tid == 0) {
                     sh.th[r] = f.theta;
                     if (f.on > 0) sh.z[r] = f.Z;
@@ -3824,44 +3821,13 @@ template <int TDT, int BT>
 __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_lz_filter_tree(const Params P) {
     __shared__ FiltShared fs;
     __shared__ WinShared ws;
-    __shared__ float msh;
-    __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
     pdl_trigger();
     pdl_wait();
     if ((int)blockIdx.x >= lz_count_of(P)) return;
     const int b = lz_seq_of(P, blockIdx.x);
     const int cur = P.level == 0 ? 0 : P.lz_seq[b].cur;
-    FiltRec* out = P.filt + (size_t)b * P.R + cur;
-    const int K = P.top_k ? P.top_k[b] : 0;
-    const float Pp = P.top_p ? P.top_p[b] : 1.f;
-    const float T = P.temperature[b];
-    if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
-        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
-        return;
-    }
-    if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
-        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
-        return;
-    }
-    const int E = P.nch * SPC;
-    if (threadIdx.x < 32) {
-        float m;
-        double z;
-        const bool bd = warp_combine(P.stats + ((size_t)b * P.R + cur) * E, E, m, z);
-        if (threadIdx.x == 0) { msh = m; bad = bd; }
-    }
-    __syncthreads();
-    if (bad) {                                   // the decision marks the sequence invalid
-        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
-        return;
-    }
-    const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
-    const float s = scale_of(T), m = msh;
-    FiltRec rec{-INFINITY, 0, 0.0};
-    if constexpr (TDT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, K, Pp, dyn, ws);
-    else if constexpr (BT == FILT_BT) rec = filter_row<TDT>(row, P.V, s, m, K, Pp, fs, FiltHist<TDT>{dyn});
-    if (threadIdx.x == 0) *out = rec;
+    filter_one_row<TDT, BT>(P, b, cur, P.tgt + ((size_t)b * P.N + cur) * P.tstride, fs, ws, dyn);
 }
 
 // Lazy filtered chain, one CTA per still-active sequence: the filter records
