@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <limits.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -766,7 +767,6 @@ __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
 constexpr int WF_NB = 4096;                       // coarse buckets (key >> 4)
 constexpr int WF_SLOTS = 8192;                    // per-key counters of the window
 constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 56 KB
-constexpr unsigned short WF_NONE = 0xFFFFu;
 
 struct WinShared {
     unsigned long long red[32];
@@ -886,11 +886,20 @@ __device__ __forceinline__ void wf_each_key(const char* row, int V, F f) {
             if (vi >= nv) break;
             const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
             const int lim = V - vi * 8;
+            if (lim >= 8) {                               // a whole vector inside the row
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t k2 = vh_keys2(xs[c]);
-                if (2 * c < lim) f(k2 & 0xFFFFu);
-                if (2 * c + 1 < lim) f(k2 >> 16);
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t k2 = vh_keys2(xs[c]);
+                    f(k2 & 0xFFFFu);
+                    f(k2 >> 16);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t k2 = vh_keys2(xs[c]);
+                    if (2 * c < lim) f(k2 & 0xFFFFu);
+                    if (2 * c + 1 < lim) f(k2 >> 16);
+                }
             }
         }
     }
@@ -909,8 +918,9 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
     const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
     if (!use_k && !use_p) return r;
     uint32_t* coarse = reinterpret_cast<uint32_t*>(smem);                        // pass 1 counts
-    unsigned short* bucket_of = reinterpret_cast<unsigned short*>(smem);         // ordinal -> bucket (reuses coarse)
-    unsigned short* ord_of = reinterpret_cast<unsigned short*>(smem + (size_t)WF_NB * 4);   // bucket -> ordinal
+    int32_t* sbase = reinterpret_cast<int32_t*>(smem);                           // bucket -> its keys' first counter
+                                                                                 // + 15 (reuses coarse)
+    unsigned short* bucket_of = reinterpret_cast<unsigned short*>(smem + (size_t)WF_NB * 4);  // ordinal -> bucket
     uint32_t* slots = reinterpret_cast<uint32_t*>(smem + (size_t)WF_NB * 6);
     // ---- pass 1: coarse counts
     for (int i = tid; i < WF_NB / 4; i += BT) reinterpret_cast<uint4*>(coarse)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -984,11 +994,11 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
         for (int j = 0; j < RB; ++j) {
             const uint32_t b = (uint32_t)(WF_NB - 1 - (p0 + j));
             if (p0 + j < nb && cnt[j]) {
-                ord_of[b] = (unsigned short)o;
+                sbase[b] = (int32_t)(o * 16u + 15u);     // key k of b counts at sbase[b] - (k & 15)
                 bucket_of[o] = (unsigned short)b;
                 ++o;
             } else {
-                ord_of[b] = WF_NONE;
+                sbase[b] = INT_MIN / 2;                  // outside the window: never a valid counter
             }
         }
     }
@@ -1005,9 +1015,8 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
         for (int i = tid; i < (used + 3) / 4; i += BT) reinterpret_cast<uint4*>(slots)[i] = make_uint4(0u, 0u, 0u, 0u);
         __syncthreads();
         wf_each_key<BT>(row, V, [&](uint32_t k) {
-            const unsigned short o = ord_of[k >> 4];
-            const int sl = (int)o * 16 + (15 - (int)(k & 15u)) - slo;
-            if (o != WF_NONE && sl >= 0 && sl < WF_SLOTS) atomicAdd(&slots[sl], 1u);
+            const int sl = sbase[k >> 4] - (int)(k & 15u) - slo;
+            if ((unsigned)sl < (unsigned)used) atomicAdd(&slots[sl], 1u);
         });
         __syncthreads();
         // this segment's keys in descending order: thread runs of RS counters
