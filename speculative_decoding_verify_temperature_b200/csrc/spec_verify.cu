@@ -662,6 +662,15 @@ __device__ int filt_scan(const T* w, int nb, int dlo, unsigned long long base, d
     return d;
 }
 
+// The mass the top-p share is taken of, in fixed-point units: the kept mass
+// of top-k (exact), or with top-k off the row's mass from its statistics
+// (zrow, fp64 across chunks, ~2e-7 relative) -- with top_p capped below
+// 1 - 2^-20 so that the target stays under the exact total; both differences
+// lie inside the oracle's 1e-6 flag on top-p decisions.
+__device__ __forceinline__ double top_p_target(bool use_k, float Pp, unsigned long long zk, double zrow) {
+    return use_k ? (double)Pp * (double)zk : fmin((double)Pp, 1.0 - 9.5367431640625e-07) * zrow * FIX_ONE;
+}
+
 // Threshold and kept mass of one row (one CTA).
 //  top-k: walk the digits of the top_k-th largest key (filt_scan over the
 //    counts, one pass per digit); every pass keeps the masses, so the mass of
@@ -675,7 +684,7 @@ __device__ int filt_scan(const T* w, int nb, int dlo, unsigned long long base, d
 //  top-p alone: one pass of the first digit over every key; the crossing
 //    bucket is refined the same way.
 template <int DT>
-__device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, float Pp, FiltShared& fs,
+__device__ FiltRec filter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp, FiltShared& fs,
                               const FiltHist<DT>& h) {
     using D = FiltDigits<DT>;
     constexpr int NL = D::NL;
@@ -703,7 +712,7 @@ __device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, f
     uint32_t key = prefix;
     unsigned long long z = mk;
     if (use_p) {
-        const double target = (double)Pp * (double)mk;
+        const double target = top_p_target(use_k, Pp, mk, zrow);
         unsigned long long base = 0ull;
         int cl = -1, cd = 0;
         for (int l = 0; l < nl && cl < 0; ++l) {                // buckets strictly above the path digit
@@ -743,6 +752,216 @@ __device__ FiltRec filter_row(const char* row, int V, float s, float m, int K, f
 __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
     x &= ~__vcmpeq2(x, 0x80008000u);
     return x ^ ((((x >> 15) & 0x00010001u) * 0xFFFFu) | 0x80008000u);
+}
+
+
+// bf16 rows: an exact histogram of the row's values (65536 order keys, two
+// 16-bit counters per 32-bit word, 128 KB of shared memory) from one pass;
+// every mass then follows exactly as count * fixed(2^(v s - m)) per value,
+// the same fixed-point numbers the radix path adds element by element.
+// (The windowed filter below forms the same numbers in 56 KB for callers
+// that cannot hold 192 KB.)
+//
+// A row has at most V distinct values, so most of the 32768 words are empty.
+// Thread t reads the 32 words of key block 1023 - t (16-byte loads, the four
+// quads of a block stored XOR-swizzled by the block index so that eight
+// consecutive threads hit eight distinct bank groups), and a block-wide scan
+// packs the indices of the non-empty words into a list in descending key
+// order.  The counts and masses are then summed over equal slices of that
+// list, so the exp2 work is spread evenly whatever the values' spread, and
+// one more scan orders the slices: the top-k key is where the running count
+// reaches top_k, the top-p key where the running mass reaches top_p times the
+// mass kept by top-k.
+constexpr int VH_WORDS = 32768;
+constexpr size_t VH_BYTES = (size_t)VH_WORDS * 4 + (size_t)VH_WORDS * 2;   // counters + word list
+
+// Physical word of logical word i (= key >> 1): block i >> 5, quad
+// ((i >> 2) & 7) ^ (block & 7), lane i & 3.
+__device__ __forceinline__ uint32_t vh_phys(uint32_t i) { return i ^ ((i >> 3) & 0x1Cu); }
+
+__device__ __forceinline__ void vh_count1(uint32_t* w, uint32_t k) {
+    atomicAdd(&w[vh_phys(k >> 1)], (k & 1u) ? 0x10000u : 1u);
+}
+__device__ __forceinline__ unsigned long long vh_mass(unsigned c, uint32_t k, float s, float m) {
+    if (c == 0u) return 0ull;
+    return (unsigned long long)c *
+           (unsigned long long)(ex2(fmaf(key_value<SPEC_BF16>(k), s, -m)) * (float)FIX_ONE);
+}
+
+// Exclusive block-wide scan, in thread order, of a u32 and a u64; the totals
+// go to *ta / *tb.  All threads call it.
+__device__ void vh_scan2(unsigned a, unsigned long long b, unsigned* ea, unsigned long long* eb, unsigned* ta,
+                         unsigned long long* tb, FiltShared& fs) {
+    static_assert(FILT_BT == 1024, "one warp scans the 32 warp totals");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned ia = a;
+    unsigned long long ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned va = __shfl_up_sync(FULL, ia, o);
+        const unsigned long long vb = __shfl_up_sync(FULL, ib, o);
+        if (lane >= o) { ia += va; ib += vb; }
+    }
+    if (lane == 31) { fs.redc[warp] = ia; fs.red[warp] = ib; }
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned xa = fs.redc[lane];
+        const unsigned long long xb = fs.red[lane];
+        unsigned sa = xa;
+        unsigned long long sb = xb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned va = __shfl_up_sync(FULL, sa, o);
+            const unsigned long long vb = __shfl_up_sync(FULL, sb, o);
+            if (lane >= o) { sa += va; sb += vb; }
+        }
+        fs.redc[lane] = sa - xa;
+        fs.red[lane] = sb - xb;
+        if (lane == 31) { fs.tc = sa; fs.tm = sb; }
+    }
+    __syncthreads();
+    *ea = fs.redc[warp] + ia - a;
+    *eb = fs.red[warp] + ib - b;
+    *ta = fs.tc;
+    *tb = fs.tm;
+    __syncthreads();                                   // fs is free again
+}
+
+// The value histogram of a bf16 row and its list of non-empty words (from the
+// logits alone, before the statistics are needed).  Returns the list length.
+// All threads call it.
+__device__ int vh_build(const char* row, int V, FiltShared& fs, uint32_t* w) {
+    const int tid = threadIdx.x;
+    uint4* w4 = reinterpret_cast<uint4*>(w);
+    unsigned short* list = reinterpret_cast<unsigned short*>(w + VH_WORDS);
+    // histogram: four 16-byte loads per thread in flight (the first four
+    // while the counters are cleared), then the updates
+    const int nv = (V + 7) / 8;
+    uint4 v[4];
+    auto load4 = [&](int v0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * FILT_BT;
+            v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    load4(tid);
+    for (int i = tid; i < VH_WORDS / 4; i += FILT_BT) w4[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int v0 = tid;;) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int vi = v0 + q * FILT_BT;
+            if (vi >= nv) break;
+            const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            const int lim = V - vi * 8;                   // elements of this vector inside the row
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t k2 = vh_keys2(xs[c]);
+                if (2 * c < lim) vh_count1(w, k2 & 0xFFFFu);
+                if (2 * c + 1 < lim) vh_count1(w, k2 >> 16);
+            }
+        }
+        v0 += 4 * FILT_BT;
+        if (v0 >= nv) break;
+        load4(v0);
+    }
+    __syncthreads();
+    // non-empty words of this thread's block, highest first
+    const uint32_t blk = (uint32_t)(VH_WORDS / 32 - 1 - tid);
+    uint32_t mask = 0u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint4 x = w4[blk * 8 + (q ^ (blk & 7u))];
+        mask |= (x.x ? 1u : 0u) << (4 * q) | (x.y ? 1u : 0u) << (4 * q + 1) | (x.z ? 1u : 0u) << (4 * q + 2) |
+                (x.w ? 1u : 0u) << (4 * q + 3);
+    }
+    unsigned off, n;
+    unsigned long long d0, d1;
+    vh_scan2((unsigned)__popc(mask), 0ull, &off, &d0, &n, &d1, fs);
+    while (mask) {
+        const int j = 31 - __clz(mask);
+        list[off++] = (unsigned short)(blk * 32 + j);
+        mask &= ~(1u << j);
+    }
+    __syncthreads();
+    return (int)n;
+}
+
+// Threshold and kept mass of a bf16 row from its value histogram and word
+// list (vh_build).  Returns false when a value occurs 65536 times or more (a
+// 16-bit counter wrapped: possible only for V > 65535); the caller then takes
+// the radix path.  All threads call it.
+__device__ bool vh_select(int V, int n, float s, float m, double zrow, int K, float Pp, FiltShared& fs,
+                          const uint32_t* w, FiltRec* out) {
+    const int tid = threadIdx.x;
+    const unsigned short* list = reinterpret_cast<const unsigned short*>(w + VH_WORDS);
+    // counts and masses of this thread's slice of the list
+    const int e0 = (int)((long long)n * tid / FILT_BT), e1 = (int)((long long)n * (tid + 1) / FILT_BT);
+    unsigned cs = 0u;
+    unsigned long long ms = 0ull;
+    for (int e = e0; e < e1; ++e) {
+        const uint32_t i = list[e];
+        const uint32_t x = w[vh_phys(i)];
+        cs += (x >> 16) + (x & 0xFFFFu);
+        ms += vh_mass(x >> 16, 2 * i + 1, s, m) + vh_mass(x & 0xFFFFu, 2 * i, s, m);
+    }
+    unsigned c0, ctot;
+    unsigned long long m0, mtot;
+    vh_scan2(cs, ms, &c0, &m0, &ctot, &mtot, fs);
+    if (V > 65535 && ctot != (unsigned)V) return false;   // a counter wrapped (the same in every thread)
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    // top-k: the first key (from the top) where the running count reaches K
+    if (tid == 0) { fs.sel = 0; fs.at = mtot; }          // top-p alone: every key is kept
+    __syncthreads();
+    if (use_k && c0 < (unsigned)K && c0 + cs >= (unsigned)K) {
+        unsigned c = c0;
+        unsigned long long mm = m0;
+        for (int e = e0; e < e1; ++e) {
+            const uint32_t i = list[e];
+            const uint32_t x = w[vh_phys(i)];
+            const unsigned ch = x >> 16, cl = x & 0xFFFFu;
+            c += ch;
+            mm += vh_mass(ch, 2 * i + 1, s, m);
+            if (c >= (unsigned)K) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
+            c += cl;
+            mm += vh_mass(cl, 2 * i, s, m);
+            if (c >= (unsigned)K) { fs.sel = (int)(2 * i); fs.at = mm; break; }
+        }
+    }
+    __syncthreads();
+    uint32_t t = (uint32_t)fs.sel;
+    const unsigned long long zk = fs.at;
+    unsigned long long z = zk;
+    if (use_p) {
+        // the first key where the running mass reaches top_p of the kept mass
+        // (a key >= the top-k key, since the running mass there is zk); with
+        // top-k off the kept mass is the row's, as wfilter_row takes it
+        const double target = top_p_target(use_k, Pp, zk, zrow);
+        __syncthreads();
+        if (tid == 0) fs.sel = -1;
+        __syncthreads();
+        if ((double)m0 < target && (double)(m0 + ms) >= target) {
+            unsigned long long mm = m0;
+            for (int e = e0; e < e1; ++e) {
+                const uint32_t i = list[e];
+                const uint32_t x = w[vh_phys(i)];
+                mm += vh_mass(x >> 16, 2 * i + 1, s, m);
+                if ((double)mm >= target) { fs.sel = (int)(2 * i + 1); fs.at = mm; break; }
+                mm += vh_mass(x & 0xFFFFu, 2 * i, s, m);
+                if ((double)mm >= target) { fs.sel = (int)(2 * i); fs.at = mm; break; }
+            }
+        }
+        __syncthreads();
+        if (fs.sel >= 0) {
+            t = (uint32_t)fs.sel;
+            z = fs.at;
+        }
+    }
+    out->theta = key_value<SPEC_BF16>(t);
+    out->on = 1;
+    out->Z = (double)z / FIX_ONE;
+    return true;
 }
 
 // bf16 rows, two passes and a sparse window.
@@ -964,7 +1183,8 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
     }
     __syncthreads();
     const int pos_k = ws.pos_k;
-    const double target_hi = (double)Pp * ws.dv * HI;   // top_p of an upper bound of the kept mass
+    // top_p of an upper bound of the kept mass (only used with top-k off)
+    const double target_hi = top_p_target(false, Pp, 0ull, zrow) * HI;
     __syncthreads();
     if (use_p && l0 < target_hi && l0 + rl >= target_hi) {
         double l = l0;
@@ -1009,7 +1229,6 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
     uint32_t tk = 0x007Fu, tp = 0x007Fu;             // -inf: keep everything (never left so)
     unsigned cb = 0u;                                  // count of the keys above this segment
     unsigned long long mb = 0ull, zk = 0ull, z = 0ull;
-    if (!use_k) zk = (unsigned long long)zfix;
     for (int seg = 0; seg * WF_SLOTS < max(nslot, 1) && !(rk && rp); ++seg) {
         const int slo = seg * WF_SLOTS, used = min(WF_SLOTS, nslot - slo);
         for (int i = tid; i < (used + 3) / 4; i += BT) reinterpret_cast<uint4*>(slots)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -1069,7 +1288,7 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
             __syncthreads();
         }
         if (rk && !rp) {
-            const double target = (double)Pp * (double)zk;
+            const double target = top_p_target(use_k, Pp, zk, zrow);
             if ((double)(mb + ftot) >= target) {            // the top-p key lies in this segment
                 find(false, target);
                 tp = (uint32_t)ws.sel;
@@ -2877,20 +3096,21 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
 
-// Filter thresholds of every row of a chain round, one CTA per (sequence,
-// row): target rows 0..gamma, then the draft-logit rows (TREE: the N node
-// rows of every tree).  bf16 rows take the windowed histogram (wfilter_row),
-// f32 rows the radix descent (filter_row, which needs FILT_BT threads); a
-// launch whose rows are all bf16 runs WF_BT threads per CTA and 32 KB of
-// shared memory, so several rows share an SM.  Every CTA waits for the
-// statistics before it exits, so the finalize kernel that follows (and reads
-// the records and the statistics) waits for them through this kernel.
-constexpr int WF_BT = 256;
+// Filter thresholds of every row of a chain round, one CTA of FILT_BT threads
+// per (sequence, row): target rows 0..gamma, then the draft-logit rows (TREE:
+// the N node rows of every tree).  bf16 rows take the value histogram
+// (vh_build / vh_select), f32 rows the radix descent (filter_row).  Every CTA
+// waits for the statistics before it exits, so the finalize kernel that
+// follows (and reads the records and the statistics) waits for them through
+// this kernel.
 
 // The filter record of one row of sequence b (statistics row r, logits at
 // `row`, element type DT): invalid top_k / top_p give on = -1; filters off, a
 // bad temperature or an unusable row (the decision marks the sequence
-// invalid) give on = 0.  All threads of the CTA call it; thread 0 writes.
+// invalid) give on = 0.  FILT_BT threads: the value histogram (bf16; the
+// radix descent when a counter wraps) or the radix descent (f32); other
+// block sizes (bf16 rows only): the windowed histogram.  All threads of the
+// CTA call it; thread 0 writes.
 template <int DT, int BT>
 __device__ void filter_one_row(const Params& P, int b, int r, const char* row, FiltShared& fs, WinShared& ws,
                                unsigned char* dyn) {
@@ -2926,8 +3146,13 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
         return;
     }
     FiltRec rec{-INFINITY, 0, 0.0};
-    if constexpr (DT == SPEC_BF16) rec = wfilter_row<BT>(row, P.V, s, m, zsh, K, Pp, dyn, ws);
-    else if constexpr (BT == FILT_BT) rec = filter_row<DT>(row, P.V, s, m, K, Pp, fs, FiltHist<DT>{dyn});
+    if constexpr (BT == FILT_BT) {
+        uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
+        if (DT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, zsh, K, Pp, fs, w, &rec))
+            rec = filter_row<DT>(row, P.V, s, m, zsh, K, Pp, fs, FiltHist<DT>{dyn});
+    } else if constexpr (DT == SPEC_BF16) {
+        rec = wfilter_row<BT>(row, P.V, s, m, zsh, K, Pp, dyn, ws);
+    }
     if (threadIdx.x == 0) *out = rec;
 }
 
@@ -2993,11 +3218,6 @@ __device__ int draw_row(const WF& wf, int nch, float u, float* wpw, FinShared& s
     return *S > 0.0 ? draw_from_chunks<CH, BT>(wf, nch, wf.V, (double)u * *S, u, sh) : -1;
 }
 
-// Filtered chain finalisation, one CTA per sequence: the decision of
-// chain_decide on the filtered distributions (p' and q' from each row's
-// statistics, threshold and kept mass), then the correction from
-// max(0, p'_k - q'_k) or the bonus from p'_gamma over the whole row.
-//
 // The last token of a filtered chain round for sequence b with k accepted:
 // the correction from max(0, p'_k - q'_k) or, for k = gamma (or an empty
 // residual), from p'_k, over the whole row (chunk masses, one chunk
@@ -3033,93 +3253,29 @@ __device__ void chain_filt_draw(const Params& P, int b, int k, float s, FinShare
     }
 }
 
-// OD (on demand: bf16 rows, no diagnostics): instead of reading every row's
-// filter record, the CTA filters the rows the decision reaches -- target row
-// i and draft row i for i = 0, 1, ... up to the first rejection, row gamma
-// after a full acceptance -- with one window histogram each (win, after the
-// per-warp sums in dynamic shared memory).  The decision then takes the same
-// steps as with every record present: it never looks past the first
-// rejection.
-template <int TDT, int DDT, int DK, bool OD = false>
+// Filtered chain finalisation, one CTA per sequence: the decision of
+// chain_decide on the filtered distributions (p' and q' from each row's
+// statistics, threshold and kept mass), then the correction from
+// max(0, p'_k - q'_k) or the bonus from p'_gamma over the whole row.
+template <int TDT, int DDT, int DK>
 __global__ void __launch_bounds__(SEQ_BT) k_chain_final_filt(const Params P) {
     __shared__ FinShared sh;
     extern __shared__ __align__(128) unsigned char dyn[];
-    constexpr int CH = chunk_elems<TDT>();
-    constexpr int QDT = DK == DK_PROBS ? SPEC_F32 : DDT;
     const int tid = threadIdx.x, b = blockIdx.x;
-    const int gamma = P.gamma, V = P.V;
+    const int gamma = P.gamma;
     float* wpw = reinterpret_cast<float*>(dyn);
     const ChainPrefetch pf = chain_prefetch<TDT, DDT, DK>(P, b);
     pdl_wait();
     combine_softmax_rows<SEQ_BT>(P, P.stats + (size_t)b * P.R * P.nch * SPC, P.R, sh);
     __syncthreads();
     const int rows = (DK == DK_LOGITS) ? 2 * gamma + 1 : gamma + 1;
-    if constexpr (!OD) {
-        for (int r = tid; r < rows; r += SEQ_BT) {
-            const FiltRec f = P.filt[(size_t)b * P.R + r];
-            sh.th[r] = f.theta;
-            if (f.on > 0) sh.z[r] = f.Z;
-            if (f.on < 0) sh.bad[r] = 1;             // invalid top_k / top_p
-        }
-        __syncthreads();
-    } else {
-        __shared__ WinShared ws;
-        unsigned char* win = dyn + P.stage_off;
-        const int K = P.top_k ? P.top_k[b] : 0;
-        const float Pp = P.top_p ? P.top_p[b] : 1.f;
-        const float T = P.temperature[b];
-        for (int r = tid; r < rows; r += SEQ_BT) sh.th[r] = -INFINITY;
-        if (tid < gamma) {                          // the prefetched decision inputs, for thread 0
-            sh.tok[tid] = pf.x;
-            sh.pch[tid] = pf.ok ? (double)pf.l : NAN;
-            sh.pch[SPEC_MAX_GAMMA + tid] = (double)pf.d;
-            sh.pch[2 * SPEC_MAX_GAMMA + tid] = (double)pf.coin;
-        }
-        __syncthreads();
-        bool go = temperature_ok(T) && K >= 0 && Pp > 0.f && Pp <= 1.f;
-        for (int r = 0; r < rows; ++r) go &= !sh.bad[r];
-        if (!(K >= 0 && Pp > 0.f && Pp <= 1.f) && tid == 0) sh.bad[0] = 1;   // invalid top_k / top_p
-        const float s = scale_of(T);
-        for (int i = 0; go && i <= gamma; ++i) {
-            // filter target row i, and draft-logit row i below gamma
-            for (int half = 0; half < ((DK == DK_LOGITS && i < gamma) ? 2 : 1); ++half) {
-                const int r = half ? gamma + 1 + i : i;
-                const char* row = half ? P.drf + ((size_t)b * gamma + i) * P.dstride
-                                       : P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride;
-                const FiltRec f = wfilter_row<SEQ_BT>(row, V, s, sh.m[r], sh.z[r], K, Pp, win, ws);
-                if (tid == 0) {
-                    sh.th[r] = f.theta;
-                    if (f.on > 0) sh.z[r] = f.Z;
-                }
-                __syncthreads();
-            }
-            if (i == gamma) break;
-            // the accept test of position i, as chain_decide takes it
-            if (tid == 0) {
-                int go_on = 0;
-                const double l = sh.pch[i];
-                if (l == l) {
-                    double p = prob_d((float)l, s, sh.m[i], sh.z[i]);
-                    if ((float)l < sh.th[i]) p = 0.0;
-                    double q;
-                    if constexpr (DK == DK_PROBS) {
-                        q = sh.pch[SPEC_MAX_GAMMA + i];
-                    } else {
-                        const float d = (float)sh.pch[SPEC_MAX_GAMMA + i];
-                        q = prob_d(d, s, sh.m[gamma + 1 + i], sh.z[gamma + 1 + i]);
-                        if (d < sh.th[gamma + 1 + i]) q = 0.0;
-                    }
-                    const double ratio = (q > 0.0) ? p / q : INFINITY;
-                    go_on = sh.pch[2 * SPEC_MAX_GAMMA + i] <= ratio;
-                }
-                sh.ivals[4] = go_on;
-            }
-            __syncthreads();
-            go = sh.ivals[4] != 0;
-            __syncthreads();
-        }
-        __syncthreads();
+    for (int r = tid; r < rows; r += SEQ_BT) {
+        const FiltRec f = P.filt[(size_t)b * P.R + r];
+        sh.th[r] = f.theta;
+        if (f.on > 0) sh.z[r] = f.Z;
+        if (f.on < 0) sh.bad[r] = 1;                 // invalid top_k / top_p
     }
+    __syncthreads();
     chain_decide<TDT, DDT, DK, true>(P, b, sh, true, pf);
     const int ok = sh.ivals[0], k = sh.ivals[1];
     if (!ok) return;
@@ -4275,30 +4431,16 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
     const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
-    // all rows bf16: windowed histograms, WF_BT threads; else FILT_BT threads
-    // and room for an f32 row's radix histograms
-    constexpr bool all_bf16 = TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16);
-    constexpr int bt = all_bf16 ? WF_BT : FILT_BT;
-    constexpr size_t hist = all_bf16 ? WF_BYTES
-                                     : (filt_hist_bytes<SPEC_F32>() > WF_BYTES ? filt_hist_bytes<SPEC_F32>() : WF_BYTES);
+    // FILT_BT threads: a bf16 row's value histogram (VH_BYTES), an f32 row's
+    // radix histograms
+    constexpr bool any_bf16 = TDT == SPEC_BF16 || (DK == DK_LOGITS && DDT == SPEC_BF16);
+    constexpr int bt = FILT_BT;
+    constexpr size_t hist = any_bf16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_filter<TDT, DDT, DK, false, bt>;
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_filter shared memory attribute");
     const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
-    if constexpr (all_bf16) {
-        // No diagnostics to fill: the finalisation filters only the rows the
-        // decision reaches.
-        if (P.diag == nullptr) {
-            P.stage_off = (int)((wpw + 127) & ~(size_t)127);
-            auto kod = k_chain_final_filt<TDT, DDT, DK, true>;
-            const size_t smem = (size_t)P.stage_off + WF_BYTES;
-            static PerDevice<bool> od_c;
-            const bool od = od_c.get([&] { return allow_smem(kod, STAGE_STATS_MAX); });
-            if (!od || smem > STAGE_STATS_MAX) return fail(SPEC_ERR_CUDA, "k_chain_final_filt shared memory");
-            return launch_dependent(kod, (unsigned)P.B, SEQ_BT, smem, P, st, "k_chain_final_filt");
-        }
-    }
     s = launch_dependent(kf, (unsigned)(P.B * rows), bt, hist, P, st, "k_filter");
     if (s != SPEC_OK) return s;
     return launch_dependent(k_chain_final_filt<TDT, DDT, DK>, (unsigned)P.B, SEQ_BT, wpw, P, st,
@@ -4349,8 +4491,8 @@ spec_status launch_tree_filtered(Params P, cudaStream_t st) {
                                     (size_t)P.stage_off + WF_BYTES, P, st, "k_tree_final");
         }
     }
-    constexpr int bt = TDT == SPEC_BF16 ? WF_BT : FILT_BT;
-    constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
+    constexpr int bt = FILT_BT;
+    constexpr size_t hist = TDT == SPEC_BF16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_filter<TDT, TDT, DK_NONE, true, bt>;
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
@@ -4408,10 +4550,9 @@ template <int TDT, int DDT, int DK>
 spec_status launch_chain_filtered_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>;
     auto kd = k_lz_decide_chain<TDT, DDT, DK, true>;
-    constexpr bool all_bf16 = TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16);
-    constexpr int fbt = all_bf16 ? WF_BT : FILT_BT;
-    constexpr size_t hist = all_bf16 ? WF_BYTES
-                                     : (filt_hist_bytes<SPEC_F32>() > WF_BYTES ? filt_hist_bytes<SPEC_F32>() : WF_BYTES);
+    constexpr bool any_bf16 = TDT == SPEC_BF16 || (DK == DK_LOGITS && DDT == SPEC_BF16);
+    constexpr int fbt = FILT_BT;
+    constexpr size_t hist = any_bf16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_lz_filter_chain<TDT, DDT, DK, fbt>;
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
@@ -4483,14 +4624,14 @@ spec_status launch_tree_lazy(Params P, cudaStream_t st) {
 template <int TDT>
 spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
     auto ks = k_lz_stats<MODE_SAMPLE, TDT, TDT>;
-    constexpr int fbt = TDT == SPEC_BF16 ? WF_BT : FILT_BT;
+    constexpr int fbt = FILT_BT;
     auto kf = k_lz_filter_tree<TDT, fbt>;
     auto kd = k_lz_decide_tree<MODE_SAMPLE, TDT, true>;
     static PerDevice<int> occ_c;
     const int occ = occ_c.get([&] { return blocks_per_sm(ks); });
     const unsigned sgrid = stats_grid((long long)P.B * P.nch, occ);
     const unsigned dgrid = (unsigned)((P.B + NWARP - 1) / NWARP);
-    constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
+    constexpr size_t hist = TDT == SPEC_BF16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
     if (!attr) return fail(SPEC_ERR_CUDA, "k_lz_filter_tree shared memory attribute");
