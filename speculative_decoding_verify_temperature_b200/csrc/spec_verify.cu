@@ -346,8 +346,10 @@ __device__ __forceinline__ float tree_sum(const float* a) {
     else return tree_sum<N / 2>(a) + tree_sum<N - N / 2>(a + N / 2);
 }
 
-// 2^(a - b) in fp64 (the rescaling of a statistic to another maximum).
-__device__ __forceinline__ double ex2d(float a, float b) { return exp2((double)a - (double)b); }
+// 2^(a - b) in fp64 (the rescaling of a statistic to another maximum).  Not
+// inlined: the fp64 exp2 needs many registers, and the callers (one call per
+// statistic) are kernels that run at high occupancy.
+__device__ __noinline__ double ex2d(float a, float b) { return exp2((double)a - (double)b); }
 
 // Per-thread online-softmax partial of NV 16-byte vectors held in registers:
 // (max x, sum 2^(x - max)), x = l * s.  `bad` is set by a NaN or +inf.
@@ -1087,20 +1089,21 @@ __device__ void wf_scan3(unsigned c, double l, double h, unsigned* ec, double* e
     __syncthreads();
 }
 
-// Calls f(key) for every element of a bf16 row (BT threads, four 16-byte
-// loads in flight per thread).
+// Calls f(key) for every element of a bf16 row (BT threads, WF_NV 16-byte
+// loads in flight per thread: one CTA per row streams it alone).
+constexpr int WF_NV = 8;
 template <int BT, class F>
 __device__ __forceinline__ void wf_each_key(const char* row, int V, F f) {
     const int nv = (V + 7) / 8;
-    for (int v0 = threadIdx.x; v0 < nv; v0 += 4 * BT) {
-        uint4 v[4];
+    for (int v0 = threadIdx.x; v0 < nv; v0 += WF_NV * BT) {
+        uint4 v[WF_NV];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < WF_NV; ++q) {
             const int vi = v0 + q * BT;
             v[q] = vi < nv ? ld_vec<SPEC_BF16>(row, (int64_t)vi * 8, V) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < WF_NV; ++q) {
             const int vi = v0 + q * BT;
             if (vi >= nv) break;
             const uint32_t xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
@@ -3158,21 +3161,59 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
 
 template <int TDT, int DDT, int DK, bool TREE, int BT>
 __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Params P) {
+    static_assert(BT == FILT_BT, "the value histogram and the radix descent take FILT_BT threads");
     __shared__ FiltShared fs;
-    __shared__ WinShared ws;
+    __shared__ float msh;
+    __shared__ double zsh;
+    __shared__ int bad;
     extern __shared__ __align__(128) unsigned char dyn[];
     pdl_trigger();
     const int rows = TREE ? P.N : ((DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1);
     const int b = blockIdx.x / rows, r = blockIdx.x - b * rows;
-    pdl_wait();
-    if (TREE || r <= P.gamma) {
-        const char* row = TREE ? P.tgt + ((size_t)b * P.N + r) * P.tstride
-                               : P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride;
-        filter_one_row<TDT, BT>(P, b, r, row, fs, ws, dyn);
-    } else {
-        filter_one_row<DDT, BT>(P, b, r, P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride, fs, ws,
-                                dyn);
+    FiltRec* out = P.filt + (size_t)b * P.R + r;
+    const int K = P.top_k ? P.top_k[b] : 0;
+    const float Pp = P.top_p ? P.top_p[b] : 1.f;
+    const float T = P.temperature[b];
+    if (K < 0 || !(Pp > 0.f && Pp <= 1.f)) {
+        pdl_wait();
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, -1, 0.0};
+        return;
     }
+    if (!temperature_ok(T) || ((K <= 0 || K >= P.V) && Pp >= 1.f)) {
+        pdl_wait();
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const bool tgt = TREE || r <= P.gamma;
+    const char* row = TREE  ? P.tgt + ((size_t)b * P.N + r) * P.tstride
+                      : tgt ? P.tgt + ((size_t)b * (P.gamma + 1) + r) * P.tstride
+                            : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
+    const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
+    uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
+    // a bf16 row's value histogram needs only its logits: built while the
+    // statistics kernel (whose row maxima the masses are relative to) runs
+    const int n = vh ? vh_build(row, P.V, fs, w) : 0;
+    pdl_wait();
+    const int E = P.nch * SPC;
+    if (threadIdx.x < 32) {
+        float m;
+        double z;
+        const bool bd = warp_combine(P.stats + ((size_t)b * P.R + r) * E, E, m, z);
+        if (threadIdx.x == 0) { msh = m; zsh = z; bad = bd; }
+    }
+    __syncthreads();
+    if (bad) {                                   // the decision marks the sequence invalid
+        if (threadIdx.x == 0) *out = FiltRec{-INFINITY, 0, 0.0};
+        return;
+    }
+    const float s = scale_of(T), m = msh;
+    const double z = zsh;
+    FiltRec rec;
+    if (!vh || !vh_select(P.V, n, s, m, z, K, Pp, fs, w, &rec)) {
+        if (tgt) rec = filter_row<TDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<TDT>{dyn});
+        else rec = filter_row<DDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<DDT>{dyn});
+    }
+    if (threadIdx.x == 0) *out = rec;
 }
 
 
