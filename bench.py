@@ -600,26 +600,18 @@ def measure(wid, dev, world, steps, warmup, local, rank=0, diag=False):
                 mean_tau=float((acc.float() + 1).mean()), hist=accept_histogram(wid, first, acc))
 
 
-ROW_KERNEL = {
-    "fused": "k_chain_fused (streams every row pair once and takes the whole round's decisions)",
-    "stats": "k_stats (streams every logit row once)",
-}
+ROW_KERNEL = "k_stats (streams every logit row once)"
 
 
-def roofline_of(m, peaks, peak_kind, row_kernel):
+def roofline_of(m, peaks, peak_kind):
     achieved = m["alg"] / (m["k_avg_ms"] / 1e3) / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": profile_traffic(m["wid"]),
-            "kernel": ROW_KERNEL[row_kernel], "kernel_ms": round(m["k_avg_ms"], 5),
+            "kernel": ROW_KERNEL, "kernel_ms": round(m["k_avg_ms"], 5),
             "algorithmic_bytes_per_launch": m["alg"],
-            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)",
+            "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)" if peak_kind == "measured"
+                            else "fallback (MEASURED_PEAKS.json absent: 6650 GB/s, an earlier copy measurement on B200)"),
             "frac_of_nominal_8000_gbs": round(achieved / 8000.0, 4)}
-
-
-def row_kernel_of(m) -> str:
-    """Which kernel the library's timing hook brackets for this workload: the
-    fused chain kernel is the only launch of its call."""
-    return "fused" if m["kps"] == 1 else "stats"
 
 
 def config_summary(m, peaks, peak_kind, cpu=None) -> dict:
@@ -628,7 +620,7 @@ def config_summary(m, peaks, peak_kind, cpu=None) -> dict:
     d = {"workload": describe(m["wid"], m["first"])["workload"], "steps": m["K"],
          "rounds_per_s": round(m["value"], 2), "step_us": round(step_s * 1e6, 3),
          "gpu_launches_per_step": m["kps"],
-         "row_kernel": roofline_of(m, peaks, peak_kind, row_kernel_of(m)),
+         "row_kernel": roofline_of(m, peaks, peak_kind),
          "round_algorithmic_bytes": int(m["round_bytes"]),
          "round_hbm_gbs": round(m["round_bytes"] / step_s / 1e9, 1),
          "round_frac": round(m["round_bytes"] / step_s / 1e9 / peaks["hbm_gbs"], 4),
@@ -689,7 +681,7 @@ def main():
     m = measure(wid, dev, ws_, args.steps, args.warmup, local, rank, diag=args.with_diag)
     first, sets, ws, K = m["first"], m["sets"], m["ws"], m["K"]
     peaks, peak_kind = measured_peaks()
-    roofline = roofline_of(m, peaks, peak_kind, row_kernel_of(m))
+    roofline = roofline_of(m, peaks, peak_kind)
     value, ms_max = m["value"], m["ms_max"]
     B = first.B
     draft_per_round = B * (first.gamma if wid in (0, 1, 4, 6, 7) else first.N - 1)

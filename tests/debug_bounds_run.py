@@ -20,7 +20,7 @@ def main():
     assert sv.LIB_PATH.endswith("libspecverify_debug.so"), sv.LIB_PATH
     assert sv.spec_debug_bounds_hits() == 0
     bad = 0
-    # chain: fused (draft logits), two-kernel (probabilities, f32 over 8 chunks), lazy, filtered
+    # chain: draft logits, draft probabilities, f32 rows over 8 chunks; then lazy and filtered
     for inp in [wl.chain_inputs(8, 4, 20000, seed=1, device="cuda", zipf=True, temperatures=(0.6, 1.0)),
                 wl.chain_inputs(6, 3, 30000, seed=2, device="cuda", draft_is_probs=True),
                 wl.chain_inputs(4, 2, 40000, seed=3, device="cuda", target_dtype=torch.float32,
