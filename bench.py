@@ -594,10 +594,20 @@ def measure(wid, dev, world, steps, warmup, local, rank=0, diag=False):
         acc.append(k.clone())
         rb += round_bytes(wid, st, k)
     acc = torch.cat(acc)
+    # --- filtered workloads: how many rows each filter path resolved (one
+    # untimed call per input set with the library's row counters on)
+    filt = None
+    if wid in (6, 8):
+        sv.spec_debug_filter_path(0, read=True)
+        for r in runners:
+            r()
+        a, b, c = sv.spec_debug_filter_path(-1, read=True)
+        filt = {"rows_by_candidates": a, "rows_by_candidates_deeper_cut": c, "rows_by_whole_row_path": b,
+                "calls": nsets}
     return dict(wid=wid, sets=sets, first=first, nsets=nsets, nbytes=nbytes, ws=ws, runners=runners, K=K,
                 ms_max=ms_max, value=value, kps=kps, k_avg_ms=k_avg_ms, clocks=sampler.summary(),
                 alg=algorithmic_bytes(wid, first), round_bytes=rb / nsets,
-                mean_tau=float((acc.float() + 1).mean()), hist=accept_histogram(wid, first, acc))
+                mean_tau=float((acc.float() + 1).mean()), hist=accept_histogram(wid, first, acc), filt=filt)
 
 
 ROW_KERNEL = "k_stats (streams every logit row once)"
@@ -710,6 +720,8 @@ def main():
         "accept_length_histogram": m["hist"],
         "e2e": e2e, "gpu_launches": K * m["kps"], "clocks": m["clocks"], "lazy": lazy,
     }
+    if m["filt"] is not None:
+        line["filter_rows"] = m["filt"]
     cpu_here = rank == 0 and ws_ == 1 and not args.no_cpu_baseline
     if cpu_here:
         cb, o, rows = cpu_baseline(wid, first, args.cpu_seconds)

@@ -575,6 +575,27 @@ spec_status spec_profile_events(void* start_event, void* stop_event);
 spec_status spec_debug_wait_budget(long long tries);
 
 /*
+ * spec_debug_filter_path -- testing hook for the top-k / top-p filters of bf16
+ * rows.  Each filtered row is first resolved from its candidates: the values
+ * within a factor 2^14 of the row's largest probability (or fewer when the
+ * row's mass bound allows), counted per value in one pass into a window of
+ * per-key counters fixed by the row statistics, and again with 2^18, then
+ * 2^24, when a cut holds too few values or too little mass.  A row whose
+ * candidates cannot hold the answer, or whose window would overflow the
+ * kernel's shared memory, is resolved by a whole-row path (the 65536-key
+ * value histogram in 1024-thread filter CTAs, else the windowed filter).
+ * Both give the same record.
+ * mode 0: the default paths, counting rows by path; mode 1: whole-row paths
+ * only, counting; mode -1: the default paths, no counting (the state at load).
+ * rows, if not NULL, receives three counts since the last read on the
+ * current device -- [0] rows the candidates resolved at the first cut, [1]
+ * rows left to a whole-row path, [2] rows the candidates resolved at a
+ * deeper cut -- and resets them (a synchronous device read).  Applies to later calls
+ * on the calling host thread.  Not for production use.
+ */
+spec_status spec_debug_filter_path(int mode, unsigned long long* rows);
+
+/*
  * spec_launch_count -- number of kernels this library has launched (or, inside
  * stream capture, added to a graph) from the calling host thread since the
  * process started.  The difference across a call is that call's launch count.

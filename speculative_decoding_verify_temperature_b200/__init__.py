@@ -8,6 +8,7 @@ from .spec_verify import (  # noqa: F401
     SpecError,
     Workspace,
     lib,
+    spec_debug_filter_path,
     spec_debug_wait_budget,
     spec_launch_count,
     spec_profile_events,

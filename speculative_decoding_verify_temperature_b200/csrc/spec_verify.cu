@@ -112,6 +112,7 @@ struct Params {
     unsigned* cnt2;                // [B]               (chain residual arrivals)
     unsigned* status;
     unsigned wait_tries;           // polls of the first wait for a CTA's own bulk copy (0: give up at once)
+    unsigned filt_mode;            // bit 0: no candidate pass in the filters; bit 1: count filtered rows by path
     // lazy (row-on-demand) verification
     struct LazySeq* lz_seq;        // [B]
     int* lz_rej;                   // [B][rej_cap]      (trees: rejected children tokens)
@@ -524,6 +525,7 @@ __device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
 // additions) and decide top-p and Z'.
 
 constexpr int FILT_BT = 1024;
+constexpr int FILT_BT_BF16 = 256;                 // filter CTAs of launches whose filtered rows are all bf16
 constexpr double FIX_ONE = 1099511627776.0;      // 2^40
 
 template <int DT> __device__ __forceinline__ uint32_t order_key(float v) {
@@ -761,7 +763,7 @@ __device__ __forceinline__ uint32_t vh_keys2(uint32_t x) {
 // 16-bit counters per 32-bit word, 128 KB of shared memory) from one pass;
 // every mass then follows exactly as count * fixed(2^(v s - m)) per value,
 // the same fixed-point numbers the radix path adds element by element.
-// (The windowed filter below forms the same numbers in 56 KB for callers
+// (The windowed filter below forms the same numbers in 52 KB for callers
 // that cannot hold 192 KB.)
 //
 // A row has at most V distinct values, so most of the 32768 words are empty.
@@ -986,8 +988,8 @@ __device__ bool vh_select(int V, int n, float s, float m, double zrow, int K, fl
 // boundary are the near-ties the oracle flags.  A window needing more than
 // WF_SLOTS counters is counted in segments, one more pass each.
 constexpr int WF_NB = 4096;                       // coarse buckets (key >> 4)
-constexpr int WF_SLOTS = 8192;                    // per-key counters of the window
-constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 56 KB
+constexpr int WF_SLOTS = 7168;                    // per-key counters of the window
+constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 52 KB
 
 struct WinShared {
     unsigned long long red[32];
@@ -1308,6 +1310,259 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
     r.on = 1;
     r.Z = (double)z / FIX_ONE;
     return r;
+}
+
+// bf16 rows, candidates first.  A cut x_c = (m - D) / s, D log2 units below
+// the row's maximum (D = 14; with top-p alone, less when the whole row's mass
+// bound V * 2^(x s - m) already proves the top-p key lies above it), rounded
+// down to a bf16 value.  The candidates' order keys lie in [key(x_c),
+// key(max)], both known from the statistics before the row is read: that
+// window of per-key counters -- without the keys of the tiny values |v| <
+// 2^-10 inside it, which a cut below zero would otherwise bring in by the
+// tens of thousands of (mostly absent) keys; those few values are counted
+// together, with their exact fixed-point mass -- is cleared, and one pass
+// over the row counts every value >= x_c into it (bf16 pair compares make a
+// survivor mask per 16-byte vector; each lane counts its own survivors with
+// 32-bit shared atomics, at the position a 512-entry table of key groups
+// gives).  The window is then scanned from its top as the
+// value histogram scans its keys -- count and fixed-point mass count *
+// fixed(2^(v s - m)) per key, a block scan, the thread whose run crosses
+// top_k or the top-p target walks it -- so the record is the same integers
+// and the same keys.  The window holds every value >= x_c, so the record is
+// exact unless the crossing falls among the tiny values: with top-k, the
+// top-p key lies at or above the top-k key; with top-p alone, the window's
+// mass must reach the top-p target.  A cut that holds fewer than top_k values
+// or too little mass is deepened (D = 18, then 24; the row is read again,
+// mostly from L2); otherwise, or when the window would outgrow the shared
+// memory, the function returns false and the caller takes a whole-row path.
+constexpr float CF_D = 14.f, CF_D2 = 18.f, CF_D3 = 24.f;
+constexpr float CF_TINY = 9.765625e-04f;          // 2^-10 (a whole number of key groups either side of 0)
+constexpr int CF_TINY_G = INT_MIN / 2;            // group table: a group of tiny values
+struct CfShared {
+    WinShared ws;                                 // block scans
+    unsigned tiny, over;
+    int sel, tz;
+    unsigned long long at, tinym;
+    int gbase[512];                               // key group (key >> 7) -> window position of its key 0
+};
+constexpr size_t CF_HEAD = ((sizeof(CfShared) + 127) / 128) * 128;
+enum { CF_OK = 0, CF_SHORT = 1, CF_FAIL = 2 };
+
+// One cut at D log2 units: CF_OK (record in *out), CF_SHORT (the cut holds
+// too few values or too little mass: a deeper cut may hold the answer) or
+// CF_FAIL.  All threads call it.
+template <int BT>
+__device__ int cf_attempt(const char* row, int V, float s, float m, double zrow, int K, float Pp, float D,
+                          unsigned char* smem, size_t bytes, FiltRec* out) {
+    CfShared& cs = *reinterpret_cast<CfShared*>(smem);
+    unsigned* win = reinterpret_cast<unsigned*>(smem + CF_HEAD);
+    const unsigned wmax = (unsigned)min((size_t)16384, (bytes - CF_HEAD) / 4);
+    const int tid = threadIdx.x;
+    const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
+    const __nv_bfloat16 tb = __float2bfloat16_rd((m - D) / s);
+    const float xc = __bfloat162float(tb);
+    if (!(xc > -INFINITY)) return CF_FAIL;            // (a cut at -inf would count the row's padding)
+    const __nv_bfloat162 t2 = __halves2bfloat162(tb, tb);
+    // the window: keys [klo, khi] less the tiny keys [g0, g1] inside it
+    const uint32_t klo = order_key<SPEC_BF16>(xc);
+    const uint32_t khi = order_key<SPEC_BF16>(__bfloat162float(__float2bfloat16_ru(m / s))) + 1u;
+    const uint32_t g0 = max(order_key<SPEC_BF16>(-CF_TINY) + 1u, klo);
+    const uint32_t g1 = min(order_key<SPEC_BF16>(CF_TINY) - 1u, khi);
+    const uint32_t glen = g0 <= g1 ? g1 - g0 + 1u : 0u;
+    if (khi < klo || khi - klo + 1u - glen > wmax) return CF_FAIL;
+    const unsigned W = khi - klo + 1u - glen;
+    for (unsigned i = tid; i < W; i += BT) win[i] = 0u;
+    // window position of key k = gbase[k >> 7] + (k & 127); outside [0, W):
+    // not in the window (a tiny group is marked)
+    for (int g = tid; g < 512; g += BT) {
+        const uint32_t k0 = (uint32_t)g << 7;
+        cs.gbase[g] = (glen && k0 >= g0 && k0 <= g1) ? CF_TINY_G
+                                                     : (int)k0 - (int)klo - ((glen && k0 > g1) ? (int)glen : 0);
+    }
+    if (tid == 0) { cs.tiny = 0u; cs.over = 0u; cs.tinym = 0ull; cs.tz = 0; }
+    __syncthreads();
+    auto count = [&](uint32_t u) {                  // one bf16 value (raw bits) >= x_c
+        u = u == 0x8000u ? 0u : u;                    // -0 counts as +0
+        const uint32_t k = u ^ (((u >> 15) * 0x7FFFu) | 0x8000u);
+        const int b = cs.gbase[k >> 7];
+        const int sl = b + (int)(k & 127u);
+        if ((unsigned)sl < W) {
+            atomicAdd(&win[sl], 1u);
+        } else if (b == CF_TINY_G) {
+            atomicAdd(&cs.tiny, 1u);
+            atomicAdd(&cs.tinym, fix_mass(key_value<SPEC_BF16>(k), s, m));
+        } else {
+            cs.over = 1u;
+        }
+    };
+    auto survivors = [&](const uint4& vq) {
+        const uint32_t xs[4] = {vq.x, vq.y, vq.z, vq.w};
+        unsigned bits = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            __nv_bfloat162 h;
+            memcpy(&h, &xs[c], 4);
+            bits |= (__hge2_mask(h, t2) & 0x10001u) << c;
+        }
+        while (bits) {
+            const int p = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            const int c = p & 3;
+            const uint32_t w = c < 2 ? (c == 0 ? xs[0] : xs[1]) : (c == 2 ? xs[2] : xs[3]);
+            count(p >= 16 ? (w >> 16) : (w & 0xFFFFu));
+        }
+    };
+    // ---- one pass: the values >= x_c.  Per 16-byte vector the four pair
+    // compares make a survivor mask (bit c: the low value of pair c, bit
+    // 16 + c: the high one); each lane then counts only its own survivors.
+    // The next step's loads are issued before this step's vectors are
+    // examined, so the examination hides under the memory latency.
+    constexpr int CF_NV = BT == 512 ? 8 : 4;
+    const int nfull = V / 8, nv = (V + 7) / 8;      // whole vectors; with the ragged tail
+    int v0 = tid;
+    if (v0 + (CF_NV - 1) * BT < nfull) {
+        uint4 a[CF_NV], b[CF_NV];
+#pragma unroll
+        for (int q = 0; q < CF_NV; ++q) a[q] = ld_stream(row + (size_t)(v0 + q * BT) * 16);
+        for (;;) {
+            const int v1 = v0 + CF_NV * BT;
+            const bool more = v1 + (CF_NV - 1) * BT < nfull;
+            if (more) {
+#pragma unroll
+                for (int q = 0; q < CF_NV; ++q) b[q] = ld_stream(row + (size_t)(v1 + q * BT) * 16);
+            }
+#pragma unroll
+            for (int q = 0; q < CF_NV; ++q) survivors(a[q]);
+            v0 = v1;
+            if (!more) break;
+#pragma unroll
+            for (int q = 0; q < CF_NV; ++q) a[q] = b[q];
+        }
+    }
+    for (; v0 < nv; v0 += BT) survivors(ld_vec<SPEC_BF16>(row, (int64_t)v0 * 8, V));   // (past V: -inf)
+    __syncthreads();
+    if (cs.over) {                                    // (the statistics' maximum disagrees with the row)
+        __syncthreads();
+        return CF_FAIL;
+    }
+    const unsigned tinyc = cs.tiny;
+    const unsigned long long tinym = cs.tinym;
+    // ---- the window from its top: thread t takes positions [t * per, (t + 1) * per);
+    // the tiny values come just before position pl (the first key below them)
+    auto key_at = [&](unsigned p) -> uint32_t {      // key of position p from the top
+        const uint32_t w = W - 1u - p;
+        return (glen && klo + w >= g0) ? klo + w + glen : klo + w;
+    };
+    const unsigned pl = glen ? W - (g0 - klo) : W;
+    const unsigned per = (W + BT - 1) / BT;
+    const unsigned p0 = min(W, tid * per), p1 = min(W, p0 + per);
+    const bool own_tiny = tinyc && p0 < p1 && ((pl >= p0 && pl < p1) || (pl == W && p1 == W));
+    unsigned sc = own_tiny ? tinyc : 0u;
+    unsigned long long sm = own_tiny ? tinym : 0ull;
+    for (unsigned p = p0; p < p1; ++p) {
+        const unsigned c = win[W - 1u - p];
+        if (c) {
+            sc += c;
+            sm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(key_at(p)), s, m);
+        }
+    }
+    unsigned c0, ctot;
+    unsigned long long m0, mtot;
+    wf_scan2<BT>(sc, sm, &c0, &m0, &ctot, &mtot, cs.ws);
+    // the thread whose run crosses the count K (by_count) or the mass target;
+    // a crossing inside the tiny values sets cs.tz.  The first barrier keeps
+    // thread 0 from resetting cs.sel before every thread has read the
+    // previous search's result: the outcome must be the same in every thread
+    // (it decides which barriers they reach next).
+    auto find = [&](bool by_count, double target) {
+        __syncthreads();
+        if (tid == 0) cs.sel = -1;
+        __syncthreads();
+        const bool cross = by_count ? (c0 < (unsigned)K && c0 + sc >= (unsigned)K)
+                                    : ((double)m0 < target && (double)(m0 + sm) >= target);
+        if (cross) {
+            unsigned c = c0;
+            unsigned long long mm = m0;
+            auto hit = [&]() { return by_count ? c >= (unsigned)K : (double)mm >= target; };
+            bool done = false;
+            for (unsigned p = p0; p < p1 && !done; ++p) {
+                if (own_tiny && p == pl) {
+                    c += tinyc;
+                    mm += tinym;
+                    if (hit()) { cs.tz = 1; done = true; break; }
+                }
+                const unsigned cj = win[W - 1u - p];
+                if (!cj) continue;
+                const uint32_t k = key_at(p);
+                c += cj;
+                mm += (unsigned long long)cj * fix_mass(key_value<SPEC_BF16>(k), s, m);
+                if (hit()) {
+                    cs.sel = (int)k;
+                    cs.at = mm;
+                    done = true;
+                }
+            }
+            if (!done && own_tiny && pl == W) cs.tz = 1;   // the tiny values close the window
+        }
+        __syncthreads();
+    };
+    int key = -1, st = CF_OK;
+    unsigned long long z = 0ull;
+    if (use_k) {
+        find(true, 0.0);
+        key = cs.sel;
+        z = cs.at;
+        st = cs.tz ? CF_FAIL : key < 0 ? CF_SHORT : CF_OK;
+    }
+    if (use_p && st == CF_OK) {
+        // with top-k the top-p key lies at or above the top-k key (the running
+        // mass there is the kept mass)
+        find(false, top_p_target(use_k, Pp, z, zrow));
+        key = cs.sel;
+        z = cs.at;
+        st = cs.tz ? CF_FAIL : key < 0 ? CF_SHORT : CF_OK;
+    }
+    __syncthreads();                                  // cs is read; the shared memory is free again
+    if (st == CF_OK) {
+        out->theta = key_value<SPEC_BF16>((uint32_t)key);
+        out->on = 1;
+        out->Z = (double)z / FIX_ONE;
+    }
+    return st;
+}
+
+// Threshold and kept mass of one bf16 row from its candidates (see above):
+// 1 (first cut) or 2 (deeper cut) with the record in *out; 0: the caller
+// takes a whole-row path.  smem: `bytes` of shared memory (up to 16384 window
+// counters).  All threads call it.
+template <int BT>
+__device__ int cfilter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp,
+                            unsigned char* smem, size_t bytes, FiltRec* out) {
+    float D = CF_D;
+    if (!(K > 0 && K < V)) {                          // top-p alone: the row's mass bound, factor-2 slack
+        const double rest = zrow - top_p_target(false, Pp, 0ull, zrow) / FIX_ONE;
+        if (rest > 0.0) D = fminf(D, log2f((float)(2.0 * V / rest)));
+    }
+    int st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out);
+    if (st != CF_SHORT) return st == CF_OK ? 1 : 0;
+    for (int i = 0; i < 2 && st == CF_SHORT; ++i)
+        st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, fmaxf(D, i == 0 ? CF_D2 : CF_D3), smem, bytes, out);
+    return st == CF_OK ? 2 : 0;
+}
+
+// Rows the candidates resolved at the first cut ([0]) or at the deeper one
+// ([2]) and rows left to a whole-row path ([1]), counted only when the caller
+// asks (spec_debug_filter_path).
+__device__ unsigned long long g_filter_rows[3];
+
+// cfilter_row unless the caller switched the candidate pass off; counts the
+// outcome when asked.
+template <int BT>
+__device__ __forceinline__ bool cand_filter(const Params& P, const char* row, float s, float m, double z, int K, float Pp,
+                                            unsigned char* smem, size_t bytes, FiltRec* out) {
+    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out);
+    if ((P.filt_mode & 2u) && threadIdx.x == 0) atomicAdd(&g_filter_rows[how == 0 ? 1 : how == 1 ? 0 : 2], 1ull);
+    return how != 0;
 }
 
 // ----------------------------------------------------------------------------- finaliser pieces
@@ -2347,7 +2602,9 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         if (tid == 0) ai[0] = 0;
         for (;;) {
             const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
-            const FiltRec f = wfilter_row<BT>(row, V, s, sh.m[cur], sh.z[cur], K, Pp, win, *ws);
+            FiltRec f{-INFINITY, 0, 0.0};
+            if (((K > 0 && K < V) || Pp < 1.f) && !cand_filter<BT>(P, row, s, sh.m[cur], sh.z[cur], K, Pp, win, WF_BYTES, &f))
+                f = wfilter_row<BT>(row, V, s, sh.m[cur], sh.z[cur], K, Pp, win, *ws);
             thc = f.theta;
             zc = f.on > 0 ? f.Z : sh.z[cur];
             for (int n = cur + 1 + tid; n < N; n += BT)
@@ -3149,20 +3406,25 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
         return;
     }
     FiltRec rec{-INFINITY, 0, 0.0};
+    bool done = false;
+    if constexpr (DT == SPEC_BF16) done = cand_filter<BT>(P, row, s, m, zsh, K, Pp, dyn, BT == FILT_BT ? VH_BYTES : WF_BYTES, &rec);
     if constexpr (BT == FILT_BT) {
         uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
-        if (DT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, zsh, K, Pp, fs, w, &rec))
+        if (!done && (DT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, zsh, K, Pp, fs, w, &rec)))
             rec = filter_row<DT>(row, P.V, s, m, zsh, K, Pp, fs, FiltHist<DT>{dyn});
     } else if constexpr (DT == SPEC_BF16) {
-        rec = wfilter_row<BT>(row, P.V, s, m, zsh, K, Pp, dyn, ws);
+        if (!done) rec = wfilter_row<BT>(row, P.V, s, m, zsh, K, Pp, dyn, ws);
     }
     if (threadIdx.x == 0) *out = rec;
 }
 
 template <int TDT, int DDT, int DK, bool TREE, int BT>
-__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Params P) {
-    static_assert(BT == FILT_BT, "the value histogram and the radix descent take FILT_BT threads");
+__global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Params P) {
+    // FILT_BT threads: the value histogram and the radix descent (any row);
+    // fewer: bf16 rows only, the windowed filter as the whole-row path
+    static_assert(BT == FILT_BT || (TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16)), "bf16 rows only");
     __shared__ FiltShared fs;
+    __shared__ WinShared ws;
     __shared__ float msh;
     __shared__ double zsh;
     __shared__ int bad;
@@ -3190,9 +3452,6 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Para
                             : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
     const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
     uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
-    // a bf16 row's value histogram needs only its logits: built while the
-    // statistics kernel (whose row maxima the masses are relative to) runs
-    const int n = vh ? vh_build(row, P.V, fs, w) : 0;
     pdl_wait();
     const int E = P.nch * SPC;
     if (threadIdx.x < 32) {
@@ -3209,7 +3468,11 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 3) k_filter(const Para
     const float s = scale_of(T), m = msh;
     const double z = zsh;
     FiltRec rec;
-    if (!vh || !vh_select(P.V, n, s, m, z, K, Pp, fs, w, &rec)) {
+    if constexpr (BT != FILT_BT) {
+        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec))
+            rec = wfilter_row<BT>(row, P.V, s, m, z, K, Pp, dyn, ws);
+    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec) ||
+                        vh_select(P.V, vh_build(row, P.V, fs, w), s, m, z, K, Pp, fs, w, &rec))) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<DDT>{dyn});
     }
@@ -4202,6 +4465,7 @@ struct NvtxRange {
 };
 thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
 thread_local unsigned g_wait_tries = WAIT_LIMIT;
+thread_local unsigned g_filt_mode = 0u;
 thread_local unsigned long long g_launches = 0;   // kernel launches issued by this host thread
 
 cudaError_t record(cudaEvent_t ev, cudaStream_t st) {
@@ -4330,6 +4594,7 @@ spec_status check_ws(void* ws, size_t bytes, const Layout& L) {
 void bind_ws(Params& P, void* ws, const Layout& L) {
     char* w = static_cast<char*>(ws);
     P.wait_tries = g_wait_tries;
+    P.filt_mode = g_filt_mode;
     P.status = reinterpret_cast<unsigned*>(w + L.status);
     P.cnt2 = reinterpret_cast<unsigned*>(w + L.cnt2);
     P.stats = reinterpret_cast<float2*>(w + L.stats);
@@ -4472,11 +4737,13 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
     const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
-    // FILT_BT threads: a bf16 row's value histogram (VH_BYTES), an f32 row's
-    // radix histograms
+    // bf16 rows only: FILT_BT_BF16 threads, several rows per SM, the windowed
+    // filter's 52 KB; else FILT_BT threads, a bf16 row's value histogram
+    // (VH_BYTES), an f32 row's radix histograms
     constexpr bool any_bf16 = TDT == SPEC_BF16 || (DK == DK_LOGITS && DDT == SPEC_BF16);
-    constexpr int bt = FILT_BT;
-    constexpr size_t hist = any_bf16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
+    constexpr bool all_bf16 = TDT == SPEC_BF16 && (DK != DK_LOGITS || DDT == SPEC_BF16);
+    constexpr int bt = all_bf16 ? FILT_BT_BF16 : FILT_BT;
+    constexpr size_t hist = all_bf16 ? WF_BYTES : any_bf16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_filter<TDT, DDT, DK, false, bt>;
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
@@ -4532,8 +4799,8 @@ spec_status launch_tree_filtered(Params P, cudaStream_t st) {
                                     (size_t)P.stage_off + WF_BYTES, P, st, "k_tree_final");
         }
     }
-    constexpr int bt = FILT_BT;
-    constexpr size_t hist = TDT == SPEC_BF16 ? VH_BYTES : filt_hist_bytes<SPEC_F32>();
+    constexpr int bt = TDT == SPEC_BF16 ? FILT_BT_BF16 : FILT_BT;
+    constexpr size_t hist = TDT == SPEC_BF16 ? WF_BYTES : filt_hist_bytes<SPEC_F32>();
     auto kf = k_filter<TDT, TDT, DK_NONE, true, bt>;
     static PerDevice<bool> attr_c;
     const bool attr = attr_c.get([&] { return allow_smem(kf, hist); });
@@ -4761,6 +5028,19 @@ spec_status spec_debug_bounds_hits(unsigned long long* hits) {
 
 spec_status spec_debug_wait_budget(long long tries) {
     g_wait_tries = tries < 0 ? WAIT_LIMIT : (tries > (long long)WAIT_LIMIT ? WAIT_LIMIT : (unsigned)tries);
+    return SPEC_OK;
+}
+
+spec_status spec_debug_filter_path(int mode, unsigned long long* rows) {
+    if (mode < -1 || mode > 1) return fail(SPEC_ERR_INVALID_ARG, "mode = %d outside [-1, 1]", mode);
+    if (rows) {
+        unsigned long long zero[3] = {0ull, 0ull, 0ull};
+        cudaError_t e = cudaMemcpyFromSymbol(rows, g_filter_rows, sizeof zero);
+        if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_filter_rows, zero, sizeof zero);
+        if (e != cudaSuccess) return fail(SPEC_ERR_CUDA, "filter row counters: %s", cudaGetErrorString(e));
+    }
+    if (mode >= 0) g_filt_mode = (mode == 1 ? 1u : 0u) | 2u;
+    else g_filt_mode = 0u;
     return SPEC_OK;
 }
 

@@ -101,6 +101,8 @@ def lib():
         L.spec_launch_count.argtypes = []
         L.spec_debug_bounds_hits.restype = i32
         L.spec_debug_bounds_hits.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+        L.spec_debug_filter_path.restype = i32
+        L.spec_debug_filter_path.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
         _lib = L
     return _lib
 
@@ -193,6 +195,22 @@ def spec_debug_wait_budget(tries: int = -1) -> None:
     kernels issue, for later calls on this thread (0 = give up at once and take
     the timeout path; negative = the default budget)."""
     _check(lib().spec_debug_wait_budget(int(tries)), "spec_debug_wait_budget")
+
+
+def spec_debug_filter_path(mode: int = -1, read: bool = False) -> tuple[int, int, int] | None:
+    """Testing hook for the bf16 top-k / top-p filters, for later calls on this
+    thread: mode 0 = candidates first (the default) and count rows by path,
+    1 = whole-row paths only and count, -1 = the default without counting.
+    With read=True, returns (rows the candidates resolved at the first cut,
+    rows left to a whole-row path, rows resolved at the deeper cut) since the
+    last read on the current device and resets them (synchronises the
+    device)."""
+    if not read:
+        _check(lib().spec_debug_filter_path(int(mode), None), "spec_debug_filter_path")
+        return None
+    v = (ctypes.c_ulonglong * 3)()
+    _check(lib().spec_debug_filter_path(int(mode), v), "spec_debug_filter_path")
+    return int(v[0]), int(v[1]), int(v[2])
 
 
 class Workspace:
