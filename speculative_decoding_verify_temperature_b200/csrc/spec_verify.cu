@@ -1313,7 +1313,7 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
 }
 
 // bf16 rows, candidates first.  A cut x_c = (m - D) / s, D log2 units below
-// the row's maximum (D = 14; with top-p alone, less when the whole row's mass
+// the row's maximum (D = 12 or 14; with top-p alone, less when the whole row's mass
 // bound V * 2^(x s - m) already proves the top-p key lies above it), rounded
 // down to a bf16 value.  The candidates' order keys lie in [key(x_c),
 // key(max)], both known from the statistics before the row is read: that
@@ -1335,7 +1335,9 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
 // or too little mass is deepened (D = 18, then 24; the row is read again,
 // mostly from L2); otherwise, or when the window would outgrow the shared
 // memory, the function returns false and the caller takes a whole-row path.
-constexpr float CF_D = 14.f, CF_D2 = 18.f, CF_D3 = 24.f;
+// first cut: 12 log2 units where many rows share the SMs (fewer candidates,
+// more rows deepened), 14 where one row's latency is the walk's
+constexpr float CF_D_MANY = 12.f, CF_D_ONE = 14.f, CF_D2 = 18.f, CF_D3 = 24.f;
 constexpr float CF_TINY = 9.765625e-04f;          // 2^-10 (a whole number of key groups either side of 0)
 constexpr int CF_TINY_G = INT_MIN / 2;            // group table: a group of tiny values
 struct CfShared {
@@ -1348,15 +1350,35 @@ struct CfShared {
 constexpr size_t CF_HEAD = ((sizeof(CfShared) + 127) / 128) * 128;
 enum { CF_OK = 0, CF_SHORT = 1, CF_FAIL = 2 };
 
+// 16-byte loads in flight per thread and step: 64 KB per SM (four 256-thread
+// CTAs, or one CTA of 512 or 1024 threads).
+template <int BT> __host__ __device__ constexpr int cf_nv() { return BT == 512 ? 8 : 4; }
+// A row's first step of loads, issued before the statistics are waited for
+// (the logits do not depend on them); have: this thread's step lies inside
+// the row's whole vectors.
+template <int BT> struct CfPre {
+    uint4 v[cf_nv<BT>()];
+    bool have;
+};
+template <int BT> __device__ __forceinline__ void cf_prefetch(const char* row, int V, CfPre<BT>& pre) {
+    constexpr int NV = cf_nv<BT>();
+    pre.have = (int)threadIdx.x + (NV - 1) * BT < V / 8;
+    if (pre.have) {
+#pragma unroll
+        for (int q = 0; q < NV; ++q) pre.v[q] = ld_stream(row + (size_t)(threadIdx.x + q * BT) * 16);
+    }
+}
+
 // One cut at D log2 units: CF_OK (record in *out), CF_SHORT (the cut holds
 // too few values or too little mass: a deeper cut may hold the answer) or
 // CF_FAIL.  All threads call it.
 template <int BT>
-__device__ int cf_attempt(const char* row, int V, float s, float m, double zrow, int K, float Pp, float D,
-                          unsigned char* smem, size_t bytes, FiltRec* out) {
+__device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float m, double zrow, int K, float Pp,
+                                          float D, unsigned char* smem, size_t bytes, FiltRec* out,
+                                          const CfPre<BT>* pre) {
     CfShared& cs = *reinterpret_cast<CfShared*>(smem);
     unsigned* win = reinterpret_cast<unsigned*>(smem + CF_HEAD);
-    const unsigned wmax = (unsigned)min((size_t)16384, (bytes - CF_HEAD) / 4);
+    const unsigned wmax = (unsigned)min((size_t)16384, ((bytes - CF_HEAD) / 4) & ~(size_t)3);
     const int tid = threadIdx.x;
     const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
     const __nv_bfloat16 tb = __float2bfloat16_rd((m - D) / s);
@@ -1371,7 +1393,7 @@ __device__ int cf_attempt(const char* row, int V, float s, float m, double zrow,
     const uint32_t glen = g0 <= g1 ? g1 - g0 + 1u : 0u;
     if (khi < klo || khi - klo + 1u - glen > wmax) return CF_FAIL;
     const unsigned W = khi - klo + 1u - glen;
-    for (unsigned i = tid; i < W; i += BT) win[i] = 0u;
+    for (unsigned i = tid; i < (W + 3u) / 4u; i += BT) reinterpret_cast<uint4*>(win)[i] = make_uint4(0u, 0u, 0u, 0u);
     // window position of key k = gbase[k >> 7] + (k & 127); outside [0, W):
     // not in the window (a tiny group is marked)
     for (int g = tid; g < 512; g += BT) {
@@ -1417,13 +1439,18 @@ __device__ int cf_attempt(const char* row, int V, float s, float m, double zrow,
     // 16 + c: the high one); each lane then counts only its own survivors.
     // The next step's loads are issued before this step's vectors are
     // examined, so the examination hides under the memory latency.
-    constexpr int CF_NV = BT == 512 ? 8 : 4;
+    constexpr int CF_NV = cf_nv<BT>();
     const int nfull = V / 8, nv = (V + 7) / 8;      // whole vectors; with the ragged tail
     int v0 = tid;
     if (v0 + (CF_NV - 1) * BT < nfull) {
         uint4 a[CF_NV], b[CF_NV];
+        if (pre && pre->have) {
 #pragma unroll
-        for (int q = 0; q < CF_NV; ++q) a[q] = ld_stream(row + (size_t)(v0 + q * BT) * 16);
+            for (int q = 0; q < CF_NV; ++q) a[q] = pre->v[q];
+        } else {
+#pragma unroll
+            for (int q = 0; q < CF_NV; ++q) a[q] = ld_stream(row + (size_t)(v0 + q * BT) * 16);
+        }
         for (;;) {
             const int v1 = v0 + CF_NV * BT;
             const bool more = v1 + (CF_NV - 1) * BT < nfull;
@@ -1459,11 +1486,25 @@ __device__ int cf_attempt(const char* row, int V, float s, float m, double zrow,
     const bool own_tiny = tinyc && p0 < p1 && ((pl >= p0 && pl < p1) || (pl == W && p1 == W));
     unsigned sc = own_tiny ? tinyc : 0u;
     unsigned long long sm = own_tiny ? tinym : 0ull;
-    for (unsigned p = p0; p < p1; ++p) {
-        const unsigned c = win[W - 1u - p];
-        if (c) {
-            sc += c;
-            sm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(key_at(p)), s, m);
+    {
+        unsigned p = p0;
+        for (; p + 4u <= p1; p += 4u) {                // four counters read before any is used
+            unsigned c4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c4[j] = win[W - 1u - (p + j)];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (c4[j]) {
+                    sc += c4[j];
+                    sm += (unsigned long long)c4[j] * fix_mass(key_value<SPEC_BF16>(key_at(p + j)), s, m);
+                }
+        }
+        for (; p < p1; ++p) {
+            const unsigned c = win[W - 1u - p];
+            if (c) {
+                sc += c;
+                sm += (unsigned long long)c * fix_mass(key_value<SPEC_BF16>(key_at(p)), s, m);
+            }
         }
     }
     unsigned c0, ctot;
@@ -1537,16 +1578,17 @@ __device__ int cf_attempt(const char* row, int V, float s, float m, double zrow,
 // counters).  All threads call it.
 template <int BT>
 __device__ int cfilter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp,
-                            unsigned char* smem, size_t bytes, FiltRec* out) {
-    float D = CF_D;
+                            unsigned char* smem, size_t bytes, FiltRec* out, const CfPre<BT>* pre, float D1) {
+    float D = D1;
     if (!(K > 0 && K < V)) {                          // top-p alone: the row's mass bound, factor-2 slack
         const double rest = zrow - top_p_target(false, Pp, 0ull, zrow) / FIX_ONE;
         if (rest > 0.0) D = fminf(D, log2f((float)(2.0 * V / rest)));
     }
-    int st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out);
+    int st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out, pre);
     if (st != CF_SHORT) return st == CF_OK ? 1 : 0;
     for (int i = 0; i < 2 && st == CF_SHORT; ++i)
-        st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, fmaxf(D, i == 0 ? CF_D2 : CF_D3), smem, bytes, out);
+        st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, fmaxf(D, i == 0 ? CF_D2 : CF_D3), smem, bytes, out,
+                            (const CfPre<BT>*)nullptr);
     return st == CF_OK ? 2 : 0;
 }
 
@@ -1559,8 +1601,9 @@ __device__ unsigned long long g_filter_rows[3];
 // outcome when asked.
 template <int BT>
 __device__ __forceinline__ bool cand_filter(const Params& P, const char* row, float s, float m, double z, int K, float Pp,
-                                            unsigned char* smem, size_t bytes, FiltRec* out) {
-    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out);
+                                            unsigned char* smem, size_t bytes, FiltRec* out,
+                                            const CfPre<BT>* pre = nullptr, float D1 = CF_D_ONE) {
+    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out, pre, D1);
     if ((P.filt_mode & 2u) && threadIdx.x == 0) atomicAdd(&g_filter_rows[how == 0 ? 1 : how == 1 ? 0 : 2], 1ull);
     return how != 0;
 }
@@ -3452,6 +3495,9 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Para
                             : P.drf + ((size_t)b * P.gamma + (r - P.gamma - 1)) * P.dstride;
     const bool vh = tgt ? TDT == SPEC_BF16 : DDT == SPEC_BF16;
     uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
+    CfPre<BT> pre;
+    pre.have = false;
+    if (vh && !(P.filt_mode & 1u)) cf_prefetch<BT>(row, P.V, pre);
     pdl_wait();
     const int E = P.nch * SPC;
     if (threadIdx.x < 32) {
@@ -3469,9 +3515,9 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Para
     const double z = zsh;
     FiltRec rec;
     if constexpr (BT != FILT_BT) {
-        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec))
+        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec, &pre, CF_D_MANY))
             rec = wfilter_row<BT>(row, P.V, s, m, z, K, Pp, dyn, ws);
-    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec) ||
+    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec, &pre, CF_D_MANY) ||
                         vh_select(P.V, vh_build(row, P.V, fs, w), s, m, z, K, Pp, fs, w, &rec))) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<DDT>{dyn});
