@@ -988,7 +988,7 @@ __device__ bool vh_select(int V, int n, float s, float m, double zrow, int K, fl
 // boundary are the near-ties the oracle flags.  A window needing more than
 // WF_SLOTS counters is counted in segments, one more pass each.
 constexpr int WF_NB = 4096;                       // coarse buckets (key >> 4)
-constexpr int WF_SLOTS = 7168;                    // per-key counters of the window
+constexpr int WF_SLOTS = 7168;                    // per-key counters of the window (a segment)
 constexpr size_t WF_BYTES = (size_t)WF_NB * 4 + (size_t)WF_NB * 2 + (size_t)WF_SLOTS * 4;   // 52 KB
 
 struct WinShared {
@@ -1294,6 +1294,15 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
         }
         if (rk && !rp) {
             const double target = top_p_target(use_k, Pp, zk, zrow);
+            if (seg > 0 && (double)mb >= target) {
+                // the top-p key lies above this segment (the top-k key, which
+                // sets the target, was found only here): count the segments
+                // again from the top for it
+                cb = 0u;
+                mb = 0ull;
+                seg = -1;
+                continue;
+            }
             if ((double)(mb + ftot) >= target) {            // the top-p key lies in this segment
                 find(false, target);
                 tp = (uint32_t)ws.sel;
@@ -4783,7 +4792,7 @@ spec_status launch_chain_filtered(Params P, cudaStream_t st) {
     spec_status s = launch_stats<MODE_CHAIN, TDT, DK == DK_PROBS ? TDT : DDT>(P, st);
     if (s != SPEC_OK) return s;
     const int rows = (DK == DK_LOGITS) ? 2 * P.gamma + 1 : P.gamma + 1;
-    // bf16 rows only: FILT_BT_BF16 threads, several rows per SM, the windowed
+    // bf16 rows only: FILT_BT_BF16 threads, four rows per SM, the windowed
     // filter's 52 KB; else FILT_BT threads, a bf16 row's value histogram
     // (VH_BYTES), an f32 row's radix histograms
     constexpr bool any_bf16 = TDT == SPEC_BF16 || (DK == DK_LOGITS && DDT == SPEC_BF16);

@@ -166,6 +166,38 @@ def test_tiny_values_around_the_crossing(cuda_device):
     assert nbad == 0, det
 
 
+def _spread(rows, V, seed):
+    """bf16 values sign * 2^u, u uniform in [-60, 3]: every 1/8-binade bucket
+    of both signs is populated."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    shape = rows.shape[:-1] + (V,)
+    u = torch.rand(shape, generator=g, device="cuda") * 63.0 - 60.0
+    sign = torch.where(torch.rand(shape, generator=g, device="cuda") < 0.5, -1.0, 1.0)
+    rows[..., :V] = (sign * torch.exp2(u)).to(rows.dtype)
+
+
+def test_windowed_filter_segments(cuda_device):
+    """The windowed filter counts a window of more than WF_SLOTS keys in
+    segments.  Values spread over 63 binades of both signs make such a window;
+    top_k = 70000 puts the top-k key in the second segment while top_p = 0.5
+    puts the top-p key in the first, so the top-p search must go back to the
+    segments above.  The whole-row-only run (the windowed filter in every row)
+    equals the oracle and the default run."""
+    B, gamma, V = 4, 2, 131072
+    inp = wl.chain_inputs(B, gamma, V, seed=9700, device="cuda", temperatures=(1.0,))
+    _spread(inp.target, V, 11)
+    _spread(inp.draft, V, 12)
+    tk = torch.tensor([70000, 70000, 0, 40000], dtype=torch.int32, device="cuda")
+    tp = torch.tensor([0.5, 0.9, 0.5, 1.0], dtype=torch.float32, device="cuda")
+    d, rd = _run(0, lambda: parity.gpu_chain_filtered(inp, tk, tp))
+    w, rw = _run(1, lambda: parity.gpu_chain_filtered(inp, tk, tp))
+    _same(d, w)
+    o = parity.oracle_chain_filtered(inp, tk, tp)
+    for out in (d, w):
+        nflag, nbad, det = parity.compare_chain(out, o, gamma)
+        assert nbad == 0, det
+
+
 def test_counting_off_by_default(cuda_device):
     """Mode -1 (the state at load) counts nothing."""
     sv.spec_debug_filter_path(-1, read=True)
