@@ -2194,15 +2194,15 @@ struct ChainPrefetch {
 template <int TDT, int DDT, int DK>
 __device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) {
     ChainPrefetch f{0, 0.f, 0.f, 0.f, false};
-    const int tid = threadIdx.x, gamma = P.gamma;
-    if (tid < gamma) {
-        f.coin = P.coins[(size_t)b * gamma + tid];
-        f.x = P.draft_tokens[(size_t)b * gamma + tid];
+    const int tid = threadIdx.x, gamma = P.gamma, i = tid & 31;
+    if (tid < 64 && i < gamma) {                      // warp 0: p side, warp 1: q side of position i
+        f.x = P.draft_tokens[(size_t)b * gamma + i];
         f.ok = f.x >= 0 && f.x < P.V;
-        if (f.ok) {
-            const char* trow = P.tgt + ((size_t)b * (gamma + 1) + tid) * P.tstride;
-            const char* drow = P.drf + ((size_t)b * gamma + tid) * P.dstride;
-            f.l = ld_elem<TDT>(trow, f.x, P.V);
+        if (tid < 32) {
+            f.coin = P.coins[(size_t)b * gamma + i];
+            if (f.ok) f.l = ld_elem<TDT>(P.tgt + ((size_t)b * (gamma + 1) + i) * P.tstride, f.x, P.V);
+        } else if (f.ok) {
+            const char* drow = P.drf + ((size_t)b * gamma + i) * P.dstride;
             if constexpr (DK == DK_PROBS) f.d = __ldg(reinterpret_cast<const float*>(drow) + f.x);
             else f.d = ld_elem<DDT>(drow, f.x, P.V);
         }
@@ -2211,9 +2211,10 @@ __device__ __forceinline__ ChainPrefetch chain_prefetch(const Params& P, int b) 
 }
 
 // Chain decision for sequence b (rule 1), after the row statistics were
-// combined into sh.m / sh.z / sh.bad.  Threads 0..gamma-1 turn their
+// combined into sh.m / sh.z / sh.bad.  Threads i of warps 0 and 1 turn their
 // prefetched logits into p_i(x_i) and q_i(x_i) (fp64 exp2 in the units of the
-// row statistics); thread 0 then takes the decisions.  Leaves sh.ivals[0] =
+// row statistics), thread i tests position i's coin, and thread 0 takes the
+// first rejection.  Leaves sh.ivals[0] =
 // valid, sh.ivals[1] = k, sh.dvals[0] = s.  When `write` is set it also writes
 // the accepted tokens, the -1 tail (position k excluded), num_accepted and
 // the p/q diagnostics, and flags invalid sequences.  Ends with __syncthreads.
@@ -2226,25 +2227,38 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
     const float T = P.temperature[b];
     const bool tok = temperature_ok(T);
     const float s = tok ? scale_of(T) : 0.f;
-    if (tid < gamma) {
+    // p(x_i) in warp 0 and q(x_i) in warp 1 (thread i of each), then each
+    // position's coin test in thread i; thread 0 finds the first rejection
+    const int wi = tid & 31;
+    if (tid < 64 && wi < gamma) {
+        const bool q_side = tid >= 32;
         bool ok = f.ok;
-        double p = 0.0, q = 0.0;
+        double v = 0.0;
         if (ok && tok) {
-            p = prob_d(f.l, s, sh.m[tid], sh.z[tid]);
-            if (FILT && f.l < sh.th[tid]) p = 0.0;               // filtered out
-            if constexpr (DK == DK_PROBS) {
-                q = (double)f.d;
-                ok &= (q >= 0.0 && q <= 3.0e38);
+            if (!q_side) {
+                v = prob_d(f.l, s, sh.m[wi], sh.z[wi]);
+                if (FILT && f.l < sh.th[wi]) v = 0.0;             // filtered out
+            } else if constexpr (DK == DK_PROBS) {
+                v = (double)f.d;
+                ok &= (v >= 0.0 && v <= 3.0e38);
             } else {
-                q = prob_d(f.d, s, sh.m[gamma + 1 + tid], sh.z[gamma + 1 + tid]);
-                if (FILT && f.d < sh.th[gamma + 1 + tid]) q = 0.0;
+                v = prob_d(f.d, s, sh.m[gamma + 1 + wi], sh.z[gamma + 1 + wi]);
+                if (FILT && f.d < sh.th[gamma + 1 + wi]) v = 0.0;
             }
         }
-        sh.pch[tid] = p;
-        sh.pch[SPEC_MAX_GAMMA + tid] = q;
-        sh.pch[2 * SPEC_MAX_GAMMA + tid] = (double)f.coin;
-        sh.rej[tid] = ok;
-        sh.tok[tid] = f.x;
+        sh.pch[(q_side ? SPEC_MAX_GAMMA : 0) + wi] = v;
+        if (q_side) {
+            sh.rej[wi] = ok;
+        } else {
+            sh.pch[2 * SPEC_MAX_GAMMA + wi] = (double)f.coin;
+            sh.tok[wi] = f.x;
+        }
+    }
+    __syncthreads();
+    if (tid < gamma) {                                // accept position tid?
+        const double pi = sh.pch[tid], qi = sh.pch[SPEC_MAX_GAMMA + tid];
+        const double ratio = (qi > 0.0) ? pi / qi : INFINITY;
+        sh.par[tid] = (sh.pch[2 * SPEC_MAX_GAMMA + tid] <= ratio) ? 1 : 0;
     }
     __syncthreads();
     if (tid == 0) {
@@ -2252,13 +2266,9 @@ __device__ void chain_decide(const Params& P, int b, FinShared& sh, bool write, 
         for (int r = 0; r < P.R; ++r) ok &= !sh.bad[r];
         for (int i = 0; i < gamma; ++i) ok &= (sh.rej[i] != 0);
         int k = gamma;
-        if (ok) {
-            for (int i = 0; i < gamma; ++i) {
-                const double pi = sh.pch[i], qi = sh.pch[SPEC_MAX_GAMMA + i];
-                const double ratio = (qi > 0.0) ? pi / qi : INFINITY;
-                if (!(sh.pch[2 * SPEC_MAX_GAMMA + i] <= ratio)) { k = i; break; }
-            }
-        }
+        if (ok)
+            for (int i = 0; i < gamma; ++i)
+                if (!sh.par[i]) { k = i; break; }
         sh.ivals[0] = ok;
         sh.ivals[1] = k;
         sh.dvals[0] = (double)s;
