@@ -577,10 +577,11 @@ spec_status spec_debug_wait_budget(long long tries);
 /*
  * spec_debug_filter_path -- testing hook for the top-k / top-p filters of bf16
  * rows.  Each filtered row is first resolved from its candidates: the values
- * within a factor 2^14 of the row's largest probability (or fewer when the
+ * within a factor 2^D of the row's largest probability (D = 12 in the filter
+ * kernel, 14 in the on-demand and lazy walks, less with top-p alone when the
  * row's mass bound allows), counted per value in one pass into a window of
- * per-key counters fixed by the row statistics, and again with 2^18, then
- * 2^24, when a cut holds too few values or too little mass.  A row whose
+ * per-key counters fixed by the row statistics, and again with D + 6, then
+ * D + 12, when a cut holds too few values or too little mass.  A row whose
  * candidates cannot hold the answer, or whose window would overflow the
  * kernel's shared memory, is resolved by a whole-row path (the 65536-key
  * value histogram in 1024-thread filter CTAs, else the windowed filter).

@@ -1322,7 +1322,7 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
 }
 
 // bf16 rows, candidates first.  A cut x_c = (m - D) / s, D log2 units below
-// the row's maximum (D = 12 or 14; with top-p alone, less when the whole row's mass
+// the row's maximum (see CfCut; with top-p alone, never more than when the whole row's mass
 // bound V * 2^(x s - m) already proves the top-p key lies above it), rounded
 // down to a bf16 value.  The candidates' order keys lie in [key(x_c),
 // key(max)], both known from the statistics before the row is read: that
@@ -1341,12 +1341,16 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
 // exact unless the crossing falls among the tiny values: with top-k, the
 // top-p key lies at or above the top-k key; with top-p alone, the window's
 // mass must reach the top-p target.  A cut that holds fewer than top_k values
-// or too little mass is deepened (D = 18, then 24; the row is read again,
+// or too little mass is deepened by 6 log2 units, twice (the row is read again,
 // mostly from L2); otherwise, or when the window would outgrow the shared
 // memory, the function returns false and the caller takes a whole-row path.
-// first cut: 12 log2 units where many rows share the SMs (fewer candidates,
-// more rows deepened), 14 where one row's latency is the walk's
-constexpr float CF_D_MANY = 12.f, CF_D_ONE = 14.f, CF_D2 = 18.f, CF_D3 = 24.f;
+// First cut, log2 units below the maximum: 12 where many rows share the SMs
+// (fewer candidates, more rows deepened), 14 where one row's latency is the
+// walk's.  (Scaling the top-k cut as 1 / T was measured: fewer rows deepened
+// on workload 6, but many more candidates on workload 8's T = 0.8 rows.)
+struct CfCut { float d; };
+constexpr CfCut CF_MANY{12.f}, CF_ONE{14.f};
+constexpr float CF_DEEPER = 6.f;                  // a cut too shallow goes 6 log2 units deeper, twice
 constexpr float CF_TINY = 9.765625e-04f;          // 2^-10 (a whole number of key groups either side of 0)
 constexpr int CF_TINY_G = INT_MIN / 2;            // group table: a group of tiny values
 struct CfShared {
@@ -1587,17 +1591,18 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
 // counters).  All threads call it.
 template <int BT>
 __device__ int cfilter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp,
-                            unsigned char* smem, size_t bytes, FiltRec* out, const CfPre<BT>* pre, float D1) {
-    float D = D1;
+                            unsigned char* smem, size_t bytes, FiltRec* out, const CfPre<BT>* pre, CfCut cut) {
+    float D = cut.d;
     if (!(K > 0 && K < V)) {                          // top-p alone: the row's mass bound, factor-2 slack
         const double rest = zrow - top_p_target(false, Pp, 0ull, zrow) / FIX_ONE;
         if (rest > 0.0) D = fminf(D, log2f((float)(2.0 * V / rest)));
     }
     int st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out, pre);
     if (st != CF_SHORT) return st == CF_OK ? 1 : 0;
-    for (int i = 0; i < 2 && st == CF_SHORT; ++i)
-        st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, fmaxf(D, i == 0 ? CF_D2 : CF_D3), smem, bytes, out,
-                            (const CfPre<BT>*)nullptr);
+    for (int i = 0; i < 2 && st == CF_SHORT; ++i) {
+        D += CF_DEEPER;
+        st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out, (const CfPre<BT>*)nullptr);
+    }
     return st == CF_OK ? 2 : 0;
 }
 
@@ -1611,8 +1616,8 @@ __device__ unsigned long long g_filter_rows[3];
 template <int BT>
 __device__ __forceinline__ bool cand_filter(const Params& P, const char* row, float s, float m, double z, int K, float Pp,
                                             unsigned char* smem, size_t bytes, FiltRec* out,
-                                            const CfPre<BT>* pre = nullptr, float D1 = CF_D_ONE) {
-    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out, pre, D1);
+                                            const CfPre<BT>* pre = nullptr, CfCut cut = CF_ONE) {
+    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out, pre, cut);
     if ((P.filt_mode & 2u) && threadIdx.x == 0) atomicAdd(&g_filter_rows[how == 0 ? 1 : how == 1 ? 0 : 2], 1ull);
     return how != 0;
 }
@@ -3534,9 +3539,9 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Para
     const double z = zsh;
     FiltRec rec;
     if constexpr (BT != FILT_BT) {
-        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec, &pre, CF_D_MANY))
+        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec, &pre, CF_MANY))
             rec = wfilter_row<BT>(row, P.V, s, m, z, K, Pp, dyn, ws);
-    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec, &pre, CF_D_MANY) ||
+    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec, &pre, CF_MANY) ||
                         vh_select(P.V, vh_build(row, P.V, fs, w), s, m, z, K, Pp, fs, w, &rec))) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<DDT>{dyn});
