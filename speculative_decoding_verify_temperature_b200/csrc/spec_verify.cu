@@ -516,13 +516,13 @@ __device__ __forceinline__ float2 chunk_argmax(const char* row, int V, int c) {
 // top_k-th largest logit (ties kept), then, within that set, theta_p = the
 // largest logit whose set {l >= theta_p} carries a top_p share of the set's
 // mass; p'(v) = 2^(x_v - m) / Z' on the kept set.  Thresholds are found over
-// order-preserving keys of the logits (-0 folded onto +0): for bf16 rows an
-// exact count histogram of a window of keys below the row's maximum
-// (wfilter_row), for f32
-// rows (and a bf16 row whose histogram counter would wrap) a radix descent of
-// 12 + 12 + 8 bit digits (filter_row).  Counts decide top-k; masses are fixed
-// point (2^-40 units, integer sums, so they do not depend on the order of the
-// additions) and decide top-p and Z'.
+// order-preserving keys of the logits (-0 folded onto +0).  bf16 rows: the
+// candidates near the row's maximum first (cfilter_row), else the whole row's
+// value histogram (vh_build / vh_select, 1024 threads) or windowed histogram
+// (wfilter_row); f32 rows (and a bf16 row whose histogram counter would wrap):
+// a radix descent of 12 + 12 + 8 bit digits (filter_row).  Counts decide
+// top-k; masses are fixed point (2^-40 units, integer sums, so they do not
+// depend on the order of the additions) and decide top-p and Z'.
 
 constexpr int FILT_BT = 1024;
 constexpr int FILT_BT_BF16 = 256;                 // filter CTAs of launches whose filtered rows are all bf16
@@ -3423,21 +3423,13 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     else finalize_mss<TDT, SEQ_BT>(P, blockIdx.x, sh, blk, reinterpret_cast<float*>(dyn + P.stage_off));
 }
 
-// Filter thresholds of every row of a chain round, one CTA of FILT_BT threads
-// per (sequence, row): target rows 0..gamma, then the draft-logit rows (TREE:
-// the N node rows of every tree).  bf16 rows take the value histogram
-// (vh_build / vh_select), f32 rows the radix descent (filter_row).  Every CTA
-// waits for the statistics before it exits, so the finalize kernel that
-// follows (and reads the records and the statistics) waits for them through
-// this kernel.
-
 // The filter record of one row of sequence b (statistics row r, logits at
 // `row`, element type DT): invalid top_k / top_p give on = -1; filters off, a
 // bad temperature or an unusable row (the decision marks the sequence
-// invalid) give on = 0.  FILT_BT threads: the value histogram (bf16; the
-// radix descent when a counter wraps) or the radix descent (f32); other
-// block sizes (bf16 rows only): the windowed histogram.  All threads of the
-// CTA call it; thread 0 writes.
+// invalid) give on = 0.  bf16 rows try their candidates first (cfilter_row);
+// the whole-row path is, with FILT_BT threads, the value histogram (the radix
+// descent when a counter wraps), else the windowed filter; f32 rows take the
+// radix descent.  All threads of the CTA call it; thread 0 writes.
 template <int DT, int BT>
 __device__ void filter_one_row(const Params& P, int b, int r, const char* row, FiltShared& fs, WinShared& ws,
                                unsigned char* dyn) {
@@ -3485,6 +3477,12 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
     if (threadIdx.x == 0) *out = rec;
 }
 
+// Filter thresholds of every row of a round, one CTA per (sequence, row):
+// target rows 0..gamma, then the draft-logit rows (TREE: the N node rows of
+// every tree).  A bf16 row's first step of loads is issued before the wait
+// for the statistics.  Every CTA waits for the statistics before it exits,
+// so the finalize kernel that follows (and reads the records and the
+// statistics) waits for them through this kernel.
 template <int TDT, int DDT, int DK, bool TREE, int BT>
 __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Params P) {
     // FILT_BT threads: the value histogram and the radix descent (any row);
