@@ -2520,6 +2520,32 @@ __device__ int tree_final_draw(const Params& P, int b, int cur, const int* rej, 
     return y;
 }
 
+// Chunk masses sh.M[0..nch) of the weights wf over a row (per-warp sums in
+// wpw, then fp64 per chunk in warp order); returns their total (fp64, chunk
+// order).  All threads of the CTA call it.
+template <int CH, int BT, class WF>
+__device__ double row_chunk_masses(const WF& wf, int nch, float* wpw, FinShared& sh) {
+    constexpr int NWB = BT / 32;
+    row_warp_sums<CH, BT>(wf, nch, wpw);
+    __syncthreads();
+    for (int c = threadIdx.x; c < nch; c += BT) {
+        double M = 0.0;
+#pragma unroll
+        for (int w = 0; w < NWB; ++w) M += (double)wpw[c * NWB + w];
+        sh.M[c] = M;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double S = 0.0;
+        for (int c = 0; c < nch; ++c) S += sh.M[c];
+        sh.dvals[0] = S;
+    }
+    __syncthreads();
+    const double S = sh.dvals[0];
+    __syncthreads();
+    return S;
+}
+
 // Bitmap (sh.bitmap) of the excluded tokens rej[0..nrej) that fall in chunk c.
 template <int CH, int BT>
 __device__ void excl_bitmap(const int* rej, int nrej, int c, FinShared& sh) {
@@ -2533,14 +2559,26 @@ __device__ void excl_bitmap(const int* rej, int nrej, int c, FinShared& sh) {
 }
 
 // Inverse-CDF draw over a whole row with the weights wf (whose bitmap is
-// sh.bitmap) and the tokens rej[0..nrej) excluded: chunk masses (block sums
-// in fp64), the chunk holding u*S, one rescan.  *S_out = the total; -1 when
-// it is not positive.  All threads call it.
+// sh.bitmap) and the tokens rej[0..nrej) excluded.  The chunk masses come
+// from one pass over the row without exclusions (row_chunk_masses; wpw holds
+// nch * BT/32 floats); the few chunks that hold an excluded token are summed
+// again with their exclusions (block sums in fp64), so no mass is subtracted.
+// Then the chunk holding u*S and one rescan.  *S_out = the total; -1 when it
+// is not positive.  All threads call it.
 template <int CH, int BT, class WF>
-__device__ int draw_excluding(WF wf, const int* rej, int nrej, int nch, int V, float u, FinShared& sh,
+__device__ int draw_excluding(WF wf, const int* rej, int nrej, int nch, int V, float u, float* wpw, FinShared& sh,
                               double* S_out) {
     const int tid = threadIdx.x;
-    for (int c = 0; c < nch; ++c) {
+    wf.bitmap = nullptr;
+    row_chunk_masses<CH, BT>(wf, nch, wpw, sh);
+    wf.bitmap = sh.bitmap;
+    for (int i = 0; i < nrej; ++i) {                  // rej is uniform across the CTA
+        const int e = rej[i];
+        if (e < 0 || e >= V) continue;
+        bool seen = false;
+        for (int j = 0; j < i; ++j) seen |= rej[j] >= 0 && rej[j] < V && rej[j] / CH == e / CH;
+        if (seen) continue;
+        const int c = e / CH;
         excl_bitmap<CH, BT>(rej, nrej, c, sh);
         wf.base = c * CH;
         double tot;
@@ -2594,18 +2632,18 @@ __device__ int draw_excluding(WF wf, const int* rej, int nrej, int nch, int V, f
 // from p'_cur itself.  *S_out = the residual's mass.
 template <int TDT, int BT, bool HD>
 __device__ int tree_filt_draw(const Params& P, int b, int cur, const int* rej, int nrej, float s, float m,
-                              double zc, float th, FinShared& sh, double* S_out) {
+                              double zc, float th, float* wpw, FinShared& sh, double* S_out) {
     constexpr int CH = chunk_elems<TDT>();
     const char* row = P.tgt + ((size_t)b * P.N + cur) * P.tstride;
     const char* drow = HD ? reinterpret_cast<const char*>(P.draft_probs) + ((size_t)b * P.N + cur) * P.dpstride
                           : nullptr;
     const float u = P.final_u[b], iz = (float)(1.0 / zc);
     WTreeFilt<TDT, HD> wr{row, drow, s, m, iz, th, sh.bitmap, 0, P.V};
-    int y = draw_excluding<CH, BT>(wr, rej, nrej, P.nch, P.V, u, sh, S_out);
+    int y = draw_excluding<CH, BT>(wr, rej, nrej, P.nch, P.V, u, wpw, sh, S_out);
     if (y < 0) {
         WTreeFilt<TDT, false> wp{row, nullptr, s, m, iz, th, sh.bitmap, 0, P.V};
         double S1;
-        y = draw_excluding<CH, BT>(wp, rej, 0, P.nch, P.V, u, sh, &S1);
+        y = draw_excluding<CH, BT>(wp, rej, 0, P.nch, P.V, u, wpw, sh, &S1);
     }
     return y;
 }
@@ -2616,7 +2654,8 @@ __device__ int tree_filt_draw(const Params& P, int b, int cur, const int* rej, i
 // top-p filtering, with each row's threshold and kept mass read from the
 // filter records (k_filter) -- or, OD (on demand, bf16 rows, no diagnostics),
 // computed here for the rows of the nodes the walk visits, one window
-// histogram each (win: WF_BYTES of shared memory).
+// histogram each (win: WF_BYTES of shared memory).  FILT: win also holds the
+// final draw's per-warp chunk sums (P.nch * BT/32 floats).
 template <int TDT, int BT, bool FILT = false, bool OD = false>
 __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const float2* blk, unsigned char* win = nullptr,
                                 WinShared* ws = nullptr) {
@@ -2712,10 +2751,11 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
             cur = next;
         }
         double S;
+        float* wpw = reinterpret_cast<float*>(win);    // (the window's shared memory is free now)
         const int y = P.draft_probs ? tree_filt_draw<TDT, BT, true>(P, b, cur, sh.rej, nrej, s, sh.m[cur], zc, thc,
-                                                                    sh, &S)
+                                                                    wpw, sh, &S)
                                     : tree_filt_draw<TDT, BT, false>(P, b, cur, sh.rej, nrej, s, sh.m[cur], zc, thc,
-                                                                     sh, &S);
+                                                                     wpw, sh, &S);
         if (tid == 0) {
             ot[k] = y;
             for (int i = k + 1; i < W; ++i) { ot[i] = -1; ai[i] = -1; }
@@ -2773,10 +2813,11 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
     double S;
     int y;
     if constexpr (FILT) {
+        float* wpw = reinterpret_cast<float*>(win);
         y = P.draft_probs ? tree_filt_draw<TDT, BT, true>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur],
-                                                          sh.th[cur], sh, &S)
+                                                          sh.th[cur], wpw, sh, &S)
                           : tree_filt_draw<TDT, BT, false>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur],
-                                                           sh.th[cur], sh, &S);
+                                                           sh.th[cur], wpw, sh, &S);
     } else {
         y = tree_final_draw<TDT, BT>(P, b, cur, sh.rej, nrej, s, sh.m[cur], sh.z[cur], sh, &S);
     }
@@ -2819,32 +2860,6 @@ __device__ int draw_from_chunks(const WF& wf, int nch, int V, double t, float u,
         __syncthreads();
     }
     return y;
-}
-
-// Chunk masses sh.M[0..nch) of the weights wf over a row (per-warp sums in
-// wpw, then fp64 per chunk in warp order); returns their total (fp64, chunk
-// order).  All threads of the CTA call it.
-template <int CH, int BT, class WF>
-__device__ double row_chunk_masses(const WF& wf, int nch, float* wpw, FinShared& sh) {
-    constexpr int NWB = BT / 32;
-    row_warp_sums<CH, BT>(wf, nch, wpw);
-    __syncthreads();
-    for (int c = threadIdx.x; c < nch; c += BT) {
-        double M = 0.0;
-#pragma unroll
-        for (int w = 0; w < NWB; ++w) M += (double)wpw[c * NWB + w];
-        sh.M[c] = M;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double S = 0.0;
-        for (int c = 0; c < nch; ++c) S += sh.M[c];
-        sh.dvals[0] = S;
-    }
-    __syncthreads();
-    const double S = sh.dvals[0];
-    __syncthreads();
-    return S;
 }
 
 // State of the multi-step sampling walk at one node: p_j = max(0, p_0 - c q)
@@ -3414,7 +3429,8 @@ __global__ void __launch_bounds__(SEQ_BT) k_tree_final(const Params P) {
     const float2* blk = stage_stats(P, blockIdx.x, P.N, dyn, P.stage_cap, &sbar);
     if constexpr (MODE == MODE_GREEDY) finalize_greedy<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
     else if constexpr (MODE == MODE_SAMPLE) finalize_sample<TDT, SEQ_BT>(P, blockIdx.x, sh, blk);
-    else if constexpr (MODE == MODE_SAMPLE_FILT) finalize_sample<TDT, SEQ_BT, true>(P, blockIdx.x, sh, blk);
+    else if constexpr (MODE == MODE_SAMPLE_FILT)
+        finalize_sample<TDT, SEQ_BT, true>(P, blockIdx.x, sh, blk, dyn + P.stage_off);
     else if constexpr (MODE == MODE_SAMPLE_FILT_OD) {
         __shared__ WinShared ws;
         finalize_sample<TDT, SEQ_BT, true, true>(P, blockIdx.x, sh, blk,
@@ -4483,10 +4499,12 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_decide_mss(const Params P) {
 
 // Last token of a lazy target-only tree walk, one CTA per sequence (those
 // left in LZ_DRAW): tree_final_draw at the node where the walk stopped, with
-// the rejected children's tokens it kept.
+// the rejected children's tokens it kept.  FILT: the dynamic shared memory
+// holds the draw's per-warp chunk sums (P.nch * SEQ_BT/32 floats).
 template <int TDT, bool FILT = false>
 __global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
     __shared__ FinShared sh;
+    extern __shared__ __align__(16) unsigned char dyn[];
     pdl_wait();
     const int b = blockIdx.x, tid = threadIdx.x;
     const LazySeq L = P.lz_seq[b];
@@ -4497,9 +4515,10 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
     double S;
     int y;
     if constexpr (FILT) {
-        y = P.draft_probs ? tree_filt_draw<TDT, SEQ_BT, true>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, sh, &S)
-                          : tree_filt_draw<TDT, SEQ_BT, false>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, sh,
-                                                               &S);
+        float* wpw = reinterpret_cast<float*>(dyn);
+        y = P.draft_probs
+                ? tree_filt_draw<TDT, SEQ_BT, true>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, wpw, sh, &S)
+                : tree_filt_draw<TDT, SEQ_BT, false>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, L.th, wpw, sh, &S);
     } else {
         y = tree_final_draw<TDT, SEQ_BT>(P, b, L.cur, sh.rej, L.nrej, L.s, L.m, L.z, sh, &S);
     }
@@ -4877,9 +4896,12 @@ spec_status launch_tree_filtered(Params P, cudaStream_t st) {
     if (s != SPEC_OK) return s;
     static PerDevice<bool> big_c;
     const bool big = big_c.get([] { return allow_stage(k_tree_final<MODE_SAMPLE_FILT, TDT>); });
-    P.stage_cap = stats_stage_bytes(P, P.N, big ? STAGE_STATS_MAX : 48 * 1024 - 1024);
-    return launch_dependent(k_tree_final<MODE_SAMPLE_FILT, TDT>, (unsigned)P.B, SEQ_BT, P.stage_cap, P, st,
-                            "k_tree_final");
+    // per-warp chunk sums of the final draw after the statistics stage
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    P.stage_cap = stats_stage_bytes(P, P.N, (big ? STAGE_STATS_MAX : 48 * 1024 - 1024) - wpw);
+    P.stage_off = (P.stage_cap + 15) & ~15;
+    return launch_dependent(k_tree_final<MODE_SAMPLE_FILT, TDT>, (unsigned)P.B, SEQ_BT, (size_t)P.stage_off + wpw, P,
+                            st, "k_tree_final");
 }
 
 // One level of the lazy walk: the statistics kernel (the first one as an
@@ -5020,7 +5042,8 @@ spec_status launch_tree_filtered_lazy(Params P, cudaStream_t st) {
         s = launch_dependent(kd, dgrid, NT, 0, P, st, "k_lz_decide");
         if (s != SPEC_OK) return s;
     }
-    spec_status s = launch_dependent(k_lz_tree_final<TDT, true>, (unsigned)P.B, SEQ_BT, 0, P, st, "k_lz_tree_final");
+    const size_t wpw = (size_t)P.nch * (SEQ_BT / 32) * sizeof(float);
+    spec_status s = launch_dependent(k_lz_tree_final<TDT, true>, (unsigned)P.B, SEQ_BT, wpw, P, st, "k_lz_tree_final");
     if (s == SPEC_OK && g_prof_stop && record(g_prof_stop, st) != cudaSuccess)
         return fail(SPEC_ERR_CUDA, "profile event");
     return s;
