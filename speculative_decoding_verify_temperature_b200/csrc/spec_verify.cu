@@ -4504,7 +4504,7 @@ __global__ void __launch_bounds__(SEQ_BT) k_lz_decide_mss(const Params P) {
 template <int TDT, bool FILT = false>
 __global__ void __launch_bounds__(SEQ_BT) k_lz_tree_final(const Params P) {
     __shared__ FinShared sh;
-    extern __shared__ __align__(16) unsigned char dyn[];
+    extern __shared__ __align__(128) unsigned char dyn[];
     pdl_wait();
     const int b = blockIdx.x, tid = threadIdx.x;
     const LazySeq L = P.lz_seq[b];
