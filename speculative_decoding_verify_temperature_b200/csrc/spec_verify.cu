@@ -1585,22 +1585,60 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
     return st;
 }
 
+// Rows with at most this many statistics entries get the top-k cut below.
+constexpr int CF_SEG_MAX = 256;
+
+// A cut that holds the top-k crossing, from the row's statistics: entry e is
+// fl(x_max * s) over the elements of one warp of one chunk, so the K-th
+// largest entry m_K belongs to K distinct elements, each >= m_K / s up to the
+// rounding of the product, and at least K values lie at or above a cut just
+// below m_K / s.  Returns that cut in log2 units below m (the margin covers
+// the product's rounding and the cut's own arithmetic), or +inf when m_K is
+// -inf.  E <= CF_SEG_MAX entries at st; smem: the candidate filter's shared
+// memory, whose window is not in use yet.  All threads call it.
+template <int BT>
+__device__ float cf_topk_cut(const float2* st, int E, int K, float m, unsigned char* smem) {
+    float* v = reinterpret_cast<float*>(smem + CF_HEAD);
+    float* res = v + CF_SEG_MAX;
+    for (int i = threadIdx.x; i < E; i += BT) v[i] = st[i].x;
+    if (threadIdx.x == 0) *res = -INFINITY;
+    __syncthreads();
+    for (int i = threadIdx.x; i < E; i += BT) {       // rank of entry i, ties by index
+        const float x = v[i];
+        int rank = 0;
+        for (int j = 0; j < E; ++j) {
+            const float y = v[j];
+            rank += (y > x || (y == x && j < i)) ? 1 : 0;
+        }
+        if (rank == K - 1) *res = x;
+    }
+    __syncthreads();
+    const float mk = *res;
+    __syncthreads();                                  // the window's memory is free again
+    if (!(mk > -INFINITY)) return INFINITY;
+    return (m - mk) + 0.015625f + fabsf(mk) * 1.52587890625e-05f;
+}
+
 // Threshold and kept mass of one bf16 row from its candidates (see above):
 // 1 (first cut) or 2 (deeper cut) with the record in *out; 0: the caller
-// takes a whole-row path.  smem: `bytes` of shared memory (up to 16384 window
-// counters).  All threads call it.
+// takes a whole-row path.  sts: the row's E statistics entries.  smem: `bytes`
+// of shared memory (up to 16384 window counters).  All threads call it.
 template <int BT>
 __device__ int cfilter_row(const char* row, int V, float s, float m, double zrow, int K, float Pp,
-                            unsigned char* smem, size_t bytes, FiltRec* out, const CfPre<BT>* pre, CfCut cut) {
-    float D = cut.d;
+                            const float2* sts, int E, unsigned char* smem, size_t bytes, FiltRec* out,
+                            const CfPre<BT>* pre, CfCut cut) {
+    float D = cut.d, Dsure = INFINITY;
     if (!(K > 0 && K < V)) {                          // top-p alone: the row's mass bound, factor-2 slack
         const double rest = zrow - top_p_target(false, Pp, 0ull, zrow) / FIX_ONE;
         if (rest > 0.0) D = fminf(D, log2f((float)(2.0 * V / rest)));
+    } else if (K <= E && E <= CF_SEG_MAX) {           // top-k: a cut that surely holds K values
+        Dsure = cf_topk_cut<BT>(sts, E, K, m, smem);
+        D = fminf(D, Dsure);
     }
     int st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out, pre);
     if (st != CF_SHORT) return st == CF_OK ? 1 : 0;
     for (int i = 0; i < 2 && st == CF_SHORT; ++i) {
-        D += CF_DEEPER;
+        D = fminf(Dsure, D + CF_DEEPER);
         st = cf_attempt<BT>(row, V, s, m, zrow, K, Pp, D, smem, bytes, out, (const CfPre<BT>*)nullptr);
     }
     return st == CF_OK ? 2 : 0;
@@ -1612,12 +1650,14 @@ __device__ int cfilter_row(const char* row, int V, float s, float m, double zrow
 __device__ unsigned long long g_filter_rows[3];
 
 // cfilter_row unless the caller switched the candidate pass off; counts the
-// outcome when asked.
+// outcome when asked.  st: the row's statistics (P.nch * SPC entries).
 template <int BT>
-__device__ __forceinline__ bool cand_filter(const Params& P, const char* row, float s, float m, double z, int K, float Pp,
-                                            unsigned char* smem, size_t bytes, FiltRec* out,
-                                            const CfPre<BT>* pre = nullptr, CfCut cut = CF_ONE) {
-    const int how = (P.filt_mode & 1u) ? 0 : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, smem, bytes, out, pre, cut);
+__device__ __forceinline__ bool cand_filter(const Params& P, const char* row, const float2* st, float s, float m,
+                                            double z, int K, float Pp, unsigned char* smem, size_t bytes,
+                                            FiltRec* out, const CfPre<BT>* pre = nullptr, CfCut cut = CF_ONE) {
+    const int how = (P.filt_mode & 1u)
+                        ? 0
+                        : cfilter_row<BT>(row, P.V, s, m, z, K, Pp, st, P.nch * SPC, smem, bytes, out, pre, cut);
     if ((P.filt_mode & 2u) && threadIdx.x == 0) atomicAdd(&g_filter_rows[how == 0 ? 1 : how == 1 ? 0 : 2], 1ull);
     return how != 0;
 }
@@ -2709,7 +2749,9 @@ __device__ void finalize_sample(const Params& P, int b, FinShared& sh, const flo
         for (;;) {
             const char* row = P.tgt + ((size_t)b * N + cur) * P.tstride;
             FiltRec f{-INFINITY, 0, 0.0};
-            if (((K > 0 && K < V) || Pp < 1.f) && !cand_filter<BT>(P, row, s, sh.m[cur], sh.z[cur], K, Pp, win, WF_BYTES, &f))
+            const float2* st = P.stats + ((size_t)b * P.R + cur) * P.nch * SPC;
+            if (((K > 0 && K < V) || Pp < 1.f) &&
+                !cand_filter<BT>(P, row, st, s, sh.m[cur], sh.z[cur], K, Pp, win, WF_BYTES, &f))
                 f = wfilter_row<BT>(row, V, s, sh.m[cur], sh.z[cur], K, Pp, win, *ws);
             thc = f.theta;
             zc = f.on > 0 ? f.Z : sh.z[cur];
@@ -3482,7 +3524,9 @@ __device__ void filter_one_row(const Params& P, int b, int r, const char* row, F
     }
     FiltRec rec{-INFINITY, 0, 0.0};
     bool done = false;
-    if constexpr (DT == SPEC_BF16) done = cand_filter<BT>(P, row, s, m, zsh, K, Pp, dyn, BT == FILT_BT ? VH_BYTES : WF_BYTES, &rec);
+    if constexpr (DT == SPEC_BF16)
+        done = cand_filter<BT>(P, row, P.stats + ((size_t)b * P.R + r) * E, s, m, zsh, K, Pp, dyn,
+                               BT == FILT_BT ? VH_BYTES : WF_BYTES, &rec);
     if constexpr (BT == FILT_BT) {
         uint32_t* w = reinterpret_cast<uint32_t*>(dyn);
         if (!done && (DT != SPEC_BF16 || !vh_select(P.V, vh_build(row, P.V, fs, w), s, m, zsh, K, Pp, fs, w, &rec)))
@@ -3553,9 +3597,11 @@ __global__ void __launch_bounds__(BT, BT == FILT_BT ? 1 : 4) k_filter(const Para
     const double z = zsh;
     FiltRec rec;
     if constexpr (BT != FILT_BT) {
-        if (!cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, WF_BYTES, &rec, &pre, CF_MANY))
+        if (!cand_filter<BT>(P, row, P.stats + ((size_t)b * P.R + r) * E, s, m, z, K, Pp, dyn, WF_BYTES, &rec, &pre,
+                             CF_MANY))
             rec = wfilter_row<BT>(row, P.V, s, m, z, K, Pp, dyn, ws);
-    } else if (!vh || !(cand_filter<BT>(P, row, s, m, z, K, Pp, dyn, VH_BYTES, &rec, &pre, CF_MANY) ||
+    } else if (!vh || !(cand_filter<BT>(P, row, P.stats + ((size_t)b * P.R + r) * E, s, m, z, K, Pp, dyn, VH_BYTES,
+                                        &rec, &pre, CF_MANY) ||
                         vh_select(P.V, vh_build(row, P.V, fs, w), s, m, z, K, Pp, fs, w, &rec))) {
         if (tgt) rec = filter_row<TDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<TDT>{dyn});
         else rec = filter_row<DDT>(row, P.V, s, m, z, K, Pp, fs, FiltHist<DDT>{dyn});
