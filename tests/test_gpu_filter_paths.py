@@ -198,6 +198,33 @@ def test_windowed_filter_segments(cuda_device):
         assert nbad == 0, det
 
 
+def test_topk_cut_from_the_statistics(cuda_device):
+    """A top-k row whose top_k is at most its number of statistics entries
+    (one per warp of each 16 KB chunk: 52 for V = 100000) is first cut at the
+    K-th largest entry, which surely holds the crossing: no row needs a
+    deeper cut or the whole-row path, also where a cut at a fixed depth holds
+    too few values or where thousands of values tie at the crossing (nearly
+    flat rows; rows of four repeated levels).  The records equal the
+    whole-row ones and the outputs equal the oracle's."""
+    B, gamma, V = 8, 2, 100000
+    inp = wl.chain_inputs(B, gamma, V, seed=9800, device="cuda", zipf=True, temperatures=(1.0,))
+    g = torch.Generator(device="cuda").manual_seed(7)
+    rows = inp.target[..., :V]
+    flat = 5.0 + torch.randn(rows.shape, generator=g, device="cuda") * 0.05
+    levels = torch.tensor([6.0, 5.5, 5.0, 4.5], device="cuda")
+    lv = levels[torch.randint(0, 4, rows.shape, generator=g, device="cuda")]
+    rows[0:2] = flat[0:2].to(rows.dtype)              # sequences 0-1: nearly flat around 5
+    rows[2:4] = lv[2:4].to(rows.dtype)                # sequences 2-3: four repeated levels
+    tk = torch.tensor([1, 20, 52, 7, 1, 20, 52, 7], dtype=torch.int32, device="cuda")
+    tp = torch.ones(B, dtype=torch.float32, device="cuda")
+    rd = _ab(lambda: parity.gpu_chain_filtered(inp, tk, tp))
+    assert rd[0] == B * (2 * gamma + 1) and rd[1] == 0 and rd[2] == 0, rd
+    out = parity.gpu_chain_filtered(inp, tk, tp)
+    o = parity.oracle_chain_filtered(inp, tk, tp)
+    nflag, nbad, det = parity.compare_chain(out, o, gamma)
+    assert nbad == 0, det
+
+
 def test_counting_off_by_default(cuda_device):
     """Mode -1 (the state at load) counts nothing."""
     sv.spec_debug_filter_path(-1, read=True)
