@@ -1361,6 +1361,7 @@ struct CfShared {
     int gbase[512];                               // key group (key >> 7) -> window position of its key 0
 };
 constexpr size_t CF_HEAD = ((sizeof(CfShared) + 127) / 128) * 128;
+constexpr int CF_STG = 256;                       // staged survivors per warp and pass step
 enum { CF_OK = 0, CF_SHORT = 1, CF_FAIL = 2 };
 
 // 16-byte loads in flight per thread and step: 64 KB per SM (four 256-thread
@@ -1391,8 +1392,11 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
                                           const CfPre<BT>* pre) {
     CfShared& cs = *reinterpret_cast<CfShared*>(smem);
     unsigned* win = reinterpret_cast<unsigned*>(smem + CF_HEAD);
-    const unsigned wmax = (unsigned)min((size_t)16384, ((bytes - CF_HEAD) / 4) & ~(size_t)3);
-    const int tid = threadIdx.x;
+    // the end of the shared memory: each warp's survivor staging (CF_STG values)
+    const size_t stg_off = (bytes - (size_t)(BT / 32) * CF_STG * sizeof(unsigned short)) & ~(size_t)15;
+    unsigned short* stg = reinterpret_cast<unsigned short*>(smem + stg_off) + (threadIdx.x >> 5) * CF_STG;
+    const unsigned wmax = (unsigned)min((size_t)16384, ((stg_off - CF_HEAD) / 4) & ~(size_t)3);
+    const int tid = threadIdx.x, lane = tid & 31;
     const bool use_k = K > 0 && K < V, use_p = Pp < 1.f;
     const __nv_bfloat16 tb = __float2bfloat16_rd((m - D) / s);
     const float xc = __bfloat162float(tb);
@@ -1430,7 +1434,9 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
             cs.over = 1u;
         }
     };
-    auto survivors = [&](const uint4& vq) {
+    // survivor mask of one 16-byte vector: bit c for the low value of pair c,
+    // bit 16 + c for the high one
+    auto smask = [&](const uint4& vq) {
         const uint32_t xs[4] = {vq.x, vq.y, vq.z, vq.w};
         unsigned bits = 0u;
 #pragma unroll
@@ -1439,13 +1445,62 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
             memcpy(&h, &xs[c], 4);
             bits |= (__hge2_mask(h, t2) & 0x10001u) << c;
         }
+        return bits;
+    };
+    auto svalue = [](const uint4& vq, int p) {       // the raw bits of survivor p of vq
+        const int c = p & 3;
+        const uint32_t w = c < 2 ? (c == 0 ? vq.x : vq.y) : (c == 2 ? vq.z : vq.w);
+        return p >= 16 ? (w >> 16) : (w & 0xFFFFu);
+    };
+    auto survivors = [&](const uint4& vq) {
+        unsigned bits = smask(vq);
         while (bits) {
             const int p = __ffs(bits) - 1;
             bits &= bits - 1u;
-            const int c = p & 3;
-            const uint32_t w = c < 2 ? (c == 0 ? xs[0] : xs[1]) : (c == 2 ? xs[2] : xs[3]);
-            count(p >= 16 ? (w >> 16) : (w & 0xFFFFu));
+            count(svalue(vq, p));
         }
+    };
+    // One step's vectors of a converged warp: the lanes' survivors are staged
+    // in the warp's slice (a warp prefix sum of their counts gives each lane
+    // its place) and counted by the whole warp, so a step costs about one
+    // shared atomic instruction per 32 survivors instead of one per vector.
+    // A step with more than CF_STG survivors counts vector by vector.
+    auto step_survivors = [&](const uint4 (&vs)[cf_nv<BT>()]) {
+        constexpr int NV = cf_nv<BT>();
+        if (__activemask() != FULL) {
+#pragma unroll
+            for (int q = 0; q < NV; ++q) survivors(vs[q]);
+            return;
+        }
+        int c = 0;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) c += __popc(smask(vs[q]));
+        if (!__any_sync(FULL, c > 0)) return;
+        int inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(FULL, inc, o);
+            if (lane >= o) inc += n;
+        }
+        const int total = __shfl_sync(FULL, inc, 31);
+        if (total > CF_STG) {
+#pragma unroll
+            for (int q = 0; q < NV; ++q) survivors(vs[q]);
+            return;
+        }
+        int at = inc - c;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) {
+            unsigned bits = smask(vs[q]);
+            while (bits) {
+                const int p = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                stg[at++] = (unsigned short)svalue(vs[q], p);
+            }
+        }
+        __syncwarp();
+        for (int j = lane; j < total; j += 32) count(stg[j]);
+        __syncwarp();                                 // the slice is read before the next step writes it
     };
     // ---- one pass: the values >= x_c.  Per 16-byte vector the four pair
     // compares make a survivor mask (bit c: the low value of pair c, bit
@@ -1471,8 +1526,7 @@ __device__ __forceinline__ int cf_attempt(const char* row, int V, float s, float
 #pragma unroll
                 for (int q = 0; q < CF_NV; ++q) b[q] = ld_stream(row + (size_t)(v1 + q * BT) * 16);
             }
-#pragma unroll
-            for (int q = 0; q < CF_NV; ++q) survivors(a[q]);
+            step_survivors(a);
             v0 = v1;
             if (!more) break;
 #pragma unroll
