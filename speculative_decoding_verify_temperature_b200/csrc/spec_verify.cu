@@ -1331,9 +1331,9 @@ __device__ FiltRec wfilter_row(const char* row, int V, float s, float m, double 
 // tens of thousands of (mostly absent) keys; those few values are counted
 // together, with their exact fixed-point mass -- is cleared, and one pass
 // over the row counts every value >= x_c into it (bf16 pair compares make a
-// survivor mask per 16-byte vector; each lane counts its own survivors with
-// 32-bit shared atomics, at the position a 512-entry table of key groups
-// gives).  The window is then scanned from its top as the
+// survivor mask per 16-byte vector; a warp stages the survivors of a pass
+// step and counts them with whole-warp 32-bit shared atomics, at the position
+// a 512-entry table of key groups gives).  The window is then scanned from its top as the
 // value histogram scans its keys -- count and fixed-point mass count *
 // fixed(2^(v s - m)) per key, a block scan, the thread whose run crosses
 // top_k or the top-p target walks it -- so the record is the same integers
